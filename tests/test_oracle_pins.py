@@ -1,0 +1,313 @@
+"""Pins for the float64 oracle: checks against things other than the oracle itself.
+
+Each test ties one oracle function to a hand-worked case, a closed form, an
+invariant, brute force, or an independent library routine (torch), so that a
+dropped term, a wrong sign or index, or a transposed operand fails here.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from head_partitioned_sparse_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                yield [c.strip() for c in line.split("|")]
+
+
+# ---------------------------------------------------------------- bf16 rounding
+def test_bf16_rounding_matches_torch_on_fp32_values():
+    rng = np.random.default_rng(1)
+    x = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32) * np.float32(10.0) ** rng.integers(-30, 30, 20000).astype(np.float32),
+        np.array([0.0, -0.0, 1.0, -1.0, 3.0e38, -3.0e38, 1e-40, -1e-40, 1.17e-38], np.float32),
+    ])
+    # exact midpoints between neighbouring bf16 values, both parities of the last kept bit
+    u = rng.integers(0x00800000, 0x7F000000, 5000, dtype=np.uint64).astype(np.uint32)
+    mid = ((u & np.uint32(0xFFFF0000)) | np.uint32(0x8000)).view(np.float32)
+    x = np.concatenate([x, mid, -mid])
+    ours = O.f64_to_bf16_bits(x.astype(np.float64))
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_bf16_rounding_from_f64_is_single_rounding():
+    # 1 + 2^-8 + 2^-40 is just above the midpoint between 1 and 1+2^-7: must round up.
+    # Rounding through fp32 first would land exactly on the midpoint and round to even (down).
+    v = 1.0 + 2.0 ** -8 + 2.0 ** -40
+    assert O.bf16_bits_to_f64(O.f64_to_bf16_bits(np.array([v])))[0] == 1.0 + 2.0 ** -7
+    assert O.bf16_bits_to_f64(O.f64_to_bf16_bits(np.array([1.0 + 2.0 ** -8])))[0] == 1.0  # tie -> even
+
+
+def test_bf16_decode_roundtrip():
+    bits = np.arange(0, 0x7F80, 7, dtype=np.uint16)
+    assert np.array_equal(O.f64_to_bf16_bits(O.bf16_bits_to_f64(bits)), bits)
+    ref = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(O.bf16_bits_to_f64(bits), ref)
+
+
+# ---------------------------------------------------------------- RoPE
+def test_rope_golden_anchors():
+    n = 0
+    for row in _rows("rope_cases.txt"):
+        if len(row) == 4:
+            theta, pos, dim, outs = float(row[0]), int(row[1]), int(row[2]), row[3]
+            x = np.zeros(128)
+            x[dim] = 1.0
+            y = O.rope(x, pos, theta)
+            want = np.zeros(128)
+            for kv in outs.split():
+                k, v = kv.split(":")
+                want[int(k)] = float(v)
+            np.testing.assert_allclose(y, want, atol=1e-12, rtol=0)
+        else:
+            theta, i, val = float(row[0]), int(row[1]), float(row[2])
+            assert O.rope_inv_freq(128, theta)[i] == pytest.approx(val, rel=1e-14)
+        n += 1
+    assert n >= 8
+
+
+def test_rope_is_a_complex_rotation():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((5, 128))
+    pos = np.array([0, 1, 17, 4095, 1048575])
+    y = O.rope(x, pos, 500000.0)
+    # independent construction: z_i = x_i + i x_{i+64}, rotated by exp(i * pos * w_i), w_i geometric
+    w = np.exp(-np.arange(64) / 64.0 * math.log(500000.0))
+    z = (x[:, :64] + 1j * x[:, 64:]) * np.exp(1j * pos[:, None] * w[None, :])
+    np.testing.assert_allclose(y[:, :64], z.real, atol=1e-9)
+    np.testing.assert_allclose(y[:, 64:], z.imag, atol=1e-9)
+
+
+def test_rope_invariants():
+    rng = np.random.default_rng(3)
+    q, k = rng.standard_normal(128), rng.standard_normal(128)
+    np.testing.assert_allclose(O.rope(q, 0, 5e5), q, atol=0)
+    assert np.linalg.norm(O.rope(q, 12345, 5e5)) == pytest.approx(np.linalg.norm(q), rel=1e-13)
+    a = O.rope(q, 100, 5e5) @ O.rope(k, 40, 5e5)
+    b = O.rope(q, 1100, 5e5) @ O.rope(k, 1040, 5e5)
+    assert a == pytest.approx(b, rel=1e-9, abs=1e-9)
+
+
+# ---------------------------------------------------------------- index projection
+def test_index_rows_unit_projector_selects_components():
+    rng = np.random.default_rng(4)
+    perm = rng.permutation(128)[:16]
+    P = np.zeros((16, 128))
+    P[np.arange(16), perm] = 1.0
+    k_bits = synth.f32_to_bf16_bits(rng.standard_normal((33, 128)).astype(np.float32))
+    k = O.bf16_bits_to_f64(k_bits)
+    got = O.index_rows(k, P)
+    assert np.array_equal(got, k_bits[:, perm])          # row r picks component perm[r]
+    got2 = O.index_rows(k, 2.0 * P)
+    assert np.array_equal(O.bf16_bits_to_f64(got2), 2.0 * k[:, perm])
+
+
+def test_index_rows_rounds_sum_at_midpoint_to_even():
+    P = np.zeros((16, 128))
+    P[0, 0] = 1.0
+    P[0, 1] = 1.0
+    k = np.zeros((2, 128))
+    k[0, :2] = [1.0, 2.0 ** -8]          # 1 + 2^-8: midpoint of 1 and 1+2^-7 -> 1 (even)
+    k[1, :2] = [1.0 + 2.0 ** -7, 2.0 ** -8]  # midpoint of 1+2^-7 and 1+2^-6 -> 1+2^-6 (even)
+    got = O.bf16_bits_to_f64(O.index_rows(k, P))[:, 0]
+    assert got[0] == 1.0 and got[1] == 1.0 + 2.0 ** -6
+
+
+# ---------------------------------------------------------------- index probabilities
+def test_index_probs_against_torch_softmax_and_group_mean():
+    rng = np.random.default_rng(5)
+    G, L = 4, 300
+    q = rng.standard_normal((G, 128))
+    P = rng.standard_normal((G, 16, 128)) / math.sqrt(128)
+    idx = rng.standard_normal((L, 16))
+    pi, a = O.index_probs(q, P, idx, 0.25)
+    tq, tP, ti = (torch.from_numpy(t) for t in (q, P, idx))
+    q_idx = torch.stack([tP[h] @ tq[h] for h in range(G)])           # [G][16]
+    ref_a = torch.softmax(0.25 * (ti @ q_idx.T).T, dim=-1)           # [G][L]
+    np.testing.assert_allclose(a, ref_a.numpy(), rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(pi, ref_a.mean(0).numpy(), rtol=1e-12, atol=1e-15)
+    assert pi.sum() == pytest.approx(1.0, abs=1e-12)
+
+
+def test_index_probs_projector_acts_on_query_side():
+    # With a unit projector, q_idx is a subset of q's components; scores are exact.
+    q = np.zeros((1, 128))
+    q[0, 7] = 2.0
+    P = np.zeros((1, 16, 128))
+    P[0, 3, 7] = 1.0                     # index dim 3 <- query dim 7
+    idx = np.zeros((3, 16))
+    idx[1, 3] = 1.0                      # token 1 matches: score 2 -> logit 0.5
+    pi, _ = O.index_probs(q, P, idx, 0.25)
+    e = math.exp(0.5)
+    np.testing.assert_allclose(pi, [1 / (2 + e), e / (2 + e), 1 / (2 + e)], rtol=1e-14)
+
+
+# ---------------------------------------------------------------- top-p
+def test_top_p_golden_cases():
+    n = 0
+    for p, masses, kept in _rows("top_p_cases.txt"):
+        pi = np.array([float(m) for m in masses.split()])
+        want = [int(k) for k in kept.split()]
+        assert list(O.top_p(pi, float(p)).kept) == want, (p, masses)
+        n += 1
+    assert n >= 15
+
+
+def test_top_p_matches_brute_force_subset_search():
+    rng = np.random.default_rng(6)
+    for trial in range(300):
+        L = int(rng.integers(1, 11))
+        pi = rng.random(L) ** 3
+        if trial % 5 == 0 and L > 2:   # inject exact ties
+            pi[rng.integers(0, L)] = pi[rng.integers(0, L)]
+        pi /= pi.sum()
+        p = float(rng.choice([0.3, 0.5, 0.8, 0.9, 0.95, 0.99]))
+        tp = O.top_p(pi, p)
+        # brute force: smallest cardinality whose best subset reaches p
+        best = None
+        for r in range(1, L + 1):
+            cands = [c for c in itertools.combinations(range(L), r) if pi[list(c)].sum() >= p]
+            if cands:
+                top = max(pi[list(c)].sum() for c in cands)
+                best = (r, top)
+                break
+        if best is None:       # rounding kept the total below p: everything is kept
+            assert len(tp.kept) == L
+            continue
+        assert len(tp.kept) == best[0]
+        assert pi[tp.kept].sum() == pytest.approx(best[1], abs=1e-12)
+
+
+def test_top_p_minimality_and_tie_order():
+    rng = np.random.default_rng(7)
+    for _ in range(50):
+        L = int(rng.integers(50, 400))
+        pi = rng.lognormal(0, 2, L)
+        pi /= pi.sum()
+        for p in (0.5, 0.9, 0.99):
+            kept = O.top_p(pi, p).kept
+            mass = pi[kept].sum()
+            assert mass >= p - 1e-12
+            assert mass - pi[kept].min() < p
+            # every kept token outranks every dropped one
+            dropped = np.setdiff1d(np.arange(L), kept)
+            if len(dropped):
+                assert pi[kept].min() >= pi[dropped].max()
+    pi = np.array([0.2, 0.1, 0.2, 0.1, 0.2, 0.2])
+    assert list(O.top_p(pi, 0.5).kept) == [0, 2, 4]   # three tied 0.2s, lowest positions
+
+
+def test_top_p_p_one_keeps_all():
+    pi = np.array([0.7, 0.3, 0.0, 0.0])
+    assert list(O.top_p(pi, 1.0).kept) == [0, 1, 2, 3]
+
+
+# ---------------------------------------------------------------- sink/window
+def test_sink_window_golden():
+    for L, ns, w, pos in _rows("sink_window_cases.txt"):
+        assert list(O.sink_window(int(L), int(ns), int(w))) == [int(x) for x in pos.split()]
+
+
+# ---------------------------------------------------------------- attention
+def test_attend_matches_torch_sdpa():
+    rng = np.random.default_rng(8)
+    q, K, V = rng.standard_normal((4, 128)), rng.standard_normal((77, 128)), rng.standard_normal((77, 128))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None, None], torch.from_numpy(K)[None, None], torch.from_numpy(V)[None, None])
+    np.testing.assert_allclose(O.attend(q, K, V), ref[0, 0].numpy(), rtol=1e-12, atol=1e-12)
+
+
+def _dense_ref(inp, b, g):
+    """Full causal-decode attention over all L tokens via torch (independent of the oracle)."""
+    L = int(inp.seq_lens[b])
+    G = inp.G
+    f = (lambda a: O.bf16_bits_to_f64(a)) if inp.dtype == "bf16" else (lambda a: np.asarray(a, np.float64))
+    q = f(inp.q_pre[b, g * G:(g + 1) * G])
+    # RoPE written independently as a complex rotation
+    w = np.exp(-np.arange(64) / 64.0 * math.log(inp.rope_theta))
+    z = (q[:, :64] + 1j * q[:, 64:]) * np.exp(1j * (L - 1) * w)
+    qr = np.concatenate([z.real, z.imag], axis=1)
+    K, V = f(inp.k_cache[b, g, :L]), f(inp.v_cache[b, g, :L])
+    return torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(qr)[None, None], torch.from_numpy(K)[None, None], torch.from_numpy(V)[None, None])[0, 0].numpy()
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_decode_p1_equals_dense_for_retrieval_heads(dtype):
+    inp = synth.make_inputs("tiny", 0, overrides={"L": 600, "window": 64, "dtype": dtype, "B": 2},
+                            seq_lens=[600, 333])
+    out, res = O.decode_inputs(inp, p=1.0)
+    for b in range(inp.B):
+        ref = _dense_ref(inp, b, 0)
+        np.testing.assert_allclose(out[b, 0:4], ref, atol=1e-10)
+        assert len(res[(b, 0)].attended) == inp.seq_lens[b]
+
+
+def test_decode_window_covering_context_equals_dense_for_all_heads():
+    inp = synth.make_inputs("tiny", 1, overrides={"L": 500, "window": 64})
+    out, _ = O.decode_inputs(inp, window=10 ** 6, p=0.5)
+    for g in range(inp.Hkv):
+        np.testing.assert_allclose(out[0, g * 4:(g + 1) * 4], _dense_ref(inp, 0, g), atol=1e-10)
+
+
+def test_decode_streaming_head_sees_only_sinks_and_window():
+    inp = synth.make_inputs("tiny", 2, overrides={"L": 700, "window": 32})
+    out, res = O.decode_inputs(inp)
+    sr = res[(0, 1)]
+    assert list(sr.attended) == list(range(4)) + list(range(700 - 32, 700))
+    # changing streaming-head keys outside sinks/window changes nothing
+    inp.k_cache[0, 1, 100:600] = inp.k_cache[0, 1, 100:600][::-1]
+    out2, _ = O.decode_inputs(inp)
+    np.testing.assert_array_equal(out[0, 4:8], out2[0, 4:8])
+
+
+def test_retrieval_output_invariant_to_permuting_kv_order():
+    inp = synth.make_inputs("tiny", 3, overrides={"L": 1024, "window": 64})
+    idx = O.index_cache_for(inp)
+    out, res = O.decode_inputs(inp, idx_cache=idx)
+    lo, hi = inp.n_sink, 1024 - inp.window
+    rng = np.random.default_rng(9)
+    perm = np.arange(1024)
+    perm[lo:hi] = lo + rng.permutation(hi - lo)       # new position j holds old row perm[j]
+    for arr in (inp.k_cache, inp.v_cache, inp.k_pre):
+        arr[0, 0] = arr[0, 0][perm]
+    idx2 = idx.copy()
+    idx2[0, 0] = idx[0, 0][perm]
+    out2, res2 = O.decode_inputs(inp, idx_cache=idx2)
+    np.testing.assert_allclose(out2[0, 0:4], out[0, 0:4], atol=1e-12)
+    inv = np.argsort(perm)
+    assert sorted(perm[res2[(0, 0)].listed]) == sorted(res[(0, 0)].listed)
+    assert len(inv) == 1024
+
+
+def test_index_append_matches_projection_of_each_head():
+    inp = synth.make_inputs("tiny", 4, overrides={"L": 64})
+    k = np.asarray(inp.k_pre, np.float64)
+    bits = O.index_append(k, inp.P_k)
+    assert bits.shape == (1, 2, 64, 16)
+    # head 1 uses P_k[1], not P_k[0]
+    v1 = O.bf16_bits_to_f64(bits[0, 1])
+    np.testing.assert_allclose(v1, k[0, 1] @ inp.P_k[1].astype(np.float64).T, rtol=2 ** -8, atol=1e-30)
+    assert not np.allclose(v1, k[0, 1] @ inp.P_k[0].astype(np.float64).T, rtol=1e-2)
+
+
+def test_planted_keys_are_recalled_in_tiny_workload():
+    inp = synth.make_inputs("tiny", 0)
+    _, res = O.decode_inputs(inp)
+    sr = res[(0, 0)]
+    planted = inp.planted[(0, 0)]
+    assert len(planted) == 4
+    assert set(planted) <= set(sr.topp.kept)
+    assert len(sr.topp.kept) < 0.05 * inp.seq_lens[0]   # concentrated: a small selected set
