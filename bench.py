@@ -1,0 +1,416 @@
+#!/usr/bin/env python3
+"""Decode-step benchmark of head-partitioned sparse attention on B200.
+
+One step = one spa_decode call on one layer's buffers for the whole batch:
+query prologue, index scoring, top-p selection, split-K attention over
+sinks + window + selected rows, and the combine.  Inputs are seeded synthetic
+tensors of the named workload (default: ctx128k, batch 4, 32/8 heads, 128K
+context), resident in HBM before timing.  Several layer copies are cycled so
+that each step reads cold data (the per-step working set exceeds L2 as well).
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the float64 CPU
+oracle on the host cores instead (a bounded sample per step).
+
+Multi-GPU: launched with torchrun, one process per GPU; every rank runs its own
+batch (weak scaling, no collective in the data path); the time is the max over
+ranks and ``value`` counts the layer-steps of all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from head_partitioned_sparse_b200 import shard, synth  # noqa: E402
+
+METRIC = "sparse decode-attention layer-steps/sec and achieved HBM GB/s at 128K ctx"
+UNIT = "layer-steps/s"
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--config", default="ctx128k", choices=synth.list_configs())
+    ap.add_argument("--p", type=float, default=None, help="top-p threshold (default: the workload's)")
+    ap.add_argument("--layers", type=int, default=2, help="layer copies cycled through")
+    ap.add_argument("--split-rows", type=int, default=0)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-sweep", action="store_true", help="skip the per-p sweep")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def workload_desc(cfg: dict, name: str, p: float) -> str:
+    return (f"{name}: batch {cfg['B']}, {cfg['Hq']}/{cfg['Hkv']} heads, head dim 128, context {cfg['L']}, "
+            f"{cfg['dtype']}, {len(cfg['retrieval'])} retrieval KV heads, r=16 index, p={p:g}, "
+            f"sinks {cfg['n_sink']}, window {cfg['window']}")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(gpu_index)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- profiles
+def recorded_traffic(kernel_file: str, summary: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", summary)
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_sha = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
+    m_b = re.search(r"dram_bytes_per_launch_full_workload:\s*([0-9.eE+]+)", text)
+    if not (m_sha and m_b):
+        return None
+    src = os.path.join(ROOT, "head_partitioned_sparse_b200", "csrc", kernel_file)
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != m_sha.group(1):
+        return None
+    return float(m_b.group(1))
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- helpers
+def algorithmic_bytes(inp, counts: np.ndarray, s_kv: int):
+    """Bytes a decode step must move: index rows of retrieval heads, sink/window K/V
+    of every head, selected K/V rows, the query and the output."""
+    idx = contig_rows = 0
+    for b in range(inp.B):
+        L = int(inp.seq_lens[b])
+        n_s = min(inp.n_sink, L)
+        w_lo = max(n_s, L - inp.window)
+        contig = n_s + (L - w_lo)
+        for g in range(inp.Hkv):
+            contig_rows += contig
+            if inp.head_mask[g]:
+                idx += L * 32
+    sel_rows = int(counts.sum())
+    kv_row = 2 * 128 * s_kv
+    q = inp.B * inp.Hq * 128 * s_kv
+    out = inp.B * inp.Hq * 128 * 4
+    return {"idx": idx, "contig_kv": contig_rows * kv_row, "selected_kv": sel_rows * kv_row, "q": q, "out": out,
+            "contig_rows": contig_rows, "selected_rows": sel_rows,
+            "total": idx + contig_rows * kv_row + sel_rows * kv_row + q + out}
+
+
+def cpu_threads() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] + [1])
+    except Exception:
+        return 1
+
+
+def run_oracle_sample(inp, idx_bits, p, seqs):
+    import oracle as O
+    slices = [(b, g) for b in seqs for g in range(inp.Hkv)]
+    t0 = time.perf_counter()
+    O.decode_inputs(inp, idx_cache=idx_bits, p=p, slices=slices)
+    return time.perf_counter() - t0
+
+
+# ----------------------------------------------------------------------------- reference arm
+def main_reference(args):
+    rank, _, world = shard.dist_env()
+    if rank != 0:
+        return 0
+    import oracle as O
+    cfg = dict(synth.CONFIGS[args.config])
+    p = float(np.float32(args.p if args.p is not None else cfg["p"]))
+    inp = synth.make_inputs(args.config, shard.rank_seed(args.seed, 0), draw_streaming_kpre=False)
+    ret = [g for g in range(inp.Hkv) if inp.head_mask[g]]
+    idx = O.index_cache_for(inp, heads=ret, precision="f64")   # BLAS: fast setup, untimed
+    # each step: the oracle's decode of one sequence of the batch (all its KV heads);
+    # a layer-step is B such samples.
+    for i in range(args.warmup):
+        run_oracle_sample(inp, idx, p, [i % inp.B])
+    times = [run_oracle_sample(inp, idx, p, [i % inp.B]) for i in range(args.steps)]
+    sec_per_layer_step = float(np.mean(times)) * inp.B
+    value = 1.0 / sec_per_layer_step
+    cores = cpu_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec_per_layer_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(cfg, args.config, p), "batch": inp.B, "seq_len": inp.Lmax, "p": p},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"float64 NumPy oracle, one sequence (all {inp.Hkv} KV heads) per step, "
+                                   f"x{inp.B} per layer-step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- native arm
+def main_native(args):
+    import torch
+    import torch.distributed as dist
+
+    from head_partitioned_sparse_b200 import binding as B
+    from head_partitioned_sparse_b200 import build as spa_build
+
+    rank, local, world = shard.dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    if not os.path.exists(B.LIB_PATH):
+        spa_build.build()
+    B.load()
+
+    cfg = dict(synth.CONFIGS[args.config])
+    p = float(np.float32(args.p if args.p is not None else cfg["p"]))
+    inp = synth.make_inputs(args.config, shard.rank_seed(args.seed, rank), draw_streaming_kpre=False)
+    s_kv = 2 if inp.dtype == "bf16" else 4
+
+    def up(a):
+        if inp.dtype == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    P_q = torch.from_numpy(inp.P_q).to(dev)
+    P_k = torch.from_numpy(inp.P_k).to(dev)
+    c = B.make_config(max_batch=inp.B, n_q_heads=inp.Hq, n_kv_heads=inp.Hkv, max_ctx=inp.Lmax,
+                      kv_dtype=B.SPA_BF16 if inp.dtype == "bf16" else B.SPA_F32, P_q=P_q, P_k=P_k,
+                      rope_theta=inp.rope_theta, idx_scale=inp.idx_scale, split_rows=args.split_rows)
+    h = B.spa_create(c)
+    stream = torch.cuda.current_stream(dev)
+    q = up(inp.q_pre)
+    lens = torch.from_numpy(inp.seq_lens).to(dev)
+    head_mask = inp.head_mask
+
+    # layer 0 from the generator; the index cache is built on the GPU by spa_index_append
+    k0, v0 = up(inp.k_cache), up(inp.v_cache)
+    kp = up(inp.k_pre)
+    idx0 = torch.zeros((inp.B, inp.Hkv, inp.Lmax, 16), dtype=torch.int16, device=dev)
+    zero = torch.zeros(inp.B, dtype=torch.int64, device=dev)
+    B.spa_index_append(h, kp, zero, inp.B, inp.Lmax, idx0, stream)
+    B.spa_device_status(h, stream)
+    del kp
+    layers = [(k0, v0, idx0)] + [(k0.clone(), v0.clone(), idx0.clone()) for _ in range(max(1, args.layers) - 1)]
+    out = torch.empty((inp.B, inp.Hq, 128), dtype=torch.float32, device=dev)
+    cnt = torch.zeros(inp.B * inp.Hkv, dtype=torch.int32, device=dev)
+    Lcap = int(inp.seq_lens.max())
+
+    def step(i, pp=p):
+        k, v, ix = layers[i % len(layers)]
+        B.spa_decode(h, q, k, v, ix, head_mask, lens, inp.B, Lcap, pp, inp.n_sink, inp.window, out, None, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def timed(n_steps, fn, profile=False):
+        torch.cuda.synchronize(dev)
+        barrier()
+        if profile:
+            B.spa_set_profiling(h, True)
+        n0 = B.spa_launch_count(h)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(n_steps):
+            fn(i)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        launches = B.spa_launch_count(h) - n0
+        return e0.elapsed_time(e1), launches
+
+    clocks = ClockSampler(local) if rank == 0 else None
+    for i in range(args.warmup):
+        step(i)
+    ms, launches = timed(args.steps, step, profile=True)
+    kern = {}
+    for kid in range(B.SPA_K_COUNT):
+        tot, n = B.spa_profile_read(h, kid)
+        if n:
+            kern[B.spa_kernel_name(kid)] = {"launches": n, "avg_us": 1e3 * tot / n}
+    B.spa_set_profiling(h, False)
+    ms_max = shard.reduce_max(ms, dev)
+    ms_per_step = ms_max / args.steps
+
+    # selected counts of this workload (identical every step)
+    B.spa_decode(h, q, layers[0][0], layers[0][1], layers[0][2], head_mask, lens, inp.B, Lcap, p, inp.n_sink,
+                 inp.window, out, cnt, stream)
+    B.spa_device_status(h, stream)
+    counts = cnt.cpu().numpy().reshape(inp.B, inp.Hkv)
+    ab = algorithmic_bytes(inp, counts, s_kv)
+
+    # p sweep (same measurement, smaller step count)
+    sweep = {}
+    if not args.no_sweep and "p_sweep" in cfg:
+        for pp in cfg["p_sweep"]:
+            pq = float(np.float32(pp))
+            for i in range(3):
+                step(i, pq)
+            n = max(10, args.steps // 4)
+            msw, _ = timed(n, lambda i: step(i, pq))
+            msw = shard.reduce_max(msw, dev) / n
+            B.spa_decode(h, q, layers[0][0], layers[0][1], layers[0][2], head_mask, lens, inp.B, Lcap, pq,
+                         inp.n_sink, inp.window, out, cnt, stream)
+            torch.cuda.synchronize(dev)
+            abw = algorithmic_bytes(inp, cnt.cpu().numpy(), s_kv)
+            sweep[f"{pp:g}"] = {"ms_per_step": msw, "layer_steps_per_s": world * 1e3 / msw,
+                                "achieved_gbs": abw["total"] / (msw * 1e-3) / 1e9,
+                                "selected_rows": abw["selected_rows"]}
+
+    # end to end through the public API: pinned host inputs in, result out, every step
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda t: t.cpu().pin_memory()
+        t_last = Lcap - 1
+        q_h = pin(q)
+        kpre_new = torch.from_numpy(np.ascontiguousarray(inp.k_pre[:, :, t_last:t_last + 1]))
+        kpre_h = (kpre_new.view(torch.int16) if inp.dtype == "bf16" else kpre_new).pin_memory()
+        knew_h = pin(layers[0][0][:, :, t_last].contiguous())
+        vnew_h = pin(layers[0][1][:, :, t_last].contiguous())
+        pos_h = torch.full((inp.B,), t_last, dtype=torch.int64).pin_memory()
+        out_h = torch.empty((inp.B, inp.Hq, 128), dtype=torch.float32).pin_memory()
+        q_d = torch.empty_like(q)
+        kpre_d = torch.empty(kpre_h.shape, dtype=kpre_h.dtype, device=dev)
+        pos_d = torch.empty(inp.B, dtype=torch.int64, device=dev)
+
+        def e2e_step(i):
+            k, v, ix = layers[i % len(layers)]
+            q_d.copy_(q_h, non_blocking=True)
+            kpre_d.copy_(kpre_h, non_blocking=True)
+            pos_d.copy_(pos_h, non_blocking=True)
+            k[:, :, t_last].copy_(knew_h, non_blocking=True)
+            v[:, :, t_last].copy_(vnew_h, non_blocking=True)
+            B.spa_index_append(h, kpre_d, pos_d, inp.B, 1, ix, stream)
+            B.spa_decode(h, q_d, k, v, ix, head_mask, lens, inp.B, Lcap, p, inp.n_sink, inp.window, out, None,
+                         stream)
+            out_h.copy_(out, non_blocking=True)
+
+        for i in range(3):
+            e2e_step(i)
+        mse, _ = timed(args.steps, e2e_step)
+        mse = shard.reduce_max(mse, dev) / args.steps
+        h2d = (q_h.numel() * q_h.element_size() + kpre_h.numel() * kpre_h.element_size() + pos_h.numel() * 8 +
+               knew_h.numel() * knew_h.element_size() + vnew_h.numel() * vnew_h.element_size())
+        d2h = out_h.numel() * 4
+        e2e = {"value": world * 1e3 / mse, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": mse}
+    clk = clocks.stop() if clocks else None
+
+    if rank == 0:
+        peak, peak_kind = measured_peaks()
+        att = kern.get("attend", {"avg_us": float("nan")})
+        att_bytes = (ab["contig_rows"] + ab["selected_rows"]) * 2 * 128 * s_kv
+        achieved = att_bytes / (att["avg_us"] * 1e-6) / 1e9
+        traffic = recorded_traffic("k_attend.cu", "attend_ctx128k.md") if args.config == "ctx128k" else None
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle as O
+            ret = [g for g in range(inp.Hkv) if inp.head_mask[g]]
+            idx_o = O.index_cache_for(inp, heads=ret, precision="f64")   # untimed setup
+            t_first = run_oracle_sample(inp, idx_o, p, list(range(inp.B)))
+            reps = max(1, min(8, math.ceil(10.0 / max(t_first, 1e-3)))) - 1
+            tot = t_first + sum(run_oracle_sample(inp, idx_o, p, list(range(inp.B))) for _ in range(reps))
+            cpu = {"value": (reps + 1) / tot, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                   "sample": f"full layer-step (all {inp.B}x{inp.Hkv} slices) x{reps + 1} with the float64 "
+                             f"NumPy oracle; index cache precomputed"}
+        step_gbs = ab["total"] / (ms_per_step * 1e-3) / 1e9
+        line = {
+            "metric": METRIC, "value": world * 1e3 / ms_per_step, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": workload_desc(cfg, args.config, p), "batch": inp.B, "seq_len": inp.Lmax,
+                       "p": p, "storage": inp.dtype, "parallelism": f"dp{world}" if world > 1 else "single",
+                       "l2": f"inputs larger than L2: {len(layers)} layer copies of "
+                             f"{(layers[0][0].numel() * 2 * s_kv + layers[0][2].numel() * 2) / 1e9:.2f} GB "
+                             f"cycled; {ab['total'] / 1e6:.0f} MB touched per step"},
+            "achieved_gbs": step_gbs,
+            "frac_of_peak": step_gbs / peak,
+            "bytes_per_step": ab,
+            "selected_counts": counts.tolist(),
+            "kernels_us": kern,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic, "kernel": "attend",
+                         "peak_kind": peak_kind},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": int(launches),
+            "clocks": clk,
+            "p_sweep": sweep or None,
+        }
+        print(json.dumps(line), flush=True)
+    B.spa_destroy(h)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return main_reference(args)
+    return main_native(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,191 @@
+"""ctypes binding of libspa (include/spa.h): argument marshalling only.
+
+Every function keeps the C name and argument order.  Tensor arguments may be
+torch tensors (their ``data_ptr()`` is passed), plain integers (raw device
+addresses) or None (NULL).  ``stream`` may be a ``torch.cuda.Stream``, a raw
+``cudaStream_t`` integer, or None for torch's current stream.  A non-zero
+status raises :class:`SpaError` carrying ``spa_last_error()``.
+
+The library must have been built (``python -m head_partitioned_sparse_b200.build``);
+there is no fallback: if ``libspa.so`` is missing or cannot be loaded, this
+module raises on first use.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libspa.so")
+
+SPA_OK = 0
+SPA_ERR_INVALID_ARG = -1
+SPA_ERR_UNSUPPORTED = -2
+SPA_ERR_WORKSPACE = -3
+SPA_ERR_CUDA = -4
+SPA_ERR_DEVICE_TIMEOUT = -5
+SPA_ERR_DEVICE_RANGE = -6
+SPA_BF16 = 0
+SPA_F32 = 1
+
+SPA_K_INDEX_APPEND, SPA_K_PROLOGUE, SPA_K_SCORE, SPA_K_MASS, SPA_K_THRESHOLD, SPA_K_COMPACT, \
+    SPA_K_ATTEND, SPA_K_COMBINE = range(8)
+SPA_K_COUNT = 8
+
+
+class SpaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"spa status {status}: {msg}")
+        self.status = status
+
+
+class spa_config(ctypes.Structure):
+    _fields_ = [
+        ("max_batch", ctypes.c_int),
+        ("n_q_heads", ctypes.c_int),
+        ("n_kv_heads", ctypes.c_int),
+        ("head_dim", ctypes.c_int),
+        ("idx_dim", ctypes.c_int),
+        ("kv_dtype", ctypes.c_int),
+        ("max_ctx", ctypes.c_int64),
+        ("rope_theta", ctypes.c_double),
+        ("idx_scale", ctypes.c_float),
+        ("split_rows", ctypes.c_int),
+        ("P_q", ctypes.c_void_p),
+        ("P_k", ctypes.c_void_p),
+    ]
+
+
+_vp, _i, _i64, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+_SIGS = {
+    "spa_create": (_i, [ctypes.POINTER(_vp), ctypes.POINTER(spa_config)]),
+    "spa_destroy": (_i, [_vp]),
+    "spa_workspace_size": (_i, [ctypes.POINTER(spa_config), ctypes.POINTER(ctypes.c_size_t)]),
+    "spa_last_error": (ctypes.c_char_p, []),
+    "spa_index_append": (_i, [_vp, _vp, _vp, _i, _i, _vp, _vp]),
+    "spa_select": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i64, _f, _i, _i, _vp, _vp, _vp]),
+    "spa_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i64, _f, _i, _i, _vp, _vp, _vp]),
+    "spa_device_status": (_i, [_vp, _vp]),
+    "spa_set_profiling": (_i, [_vp, _i]),
+    "spa_profile_read": (_i, [_vp, _i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
+    "spa_kernel_name": (ctypes.c_char_p, [_i]),
+    "spa_launch_count": (_i, [_vp, ctypes.POINTER(ctypes.c_int64)]),
+}
+EXPORTED = tuple(_SIGS)
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libspa.so (once) and declare every exported signature."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m head_partitioned_sparse_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _ptr(x) -> Optional[int]:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        return x.data_ptr()
+    raise TypeError(f"expected a tensor, an int address or None, got {type(x)!r}")
+
+
+def _stream(s) -> Optional[int]:
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _host_u8(mask) -> ctypes.Array:
+    vals = [int(v) for v in (mask.tolist() if hasattr(mask, "tolist") else mask)]
+    return (ctypes.c_uint8 * len(vals))(*vals)
+
+
+def _check(status: int) -> None:
+    if status != SPA_OK:
+        raise SpaError(status, load().spa_last_error().decode())
+
+
+def spa_last_error() -> str:
+    return load().spa_last_error().decode()
+
+
+def spa_workspace_size(cfg: spa_config) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load().spa_workspace_size(ctypes.byref(cfg), ctypes.byref(n)))
+    return n.value
+
+
+def spa_create(cfg: spa_config) -> int:
+    h = ctypes.c_void_p(None)
+    _check(load().spa_create(ctypes.byref(h), ctypes.byref(cfg)))
+    return h.value
+
+
+def spa_destroy(h) -> None:
+    _check(load().spa_destroy(h))
+
+
+def spa_index_append(h, k_pre, start_pos, B: int, T: int, idx_cache, stream=None) -> None:
+    _check(load().spa_index_append(h, _ptr(k_pre), _ptr(start_pos), B, T, _ptr(idx_cache), _stream(stream)))
+
+
+def spa_select(h, q_pre, idx_cache, head_mask, seq_lens, B: int, max_seq_len: int, p: float, n_sink: int,
+               window: int, sel_idx, sel_count, stream=None) -> None:
+    _check(load().spa_select(h, _ptr(q_pre), _ptr(idx_cache), _host_u8(head_mask), _ptr(seq_lens), B,
+                             max_seq_len, p, n_sink, window, _ptr(sel_idx), _ptr(sel_count), _stream(stream)))
+
+
+def spa_decode(h, q_pre, k_cache, v_cache, idx_cache, head_mask, seq_lens, B: int, max_seq_len: int, p: float,
+               n_sink: int, window: int, out, sel_count_opt=None, stream=None) -> None:
+    _check(load().spa_decode(h, _ptr(q_pre), _ptr(k_cache), _ptr(v_cache), _ptr(idx_cache), _host_u8(head_mask),
+                             _ptr(seq_lens), B, max_seq_len, p, n_sink, window, _ptr(out), _ptr(sel_count_opt),
+                             _stream(stream)))
+
+
+def spa_device_status(h, stream=None) -> None:
+    _check(load().spa_device_status(h, _stream(stream)))
+
+
+def spa_set_profiling(h, enable: bool) -> None:
+    _check(load().spa_set_profiling(h, 1 if enable else 0))
+
+
+def spa_profile_read(h, kernel_id: int) -> Tuple[float, int]:
+    ms, n = ctypes.c_double(0.0), ctypes.c_int64(0)
+    _check(load().spa_profile_read(h, kernel_id, ctypes.byref(ms), ctypes.byref(n)))
+    return ms.value, n.value
+
+
+def spa_kernel_name(kernel_id: int) -> str:
+    return load().spa_kernel_name(kernel_id).decode()
+
+
+def spa_launch_count(h) -> int:
+    n = ctypes.c_int64(0)
+    _check(load().spa_launch_count(h, ctypes.byref(n)))
+    return n.value
+
+
+def make_config(*, max_batch: int, n_q_heads: int, n_kv_heads: int, max_ctx: int, kv_dtype: int,
+                P_q, P_k, rope_theta: float = 500000.0, idx_scale: float = 0.25, split_rows: int = 0,
+                head_dim: int = 128, idx_dim: int = 16) -> spa_config:
+    """Fill a spa_config; P_q / P_k are device float32 tensors (or addresses)."""
+    return spa_config(max_batch=max_batch, n_q_heads=n_q_heads, n_kv_heads=n_kv_heads, head_dim=head_dim,
+                      idx_dim=idx_dim, kv_dtype=kv_dtype, max_ctx=max_ctx, rope_theta=rope_theta,
+                      idx_scale=idx_scale, split_rows=split_rows, P_q=_ptr(P_q), P_k=_ptr(P_k))

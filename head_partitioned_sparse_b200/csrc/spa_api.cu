@@ -1,0 +1,432 @@
+// Host side of the libspa C ABI: argument checks, workspace, launch sequencing.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/spa.h"
+#include "spa_internal.cuh"
+
+namespace {
+
+thread_local std::string g_err;
+
+spa_status fail(spa_status code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+spa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(SPA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Layout {
+  size_t off[16];
+  size_t total;
+  int64_t max_items;
+  int n_chunks_max;
+};
+
+// Sizes every workspace region for a configuration (offsets 256-byte aligned).
+Layout plan(const spa_config& c, int split_rows) {
+  Layout L{};
+  const int G = c.n_q_heads / c.n_kv_heads;
+  const size_t slices = (size_t)c.max_batch * c.n_kv_heads;
+  const int64_t Lmax = c.max_ctx;
+  L.n_chunks_max = (int)((Lmax + spa::kChunk - 1) / spa::kChunk);
+  L.max_items = (int64_t)slices * ((Lmax + split_rows - 1) / split_rows);
+  size_t sz[16] = {
+      (size_t)c.n_q_heads * 16 * 128 * 4,                  // 0 P_q
+      (size_t)c.n_kv_heads * 16 * 128 * 4,                 // 1 P_k
+      64 * 8,                                              // 2 inv_freq
+      (size_t)c.max_batch * c.n_q_heads * 128 * 4,         // 3 q_rot
+      (size_t)c.max_batch * c.n_q_heads * 16 * 4,          // 4 q_idx
+      slices * L.n_chunks_max * G * 8,                     // 5 stats
+      slices * (size_t)Lmax * 4,                           // 6 pi
+      slices * spa::kBins1 * 8,                            // 7 hist1
+      slices * (size_t)Lmax * 8,                           // 8 cand
+      slices * L.n_chunks_max * 4,                         // 9 chunk_gt
+      slices * L.n_chunks_max * 4,                         // 10 chunk_off
+      slices * sizeof(spa::SliceState),                    // 11 st
+      slices * (size_t)Lmax * 4,                           // 12 list
+      (slices + 1) * 4,                                    // 13 item_base
+      (size_t)L.max_items * G * (spa::kHeadDim + 2) * 4,   // 14 part
+      256,                                                 // 15 dev_err
+  };
+  size_t o = 0;
+  for (int i = 0; i < 16; ++i) {
+    L.off[i] = o;
+    o += round_up(sz[i], 256);
+  }
+  L.total = o;
+  return L;
+}
+
+}  // namespace
+
+struct spa_ctx {
+  spa_config cfg{};
+  int G = 0;
+  int split_rows = 0;
+  float idx_scale = 0.f;
+  int device = 0;
+  int num_sms = 0;
+  int attend_occ = 1;
+  void* mem = nullptr;
+  size_t mem_bytes = 0;
+  spa::Workspace ws{};
+  int n_chunks_max = 0;
+  // instrumentation
+  bool prof = false;
+  std::vector<cudaEvent_t> ev;   // pairs: 2*i start, 2*i+1 stop
+  std::vector<int> ev_kid;
+  size_t ev_next = 0;
+  int64_t launches = 0;
+};
+
+namespace {
+
+constexpr size_t kEventPairs = 1 << 14;
+
+spa_status check_config(const spa_config* c) {
+  if (!c) return fail(SPA_ERR_INVALID_ARG, "config is NULL");
+  if (c->head_dim != 128) return fail(SPA_ERR_UNSUPPORTED, "head_dim must be 128 (got %d)", c->head_dim);
+  if (c->idx_dim != 16) return fail(SPA_ERR_UNSUPPORTED, "idx_dim must be 16 (got %d)", c->idx_dim);
+  if (c->kv_dtype != SPA_BF16 && c->kv_dtype != SPA_F32)
+    return fail(SPA_ERR_UNSUPPORTED, "kv_dtype must be SPA_BF16 or SPA_F32 (got %d)", c->kv_dtype);
+  if (c->n_kv_heads < 1 || c->n_kv_heads > spa::kMaxKvHeads)
+    return fail(SPA_ERR_UNSUPPORTED, "n_kv_heads must be in [1, %d] (got %d)", spa::kMaxKvHeads, c->n_kv_heads);
+  if (c->n_q_heads < 1 || c->n_q_heads % c->n_kv_heads != 0)
+    return fail(SPA_ERR_INVALID_ARG, "n_q_heads (%d) must be a positive multiple of n_kv_heads (%d)",
+                c->n_q_heads, c->n_kv_heads);
+  const int G = c->n_q_heads / c->n_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8)
+    return fail(SPA_ERR_UNSUPPORTED, "GQA group size must be 1, 2, 4 or 8 (got %d)", G);
+  if (c->max_batch < 1 || (int64_t)c->max_batch * c->n_kv_heads > 65535)
+    return fail(SPA_ERR_INVALID_ARG, "max_batch must be >= 1 with max_batch*n_kv_heads <= 65535 (got %d)",
+                c->max_batch);
+  if (c->max_ctx < 1 || c->max_ctx > spa::kMaxCtx)
+    return fail(SPA_ERR_INVALID_ARG, "max_ctx must be in [1, 2^24] (got %lld)", (long long)c->max_ctx);
+  if (!(c->rope_theta > 0.0) || !std::isfinite(c->rope_theta))
+    return fail(SPA_ERR_INVALID_ARG, "rope_theta must be positive and finite");
+  if (!std::isfinite(c->idx_scale)) return fail(SPA_ERR_INVALID_ARG, "idx_scale must be finite");
+  if (c->split_rows < 0 || c->split_rows % spa::kTile != 0)
+    return fail(SPA_ERR_INVALID_ARG, "split_rows must be 0 or a positive multiple of %d (got %d)", spa::kTile,
+                c->split_rows);
+  if (!c->P_q || !c->P_k) return fail(SPA_ERR_INVALID_ARG, "P_q and P_k must be device pointers");
+  if (!aligned16(c->P_q) || !aligned16(c->P_k)) return fail(SPA_ERR_INVALID_ARG, "P_q/P_k must be 16-byte aligned");
+  return SPA_OK;
+}
+
+template <class F>
+spa_status run(spa_ctx* h, int kid, cudaStream_t st, const char* name, F&& f) {
+  const bool timed = h->prof && h->ev_next < kEventPairs;
+  if (timed) cudaEventRecord(h->ev[2 * h->ev_next], st);
+  cudaError_t e = f();
+  if (timed) {
+    cudaEventRecord(h->ev[2 * h->ev_next + 1], st);
+    h->ev_kid[h->ev_next++] = kid;
+  }
+  ++h->launches;
+  if (e != cudaSuccess) return cuda_fail(e, name);
+  return SPA_OK;
+}
+
+struct StepArgs {
+  const void* q_pre;
+  const void* idx_cache;
+  const uint8_t* head_mask;
+  const int64_t* seq_lens;
+  int B;
+  int64_t max_seq_len;
+  float p;
+  int n_sink, window;
+};
+
+spa_status check_step(spa_ctx* h, const StepArgs& a, spa::StepParams* P) {
+  if (!h) return fail(SPA_ERR_INVALID_ARG, "handle is NULL");
+  if (!a.q_pre || !a.idx_cache || !a.seq_lens || !a.head_mask)
+    return fail(SPA_ERR_INVALID_ARG, "q_pre, idx_cache, seq_lens and head_mask must be non-NULL");
+  if (!aligned16(a.q_pre) || !aligned16(a.idx_cache) || ((uintptr_t)a.seq_lens & 7u))
+    return fail(SPA_ERR_INVALID_ARG, "q_pre/idx_cache must be 16-byte aligned, seq_lens 8-byte aligned");
+  if (a.B < 1 || a.B > h->cfg.max_batch)
+    return fail(SPA_ERR_INVALID_ARG, "B must be in [1, max_batch=%d] (got %d)", h->cfg.max_batch, a.B);
+  if (!(a.p > 0.f) || !(a.p <= 1.f)) return fail(SPA_ERR_INVALID_ARG, "p must be in (0, 1] (got %g)", (double)a.p);
+  if (a.n_sink < 0 || a.window < 0) return fail(SPA_ERR_INVALID_ARG, "n_sink and window must be >= 0");
+  if ((int64_t)a.n_sink + a.window < 1)
+    return fail(SPA_ERR_INVALID_ARG, "n_sink + window must be >= 1 (a streaming head needs a token)");
+  if (a.max_seq_len < 0 || a.max_seq_len > h->cfg.max_ctx)
+    return fail(SPA_ERR_INVALID_ARG, "max_seq_len must be in [0, max_ctx=%lld] (got %lld)",
+                (long long)h->cfg.max_ctx, (long long)a.max_seq_len);
+  std::memset(P, 0, sizeof *P);
+  const int Hkv = h->cfg.n_kv_heads;
+  for (int g = 0; g < Hkv; ++g) {
+    P->is_ret[g] = a.head_mask[g] ? 1 : 0;
+    if (P->is_ret[g]) P->ret_heads[P->n_ret++] = g;
+  }
+  P->q_pre = a.q_pre;
+  P->idx_cache = static_cast<const uint16_t*>(a.idx_cache);
+  P->seq_lens = a.seq_lens;
+  P->B = a.B;
+  P->Hq = h->cfg.n_q_heads;
+  P->Hkv = Hkv;
+  P->G = h->G;
+  P->Lmax = h->cfg.max_ctx;
+  P->Lcap = (int)(a.max_seq_len ? a.max_seq_len : h->cfg.max_ctx);
+  P->n_chunks = (P->Lcap + spa::kChunk - 1) / spa::kChunk;
+  P->n_slices = a.B * Hkv;
+  P->p = a.p;
+  P->keep_all = a.p >= 1.f ? 1 : 0;
+  P->n_sink = a.n_sink;
+  P->window = a.window;
+  P->idx_scale_log2 = h->idx_scale * 1.4426950408889634f;
+  P->attn_scale_log2 = (float)(1.4426950408889634 / std::sqrt(128.0));
+  P->split_rows = h->split_rows;
+  P->ws = h->ws;
+  return SPA_OK;
+}
+
+spa_status run_selection(spa_ctx* h, spa::StepParams& P, cudaStream_t st) {
+  spa_status r;
+  if ((r = run(h, SPA_K_PROLOGUE, st, "prologue", [&] { return spa::launch_prologue(P, h->cfg.kv_dtype, st); })))
+    return r;
+  if (P.n_ret == 0) return SPA_OK;
+  if ((r = run(h, SPA_K_SCORE, st, "index score", [&] { return spa::launch_score(P, st); }))) return r;
+  if ((r = run(h, SPA_K_MASS, st, "index mass", [&] { return spa::launch_mass(P, st); }))) return r;
+  if ((r = run(h, SPA_K_THRESHOLD, st, "threshold", [&] { return spa::launch_threshold(P, st); }))) return r;
+  if ((r = run(h, SPA_K_COMPACT, st, "compact", [&] { return spa::launch_compact(P, st); }))) return r;
+  return SPA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* spa_last_error(void) { return g_err.c_str(); }
+
+spa_status spa_workspace_size(const spa_config* cfg, size_t* bytes) {
+  spa_status r = check_config(cfg);
+  if (r) return r;
+  if (!bytes) return fail(SPA_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = plan(*cfg, cfg->split_rows ? cfg->split_rows : spa::kDefaultSplitRows).total;
+  return SPA_OK;
+}
+
+spa_status spa_create(spa_handle* out, const spa_config* cfg) {
+  if (!out) return fail(SPA_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  spa_status r = check_config(cfg);
+  if (r) return r;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0)
+    return fail(SPA_ERR_UNSUPPORTED, "libspa is built for sm_100a (B200); device %d is sm_%d%d", dev, major, minor);
+
+  spa_ctx* h = new (std::nothrow) spa_ctx;
+  if (!h) return fail(SPA_ERR_WORKSPACE, "out of host memory");
+  h->cfg = *cfg;
+  h->G = cfg->n_q_heads / cfg->n_kv_heads;
+  h->split_rows = cfg->split_rows ? cfg->split_rows : spa::kDefaultSplitRows;
+  h->idx_scale = cfg->idx_scale > 0.f ? cfg->idx_scale : 0.25f;
+  h->device = dev;
+  cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev);
+  const Layout L = plan(*cfg, h->split_rows);
+  e = cudaMalloc(&h->mem, L.total);
+  if (e != cudaSuccess) {
+    delete h;
+    return fail(SPA_ERR_WORKSPACE, "cudaMalloc of %zu workspace bytes failed: %s", L.total, cudaGetErrorString(e));
+  }
+  h->mem_bytes = L.total;
+  char* base = static_cast<char*>(h->mem);
+  spa::Workspace& w = h->ws;
+  w.P_q = (float*)(base + L.off[0]);
+  w.P_k = (float*)(base + L.off[1]);
+  w.inv_freq = (double*)(base + L.off[2]);
+  w.q_rot = (float*)(base + L.off[3]);
+  w.q_idx = (float*)(base + L.off[4]);
+  w.stats = (float2*)(base + L.off[5]);
+  w.pi = (float*)(base + L.off[6]);
+  w.hist1 = (unsigned long long*)(base + L.off[7]);
+  w.cand = (uint2*)(base + L.off[8]);
+  w.chunk_gt = (int*)(base + L.off[9]);
+  w.chunk_off = (int*)(base + L.off[10]);
+  w.st = (spa::SliceState*)(base + L.off[11]);
+  w.list = (int*)(base + L.off[12]);
+  w.item_base = (int*)(base + L.off[13]);
+  w.part = (float*)(base + L.off[14]);
+  w.dev_err = (unsigned*)(base + L.off[15]);
+  w.max_items = L.max_items;
+  h->n_chunks_max = L.n_chunks_max;
+
+  double invf[64];
+  for (int i = 0; i < 64; ++i) invf[i] = std::pow(cfg->rope_theta, -2.0 * i / 128.0);
+  const size_t pq = (size_t)cfg->n_q_heads * 16 * 128 * 4, pk = (size_t)cfg->n_kv_heads * 16 * 128 * 4;
+  if ((e = cudaMemcpy(w.P_q, cfg->P_q, pq, cudaMemcpyDeviceToDevice)) != cudaSuccess ||
+      (e = cudaMemcpy(w.P_k, cfg->P_k, pk, cudaMemcpyDeviceToDevice)) != cudaSuccess ||
+      (e = cudaMemcpy(w.inv_freq, invf, sizeof invf, cudaMemcpyHostToDevice)) != cudaSuccess ||
+      (e = cudaMemset(w.dev_err, 0, 4)) != cudaSuccess || (e = cudaDeviceSynchronize()) != cudaSuccess) {
+    cudaFree(h->mem);
+    delete h;
+    return cuda_fail(e, "spa_create: copying projectors");
+  }
+  const int occ = spa::attend_setup(cfg->kv_dtype, h->G, cfg->max_batch * cfg->n_kv_heads);
+  if (occ < 1) {
+    cudaFree(h->mem);
+    delete h;
+    return fail(SPA_ERR_UNSUPPORTED, "attention kernel cannot be resident with this configuration");
+  }
+  h->attend_occ = occ;
+  *out = h;
+  return SPA_OK;
+}
+
+spa_status spa_destroy(spa_handle h) {
+  if (!h) return SPA_OK;
+  cudaDeviceSynchronize();
+  for (cudaEvent_t ev : h->ev) cudaEventDestroy(ev);
+  cudaError_t e = cudaFree(h->mem);
+  delete h;
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFree");
+  return SPA_OK;
+}
+
+spa_status spa_index_append(spa_handle h, const void* k_pre, const int64_t* start_pos, int B, int T,
+                            void* idx_cache, spa_stream stream) {
+  if (!h) return fail(SPA_ERR_INVALID_ARG, "handle is NULL");
+  if (!k_pre || !start_pos || !idx_cache) return fail(SPA_ERR_INVALID_ARG, "k_pre, start_pos, idx_cache must be non-NULL");
+  if (!aligned16(k_pre) || !aligned16(idx_cache) || ((uintptr_t)start_pos & 7u))
+    return fail(SPA_ERR_INVALID_ARG, "k_pre/idx_cache must be 16-byte aligned, start_pos 8-byte aligned");
+  if (B < 1 || B > h->cfg.max_batch)
+    return fail(SPA_ERR_INVALID_ARG, "B must be in [1, max_batch=%d] (got %d)", h->cfg.max_batch, B);
+  if (T < 1 || (int64_t)T > h->cfg.max_ctx)
+    return fail(SPA_ERR_INVALID_ARG, "T must be in [1, max_ctx] (got %d)", T);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return run(h, SPA_K_INDEX_APPEND, st, "index append", [&] {
+    return spa::launch_index_append(k_pre, start_pos, B, T, h->cfg.n_kv_heads, h->cfg.max_ctx, h->cfg.kv_dtype,
+                                    h->ws.P_k, static_cast<uint16_t*>(idx_cache), h->ws.dev_err, st);
+  });
+}
+
+spa_status spa_select(spa_handle h, const void* q_pre, const void* idx_cache, const uint8_t* head_mask,
+                      const int64_t* seq_lens, int B, int64_t max_seq_len, float p, int n_sink, int window,
+                      int32_t* sel_idx, int32_t* sel_count, spa_stream stream) {
+  spa::StepParams P;
+  spa_status r = check_step(h, StepArgs{q_pre, idx_cache, head_mask, seq_lens, B, max_seq_len, p, n_sink, window}, &P);
+  if (r) return r;
+  if (!sel_idx || !sel_count) return fail(SPA_ERR_INVALID_ARG, "sel_idx and sel_count must be non-NULL");
+  if (!aligned16(sel_idx) || ((uintptr_t)sel_count & 3u))
+    return fail(SPA_ERR_INVALID_ARG, "sel_idx must be 16-byte aligned, sel_count 4-byte aligned");
+  P.sel_list = sel_idx;
+  P.sel_count = sel_count;
+  return run_selection(h, P, reinterpret_cast<cudaStream_t>(stream));
+}
+
+spa_status spa_decode(spa_handle h, const void* q_pre, const void* k_cache, const void* v_cache,
+                      const void* idx_cache, const uint8_t* head_mask, const int64_t* seq_lens, int B,
+                      int64_t max_seq_len, float p, int n_sink, int window, float* out, int32_t* sel_count_opt,
+                      spa_stream stream) {
+  spa::StepParams P;
+  spa_status r = check_step(h, StepArgs{q_pre, idx_cache, head_mask, seq_lens, B, max_seq_len, p, n_sink, window}, &P);
+  if (r) return r;
+  if (!k_cache || !v_cache || !out) return fail(SPA_ERR_INVALID_ARG, "k_cache, v_cache and out must be non-NULL");
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return fail(SPA_ERR_INVALID_ARG, "k_cache, v_cache and out must be 16-byte aligned");
+  if (sel_count_opt && ((uintptr_t)sel_count_opt & 3u)) return fail(SPA_ERR_INVALID_ARG, "sel_count_opt misaligned");
+  P.k_cache = k_cache;
+  P.v_cache = v_cache;
+  P.out = out;
+  P.sel_list = h->ws.list;
+  P.sel_count = nullptr;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if ((r = run_selection(h, P, st))) return r;
+  // upper bound on splits: every slice has at most Lcap rows
+  const int64_t per_slice = (P.Lcap + P.split_rows - 1) / P.split_rows;
+  const int64_t max_items = per_slice * P.n_slices;
+  const int64_t cap = (int64_t)h->num_sms * h->attend_occ;
+  const int grid = (int)(max_items < cap ? max_items : cap);
+  if ((r = run(h, SPA_K_ATTEND, st, "attend", [&] { return spa::launch_attend(P, h->cfg.kv_dtype, grid, st); })))
+    return r;
+  P.sel_count = sel_count_opt;
+  return run(h, SPA_K_COMBINE, st, "combine", [&] { return spa::launch_combine(P, st); });
+}
+
+spa_status spa_device_status(spa_handle h, spa_stream stream) {
+  if (!h) return fail(SPA_ERR_INVALID_ARG, "handle is NULL");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned flags = 0;
+  if ((e = cudaMemcpy(&flags, h->ws.dev_err, 4, cudaMemcpyDeviceToHost)) != cudaSuccess) return cuda_fail(e, "read status");
+  if (flags) {
+    if ((e = cudaMemset(h->ws.dev_err, 0, 4)) != cudaSuccess) return cuda_fail(e, "clear status");
+    if (flags & spa::kErrInternal)
+      return fail(SPA_ERR_CUDA, "internal consistency check failed in the selection kernels (flags 0x%x)", flags);
+    return fail(SPA_ERR_DEVICE_RANGE, "device range check failed:%s%s",
+                (flags & spa::kErrSeqLen) ? " seq_lens outside [1, max_seq_len]" : "",
+                (flags & spa::kErrStartPos) ? " start_pos + t outside [0, max_ctx)" : "");
+  }
+  return SPA_OK;
+}
+
+spa_status spa_set_profiling(spa_handle h, int enable) {
+  if (!h) return fail(SPA_ERR_INVALID_ARG, "handle is NULL");
+  if (enable && h->ev.empty()) {
+    h->ev.resize(2 * kEventPairs);
+    h->ev_kid.resize(kEventPairs);
+    for (auto& ev : h->ev) {
+      cudaError_t e = cudaEventCreate(&ev);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaEventCreate");
+    }
+  }
+  h->prof = enable != 0;
+  h->ev_next = 0;
+  return SPA_OK;
+}
+
+spa_status spa_profile_read(spa_handle h, int kernel_id, double* total_ms, int64_t* launches) {
+  if (!h || !total_ms || !launches) return fail(SPA_ERR_INVALID_ARG, "NULL argument");
+  double sum = 0.0;
+  int64_t n = 0;
+  for (size_t i = 0; i < h->ev_next; ++i) {
+    if (h->ev_kid[i] != kernel_id) continue;
+    cudaError_t e = cudaEventSynchronize(h->ev[2 * i + 1]);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+    float ms = 0.f;
+    e = cudaEventElapsedTime(&ms, h->ev[2 * i], h->ev[2 * i + 1]);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventElapsedTime");
+    sum += ms;
+    ++n;
+  }
+  *total_ms = sum;
+  *launches = n;
+  return SPA_OK;
+}
+
+const char* spa_kernel_name(int kernel_id) {
+  static const char* names[SPA_K_COUNT] = {"index_append", "prologue", "index_score", "index_mass",
+                                           "threshold",    "compact",  "attend",      "combine"};
+  return (kernel_id >= 0 && kernel_id < SPA_K_COUNT) ? names[kernel_id] : "";
+}
+
+spa_status spa_launch_count(spa_handle h, int64_t* launches) {
+  if (!h || !launches) return fail(SPA_ERR_INVALID_ARG, "NULL argument");
+  *launches = h->launches;
+  return SPA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,167 @@
+// Internal definitions shared by the libspa kernels and the host entry points.
+// Not part of the public ABI (see include/spa.h).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace spa {
+
+constexpr int kHeadDim = 128;          // d
+constexpr int kIdxDim = 16;            // r, the index dimension
+constexpr int kMaxKvHeads = 64;
+constexpr int kMaxGroup = 8;           // largest GQA group size G
+constexpr int64_t kMaxCtx = int64_t(1) << 24;
+
+// Selection works on chunks of kChunk consecutive tokens of one (b, kv head) slice.
+constexpr int kChunk = 4096;
+constexpr int kSelThreads = 256;
+constexpr int kTokPerThread = kChunk / kSelThreads;  // 16
+constexpr int kMaxChunks = int(kMaxCtx / kChunk);    // 4096
+
+// Radix digits of the fp32 bit pattern u of a probability in [0, 1]:
+// bits 31..30 are zero, digit1 = u >> 18 (12 bits), digit2 = (u >> 6) & 0xfff
+// (12 bits), digit3 = u & 0x3f (6 bits).
+constexpr int kBins1 = 4096;
+constexpr int kBins2 = 4096;
+constexpr int kBins3 = 64;
+constexpr float kMassScale = 1152921504606846976.0f;  // 2^60: mass unit is 2^-60
+
+// Attention splits ("items") cover up to split_rows rows of one slice; rows are
+// staged through shared memory kTile rows at a time.
+constexpr int kTile = 64;
+constexpr int kAttnThreads = 256;
+constexpr int kDefaultSplitRows = 512;
+
+// Device status bits.
+constexpr unsigned kErrSeqLen = 1u;
+constexpr unsigned kErrStartPos = 2u;
+constexpr unsigned kErrInternal = 4u;
+
+// Per (b, kv head) selection state.  Written by the threshold kernels, read by
+// compaction and attention.
+struct __align__(16) SliceState {
+  unsigned long long q_total;   // sum of quantised masses (units of 2^-60)
+  unsigned long long target;    // ceil(p * q_total)
+  unsigned long long m_above;   // mass of all tokens in digit1 bins above b1
+  int b1;                       // round-1 bin holding the cut; -1 = keep everything
+  unsigned tau_bits;            // fp32 bits of the cut probability tau
+  int pos_cut;                  // tied tokens (prob == tau) are kept iff pos <= pos_cut
+  int count;                    // listed tokens (kept, outside sinks/window)
+  unsigned ticket_mass;         // last-block tickets
+  unsigned ticket_thr;
+  unsigned cand_count;          // candidates appended (tokens in bin b1)
+  int pad_;
+};
+
+// Device workspace carved out of one allocation.
+struct Workspace {
+  float* P_q;            // [Hq][16][128]
+  float* P_k;            // [Hkv][16][128]
+  double* inv_freq;      // [64]
+  float* q_rot;          // [Bm][Hq][128]
+  float* q_idx;          // [Bm][Hq][16]
+  float2* stats;         // [Bm*Hkv][n_chunks_max][G]  (m in log2 units, z)
+  float* pi;             // [Bm*Hkv][Lmax]
+  unsigned long long* hist1;  // [Bm*Hkv][kBins1]
+  uint2* cand;           // [Bm*Hkv][Lmax]  (prob bits, position)
+  int* chunk_gt;         // [Bm*Hkv][n_chunks_max]
+  int* chunk_off;        // [Bm*Hkv][n_chunks_max]
+  SliceState* st;        // [Bm*Hkv]
+  int* list;             // [Bm*Hkv][Lmax]  selected positions (decode)
+  int* item_base;        // [Bm*Hkv + 1]
+  float* part;           // [max_items][G][kHeadDim + 2]
+  unsigned* dev_err;     // [1]
+  int64_t max_items;
+};
+
+// Arguments common to the selection / attention kernels of one call.
+struct StepParams {
+  const void* q_pre;
+  const void* k_cache;
+  const void* v_cache;
+  const uint16_t* idx_cache;
+  const int64_t* seq_lens;
+  float* out;
+  int* sel_list;         // [B*Hkv][Lmax] output list (workspace or caller's)
+  int* sel_count;        // [B*Hkv] or null
+  int B, Hq, Hkv, G;
+  int64_t Lmax;          // cache row capacity (row stride of the caches)
+  int Lcap;              // max_seq_len of this call
+  int n_chunks;          // ceil(Lcap / kChunk)
+  int n_slices;          // B * Hkv
+  float p;
+  int keep_all;          // p >= 1
+  int n_sink, window;
+  float idx_scale_log2;  // idx_scale * log2(e)
+  float attn_scale_log2; // log2(e) / sqrt(128)
+  int split_rows;
+  int n_ret;
+  int ret_heads[kMaxKvHeads];
+  unsigned char is_ret[kMaxKvHeads];
+  Workspace ws;
+};
+
+// ---------------------------------------------------------------- helpers
+__device__ __forceinline__ int load_len(const int64_t* seq_lens, int b, int Lcap, unsigned* err) {
+  int64_t L = seq_lens[b];
+  if (L < 1 || L > Lcap) {
+    atomicOr(err, kErrSeqLen);
+    L = L < 1 ? 1 : Lcap;
+  }
+  return int(L);
+}
+
+// Sinks are [0, n_s); the window is [w_lo, L).  w_lo >= n_s so the two never overlap.
+struct SinkWindow {
+  int n_s, w_lo, L;
+  __device__ __forceinline__ SinkWindow(int L_, int n_sink, int window) : L(L_) {
+    n_s = n_sink < L_ ? n_sink : L_;
+    long long lo = (long long)L_ - (long long)window;
+    w_lo = lo > n_s ? int(lo) : n_s;
+  }
+  __device__ __forceinline__ int n_contig() const { return n_s + (L - w_lo); }
+  __device__ __forceinline__ bool always(int j) const { return j < n_s || j >= w_lo; }
+  __device__ __forceinline__ int contig_pos(int v) const { return v < n_s ? v : w_lo + (v - n_s); }
+};
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+template <typename T> struct Elem;
+template <> struct Elem<__nv_bfloat16> {
+  static __device__ __forceinline__ float get(const __nv_bfloat16* p, int i) { return __bfloat162float(p[i]); }
+};
+template <> struct Elem<float> {
+  static __device__ __forceinline__ float get(const float* p, int i) { return p[i]; }
+};
+
+__device__ __forceinline__ unsigned long long mass_q(float pr) {
+  return __float2ull_rn(pr * kMassScale);
+}
+
+// Merge two online-softmax states (m in log2 units).
+__device__ __forceinline__ void merge_mz(float& m, float& z, float m2, float z2) {
+  float mn = fmaxf(m, m2);
+  if (mn == -INFINITY) { m = mn; z = 0.f; return; }
+  z = z * exp2f(m - mn) + z2 * exp2f(m2 - mn);
+  m = mn;
+}
+
+}  // namespace spa
+
+// Launchers (defined in the kernel translation units).
+namespace spa {
+cudaError_t launch_index_append(const void* k_pre, const int64_t* start_pos, int B, int T, int Hkv,
+                                int64_t Lmax, int kv_dtype, const float* P_k, uint16_t* idx_cache,
+                                unsigned* dev_err, cudaStream_t st);
+cudaError_t launch_prologue(const StepParams& P, int kv_dtype, cudaStream_t st);
+cudaError_t launch_score(const StepParams& P, cudaStream_t st);
+cudaError_t launch_mass(const StepParams& P, cudaStream_t st);
+cudaError_t launch_threshold(const StepParams& P, cudaStream_t st);
+cudaError_t launch_compact(const StepParams& P, cudaStream_t st);
+cudaError_t launch_attend(const StepParams& P, int kv_dtype, int grid, cudaStream_t st);
+cudaError_t launch_combine(const StepParams& P, cudaStream_t st);
+int attend_setup(int kv_dtype, int G, int max_slices);
+}  // namespace spa

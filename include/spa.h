@@ -1,0 +1,209 @@
+/*
+ * spa.h -- C ABI of libspa: one decode step of head-partitioned sparse attention
+ * on an NVIDIA B200 (sm_100a).
+ *
+ * The method ("Full Attention Strikes Back" (RTPurbo summary), Methodology §1-§3,
+ * §5) splits the KV heads of an attention layer in two:
+ *   - streaming (local) heads attend to the attention sinks plus a sliding window;
+ *   - retrieval heads score every cached token in a 16-dim index space built from
+ *     the keys *before* RoPE, keep the smallest set of tokens whose index
+ *     probability mass reaches p (top-p, not a fixed top-k), and run exact softmax
+ *     attention over that set plus the sinks and window.
+ * Conventions fixed by this library where the pages are silent:
+ *   - index probabilities are computed per query head (softmax of idx_scale *
+ *     <P_q[h] q_pre[h], idx_j>) and averaged over the heads of each GQA group
+ *     ("Autonomy of Heads" summary, Deployment strategy: group mean), giving
+ *     one selected set per (sequence, KV head);
+ *   - tokens are ranked by (probability desc, position asc); the kept set is the
+ *     shortest prefix whose mass reaches p (token kept iff the mass ranked ahead
+ *     of it is < p); p >= 1 keeps every token;
+ *   - sinks are positions [0, n_sink); the window is the last `window` positions,
+ *     the current token (position seq_len-1) included; both are always attended;
+ *   - RoPE is rotate-half with inv_freq_i = rope_theta^(-2i/128), applied by the
+ *     library to the query at position seq_len-1.  k_cache holds post-RoPE keys
+ *     written by the caller; the index cache is built from pre-RoPE keys.
+ *
+ * Memory and ownership
+ *   Every tensor pointer is a DEVICE pointer owned by the caller, except
+ *   `head_mask` (HOST memory, read during the call) and the handle.  Tensors are
+ *   dense, row-major, 16-byte aligned.  Storage dtype of q/k/v is the handle's
+ *   kv_dtype (SPA_BF16 or SPA_F32); the index cache is always bf16; outputs are
+ *   float32.  The handle owns a device workspace allocated in spa_create.
+ *
+ * Execution
+ *   Every compute call only enqueues kernels on `stream` (no host sync, no
+ *   device->host copy), so a call can be captured in a CUDA graph.  Calls on one
+ *   handle share its workspace: do not run two of them concurrently on
+ *   different streams.  Argument errors are reported before anything is
+ *   launched.  Values that live on the device (seq_lens, start_pos) are range
+ *   checked by the kernels: an out-of-range value is clamped into range, a
+ *   device status bit is set, and spa_device_status() reports it.
+ *
+ * Errors
+ *   Every call returns SPA_OK (0) or a negative spa_status; spa_last_error()
+ *   returns a thread-local message for the last failing call.  No C++ exception
+ *   crosses this boundary.  There is no CPU fallback: without a usable CUDA
+ *   device, calls that need one return SPA_ERR_CUDA.
+ */
+#ifndef SPA_H_
+#define SPA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SPA_API __attribute__((visibility("default")))
+#else
+#define SPA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int spa_status;
+#define SPA_OK 0
+#define SPA_ERR_INVALID_ARG (-1)    /* null/misaligned pointer, bad size, p out of (0,1] ... */
+#define SPA_ERR_UNSUPPORTED (-2)    /* head_dim != 128, idx_dim != 16, unsupported GQA ratio or dtype */
+#define SPA_ERR_WORKSPACE (-3)      /* workspace allocation failed / request exceeds the handle's capacity */
+#define SPA_ERR_CUDA (-4)           /* a CUDA runtime call or kernel launch failed */
+#define SPA_ERR_DEVICE_TIMEOUT (-5) /* reserved: a bounded device-side wait gave up */
+#define SPA_ERR_DEVICE_RANGE (-6)   /* spa_device_status: a device-resident length/position was out of range */
+
+/* storage dtypes of q / k / v */
+#define SPA_BF16 0
+#define SPA_F32 1
+
+typedef struct spa_ctx* spa_handle;
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* spa_stream;
+
+typedef struct {
+  int max_batch;      /* largest B a call may pass (>= 1) */
+  int n_q_heads;      /* Hq */
+  int n_kv_heads;     /* Hkv; Hq / Hkv (the GQA group size G) must be 1, 2, 4 or 8; Hkv <= 64 */
+  int head_dim;       /* must be 128 */
+  int idx_dim;        /* index dimension r; must be 16 */
+  int kv_dtype;       /* SPA_BF16 or SPA_F32 */
+  int64_t max_ctx;    /* Lmax: cache capacity in tokens per (sequence, KV head); 1 <= Lmax <= 2^24 */
+  double rope_theta;  /* RoPE base (e.g. 500000) */
+  float idx_scale;    /* index softmax temperature; <= 0 selects 1/sqrt(idx_dim) = 0.25 */
+  int split_rows;     /* rows of K/V per attention split; 0 selects the default (a multiple of 64) */
+  const float* P_q;   /* device [Hq][16][128] float32 query projectors; copied at create */
+  const float* P_k;   /* device [Hkv][16][128] float32 key projectors; copied at create */
+} spa_config;
+
+/* Validate `cfg`, allocate the device workspace on the current device and copy
+ * the projectors.  Synchronous.  On failure *out is NULL. */
+SPA_API spa_status spa_create(spa_handle* out, const spa_config* cfg);
+
+/* Free the workspace (synchronises the device first).  NULL is accepted. */
+SPA_API spa_status spa_destroy(spa_handle h);
+
+/* Bytes of device workspace spa_create would allocate for `cfg`. Host only. */
+SPA_API spa_status spa_workspace_size(const spa_config* cfg, size_t* bytes);
+
+/* Thread-local text of the last error ("" if none).  Valid until the next call
+ * on this thread. */
+SPA_API const char* spa_last_error(void);
+
+/*
+ * Index append ("Full Attention Strikes Back", Methodology §2: a 16-dim projector
+ * applied to the key features before RoPE is injected).
+ *   idx_cache[b][g][start_pos[b] + t][r] = bf16_rne( sum_d P_k[g][r][d] * k_pre[b][g][t][d] )
+ * for b < B, g < Hkv, t < T, r < 16; each product is rounded to float32 and added
+ * to a float32 running sum in ascending d (no fused multiply-add), so the code is
+ * reproducible bit for bit.
+ *   k_pre     device [B][Hkv][T][128], kv_dtype: pre-RoPE keys of T new tokens
+ *   start_pos device int64 [B]: cache position of token t = 0 for each sequence
+ *   idx_cache device bf16 [max_batch][Hkv][Lmax][16] (32 bytes per row), written
+ * Rows whose position falls outside [0, Lmax) are skipped and flagged (device status).
+ * Works for a prefill chunk (T large) and for the decode token (T = 1).
+ */
+SPA_API spa_status spa_index_append(spa_handle h, const void* k_pre, const int64_t* start_pos,
+                            int B, int T, void* idx_cache, spa_stream stream);
+
+/*
+ * Top-p token selection for the retrieval heads ("Full Attention Strikes Back",
+ * Methodology §2-§3, §5 histogram thresholding).  For each b < B and each KV head
+ * g with head_mask[g] != 0, with L = seq_lens[b]:
+ *   pi_j = mean_{h in group g} softmax_j( idx_scale * <P_q[h] q_pre[b][h], idx_cache[b][g][j]> ), j < L
+ *   T    = shortest prefix of (pi desc, position asc) whose mass reaches p (all of [0,L) if p >= 1)
+ *   sel_idx[b][g][0 .. count)  = T minus sinks/window, positions ascending
+ *   sel_count[b * Hkv + g]     = count
+ * Streaming heads get count 0.  Entries of sel_idx at or beyond the count are
+ * left unspecified.
+ *   q_pre      device [B][Hq][128], kv_dtype: pre-RoPE queries of the current token
+ *   idx_cache  device bf16 [max_batch][Hkv][Lmax][16]
+ *   head_mask  HOST uint8 [Hkv]: 1 = retrieval head, 0 = streaming head
+ *   seq_lens   device int64 [B]: context length including the current token, 1..max_seq_len
+ *   max_seq_len host upper bound on seq_lens for this call (sizes the launch); 0 = Lmax
+ *   p          in (0, 1]; n_sink >= 0; window >= 0; n_sink + window >= 1
+ *   sel_idx    device int32 [B][Hkv][Lmax]; sel_count device int32 [B * Hkv]
+ * Selection is computed in float32 probabilities with exact integer mass sums
+ * (probabilities quantised to multiples of 2^-60) and is deterministic.
+ */
+SPA_API spa_status spa_select(spa_handle h, const void* q_pre, const void* idx_cache,
+                      const uint8_t* head_mask, const int64_t* seq_lens, int B,
+                      int64_t max_seq_len, float p, int n_sink, int window,
+                      int32_t* sel_idx, int32_t* sel_count, spa_stream stream);
+
+/*
+ * One decode step ("Full Attention Strikes Back", Methodology §1-§3, §5;
+ * exact token attention as in "Hierarchical Global Attention", §4).
+ * For every b < B and query head h (KV head g = h / G), with L = seq_lens[b]:
+ *   S   = sinks ∪ window                    (streaming head)
+ *       = sinks ∪ window ∪ T               (retrieval head, T as in spa_select)
+ *   out[b][h] = sum_{j in S} softmax_j( <RoPE(q_pre[b][h], L-1), k_cache[b][g][j]> / sqrt(128) ) v_cache[b][g][j]
+ *   q_pre, idx_cache, head_mask, seq_lens, max_seq_len, p, n_sink, window: as in spa_select
+ *   k_cache, v_cache device [max_batch][Hkv][Lmax][128], kv_dtype (k post-RoPE)
+ *   out             device float32 [B][Hq][128], written
+ *   sel_count_opt   NULL, or device int32 [B * Hkv] receiving the selected counts
+ * Attention is split over rows (split-K), each split keeping an online-softmax
+ * state (m, l, acc) that a combine kernel merges with log-sum-exp weights.
+ */
+SPA_API spa_status spa_decode(spa_handle h, const void* q_pre, const void* k_cache, const void* v_cache,
+                      const void* idx_cache, const uint8_t* head_mask, const int64_t* seq_lens,
+                      int B, int64_t max_seq_len, float p, int n_sink, int window,
+                      float* out, int32_t* sel_count_opt, spa_stream stream);
+
+/*
+ * Synchronise `stream`, then read and clear the handle's device status word.
+ * Returns SPA_ERR_DEVICE_RANGE (with the offending field named in
+ * spa_last_error) if a kernel clamped an out-of-range seq_lens/start_pos value
+ * since the last check, else SPA_OK.
+ */
+SPA_API spa_status spa_device_status(spa_handle h, spa_stream stream);
+
+/* ---- instrumentation (used by the benchmark; off by default) ---- */
+
+/* Kernel ids for spa_profile_read / spa_kernel_name. */
+#define SPA_K_INDEX_APPEND 0
+#define SPA_K_PROLOGUE 1
+#define SPA_K_SCORE 2
+#define SPA_K_MASS 3
+#define SPA_K_THRESHOLD 4
+#define SPA_K_COMPACT 5
+#define SPA_K_ATTEND 6
+#define SPA_K_COMBINE 7
+#define SPA_K_COUNT 8
+
+/* When enabled, every kernel launch of this handle is bracketed by two CUDA
+ * events recorded on the launch stream (a bounded pool; launches beyond it are
+ * not timed).  Enabling resets the pool. */
+SPA_API spa_status spa_set_profiling(spa_handle h, int enable);
+
+/* Synchronise the recorded events and return, for kernel `kernel_id`, the
+ * summed device time in milliseconds and the number of timed launches. */
+SPA_API spa_status spa_profile_read(spa_handle h, int kernel_id, double* total_ms, int64_t* launches);
+
+/* Name of a kernel id ("" if unknown). */
+SPA_API const char* spa_kernel_name(int kernel_id);
+
+/* Number of kernel launches this handle has issued since it was created. */
+SPA_API spa_status spa_launch_count(spa_handle h, int64_t* launches);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPA_H_ */

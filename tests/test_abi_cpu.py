@@ -1,0 +1,105 @@
+"""The C ABI library: it loads, exports what include/spa.h declares, and rejects
+bad arguments on the host before touching a GPU.  No compute calls here."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+from head_partitioned_sparse_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "spa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from head_partitioned_sparse_b200 import build
+    build.build()
+    return B.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^SPA_API\s+[\w\s\*]+?\b(spa_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("spa_create", "spa_destroy", "spa_index_append", "spa_select", "spa_decode",
+                     "spa_workspace_size", "spa_last_error", "spa_device_status"):
+        assert required in names
+    assert sorted(B.EXPORTED) == names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (spa_\w+)", out))
+    assert set(declared_functions()) <= exported
+    # nothing but the C ABI is exported by name
+    assert exported == set(declared_functions())
+
+
+def _cfg(**kw):
+    base = dict(max_batch=2, n_q_heads=8, n_kv_heads=2, max_ctx=4096, kv_dtype=B.SPA_BF16,
+                P_q=0x10000, P_k=0x20000)   # never dereferenced by the host checks
+    base.update(kw)
+    return B.make_config(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(head_dim=64), B.SPA_ERR_UNSUPPORTED),
+    (dict(idx_dim=8), B.SPA_ERR_UNSUPPORTED),
+    (dict(kv_dtype=7), B.SPA_ERR_UNSUPPORTED),
+    (dict(n_q_heads=6, n_kv_heads=2), B.SPA_ERR_UNSUPPORTED),     # G = 3
+    (dict(n_q_heads=32, n_kv_heads=2), B.SPA_ERR_UNSUPPORTED),    # G = 16
+    (dict(n_q_heads=7, n_kv_heads=2), B.SPA_ERR_INVALID_ARG),
+    (dict(max_ctx=0), B.SPA_ERR_INVALID_ARG),
+    (dict(max_ctx=(1 << 24) + 1), B.SPA_ERR_INVALID_ARG),
+    (dict(max_batch=0), B.SPA_ERR_INVALID_ARG),
+    (dict(split_rows=100), B.SPA_ERR_INVALID_ARG),
+    (dict(P_q=None), B.SPA_ERR_INVALID_ARG),
+    (dict(P_k=0x20004), B.SPA_ERR_INVALID_ARG),                    # misaligned
+    (dict(rope_theta=-1.0), B.SPA_ERR_INVALID_ARG),
+])
+def test_config_validation(lib, kw, status):
+    with pytest.raises(B.SpaError) as e:
+        B.spa_workspace_size(_cfg(**kw))
+    assert e.value.status == status
+    assert B.spa_last_error()
+
+
+def test_workspace_size_grows_with_context(lib):
+    a = B.spa_workspace_size(_cfg(max_ctx=4096))
+    b = B.spa_workspace_size(_cfg(max_ctx=8192))
+    assert 0 < a < b
+    # dominated by per-token buffers: probabilities, candidates, list (16 B/token/slice) + splits
+    assert b - a >= 2 * 2 * 4096 * 16
+
+
+def test_null_handle_is_rejected_without_a_device(lib):
+    with pytest.raises(B.SpaError) as e:
+        B.spa_decode(None, 16, 16, 16, 16, [1, 0], 16, 1, 0, 0.9, 4, 16, 16, None, stream=0)
+    assert e.value.status == B.SPA_ERR_INVALID_ARG
+    with pytest.raises(B.SpaError) as e:
+        B.spa_index_append(None, 16, 16, 1, 1, 16, stream=0)
+    assert e.value.status == B.SPA_ERR_INVALID_ARG
+    with pytest.raises(B.SpaError) as e:
+        B.spa_select(None, 16, 16, [1, 0], 16, 1, 0, 0.9, 4, 16, 16, 16, stream=0)
+    assert e.value.status == B.SPA_ERR_INVALID_ARG
+    assert B.spa_destroy(None) is None
+
+
+def test_kernel_names(lib):
+    names = [B.spa_kernel_name(i) for i in range(B.SPA_K_COUNT)]
+    assert names[B.SPA_K_ATTEND] == "attend" and all(names)
+    assert B.spa_kernel_name(99) == ""
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_create_without_device_fails_loudly(lib):
+    with pytest.raises(B.SpaError) as e:
+        B.spa_create(_cfg())
+    assert e.value.status in (B.SPA_ERR_CUDA, B.SPA_ERR_UNSUPPORTED)
