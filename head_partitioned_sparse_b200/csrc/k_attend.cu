@@ -233,37 +233,66 @@ __global__ void __launch_bounds__(kAttnThreads) k_attend(StepParams P) {
       }
       __syncthreads();
     }
-    // write the split's state
-    float* dst = P.ws.part + (size_t)item * G * (kHeadDim + 2);
+    // write the split's state: [acc 128][m][l][pad 2] per head
+    float* dst = P.ws.part + (size_t)item * G * kPartStride;
     if (pv_active)
 #pragma unroll
-      for (int k = 0; k < HP; ++k) dst[(h0 + k) * (kHeadDim + 2) + 2 + d] = acc[k];
+      for (int k = 0; k < HP; ++k) dst[(h0 + k) * kPartStride + d] = acc[k];
     if (tid < G) {
-      dst[tid * (kHeadDim + 2)] = mrun[tid];
-      dst[tid * (kHeadDim + 2) + 1] = lrun[tid];
+      dst[tid * kPartStride + kHeadDim] = mrun[tid];
+      dst[tid * kPartStride + kHeadDim + 1] = lrun[tid];
     }
   }
 }
 
+// One CTA per (slice, head): warp w merges the splits w, w + 8, ... of the slice
+// (lane = 4 dims), then warp states are merged in warp order.  Deterministic.
 template <int G>
-__global__ void __launch_bounds__(kHeadDim) k_combine(StepParams P) {
-  const int s = blockIdx.x;
+__global__ void __launch_bounds__(256) k_combine(StepParams P) {
+  __shared__ float wm[8], wl[8];
+  __shared__ __align__(16) float wacc[8][kHeadDim];
+  const int s = blockIdx.x / G, h = blockIdx.x % G;
   const int b = s / P.Hkv, g = s % P.Hkv;
-  const int d = threadIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int i0 = P.ws.item_base[s], i1 = P.ws.item_base[s + 1];
-  for (int h = 0; h < G; ++h) {
-    float M = -INFINITY;
-    for (int i = i0; i < i1; ++i) M = fmaxf(M, P.ws.part[((size_t)i * G + h) * (kHeadDim + 2)]);
-    float num = 0.f, den = 0.f;
-    for (int i = i0; i < i1; ++i) {
-      const float* pp = P.ws.part + ((size_t)i * G + h) * (kHeadDim + 2);
-      const float w = exp2f(pp[0] - M);
-      den = fmaf(w, pp[1], den);
-      num = fmaf(w, pp[2 + d], num);
-    }
-    P.out[((size_t)b * P.Hq + (size_t)g * G + h) * kHeadDim + d] = num / den;
+  float m = -INFINITY, l = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = i0 + warp; i < i1; i += 8) {
+    const float* pp = P.ws.part + ((size_t)i * G + h) * kPartStride;
+    const float4 a = *reinterpret_cast<const float4*>(pp + 4 * lane);
+    const float mi = pp[kHeadDim], li = pp[kHeadDim + 1];
+    const float mn = fmaxf(m, mi);
+    const float sa = exp2f(m - mn), sb = exp2f(mi - mn);
+    l = l * sa + li * sb;
+    acc.x = acc.x * sa + a.x * sb;
+    acc.y = acc.y * sa + a.y * sb;
+    acc.z = acc.z * sa + a.z * sb;
+    acc.w = acc.w * sa + a.w * sb;
+    m = mn;
   }
-  if (d == 0 && P.sel_count) P.sel_count[s] = P.is_ret[g] ? P.ws.st[s].count : 0;
+  if (lane == 0) { wm[warp] = m; wl[warp] = l; }
+  *reinterpret_cast<float4*>(&wacc[warp][4 * lane]) = acc;
+  __syncthreads();
+  if (warp == 0) {
+    float M = -INFINITY;
+    for (int w = 0; w < 8; ++w) M = fmaxf(M, wm[w]);
+    float den = 0.f;
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int w = 0; w < 8; ++w) {
+      if (wm[w] == -INFINITY) continue;
+      const float sc = exp2f(wm[w] - M);
+      den = fmaf(sc, wl[w], den);
+      const float4 a = *reinterpret_cast<const float4*>(&wacc[w][4 * lane]);
+      num.x = fmaf(sc, a.x, num.x);
+      num.y = fmaf(sc, a.y, num.y);
+      num.z = fmaf(sc, a.z, num.z);
+      num.w = fmaf(sc, a.w, num.w);
+    }
+    const float inv = 1.f / den;
+    float4 o = make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
+    *reinterpret_cast<float4*>(P.out + ((size_t)b * P.Hq + (size_t)g * G + h) * kHeadDim + 4 * lane) = o;
+  }
+  if (threadIdx.x == 0 && h == 0 && P.sel_count) P.sel_count[s] = P.is_ret[g] ? P.ws.st[s].count : 0;
 }
 
 template <typename T, int G>
@@ -302,10 +331,10 @@ cudaError_t launch_attend(const StepParams& P, int kv_dtype, int grid, cudaStrea
 
 cudaError_t launch_combine(const StepParams& P, cudaStream_t st) {
   switch (P.G) {
-    case 1: k_combine<1><<<P.n_slices, kHeadDim, 0, st>>>(P); break;
-    case 2: k_combine<2><<<P.n_slices, kHeadDim, 0, st>>>(P); break;
-    case 4: k_combine<4><<<P.n_slices, kHeadDim, 0, st>>>(P); break;
-    case 8: k_combine<8><<<P.n_slices, kHeadDim, 0, st>>>(P); break;
+    case 1: k_combine<1><<<P.n_slices * 1, 256, 0, st>>>(P); break;
+    case 2: k_combine<2><<<P.n_slices * 2, 256, 0, st>>>(P); break;
+    case 4: k_combine<4><<<P.n_slices * 4, 256, 0, st>>>(P); break;
+    case 8: k_combine<8><<<P.n_slices * 8, 256, 0, st>>>(P); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

@@ -161,33 +161,44 @@ __device__ __forceinline__ void load_qidx(const StepParams& P, const SliceCoord&
 }
 
 // ------------------------------------------------------------------ prologue
+// One CTA per (b, kv head), 256 threads.  cos/sin of the 64 RoPE angles are formed
+// once in float64 and shared; each warp owns index outputs (h, r) and reduces the
+// 128-term float64 dot product P_q[h][r] . q_pre[h] across its lanes.
 template <typename T>
-__global__ void __launch_bounds__(128) k_prologue(StepParams P) {
+__global__ void __launch_bounds__(256) k_prologue(StepParams P) {
+  __shared__ double cs_s[kHeadDim / 2], sn_s[kHeadDim / 2];
   const int s = blockIdx.x;
   const int b = s / P.Hkv, g = s % P.Hkv, G = P.G;
   const int L = load_len(P.seq_lens, b, P.Lcap, P.ws.dev_err);
   const T* q = (const T*)P.q_pre + ((size_t)b * P.Hq + (size_t)g * G) * kHeadDim;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid < kHeadDim / 2) {
     // rotate-half RoPE at position L-1; the angle is formed and reduced in float64
     const double ang = (double)(L - 1) * P.ws.inv_freq[tid];
-    double sn, cs;
-    sincos(ang, &sn, &cs);
-    for (int h = 0; h < G; ++h) {
-      const double x1 = Elem<T>::get(q, h * kHeadDim + tid);
-      const double x2 = Elem<T>::get(q, h * kHeadDim + tid + kHeadDim / 2);
-      float* o = P.ws.q_rot + ((size_t)b * P.Hq + (size_t)g * G + h) * kHeadDim;
-      o[tid] = (float)(x1 * cs - x2 * sn);
-      o[tid + kHeadDim / 2] = (float)(x2 * cs + x1 * sn);
-    }
+    sincos(ang, &sn_s[tid], &cs_s[tid]);
+  }
+  __syncthreads();
+  for (int t = tid; t < G * (kHeadDim / 2); t += blockDim.x) {
+    const int h = t / (kHeadDim / 2), i = t % (kHeadDim / 2);
+    const double x1 = Elem<T>::get(q, h * kHeadDim + i);
+    const double x2 = Elem<T>::get(q, h * kHeadDim + i + kHeadDim / 2);
+    float* o = P.ws.q_rot + ((size_t)b * P.Hq + (size_t)g * G + h) * kHeadDim;
+    o[i] = (float)(x1 * cs_s[i] - x2 * sn_s[i]);
+    o[i + kHeadDim / 2] = (float)(x2 * cs_s[i] + x1 * sn_s[i]);
   }
   if (P.is_ret[g]) {
-    for (int t = tid; t < G * kIdxDim; t += blockDim.x) {
-      const int h = t / kIdxDim, r = t % kIdxDim;
+    for (int o = warp; o < G * kIdxDim; o += blockDim.x / 32) {
+      const int h = o / kIdxDim, r = o % kIdxDim;
       const float* pq = P.ws.P_q + ((size_t)(g * G + h) * kIdxDim + r) * kHeadDim;
       double acc = 0.0;
-      for (int d = 0; d < kHeadDim; ++d) acc += (double)pq[d] * (double)Elem<T>::get(q, h * kHeadDim + d);
-      P.ws.q_idx[((size_t)b * P.Hq + (size_t)g * G + h) * kIdxDim + r] = (float)acc;
+#pragma unroll
+      for (int k = 0; k < kHeadDim / 32; ++k) {
+        const int d = lane + 32 * k;
+        acc += (double)pq[d] * (double)Elem<T>::get(q, h * kHeadDim + d);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(kFull, acc, off);
+      if (lane == 0) P.ws.q_idx[((size_t)b * P.Hq + (size_t)g * G + h) * kIdxDim + r] = (float)acc;
     }
     unsigned long long* h1 = P.ws.hist1 + (size_t)s * kBins1;
     for (int i = tid; i < kBins1; i += blockDim.x) h1[i] = 0ull;
@@ -606,8 +617,8 @@ cudaError_t launch_mass_g(const StepParams& P, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_prologue(const StepParams& P, int kv_dtype, cudaStream_t st) {
-  if (kv_dtype == 0) k_prologue<__nv_bfloat16><<<P.n_slices, 128, 0, st>>>(P);
-  else k_prologue<float><<<P.n_slices, 128, 0, st>>>(P);
+  if (kv_dtype == 0) k_prologue<__nv_bfloat16><<<P.n_slices, 256, 0, st>>>(P);
+  else k_prologue<float><<<P.n_slices, 256, 0, st>>>(P);
   return cudaGetLastError();
 }
 

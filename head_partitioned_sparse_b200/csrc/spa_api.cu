@@ -61,7 +61,7 @@ Layout plan(const spa_config& c, int split_rows) {
       slices * sizeof(spa::SliceState),                    // 11 st
       slices * (size_t)Lmax * 4,                           // 12 list
       (slices + 1) * 4,                                    // 13 item_base
-      (size_t)L.max_items * G * (spa::kHeadDim + 2) * 4,   // 14 part
+      (size_t)L.max_items * G * spa::kPartStride * 4,      // 14 part
       256,                                                 // 15 dev_err
   };
   size_t o = 0;

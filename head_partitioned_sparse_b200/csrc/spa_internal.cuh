@@ -33,6 +33,8 @@ constexpr float kMassScale = 1152921504606846976.0f;  // 2^60: mass unit is 2^-6
 constexpr int kTile = 64;
 constexpr int kAttnThreads = 256;
 constexpr int kDefaultSplitRows = 512;
+// One split's state per head: acc[128], m, l, 2 floats of padding (16-byte rows).
+constexpr int kPartStride = kHeadDim + 4;
 
 // Device status bits.
 constexpr unsigned kErrSeqLen = 1u;
@@ -71,7 +73,7 @@ struct Workspace {
   SliceState* st;        // [Bm*Hkv]
   int* list;             // [Bm*Hkv][Lmax]  selected positions (decode)
   int* item_base;        // [Bm*Hkv + 1]
-  float* part;           // [max_items][G][kHeadDim + 2]
+  float* part;           // [max_items][G][kPartStride]
   unsigned* dev_err;     // [1]
   int64_t max_items;
 };
