@@ -71,6 +71,8 @@ _SIGS = {
     "spa_profile_read": (_i, [_vp, _i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
     "spa_kernel_name": (ctypes.c_char_p, [_i]),
     "spa_launch_count": (_i, [_vp, ctypes.POINTER(ctypes.c_int64)]),
+    "spa_select_noalloc": (_i, [_vp, _i, _i, _i, _f, _i64, _vp, _vp, _vp, _vp, _i, _i64, _f, _i, _i, _vp, _vp,
+                                _vp]),
 }
 EXPORTED = tuple(_SIGS)
 
@@ -189,3 +191,12 @@ def make_config(*, max_batch: int, n_q_heads: int, n_kv_heads: int, max_ctx: int
     return spa_config(max_batch=max_batch, n_q_heads=n_q_heads, n_kv_heads=n_kv_heads, head_dim=head_dim,
                       idx_dim=idx_dim, kv_dtype=kv_dtype, max_ctx=max_ctx, rope_theta=rope_theta,
                       idx_scale=idx_scale, split_rows=split_rows, P_q=_ptr(P_q), P_k=_ptr(P_k))
+
+
+def spa_select_noalloc(P_q, n_q_heads: int, n_kv_heads: int, kv_dtype: int, idx_scale: float, max_ctx: int,
+                       q_pre, idx_cache, head_mask, seq_lens, B: int, max_seq_len: int, p: float, n_sink: int,
+                       window: int, sel_idx, sel_count, stream=None) -> None:
+    """spa_select with no handle and no allocation (static scratch; see include/spa.h)."""
+    _check(load().spa_select_noalloc(_ptr(P_q), n_q_heads, n_kv_heads, kv_dtype, idx_scale, max_ctx, _ptr(q_pre),
+                                     _ptr(idx_cache), _host_u8(head_mask), _ptr(seq_lens), B, max_seq_len, p,
+                                     n_sink, window, _ptr(sel_idx), _ptr(sel_count), _stream(stream)))

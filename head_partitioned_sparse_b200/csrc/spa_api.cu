@@ -75,6 +75,14 @@ Layout plan(const spa_config& c, int split_rows) {
 
 }  // namespace
 
+namespace spa {
+// Records `msg` as the calling thread's spa_last_error() text; returns `code`.
+int set_last_error(int code, const char* msg) {
+  g_err = msg;
+  return code;
+}
+}  // namespace spa
+
 struct spa_ctx {
   spa_config cfg{};
   int G = 0;

@@ -166,4 +166,5 @@ cudaError_t launch_compact(const StepParams& P, cudaStream_t st);
 cudaError_t launch_attend(const StepParams& P, int kv_dtype, int grid, cudaStream_t st);
 cudaError_t launch_combine(const StepParams& P, cudaStream_t st);
 int attend_setup(int kv_dtype, int G, int max_slices);
+int set_last_error(int code, const char* msg);
 }  // namespace spa

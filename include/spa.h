@@ -203,6 +203,32 @@ SPA_API const char* spa_kernel_name(int kernel_id);
 /* Number of kernel launches this handle has issued since it was created. */
 SPA_API spa_status spa_launch_count(spa_handle h, int64_t* launches);
 
+/*
+ * spa_select without a handle and without allocating anything, for callers that
+ * cannot call cudaMalloc: code inside a host framework that has reserved the GPU's
+ * memory for its own pool, or a decode loop that cannot afford the implicit device
+ * synchronisation an allocation may cause.  The paper has no counterpart to this
+ * entry point; it exists for those callers only.
+ * Inputs, outputs and result are those of spa_select; the query projectors are
+ * passed directly (P_q: device float32 [n_q_heads][16][128]) and max_ctx is the row
+ * stride of idx_cache and sel_idx; idx_scale <= 0 selects 0.25.
+ * All scratch is one static 12 MiB device array, held by every GPU that loads the
+ * library until the process exits.  Limits: B*n_kv_heads <= 64, B*n_q_heads <= 512,
+ * B*n_kv_heads*max_ctx <= 2^19 tokens; larger requests return SPA_ERR_WORKSPACE
+ * before anything is launched.  The first call on a device looks up the array's
+ * device address there (cudaGetSymbolAddress, with that device current): make that
+ * first call before any stream capture.  Every call shares the array and the next
+ * call overwrites it, so calls that overlap on the GPU race: serialise them.
+ * Out-of-range seq_lens values are clamped but not reported (no handle to hold the
+ * status word).
+ */
+SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads, int n_kv_heads, int kv_dtype,
+                                      float idx_scale, int64_t max_ctx, const void* q_pre,
+                                      const void* idx_cache, const uint8_t* head_mask,
+                                      const int64_t* seq_lens, int B, int64_t max_seq_len, float p,
+                                      int n_sink, int window, int32_t* sel_idx, int32_t* sel_count,
+                                      spa_stream stream);
+
 #ifdef __cplusplus
 }
 #endif
