@@ -326,7 +326,8 @@ int setup_tg(int max_slices) {
 }  // namespace
 
 cudaError_t launch_attend(const StepParams& P, int kv_dtype, int grid, cudaStream_t st) {
-  return kv_dtype == 0 ? launch_attend_t<__nv_bfloat16>(P, grid, st) : launch_attend_t<float>(P, grid, st);
+  // bf16 caches: tensor-core kernel (k_attend_mma.cu); float32 caches: this file's kernel
+  return kv_dtype == 0 ? launch_attend_bf16(P, grid, st) : launch_attend_t<float>(P, grid, st);
 }
 
 cudaError_t launch_combine(const StepParams& P, cudaStream_t st) {
@@ -343,20 +344,12 @@ cudaError_t launch_combine(const StepParams& P, cudaStream_t st) {
 // Sets the dynamic shared-memory limit for the (dtype, G) instantiation and returns
 // resident CTAs per SM (or -1).
 int attend_setup(int kv_dtype, int G, int max_slices) {
-  if (kv_dtype == 0) {
-    switch (G) {
-      case 1: return setup_tg<__nv_bfloat16, 1>(max_slices);
-      case 2: return setup_tg<__nv_bfloat16, 2>(max_slices);
-      case 4: return setup_tg<__nv_bfloat16, 4>(max_slices);
-      case 8: return setup_tg<__nv_bfloat16, 8>(max_slices);
-    }
-  } else {
-    switch (G) {
-      case 1: return setup_tg<float, 1>(max_slices);
-      case 2: return setup_tg<float, 2>(max_slices);
-      case 4: return setup_tg<float, 4>(max_slices);
-      case 8: return setup_tg<float, 8>(max_slices);
-    }
+  if (kv_dtype == 0) return attend_bf16_setup(G, max_slices);
+  switch (G) {
+    case 1: return setup_tg<float, 1>(max_slices);
+    case 2: return setup_tg<float, 2>(max_slices);
+    case 4: return setup_tg<float, 4>(max_slices);
+    case 8: return setup_tg<float, 8>(max_slices);
   }
   return -1;
 }

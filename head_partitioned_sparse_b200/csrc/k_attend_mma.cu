@@ -1,0 +1,404 @@
+// Split-K attention for bf16 caches on the tensor cores (mma.sync m16n8k16).
+//
+// Same computation as the float32 kernel in k_attend.cu ("Full Attention Strikes
+// Back" (RTPurbo summary), Methodology §1; exact token attention as in
+// "Hierarchical Global Attention", Central mechanism §4): for every split of a
+// slice's attended rows, the online-softmax state (m, l, acc) of each query head
+// of the GQA group.
+//
+// Work layout.  One CTA per SM, 8 warps.  A split ("item") is split_rows virtual
+// rows of one slice (sinks, window, then the gathered list); CTAs take items
+// c, c + gridDim.x, ...; inside an item, warp w takes the 16-row chunks
+// w, w + 8, ...  Each warp streams its chunks through its own 3-stage ring in
+// shared memory with 16-byte cp.async (one K row = 256 bytes = 16 lanes), keeps
+// prefetching across item boundaries, and keeps its own online softmax.  At the
+// end of an item the 8 warp states are merged in a fixed 3-round tree and warp 0
+// writes the split's state.
+//
+// Tensor-core mapping (G <= 8 heads of the group, M = 16 rows):
+//   S[16 x 16 tokens] = Q[16 x 128] . K^T:  A rows 0..7 = bf16 high parts of the
+//       G rotated queries, rows 8..15 = the bf16 residuals (q - hi), so the two
+//       halves of the accumulator sum to the score at ~2^-17 relative precision;
+//       B = K rows straight from shared memory (ldmatrix, rows are tokens).
+//   O[16 x 128] += P[16 x 16 tokens] . V:  the probabilities, split the same way
+//       into bf16 high parts (rows 0..7) and residuals (rows 8..15), come from the
+//       score accumulators without a shuffle; B = V via ldmatrix.trans.
+// Rows of a stage are padded to 272 bytes so the 8 row addresses of an ldmatrix
+// fall in 8 different bank groups.
+#include <climits>
+
+#include "spa_internal.cuh"
+
+namespace spa {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kWarps = 8;
+constexpr int kChunkRows = 16;
+constexpr int kStages = 3;
+constexpr int kRowPad = kHeadDim + 8;                               // 136 bf16 = 272 bytes
+constexpr int kStageElems = 2 * kChunkRows * kRowPad;               // K then V
+constexpr size_t kRingBytes = (size_t)kWarps * kStages * kStageElems * 2;
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_stages() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(kStages - 2) : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  const unsigned a = (unsigned)__cvta_generic_to_shared(p);
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
+  const unsigned a = (unsigned)__cvta_generic_to_shared(p);
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// bf16 pair: x in the low half (lower column), y in the high half.
+__device__ __forceinline__ uint32_t pack2(float x, float y) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(x, y);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+__device__ __forceinline__ float bf16r(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
+// Where an item's rows come from.
+struct ItemInfo {
+  int s;          // slice b * Hkv + g
+  int v0, v1;     // virtual rows [v0, v1)
+  int nc;         // contiguous (sink + window) rows of the slice
+  int n_s, w_lo;  // sinks [0, n_s), window [w_lo, L)
+  int nch;        // 16-row chunks
+};
+
+__device__ __forceinline__ ItemInfo decode_item(const StepParams& P, const int* pref, int item) {
+  int lo = 0, hi = P.n_slices - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pref[mid] <= item) lo = mid; else hi = mid - 1;
+  }
+  ItemInfo it;
+  it.s = lo;
+  const int b = lo / P.Hkv, g = lo % P.Hkv;
+  const int L = load_len(P.seq_lens, b, P.Lcap, P.ws.dev_err);
+  const SinkWindow sw(L, P.n_sink, P.window);
+  const int n_rows = sw.n_contig() + (P.is_ret[g] ? P.ws.st[lo].count : 0);
+  it.nc = sw.n_contig();
+  it.n_s = sw.n_s;
+  it.w_lo = sw.w_lo;
+  it.v0 = (item - pref[lo]) * P.split_rows;
+  it.v1 = min(it.v0 + P.split_rows, n_rows);
+  it.nch = (it.v1 - it.v0 + kChunkRows - 1) / kChunkRows;
+  return it;
+}
+
+template <int G>
+__global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __nv_bfloat16* ring = reinterpret_cast<__nv_bfloat16*>(smem);
+  float* mbuf = reinterpret_cast<float*>(smem + kRingBytes);         // [4][G][kPartStride]
+  int* pref = reinterpret_cast<int*>(mbuf + 4 * G * kPartStride);    // [n_slices + 1]
+  __shared__ int shi[32];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gid = lane >> 2, t4 = lane & 3;
+  const int NS = P.n_slices;
+
+  // ---- item prefix over slices (CTA 0 publishes it for the combine)
+  {
+    int carry = 0;
+    for (int base = 0; base < NS; base += kWarps * 32) {
+      const int s = base + tid;
+      int it = 0;
+      if (s < NS) {
+        const int b = s / P.Hkv, g = s % P.Hkv;
+        const int L = load_len(P.seq_lens, b, P.Lcap, P.ws.dev_err);
+        const SinkWindow sw(L, P.n_sink, P.window);
+        const int n = sw.n_contig() + (P.is_ret[g] ? P.ws.st[s].count : 0);
+        it = (n + P.split_rows - 1) / P.split_rows;
+      }
+      int v = it;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, v, o);
+        if (lane >= o) v += y;
+      }
+      if (lane == 31) shi[warp] = v;
+      __syncthreads();
+      if (warp == 0) {
+        int w = lane < kWarps ? shi[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(kFull, w, o);
+          if (lane >= o) w += y;
+        }
+        if (lane < kWarps) shi[lane] = w;
+      }
+      __syncthreads();
+      if (s < NS) pref[s] = carry + (warp ? shi[warp - 1] : 0) + v - it;
+      carry += shi[kWarps - 1];
+      __syncthreads();
+    }
+    if (tid == 0) pref[NS] = carry;
+    __syncthreads();
+  }
+  const int total = pref[NS];
+  if (blockIdx.x == 0)
+    for (int s = tid; s <= NS; s += kWarps * 32) P.ws.item_base[s] = pref[s];
+
+  __nv_bfloat16* myring = ring + (size_t)warp * kStages * kStageElems;
+
+  // ---- prefetch cursor over this warp's (item, chunk) units
+  int pf_item = blockIdx.x, pf_ch = warp;
+  ItemInfo pf = {};
+  if (pf_item < total) pf = decode_item(P, pref, pf_item);
+  auto pf_normalise = [&]() {
+    while (pf_item < total && pf_ch >= pf.nch) {
+      pf_item += gridDim.x;
+      pf_ch = warp;
+      if (pf_item < total) pf = decode_item(P, pref, pf_item);
+    }
+  };
+  pf_normalise();
+  int issued = 0;  // units issued so far (selects the ring slot)
+  auto issue_next = [&]() {
+    __nv_bfloat16* dst = myring + (size_t)(issued % kStages) * kStageElems;
+    if (pf_item < total) {
+      const int r0 = pf.v0 + pf_ch * kChunkRows;
+      const int* list = P.sel_list + (size_t)pf.s * P.Lmax;
+      // lane r < 16 resolves the position of row r (rows past the item repeat row 0)
+      int pos = 0;
+      if (lane < kChunkRows) {
+        int v = r0 + lane;
+        if (v >= pf.v1) v = r0;
+        pos = v < pf.nc ? (v < pf.n_s ? v : pf.w_lo + (v - pf.n_s)) : list[v - pf.nc];
+      }
+      const __nv_bfloat16* kb = (const __nv_bfloat16*)P.k_cache + (size_t)pf.s * P.Lmax * kHeadDim;
+      const __nv_bfloat16* vb = (const __nv_bfloat16*)P.v_cache + (size_t)pf.s * P.Lmax * kHeadDim;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int idx = i * 32 + lane;   // 512 pieces of 16 bytes: [K|V][row][piece]
+        const int tv = idx >> 8, rem = idx & 255, r = rem >> 4, c = rem & 15;
+        const int prow = __shfl_sync(kFull, pos, r);
+        const __nv_bfloat16* src = (tv ? vb : kb) + (size_t)prow * kHeadDim + c * 8;
+        cp_async16(dst + tv * kChunkRows * kRowPad + r * kRowPad + c * 8, src);
+      }
+      pf_ch += kWarps;
+      pf_normalise();
+    }
+    cp_async_commit();
+    ++issued;
+  };
+#pragma unroll
+  for (int i = 0; i < kStages - 1; ++i) issue_next();
+
+  int consumed = 0;
+  int cur_slice = -1;
+  uint32_t qa[8][4];   // A fragments of Q (hi rows 0..7, residual rows 8..15), per 16-dim k-step
+  const float scale = P.attn_scale_log2;
+
+  for (int item = blockIdx.x; item < total; item += gridDim.x) {
+    const ItemInfo it = decode_item(P, pref, item);
+    if (it.s != cur_slice) {
+      cur_slice = it.s;
+      const int b = it.s / P.Hkv, g = it.s % P.Hkv;
+      const float* q = P.ws.q_rot + ((size_t)b * P.Hq + (size_t)g * G + (gid < G ? gid : 0)) * kHeadDim;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        float x[4];
+        x[0] = q[16 * kk + 2 * t4];
+        x[1] = q[16 * kk + 2 * t4 + 1];
+        x[2] = q[16 * kk + 2 * t4 + 8];
+        x[3] = q[16 * kk + 2 * t4 + 9];
+        if (gid >= G) x[0] = x[1] = x[2] = x[3] = 0.f;
+        float hi[4], lo[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          hi[j] = bf16r(x[j]);
+          lo[j] = x[j] - hi[j];
+        }
+        qa[kk][0] = pack2(hi[0], hi[1]);
+        qa[kk][1] = pack2(lo[0], lo[1]);
+        qa[kk][2] = pack2(hi[2], hi[3]);
+        qa[kk][3] = pack2(lo[2], lo[3]);
+      }
+    }
+    float m = -INFINITY, l = 0.f;
+    float acc[16][4];
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+
+    for (int ch = warp; ch < it.nch; ch += kWarps) {
+      cp_async_wait_stages();
+      __syncwarp();
+      const __nv_bfloat16* ks = myring + (size_t)(consumed % kStages) * kStageElems;
+      const __nv_bfloat16* vs = ks + kChunkRows * kRowPad;
+      ++consumed;
+      issue_next();   // refill the slot consumed last time
+      const int nr = min(kChunkRows, it.v1 - (it.v0 + ch * kChunkRows));
+
+      // S = Q K^T for 16 tokens (two n-tiles of 8)
+      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      const int mi = lane >> 3, rr = lane & 7;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        uint32_t bk[4];
+        ldsm_x4(bk, ks + (8 * (mi >> 1) + rr) * kRowPad + 16 * kk + 8 * (mi & 1));
+        mma16816(sc[0], qa[kk], bk[0], bk[1]);
+        mma16816(sc[1], qa[kk], bk[2], bk[3]);
+      }
+      // scores of head gid for tokens 8j + 2 t4 + c (hi row + residual row)
+      float s[2][2];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int tok = 8 * j + 2 * t4 + c;
+          const float v = (sc[j][c] + sc[j][2 + c]) * scale;
+          s[j][c] = tok < nr ? v : -INFINITY;
+          mx = fmaxf(mx, s[j][c]);
+        }
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+      const float mn = fmaxf(m, mx);
+      const float alpha = exp2f(m - mn);   // m = -inf on the first chunk: alpha = 0
+      m = mn;
+      if (__any_sync(kFull, alpha != 1.f)) {
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+          acc[nt][0] *= alpha;
+          acc[nt][1] *= alpha;
+          acc[nt][2] *= alpha;
+          acc[nt][3] *= alpha;
+        }
+        l *= alpha;
+      }
+      float p[2][2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          p[j][c] = exp2f(s[j][c] - mn);
+          l += p[j][c];
+        }
+      // P as the A operand: rows gid = bf16(p), rows gid + 8 = p - bf16(p)
+      uint32_t pa[4];
+      {
+        const float h00 = bf16r(p[0][0]), h01 = bf16r(p[0][1]), h10 = bf16r(p[1][0]), h11 = bf16r(p[1][1]);
+        pa[0] = pack2(h00, h01);
+        pa[1] = pack2(p[0][0] - h00, p[0][1] - h01);
+        pa[2] = pack2(h10, h11);
+        pa[3] = pack2(p[1][0] - h10, p[1][1] - h11);
+      }
+      // O += P V over 128 dims (16 n-tiles of 8)
+#pragma unroll
+      for (int nt = 0; nt < 16; nt += 2) {
+        uint32_t bv[4];
+        ldsm_x4_t(bv, vs + (8 * (mi & 1) + rr) * kRowPad + 8 * (nt + (mi >> 1)));
+        mma16816(acc[nt], pa, bv[0], bv[1]);
+        mma16816(acc[nt + 1], pa, bv[2], bv[3]);
+      }
+    }
+
+    // ---- warp state: row sums over the 4 lanes of a head, hi + residual rows combined
+    l += __shfl_xor_sync(kFull, l, 1);
+    l += __shfl_xor_sync(kFull, l, 2);
+    float o[16][2];
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+      o[nt][0] = acc[nt][0] + acc[nt][2];
+      o[nt][1] = acc[nt][1] + acc[nt][3];
+    }
+    // ---- merge the 8 warp states: 8 -> 4 -> 2 -> 1
+#pragma unroll
+    for (int half = kWarps / 2; half >= 1; half >>= 1) {
+      if (warp >= half && warp < 2 * half && gid < G) {
+        float* dst = mbuf + ((size_t)(warp - half) * G + gid) * kPartStride;
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt)
+          *reinterpret_cast<float2*>(dst + 8 * nt + 2 * t4) = make_float2(o[nt][0], o[nt][1]);
+        if (t4 == 0) { dst[kHeadDim] = m; dst[kHeadDim + 1] = l; }
+      }
+      __syncthreads();
+      if (warp < half && gid < G) {
+        const float* src = mbuf + ((size_t)warp * G + gid) * kPartStride;
+        const float m2 = src[kHeadDim], l2 = src[kHeadDim + 1];
+        const float mn = fmaxf(m, m2);
+        if (mn != -INFINITY) {
+          const float sa = exp2f(m - mn), sb = exp2f(m2 - mn);
+          l = l * sa + l2 * sb;
+#pragma unroll
+          for (int nt = 0; nt < 16; ++nt) {
+            const float2 v = *reinterpret_cast<const float2*>(src + 8 * nt + 2 * t4);
+            o[nt][0] = o[nt][0] * sa + v.x * sb;
+            o[nt][1] = o[nt][1] * sa + v.y * sb;
+          }
+          m = mn;
+        }
+      }
+      __syncthreads();
+    }
+    if (warp == 0 && gid < G) {
+      float* dst = P.ws.part + ((size_t)item * G + gid) * kPartStride;
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt)
+        *reinterpret_cast<float2*>(dst + 8 * nt + 2 * t4) = make_float2(o[nt][0], o[nt][1]);
+      if (t4 == 0) { dst[kHeadDim] = m; dst[kHeadDim + 1] = l; }
+    }
+  }
+  asm volatile("cp.async.wait_all;\n" ::: "memory");
+}
+
+size_t smem_bytes(int G, int max_slices) {
+  return kRingBytes + (size_t)4 * G * kPartStride * 4 + (size_t)(max_slices + 1) * 4;
+}
+
+template <int G>
+int setup_g(int max_slices) {
+  const size_t sm = smem_bytes(G, max_slices);
+  if (cudaFuncSetAttribute(k_attend_bf16<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
+    return -1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_attend_bf16<G>, kWarps * 32, sm) != cudaSuccess) return -1;
+  return n;
+}
+
+}  // namespace
+
+cudaError_t launch_attend_bf16(const StepParams& P, int grid, cudaStream_t st) {
+  const size_t sm = smem_bytes(P.G, P.n_slices);
+  switch (P.G) {
+    case 1: k_attend_bf16<1><<<grid, kWarps * 32, sm, st>>>(P); break;
+    case 2: k_attend_bf16<2><<<grid, kWarps * 32, sm, st>>>(P); break;
+    case 4: k_attend_bf16<4><<<grid, kWarps * 32, sm, st>>>(P); break;
+    case 8: k_attend_bf16<8><<<grid, kWarps * 32, sm, st>>>(P); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+int attend_bf16_setup(int G, int max_slices) {
+  switch (G) {
+    case 1: return setup_g<1>(max_slices);
+    case 2: return setup_g<2>(max_slices);
+    case 4: return setup_g<4>(max_slices);
+    case 8: return setup_g<8>(max_slices);
+  }
+  return -1;
+}
+
+}  // namespace spa

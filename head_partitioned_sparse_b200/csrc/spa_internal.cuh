@@ -166,5 +166,7 @@ cudaError_t launch_compact(const StepParams& P, cudaStream_t st);
 cudaError_t launch_attend(const StepParams& P, int kv_dtype, int grid, cudaStream_t st);
 cudaError_t launch_combine(const StepParams& P, cudaStream_t st);
 int attend_setup(int kv_dtype, int G, int max_slices);
+cudaError_t launch_attend_bf16(const StepParams& P, int grid, cudaStream_t st);
+int attend_bf16_setup(int G, int max_slices);
 int set_last_error(int code, const char* msg);
 }  // namespace spa
