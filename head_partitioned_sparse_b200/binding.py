@@ -67,7 +67,7 @@ _SIGS = {
     "spa_select": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i64, _f, _i, _i, _vp, _vp, _vp]),
     "spa_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i64, _f, _i, _i, _vp, _vp, _vp]),
     "spa_device_status": (_i, [_vp, _vp]),
-    "spa_set_profiling": (_i, [_vp, _i]),
+    "spa_set_profiling": (_i, [_vp, ctypes.c_uint]),
     "spa_profile_read": (_i, [_vp, _i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
     "spa_kernel_name": (ctypes.c_char_p, [_i]),
     "spa_launch_count": (_i, [_vp, ctypes.POINTER(ctypes.c_int64)]),
@@ -164,8 +164,9 @@ def spa_device_status(h, stream=None) -> None:
     _check(load().spa_device_status(h, _stream(stream)))
 
 
-def spa_set_profiling(h, enable: bool) -> None:
-    _check(load().spa_set_profiling(h, 1 if enable else 0))
+def spa_set_profiling(h, kernel_mask: int) -> None:
+    """kernel_mask: bit (1 << SPA_K_...) per kernel to time with CUDA events; 0 = off."""
+    _check(load().spa_set_profiling(h, int(kernel_mask)))
 
 
 def spa_profile_read(h, kernel_id: int) -> Tuple[float, int]:

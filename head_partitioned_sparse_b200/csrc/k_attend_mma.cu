@@ -11,7 +11,10 @@
 // c, c + gridDim.x, ...; inside an item, warp w takes the 16-row chunks
 // w, w + 8, ...  Each warp streams its chunks through its own 3-stage ring in
 // shared memory with 16-byte cp.async (one K row = 256 bytes = 16 lanes), keeps
-// prefetching across item boundaries, and keeps its own online softmax.  At the
+// prefetching across item boundaries, loads the row positions of the next chunk
+// one issue ahead (no copy waits on a list load), and keeps its own online softmax.
+// (One 256-byte TMA bulk copy per row was measured 4.6x slower than this: the
+// per-request cost of the bulk-copy engine dominates at row granularity.)  At the
 // end of an item the 8 warp states are merged in a fixed 3-round tree and warp 0
 // writes the split's state.
 //
@@ -161,7 +164,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
 
   __nv_bfloat16* myring = ring + (size_t)warp * kStages * kStageElems;
 
-  // ---- prefetch cursor over this warp's (item, chunk) units
+  // ---- prefetch cursor over this warp's (item, chunk) units.  The row positions of
+  // the unit to issue next are loaded one issue ahead (apos, lane r < 16 holds row r),
+  // so no copy address waits on a load from the selected list.
   int pf_item = blockIdx.x, pf_ch = warp;
   ItemInfo pf = {};
   if (pf_item < total) pf = decode_item(P, pref, pf_item);
@@ -172,32 +177,36 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
       if (pf_item < total) pf = decode_item(P, pref, pf_item);
     }
   };
+  auto load_pos = [&]() -> int {
+    int pos = 0;
+    if (pf_item < total && lane < kChunkRows) {
+      const int r0 = pf.v0 + pf_ch * kChunkRows;
+      int v = r0 + lane;
+      if (v >= pf.v1) v = r0;   // rows past the item repeat row 0 (finite, masked later)
+      pos = v < pf.nc ? (v < pf.n_s ? v : pf.w_lo + (v - pf.n_s))
+                      : P.sel_list[(size_t)pf.s * P.Lmax + (v - pf.nc)];
+    }
+    return pos;
+  };
   pf_normalise();
+  int apos = load_pos();
   int issued = 0;  // units issued so far (selects the ring slot)
   auto issue_next = [&]() {
     __nv_bfloat16* dst = myring + (size_t)(issued % kStages) * kStageElems;
     if (pf_item < total) {
-      const int r0 = pf.v0 + pf_ch * kChunkRows;
-      const int* list = P.sel_list + (size_t)pf.s * P.Lmax;
-      // lane r < 16 resolves the position of row r (rows past the item repeat row 0)
-      int pos = 0;
-      if (lane < kChunkRows) {
-        int v = r0 + lane;
-        if (v >= pf.v1) v = r0;
-        pos = v < pf.nc ? (v < pf.n_s ? v : pf.w_lo + (v - pf.n_s)) : list[v - pf.nc];
-      }
       const __nv_bfloat16* kb = (const __nv_bfloat16*)P.k_cache + (size_t)pf.s * P.Lmax * kHeadDim;
       const __nv_bfloat16* vb = (const __nv_bfloat16*)P.v_cache + (size_t)pf.s * P.Lmax * kHeadDim;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int idx = i * 32 + lane;   // 512 pieces of 16 bytes: [K|V][row][piece]
         const int tv = idx >> 8, rem = idx & 255, r = rem >> 4, c = rem & 15;
-        const int prow = __shfl_sync(kFull, pos, r);
+        const int prow = __shfl_sync(kFull, apos, r);
         const __nv_bfloat16* src = (tv ? vb : kb) + (size_t)prow * kHeadDim + c * 8;
         cp_async16(dst + tv * kChunkRows * kRowPad + r * kRowPad + c * 8, src);
       }
       pf_ch += kWarps;
       pf_normalise();
+      apos = load_pos();
     }
     cp_async_commit();
     ++issued;
@@ -250,15 +259,20 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
       issue_next();   // refill the slot consumed last time
       const int nr = min(kChunkRows, it.v1 - (it.v0 + ch * kChunkRows));
 
-      // S = Q K^T for 16 tokens (two n-tiles of 8)
-      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      // S = Q K^T for 16 tokens (two n-tiles of 8); two accumulators per n-tile
+      // (even / odd k-steps) halve the dependent mma chain
+      float sc[2][2][4];
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) sc[a][e][0] = sc[a][e][1] = sc[a][e][2] = sc[a][e][3] = 0.f;
       const int mi = lane >> 3, rr = lane & 7;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         uint32_t bk[4];
         ldsm_x4(bk, ks + (8 * (mi >> 1) + rr) * kRowPad + 16 * kk + 8 * (mi & 1));
-        mma16816(sc[0], qa[kk], bk[0], bk[1]);
-        mma16816(sc[1], qa[kk], bk[2], bk[3]);
+        mma16816(sc[0][kk & 1], qa[kk], bk[0], bk[1]);
+        mma16816(sc[1][kk & 1], qa[kk], bk[2], bk[3]);
       }
       // scores of head gid for tokens 8j + 2 t4 + c (hi row + residual row)
       float s[2][2];
@@ -268,7 +282,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int tok = 8 * j + 2 * t4 + c;
-          const float v = (sc[j][c] + sc[j][2 + c]) * scale;
+          const float v = ((sc[j][0][c] + sc[j][1][c]) + (sc[j][0][2 + c] + sc[j][1][2 + c])) * scale;
           s[j][c] = tok < nr ? v : -INFINITY;
           mx = fmaxf(mx, s[j][c]);
         }

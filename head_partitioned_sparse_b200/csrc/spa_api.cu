@@ -96,7 +96,7 @@ struct spa_ctx {
   spa::Workspace ws{};
   int n_chunks_max = 0;
   // instrumentation
-  bool prof = false;
+  unsigned prof_mask = 0;
   std::vector<cudaEvent_t> ev;   // pairs: 2*i start, 2*i+1 stop
   std::vector<int> ev_kid;
   size_t ev_next = 0;
@@ -139,7 +139,7 @@ spa_status check_config(const spa_config* c) {
 
 template <class F>
 spa_status run(spa_ctx* h, int kid, cudaStream_t st, const char* name, F&& f) {
-  const bool timed = h->prof && h->ev_next < kEventPairs;
+  const bool timed = ((h->prof_mask >> kid) & 1u) && h->ev_next < kEventPairs;
   if (timed) cudaEventRecord(h->ev[2 * h->ev_next], st);
   cudaError_t e = f();
   if (timed) {
@@ -382,6 +382,8 @@ spa_status spa_device_status(spa_handle h, spa_stream stream) {
   if ((e = cudaMemcpy(&flags, h->ws.dev_err, 4, cudaMemcpyDeviceToHost)) != cudaSuccess) return cuda_fail(e, "read status");
   if (flags) {
     if ((e = cudaMemset(h->ws.dev_err, 0, 4)) != cudaSuccess) return cuda_fail(e, "clear status");
+    if (flags & spa::kErrTimeout)
+      return fail(SPA_ERR_DEVICE_TIMEOUT, "a bounded device-side wait gave up (flags 0x%x)", flags);
     if (flags & spa::kErrInternal)
       return fail(SPA_ERR_CUDA, "internal consistency check failed in the selection kernels (flags 0x%x)", flags);
     return fail(SPA_ERR_DEVICE_RANGE, "device range check failed:%s%s",
@@ -391,9 +393,9 @@ spa_status spa_device_status(spa_handle h, spa_stream stream) {
   return SPA_OK;
 }
 
-spa_status spa_set_profiling(spa_handle h, int enable) {
+spa_status spa_set_profiling(spa_handle h, unsigned kernel_mask) {
   if (!h) return fail(SPA_ERR_INVALID_ARG, "handle is NULL");
-  if (enable && h->ev.empty()) {
+  if (kernel_mask && h->ev.empty()) {
     h->ev.resize(2 * kEventPairs);
     h->ev_kid.resize(kEventPairs);
     for (auto& ev : h->ev) {
@@ -401,7 +403,7 @@ spa_status spa_set_profiling(spa_handle h, int enable) {
       if (e != cudaSuccess) return cuda_fail(e, "cudaEventCreate");
     }
   }
-  h->prof = enable != 0;
+  h->prof_mask = kernel_mask;
   h->ev_next = 0;
   return SPA_OK;
 }

@@ -40,6 +40,7 @@ constexpr int kPartStride = kHeadDim + 4;
 constexpr unsigned kErrSeqLen = 1u;
 constexpr unsigned kErrStartPos = 2u;
 constexpr unsigned kErrInternal = 4u;
+constexpr unsigned kErrTimeout = 8u;   // a bounded device-side wait gave up
 
 // Per (b, kv head) selection state.  Written by the threshold kernels, read by
 // compaction and attention.

@@ -67,7 +67,7 @@ typedef int spa_status;
 #define SPA_ERR_UNSUPPORTED (-2)    /* head_dim != 128, idx_dim != 16, unsupported GQA ratio or dtype */
 #define SPA_ERR_WORKSPACE (-3)      /* workspace allocation failed / request exceeds the handle's capacity */
 #define SPA_ERR_CUDA (-4)           /* a CUDA runtime call or kernel launch failed */
-#define SPA_ERR_DEVICE_TIMEOUT (-5) /* reserved: a bounded device-side wait gave up */
+#define SPA_ERR_DEVICE_TIMEOUT (-5) /* spa_device_status: a bounded device-side wait gave up */
 #define SPA_ERR_DEVICE_RANGE (-6)   /* spa_device_status: a device-resident length/position was out of range */
 
 /* storage dtypes of q / k / v */
@@ -188,10 +188,12 @@ SPA_API spa_status spa_device_status(spa_handle h, spa_stream stream);
 #define SPA_K_COMBINE 7
 #define SPA_K_COUNT 8
 
-/* When enabled, every kernel launch of this handle is bracketed by two CUDA
- * events recorded on the launch stream (a bounded pool; launches beyond it are
- * not timed).  Enabling resets the pool. */
-SPA_API spa_status spa_set_profiling(spa_handle h, int enable);
+/* kernel_mask = 0 disables timing.  Otherwise every launch of a kernel whose bit
+ * (1 << SPA_K_...) is set is bracketed by two CUDA events recorded on the launch
+ * stream (a bounded pool; launches beyond it are not timed).  Each event pair
+ * adds a few microseconds of stream time, so time only what is needed.  Setting
+ * a mask resets the pool. */
+SPA_API spa_status spa_set_profiling(spa_handle h, unsigned kernel_mask);
 
 /* Synchronise the recorded events and return, for kernel `kernel_id`, the
  * summed device time in milliseconds and the number of timed launches. */
