@@ -245,51 +245,72 @@ __global__ void __launch_bounds__(kAttnThreads) k_attend(StepParams P) {
   }
 }
 
-// One CTA per (slice, head): warp w merges the splits w, w + 8, ... of the slice
-// (lane = 4 dims), then warp states are merged in warp order.  Deterministic.
+// One CTA per (slice, head): warp w merges the splits w, w + kCombWarps, ... of the
+// slice (lane = 4 dims), loading kCombBatch splits before merging any, then warp
+// states are merged in warp order.  Deterministic.
+constexpr int kCombWarps = 16;
+constexpr int kCombBatch = 4;
+
 template <int G>
-__global__ void __launch_bounds__(256) k_combine(StepParams P) {
-  __shared__ float wm[8], wl[8];
-  __shared__ __align__(16) float wacc[8][kHeadDim];
+__global__ void __launch_bounds__(kCombWarps * 32) k_combine(StepParams P) {
+  __shared__ float wm[kCombWarps], wl[kCombWarps];
+  __shared__ __align__(16) float wacc[kCombWarps][kHeadDim];
   const int s = blockIdx.x / G, h = blockIdx.x % G;
   const int b = s / P.Hkv, g = s % P.Hkv;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int i0 = P.ws.item_base[s], i1 = P.ws.item_base[s + 1];
   float m = -INFINITY, l = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int i = i0 + warp; i < i1; i += 8) {
-    const float* pp = P.ws.part + ((size_t)i * G + h) * kPartStride;
-    const float4 a = *reinterpret_cast<const float4*>(pp + 4 * lane);
-    const float mi = pp[kHeadDim], li = pp[kHeadDim + 1];
-    const float mn = fmaxf(m, mi);
-    const float sa = exp2f(m - mn), sb = exp2f(mi - mn);
-    l = l * sa + li * sb;
-    acc.x = acc.x * sa + a.x * sb;
-    acc.y = acc.y * sa + a.y * sb;
-    acc.z = acc.z * sa + a.z * sb;
-    acc.w = acc.w * sa + a.w * sb;
-    m = mn;
+  for (int ib = i0 + warp; ib < i1; ib += kCombWarps * kCombBatch) {
+    float4 a[kCombBatch];
+    float mi[kCombBatch], li[kCombBatch];
+#pragma unroll
+    for (int u = 0; u < kCombBatch; ++u) {
+      const int i = ib + u * kCombWarps;
+      if (i < i1) {
+        const float* pp = P.ws.part + ((size_t)i * G + h) * kPartStride;
+        a[u] = *reinterpret_cast<const float4*>(pp + 4 * lane);
+        mi[u] = pp[kHeadDim];
+        li[u] = pp[kHeadDim + 1];
+      } else {
+        a[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        mi[u] = -INFINITY;
+        li[u] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kCombBatch; ++u) {
+      const float mn = fmaxf(m, mi[u]);
+      if (mn == -INFINITY) continue;
+      const float sa = exp2f(m - mn), sb = exp2f(mi[u] - mn);
+      l = l * sa + li[u] * sb;
+      acc.x = acc.x * sa + a[u].x * sb;
+      acc.y = acc.y * sa + a[u].y * sb;
+      acc.z = acc.z * sa + a[u].z * sb;
+      acc.w = acc.w * sa + a[u].w * sb;
+      m = mn;
+    }
   }
   if (lane == 0) { wm[warp] = m; wl[warp] = l; }
   *reinterpret_cast<float4*>(&wacc[warp][4 * lane]) = acc;
   __syncthreads();
   if (warp == 0) {
     float M = -INFINITY;
-    for (int w = 0; w < 8; ++w) M = fmaxf(M, wm[w]);
+    for (int w = 0; w < kCombWarps; ++w) M = fmaxf(M, wm[w]);
     float den = 0.f;
     float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int w = 0; w < 8; ++w) {
+    for (int w = 0; w < kCombWarps; ++w) {
       if (wm[w] == -INFINITY) continue;
       const float sc = exp2f(wm[w] - M);
       den = fmaf(sc, wl[w], den);
-      const float4 a = *reinterpret_cast<const float4*>(&wacc[w][4 * lane]);
-      num.x = fmaf(sc, a.x, num.x);
-      num.y = fmaf(sc, a.y, num.y);
-      num.z = fmaf(sc, a.z, num.z);
-      num.w = fmaf(sc, a.w, num.w);
+      const float4 v = *reinterpret_cast<const float4*>(&wacc[w][4 * lane]);
+      num.x = fmaf(sc, v.x, num.x);
+      num.y = fmaf(sc, v.y, num.y);
+      num.z = fmaf(sc, v.z, num.z);
+      num.w = fmaf(sc, v.w, num.w);
     }
     const float inv = 1.f / den;
-    float4 o = make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
+    const float4 o = make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
     *reinterpret_cast<float4*>(P.out + ((size_t)b * P.Hq + (size_t)g * G + h) * kHeadDim + 4 * lane) = o;
   }
   if (threadIdx.x == 0 && h == 0 && P.sel_count) P.sel_count[s] = P.is_ret[g] ? P.ws.st[s].count : 0;
@@ -332,10 +353,10 @@ cudaError_t launch_attend(const StepParams& P, int kv_dtype, int grid, cudaStrea
 
 cudaError_t launch_combine(const StepParams& P, cudaStream_t st) {
   switch (P.G) {
-    case 1: k_combine<1><<<P.n_slices * 1, 256, 0, st>>>(P); break;
-    case 2: k_combine<2><<<P.n_slices * 2, 256, 0, st>>>(P); break;
-    case 4: k_combine<4><<<P.n_slices * 4, 256, 0, st>>>(P); break;
-    case 8: k_combine<8><<<P.n_slices * 8, 256, 0, st>>>(P); break;
+    case 1: k_combine<1><<<P.n_slices * 1, kCombWarps * 32, 0, st>>>(P); break;
+    case 2: k_combine<2><<<P.n_slices * 2, kCombWarps * 32, 0, st>>>(P); break;
+    case 4: k_combine<4><<<P.n_slices * 4, kCombWarps * 32, 0, st>>>(P); break;
+    case 8: k_combine<8><<<P.n_slices * 8, kCombWarps * 32, 0, st>>>(P); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

@@ -32,7 +32,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
-  size_t off[16];
+  size_t off[17];
   size_t total;
   int64_t max_items;
   int n_chunks_max;
@@ -46,14 +46,14 @@ Layout plan(const spa_config& c, int split_rows) {
   const int64_t Lmax = c.max_ctx;
   L.n_chunks_max = (int)((Lmax + spa::kChunk - 1) / spa::kChunk);
   L.max_items = (int64_t)slices * ((Lmax + split_rows - 1) / split_rows);
-  size_t sz[16] = {
+  size_t sz[17] = {
       (size_t)c.n_q_heads * 16 * 128 * 4,                  // 0 P_q
       (size_t)c.n_kv_heads * 16 * 128 * 4,                 // 1 P_k
       64 * 8,                                              // 2 inv_freq
       (size_t)c.max_batch * c.n_q_heads * 128 * 4,         // 3 q_rot
       (size_t)c.max_batch * c.n_q_heads * 16 * 4,          // 4 q_idx
       slices * L.n_chunks_max * G * 8,                     // 5 stats
-      slices * (size_t)Lmax * 4,                           // 6 pi
+      slices * (size_t)spa::pi_row_stride(Lmax) * 4,       // 6 pi
       slices * spa::kBins1 * 8,                            // 7 hist1
       slices * (size_t)Lmax * 8,                           // 8 cand
       slices * L.n_chunks_max * 4,                         // 9 chunk_gt
@@ -63,9 +63,10 @@ Layout plan(const spa_config& c, int split_rows) {
       (slices + 1) * 4,                                    // 13 item_base
       (size_t)L.max_items * G * spa::kPartStride * 4,      // 14 part
       256,                                                 // 15 dev_err
+      slices * spa::kBins2 * 8,                            // 16 hist2
   };
   size_t o = 0;
-  for (int i = 0; i < 16; ++i) {
+  for (int i = 0; i < 17; ++i) {
     L.off[i] = o;
     o += round_up(sz[i], 256);
   }
@@ -269,6 +270,7 @@ spa_status spa_create(spa_handle* out, const spa_config* cfg) {
   w.q_idx = (float*)(base + L.off[4]);
   w.stats = (float2*)(base + L.off[5]);
   w.pi = (float*)(base + L.off[6]);
+  w.pi_stride = spa::pi_row_stride(cfg->max_ctx);
   w.hist1 = (unsigned long long*)(base + L.off[7]);
   w.cand = (uint2*)(base + L.off[8]);
   w.chunk_gt = (int*)(base + L.off[9]);
@@ -278,11 +280,14 @@ spa_status spa_create(spa_handle* out, const spa_config* cfg) {
   w.item_base = (int*)(base + L.off[13]);
   w.part = (float*)(base + L.off[14]);
   w.dev_err = (unsigned*)(base + L.off[15]);
+  w.hist2 = (unsigned long long*)(base + L.off[16]);
   w.max_items = L.max_items;
   h->n_chunks_max = L.n_chunks_max;
 
   double invf[64];
-  for (int i = 0; i < 64; ++i) invf[i] = std::pow(cfg->rope_theta, -2.0 * i / 128.0);
+  // inverse frequencies theta^(-2i/128), stored divided by pi (the device works in units of pi)
+  const double kPi = 3.141592653589793238462643383279502884;
+  for (int i = 0; i < 64; ++i) invf[i] = std::pow(cfg->rope_theta, -2.0 * i / 128.0) / kPi;
   const size_t pq = (size_t)cfg->n_q_heads * 16 * 128 * 4, pk = (size_t)cfg->n_kv_heads * 16 * 128 * 4;
   if ((e = cudaMemcpy(w.P_q, cfg->P_q, pq, cudaMemcpyDeviceToDevice)) != cudaSuccess ||
       (e = cudaMemcpy(w.P_k, cfg->P_k, pk, cudaMemcpyDeviceToDevice)) != cudaSuccess ||

@@ -58,16 +58,20 @@ struct __align__(16) SliceState {
   int pad_;
 };
 
+__host__ __device__ inline int64_t pi_row_stride(int64_t Lmax) { return (Lmax + 63) / 64 * 64; }
+
 // Device workspace carved out of one allocation.
 struct Workspace {
   float* P_q;            // [Hq][16][128]
   float* P_k;            // [Hkv][16][128]
-  double* inv_freq;      // [64]
+  double* inv_freq;      // [64] RoPE inverse frequencies divided by pi
   float* q_rot;          // [Bm][Hq][128]
   float* q_idx;          // [Bm][Hq][16]
   float2* stats;         // [Bm*Hkv][n_chunks_max][G]  (m in log2 units, z)
-  float* pi;             // [Bm*Hkv][Lmax]
+  float* pi;             // [Bm*Hkv][pi_stride]
+  int64_t pi_stride;     // Lmax rounded up to 64 floats (256-byte rows)
   unsigned long long* hist1;  // [Bm*Hkv][kBins1]
+  unsigned long long* hist2;  // [Bm*Hkv][kBins2] round-2 masses of the round-1 cut bin
   uint2* cand;           // [Bm*Hkv][Lmax]  (prob bits, position)
   int* chunk_gt;         // [Bm*Hkv][n_chunks_max]
   int* chunk_off;        // [Bm*Hkv][n_chunks_max]

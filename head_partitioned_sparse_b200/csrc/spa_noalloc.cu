@@ -125,13 +125,14 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
       (size_t)B * n_q_heads * spa::kHeadDim * 4,               // q_rot
       (size_t)B * n_q_heads * spa::kIdxDim * 4,                // q_idx
       (size_t)slices * P.n_chunks * G * 8,                     // stats
-      (size_t)slices * max_ctx * 4,                            // pi
+      (size_t)slices * spa::pi_row_stride(max_ctx) * 4,        // pi
       (size_t)slices * spa::kBins1 * 8,                        // hist1
       (size_t)slices * max_ctx * 8,                            // candidates
       (size_t)slices * P.n_chunks * 4,                         // chunk_gt
       (size_t)slices * P.n_chunks * 4,                         // chunk_off
       (size_t)slices * sizeof(spa::SliceState),                // state
       256,                                                     // device status word
+      (size_t)slices * spa::kBins2 * 8,                        // hist2
   };
   size_t off[sizeof sz / sizeof sz[0]];
   size_t o = 0;
@@ -147,12 +148,14 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
   w.q_idx = (float*)(base + off[2]);
   w.stats = (float2*)(base + off[3]);
   w.pi = (float*)(base + off[4]);
+  w.pi_stride = spa::pi_row_stride(max_ctx);
   w.hist1 = (unsigned long long*)(base + off[5]);
   w.cand = (uint2*)(base + off[6]);
   w.chunk_gt = (int*)(base + off[7]);
   w.chunk_off = (int*)(base + off[8]);
   w.st = (spa::SliceState*)(base + off[9]);
   w.dev_err = (unsigned*)(base + off[10]);
+  w.hist2 = (unsigned long long*)(base + off[11]);
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = spa::launch_prologue(P, kv_dtype, st);
