@@ -29,9 +29,8 @@ SPA_ERR_DEVICE_RANGE = -6
 SPA_BF16 = 0
 SPA_F32 = 1
 
-SPA_K_INDEX_APPEND, SPA_K_PROLOGUE, SPA_K_SCORE, SPA_K_MASS, SPA_K_THRESHOLD, SPA_K_COMPACT, \
-    SPA_K_ATTEND, SPA_K_COMBINE = range(8)
-SPA_K_COUNT = 8
+SPA_K_INDEX_APPEND, SPA_K_SELECT, SPA_K_ATTEND, SPA_K_COMBINE = range(4)
+SPA_K_COUNT = 4
 
 
 class SpaError(RuntimeError):

@@ -1,4 +1,5 @@
-// Query prologue and top-p token selection for the retrieval heads.
+// Query prologue and top-p token selection for the retrieval heads, as one
+// cooperative persistent kernel.
 //
 // "Full Attention Strikes Back" (RTPurbo summary):
 //   Methodology §2  index scores in a 16-dim pre-RoPE subspace;
@@ -7,24 +8,29 @@
 // Group mean of per-head probabilities: "Autonomy of Heads" summary, Deployment
 // strategy (GQA scores aggregated to the group by their mean).
 //
-// Pipeline for every retrieval slice s = (b, g), over chunks of kChunk tokens:
-//   k_prologue   q_rot = RoPE(q_pre, L-1) (float64 angles), q_idx = P_q q_pre,
-//                reset of the slice's selection state;
-//   k_score      per chunk and head h: m = max_j l_hj, z = sum_j 2^(l_hj - m),
-//                l_hj = log2(e) * idx_scale * <q_idx[h], idx_j>   (idx read #1);
-//   k_mass       merge (m, z) over chunks -> M_h, Z_h; recompute l_hj (idx read #2),
-//                pi_j = sum_h 2^(l_hj - M_h) / (G Z_h), stored as fp32; a mass
-//                histogram over the top 12 bits of pi_j's bit pattern, with
-//                masses quantised to integer multiples of 2^-60 so every sum is
-//                exact and order independent.  The last CTA of the slice finds
-//                the bin b1 where the descending cumulative mass reaches p;
-//   k_threshold  counts tokens above b1 per chunk and appends the tokens of bin
-//                b1 to a candidate list; the last CTA resolves the exact cut value
-//                tau (two more radix rounds over the candidates), the tie quota
-//                at tau (lowest positions first) and per-chunk output offsets;
-//   k_compact    writes kept positions outside sinks/window, ascending.
-// No kernel waits on another CTA: cross-CTA steps use kernel boundaries or a
-// "last CTA to finish" ticket.
+// Phases, separated by grid-wide barriers (units: retrieval slices s = (b, g) and
+// their chunks of kChunk tokens; CTAs take units in grid-stride order):
+//   prologue  q_rot = RoPE(q_pre, L-1) for every head (angles in float64, reduced
+//             exactly in units of pi), q_idx = P_q q_pre (float64 dot products),
+//             reset of each retrieval slice's selection state;
+//   score     per chunk and head h: m = max_j l_hj, z = sum_j 2^(l_hj - m),
+//             l_hj = log2(e) * idx_scale * <q_idx[h], idx_j>   (index read #1);
+//   mass      merge (m, z) over chunks -> M_h, Z_h; recompute l_hj (index read #2),
+//             pi_j = sum_h 2^(l_hj - M_h) / (G Z_h), stored as fp32; a mass histogram
+//             over the top 12 bits of pi_j's bit pattern, masses quantised to integer
+//             multiples of 2^-60 so every sum is exact and order independent;
+//   cut 1     per slice: total mass, target ceil(p * total) and the bin b1 where the
+//             descending cumulative mass reaches it;
+//   threshold per chunk: tokens above b1 counted, tokens of bin b1 appended as
+//             candidates with their round-2 masses added to the slice histogram;
+//   refine    per slice: round-2 bin b2 from the histogram, one pass over the
+//             candidates for round 3 (exact cut value tau), the tie quota at tau
+//             (lowest positions first) and per-chunk output offsets;
+//   compact   per chunk: kept positions outside sinks/window, ascending.
+// One launch replaces a chain of small kernels whose fixed launch cost dominated.
+// Grid barriers spin on a generation word with a clock budget; on timeout they set a
+// device status bit and every CTA leaves the kernel.  The launch is cooperative, so
+// all CTAs are resident together.
 #include <climits>
 
 #include "spa_internal.cuh"
@@ -148,16 +154,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float x, float y) {
 template <int G>
 __device__ __forceinline__ int lane_head(int t4, int nh) { return G <= 4 ? t4 : t4 + 4 * nh; }
 
-struct SliceCoord {
-  int s, b, g, c, L;
-};
 
+// Stages the group's query index vectors in shared memory (qsm, G * 16 floats), then
+// builds the lane's B fragments from there.  Called by every thread of the CTA.
 template <int G>
-__device__ __forceinline__ void load_qidx_frag(const StepParams& P, int b, int g,
+__device__ __forceinline__ void load_qidx_frag(const StepParams& P, int b, int g, float* qsm,
                                                uint32_t (&qb)[IdxTiles<G>::NT][2]) {
-  __shared__ float qsm[G * kIdxDim];
   const int lane = threadIdx.x & 31, gid = lane >> 2, t4 = lane & 3;
-  if (threadIdx.x < G * kIdxDim) qsm[threadIdx.x] = P.ws.q_idx[((size_t)b * P.Hq + (size_t)g * G) * kIdxDim + threadIdx.x];
+  if (threadIdx.x < G * kIdxDim)   // written by another CTA in an earlier phase: read through L2
+    qsm[threadIdx.x] = __ldcg(&P.ws.q_idx[((size_t)b * P.Hq + (size_t)g * G) * kIdxDim + threadIdx.x]);
   __syncthreads();
   const float* qbase = qsm;
 #pragma unroll
@@ -251,32 +256,113 @@ __device__ __forceinline__ void online_add(float& m, float& z, float l) {
 }
 
 
-// Every CTA of a slice needs the same few scalars; one thread loads each of them and
-// shares it, so thousands of warps do not queue on one L2 line.
-__device__ __forceinline__ SliceCoord slice_coord(const StepParams& P) {
-  __shared__ int s_len;
-  SliceCoord sc;
-  const int y = blockIdx.y;
-  sc.b = y / P.n_ret;
-  sc.g = P.ret_heads[y % P.n_ret];
-  sc.s = sc.b * P.Hkv + sc.g;
-  sc.c = blockIdx.x;
-  if (threadIdx.x == 0) s_len = load_len(P.seq_lens, sc.b, P.Lcap, P.ws.dev_err);
+
+// ------------------------------------------------------------------ grid barrier
+constexpr long long kBarrierCycles = 4000000000LL;   // ~2 s bound per barrier
+
+// Sense-reversing barrier over all CTAs of a cooperative launch: bar[0] counts
+// arrivals (reset by the last arriver), bar[32] is the generation (a separate
+// 128-byte line, so polling does not delay the arrivals).  Returns false (on every
+// thread of the CTA) if the wait gave up.
+__device__ bool grid_barrier(unsigned* bar, unsigned* err, int* s_ok) {
   __syncthreads();
-  sc.L = s_len;
-  return sc;
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    volatile unsigned* gen = bar + 32;
+    const unsigned g = *gen;
+    __threadfence();
+    const unsigned arrived = atomicAdd(bar, 1u);
+    if (arrived == gridDim.x - 1) {
+      atomicExch(bar, 0u);
+      __threadfence();
+      atomicAdd(bar + 32, 1u);
+    } else {
+      const long long t0 = clock64();
+      unsigned ns = 32;
+      while (*gen == g) {
+        if (clock64() - t0 > kBarrierCycles) {
+          atomicOr(err, kErrTimeout);
+          ok = 0;
+          break;
+        }
+        __nanosleep(ns);
+        if (ns < 256) ns <<= 1;
+      }
+    }
+    __threadfence();
+    *s_ok = ok;
+  }
+  __syncthreads();
+  return *s_ok != 0;
 }
 
-// ------------------------------------------------------------------ prologue
-// One CTA per (b, kv head), 256 threads.  cos/sin of the 64 RoPE angles are formed
-// once in float64 and shared; each warp owns index outputs (h, r) and reduces the
-// 128-term float64 dot product P_q[h][r] . q_pre[h] across its lanes.
+// "Last CTA of the slice" ticket: every unit of the slice takes one; the CTA that
+// takes the last runs the per-slice step.  Called by every thread of the CTA.
+__device__ bool last_of_slice(unsigned* ticket, unsigned n_units, int* s_flag) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) *s_flag = atomicAdd(ticket, 1u) == n_units - 1;
+  __syncthreads();
+  if (*s_flag) __threadfence();
+  return *s_flag != 0;
+}
+
+// ------------------------------------------------------------------ shared memory
+constexpr int kSmallCap = 1024;   // candidates of the round-2 cut bin held in shared memory
+constexpr int kCandBatch = 8;     // candidates loaded per thread before any is used
+
+struct SmemPro { double cs[kHeadDim / 2], sn[kHeadDim / 2]; };
+struct SmemScore { float2 red[kSelThreads / 32][kMaxGroup]; };
+struct SmemMass { unsigned long long hist[kBins1]; float Mh[kMaxGroup], Wh[kMaxGroup]; };
+struct SmemRefine {
+  int chunk_sel[kMaxChunks];      // kept candidates per chunk (listed ones)
+  unsigned cnt4k[4096];           // position-select histogram
+  uint2 small[kSmallCap];         // candidates of the round-2 cut bin
+  unsigned long long m3[kBins3];
+  unsigned c3[kBins3];
+};
+union SelSmem {
+  SmemPro pro;
+  SmemScore score;
+  SmemMass mass;
+  SmemRefine ref;
+};
+// Scalars shared by the threads of a CTA (outside the union: live across calls).
+struct SelScalars {
+  float qsm[kMaxGroup * kIdxDim];
+  unsigned long long shl[32];
+  unsigned shu[32];
+  int shi[32];
+  int L, b1, b2, b3, kbin, fbin, cut_bin, pos_cut, off, ok;
+  unsigned small_n, kbefore, fbefore, tau;
+  unsigned long long above2, cut_above;
+};
+
+// Unit coordinates: retrieval slice y -> (b, g, s).
+struct Unit {
+  int b, g, s;
+};
+__device__ __forceinline__ Unit unit_of(const StepParams& P, int y) {
+  Unit u;
+  u.b = y / P.n_ret;
+  u.g = P.ret_heads[y % P.n_ret];
+  u.s = u.b * P.Hkv + u.g;
+  return u;
+}
+// Sequence length of b, loaded by one thread and shared (every CTA of a slice needs it).
+__device__ __forceinline__ int cta_len(const StepParams& P, int b, SelScalars& sc) {
+  __syncthreads();   // previous readers of sc.L are done
+  if (threadIdx.x == 0) sc.L = load_len(P.seq_lens, b, P.Lcap, P.ws.dev_err);
+  __syncthreads();
+  return sc.L;
+}
+
+// ------------------------------------------------------------------ prologue phase
+// Unit: one (b, kv head) slice of every head (streaming ones included).
 template <typename T>
-__global__ void __launch_bounds__(256) k_prologue(StepParams P) {
-  __shared__ double cs_s[kHeadDim / 2], sn_s[kHeadDim / 2];
-  const int s = blockIdx.x;
+__device__ void prologue_unit(const StepParams& P, SmemPro& sm, SelScalars& sc, int s) {
   const int b = s / P.Hkv, g = s % P.Hkv, G = P.G;
-  const int L = load_len(P.seq_lens, b, P.Lcap, P.ws.dev_err);
+  const int L = cta_len(P, b, sc);
   const T* q = (const T*)P.q_pre + ((size_t)b * P.Hq + (size_t)g * G) * kHeadDim;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid < kHeadDim / 2) {
@@ -285,7 +371,7 @@ __global__ void __launch_bounds__(256) k_prologue(StepParams P) {
     // sincospi evaluates the reduced angle: no large-argument reduction on the device.
     const double t = (double)(L - 1) * P.ws.inv_freq[tid];
     const double r = t - 2.0 * rint(0.5 * t);
-    sincospi(r, &sn_s[tid], &cs_s[tid]);
+    sincospi(r, &sm.sn[tid], &sm.cs[tid]);
   }
   __syncthreads();
   for (int t = tid; t < G * (kHeadDim / 2); t += blockDim.x) {
@@ -293,36 +379,40 @@ __global__ void __launch_bounds__(256) k_prologue(StepParams P) {
     const double x1 = Elem<T>::get(q, h * kHeadDim + i);
     const double x2 = Elem<T>::get(q, h * kHeadDim + i + kHeadDim / 2);
     float* o = P.ws.q_rot + ((size_t)b * P.Hq + (size_t)g * G + h) * kHeadDim;
-    o[i] = (float)(x1 * cs_s[i] - x2 * sn_s[i]);
-    o[i + kHeadDim / 2] = (float)(x2 * cs_s[i] + x1 * sn_s[i]);
+    o[i] = (float)(x1 * sm.cs[i] - x2 * sm.sn[i]);
+    o[i + kHeadDim / 2] = (float)(x2 * sm.cs[i] + x1 * sm.sn[i]);
   }
   if (P.is_ret[g]) {
-    // warp w owns outputs o = w + 8k (k < 2G); every projector load of the warp is issued
-    // before the first reduction
+    // warp w owns index outputs o = w + 8k; projector rows are loaded four outputs at a
+    // time before their float64 dot products are reduced across the warp
     constexpr int kMaxOut = kMaxGroup * kIdxDim / 8;
+    constexpr int kBatch = 4;
     const int nw = blockDim.x / 32;
-    float pv[kMaxOut][kHeadDim / 32];
 #pragma unroll
-    for (int k = 0; k < kMaxOut; ++k) {
-      const int o = warp + nw * k;
-      if (o < G * kIdxDim) {
-        const float* pq = P.ws.P_q + ((size_t)g * G * kIdxDim + o) * kHeadDim;
+    for (int k0 = 0; k0 < kMaxOut; k0 += kBatch) {
+      float pv[kBatch][kHeadDim / 32];
 #pragma unroll
-        for (int e = 0; e < kHeadDim / 32; ++e) pv[k][e] = pq[lane + 32 * e];
+      for (int k = 0; k < kBatch; ++k) {
+        const int o = warp + nw * (k0 + k);
+        if (o < G * kIdxDim) {
+          const float* pq = P.ws.P_q + ((size_t)g * G * kIdxDim + o) * kHeadDim;
+#pragma unroll
+          for (int e = 0; e < kHeadDim / 32; ++e) pv[k][e] = pq[lane + 32 * e];
+        }
       }
-    }
 #pragma unroll
-    for (int k = 0; k < kMaxOut; ++k) {
-      const int o = warp + nw * k;
-      if (o < G * kIdxDim) {
-        const int h = o / kIdxDim, r = o % kIdxDim;
-        double acc = 0.0;
+      for (int k = 0; k < kBatch; ++k) {
+        const int o = warp + nw * (k0 + k);
+        if (o < G * kIdxDim) {
+          const int h = o / kIdxDim, r = o % kIdxDim;
+          double acc = 0.0;
 #pragma unroll
-        for (int e = 0; e < kHeadDim / 32; ++e)
-          acc += (double)pv[k][e] * (double)Elem<T>::get(q, h * kHeadDim + lane + 32 * e);
+          for (int e = 0; e < kHeadDim / 32; ++e)
+            acc += (double)pv[k][e] * (double)Elem<T>::get(q, h * kHeadDim + lane + 32 * e);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(kFull, acc, off);
-        if (lane == 0) P.ws.q_idx[((size_t)b * P.Hq + (size_t)g * G + h) * kIdxDim + r] = (float)acc;
+          for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(kFull, acc, off);
+          if (lane == 0) P.ws.q_idx[((size_t)b * P.Hq + (size_t)g * G + h) * kIdxDim + r] = (float)acc;
+        }
       }
     }
     unsigned long long* h1 = P.ws.hist1 + (size_t)s * kBins1;
@@ -336,7 +426,8 @@ __global__ void __launch_bounds__(256) k_prologue(StepParams P) {
       z.tau_bits = 0u;
       z.pos_cut = INT_MAX;
       z.count = 0;
-      z.ticket_mass = z.ticket_thr = z.cand_count = 0u;
+      z.cand_count = 0u;
+      z.ticket_mass = z.ticket_thr = 0u;
       z.pad_ = 0;
       P.ws.st[s] = z;
     }
@@ -344,35 +435,34 @@ __global__ void __launch_bounds__(256) k_prologue(StepParams P) {
     P.ws.st[s].count = 0;
     if (P.sel_count) P.sel_count[s] = 0;
   }
+  __syncthreads();   // sm.cs / sm.sn reused by the next unit
 }
 
-// ------------------------------------------------------------------ k_score
-// Warp w of a chunk's CTA takes the 16-token groups w, w + 8, ... (4 in flight).
+// ------------------------------------------------------------------ score phase
+// Warp w of the CTA takes the 16-token groups w, w + 8, ... of the chunk (8 in flight).
 template <int G>
-__global__ void __launch_bounds__(kSelThreads) k_score(StepParams P) {
+__device__ void score_unit(const StepParams& P, SmemScore& sm, SelScalars& sc, int y, int c) {
   constexpr int NH = IdxTiles<G>::NH, U = 8;
   constexpr int kGroups = kChunk / 16, kWarps = kSelThreads / 32;
-  __shared__ float2 red[kWarps][G];
-  const SliceCoord sc = slice_coord(P);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, t4 = lane & 3;
-  const int j0 = sc.c * kChunk;
-  float2* out = P.ws.stats + ((size_t)sc.s * P.n_chunks + sc.c) * G;
-  if (j0 >= sc.L) {
+  const Unit un = unit_of(P, y);
+  const int L = cta_len(P, un.b, sc);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, t4 = lane & 3, gid = lane >> 2;
+  const int j0 = c * kChunk;
+  float2* out = P.ws.stats + ((size_t)un.s * P.n_chunks + c) * G;
+  if (j0 >= L) {
     if (threadIdx.x < G) out[threadIdx.x] = make_float2(-INFINITY, 0.f);
     return;
   }
   uint32_t qb[IdxTiles<G>::NT][2];
-  load_qidx_frag<G>(P, sc.b, sc.g, qb);
+  load_qidx_frag<G>(P, un.b, un.g, sc.qsm, qb);
   const float scale = P.idx_scale_log2;
-  const int jend = min(sc.L, j0 + kChunk);
-  const uint2* rows = reinterpret_cast<const uint2*>(P.idx_cache + (size_t)sc.s * P.Lmax * kIdxDim);
-  // two independent online accumulators per head (tokens gid and gid + 8) keep the
-  // exp2 dependency chains short; merged below
+  const int jend = min(L, j0 + kChunk);
+  const uint2* rows = reinterpret_cast<const uint2*>(P.idx_cache + (size_t)un.s * P.Lmax * kIdxDim);
+  // two independent online accumulators per head (tokens gid and gid + 8)
   float m[NH][2], z[NH][2];
 #pragma unroll
   for (int h = 0; h < NH; ++h) { m[h][0] = m[h][1] = -INFINITY; z[h][0] = z[h][1] = 0.f; }
   const uint64_t pol = l2_policy_keep();
-  const int gid = lane >> 2;
   for (int k = 0; k < kGroups / kWarps; k += U) {
     uint2 ra[U], rb[U];
 #pragma unroll
@@ -389,52 +479,44 @@ __global__ void __launch_bounds__(kSelThreads) k_score(StepParams P) {
       }
     }
   }
-#pragma unroll
-  for (int h = 0; h < NH; ++h) merge_mz(m[h][0], z[h][0], m[h][1], z[h][1]);
-  float mf[NH], zf[NH];
-#pragma unroll
-  for (int h = 0; h < NH; ++h) { mf[h] = m[h][0]; zf[h] = z[h][0]; }
   // lanes with the same t4 hold the same heads: merge over gid, then over warps
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
+    merge_mz(m[h][0], z[h][0], m[h][1], z[h][1]);
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
-      const float m2 = __shfl_xor_sync(kFull, mf[h], o);
-      const float z2 = __shfl_xor_sync(kFull, zf[h], o);
-      merge_mz(mf[h], zf[h], m2, z2);
+      const float m2 = __shfl_xor_sync(kFull, m[h][0], o);
+      const float z2 = __shfl_xor_sync(kFull, z[h][0], o);
+      merge_mz(m[h][0], z[h][0], m2, z2);
     }
     const int head = lane_head<G>(t4, h);
-    if (lane < 4 && head < G) red[warp][head] = make_float2(mf[h], zf[h]);
+    if (lane < 4 && head < G) sm.red[warp][head] = make_float2(m[h][0], z[h][0]);
   }
   __syncthreads();
   if (threadIdx.x < G) {
     const int h = threadIdx.x;
     float mm = -INFINITY, zz = 0.f;
-    for (int w = 0; w < kWarps; ++w) merge_mz(mm, zz, red[w][h].x, red[w][h].y);
+    for (int w = 0; w < kWarps; ++w) merge_mz(mm, zz, sm.red[w][h].x, sm.red[w][h].y);
     out[h] = make_float2(mm, zz);
   }
+  __syncthreads();   // sm.red reused by the next unit
 }
 
-// ------------------------------------------------------------------ k_mass
+// ------------------------------------------------------------------ mass phase
 template <int G>
-__global__ void __launch_bounds__(kSelThreads) k_mass(StepParams P) {
-  __shared__ unsigned long long hist[kBins1];
-  __shared__ float Mh[G], Wh[G];
-  __shared__ unsigned long long sh[32];
-  __shared__ int last_flag;
-  __shared__ int cut_bin;
-  __shared__ unsigned long long cut_above;
-  const SliceCoord sc = slice_coord(P);
+__device__ void mass_unit(const StepParams& P, SmemMass& sm, SelScalars& sc, int y, int c) {
+  const Unit un = unit_of(P, y);
+  const int L = cta_len(P, un.b, sc);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int j0 = sc.c * kChunk;
-
-  for (int i = tid; i < kBins1; i += kSelThreads) hist[i] = 0ull;
+  const int j0 = c * kChunk;
+  if (j0 >= L) return;
+  for (int i = tid; i < kBins1; i += kSelThreads) sm.hist[i] = 0ull;
   // global (M_h, Z_h): warp h merges the chunk partials, in a fixed order
   if (warp < G) {
-    const int nc = (sc.L + kChunk - 1) / kChunk;
+    const int nc = (L + kChunk - 1) / kChunk;
     float m = -INFINITY, z = 0.f;
-    for (int c = lane; c < nc; c += 32) {
-      const float2 v = P.ws.stats[((size_t)sc.s * P.n_chunks + c) * G + warp];
+    for (int cc = lane; cc < nc; cc += 32) {
+      const float2 v = __ldcg(&P.ws.stats[((size_t)un.s * P.n_chunks + cc) * G + warp]);
       merge_mz(m, z, v.x, v.y);
     }
 #pragma unroll
@@ -444,29 +526,28 @@ __global__ void __launch_bounds__(kSelThreads) k_mass(StepParams P) {
       merge_mz(m, z, m2, z2);
     }
     if (lane == 0) {
-      Mh[warp] = m;
-      Wh[warp] = 1.f / ((float)G * z);
+      sm.Mh[warp] = m;
+      sm.Wh[warp] = 1.f / ((float)G * z);
     }
   }
   __syncthreads();
-
-  if (j0 < sc.L) {
+  {
     constexpr int NH = IdxTiles<G>::NH, U = 8;
     constexpr int kGroups = kChunk / 16, kWarps = kSelThreads / 32;
     uint32_t qb[IdxTiles<G>::NT][2];
-    load_qidx_frag<G>(P, sc.b, sc.g, qb);
+    load_qidx_frag<G>(P, un.b, un.g, sc.qsm, qb);
     const float scale = P.idx_scale_log2;
     const int gid = lane >> 2, t4 = lane & 3;
     float M[NH], W[NH];
 #pragma unroll
     for (int h = 0; h < NH; ++h) {
       const int head = lane_head<G>(t4, h);
-      M[h] = head < G ? Mh[head] : 0.f;
-      W[h] = head < G ? Wh[head] : 0.f;   // lanes of absent heads contribute nothing
+      M[h] = head < G ? sm.Mh[head] : 0.f;
+      W[h] = head < G ? sm.Wh[head] : 0.f;   // lanes of absent heads contribute nothing
     }
-    const int jend = min(sc.L, j0 + kChunk);
-    const uint2* rows = reinterpret_cast<const uint2*>(P.idx_cache + (size_t)sc.s * P.Lmax * kIdxDim);
-    float* pi = P.ws.pi + (size_t)sc.s * P.ws.pi_stride;
+    const int jend = min(L, j0 + kChunk);
+    const uint2* rows = reinterpret_cast<const uint2*>(P.idx_cache + (size_t)un.s * P.Lmax * kIdxDim);
+    float* pi = P.ws.pi + (size_t)un.s * P.ws.pi_stride;
     const uint64_t pol = l2_policy_drop();
     for (int k = 0; k < kGroups / kWarps; k += U) {
       uint2 ra[U], rb[U];
@@ -481,13 +562,13 @@ __global__ void __launch_bounds__(kSelThreads) k_mass(StepParams P) {
         // then the 4 lanes of a token (fixed order, identical result in every lane)
         float pr[2];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int cc = 0; cc < 2; ++cc) {
           float acc = 0.f;
 #pragma unroll
-          for (int h = 0; h < NH; ++h) acc += W[h] == 0.f ? 0.f : exp2f(lg[h][c] - M[h]) * W[h];
+          for (int h = 0; h < NH; ++h) acc += W[h] == 0.f ? 0.f : exp2f(lg[h][cc] - M[h]) * W[h];
           acc += __shfl_xor_sync(kFull, acc, 1);
           acc += __shfl_xor_sync(kFull, acc, 2);
-          pr[c] = acc;
+          pr[cc] = acc;
         }
         if (t4 < 2) {   // lane t4 = 0 stores token gid, t4 = 1 token gid + 8
           const int jt = j + gid + 8 * t4;
@@ -495,24 +576,24 @@ __global__ void __launch_bounds__(kSelThreads) k_mass(StepParams P) {
           if (jt < jend) {
             pi[jt] = v;
             const unsigned bits = __float_as_uint(v);
-            atomicAdd(&hist[min(bits >> 18, (unsigned)(kBins1 - 1))], mass_q(v));
+            atomicAdd(&sm.hist[min(bits >> 18, (unsigned)(kBins1 - 1))], mass_q(v));
           }
         }
       }
     }
   }
   __syncthreads();
-  unsigned long long* g1 = P.ws.hist1 + (size_t)sc.s * kBins1;
+  unsigned long long* g1 = P.ws.hist1 + (size_t)un.s * kBins1;
   for (int i = tid; i < kBins1; i += kSelThreads)
-    if (hist[i]) atomicAdd(g1 + i, hist[i]);
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) last_flag = (atomicAdd(&P.ws.st[sc.s].ticket_mass, 1u) == gridDim.x - 1);
-  __syncthreads();
-  if (!last_flag) return;
-  __threadfence();
+    if (sm.hist[i]) atomicAdd(g1 + i, sm.hist[i]);
+  __syncthreads();   // sm.hist reused by the next unit
+}
 
-  // ---- last CTA of this slice: total mass, target and the round-1 cut bin
+// ------------------------------------------------------------------ cut 1 (per slice)
+__device__ void cut1_slice(const StepParams& P, SelScalars& sc, int y) {
+  const Unit un = unit_of(P, y);
+  const int tid = threadIdx.x;
+  const unsigned long long* g1 = P.ws.hist1 + (size_t)un.s * kBins1;
   unsigned long long m16[16];
   unsigned long long tsum = 0;
 #pragma unroll
@@ -520,33 +601,28 @@ __global__ void __launch_bounds__(kSelThreads) k_mass(StepParams P) {
     m16[k] = __ldcg(g1 + (4095 - 16 * tid - k));
     tsum += m16[k];
   }
-  const unsigned long long total = block_sum(tsum, sh);
-  SliceState* st = P.ws.st + sc.s;
-  if (P.keep_all || total == 0ull) {
-    if (tid == 0) { st->q_total = total; st->target = total; st->b1 = -1; st->m_above = 0ull; }
-    return;
+  const unsigned long long total = block_sum(tsum, sc.shl);
+  SliceState* st = P.ws.st + un.s;
+  unsigned long long target = total;
+  bool keep_all = P.keep_all || total == 0ull;
+  if (!keep_all) {
+    target = (unsigned long long)ceil((double)P.p * (double)total);
+    if (target < 1ull) target = 1ull;
+    keep_all = target > total;   // cannot happen for p < 1; keep everything if it does
   }
-  unsigned long long target = (unsigned long long)ceil((double)P.p * (double)total);
-  if (target < 1ull) target = 1ull;
-  if (target > total) {  // cannot happen for p < 1; keep everything if it does
-    if (tid == 0) { st->q_total = total; st->target = target; st->b1 = -1; st->m_above = 0ull; }
-    return;
-  }
-  if (tid == 0) cut_bin = -1;
+  if (tid == 0) sc.cut_bin = -1;
   __syncthreads();
-  find_cut_desc_4096(m16, 0ull, target, sh, &cut_bin, &cut_above);
+  if (!keep_all) find_cut_desc_4096(m16, 0ull, target, sc.shl, &sc.cut_bin, &sc.cut_above);
   if (tid == 0) {
     st->q_total = total;
     st->target = target;
-    st->b1 = cut_bin;
-    st->m_above = cut_above;
+    st->b1 = keep_all ? -1 : sc.cut_bin;
+    st->m_above = keep_all ? 0ull : sc.cut_above;
   }
+  __syncthreads();
 }
 
-// ------------------------------------------------------------------ k_threshold
-constexpr int kSmallCap = 1024;   // candidates of the round-2 cut bin held in shared memory
-constexpr int kCandBatch = 8;     // candidates loaded per thread before any is used
-
+// ------------------------------------------------------------------ threshold phase
 // Calls f(bits, pos) for every candidate (in no particular order), kCandBatch
 // independent loads per thread at a time.
 template <class F>
@@ -571,36 +647,24 @@ __device__ __forceinline__ int listed_in(const SinkWindow& sw, int lo, int hi) {
   return b > a ? b - a : 0;
 }
 
-__global__ void __launch_bounds__(kSelThreads) k_threshold(StepParams P) {
-  __shared__ int chunk_sel[kMaxChunks];        // kept candidates per chunk (listed ones)
-  __shared__ unsigned cnt4k[4096];             // position-select histogram
-  __shared__ uint2 small[kSmallCap];           // candidates of the round-2 cut bin
-  __shared__ unsigned long long m3[kBins3];
-  __shared__ unsigned c3[kBins3];
-  __shared__ unsigned long long shl[32];
-  __shared__ unsigned shu[32];
-  __shared__ int shi[32];
-  __shared__ int last_flag, b2, b3, kbin, fbin;
-  __shared__ unsigned small_n, kbefore, fbefore;
-  __shared__ unsigned long long above2;
-  const SliceCoord sc = slice_coord(P);
+// Unit: one chunk.  Tokens above bin b1 counted (listed ones), tokens of bin b1
+// appended as candidates with their round-2 masses added to the slice histogram.
+__device__ void threshold_unit(const StepParams& P, SelScalars& sc, int y, int c) {
+  const Unit un = unit_of(P, y);
+  const int L = cta_len(P, un.b, sc);
   const int tid = threadIdx.x, lane = tid & 31;
-  const int j0 = sc.c * kChunk;
-  SliceState* st = P.ws.st + sc.s;
-  __shared__ int s_b1;
-  if (tid == 0) s_b1 = st->b1;
+  const int j0 = c * kChunk;
+  SliceState* st = P.ws.st + un.s;
+  if (tid == 0) sc.b1 = __ldcg(&st->b1);
   __syncthreads();
-  const int b1 = s_b1;
-  const SinkWindow sw(sc.L, P.n_sink, P.window);
-  const unsigned* pib = reinterpret_cast<const unsigned*>(P.ws.pi + (size_t)sc.s * P.ws.pi_stride);
-  uint2* cand = P.ws.cand + (size_t)sc.s * P.Lmax;
-  unsigned long long* h2 = P.ws.hist2 + (size_t)sc.s * kBins2;
-
-  // ---- every chunk: tokens above bin b1 (listed ones counted), tokens of bin b1
-  // appended as candidates with their round-2 masses added to the slice histogram
+  const int b1 = sc.b1;
+  const SinkWindow sw(L, P.n_sink, P.window);
+  const unsigned* pib = reinterpret_cast<const unsigned*>(P.ws.pi + (size_t)un.s * P.ws.pi_stride);
+  uint2* cand = P.ws.cand + (size_t)un.s * P.Lmax;
+  unsigned long long* h2 = P.ws.hist2 + (size_t)un.s * kBins2;
   int cnt = 0;
-  if (j0 < sc.L) {
-    const int jend = min(sc.L, j0 + kChunk);
+  if (j0 < L) {
+    const int jend = min(L, j0 + kChunk);
     unsigned bits[kTokPerThread];
 #pragma unroll
     for (int i = 0; i < kTokPerThread; ++i) {
@@ -640,21 +704,31 @@ __global__ void __launch_bounds__(kSelThreads) k_threshold(StepParams P) {
       }
     }
   }
-  const int chunk_total = block_sum(cnt, shi);
-  if (tid == 0) P.ws.chunk_gt[(size_t)sc.s * P.n_chunks + sc.c] = chunk_total;
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) last_flag = (atomicAdd(&st->ticket_thr, 1u) == gridDim.x - 1);
-  __syncthreads();
-  if (!last_flag) return;
-  __threadfence();
+  const int chunk_total = block_sum(cnt, sc.shi);
+  if (tid == 0) P.ws.chunk_gt[(size_t)un.s * P.n_chunks + c] = chunk_total;
+}
 
-  // ---- last CTA of the slice: exact cut value, tie quota, per-chunk output offsets
+// ------------------------------------------------------------------ refine (per slice)
+__device__ void refine_slice(const StepParams& P, SmemRefine& sm, SelScalars& sc, int y) {
+  const Unit un = unit_of(P, y);
+  const int L = cta_len(P, un.b, sc);
+  const int tid = threadIdx.x;
+  SliceState* st = P.ws.st + un.s;
+  if (tid == 0) sc.b1 = __ldcg(&st->b1);
+  __syncthreads();
+  const int b1 = sc.b1;
+  const SinkWindow sw(L, P.n_sink, P.window);
+  const uint2* cand = P.ws.cand + (size_t)un.s * P.Lmax;
+  const unsigned long long* h2 = P.ws.hist2 + (size_t)un.s * kBins2;
+  int* chunk_sel = sm.chunk_sel;
+  unsigned* cnt4k = sm.cnt4k;
+  uint2* small = sm.small;
+  // exact cut value, tie quota, per-chunk output offsets
   unsigned tau = 0u;
   int pos_cut = INT_MAX;
   for (int c = tid; c < P.n_chunks; c += kSelThreads) chunk_sel[c] = 0;
-  if (tid < kBins3) { m3[tid] = 0ull; c3[tid] = 0u; }
-  if (tid == 0) { b2 = -1; b3 = -1; small_n = 0u; kbin = -1; }
+  if (tid < kBins3) { sm.m3[tid] = 0ull; sm.c3[tid] = 0u; }
+  if (tid == 0) { sc.b2 = -1; sc.b3 = -1; sc.small_n = 0u; sc.kbin = -1; }
   __syncthreads();
   bool found = b1 < 0;   // keep-everything mode needs no cut
   if (b1 >= 0) {
@@ -665,8 +739,8 @@ __global__ void __launch_bounds__(kSelThreads) k_threshold(StepParams P) {
     unsigned long long m16[16];
 #pragma unroll
     for (int k = 0; k < 16; ++k) m16[k] = __ldcg(h2 + (4095 - 16 * tid - k));
-    find_cut_desc_4096(m16, mab, target, shl, &b2, &above2);
-    const int cb2 = b2;
+    find_cut_desc_4096(m16, mab, target, sc.shl, &sc.b2, &sc.above2);
+    const int cb2 = sc.b2;
     // one pass over the candidates: above the round-2 bin they are kept; inside it
     // they feed round 3 (bits 5..0) and are parked in shared memory
     for_each_candidate(cand, n, [&](unsigned bits, int pos) {
@@ -674,31 +748,31 @@ __global__ void __launch_bounds__(kSelThreads) k_threshold(StepParams P) {
       if (d2 > cb2) {
         if (!sw.always(pos)) atomicAdd(&chunk_sel[pos / kChunk], 1);
       } else if (d2 == cb2) {
-        atomicAdd(&m3[bits & 63u], mass_q(__uint_as_float(bits)));
-        atomicAdd(&c3[bits & 63u], 1u);
-        const unsigned slot = atomicAdd(&small_n, 1u);
+        atomicAdd(&sm.m3[bits & 63u], mass_q(__uint_as_float(bits)));
+        atomicAdd(&sm.c3[bits & 63u], 1u);
+        const unsigned slot = atomicAdd(&sc.small_n, 1u);
         if (slot < kSmallCap) small[slot] = make_uint2(bits, (unsigned)pos);
       }
     });
     __syncthreads();
     if (tid == 0 && cb2 >= 0) {
-      unsigned long long cum = above2;
+      unsigned long long cum = sc.above2;
       for (int k = kBins3 - 1; k >= 0; --k) {
-        if (cum < target && cum + m3[k] >= target) { b3 = k; break; }
-        cum += m3[k];
+        if (cum < target && cum + sm.m3[k] >= target) { sc.b3 = k; break; }
+        cum += sm.m3[k];
       }
-      above2 = cum;   // mass strictly above tau
+      sc.above2 = cum;   // mass strictly above tau
     }
     __syncthreads();
     // b2 and b3 always exist (the candidates carry the mass of bin b1); if a search ever
     // failed, every token is kept rather than a missing bin indexed
-    found = cb2 >= 0 && b3 >= 0;
-    const bool small_ok = small_n <= (unsigned)kSmallCap;
-    const unsigned sn = small_ok ? small_n : 0u;
+    found = cb2 >= 0 && sc.b3 >= 0;
+    const bool small_ok = sc.small_n <= (unsigned)kSmallCap;
+    const unsigned sn = small_ok ? sc.small_n : 0u;
     if (found) {
-      tau = ((unsigned)b1 << 18) | ((unsigned)cb2 << 6) | (unsigned)b3;
-      const unsigned long long m_gt = above2;
-      const unsigned n_eq = c3[b3];
+      tau = ((unsigned)b1 << 18) | ((unsigned)cb2 << 6) | (unsigned)sc.b3;
+      const unsigned long long m_gt = sc.above2;
+      const unsigned n_eq = sm.c3[sc.b3];
       const unsigned long long q_tau = mass_q(__uint_as_float(tau));
       const unsigned long long need =
           (q_tau > 0ull && target > m_gt) ? (target - m_gt + q_tau - 1ull) / q_tau : ~0ull;
@@ -708,7 +782,7 @@ __global__ void __launch_bounds__(kSelThreads) k_threshold(StepParams P) {
         for (int pass = 0; pass < 2; ++pass) {
           for (int i = tid; i < 4096; i += kSelThreads) cnt4k[i] = 0u;
           __syncthreads();
-          const int kb = kbin;
+          const int kb = sc.kbin;
           auto add = [&](unsigned bits, int pos) {
             if (bits != tau) return;
             if (pass == 0) atomicAdd(&cnt4k[(unsigned)pos >> 12], 1u);
@@ -723,18 +797,18 @@ __global__ void __launch_bounds__(kSelThreads) k_threshold(StepParams P) {
           unsigned c16[16];
 #pragma unroll
           for (int k = 0; k < 16; ++k) c16[k] = cnt4k[16 * tid + k];
-          if (tid == 0) fbin = -1;
+          if (tid == 0) sc.fbin = -1;
           __syncthreads();
-          find_kth_asc_4096(c16, pass == 0 ? 0u : kbefore, qk, shu, &fbin, &fbefore);
+          find_kth_asc_4096(c16, pass == 0 ? 0u : sc.kbefore, qk, sc.shu, &sc.fbin, &sc.fbefore);
           if (tid == 0) {
-            if (fbin < 0) kbin = -1;
-            else if (pass == 0) { kbin = fbin; kbefore = fbefore; }
-            else if (kbin >= 0) kbin = (kbin << 12) | fbin;
+            if (sc.fbin < 0) sc.kbin = -1;
+            else if (pass == 0) { sc.kbin = sc.fbin; sc.kbefore = sc.fbefore; }
+            else if (sc.kbin >= 0) sc.kbin = (sc.kbin << 12) | sc.fbin;
           }
           __syncthreads();
-          if (kbin < 0) break;
+          if (sc.kbin < 0) break;
         }
-        pos_cut = kbin >= 0 ? kbin : INT_MAX;
+        pos_cut = sc.kbin >= 0 ? sc.kbin : INT_MAX;
       }
       // kept candidates of the round-2 cut bin
       const int pc = pos_cut;
@@ -755,8 +829,8 @@ __global__ void __launch_bounds__(kSelThreads) k_threshold(StepParams P) {
     tau = 0u;
     pos_cut = INT_MAX;
     for (int c = tid; c < P.n_chunks; c += kSelThreads)
-      chunk_sel[c] = listed_in(sw, c * kChunk, min(sc.L, (c + 1) * kChunk)) -
-                     __ldcg(&P.ws.chunk_gt[(size_t)sc.s * P.n_chunks + c]);
+      chunk_sel[c] = listed_in(sw, c * kChunk, min(L, (c + 1) * kChunk)) -
+                     __ldcg(&P.ws.chunk_gt[(size_t)un.s * P.n_chunks + c]);
     __syncthreads();
   }
   // offsets: exclusive scan over chunks of (above-b1 count + kept candidates)
@@ -765,47 +839,46 @@ __global__ void __launch_bounds__(kSelThreads) k_threshold(StepParams P) {
   int loc = 0;
   for (int k = 0; k < per; ++k) {
     const int c = c0 + k;
-    if (c < P.n_chunks) loc += __ldcg(&P.ws.chunk_gt[(size_t)sc.s * P.n_chunks + c]) + chunk_sel[c];
+    if (c < P.n_chunks) loc += __ldcg(&P.ws.chunk_gt[(size_t)un.s * P.n_chunks + c]) + chunk_sel[c];
   }
   int total = 0;
-  int run = block_excl_scan(loc, shi, &total);
+  int run = block_excl_scan(loc, sc.shi, &total);
   for (int k = 0; k < per; ++k) {
     const int c = c0 + k;
     if (c < P.n_chunks) {
-      P.ws.chunk_off[(size_t)sc.s * P.n_chunks + c] = run;
-      run += __ldcg(&P.ws.chunk_gt[(size_t)sc.s * P.n_chunks + c]) + chunk_sel[c];
+      P.ws.chunk_off[(size_t)un.s * P.n_chunks + c] = run;
+      run += __ldcg(&P.ws.chunk_gt[(size_t)un.s * P.n_chunks + c]) + chunk_sel[c];
     }
   }
   if (tid == 0) {
     st->tau_bits = tau;
     st->pos_cut = pos_cut;
     st->count = total;
-    if (P.sel_count) P.sel_count[sc.s] = total;
+    if (P.sel_count) P.sel_count[un.s] = total;
   }
+  __syncthreads();   // shared memory reused by the next unit
 }
 
-// ------------------------------------------------------------------ k_compact
-__global__ void __launch_bounds__(kSelThreads) k_compact(StepParams P) {
-  __shared__ int shi[32];
-  const SliceCoord sc = slice_coord(P);
-  const int j0 = sc.c * kChunk;
-  if (j0 >= sc.L) return;
-  __shared__ unsigned s_tau;
-  __shared__ int s_cut, s_off;
+// ------------------------------------------------------------------ compact phase
+__device__ void compact_unit(const StepParams& P, SelScalars& sc, int y, int c) {
+  const Unit un = unit_of(P, y);
+  const int L = cta_len(P, un.b, sc);
+  const int j0 = c * kChunk;
+  if (j0 >= L) return;
   if (threadIdx.x == 0) {
-    const SliceState* st = P.ws.st + sc.s;
-    s_tau = st->tau_bits;
-    s_cut = st->pos_cut;
-    s_off = P.ws.chunk_off[(size_t)sc.s * P.n_chunks + sc.c];
+    const SliceState* st = P.ws.st + un.s;
+    sc.tau = __ldcg(&st->tau_bits);
+    sc.pos_cut = __ldcg(&st->pos_cut);
+    sc.off = __ldcg(&P.ws.chunk_off[(size_t)un.s * P.n_chunks + c]);
   }
   __syncthreads();
-  const unsigned tau = s_tau;
-  const int pos_cut = s_cut;
-  const SinkWindow sw(sc.L, P.n_sink, P.window);
-  const unsigned* pib = reinterpret_cast<const unsigned*>(P.ws.pi + (size_t)sc.s * P.ws.pi_stride);
+  const unsigned tau = sc.tau;
+  const int pos_cut = sc.pos_cut;
+  const SinkWindow sw(L, P.n_sink, P.window);
+  const unsigned* pib = reinterpret_cast<const unsigned*>(P.ws.pi + (size_t)un.s * P.ws.pi_stride);
   const int jb = j0 + threadIdx.x * kTokPerThread;  // this thread's 16 consecutive tokens
   unsigned keep = 0u;
-  if (jb < sc.L) {
+  if (jb < L) {
     // rows of the probability buffer are padded to 64 floats: four 16-byte loads stay in the row
     const uint4* v4 = reinterpret_cast<const uint4*>(pib + jb);
     unsigned bits[kTokPerThread];
@@ -820,13 +893,13 @@ __global__ void __launch_bounds__(kSelThreads) k_compact(StepParams P) {
 #pragma unroll
     for (int i = 0; i < kTokPerThread; ++i) {
       const int j = jb + i;
-      const bool k = j < sc.L && (bits[i] > tau || (bits[i] == tau && j <= pos_cut)) && !sw.always(j);
+      const bool k = j < L && (bits[i] > tau || (bits[i] == tau && j <= pos_cut)) && !sw.always(j);
       keep |= (k ? 1u : 0u) << i;
     }
   }
-  const int off = block_excl_scan(__popc(keep), shi, (int*)nullptr);
-  const int64_t first = (int64_t)s_off + off;
-  int* dst = P.sel_list + (size_t)sc.s * P.Lmax;
+  const int off = block_excl_scan(__popc(keep), sc.shi, (int*)nullptr);
+  const int64_t first = (int64_t)sc.off + off;
+  int* dst = P.sel_list + (size_t)un.s * P.Lmax;
   int k = 0;
 #pragma unroll
   for (int i = 0; i < kTokPerThread; ++i) {
@@ -838,53 +911,95 @@ __global__ void __launch_bounds__(kSelThreads) k_compact(StepParams P) {
   }
 }
 
-template <int G>
-cudaError_t launch_score_g(const StepParams& P, cudaStream_t st) {
-  k_score<G><<<dim3(P.n_chunks, P.B * P.n_ret), kSelThreads, 0, st>>>(P);
-  return cudaGetLastError();
+// ------------------------------------------------------------------ the kernel
+template <typename T, int G>
+__global__ void __launch_bounds__(kSelThreads, 4) k_select(StepParams P) {
+  __shared__ SelSmem sm;
+  __shared__ SelScalars sc;
+  const int nb = gridDim.x;
+  for (int s = blockIdx.x; s < P.n_slices; s += nb) prologue_unit<T>(P, sm.pro, sc, s);
+  if (!grid_barrier(P.ws.bar, P.ws.dev_err, &sc.ok)) return;
+  if (P.n_ret == 0) return;
+  const int n_rs = P.B * P.n_ret;
+  const int n_units = n_rs * P.n_chunks;
+  for (int u = blockIdx.x; u < n_units; u += nb) score_unit<G>(P, sm.score, sc, u / P.n_chunks, u % P.n_chunks);
+  if (!grid_barrier(P.ws.bar, P.ws.dev_err, &sc.ok)) return;
+  for (int u = blockIdx.x; u < n_units; u += nb) {
+    const int y = u / P.n_chunks;
+    mass_unit<G>(P, sm.mass, sc, y, u % P.n_chunks);
+    if (last_of_slice(&P.ws.st[unit_of(P, y).s].ticket_mass, P.n_chunks, &sc.ok)) cut1_slice(P, sc, y);
+  }
+  if (!grid_barrier(P.ws.bar, P.ws.dev_err, &sc.ok)) return;
+  for (int u = blockIdx.x; u < n_units; u += nb) {
+    const int y = u / P.n_chunks;
+    threshold_unit(P, sc, y, u % P.n_chunks);
+    if (last_of_slice(&P.ws.st[unit_of(P, y).s].ticket_thr, P.n_chunks, &sc.ok)) refine_slice(P, sm.ref, sc, y);
+  }
+  if (!grid_barrier(P.ws.bar, P.ws.dev_err, &sc.ok)) return;
+  for (int u = blockIdx.x; u < n_units; u += nb) compact_unit(P, sc, u / P.n_chunks, u % P.n_chunks);
 }
-template <int G>
-cudaError_t launch_mass_g(const StepParams& P, cudaStream_t st) {
-  k_mass<G><<<dim3(P.n_chunks, P.B * P.n_ret), kSelThreads, 0, st>>>(P);
-  return cudaGetLastError();
+
+template <typename T, int G>
+cudaError_t launch_tg(const StepParams& P, int grid, cudaStream_t st) {
+  StepParams local = P;
+  void* args[] = {&local};
+  return cudaLaunchCooperativeKernel((const void*)k_select<T, G>, dim3(grid), dim3(kSelThreads), args, 0, st);
+}
+
+template <typename T, int G>
+int resident_tg() {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_select<T, G>, kSelThreads, 0) != cudaSuccess) return -1;
+  return n;
 }
 
 }  // namespace
 
-cudaError_t launch_prologue(const StepParams& P, int kv_dtype, cudaStream_t st) {
-  if (kv_dtype == 0) k_prologue<__nv_bfloat16><<<P.n_slices, 256, 0, st>>>(P);
-  else k_prologue<float><<<P.n_slices, 256, 0, st>>>(P);
-  return cudaGetLastError();
+// Grid of the selection launch: one CTA per unit of work, capped at what is resident.
+int select_grid(const StepParams& P, int max_resident) {
+  const int units = P.n_ret > 0 ? P.B * P.n_ret * P.n_chunks : 0;
+  int want = units > P.n_slices ? units : P.n_slices;
+  if (want < 1) want = 1;
+  return want < max_resident ? want : max_resident;
 }
 
-cudaError_t launch_score(const StepParams& P, cudaStream_t st) {
-  switch (P.G) {
-    case 1: return launch_score_g<1>(P, st);
-    case 2: return launch_score_g<2>(P, st);
-    case 4: return launch_score_g<4>(P, st);
-    case 8: return launch_score_g<8>(P, st);
+cudaError_t launch_select(const StepParams& P, int kv_dtype, int grid, cudaStream_t st) {
+  if (kv_dtype == 0) {
+    switch (P.G) {
+      case 1: return launch_tg<__nv_bfloat16, 1>(P, grid, st);
+      case 2: return launch_tg<__nv_bfloat16, 2>(P, grid, st);
+      case 4: return launch_tg<__nv_bfloat16, 4>(P, grid, st);
+      case 8: return launch_tg<__nv_bfloat16, 8>(P, grid, st);
+    }
+  } else {
+    switch (P.G) {
+      case 1: return launch_tg<float, 1>(P, grid, st);
+      case 2: return launch_tg<float, 2>(P, grid, st);
+      case 4: return launch_tg<float, 4>(P, grid, st);
+      case 8: return launch_tg<float, 8>(P, grid, st);
+    }
   }
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_mass(const StepParams& P, cudaStream_t st) {
-  switch (P.G) {
-    case 1: return launch_mass_g<1>(P, st);
-    case 2: return launch_mass_g<2>(P, st);
-    case 4: return launch_mass_g<4>(P, st);
-    case 8: return launch_mass_g<8>(P, st);
+// Co-resident CTAs of the selection kernel per SM for (dtype, G), or -1.
+int select_resident_per_sm(int kv_dtype, int G) {
+  if (kv_dtype == 0) {
+    switch (G) {
+      case 1: return resident_tg<__nv_bfloat16, 1>();
+      case 2: return resident_tg<__nv_bfloat16, 2>();
+      case 4: return resident_tg<__nv_bfloat16, 4>();
+      case 8: return resident_tg<__nv_bfloat16, 8>();
+    }
+  } else {
+    switch (G) {
+      case 1: return resident_tg<float, 1>();
+      case 2: return resident_tg<float, 2>();
+      case 4: return resident_tg<float, 4>();
+      case 8: return resident_tg<float, 8>();
+    }
   }
-  return cudaErrorInvalidValue;
-}
-
-cudaError_t launch_threshold(const StepParams& P, cudaStream_t st) {
-  k_threshold<<<dim3(P.n_chunks, P.B * P.n_ret), kSelThreads, 0, st>>>(P);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_compact(const StepParams& P, cudaStream_t st) {
-  k_compact<<<dim3(P.n_chunks, P.B * P.n_ret), kSelThreads, 0, st>>>(P);
-  return cudaGetLastError();
+  return -1;
 }
 
 }  // namespace spa

@@ -32,7 +32,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
-  size_t off[17];
+  size_t off[18];
   size_t total;
   int64_t max_items;
   int n_chunks_max;
@@ -46,7 +46,7 @@ Layout plan(const spa_config& c, int split_rows) {
   const int64_t Lmax = c.max_ctx;
   L.n_chunks_max = (int)((Lmax + spa::kChunk - 1) / spa::kChunk);
   L.max_items = (int64_t)slices * ((Lmax + split_rows - 1) / split_rows);
-  size_t sz[17] = {
+  size_t sz[18] = {
       (size_t)c.n_q_heads * 16 * 128 * 4,                  // 0 P_q
       (size_t)c.n_kv_heads * 16 * 128 * 4,                 // 1 P_k
       64 * 8,                                              // 2 inv_freq
@@ -64,9 +64,10 @@ Layout plan(const spa_config& c, int split_rows) {
       (size_t)L.max_items * G * spa::kPartStride * 4,      // 14 part
       256,                                                 // 15 dev_err
       slices * spa::kBins2 * 8,                            // 16 hist2
+      256,                                                 // 17 selection grid barrier
   };
   size_t o = 0;
-  for (int i = 0; i < 17; ++i) {
+  for (int i = 0; i < 18; ++i) {
     L.off[i] = o;
     o += round_up(sz[i], 256);
   }
@@ -92,6 +93,7 @@ struct spa_ctx {
   int device = 0;
   int num_sms = 0;
   int attend_occ = 1;
+  int select_max_grid = 1;   // co-resident CTAs of the cooperative selection kernel
   void* mem = nullptr;
   size_t mem_bytes = 0;
   spa::Workspace ws{};
@@ -207,15 +209,8 @@ spa_status check_step(spa_ctx* h, const StepArgs& a, spa::StepParams* P) {
 }
 
 spa_status run_selection(spa_ctx* h, spa::StepParams& P, cudaStream_t st) {
-  spa_status r;
-  if ((r = run(h, SPA_K_PROLOGUE, st, "prologue", [&] { return spa::launch_prologue(P, h->cfg.kv_dtype, st); })))
-    return r;
-  if (P.n_ret == 0) return SPA_OK;
-  if ((r = run(h, SPA_K_SCORE, st, "index score", [&] { return spa::launch_score(P, st); }))) return r;
-  if ((r = run(h, SPA_K_MASS, st, "index mass", [&] { return spa::launch_mass(P, st); }))) return r;
-  if ((r = run(h, SPA_K_THRESHOLD, st, "threshold", [&] { return spa::launch_threshold(P, st); }))) return r;
-  if ((r = run(h, SPA_K_COMPACT, st, "compact", [&] { return spa::launch_compact(P, st); }))) return r;
-  return SPA_OK;
+  const int grid = spa::select_grid(P, h->select_max_grid);
+  return run(h, SPA_K_SELECT, st, "select", [&] { return spa::launch_select(P, h->cfg.kv_dtype, grid, st); });
 }
 
 }  // namespace
@@ -281,6 +276,7 @@ spa_status spa_create(spa_handle* out, const spa_config* cfg) {
   w.part = (float*)(base + L.off[14]);
   w.dev_err = (unsigned*)(base + L.off[15]);
   w.hist2 = (unsigned long long*)(base + L.off[16]);
+  w.bar = (unsigned*)(base + L.off[17]);
   w.max_items = L.max_items;
   h->n_chunks_max = L.n_chunks_max;
 
@@ -292,7 +288,8 @@ spa_status spa_create(spa_handle* out, const spa_config* cfg) {
   if ((e = cudaMemcpy(w.P_q, cfg->P_q, pq, cudaMemcpyDeviceToDevice)) != cudaSuccess ||
       (e = cudaMemcpy(w.P_k, cfg->P_k, pk, cudaMemcpyDeviceToDevice)) != cudaSuccess ||
       (e = cudaMemcpy(w.inv_freq, invf, sizeof invf, cudaMemcpyHostToDevice)) != cudaSuccess ||
-      (e = cudaMemset(w.dev_err, 0, 4)) != cudaSuccess || (e = cudaDeviceSynchronize()) != cudaSuccess) {
+      (e = cudaMemset(w.dev_err, 0, 4)) != cudaSuccess || (e = cudaMemset(w.bar, 0, 256)) != cudaSuccess ||
+      (e = cudaDeviceSynchronize()) != cudaSuccess) {
     cudaFree(h->mem);
     delete h;
     return cuda_fail(e, "spa_create: copying projectors");
@@ -304,6 +301,13 @@ spa_status spa_create(spa_handle* out, const spa_config* cfg) {
     return fail(SPA_ERR_UNSUPPORTED, "attention kernel cannot be resident with this configuration");
   }
   h->attend_occ = occ;
+  const int sel_occ = spa::select_resident_per_sm(cfg->kv_dtype, h->G);
+  if (sel_occ < 1) {
+    cudaFree(h->mem);
+    delete h;
+    return fail(SPA_ERR_UNSUPPORTED, "selection kernel cannot be resident with this configuration");
+  }
+  h->select_max_grid = sel_occ * h->num_sms;
   *out = h;
   return SPA_OK;
 }
@@ -387,8 +391,12 @@ spa_status spa_device_status(spa_handle h, spa_stream stream) {
   if ((e = cudaMemcpy(&flags, h->ws.dev_err, 4, cudaMemcpyDeviceToHost)) != cudaSuccess) return cuda_fail(e, "read status");
   if (flags) {
     if ((e = cudaMemset(h->ws.dev_err, 0, 4)) != cudaSuccess) return cuda_fail(e, "clear status");
-    if (flags & spa::kErrTimeout)
+    if (flags & spa::kErrTimeout) {
+      // the grid barrier may have been left mid-way: start the next call from a clean barrier
+      cudaMemset(h->ws.bar, 0, 256);
+      cudaDeviceSynchronize();
       return fail(SPA_ERR_DEVICE_TIMEOUT, "a bounded device-side wait gave up (flags 0x%x)", flags);
+    }
     if (flags & spa::kErrInternal)
       return fail(SPA_ERR_CUDA, "internal consistency check failed in the selection kernels (flags 0x%x)", flags);
     return fail(SPA_ERR_DEVICE_RANGE, "device range check failed:%s%s",
@@ -433,8 +441,7 @@ spa_status spa_profile_read(spa_handle h, int kernel_id, double* total_ms, int64
 }
 
 const char* spa_kernel_name(int kernel_id) {
-  static const char* names[SPA_K_COUNT] = {"index_append", "prologue", "index_score", "index_mass",
-                                           "threshold",    "compact",  "attend",      "combine"};
+  static const char* names[SPA_K_COUNT] = {"index_append", "select", "attend", "combine"};
   return (kernel_id >= 0 && kernel_id < SPA_K_COUNT) ? names[kernel_id] : "";
 }
 

@@ -42,8 +42,8 @@ constexpr unsigned kErrStartPos = 2u;
 constexpr unsigned kErrInternal = 4u;
 constexpr unsigned kErrTimeout = 8u;   // a bounded device-side wait gave up
 
-// Per (b, kv head) selection state.  Written by the threshold kernels, read by
-// compaction and attention.
+// Per (b, kv head) selection state.  Written by the selection kernel, read by its
+// later phases and by attention.
 struct __align__(16) SliceState {
   unsigned long long q_total;   // sum of quantised masses (units of 2^-60)
   unsigned long long target;    // ceil(p * q_total)
@@ -52,7 +52,7 @@ struct __align__(16) SliceState {
   unsigned tau_bits;            // fp32 bits of the cut probability tau
   int pos_cut;                  // tied tokens (prob == tau) are kept iff pos <= pos_cut
   int count;                    // listed tokens (kept, outside sinks/window)
-  unsigned ticket_mass;         // last-block tickets
+  unsigned ticket_mass;         // last-CTA tickets of the mass and threshold phases
   unsigned ticket_thr;
   unsigned cand_count;          // candidates appended (tokens in bin b1)
   int pad_;
@@ -80,6 +80,7 @@ struct Workspace {
   int* item_base;        // [Bm*Hkv + 1]
   float* part;           // [max_items][G][kPartStride]
   unsigned* dev_err;     // [1]
+  unsigned* bar;         // [64] grid barrier of the selection kernel: [0] arrivals, [32] generation
   int64_t max_items;
 };
 
@@ -163,11 +164,9 @@ namespace spa {
 cudaError_t launch_index_append(const void* k_pre, const int64_t* start_pos, int B, int T, int Hkv,
                                 int64_t Lmax, int kv_dtype, const float* P_k, uint16_t* idx_cache,
                                 unsigned* dev_err, cudaStream_t st);
-cudaError_t launch_prologue(const StepParams& P, int kv_dtype, cudaStream_t st);
-cudaError_t launch_score(const StepParams& P, cudaStream_t st);
-cudaError_t launch_mass(const StepParams& P, cudaStream_t st);
-cudaError_t launch_threshold(const StepParams& P, cudaStream_t st);
-cudaError_t launch_compact(const StepParams& P, cudaStream_t st);
+cudaError_t launch_select(const StepParams& P, int kv_dtype, int grid, cudaStream_t st);
+int select_grid(const StepParams& P, int max_resident);
+int select_resident_per_sm(int kv_dtype, int G);
 cudaError_t launch_attend(const StepParams& P, int kv_dtype, int grid, cudaStream_t st);
 cudaError_t launch_combine(const StepParams& P, cudaStream_t st);
 int attend_setup(int kv_dtype, int G, int max_slices);

@@ -133,6 +133,7 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
       (size_t)slices * sizeof(spa::SliceState),                // state
       256,                                                     // device status word
       (size_t)slices * spa::kBins2 * 8,                        // hist2
+      256,                                                     // selection grid barrier
   };
   size_t off[sizeof sz / sizeof sz[0]];
   size_t o = 0;
@@ -156,14 +157,15 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
   w.st = (spa::SliceState*)(base + off[9]);
   w.dev_err = (unsigned*)(base + off[10]);
   w.hist2 = (unsigned long long*)(base + off[11]);
+  w.bar = (unsigned*)(base + off[12]);
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = spa::launch_prologue(P, kv_dtype, st);
-  if (e == cudaSuccess && P.n_ret > 0) {
-    if ((e = spa::launch_score(P, st)) == cudaSuccess && (e = spa::launch_mass(P, st)) == cudaSuccess &&
-        (e = spa::launch_threshold(P, st)) == cudaSuccess)
-      e = spa::launch_compact(P, st);
-  }
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int per_sm = spa::select_resident_per_sm(kv_dtype, G);
+  if (per_sm < 1 || sms < 1) return err(SPA_ERR_UNSUPPORTED, "spa_select_noalloc: selection kernel cannot be resident");
+  cudaError_t e = spa::launch_select(P, kv_dtype, spa::select_grid(P, per_sm * sms), st);
   if (e != cudaSuccess) return err(SPA_ERR_CUDA, cudaGetErrorString(e));
   return SPA_OK;
 }

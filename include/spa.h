@@ -177,16 +177,13 @@ SPA_API spa_status spa_device_status(spa_handle h, spa_stream stream);
 
 /* ---- instrumentation (used by the benchmark; off by default) ---- */
 
-/* Kernel ids for spa_profile_read / spa_kernel_name. */
+/* Kernel ids for spa_profile_read / spa_kernel_name.  Selection (query prologue,
+ * index scores, mass histogram, threshold, compaction) is one cooperative kernel. */
 #define SPA_K_INDEX_APPEND 0
-#define SPA_K_PROLOGUE 1
-#define SPA_K_SCORE 2
-#define SPA_K_MASS 3
-#define SPA_K_THRESHOLD 4
-#define SPA_K_COMPACT 5
-#define SPA_K_ATTEND 6
-#define SPA_K_COMBINE 7
-#define SPA_K_COUNT 8
+#define SPA_K_SELECT 1
+#define SPA_K_ATTEND 2
+#define SPA_K_COMBINE 3
+#define SPA_K_COUNT 4
 
 /* kernel_mask = 0 disables timing.  Otherwise every launch of a kernel whose bit
  * (1 << SPA_K_...) is set is bracketed by two CUDA events recorded on the launch
