@@ -18,7 +18,8 @@
 //   mass      merge (m, z) over chunks -> M_h, Z_h; recompute l_hj (index read #2),
 //             pi_j = sum_h 2^(l_hj - M_h) / (G Z_h), stored as fp32; a mass histogram
 //             over the top 12 bits of pi_j's bit pattern, masses quantised to integer
-//             multiples of 2^-60 so every sum is exact and order independent;
+//             multiples of 2^-63 so every sum is exact and order independent (per chunk
+//             as a count and a sum of low significand bits per bin, 32-bit atomics);
 //   cut 1     per slice: total mass, target ceil(p * total) and the bin b1 where the
 //             descending cumulative mass reaches it;
 //   threshold per chunk: tokens above b1 counted, tokens of bin b1 appended as
@@ -155,16 +156,11 @@ template <int G>
 __device__ __forceinline__ int lane_head(int t4, int nh) { return G <= 4 ? t4 : t4 + 4 * nh; }
 
 
-// Stages the group's query index vectors in shared memory (qsm, G * 16 floats), then
-// builds the lane's B fragments from there.  Called by every thread of the CTA.
+// The lane's B fragments of the group's query index vectors (qsm, G * 16 floats in
+// shared memory).
 template <int G>
-__device__ __forceinline__ void load_qidx_frag(const StepParams& P, int b, int g, float* qsm,
-                                               uint32_t (&qb)[IdxTiles<G>::NT][2]) {
+__device__ __forceinline__ void qidx_frag(const float* qbase, uint32_t (&qb)[IdxTiles<G>::NT][2]) {
   const int lane = threadIdx.x & 31, gid = lane >> 2, t4 = lane & 3;
-  if (threadIdx.x < G * kIdxDim)   // written by another CTA in an earlier phase: read through L2
-    qsm[threadIdx.x] = __ldcg(&P.ws.q_idx[((size_t)b * P.Hq + (size_t)g * G) * kIdxDim + threadIdx.x]);
-  __syncthreads();
-  const float* qbase = qsm;
 #pragma unroll
   for (int t = 0; t < IdxTiles<G>::NT; ++t) {
     int head, part;   // part 0 = hi, 1 = mid, 2 = lo, -1 = zero column
@@ -190,6 +186,17 @@ __device__ __forceinline__ void load_qidx_frag(const StepParams& P, int b, int g
     qb[t][0] = pack_bf16x2(v[0], v[1]);
     qb[t][1] = pack_bf16x2(v[2], v[3]);
   }
+}
+
+// Stages the group's query index vectors (written by an earlier phase, read through L2)
+// in shared memory and builds the fragments.  Called by every thread of the CTA.
+template <int G>
+__device__ __forceinline__ void load_qidx_frag(const StepParams& P, int b, int g, float* qsm,
+                                               uint32_t (&qb)[IdxTiles<G>::NT][2]) {
+  if (threadIdx.x < G * kIdxDim)
+    qsm[threadIdx.x] = __ldcg(&P.ws.q_idx[((size_t)b * P.Hq + (size_t)g * G) * kIdxDim + threadIdx.x]);
+  __syncthreads();
+  qidx_frag<G>(qsm, qb);
 }
 
 // Log2-domain logits of tokens gid (ra) and gid + 8 (rb) for the lane's heads.
@@ -308,12 +315,14 @@ __device__ bool last_of_slice(unsigned* ticket, unsigned n_units, int* s_flag) {
 }
 
 // ------------------------------------------------------------------ shared memory
+constexpr int kWarps = kSelThreads / 32;
+constexpr int kGroupBatch = 4;                // groups per warp loaded together (double-buffered)
 constexpr int kSmallCap = 1024;   // candidates of the round-2 cut bin held in shared memory
 constexpr int kCandBatch = 8;     // candidates loaded per thread before any is used
 
 struct SmemPro { double cs[kHeadDim / 2], sn[kHeadDim / 2]; };
 struct SmemScore { float2 red[kSelThreads / 32][kMaxGroup]; };
-struct SmemMass { unsigned long long hist[kBins1]; float Mh[kMaxGroup], Wh[kMaxGroup]; };
+struct SmemMass { unsigned cnt[kBins1], low[kBins1]; float Mh[kMaxGroup], Wh[kMaxGroup]; };
 struct SmemRefine {
   int chunk_sel[kMaxChunks];      // kept candidates per chunk (listed ones)
   unsigned cnt4k[4096];           // position-select histogram
@@ -333,8 +342,8 @@ struct SelScalars {
   unsigned long long shl[32];
   unsigned shu[32];
   int shi[32];
-  int L, b1, b2, b3, kbin, fbin, cut_bin, pos_cut, off, ok;
-  unsigned small_n, kbefore, fbefore, tau;
+  int L, b1, b2, b3, kbin, fbin, cut_bin, pos_cut, off, ok, duty;
+  unsigned small_n, kbefore, fbefore, tau, gen;
   unsigned long long above2, cut_above;
 };
 
@@ -357,14 +366,16 @@ __device__ __forceinline__ int cta_len(const StepParams& P, int b, SelScalars& s
   return sc.L;
 }
 
-// ------------------------------------------------------------------ prologue phase
-// Unit: one (b, kv head) slice of every head (streaming ones included).
+// ------------------------------------------------------------------ query rotation
+// RoPE of slice s's G query heads at position L-1 (streaming slices included), read by
+// the attention kernels after this launch; a streaming slice's selection count is 0.
+// Taken as a "duty" by CTAs that wait at the last barrier anyway.
 template <typename T>
-__device__ void prologue_unit(const StepParams& P, SmemPro& sm, SelScalars& sc, int s) {
+__device__ void qrot_slice(const StepParams& P, SmemPro& sm, SelScalars& sc, int s) {
   const int b = s / P.Hkv, g = s % P.Hkv, G = P.G;
   const int L = cta_len(P, b, sc);
   const T* q = (const T*)P.q_pre + ((size_t)b * P.Hq + (size_t)g * G) * kHeadDim;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   if (tid < kHeadDim / 2) {
     // rotate-half RoPE at position L-1.  The angle is carried in units of pi,
     // t = (L-1) * inv_freq / pi in float64, reduced exactly modulo 2 (|t| < 2^52), and
@@ -382,94 +393,220 @@ __device__ void prologue_unit(const StepParams& P, SmemPro& sm, SelScalars& sc, 
     o[i] = (float)(x1 * sm.cs[i] - x2 * sm.sn[i]);
     o[i + kHeadDim / 2] = (float)(x2 * sm.cs[i] + x1 * sm.sn[i]);
   }
-  if (P.is_ret[g]) {
-    // warp w owns index outputs o = w + 8k; projector rows are loaded four outputs at a
-    // time before their float64 dot products are reduced across the warp
-    constexpr int kMaxOut = kMaxGroup * kIdxDim / 8;
-    constexpr int kBatch = 4;
-    const int nw = blockDim.x / 32;
-#pragma unroll
-    for (int k0 = 0; k0 < kMaxOut; k0 += kBatch) {
-      float pv[kBatch][kHeadDim / 32];
-#pragma unroll
-      for (int k = 0; k < kBatch; ++k) {
-        const int o = warp + nw * (k0 + k);
-        if (o < G * kIdxDim) {
-          const float* pq = P.ws.P_q + ((size_t)g * G * kIdxDim + o) * kHeadDim;
-#pragma unroll
-          for (int e = 0; e < kHeadDim / 32; ++e) pv[k][e] = pq[lane + 32 * e];
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < kBatch; ++k) {
-        const int o = warp + nw * (k0 + k);
-        if (o < G * kIdxDim) {
-          const int h = o / kIdxDim, r = o % kIdxDim;
-          double acc = 0.0;
-#pragma unroll
-          for (int e = 0; e < kHeadDim / 32; ++e)
-            acc += (double)pv[k][e] * (double)Elem<T>::get(q, h * kHeadDim + lane + 32 * e);
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(kFull, acc, off);
-          if (lane == 0) P.ws.q_idx[((size_t)b * P.Hq + (size_t)g * G + h) * kIdxDim + r] = (float)acc;
-        }
-      }
-    }
-    unsigned long long* h1 = P.ws.hist1 + (size_t)s * kBins1;
-    unsigned long long* h2 = P.ws.hist2 + (size_t)s * kBins2;
-    for (int i = tid; i < kBins1; i += blockDim.x) h1[i] = 0ull;
-    for (int i = tid; i < kBins2; i += blockDim.x) h2[i] = 0ull;
-    if (tid == 0) {
-      SliceState z;
-      z.q_total = z.target = z.m_above = 0ull;
-      z.b1 = -1;
-      z.tau_bits = 0u;
-      z.pos_cut = INT_MAX;
-      z.count = 0;
-      z.cand_count = 0u;
-      z.ticket_mass = z.ticket_thr = 0u;
-      z.pad_ = 0;
-      P.ws.st[s] = z;
-    }
-  } else if (tid == 0) {
+  if (!P.is_ret[g] && tid == 0) {
     P.ws.st[s].count = 0;
     if (P.sel_count) P.sel_count[s] = 0;
   }
-  __syncthreads();   // sm.cs / sm.sn reused by the next unit
+  __syncthreads();   // sm.cs / sm.sn reused by the next duty
+}
+
+// Takes q_rot duties (slices) from a grid-wide ticket until none is left.
+template <typename T>
+__device__ void qrot_duties(const StepParams& P, SmemPro& sm, SelScalars& sc) {
+  for (;;) {
+    __syncthreads();
+    if (threadIdx.x == 0) sc.duty = (int)atomicAdd(P.ws.bar + kBarDuty, 1u);
+    __syncthreads();
+    const int s = sc.duty;
+    if (s >= P.n_slices) return;
+    qrot_slice<T>(P, sm, sc, s);
+  }
+}
+
+// ------------------------------------------------------------------ query index vectors
+// q_idx[h] = P_q[g G + h] q_pre[h] for the G heads of slice (b, g): float64 dot products,
+// thread w of G * 64 sums a quarter (32 dims) of output w / 4 in order, the quarters are
+// added pairwise.  Result in sc.qsm (G * 16 floats) with the sequence length of b in
+// sc.L (validated as load_len does), both visible after the call.
+template <typename T, int G>
+__device__ void compute_qidx(const StepParams& P, int b, int g, SelScalars& sc) {
+  const int tid = threadIdx.x;
+  float* qsm = sc.qsm;
+  int64_t len_raw = 0;
+  if (tid == 0) len_raw = P.seq_lens[b];   // validated after the dot products are issued
+  const T* q = (const T*)P.q_pre + ((size_t)b * P.Hq + (size_t)g * G) * kHeadDim;
+  for (int w = tid; w < G * kIdxDim * 4; w += kSelThreads) {   // whole warps (G * 64 = 64k)
+    const int o = w >> 2, qd = w & 3, h = o / kIdxDim;
+    const float4* prow = reinterpret_cast<const float4*>(P.ws.P_q + ((size_t)g * G * kIdxDim + o) * kHeadDim) + 8 * qd;
+    const T* qrow = q + h * kHeadDim + 32 * qd;
+    double acc = 0.0;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float4 pv[4];
+      float qv[16];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) pv[k] = __ldg(prow + 4 * half + k);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) qv[k] = Elem<T>::get(qrow, 16 * half + k);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        acc += (double)pv[k].x * (double)qv[4 * k];
+        acc += (double)pv[k].y * (double)qv[4 * k + 1];
+        acc += (double)pv[k].z * (double)qv[4 * k + 2];
+        acc += (double)pv[k].w * (double)qv[4 * k + 3];
+      }
+    }
+    acc += __shfl_xor_sync(kFull, acc, 1);
+    acc += __shfl_xor_sync(kFull, acc, 2);
+    if (qd == 0) qsm[o] = (float)acc;
+  }
+  if (tid == 0) {
+    if (len_raw < 1 || len_raw > P.Lcap) {
+      atomicOr(P.ws.dev_err, kErrSeqLen);
+      len_raw = len_raw < 1 ? 1 : P.Lcap;
+    }
+    sc.L = (int)len_raw;
+  }
+  __syncthreads();
+}
+
+// ------------------------------------------------------------------ work partition
+// The score and mass phases split the retrieval slices' capacity (max_seq_len tokens
+// each, as ngc 16-token groups; slice y = b * n_ret + r owns global groups
+// [y ngc, (y+1) ngc)) into equal contiguous group ranges, one per CTA, so every SM of a
+// full-occupancy grid gets the same share.  A range may span slices; groups past a
+// sequence's length are empty.  CTA c covers [c T / nb, (c+1) T / nb), T = n_rs ngc.
+struct Ranges {
+  long long ngc, total;
+  int nb;
+  __device__ __forceinline__ Ranges(const StepParams& P) {
+    ngc = ((long long)P.Lcap + 15) / 16;
+    total = (long long)P.B * P.n_ret * ngc;
+    nb = (int)gridDim.x;
+  }
+  __device__ __forceinline__ long long begin(int c) const { return (long long)c * total / nb; }
+  // CTA whose range holds global group g
+  __device__ __forceinline__ int owner(long long g) const { return (int)(((g + 1) * nb - 1) / total); }
+  __device__ __forceinline__ int first_cta(int y) const { return owner((long long)y * ngc); }
+  __device__ __forceinline__ int last_cta(int y) const { return owner((long long)(y + 1) * ngc - 1); }
+};
+// Per-range statistics of slice y live at stats[(cta + y) * G]: the CTAs of slice y
+// are consecutive and the last one of y may be the first one of y + 1, so the slots
+// of different slices never overlap (at most nb + n_rs of them).
+__device__ __forceinline__ size_t stats_slot(int cta, int y) { return (size_t)cta + (size_t)y; }
+
+// Visits the CTA's range as segments f(y, l0, l1) of local groups [l0, l1) of slice y.
+template <class F>
+__device__ __forceinline__ void for_each_segment(const Ranges& R, F&& f) {
+  const long long ge = R.begin(blockIdx.x + 1);
+  for (long long g = R.begin(blockIdx.x); g < ge;) {
+    const int y = (int)(g / R.ngc);
+    const long long gend = min(ge, (long long)(y + 1) * R.ngc);
+    f(y, (int)(g - (long long)y * R.ngc), (int)(gend - (long long)y * R.ngc));
+    g = gend;
+  }
 }
 
 // ------------------------------------------------------------------ score phase
-// Warp w of the CTA takes the 16-token groups w, w + 8, ... of the chunk (8 in flight).
-template <int G>
-__device__ void score_unit(const StepParams& P, SmemScore& sm, SelScalars& sc, int y, int c) {
-  constexpr int NH = IdxTiles<G>::NH, U = 8;
-  constexpr int kGroups = kChunk / 16, kWarps = kSelThreads / 32;
+// The leader of slice y (the CTA holding its first group) resets the slice state,
+// computes the group's query index vectors, stores them and publishes them with a flag
+// tagged with this call's barrier generation; every range of the slice reads them after
+// the flag (bounded wait).  A CTA leads its slices before it scores any range, and only
+// waits for lower-numbered CTAs, so the waits always end.
+template <typename T, int G>
+__device__ void lead_slice(const StepParams& P, SelScalars& sc, int y) {
   const Unit un = unit_of(P, y);
-  const int L = cta_len(P, un.b, sc);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, t4 = lane & 3, gid = lane >> 2;
-  const int j0 = c * kChunk;
-  float2* out = P.ws.stats + ((size_t)un.s * P.n_chunks + c) * G;
-  if (j0 >= L) {
-    if (threadIdx.x < G) out[threadIdx.x] = make_float2(-INFINITY, 0.f);
+  SliceState* st = P.ws.st + un.s;
+  __syncthreads();   // earlier readers of sc.qsm / sc.L are done
+  if (threadIdx.x == 0) {
+    SliceState z;
+    z.q_total = z.target = z.m_above = 0ull;
+    z.b1 = -1;
+    z.tau_bits = 0u;
+    z.pos_cut = INT_MAX;
+    z.count = 0;
+    z.cand_count = 0u;
+    z.ticket_mass = z.ticket_thr = 0u;
+    z.qidx_ready = 0u;
+    *st = z;
+  }
+  compute_qidx<T, G>(P, un.b, un.g, sc);
+  if (threadIdx.x < G * kIdxDim) {
+    P.ws.q_idx[((size_t)un.b * P.Hq + (size_t)un.g * G) * kIdxDim + threadIdx.x] = sc.qsm[threadIdx.x];
+    __threadfence();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) atomicExch(&st->qidx_ready, sc.gen + 1u);
+}
+
+// Waits (thread 0, bounded) for slice s's q_idx flag of this call; the caller
+// synchronises the CTA afterwards.
+__device__ __forceinline__ void wait_qidx(const StepParams& P, int s, unsigned gen) {
+  volatile unsigned* flag = &P.ws.st[s].qidx_ready;
+  const unsigned want = gen + 1u;
+  const long long t0 = clock64();
+  unsigned ns = 32;
+  while (*flag != want) {
+    if (clock64() - t0 > kBarrierCycles) {
+      atomicOr(P.ws.dev_err, kErrTimeout);
+      break;
+    }
+    __nanosleep(ns);
+    if (ns < 128) ns <<= 1;
+  }
+  __threadfence();
+}
+
+// Clears the CTA's share of slice y's round-1 / round-2 histograms (read after a barrier).
+__device__ __forceinline__ void clear_hist_share(const StepParams& P, const Ranges& R, int y, int s) {
+  static_assert(kBins1 == kBins2, "histogram reset assumes equal round-1 / round-2 bin counts");
+  const int first = R.first_cta(y), n = R.last_cta(y) - first + 1, k = (int)blockIdx.x - first;
+  unsigned long long* h1 = P.ws.hist1 + (size_t)s * kBins1;
+  unsigned long long* h2 = P.ws.hist2 + (size_t)s * kBins2;
+  for (int i = k * kSelThreads + (int)threadIdx.x; i < kBins1; i += n * kSelThreads) {
+    h1[i] = 0ull;
+    h2[i] = 0ull;
+  }
+}
+
+// One range of slice y: per head m = max_j l_hj, z = sum_j 2^(l_hj - m) over the tokens
+// of local groups [l0, l1), l_hj = log2(e) * idx_scale * <q_idx[h], idx_j>.  Warp w takes
+// groups l0 + w, l0 + w + 8, ..., kGroupBatch at a time; the first batch is requested
+// before the query vectors arrive (bounded by the call's max length; rows past the
+// sequence are masked).
+template <int G>
+__device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc, const Ranges& R, int y,
+                              int l0, int l1) {
+  constexpr int NH = IdxTiles<G>::NH, U = kGroupBatch;
+  const Unit un = unit_of(P, y);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, t4 = lane & 3, gid = lane >> 2;
+  clear_hist_share(P, R, y, un.s);
+  const uint2* rows = reinterpret_cast<const uint2*>(P.idx_cache + (size_t)un.s * P.Lmax * kIdxDim);
+  const uint64_t pol = l2_policy_keep();
+  uint2 ra[U], rb[U];
+  {
+    const int jpf = min(P.Lcap, 16 * l1);
+#pragma unroll
+    for (int u = 0; u < U; ++u) load_group(rows, 16 * (l0 + warp + kWarps * u), jpf, pol, ra[u], rb[u]);
+  }
+  __syncthreads();   // earlier readers of sc.L and sc.qsm are done
+  if (tid == 0) {
+    sc.L = load_len(P.seq_lens, un.b, P.Lcap, P.ws.dev_err);
+    if (16 * l0 < sc.L) wait_qidx(P, un.s, sc.gen);
+  }
+  __syncthreads();
+  const int L = sc.L;
+  float2* out = P.ws.stats + stats_slot(blockIdx.x, y) * G;
+  if (16 * l0 >= L) {
+    if (tid < G) out[tid] = make_float2(-INFINITY, 0.f);
     return;
   }
   uint32_t qb[IdxTiles<G>::NT][2];
   load_qidx_frag<G>(P, un.b, un.g, sc.qsm, qb);
   const float scale = P.idx_scale_log2;
-  const int jend = min(L, j0 + kChunk);
-  const uint2* rows = reinterpret_cast<const uint2*>(P.idx_cache + (size_t)un.s * P.Lmax * kIdxDim);
+  const int jend = min(L, 16 * l1);
   // two independent online accumulators per head (tokens gid and gid + 8)
   float m[NH][2], z[NH][2];
 #pragma unroll
   for (int h = 0; h < NH; ++h) { m[h][0] = m[h][1] = -INFINITY; z[h][0] = z[h][1] = 0.f; }
-  const uint64_t pol = l2_policy_keep();
-  for (int k = 0; k < kGroups / kWarps; k += U) {
-    uint2 ra[U], rb[U];
+  for (int gb = l0; 16 * gb < jend; gb += kWarps * U) {
+    if (gb > l0) {
 #pragma unroll
-    for (int u = 0; u < U; ++u) load_group(rows, j0 + 16 * (warp + kWarps * (k + u)), jend, pol, ra[u], rb[u]);
+      for (int u = 0; u < U; ++u) load_group(rows, 16 * (gb + warp + kWarps * u), jend, pol, ra[u], rb[u]);
+    }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int j = j0 + 16 * (warp + kWarps * (k + u));
+      const int j = 16 * (gb + warp + kWarps * u);
       float lg[NH][2];
       group_logits<G>(ra[u], rb[u], qb, scale, lg);
 #pragma unroll
@@ -493,100 +630,20 @@ __device__ void score_unit(const StepParams& P, SmemScore& sm, SelScalars& sc, i
     if (lane < 4 && head < G) sm.red[warp][head] = make_float2(m[h][0], z[h][0]);
   }
   __syncthreads();
-  if (threadIdx.x < G) {
-    const int h = threadIdx.x;
+  if (tid < G) {
     float mm = -INFINITY, zz = 0.f;
-    for (int w = 0; w < kWarps; ++w) merge_mz(mm, zz, sm.red[w][h].x, sm.red[w][h].y);
-    out[h] = make_float2(mm, zz);
+    for (int w = 0; w < kWarps; ++w) merge_mz(mm, zz, sm.red[w][tid].x, sm.red[w][tid].y);
+    out[tid] = make_float2(mm, zz);
   }
-  __syncthreads();   // sm.red reused by the next unit
+  __syncthreads();   // sm.red reused by the next range
 }
 
-// ------------------------------------------------------------------ mass phase
-template <int G>
-__device__ void mass_unit(const StepParams& P, SmemMass& sm, SelScalars& sc, int y, int c) {
-  const Unit un = unit_of(P, y);
-  const int L = cta_len(P, un.b, sc);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int j0 = c * kChunk;
-  if (j0 >= L) return;
-  for (int i = tid; i < kBins1; i += kSelThreads) sm.hist[i] = 0ull;
-  // global (M_h, Z_h): warp h merges the chunk partials, in a fixed order
-  if (warp < G) {
-    const int nc = (L + kChunk - 1) / kChunk;
-    float m = -INFINITY, z = 0.f;
-    for (int cc = lane; cc < nc; cc += 32) {
-      const float2 v = __ldcg(&P.ws.stats[((size_t)un.s * P.n_chunks + cc) * G + warp]);
-      merge_mz(m, z, v.x, v.y);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float m2 = __shfl_xor_sync(kFull, m, o);
-      const float z2 = __shfl_xor_sync(kFull, z, o);
-      merge_mz(m, z, m2, z2);
-    }
-    if (lane == 0) {
-      sm.Mh[warp] = m;
-      sm.Wh[warp] = 1.f / ((float)G * z);
-    }
-  }
-  __syncthreads();
-  {
-    constexpr int NH = IdxTiles<G>::NH, U = 8;
-    constexpr int kGroups = kChunk / 16, kWarps = kSelThreads / 32;
-    uint32_t qb[IdxTiles<G>::NT][2];
-    load_qidx_frag<G>(P, un.b, un.g, sc.qsm, qb);
-    const float scale = P.idx_scale_log2;
-    const int gid = lane >> 2, t4 = lane & 3;
-    float M[NH], W[NH];
-#pragma unroll
-    for (int h = 0; h < NH; ++h) {
-      const int head = lane_head<G>(t4, h);
-      M[h] = head < G ? sm.Mh[head] : 0.f;
-      W[h] = head < G ? sm.Wh[head] : 0.f;   // lanes of absent heads contribute nothing
-    }
-    const int jend = min(L, j0 + kChunk);
-    const uint2* rows = reinterpret_cast<const uint2*>(P.idx_cache + (size_t)un.s * P.Lmax * kIdxDim);
-    float* pi = P.ws.pi + (size_t)un.s * P.ws.pi_stride;
-    const uint64_t pol = l2_policy_drop();
-    for (int k = 0; k < kGroups / kWarps; k += U) {
-      uint2 ra[U], rb[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) load_group(rows, j0 + 16 * (warp + kWarps * (k + u)), jend, pol, ra[u], rb[u]);
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int j = j0 + 16 * (warp + kWarps * (k + u));
-        float lg[NH][2];
-        group_logits<G>(ra[u], rb[u], qb, scale, lg);
-        // pi = sum over the group's heads of 2^(l - M_h) / (G Z_h): lane-local heads first,
-        // then the 4 lanes of a token (fixed order, identical result in every lane)
-        float pr[2];
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          float acc = 0.f;
-#pragma unroll
-          for (int h = 0; h < NH; ++h) acc += W[h] == 0.f ? 0.f : exp2f(lg[h][cc] - M[h]) * W[h];
-          acc += __shfl_xor_sync(kFull, acc, 1);
-          acc += __shfl_xor_sync(kFull, acc, 2);
-          pr[cc] = acc;
-        }
-        if (t4 < 2) {   // lane t4 = 0 stores token gid, t4 = 1 token gid + 8
-          const int jt = j + gid + 8 * t4;
-          const float v = t4 == 0 ? pr[0] : pr[1];
-          if (jt < jend) {
-            pi[jt] = v;
-            const unsigned bits = __float_as_uint(v);
-            atomicAdd(&sm.hist[min(bits >> 18, (unsigned)(kBins1 - 1))], mass_q(v));
-          }
-        }
-      }
-    }
-  }
-  __syncthreads();
-  unsigned long long* g1 = P.ws.hist1 + (size_t)un.s * kBins1;
-  for (int i = tid; i < kBins1; i += kSelThreads)
-    if (sm.hist[i]) atomicAdd(g1 + i, sm.hist[i]);
-  __syncthreads();   // sm.hist reused by the next unit
+template <typename T, int G>
+__device__ void score_phase(const StepParams& P, SmemScore& sm, SelScalars& sc) {
+  const Ranges R(P);
+  const long long ga = R.begin(blockIdx.x), ge = R.begin(blockIdx.x + 1);
+  for (long long y = (ga + R.ngc - 1) / R.ngc; y * R.ngc < ge; ++y) lead_slice<T, G>(P, sc, (int)y);
+  for_each_segment(R, [&](int y, int l0, int l1) { score_segment<G>(P, sm, sc, R, y, l0, l1); });
 }
 
 // ------------------------------------------------------------------ cut 1 (per slice)
@@ -620,6 +677,114 @@ __device__ void cut1_slice(const StepParams& P, SelScalars& sc, int y) {
     st->m_above = keep_all ? 0ull : sc.cut_above;
   }
   __syncthreads();
+}
+
+// ------------------------------------------------------------------ mass phase
+// One range of slice y: M_h, Z_h merged from the slice's range statistics (fixed
+// order), the logits recomputed (index read #2, mostly from L2),
+// pi_j = sum_h 2^(l_hj - M_h) / (G Z_h) stored, and its mass added to the slice's
+// round-1 histogram via a per-range shared histogram of counts and low significand
+// bits (32-bit atomics; a range holds at most kMaxRangeGroups groups, so a bin's
+// low-bit sum stays below 2^32).
+constexpr int kMaxRangeGroups = 1024;   // 16384 tokens: 16384 * 2^18 = 2^32
+template <int G>
+__device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, const Ranges& R, int y, int l0,
+                             int l1) {
+  constexpr int NH = IdxTiles<G>::NH, U = kGroupBatch;
+  const Unit un = unit_of(P, y);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, gid = lane >> 2, t4 = lane & 3;
+  const uint2* rows = reinterpret_cast<const uint2*>(P.idx_cache + (size_t)un.s * P.Lmax * kIdxDim);
+  const uint64_t pol = l2_policy_drop();
+  uint2 ra[U], rb[U];
+  {
+    const int jpf = min(P.Lcap, 16 * l1);
+#pragma unroll
+    for (int u = 0; u < U; ++u) load_group(rows, 16 * (l0 + warp + kWarps * u), jpf, pol, ra[u], rb[u]);
+  }
+  const int L = cta_len(P, un.b, sc);
+  if (16 * l0 >= L) return;
+  for (int i = tid; i < kBins1; i += kSelThreads) sm.cnt[i] = sm.low[i] = 0u;
+  // global (M_h, Z_h): warp h merges the ranges' partials, in a fixed order
+  if (warp < G) {
+    const int c0 = R.first_cta(y), c1 = R.last_cta(y);
+    float m = -INFINITY, z = 0.f;
+    for (int c = c0 + lane; c <= c1; c += 32) {
+      const float2 v = __ldcg(&P.ws.stats[stats_slot(c, y) * G + warp]);
+      merge_mz(m, z, v.x, v.y);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(kFull, m, o);
+      const float z2 = __shfl_xor_sync(kFull, z, o);
+      merge_mz(m, z, m2, z2);
+    }
+    if (lane == 0) {
+      sm.Mh[warp] = m;
+      sm.Wh[warp] = 1.f / ((float)G * z);
+    }
+  }
+  uint32_t qb[IdxTiles<G>::NT][2];
+  load_qidx_frag<G>(P, un.b, un.g, sc.qsm, qb);   // its CTA barrier also publishes sm.Mh / sm.Wh
+  const float scale = P.idx_scale_log2;
+  float M[NH], W[NH];
+#pragma unroll
+  for (int h = 0; h < NH; ++h) {
+    const int head = lane_head<G>(t4, h);
+    M[h] = head < G ? sm.Mh[head] : 0.f;
+    W[h] = head < G ? sm.Wh[head] : 0.f;   // lanes of absent heads contribute nothing
+  }
+  const int jend = min(L, 16 * l1);
+  float* pi = P.ws.pi + (size_t)un.s * P.ws.pi_stride;
+  for (int gb = l0; 16 * gb < jend; gb += kWarps * U) {
+    if (gb > l0) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) load_group(rows, 16 * (gb + warp + kWarps * u), jend, pol, ra[u], rb[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = 16 * (gb + warp + kWarps * u);
+      float lg[NH][2];
+      group_logits<G>(ra[u], rb[u], qb, scale, lg);
+      // pi = sum over the group's heads of 2^(l - M_h) / (G Z_h): lane-local heads first,
+      // then the 4 lanes of a token (fixed order, identical result in every lane)
+      float pr[2];
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        float acc = 0.f;
+#pragma unroll
+        for (int h = 0; h < NH; ++h) acc += W[h] == 0.f ? 0.f : exp2f(lg[h][cc] - M[h]) * W[h];
+        acc += __shfl_xor_sync(kFull, acc, 1);
+        acc += __shfl_xor_sync(kFull, acc, 2);
+        pr[cc] = acc;
+      }
+      if (t4 < 2) {   // lane t4 = 0 stores token gid, t4 = 1 token gid + 8
+        const int jt = j + gid + 8 * t4;
+        const float v = t4 == 0 ? pr[0] : pr[1];
+        if (jt < jend) {
+          pi[jt] = v;
+          const unsigned bits = __float_as_uint(v);
+          const unsigned d = min(bits >> 18, (unsigned)(kBins1 - 1));
+          atomicAdd(&sm.cnt[d], 1u);
+          atomicAdd(&sm.low[d], bits & 0x3ffffu);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  unsigned long long* g1 = P.ws.hist1 + (size_t)un.s * kBins1;
+  for (int i = tid; i < kBins1; i += kSelThreads)
+    if (sm.cnt[i]) atomicAdd(g1 + i, bin1_mass((unsigned)i, sm.cnt[i], sm.low[i]));
+  __syncthreads();   // the histogram is reused by the next range
+}
+
+template <int G>
+__device__ void mass_phase(const StepParams& P, SmemMass& sm, SelScalars& sc) {
+  const Ranges R(P);
+  for_each_segment(R, [&](int y, int l0, int l1) {
+    for (int a = l0; a < l1; a += kMaxRangeGroups) mass_segment<G>(P, sm, sc, R, y, a, min(l1, a + kMaxRangeGroups));
+    const int n = R.last_cta(y) - R.first_cta(y) + 1;
+    if (last_of_slice(&P.ws.st[unit_of(P, y).s].ticket_mass, (unsigned)n, &sc.ok)) cut1_slice(P, sc, y);
+  });
 }
 
 // ------------------------------------------------------------------ threshold phase
@@ -698,7 +863,7 @@ __device__ void threshold_unit(const StepParams& P, SelScalars& sc, int y, int c
       for (int i = 0; i < kTokPerThread; ++i) {
         if ((cflags >> i) & 1u) {
           cand[base + __popc(masks[i] & lt)] = make_uint2(bits[i], (unsigned)(j0 + tid + kSelThreads * i));
-          atomicAdd(&h2[(bits[i] >> 6) & 0xfffu], mass_q(__uint_as_float(bits[i])));
+          atomicAdd(&h2[(bits[i] >> 6) & 0xfffu], mass_q(bits[i]));
         }
         base += __popc(masks[i]);
       }
@@ -748,7 +913,7 @@ __device__ void refine_slice(const StepParams& P, SmemRefine& sm, SelScalars& sc
       if (d2 > cb2) {
         if (!sw.always(pos)) atomicAdd(&chunk_sel[pos / kChunk], 1);
       } else if (d2 == cb2) {
-        atomicAdd(&sm.m3[bits & 63u], mass_q(__uint_as_float(bits)));
+        atomicAdd(&sm.m3[bits & 63u], mass_q(bits));
         atomicAdd(&sm.c3[bits & 63u], 1u);
         const unsigned slot = atomicAdd(&sc.small_n, 1u);
         if (slot < kSmallCap) small[slot] = make_uint2(bits, (unsigned)pos);
@@ -773,7 +938,7 @@ __device__ void refine_slice(const StepParams& P, SmemRefine& sm, SelScalars& sc
       tau = ((unsigned)b1 << 18) | ((unsigned)cb2 << 6) | (unsigned)sc.b3;
       const unsigned long long m_gt = sc.above2;
       const unsigned n_eq = sm.c3[sc.b3];
-      const unsigned long long q_tau = mass_q(__uint_as_float(tau));
+      const unsigned long long q_tau = mass_q(tau);
       const unsigned long long need =
           (q_tau > 0ull && target > m_gt) ? (target - m_gt + q_tau - 1ull) / q_tau : ~0ull;
       if (need < (unsigned long long)n_eq) {
@@ -917,24 +1082,26 @@ __global__ void __launch_bounds__(kSelThreads, 4) k_select(StepParams P) {
   __shared__ SelSmem sm;
   __shared__ SelScalars sc;
   const int nb = gridDim.x;
-  for (int s = blockIdx.x; s < P.n_slices; s += nb) prologue_unit<T>(P, sm.pro, sc, s);
-  if (!grid_barrier(P.ws.bar, P.ws.dev_err, &sc.ok)) return;
-  if (P.n_ret == 0) return;
+  if (P.n_ret == 0) {   // nothing to select: only the query rotation
+    for (int s = blockIdx.x; s < P.n_slices; s += nb) qrot_slice<T>(P, sm.pro, sc, s);
+    return;
+  }
   const int n_rs = P.B * P.n_ret;
   const int n_units = n_rs * P.n_chunks;
-  for (int u = blockIdx.x; u < n_units; u += nb) score_unit<G>(P, sm.score, sc, u / P.n_chunks, u % P.n_chunks);
+  // the barrier generation is constant until every CTA has finished the score phase:
+  // it tags this call's q_idx flags
+  if (threadIdx.x == 0) sc.gen = *reinterpret_cast<volatile unsigned*>(P.ws.bar + 32);
+  if (blockIdx.x == 0 && threadIdx.x == 0) P.ws.bar[kBarDuty] = 0u;   // taken after two barriers
+  score_phase<T, G>(P, sm.score, sc);
   if (!grid_barrier(P.ws.bar, P.ws.dev_err, &sc.ok)) return;
-  for (int u = blockIdx.x; u < n_units; u += nb) {
-    const int y = u / P.n_chunks;
-    mass_unit<G>(P, sm.mass, sc, y, u % P.n_chunks);
-    if (last_of_slice(&P.ws.st[unit_of(P, y).s].ticket_mass, P.n_chunks, &sc.ok)) cut1_slice(P, sc, y);
-  }
+  mass_phase<G>(P, sm.mass, sc);
   if (!grid_barrier(P.ws.bar, P.ws.dev_err, &sc.ok)) return;
   for (int u = blockIdx.x; u < n_units; u += nb) {
     const int y = u / P.n_chunks;
     threshold_unit(P, sc, y, u % P.n_chunks);
     if (last_of_slice(&P.ws.st[unit_of(P, y).s].ticket_thr, P.n_chunks, &sc.ok)) refine_slice(P, sm.ref, sc, y);
   }
+  qrot_duties<T>(P, sm.pro, sc);   // off the critical path: refine steps run meanwhile
   if (!grid_barrier(P.ws.bar, P.ws.dev_err, &sc.ok)) return;
   for (int u = blockIdx.x; u < n_units; u += nb) compact_unit(P, sc, u / P.n_chunks, u % P.n_chunks);
 }
@@ -955,12 +1122,18 @@ int resident_tg() {
 
 }  // namespace
 
-// Grid of the selection launch: one CTA per unit of work, capped at what is resident.
+// Grid of the selection launch.  When there is at least half a full wave of work it is
+// every resident CTA (the same count on every SM, so the range-partitioned phases are
+// balanced per SM); never more CTAs than 16-token groups, so no CTA has an empty range.
 int select_grid(const StepParams& P, int max_resident) {
-  const int units = P.n_ret > 0 ? P.B * P.n_ret * P.n_chunks : 0;
-  int want = units > P.n_slices ? units : P.n_slices;
+  if (P.n_ret <= 0) return P.n_slices < max_resident ? P.n_slices : max_resident;
+  const long long groups = (long long)P.B * P.n_ret * (((long long)P.Lcap + 15) / 16);
+  long long want = (long long)P.B * P.n_ret * P.n_chunks;
+  if (want < P.n_slices) want = P.n_slices;
+  if (2 * want >= max_resident) want = max_resident;
+  if (want > groups) want = groups;
   if (want < 1) want = 1;
-  return want < max_resident ? want : max_resident;
+  return (int)want;
 }
 
 cudaError_t launch_select(const StepParams& P, int kv_dtype, int grid, cudaStream_t st) {

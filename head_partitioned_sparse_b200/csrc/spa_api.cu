@@ -52,7 +52,7 @@ Layout plan(const spa_config& c, int split_rows) {
       64 * 8,                                              // 2 inv_freq
       (size_t)c.max_batch * c.n_q_heads * 128 * 4,         // 3 q_rot
       (size_t)c.max_batch * c.n_q_heads * 16 * 4,          // 4 q_idx
-      slices * L.n_chunks_max * G * 8,                     // 5 stats
+      (spa::kMaxSelectGrid + slices) * G * 8,              // 5 stats
       slices * (size_t)spa::pi_row_stride(Lmax) * 4,       // 6 pi
       slices * spa::kBins1 * 8,                            // 7 hist1
       slices * (size_t)Lmax * 8,                           // 8 cand
@@ -64,7 +64,7 @@ Layout plan(const spa_config& c, int split_rows) {
       (size_t)L.max_items * G * spa::kPartStride * 4,      // 14 part
       256,                                                 // 15 dev_err
       slices * spa::kBins2 * 8,                            // 16 hist2
-      256,                                                 // 17 selection grid barrier
+      spa::kBarWords * 4,                                  // 17 selection grid barrier
   };
   size_t o = 0;
   for (int i = 0; i < 18; ++i) {
@@ -288,7 +288,8 @@ spa_status spa_create(spa_handle* out, const spa_config* cfg) {
   if ((e = cudaMemcpy(w.P_q, cfg->P_q, pq, cudaMemcpyDeviceToDevice)) != cudaSuccess ||
       (e = cudaMemcpy(w.P_k, cfg->P_k, pk, cudaMemcpyDeviceToDevice)) != cudaSuccess ||
       (e = cudaMemcpy(w.inv_freq, invf, sizeof invf, cudaMemcpyHostToDevice)) != cudaSuccess ||
-      (e = cudaMemset(w.dev_err, 0, 4)) != cudaSuccess || (e = cudaMemset(w.bar, 0, 256)) != cudaSuccess ||
+      (e = cudaMemset(w.dev_err, 0, 4)) != cudaSuccess || (e = cudaMemset(w.bar, 0, spa::kBarWords * 4)) != cudaSuccess ||
+      (e = cudaMemset(w.st, 0, L.off[12] - L.off[11])) != cudaSuccess ||
       (e = cudaDeviceSynchronize()) != cudaSuccess) {
     cudaFree(h->mem);
     delete h;
@@ -308,6 +309,7 @@ spa_status spa_create(spa_handle* out, const spa_config* cfg) {
     return fail(SPA_ERR_UNSUPPORTED, "selection kernel cannot be resident with this configuration");
   }
   h->select_max_grid = sel_occ * h->num_sms;
+  if (h->select_max_grid > spa::kMaxSelectGrid) h->select_max_grid = spa::kMaxSelectGrid;
   *out = h;
   return SPA_OK;
 }
@@ -393,7 +395,9 @@ spa_status spa_device_status(spa_handle h, spa_stream stream) {
     if ((e = cudaMemset(h->ws.dev_err, 0, 4)) != cudaSuccess) return cuda_fail(e, "clear status");
     if (flags & spa::kErrTimeout) {
       // the grid barrier may have been left mid-way: start the next call from a clean barrier
-      cudaMemset(h->ws.bar, 0, 256);
+      cudaMemset(h->ws.bar, 0, spa::kBarWords * 4);
+      // q_idx flags are tagged with the barrier generation, which restarts at 0
+      cudaMemset(h->ws.st, 0, sizeof(spa::SliceState) * (size_t)h->cfg.max_batch * h->cfg.n_kv_heads);
       cudaDeviceSynchronize();
       return fail(SPA_ERR_DEVICE_TIMEOUT, "a bounded device-side wait gave up (flags 0x%x)", flags);
     }

@@ -26,15 +26,25 @@ constexpr int kMaxChunks = int(kMaxCtx / kChunk);    // 4096
 constexpr int kBins1 = 4096;
 constexpr int kBins2 = 4096;
 constexpr int kBins3 = 64;
-constexpr float kMassScale = 1152921504606846976.0f;  // 2^60: mass unit is 2^-60
+// Masses are integers in units of 2^-63 (see mass_q): exact below 2^64 for any sum of
+// probabilities that add up to at most 1 (plus fp32 rounding).
+constexpr int kMassMinExp = 87;
+
+// Largest grid of the selection kernel (sizes the per-range statistics).
+constexpr int kMaxSelectGrid = 8192;
 
 // Attention splits ("items") cover up to split_rows rows of one slice; rows are
 // staged through shared memory kTile rows at a time.
 constexpr int kTile = 64;
 constexpr int kAttnThreads = 256;
-constexpr int kDefaultSplitRows = 512;
+constexpr int kDefaultSplitRows = 1024;
 // One split's state per head: acc[128], m, l, 2 floats of padding (16-byte rows).
 constexpr int kPartStride = kHeadDim + 4;
+
+// Words of the selection kernel's synchronisation block, one 128-byte line each:
+// [0] barrier arrivals, [32] barrier generation, [kBarDuty] q_rot duty ticket.
+constexpr int kBarWords = 96;
+constexpr int kBarDuty = 64;
 
 // Device status bits.
 constexpr unsigned kErrSeqLen = 1u;
@@ -45,7 +55,7 @@ constexpr unsigned kErrTimeout = 8u;   // a bounded device-side wait gave up
 // Per (b, kv head) selection state.  Written by the selection kernel, read by its
 // later phases and by attention.
 struct __align__(16) SliceState {
-  unsigned long long q_total;   // sum of quantised masses (units of 2^-60)
+  unsigned long long q_total;   // sum of quantised masses (units of 2^-63)
   unsigned long long target;    // ceil(p * q_total)
   unsigned long long m_above;   // mass of all tokens in digit1 bins above b1
   int b1;                       // round-1 bin holding the cut; -1 = keep everything
@@ -55,7 +65,7 @@ struct __align__(16) SliceState {
   unsigned ticket_mass;         // last-CTA tickets of the mass and threshold phases
   unsigned ticket_thr;
   unsigned cand_count;          // candidates appended (tokens in bin b1)
-  int pad_;
+  unsigned qidx_ready;          // barrier generation + 1 once this call's q_idx is stored
 };
 
 __host__ __device__ inline int64_t pi_row_stride(int64_t Lmax) { return (Lmax + 63) / 64 * 64; }
@@ -67,7 +77,7 @@ struct Workspace {
   double* inv_freq;      // [64] RoPE inverse frequencies divided by pi
   float* q_rot;          // [Bm][Hq][128]
   float* q_idx;          // [Bm][Hq][16]
-  float2* stats;         // [Bm*Hkv][n_chunks_max][G]  (m in log2 units, z)
+  float2* stats;         // [kMaxSelectGrid + Bm*Hkv][G] per-range (m in log2 units, z)
   float* pi;             // [Bm*Hkv][pi_stride]
   int64_t pi_stride;     // Lmax rounded up to 64 floats (256-byte rows)
   unsigned long long* hist1;  // [Bm*Hkv][kBins1]
@@ -80,7 +90,7 @@ struct Workspace {
   int* item_base;        // [Bm*Hkv + 1]
   float* part;           // [max_items][G][kPartStride]
   unsigned* dev_err;     // [1]
-  unsigned* bar;         // [64] grid barrier of the selection kernel: [0] arrivals, [32] generation
+  unsigned* bar;         // [kBarWords] selection kernel: grid barrier and q_rot duty ticket
   int64_t max_items;
 };
 
@@ -145,8 +155,27 @@ template <> struct Elem<float> {
   static __device__ __forceinline__ float get(const float* p, int i) { return p[i]; }
 };
 
-__device__ __forceinline__ unsigned long long mass_q(float pr) {
-  return __float2ull_rn(pr * kMassScale);
+// Quantised mass of a probability from its fp32 bit pattern u: the exact value in units
+// of 2^-63, M * 2^(E - 87) for the 24-bit significand M and exponent field E >= 87
+// (values >= 2^-40); smaller values count as 0.  Integer sums of these masses are exact,
+// so every total is independent of the order of accumulation.  Probabilities are at most
+// 1 plus fp32 rounding (E <= 127), so one mass is below 2^64.
+__device__ __forceinline__ unsigned long long mass_q(unsigned u) {
+  int e = (int)((u >> 23) & 0xffu);
+  if (e < kMassMinExp) return 0ull;
+  e = e > 127 ? 127 : e;
+  return (unsigned long long)((u & 0x7fffffu) | 0x800000u) << (e - kMassMinExp);
+}
+
+// Total mass_q of n probabilities of round-1 bin d (u >> 18 == d: same exponent and top
+// five significand bits) whose low 18 bits sum to s_low.  Equal to the sum of their
+// mass_q, which lets the per-chunk histograms count with 32-bit shared-memory atomics.
+__device__ __forceinline__ unsigned long long bin1_mass(unsigned d, unsigned n, unsigned long long s_low) {
+  int e = (int)(d >> 5);
+  if (e < kMassMinExp || n == 0u) return 0ull;
+  e = e > 127 ? 127 : e;
+  const unsigned long long base = (unsigned long long)(32u | (d & 31u)) << 18;
+  return (base * n + s_low) << (e - kMassMinExp);
 }
 
 // Merge two online-softmax states (m in log2 units).

@@ -116,6 +116,13 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
   P.attn_scale_log2 = (float)(1.4426950408889634 / std::sqrt(128.0));
   P.split_rows = spa::kDefaultSplitRows;
 
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int per_sm = spa::select_resident_per_sm(kv_dtype, G);
+  if (per_sm < 1 || sms < 1) return err(SPA_ERR_UNSUPPORTED, "spa_select_noalloc: selection kernel cannot be resident");
+  const int grid = spa::select_grid(P, per_sm * sms < spa::kMaxSelectGrid ? per_sm * sms : spa::kMaxSelectGrid);
+
   void* base_v = nullptr;
   spa_status r = scratch_on_current_device(&base_v);
   if (r) return r;
@@ -124,7 +131,7 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
       64 * 8,                                                  // inv_freq (unused by selection; zero)
       (size_t)B * n_q_heads * spa::kHeadDim * 4,               // q_rot
       (size_t)B * n_q_heads * spa::kIdxDim * 4,                // q_idx
-      (size_t)slices * P.n_chunks * G * 8,                     // stats
+      (size_t)(grid + slices) * G * 8,                         // per-range statistics
       (size_t)slices * spa::pi_row_stride(max_ctx) * 4,        // pi
       (size_t)slices * spa::kBins1 * 8,                        // hist1
       (size_t)slices * max_ctx * 8,                            // candidates
@@ -133,7 +140,7 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
       (size_t)slices * sizeof(spa::SliceState),                // state
       256,                                                     // device status word
       (size_t)slices * spa::kBins2 * 8,                        // hist2
-      256,                                                     // selection grid barrier
+      spa::kBarWords * 4,                                      // selection grid barrier
   };
   size_t off[sizeof sz / sizeof sz[0]];
   size_t o = 0;
@@ -160,12 +167,7 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
   w.bar = (unsigned*)(base + off[12]);
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int per_sm = spa::select_resident_per_sm(kv_dtype, G);
-  if (per_sm < 1 || sms < 1) return err(SPA_ERR_UNSUPPORTED, "spa_select_noalloc: selection kernel cannot be resident");
-  cudaError_t e = spa::launch_select(P, kv_dtype, spa::select_grid(P, per_sm * sms), st);
+  cudaError_t e = spa::launch_select(P, kv_dtype, grid, st);
   if (e != cudaSuccess) return err(SPA_ERR_CUDA, cudaGetErrorString(e));
   return SPA_OK;
 }
