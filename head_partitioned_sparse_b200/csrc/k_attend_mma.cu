@@ -87,18 +87,25 @@ struct ItemInfo {
   int nch;        // 16-row chunks
 };
 
-__device__ __forceinline__ ItemInfo decode_item(const StepParams& P, const int* pref, int item) {
-  int lo = 0, hi = P.n_slices - 1;
+// Slice of an item (binary search over the item prefix).
+__device__ __forceinline__ int slice_of(const int* pref, int n_slices, int item) {
+  int lo = 0, hi = n_slices - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (pref[mid] <= item) lo = mid; else hi = mid - 1;
   }
+  return lo;
+}
+
+// Decodes an item from shared memory only: the item prefix over slices and each slice's
+// (sequence length, listed rows), both filled at kernel start.
+__device__ __forceinline__ ItemInfo decode_item(const StepParams& P, const int* pref, const int2* sinfo, int item) {
+  const int lo = slice_of(pref, P.n_slices, item);
   ItemInfo it;
   it.s = lo;
-  const int b = lo / P.Hkv, g = lo % P.Hkv;
-  const int L = load_len(P.seq_lens, b, P.Lcap, P.ws.dev_err);
-  const SinkWindow sw(L, P.n_sink, P.window);
-  const int n_rows = sw.n_contig() + (P.is_ret[g] ? P.ws.st[lo].count : 0);
+  const int2 si = sinfo[lo];
+  const SinkWindow sw(si.x, P.n_sink, P.window);
+  const int n_rows = sw.n_contig() + si.y;
   it.nc = sw.n_contig();
   it.n_s = sw.n_s;
   it.w_lo = sw.w_lo;
@@ -114,6 +121,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
   __nv_bfloat16* ring = reinterpret_cast<__nv_bfloat16*>(smem);
   float* mbuf = reinterpret_cast<float*>(smem + kRingBytes);         // [4][G][kPartStride]
   int* pref = reinterpret_cast<int*>(mbuf + 4 * G * kPartStride);    // [n_slices + 1]
+  int2* sinfo = reinterpret_cast<int2*>(pref + ((P.n_slices + 2) & ~1));   // [n_slices] (L, listed rows)
   __shared__ int shi[32];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -130,8 +138,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
         const int b = s / P.Hkv, g = s % P.Hkv;
         const int L = load_len(P.seq_lens, b, P.Lcap, P.ws.dev_err);
         const SinkWindow sw(L, P.n_sink, P.window);
-        const int n = sw.n_contig() + (P.is_ret[g] ? P.ws.st[s].count : 0);
-        it = (n + P.split_rows - 1) / P.split_rows;
+        const int cnt = P.is_ret[g] ? P.ws.st[s].count : 0;
+        sinfo[s] = make_int2(L, cnt);
+        it = (sw.n_contig() + cnt + P.split_rows - 1) / P.split_rows;
       }
       int v = it;
 #pragma unroll
@@ -169,12 +178,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
   // so no copy address waits on a load from the selected list.
   int pf_item = blockIdx.x, pf_ch = warp;
   ItemInfo pf = {};
-  if (pf_item < total) pf = decode_item(P, pref, pf_item);
+  if (pf_item < total) pf = decode_item(P, pref, sinfo, pf_item);
   auto pf_normalise = [&]() {
     while (pf_item < total && pf_ch >= pf.nch) {
       pf_item += gridDim.x;
       pf_ch = warp;
-      if (pf_item < total) pf = decode_item(P, pref, pf_item);
+      if (pf_item < total) pf = decode_item(P, pref, sinfo, pf_item);
     }
   };
   auto load_pos = [&]() -> int {
@@ -220,7 +229,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
   const float scale = P.attn_scale_log2;
 
   for (int item = blockIdx.x; item < total; item += gridDim.x) {
-    const ItemInfo it = decode_item(P, pref, item);
+    const ItemInfo it = decode_item(P, pref, sinfo, item);
     if (it.s != cur_slice) {
       cur_slice = it.s;
       const int b = it.s / P.Hkv, g = it.s % P.Hkv;
@@ -243,6 +252,18 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
         qa[kk][1] = pack2(lo[0], lo[1]);
         qa[kk][2] = pack2(hi[2], hi[3]);
         qa[kk][3] = pack2(lo[2], lo[3]);
+      }
+    }
+    {
+      // the next item of this CTA: bring its slice's rotated query rows into L1 now
+      // (lane (gid, t4): 128-byte line t4 of head gid)
+      const int nx = item + (int)gridDim.x;
+      if (nx < total && gid < G) {
+        const int ns = slice_of(pref, NS, nx);
+        if (ns != it.s) {
+          const float* qn = P.ws.q_rot + ((size_t)(ns / P.Hkv) * P.Hq + (size_t)(ns % P.Hkv) * G + gid) * kHeadDim + 32 * t4;
+          asm volatile("prefetch.global.L1 [%0];\n" ::"l"(qn));
+        }
       }
     }
     float m = -INFINITY, l = 0.f;
@@ -378,7 +399,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
 }
 
 size_t smem_bytes(int G, int max_slices) {
-  return kRingBytes + (size_t)4 * G * kPartStride * 4 + (size_t)(max_slices + 1) * 4;
+  return kRingBytes + (size_t)4 * G * kPartStride * 4 + (size_t)((max_slices + 2) & ~1) * 4 + (size_t)max_slices * 8;
 }
 
 template <int G>

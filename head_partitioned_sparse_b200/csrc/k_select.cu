@@ -122,6 +122,29 @@ __device__ void find_kth_asc_4096(const unsigned (&c)[16], unsigned base, unsign
   __syncthreads();
 }
 
+// Thread t's 16 coalesced histogram words (bins t + 256 k), issued before they are used.
+__device__ __forceinline__ void hist_issue(const unsigned long long* g, unsigned long long (&v)[16]) {
+#pragma unroll
+  for (int k = 0; k < 16; ++k) v[k] = __ldcg(g + threadIdx.x + 256 * k);
+}
+// Redistributes them through shared memory so that thread t holds bins 4095 - 16 t - k,
+// k = 0..15 (the layout of the descending cut search).  Ends with a CTA barrier.
+__device__ __forceinline__ void hist_desc(unsigned long long* stage, const unsigned long long (&v)[16],
+                                          unsigned long long (&m)[16]) {
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const int i = (int)threadIdx.x + 256 * k;
+    stage[i + (i >> 4)] = v[k];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const int i = 4095 - 16 * (int)threadIdx.x - k;
+    m[k] = stage[i + (i >> 4)];
+  }
+  __syncthreads();
+}
+
 // ------------------------------------------------------------------ index scores
 // Scores of 16 tokens at a time on the tensor cores (mma.sync m16n8k16, bf16 in,
 // float32 accumulate): A = the 16 tokens' bf16 index rows (16 x 16 dims), B = the
@@ -330,7 +353,11 @@ struct SmemRefine {
   unsigned long long m3[kBins3];
   unsigned c3[kBins3];
 };
+// Round-1 / round-2 histogram staged for the cut search: loaded coalesced, read back as
+// 16 consecutive bins per thread (index i stored at i + i / 16 against bank conflicts).
+struct SmemStage { unsigned long long h[kBins1 + kBins1 / 16]; };
 union SelSmem {
+  SmemStage stage;
   SmemPro pro;
   SmemScore score;
   SmemMass mass;
@@ -343,7 +370,7 @@ struct SelScalars {
   unsigned shu[32];
   int shi[32];
   int L, b1, b2, b3, kbin, fbin, cut_bin, pos_cut, off, ok, duty;
-  unsigned small_n, kbefore, fbefore, tau, gen;
+  unsigned small_n, kbefore, fbefore, tau;
   unsigned long long above2, cut_above;
 };
 
@@ -507,6 +534,8 @@ template <typename T, int G>
 __device__ void lead_slice(const StepParams& P, SelScalars& sc, int y) {
   const Unit un = unit_of(P, y);
   SliceState* st = P.ws.st + un.s;
+  unsigned gen = 0u;   // barrier generation (thread 0): constant while any CTA scores
+  if (threadIdx.x == 0) gen = *reinterpret_cast<volatile unsigned*>(P.ws.bar + 32);
   __syncthreads();   // earlier readers of sc.qsm / sc.L are done
   if (threadIdx.x == 0) {
     SliceState z;
@@ -526,14 +555,15 @@ __device__ void lead_slice(const StepParams& P, SelScalars& sc, int y) {
     __threadfence();
   }
   __syncthreads();
-  if (threadIdx.x == 0) atomicExch(&st->qidx_ready, sc.gen + 1u);
+  if (threadIdx.x == 0) atomicExch(&st->qidx_ready, gen + 1u);
 }
 
 // Waits (thread 0, bounded) for slice s's q_idx flag of this call; the caller
-// synchronises the CTA afterwards.
-__device__ __forceinline__ void wait_qidx(const StepParams& P, int s, unsigned gen) {
+// synchronises the CTA afterwards.  The barrier generation that tags the flag cannot
+// change before this CTA reaches the first grid barrier.
+__device__ __forceinline__ void wait_qidx(const StepParams& P, int s) {
   volatile unsigned* flag = &P.ws.st[s].qidx_ready;
-  const unsigned want = gen + 1u;
+  const unsigned want = *reinterpret_cast<volatile unsigned*>(P.ws.bar + 32) + 1u;
   const long long t0 = clock64();
   unsigned ns = 32;
   while (*flag != want) {
@@ -582,7 +612,7 @@ __device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc
   __syncthreads();   // earlier readers of sc.L and sc.qsm are done
   if (tid == 0) {
     sc.L = load_len(P.seq_lens, un.b, P.Lcap, P.ws.dev_err);
-    if (16 * l0 < sc.L) wait_qidx(P, un.s, sc.gen);
+    if (16 * l0 < sc.L) wait_qidx(P, un.s);
   }
   __syncthreads();
   const int L = sc.L;
@@ -647,18 +677,16 @@ __device__ void score_phase(const StepParams& P, SmemScore& sm, SelScalars& sc) 
 }
 
 // ------------------------------------------------------------------ cut 1 (per slice)
-__device__ void cut1_slice(const StepParams& P, SelScalars& sc, int y) {
+__device__ void cut1_slice(const StepParams& P, SmemStage& sm, SelScalars& sc, int y) {
   const Unit un = unit_of(P, y);
   const int tid = threadIdx.x;
-  const unsigned long long* g1 = P.ws.hist1 + (size_t)un.s * kBins1;
-  unsigned long long m16[16];
+  unsigned long long v[16], m16[16];
+  hist_issue(P.ws.hist1 + (size_t)un.s * kBins1, v);
   unsigned long long tsum = 0;
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    m16[k] = __ldcg(g1 + (4095 - 16 * tid - k));
-    tsum += m16[k];
-  }
+  for (int k = 0; k < 16; ++k) tsum += v[k];
   const unsigned long long total = block_sum(tsum, sc.shl);
+  hist_desc(sm.h, v, m16);
   SliceState* st = P.ws.st + un.s;
   unsigned long long target = total;
   bool keep_all = P.keep_all || total == 0ull;
@@ -701,8 +729,13 @@ __device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
 #pragma unroll
     for (int u = 0; u < U; ++u) load_group(rows, 16 * (l0 + warp + kWarps * u), jpf, pol, ra[u], rb[u]);
   }
-  const int L = cta_len(P, un.b, sc);
-  if (16 * l0 >= L) return;
+  // the sequence length, the query index vectors and the slice statistics are
+  // requested together; one CTA barrier publishes them
+  __syncthreads();   // earlier readers of sc.L, sc.qsm and the histogram are done
+  int64_t len_raw = 0;
+  if (tid == 0) len_raw = P.seq_lens[un.b];
+  float qv = 0.f;
+  if (tid < G * kIdxDim) qv = __ldcg(&P.ws.q_idx[((size_t)un.b * P.Hq + (size_t)un.g * G) * kIdxDim + tid]);
   for (int i = tid; i < kBins1; i += kSelThreads) sm.cnt[i] = sm.low[i] = 0u;
   // global (M_h, Z_h): warp h merges the ranges' partials, in a fixed order
   if (warp < G) {
@@ -723,8 +756,19 @@ __device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
       sm.Wh[warp] = 1.f / ((float)G * z);
     }
   }
+  if (tid < G * kIdxDim) sc.qsm[tid] = qv;
+  if (tid == 0) {
+    if (len_raw < 1 || len_raw > P.Lcap) {
+      atomicOr(P.ws.dev_err, kErrSeqLen);
+      len_raw = len_raw < 1 ? 1 : P.Lcap;
+    }
+    sc.L = (int)len_raw;
+  }
+  __syncthreads();
+  const int L = sc.L;
+  if (16 * l0 >= L) return;
   uint32_t qb[IdxTiles<G>::NT][2];
-  load_qidx_frag<G>(P, un.b, un.g, sc.qsm, qb);   // its CTA barrier also publishes sm.Mh / sm.Wh
+  qidx_frag<G>(sc.qsm, qb);
   const float scale = P.idx_scale_log2;
   float M[NH], W[NH];
 #pragma unroll
@@ -778,12 +822,13 @@ __device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
 }
 
 template <int G>
-__device__ void mass_phase(const StepParams& P, SmemMass& sm, SelScalars& sc) {
+__device__ void mass_phase(const StepParams& P, SelSmem& sm_all, SelScalars& sc) {
+  SmemMass& sm = sm_all.mass;
   const Ranges R(P);
   for_each_segment(R, [&](int y, int l0, int l1) {
     for (int a = l0; a < l1; a += kMaxRangeGroups) mass_segment<G>(P, sm, sc, R, y, a, min(l1, a + kMaxRangeGroups));
     const int n = R.last_cta(y) - R.first_cta(y) + 1;
-    if (last_of_slice(&P.ws.st[unit_of(P, y).s].ticket_mass, (unsigned)n, &sc.ok)) cut1_slice(P, sc, y);
+    if (last_of_slice(&P.ws.st[unit_of(P, y).s].ticket_mass, (unsigned)n, &sc.ok)) cut1_slice(P, sm_all.stage, sc, y);
   });
 }
 
@@ -874,17 +919,36 @@ __device__ void threshold_unit(const StepParams& P, SelScalars& sc, int y, int c
 }
 
 // ------------------------------------------------------------------ refine (per slice)
-__device__ void refine_slice(const StepParams& P, SmemRefine& sm, SelScalars& sc, int y) {
+__device__ void refine_slice(const StepParams& P, SelSmem& smu, SelScalars& sc, int y) {
+  SmemRefine& sm = smu.ref;
   const Unit un = unit_of(P, y);
-  const int L = cta_len(P, un.b, sc);
   const int tid = threadIdx.x;
   SliceState* st = P.ws.st + un.s;
-  if (tid == 0) sc.b1 = __ldcg(&st->b1);
+  // every input of this step is requested at once: the round-2 histogram (bits 17..6,
+  // filled by the chunks), the slice state and the sequence length
+  unsigned long long v2[16];
+  hist_issue(P.ws.hist2 + (size_t)un.s * kBins2, v2);
+  const unsigned n = __ldcg(&st->cand_count);
+  const unsigned long long target = __ldcg(&st->target);
+  const unsigned long long mab = __ldcg(&st->m_above);
+  __syncthreads();   // earlier readers of the scalars are done
+  if (tid == 32) sc.b1 = __ldcg(&st->b1);
+  if (tid == 0) {
+    sc.L = load_len(P.seq_lens, un.b, P.Lcap, P.ws.dev_err);
+    sc.b2 = -1;
+    sc.b3 = -1;
+    sc.small_n = 0u;
+    sc.kbin = -1;
+  }
   __syncthreads();
-  const int b1 = sc.b1;
+  const int L = sc.L, b1 = sc.b1;
   const SinkWindow sw(L, P.n_sink, P.window);
   const uint2* cand = P.ws.cand + (size_t)un.s * P.Lmax;
-  const unsigned long long* h2 = P.ws.hist2 + (size_t)un.s * kBins2;
+  if (b1 >= 0) {   // round 2 cut (the staging buffer aliases chunk_sel / cnt4k)
+    unsigned long long m16[16];
+    hist_desc(smu.stage.h, v2, m16);
+    find_cut_desc_4096(m16, mab, target, sc.shl, &sc.b2, &sc.above2);
+  }
   int* chunk_sel = sm.chunk_sel;
   unsigned* cnt4k = sm.cnt4k;
   uint2* small = sm.small;
@@ -893,18 +957,9 @@ __device__ void refine_slice(const StepParams& P, SmemRefine& sm, SelScalars& sc
   int pos_cut = INT_MAX;
   for (int c = tid; c < P.n_chunks; c += kSelThreads) chunk_sel[c] = 0;
   if (tid < kBins3) { sm.m3[tid] = 0ull; sm.c3[tid] = 0u; }
-  if (tid == 0) { sc.b2 = -1; sc.b3 = -1; sc.small_n = 0u; sc.kbin = -1; }
   __syncthreads();
   bool found = b1 < 0;   // keep-everything mode needs no cut
   if (b1 >= 0) {
-    const unsigned n = __ldcg(&st->cand_count);
-    const unsigned long long target = __ldcg(&st->target);
-    const unsigned long long mab = __ldcg(&st->m_above);
-    // round 2 (bits 17..6): the chunks filled the slice histogram
-    unsigned long long m16[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) m16[k] = __ldcg(h2 + (4095 - 16 * tid - k));
-    find_cut_desc_4096(m16, mab, target, sc.shl, &sc.b2, &sc.above2);
     const int cb2 = sc.b2;
     // one pass over the candidates: above the round-2 bin they are kept; inside it
     // they feed round 3 (bits 5..0) and are parked in shared memory
@@ -920,13 +975,25 @@ __device__ void refine_slice(const StepParams& P, SmemRefine& sm, SelScalars& sc
       }
     });
     __syncthreads();
-    if (tid == 0 && cb2 >= 0) {
-      unsigned long long cum = sc.above2;
-      for (int k = kBins3 - 1; k >= 0; --k) {
-        if (cum < target && cum + sm.m3[k] >= target) { sc.b3 = k; break; }
-        cum += sm.m3[k];
+    if (tid < 32 && cb2 >= 0) {
+      // round 3 (bits 5..0), descending: lane i holds bins 63 - 2i and 62 - 2i
+      const unsigned long long ma = sm.m3[63 - 2 * tid], mb = sm.m3[62 - 2 * tid];
+      unsigned long long x = ma + mb;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long t = __shfl_up_sync(kFull, x, o);
+        if (tid >= o) x += t;
       }
-      sc.above2 = cum;   // mass strictly above tau
+      const unsigned long long before = sc.above2 + x - (ma + mb);   // mass above bin 63 - 2i
+      int hit = -1;
+      unsigned long long above = 0ull;
+      if (before < target && before + ma >= target) { hit = 63 - 2 * tid; above = before; }
+      else if (before + ma < target && before + ma + mb >= target) { hit = 62 - 2 * tid; above = before + ma; }
+      const unsigned who = __ballot_sync(kFull, hit >= 0);
+      if (who != 0u && tid == __ffs(who) - 1) {
+        sc.b3 = hit;
+        sc.above2 = above;   // mass strictly above tau
+      }
     }
     __syncthreads();
     // b2 and b3 always exist (the candidates carry the mass of bin b1); if a search ever
@@ -1088,18 +1155,15 @@ __global__ void __launch_bounds__(kSelThreads, 4) k_select(StepParams P) {
   }
   const int n_rs = P.B * P.n_ret;
   const int n_units = n_rs * P.n_chunks;
-  // the barrier generation is constant until every CTA has finished the score phase:
-  // it tags this call's q_idx flags
-  if (threadIdx.x == 0) sc.gen = *reinterpret_cast<volatile unsigned*>(P.ws.bar + 32);
   if (blockIdx.x == 0 && threadIdx.x == 0) P.ws.bar[kBarDuty] = 0u;   // taken after two barriers
   score_phase<T, G>(P, sm.score, sc);
   if (!grid_barrier(P.ws.bar, P.ws.dev_err, &sc.ok)) return;
-  mass_phase<G>(P, sm.mass, sc);
+  mass_phase<G>(P, sm, sc);
   if (!grid_barrier(P.ws.bar, P.ws.dev_err, &sc.ok)) return;
   for (int u = blockIdx.x; u < n_units; u += nb) {
     const int y = u / P.n_chunks;
     threshold_unit(P, sc, y, u % P.n_chunks);
-    if (last_of_slice(&P.ws.st[unit_of(P, y).s].ticket_thr, P.n_chunks, &sc.ok)) refine_slice(P, sm.ref, sc, y);
+    if (last_of_slice(&P.ws.st[unit_of(P, y).s].ticket_thr, P.n_chunks, &sc.ok)) refine_slice(P, sm, sc, y);
   }
   qrot_duties<T>(P, sm.pro, sc);   // off the critical path: refine steps run meanwhile
   if (!grid_barrier(P.ws.bar, P.ws.dev_err, &sc.ok)) return;
