@@ -381,7 +381,7 @@ def main_native(args):
         peak, peak_kind = measured_peaks()
         att_bytes = (ab["contig_rows"] + ab["selected_rows"]) * 2 * 128 * s_kv
         achieved = att_bytes / (attend_us * 1e-6) / 1e9
-        traffic = recorded_traffic("k_attend.cu", "attend_ctx128k.md") if args.config == "ctx128k" else None
+        traffic = recorded_traffic("k_attend_mma.cu", "attend_ctx128k.md") if args.config == "ctx128k" else None
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             import oracle as O

@@ -141,7 +141,8 @@ SPA_API spa_status spa_index_append(spa_handle h, const void* k_pre, const int64
  *   p          in (0, 1]; n_sink >= 0; window >= 0; n_sink + window >= 1
  *   sel_idx    device int32 [B][Hkv][Lmax]; sel_count device int32 [B * Hkv]
  * Selection is computed in float32 probabilities with exact integer mass sums
- * (probabilities quantised to multiples of 2^-60) and is deterministic.
+ * (each probability's mass taken exactly from its float32 bit pattern in units of
+ * 2^-63; probabilities below 2^-40 count as 0) and is deterministic.
  */
 SPA_API spa_status spa_select(spa_handle h, const void* q_pre, const void* idx_cache,
                       const uint8_t* head_mask, const int64_t* seq_lens, int B,
