@@ -6,17 +6,18 @@
 // slice's attended rows, the online-softmax state (m, l, acc) of each query head
 // of the GQA group.
 //
-// Work layout.  One CTA per SM, 8 warps.  A split ("item") is split_rows virtual
-// rows of one slice (sinks, window, then the gathered list); CTAs take items
-// c, c + gridDim.x, ...; inside an item, warp w takes the 16-row chunks
-// w, w + 8, ...  Each warp streams its chunks through its own 3-stage ring in
-// shared memory with 16-byte cp.async (one K row = 256 bytes = 16 lanes), keeps
-// prefetching across item boundaries, loads the row positions of the next chunk
-// one issue ahead (no copy waits on a list load), and keeps its own online softmax.
+// Work layout.  One CTA per SM, 8 warps.  The attended rows of all slices form one
+// virtual row space (per slice: sinks, window, then the gathered list); each CTA takes
+// an equal contiguous share of it, i.e. one piece per slice it touches, so every SM gets
+// the same number of rows whatever the slices' lengths.  Inside a piece, warp w takes
+// the 16-row chunks w, w + 8, ...  Each warp streams its chunks through its own 3-stage
+// ring in shared memory with 16-byte cp.async (one K row = 256 bytes = 16 lanes), keeps
+// prefetching across pieces, loads the row positions of the next chunk one issue ahead
+// (no copy waits on a list load), and keeps its own online softmax.
 // (One 256-byte TMA bulk copy per row was measured 4.6x slower than this: the
 // per-request cost of the bulk-copy engine dominates at row granularity.)  At the
-// end of an item the 8 warp states are merged in a fixed 3-round tree and warp 0
-// writes the split's state.
+// end of a piece the 8 warp states are merged in a fixed 3-round tree and warp 0
+// writes the split state of (CTA, slice).
 //
 // Tensor-core mapping (G <= 8 heads of the group, M = 16 rows):
 //   S[16 x 16 tokens] = Q[16 x 128] . K^T:  A rows 0..7 = bf16 high parts of the
@@ -87,31 +88,33 @@ struct ItemInfo {
   int nch;        // 16-row chunks
 };
 
-// Slice of an item (binary search over the item prefix).
-__device__ __forceinline__ int slice_of(const int* pref, int n_slices, int item) {
+// Slice holding virtual row r of the concatenated row space (binary search over the
+// row prefix: the largest s with rpre[s] <= r).
+__device__ __forceinline__ int slice_of_row(const long long* rpre, int n_slices, long long r) {
   int lo = 0, hi = n_slices - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (pref[mid] <= item) lo = mid; else hi = mid - 1;
+    if (rpre[mid] <= r) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
 
-// Decodes an item from shared memory only: the item prefix over slices and each slice's
-// (sequence length, listed rows), both filled at kernel start.
-__device__ __forceinline__ ItemInfo decode_item(const StepParams& P, const int* pref, const int2* sinfo, int item) {
-  const int lo = slice_of(pref, P.n_slices, item);
+// The piece of slice s inside the CTA's row range [r_lo, r_hi), from shared memory only:
+// the row prefix over slices and each slice's (sequence length, listed rows).
+__device__ __forceinline__ ItemInfo piece_info(const StepParams& P, const long long* rpre, const int2* sinfo,
+                                              long long r_lo, long long r_hi, int s) {
   ItemInfo it;
-  it.s = lo;
-  const int2 si = sinfo[lo];
+  it.s = s;
+  const int2 si = sinfo[s];
   const SinkWindow sw(si.x, P.n_sink, P.window);
-  const int n_rows = sw.n_contig() + si.y;
   it.nc = sw.n_contig();
   it.n_s = sw.n_s;
   it.w_lo = sw.w_lo;
-  it.v0 = (item - pref[lo]) * P.split_rows;
-  it.v1 = min(it.v0 + P.split_rows, n_rows);
-  it.nch = (it.v1 - it.v0 + kChunkRows - 1) / kChunkRows;
+  const long long a = r_lo > rpre[s] ? r_lo : rpre[s];
+  const long long e = r_hi < rpre[s + 1] ? r_hi : rpre[s + 1];
+  it.v0 = (int)(a - rpre[s]);
+  it.v1 = (int)(e - rpre[s]);
+  it.nch = it.v1 > it.v0 ? (it.v1 - it.v0 + kChunkRows - 1) / kChunkRows : 0;
   return it;
 }
 
@@ -120,75 +123,95 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
   extern __shared__ __align__(16) unsigned char smem[];
   __nv_bfloat16* ring = reinterpret_cast<__nv_bfloat16*>(smem);
   float* mbuf = reinterpret_cast<float*>(smem + kRingBytes);         // [4][G][kPartStride]
-  int* pref = reinterpret_cast<int*>(mbuf + 4 * G * kPartStride);    // [n_slices + 1]
-  int2* sinfo = reinterpret_cast<int2*>(pref + ((P.n_slices + 2) & ~1));   // [n_slices] (L, listed rows)
+  long long* rpre = reinterpret_cast<long long*>(mbuf + 4 * G * kPartStride);   // [n_slices + 1] row prefix
+  int2* sinfo = reinterpret_cast<int2*>(rpre + P.n_slices + 1);                  // [n_slices] (L, listed rows)
   __shared__ int shi[32];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gid = lane >> 2, t4 = lane & 3;
   const int NS = P.n_slices;
 
-  // ---- item prefix over slices (CTA 0 publishes it for the combine)
+  // ---- row prefix over slices: slice s owns virtual rows [rpre[s], rpre[s + 1]) of the
+  // concatenated row space (its sinks, window, then its gathered list)
   {
-    int carry = 0;
+    __shared__ long long shl[32];
+    long long carry = 0;
     for (int base = 0; base < NS; base += kWarps * 32) {
       const int s = base + tid;
-      int it = 0;
+      long long rows = 0;
       if (s < NS) {
         const int b = s / P.Hkv, g = s % P.Hkv;
         const int L = load_len(P.seq_lens, b, P.Lcap, P.ws.dev_err);
         const SinkWindow sw(L, P.n_sink, P.window);
         const int cnt = P.is_ret[g] ? P.ws.st[s].count : 0;
         sinfo[s] = make_int2(L, cnt);
-        it = (sw.n_contig() + cnt + P.split_rows - 1) / P.split_rows;
+        rows = sw.n_contig() + cnt;
       }
-      int v = it;
+      long long v = rows;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(kFull, v, o);
+        const long long y = __shfl_up_sync(kFull, v, o);
         if (lane >= o) v += y;
       }
-      if (lane == 31) shi[warp] = v;
+      if (lane == 31) shl[warp] = v;
       __syncthreads();
       if (warp == 0) {
-        int w = lane < kWarps ? shi[lane] : 0;
+        long long w = lane < kWarps ? shl[lane] : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(kFull, w, o);
+          const long long y = __shfl_up_sync(kFull, w, o);
           if (lane >= o) w += y;
         }
-        if (lane < kWarps) shi[lane] = w;
+        if (lane < kWarps) shl[lane] = w;
       }
       __syncthreads();
-      if (s < NS) pref[s] = carry + (warp ? shi[warp - 1] : 0) + v - it;
-      carry += shi[kWarps - 1];
+      if (s < NS) rpre[s] = carry + (warp ? shl[warp - 1] : 0) + v - rows;
+      carry += shl[kWarps - 1];
       __syncthreads();
     }
-    if (tid == 0) pref[NS] = carry;
+    if (tid == 0) rpre[NS] = carry;
     __syncthreads();
   }
-  const int total = pref[NS];
-  if (blockIdx.x == 0)
-    for (int s = tid; s <= NS; s += kWarps * 32) P.ws.item_base[s] = pref[s];
+  // ---- the CTA's equal share of the row space, as one piece per slice it touches.  The
+  // split state of the piece of slice s goes to partial slot blockIdx.x + s, so each
+  // slice's slots are consecutive; CTA 0 publishes where they start for the combine.  A
+  // CTA whose range starts exactly at a slice boundary writes an empty state into the one
+  // slot (its index + s - 1) that the previous slice's range would otherwise skip.
+  const long long T = rpre[NS];
+  const int nb = gridDim.x;
+  const long long r_lo = (long long)blockIdx.x * T / nb, r_hi = (long long)(blockIdx.x + 1) * T / nb;
+  auto owner = [&](long long r) { return (int)(((r + 1) * nb - 1) / T); };
+  if (blockIdx.x == 0) {
+    for (int s = tid; s < NS; s += kWarps * 32) P.ws.item_base[s] = owner(rpre[s]) + s;
+    if (tid == 0) P.ws.item_base[NS] = owner(T - 1) + NS;
+  }
+  const int s_first = r_lo < r_hi ? slice_of_row(rpre, NS, r_lo) : 1;
+  const int s_last = r_lo < r_hi ? slice_of_row(rpre, NS, r_hi - 1) : 0;
+  if (r_lo < r_hi && s_first > 0 && rpre[s_first] == r_lo && warp == 0 && gid < G) {
+    float* dst = P.ws.part + ((size_t)(blockIdx.x + s_first - 1) * G + gid) * kPartStride;
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) *reinterpret_cast<float2*>(dst + 8 * nt + 2 * t4) = make_float2(0.f, 0.f);
+    if (t4 == 0) { dst[kHeadDim] = -INFINITY; dst[kHeadDim + 1] = 0.f; }
+  }
 
   __nv_bfloat16* myring = ring + (size_t)warp * kStages * kStageElems;
 
   // ---- prefetch cursor over this warp's (item, chunk) units.  The row positions of
   // the unit to issue next are loaded one issue ahead (apos, lane r < 16 holds row r),
   // so no copy address waits on a load from the selected list.
-  int pf_item = blockIdx.x, pf_ch = warp;
+  int pf_item = s_first, pf_ch = warp;   // pf_item: the slice of the piece
   ItemInfo pf = {};
-  if (pf_item < total) pf = decode_item(P, pref, sinfo, pf_item);
+  if (pf_item <= s_last) pf = piece_info(P, rpre, sinfo, r_lo, r_hi, pf_item);
   auto pf_normalise = [&]() {
-    while (pf_item < total && pf_ch >= pf.nch) {
-      pf_item += gridDim.x;
+    while (pf_item <= s_last && pf_ch >= pf.nch) {
+      ++pf_item;
       pf_ch = warp;
-      if (pf_item < total) pf = decode_item(P, pref, sinfo, pf_item);
+      if (pf_item <= s_last) pf = piece_info(P, rpre, sinfo, r_lo, r_hi, pf_item);
     }
   };
   auto load_pos = [&]() -> int {
     int pos = 0;
-    if (pf_item < total && lane < kChunkRows) {
+    if (pf_item <= s_last && lane < kChunkRows) {
       const int r0 = pf.v0 + pf_ch * kChunkRows;
       int v = r0 + lane;
       if (v >= pf.v1) v = r0;   // rows past the item repeat row 0 (finite, masked later)
@@ -202,7 +225,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
   int issued = 0;  // units issued so far (selects the ring slot)
   auto issue_next = [&]() {
     __nv_bfloat16* dst = myring + (size_t)(issued % kStages) * kStageElems;
-    if (pf_item < total) {
+    if (pf_item <= s_last) {
       const __nv_bfloat16* kb = (const __nv_bfloat16*)P.k_cache + (size_t)pf.s * P.Lmax * kHeadDim;
       const __nv_bfloat16* vb = (const __nv_bfloat16*)P.v_cache + (size_t)pf.s * P.Lmax * kHeadDim;
 #pragma unroll
@@ -228,8 +251,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
   uint32_t qa[8][4];   // A fragments of Q (hi rows 0..7, residual rows 8..15), per 16-dim k-step
   const float scale = P.attn_scale_log2;
 
-  for (int item = blockIdx.x; item < total; item += gridDim.x) {
-    const ItemInfo it = decode_item(P, pref, sinfo, item);
+  for (int ps = s_first; ps <= s_last; ++ps) {
+    const ItemInfo it = piece_info(P, rpre, sinfo, r_lo, r_hi, ps);
     if (it.s != cur_slice) {
       cur_slice = it.s;
       const int b = it.s / P.Hkv, g = it.s % P.Hkv;
@@ -255,15 +278,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
       }
     }
     {
-      // the next item of this CTA: bring its slice's rotated query rows into L1 now
+      // the next piece of this CTA: bring its slice's rotated query rows into L1 now
       // (lane (gid, t4): 128-byte line t4 of head gid)
-      const int nx = item + (int)gridDim.x;
-      if (nx < total && gid < G) {
-        const int ns = slice_of(pref, NS, nx);
-        if (ns != it.s) {
-          const float* qn = P.ws.q_rot + ((size_t)(ns / P.Hkv) * P.Hq + (size_t)(ns % P.Hkv) * G + gid) * kHeadDim + 32 * t4;
-          asm volatile("prefetch.global.L1 [%0];\n" ::"l"(qn));
-        }
+      const int ns = ps + 1;
+      if (ns <= s_last && gid < G) {
+        const float* qn = P.ws.q_rot + ((size_t)(ns / P.Hkv) * P.Hq + (size_t)(ns % P.Hkv) * G + gid) * kHeadDim + 32 * t4;
+        asm volatile("prefetch.global.L1 [%0];\n" ::"l"(qn));
       }
     }
     float m = -INFINITY, l = 0.f;
@@ -388,7 +408,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
       __syncthreads();
     }
     if (warp == 0 && gid < G) {
-      float* dst = P.ws.part + ((size_t)item * G + gid) * kPartStride;
+      float* dst = P.ws.part + ((size_t)(blockIdx.x + it.s) * G + gid) * kPartStride;
 #pragma unroll
       for (int nt = 0; nt < 16; ++nt)
         *reinterpret_cast<float2*>(dst + 8 * nt + 2 * t4) = make_float2(o[nt][0], o[nt][1]);
@@ -399,7 +419,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
 }
 
 size_t smem_bytes(int G, int max_slices) {
-  return kRingBytes + (size_t)4 * G * kPartStride * 4 + (size_t)((max_slices + 2) & ~1) * 4 + (size_t)max_slices * 8;
+  return kRingBytes + (size_t)4 * G * kPartStride * 4 + (size_t)(max_slices + 1) * 8 + (size_t)max_slices * 8;
 }
 
 template <int G>

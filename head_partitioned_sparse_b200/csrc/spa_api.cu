@@ -46,6 +46,8 @@ Layout plan(const spa_config& c, int split_rows) {
   const int64_t Lmax = c.max_ctx;
   L.n_chunks_max = (int)((Lmax + spa::kChunk - 1) / spa::kChunk);
   L.max_items = (int64_t)slices * ((Lmax + split_rows - 1) / split_rows);
+  const int64_t part_slots = L.max_items > (int64_t)(spa::kMaxAttendCtas + slices + 1)
+                                 ? L.max_items : (int64_t)(spa::kMaxAttendCtas + slices + 1);
   size_t sz[18] = {
       (size_t)c.n_q_heads * 16 * 128 * 4,                  // 0 P_q
       (size_t)c.n_kv_heads * 16 * 128 * 4,                 // 1 P_k
@@ -61,7 +63,7 @@ Layout plan(const spa_config& c, int split_rows) {
       slices * sizeof(spa::SliceState),                    // 11 st
       slices * (size_t)Lmax * 4,                           // 12 list
       (slices + 1) * 4,                                    // 13 item_base
-      (size_t)L.max_items * G * spa::kPartStride * 4,      // 14 part
+      (size_t)part_slots * G * spa::kPartStride * 4,       // 14 split states
       256,                                                 // 15 dev_err
       slices * spa::kBins2 * 8,                            // 16 hist2
       spa::kBarWords * 4,                                  // 17 selection grid barrier
@@ -376,7 +378,8 @@ spa_status spa_decode(spa_handle h, const void* q_pre, const void* k_cache, cons
   // upper bound on splits: every slice has at most Lcap rows
   const int64_t per_slice = (P.Lcap + P.split_rows - 1) / P.split_rows;
   const int64_t max_items = per_slice * P.n_slices;
-  const int64_t cap = (int64_t)h->num_sms * h->attend_occ;
+  int64_t cap = (int64_t)h->num_sms * h->attend_occ;
+  if (cap > spa::kMaxAttendCtas) cap = spa::kMaxAttendCtas;
   const int grid = (int)(max_items < cap ? max_items : cap);
   if ((r = run(h, SPA_K_ATTEND, st, "attend", [&] { return spa::launch_attend(P, h->cfg.kv_dtype, grid, st); })))
     return r;

@@ -32,6 +32,9 @@ constexpr int kMassMinExp = 87;
 
 // Largest grid of the selection kernel (sizes the per-range statistics).
 constexpr int kMaxSelectGrid = 8192;
+// Largest grid of the attention kernels (the bf16 kernel writes one split state per
+// (CTA, slice) it touches: at most grid + slices of them).
+constexpr int kMaxAttendCtas = 1024;
 
 // Attention splits ("items") cover up to split_rows rows of one slice; rows are
 // staged through shared memory kTile rows at a time.
@@ -88,7 +91,7 @@ struct Workspace {
   SliceState* st;        // [Bm*Hkv]
   int* list;             // [Bm*Hkv][Lmax]  selected positions (decode)
   int* item_base;        // [Bm*Hkv + 1]
-  float* part;           // [max_items][G][kPartStride]
+  float* part;           // [max(max_items, kMaxAttendCtas + Bm*Hkv + 1)][G][kPartStride]
   unsigned* dev_err;     // [1]
   unsigned* bar;         // [kBarWords] selection kernel: grid barrier and q_rot duty ticket
   int64_t max_items;
