@@ -17,7 +17,9 @@
 // (One 256-byte TMA bulk copy per row was measured 4.6x slower than this: the
 // per-request cost of the bulk-copy engine dominates at row granularity.)  At the
 // end of a piece the 8 warp states are merged in a fixed 3-round tree and warp 0
-// writes the split state of (CTA, slice).
+// writes the split state of (CTA, slice); the last CTA to finish a piece of a slice
+// (a per-slice ticket) combines the slice's states into the output, so a decode step
+// needs no separate combine launch.
 //
 // Tensor-core mapping (G <= 8 heads of the group, M = 16 rows):
 //   S[16 x 16 tokens] = Q[16 x 128] . K^T:  A rows 0..7 = bf16 high parts of the
@@ -118,6 +120,81 @@ __device__ __forceinline__ ItemInfo piece_info(const StepParams& P, const long l
   return it;
 }
 
+// Combines slice s's split states (slots c + s for CTAs c0..c1) into out[b][g G + h]:
+// warp w takes head w % G and the slots c0 + w / G, c0 + w / G + 8 / G, ... (merged in
+// order), then the warps of a head are merged in warp order through shared memory.
+// Lane l holds dims 4l..4l+3.  Called by every thread of the CTA.
+template <int G>
+__device__ void combine_slice(const StepParams& P, int s, int c0, int c1, float* cbuf) {
+  constexpr int kPer = kWarps / G;   // warps per head
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int h = warp % G, sub = warp / G;
+  float m = -INFINITY, l = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  constexpr int kB = 4;
+  for (int c = c0 + sub; c <= c1; c += kPer * kB) {
+    float4 a[kB];
+    float mi[kB], li[kB];
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int cc = c + u * kPer;
+      if (cc <= c1) {
+        const float* pp = P.ws.part + ((size_t)(cc + s) * G + h) * kPartStride;
+        a[u] = __ldcg(reinterpret_cast<const float4*>(pp) + lane);
+        mi[u] = __ldcg(pp + kHeadDim);
+        li[u] = __ldcg(pp + kHeadDim + 1);
+      } else {
+        a[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        mi[u] = -INFINITY;
+        li[u] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const float mn = fmaxf(m, mi[u]);
+      if (mn == -INFINITY) continue;
+      const float sa = exp2f(m - mn), sb = exp2f(mi[u] - mn);
+      l = l * sa + li[u] * sb;
+      acc.x = acc.x * sa + a[u].x * sb;
+      acc.y = acc.y * sa + a[u].y * sb;
+      acc.z = acc.z * sa + a[u].z * sb;
+      acc.w = acc.w * sa + a[u].w * sb;
+      m = mn;
+    }
+  }
+  float* mine = cbuf + (size_t)warp * kPartStride;
+  *reinterpret_cast<float4*>(mine + 4 * lane) = acc;
+  if (lane == 0) { mine[kHeadDim] = m; mine[kHeadDim + 1] = l; }
+  __syncthreads();
+  if (warp < G) {
+    float M = -INFINITY, Ls = 0.f;
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k = 0; k < kPer; ++k) {
+      const float* src = cbuf + (size_t)(h + G * k) * kPartStride;
+      const float m2 = src[kHeadDim], l2 = src[kHeadDim + 1];
+      const float mn = fmaxf(M, m2);
+      if (mn == -INFINITY) continue;
+      const float sa = exp2f(M - mn), sb = exp2f(m2 - mn);
+      const float4 v = *reinterpret_cast<const float4*>(src + 4 * lane);
+      Ls = Ls * sa + l2 * sb;
+      num.x = num.x * sa + v.x * sb;
+      num.y = num.y * sa + v.y * sb;
+      num.z = num.z * sa + v.z * sb;
+      num.w = num.w * sa + v.w * sb;
+      M = mn;
+    }
+    const float inv = 1.f / Ls;
+    const int b = s / P.Hkv, g = s % P.Hkv;
+    *reinterpret_cast<float4*>(P.out + ((size_t)b * P.Hq + (size_t)g * G + h) * kHeadDim + 4 * lane) =
+        make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
+  }
+  if (threadIdx.x == 0 && P.sel_count) {
+    const int g = s % P.Hkv;
+    P.sel_count[s] = P.is_ret[g] ? P.ws.st[s].count : 0;
+  }
+  __syncthreads();   // cbuf reused by the next combine
+}
+
 template <int G>
 __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -125,7 +202,10 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
   float* mbuf = reinterpret_cast<float*>(smem + kRingBytes);         // [4][G][kPartStride]
   long long* rpre = reinterpret_cast<long long*>(mbuf + 4 * G * kPartStride);   // [n_slices + 1] row prefix
   int2* sinfo = reinterpret_cast<int2*>(rpre + P.n_slices + 1);                  // [n_slices] (L, listed rows)
+  // [8 warps][kPartStride], 16-byte aligned (float4 accesses)
+  float* cbuf = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(sinfo + P.n_slices) + 15) & ~uintptr_t(15));
   __shared__ int shi[32];
+  __shared__ int s_merge;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gid = lane >> 2, t4 = lane & 3;
@@ -178,21 +258,11 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
   // CTA whose range starts exactly at a slice boundary writes an empty state into the one
   // slot (its index + s - 1) that the previous slice's range would otherwise skip.
   const long long T = rpre[NS];
-  const int nb = gridDim.x;
-  const long long r_lo = (long long)blockIdx.x * T / nb, r_hi = (long long)(blockIdx.x + 1) * T / nb;
+  const int nb = (long long)gridDim.x < T ? (int)gridDim.x : (int)T;   // active CTAs: >= 1 row each
+  const long long r_lo = (long long)blockIdx.x * T / nb, r_hi = blockIdx.x < nb ? (long long)(blockIdx.x + 1) * T / nb : r_lo;
   auto owner = [&](long long r) { return (int)(((r + 1) * nb - 1) / T); };
-  if (blockIdx.x == 0) {
-    for (int s = tid; s < NS; s += kWarps * 32) P.ws.item_base[s] = owner(rpre[s]) + s;
-    if (tid == 0) P.ws.item_base[NS] = owner(T - 1) + NS;
-  }
   const int s_first = r_lo < r_hi ? slice_of_row(rpre, NS, r_lo) : 1;
   const int s_last = r_lo < r_hi ? slice_of_row(rpre, NS, r_hi - 1) : 0;
-  if (r_lo < r_hi && s_first > 0 && rpre[s_first] == r_lo && warp == 0 && gid < G) {
-    float* dst = P.ws.part + ((size_t)(blockIdx.x + s_first - 1) * G + gid) * kPartStride;
-#pragma unroll
-    for (int nt = 0; nt < 16; ++nt) *reinterpret_cast<float2*>(dst + 8 * nt + 2 * t4) = make_float2(0.f, 0.f);
-    if (t4 == 0) { dst[kHeadDim] = -INFINITY; dst[kHeadDim + 1] = 0.f; }
-  }
 
   __nv_bfloat16* myring = ring + (size_t)warp * kStages * kStageElems;
 
@@ -413,13 +483,25 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
       for (int nt = 0; nt < 16; ++nt)
         *reinterpret_cast<float2*>(dst + 8 * nt + 2 * t4) = make_float2(o[nt][0], o[nt][1]);
       if (t4 == 0) { dst[kHeadDim] = m; dst[kHeadDim + 1] = l; }
+      __threadfence();
+    }
+    // ---- the last CTA to finish a piece of this slice combines its split states
+    __syncthreads();
+    const int c0 = owner(rpre[it.s]), c1 = owner(rpre[it.s + 1] - 1);
+    if (tid == 0) s_merge = atomicAdd(&P.ws.attn_ticket[it.s], 1u) == (unsigned)(c1 - c0);
+    __syncthreads();
+    if (s_merge) {
+      __threadfence();
+      combine_slice<G>(P, it.s, c0, c1, cbuf);
+      if (tid == 0) P.ws.attn_ticket[it.s] = 0u;   // ready for the next call
     }
   }
   asm volatile("cp.async.wait_all;\n" ::: "memory");
 }
 
 size_t smem_bytes(int G, int max_slices) {
-  return kRingBytes + (size_t)4 * G * kPartStride * 4 + (size_t)(max_slices + 1) * 8 + (size_t)max_slices * 8;
+  return kRingBytes + (size_t)4 * G * kPartStride * 4 + (size_t)(max_slices + 1) * 8 + (size_t)max_slices * 8 +
+         16 + (size_t)kWarps * kPartStride * 4;
 }
 
 template <int G>

@@ -32,7 +32,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
-  size_t off[18];
+  size_t off[19];
   size_t total;
   int64_t max_items;
   int n_chunks_max;
@@ -48,7 +48,7 @@ Layout plan(const spa_config& c, int split_rows) {
   L.max_items = (int64_t)slices * ((Lmax + split_rows - 1) / split_rows);
   const int64_t part_slots = L.max_items > (int64_t)(spa::kMaxAttendCtas + slices + 1)
                                  ? L.max_items : (int64_t)(spa::kMaxAttendCtas + slices + 1);
-  size_t sz[18] = {
+  size_t sz[19] = {
       (size_t)c.n_q_heads * 16 * 128 * 4,                  // 0 P_q
       (size_t)c.n_kv_heads * 16 * 128 * 4,                 // 1 P_k
       64 * 8,                                              // 2 inv_freq
@@ -67,9 +67,10 @@ Layout plan(const spa_config& c, int split_rows) {
       256,                                                 // 15 dev_err
       slices * spa::kBins2 * 8,                            // 16 hist2
       spa::kBarWords * 4,                                  // 17 selection grid barrier
+      slices * 4,                                          // 18 attention tickets
   };
   size_t o = 0;
-  for (int i = 0; i < 18; ++i) {
+  for (int i = 0; i < 19; ++i) {
     L.off[i] = o;
     o += round_up(sz[i], 256);
   }
@@ -279,6 +280,7 @@ spa_status spa_create(spa_handle* out, const spa_config* cfg) {
   w.dev_err = (unsigned*)(base + L.off[15]);
   w.hist2 = (unsigned long long*)(base + L.off[16]);
   w.bar = (unsigned*)(base + L.off[17]);
+  w.attn_ticket = (unsigned*)(base + L.off[18]);
   w.max_items = L.max_items;
   h->n_chunks_max = L.n_chunks_max;
 
@@ -292,6 +294,7 @@ spa_status spa_create(spa_handle* out, const spa_config* cfg) {
       (e = cudaMemcpy(w.inv_freq, invf, sizeof invf, cudaMemcpyHostToDevice)) != cudaSuccess ||
       (e = cudaMemset(w.dev_err, 0, 4)) != cudaSuccess || (e = cudaMemset(w.bar, 0, spa::kBarWords * 4)) != cudaSuccess ||
       (e = cudaMemset(w.st, 0, L.off[12] - L.off[11])) != cudaSuccess ||
+      (e = cudaMemset(w.attn_ticket, 0, (size_t)cfg->max_batch * cfg->n_kv_heads * 4)) != cudaSuccess ||
       (e = cudaDeviceSynchronize()) != cudaSuccess) {
     cudaFree(h->mem);
     delete h;
@@ -381,8 +384,11 @@ spa_status spa_decode(spa_handle h, const void* q_pre, const void* k_cache, cons
   int64_t cap = (int64_t)h->num_sms * h->attend_occ;
   if (cap > spa::kMaxAttendCtas) cap = spa::kMaxAttendCtas;
   const int grid = (int)(max_items < cap ? max_items : cap);
+  // bf16 caches: the attention kernel combines the splits and reports the counts itself
+  if (h->cfg.kv_dtype == 0) P.sel_count = sel_count_opt;
   if ((r = run(h, SPA_K_ATTEND, st, "attend", [&] { return spa::launch_attend(P, h->cfg.kv_dtype, grid, st); })))
     return r;
+  if (h->cfg.kv_dtype == 0) return SPA_OK;
   P.sel_count = sel_count_opt;
   return run(h, SPA_K_COMBINE, st, "combine", [&] { return spa::launch_combine(P, st); });
 }
@@ -399,6 +405,7 @@ spa_status spa_device_status(spa_handle h, spa_stream stream) {
     if (flags & spa::kErrTimeout) {
       // the grid barrier may have been left mid-way: start the next call from a clean barrier
       cudaMemset(h->ws.bar, 0, spa::kBarWords * 4);
+      cudaMemset(h->ws.attn_ticket, 0, sizeof(unsigned) * (size_t)h->cfg.max_batch * h->cfg.n_kv_heads);
       // q_idx flags are tagged with the barrier generation, which restarts at 0
       cudaMemset(h->ws.st, 0, sizeof(spa::SliceState) * (size_t)h->cfg.max_batch * h->cfg.n_kv_heads);
       cudaDeviceSynchronize();

@@ -91,6 +91,7 @@ struct Workspace {
   SliceState* st;        // [Bm*Hkv]
   int* list;             // [Bm*Hkv][Lmax]  selected positions (decode)
   int* item_base;        // [Bm*Hkv + 1]
+  unsigned* attn_ticket; // [Bm*Hkv] pieces of each slice finished (bf16 attention; reset by its combiner)
   float* part;           // [max(max_items, kMaxAttendCtas + Bm*Hkv + 1)][G][kPartStride]
   unsigned* dev_err;     // [1]
   unsigned* bar;         // [kBarWords] selection kernel: grid barrier and q_rot duty ticket

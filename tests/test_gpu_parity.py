@@ -246,7 +246,7 @@ def test_all_streaming_and_all_retrieval(retrieval):
         n0 = B.spa_launch_count(h.h)
         out, cnt = gpu_decode(h, inp, dev)
         launches = B.spa_launch_count(h.h) - n0
-    assert launches == 3   # one cooperative selection kernel, attention, combine
+    assert launches == (2 if inp.dtype == "bf16" else 3)   # selection, attention (+ combine for float32 caches)
     _, res = O.decode_inputs(inp, idx_cache=idx)
     for g in retrieval:
         check_selection(lists[(0, g)], res[(0, g)], inp.p, inp.n_sink, inp.window)
