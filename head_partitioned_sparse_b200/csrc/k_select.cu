@@ -274,14 +274,22 @@ __device__ __forceinline__ void load_group(const uint2* rows, int j, int jend, u
   rb = jb < jend ? ld_hint(rows + 4 * (size_t)jb + t4, pol) : make_uint2(0u, 0u);
 }
 
+// 2^x with the hardware approximation (relative error about 2^-22, results below 2^-126
+// flushed to 0), used by both index passes so that sums and probabilities agree.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Online max / sum-of-exp2 with one exp2 per value; -inf values are skipped.
 __device__ __forceinline__ void online_add(float& m, float& z, float l) {
   if (l == -INFINITY) return;
   if (l > m) {
-    z = z * exp2f(m - l) + 1.f;
+    z = z * ex2(m - l) + 1.f;
     m = l;
   } else {
-    z += exp2f(l - m);
+    z += ex2(l - m);
   }
 }
 
@@ -796,7 +804,10 @@ __device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
       for (int cc = 0; cc < 2; ++cc) {
         float acc = 0.f;
 #pragma unroll
-        for (int h = 0; h < NH; ++h) acc += W[h] == 0.f ? 0.f : exp2f(lg[h][cc] - M[h]) * W[h];
+        for (int h = 0; h < NH; ++h) {
+          if (G < 4 && W[h] == 0.f) continue;   // lanes of absent heads (G < 4) add nothing
+          acc += ex2(lg[h][cc] - M[h]) * W[h];
+        }
         acc += __shfl_xor_sync(kFull, acc, 1);
         acc += __shfl_xor_sync(kFull, acc, 2);
         pr[cc] = acc;
