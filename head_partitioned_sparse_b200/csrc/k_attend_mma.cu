@@ -46,9 +46,16 @@ constexpr int kRowPad = kHeadDim + 8;                               // 136 bf16 
 constexpr int kStageElems = 2 * kChunkRows * kRowPad;               // K then V
 constexpr size_t kRingBytes = (size_t)kWarps * kStages * kStageElems * 2;
 
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+// K/V rows are read once per step: their L2 lines are marked first to go, so the
+// stream does not push out the small tensors the next call reads first.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, uint64_t pol) {
   const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "l"(pol) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_stages() {
@@ -299,6 +306,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
   pf_normalise();
   int apos = load_pos();
   int issued = 0;  // units issued so far (selects the ring slot)
+  const uint64_t kv_pol = l2_evict_first();
   auto issue_next = [&]() {
     __nv_bfloat16* dst = myring + (size_t)(issued % kStages) * kStageElems;
     if (pf_item <= s_last) {
@@ -310,7 +318,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
         const int tv = idx >> 8, rem = idx & 255, r = rem >> 4, c = rem & 15;
         const int prow = __shfl_sync(kFull, apos, r);
         const __nv_bfloat16* src = (tv ? vb : kb) + (size_t)prow * kHeadDim + c * 8;
-        cp_async16(dst + tv * kChunkRows * kRowPad + r * kRowPad + c * 8, src);
+        cp_async16(dst + tv * kChunkRows * kRowPad + r * kRowPad + c * 8, src, kv_pol);
       }
       pf_ch += kWarps;
       pf_normalise();

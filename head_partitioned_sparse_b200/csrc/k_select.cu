@@ -257,6 +257,13 @@ __device__ __forceinline__ uint64_t l2_policy_drop() {
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
   return p;
 }
+__device__ __forceinline__ float4 ld_keep(const float4* ptr, uint64_t pol) {
+  float4 v;
+  asm volatile("ld.global.nc.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;\n"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(ptr), "l"(pol));
+  return v;
+}
 __device__ __forceinline__ uint2 ld_hint(const uint2* ptr, uint64_t pol) {
   uint2 v;
   asm volatile("ld.global.nc.L2::cache_hint.v2.u32 {%0, %1}, [%2], %3;\n"
@@ -460,6 +467,7 @@ __device__ void compute_qidx(const StepParams& P, int b, int g, SelScalars& sc) 
   int64_t len_raw = 0;
   if (tid == 0) len_raw = P.seq_lens[b];   // validated after the dot products are issued
   const T* q = (const T*)P.q_pre + ((size_t)b * P.Hq + (size_t)g * G) * kHeadDim;
+  const uint64_t keep = l2_policy_keep();   // projectors are reread by the next call
   for (int w = tid; w < G * kIdxDim * 4; w += kSelThreads) {   // whole warps (G * 64 = 64k)
     const int o = w >> 2, qd = w & 3, h = o / kIdxDim;
     const float4* prow = reinterpret_cast<const float4*>(P.ws.P_q + ((size_t)g * G * kIdxDim + o) * kHeadDim) + 8 * qd;
@@ -470,7 +478,7 @@ __device__ void compute_qidx(const StepParams& P, int b, int g, SelScalars& sc) 
       float4 pv[4];
       float qv[16];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) pv[k] = __ldg(prow + 4 * half + k);
+      for (int k = 0; k < 4; ++k) pv[k] = ld_keep(prow + 4 * half + k, keep);
 #pragma unroll
       for (int k = 0; k < 16; ++k) qv[k] = Elem<T>::get(qrow, 16 * half + k);
 #pragma unroll
