@@ -473,20 +473,40 @@ __device__ void compute_qidx(const StepParams& P, int b, int g, SelScalars& sc) 
     const float4* prow = reinterpret_cast<const float4*>(P.ws.P_q + ((size_t)g * G * kIdxDim + o) * kHeadDim) + 8 * qd;
     const T* qrow = q + h * kHeadDim + 32 * qd;
     double acc = 0.0;
+    if (sizeof(T) == 2) {
+      // bf16 queries: all 32 projector values and the 32 query values in one round trip
+      // (q_pre is 16-byte aligned and the quarter starts at a 64-byte offset)
+      float4 pv[8];
+      uint4 qw[4];
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      float4 pv[4];
-      float qv[16];
+      for (int k = 0; k < 8; ++k) pv[k] = ld_keep(prow + k, keep);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) pv[k] = ld_keep(prow + 4 * half + k, keep);
+      for (int k = 0; k < 4; ++k) qw[k] = __ldg(reinterpret_cast<const uint4*>(qrow) + k);
 #pragma unroll
-      for (int k = 0; k < 16; ++k) qv[k] = Elem<T>::get(qrow, 16 * half + k);
+      for (int k = 0; k < 8; ++k) {
+        const uint4 w4 = qw[k >> 1];
+        const uint32_t wa = (k & 1) ? w4.z : w4.x, wb = (k & 1) ? w4.w : w4.y;
+        acc += (double)pv[k].x * (double)bf16_lo(wa);
+        acc += (double)pv[k].y * (double)bf16_hi(wa);
+        acc += (double)pv[k].z * (double)bf16_lo(wb);
+        acc += (double)pv[k].w * (double)bf16_hi(wb);
+      }
+    } else {
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        acc += (double)pv[k].x * (double)qv[4 * k];
-        acc += (double)pv[k].y * (double)qv[4 * k + 1];
-        acc += (double)pv[k].z * (double)qv[4 * k + 2];
-        acc += (double)pv[k].w * (double)qv[4 * k + 3];
+      for (int half = 0; half < 2; ++half) {
+        float4 pv[4];
+        float qv[16];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) pv[k] = ld_keep(prow + 4 * half + k, keep);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) qv[k] = Elem<T>::get(qrow, 16 * half + k);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          acc += (double)pv[k].x * (double)qv[4 * k];
+          acc += (double)pv[k].y * (double)qv[4 * k + 1];
+          acc += (double)pv[k].z * (double)qv[4 * k + 2];
+          acc += (double)pv[k].w * (double)qv[4 * k + 3];
+        }
       }
     }
     acc += __shfl_xor_sync(kFull, acc, 1);
