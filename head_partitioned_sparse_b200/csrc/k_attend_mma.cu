@@ -217,7 +217,6 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
   int2* sinfo = reinterpret_cast<int2*>(rpre + P.n_slices + 1);                  // [n_slices] (L, listed rows)
   // [8 warps][kPartStride], 16-byte aligned (float4 accesses)
   float* cbuf = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(sinfo + P.n_slices) + 15) & ~uintptr_t(15));
-  __shared__ int shi[32];
   __shared__ int s_merge;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
