@@ -354,7 +354,7 @@ __device__ bool last_of_slice(unsigned* ticket, unsigned n_units, int* s_flag) {
 
 // ------------------------------------------------------------------ shared memory
 constexpr int kWarps = kSelThreads / 32;
-constexpr int kGroupBatch = 4;                // groups per warp loaded together (double-buffered)
+constexpr int kGroupBatch = 4;                // groups per warp loaded together (8 spills at 64 registers)
 constexpr int kSmallCap = 1024;   // candidates of the round-2 cut bin held in shared memory
 constexpr int kCandBatch = 8;     // candidates loaded per thread before any is used
 
