@@ -1225,15 +1225,13 @@ int resident_tg() {
 
 }  // namespace
 
-// Grid of the selection launch.  When there is at least half a full wave of work it is
-// every resident CTA (the same count on every SM, so the range-partitioned phases are
-// balanced per SM); never more CTAs than 16-token groups, so no CTA has an empty range.
+// Grid of the selection launch: every resident CTA (the same count on every SM, so the
+// range-partitioned score and mass phases are balanced per SM), but never more CTAs than
+// 16-token groups, so no CTA has an empty range.
 int select_grid(const StepParams& P, int max_resident) {
   if (P.n_ret <= 0) return P.n_slices < max_resident ? P.n_slices : max_resident;
   const long long groups = (long long)P.B * P.n_ret * (((long long)P.Lcap + 15) / 16);
-  long long want = (long long)P.B * P.n_ret * P.n_chunks;
-  if (want < P.n_slices) want = P.n_slices;
-  if (2 * want >= max_resident) want = max_resident;
+  long long want = max_resident;
   if (want > groups) want = groups;
   if (want < 1) want = 1;
   return (int)want;
