@@ -17,7 +17,8 @@ Sources (page title, section):
          §2 low-dimensional token indexing: a 16-dim projector applied to query and
             key features before RoPE is injected; relevance is estimated there;
          §3 dynamic top-p: attention mass in the low-dim space is accumulated until
-            the cumulative threshold p is reached;
+            the cumulative threshold p is reached (contrasted there with a fixed
+            top-k budget, built here as the selector variant ``top_k``);
          §5 hardware-aware kernels (histogram thresholding, sparse decode).
   [HGA]  "Hierarchical Global Attention" summary, Central mechanism §4: exact
          token attention, plain softmax over the bounded selected set.
@@ -32,6 +33,8 @@ Readings where the pages are silent (each is listed in the design notes):
   * tokens are ordered by (probability desc, position asc); token j is kept
     iff the running mass *before* it is < p ("until p is reached"), so the
     kept set is the shortest prefix whose mass is >= p; p >= 1 keeps all;
+  * the top-k variant keeps the first k tokens of that same order (all L when
+    k >= L), over all L tokens like top-p, sinks and window attended anyway;
   * sinks = positions [0, n_sink), window = the last ``window`` positions
     (the current token included); both are always attended, the union
     de-duplicated;
@@ -192,6 +195,24 @@ def top_p(pi: np.ndarray, p: float) -> TopP:
     return TopP(kept=kept, order=order, c_before=c_before)
 
 
+def top_k(pi: np.ndarray, k: int) -> TopP:
+    """The first k tokens of the (pi desc, position asc) order (all L when k >= L).
+
+    A fixed budget in place of the mass threshold of ``top_p``; ``c_before`` is
+    still the running mass before each position in that order.
+    """
+    pi = np.asarray(pi, np.float64)
+    L = pi.shape[0]
+    pos = np.arange(L)
+    order = np.lexsort((pos, -pi))
+    run = np.cumsum(pi[order])
+    before_sorted = np.concatenate([[0.0], run[:-1]])
+    c_before = np.empty(L, np.float64)
+    c_before[order] = before_sorted
+    kept = pos.copy() if k >= L else np.sort(order[:max(int(k), 0)])
+    return TopP(kept=kept, order=order, c_before=c_before)
+
+
 def sink_window(L: int, n_sink: int, window: int) -> np.ndarray:
     """Positions always attended: [0, n_sink) union [L - window, L), clipped to [0, L)."""
     s = set(range(min(max(n_sink, 0), L)))
@@ -227,8 +248,10 @@ class SliceResult:
 
 def decode(q_pre, k_cache, v_cache, idx_cache, head_mask, seq_lens, p, n_sink, window,
            P_q, rope_theta, idx_scale, *, to_f64=None, slices=None,
-           attend_sets: Optional[Dict[Tuple[int, int], np.ndarray]] = None):
+           attend_sets: Optional[Dict[Tuple[int, int], np.ndarray]] = None, k: Optional[int] = None):
     """One decode step for every (b, kv head) in ``slices`` (default: all).
+
+    Retrieval heads select by top-p (``p``), or by top-k when ``k`` is given.
 
     Array arguments hold storage values; ``to_f64`` maps a storage array to its
     exact float64 values (bf16 bits -> values, or identity for float32).
@@ -257,7 +280,7 @@ def decode(q_pre, k_cache, v_cache, idx_cache, head_mask, seq_lens, p, n_sink, w
         if retrieval:
             idx = bf16_bits_to_f64(idx_cache[b, g, :L])
             pi, _ = index_probs(qp, np.asarray(P_q, np.float64)[heads], idx, idx_scale)
-            tp = top_p(pi, p)
+            tp = top_p(pi, p) if k is None else top_k(pi, k)
             sr.topp, sr.pi = tp, pi
             listed = np.setdiff1d(tp.kept, base)
             if attend_sets is not None and (b, g) in attend_sets:
@@ -273,7 +296,7 @@ def decode(q_pre, k_cache, v_cache, idx_cache, head_mask, seq_lens, p, n_sink, w
 
 
 def decode_inputs(inp, *, slices=None, attend_sets=None, p=None, n_sink=None, window=None,
-                  idx_cache=None):
+                  idx_cache=None, k=None):
     """``decode`` on a ``synth.Inputs`` bundle (index cache built by ``index_append``)."""
     to_f64 = (lambda a: bf16_bits_to_f64(a)) if inp.dtype == "bf16" else (lambda a: np.asarray(a, np.float64))
     if idx_cache is None:
@@ -283,7 +306,7 @@ def decode_inputs(inp, *, slices=None, attend_sets=None, p=None, n_sink=None, wi
                   inp.n_sink if n_sink is None else n_sink,
                   inp.window if window is None else window,
                   inp.P_q, inp.rope_theta, inp.idx_scale, to_f64=to_f64, slices=slices,
-                  attend_sets=attend_sets)
+                  attend_sets=attend_sets, k=k)
 
 
 def index_cache_for(inp, heads: Optional[List[int]] = None, precision: str = "f32") -> np.ndarray:

@@ -215,6 +215,58 @@ def test_top_p_p_one_keeps_all():
 
 
 # ---------------------------------------------------------------- sink/window
+# ---------------------------------------------------------------- top-k
+def test_top_k_golden_cases():
+    n = 0
+    for k, masses, kept in _rows("top_k_cases.txt"):
+        pi = np.array([float(m) for m in masses.split()])
+        want = [int(x) for x in kept.split()]
+        assert list(O.top_k(pi, int(k)).kept) == want, (k, masses)
+        n += 1
+    assert n >= 13
+
+
+def test_top_k_is_the_heaviest_k_subset_with_lowest_positions_on_ties():
+    rng = np.random.default_rng(16)
+    for trial in range(300):
+        L = int(rng.integers(1, 10))
+        pi = np.round(rng.random(L) * 8) / 8      # coarse values: many exact ties
+        k = int(rng.integers(1, L + 2))
+        got = list(O.top_k(pi, k).kept)
+        if k >= L:
+            assert got == list(range(L))
+            continue
+        # brute force over every k-subset: the largest mass, then the smallest
+        # ascending position tuple among subsets of that mass
+        best = None
+        for c in itertools.combinations(range(L), k):
+            key = (-pi[list(c)].sum(), c)
+            if best is None or key < best:
+                best = key
+        assert got == list(best[1]), (pi, k)
+
+
+def test_top_k_with_the_top_p_count_is_the_top_p_set():
+    rng = np.random.default_rng(17)
+    for _ in range(100):
+        L = int(rng.integers(20, 300))
+        pi = rng.lognormal(0, 2, L)
+        pi /= pi.sum()
+        for p in (0.5, 0.9, 0.99):
+            tp = O.top_p(pi, p).kept
+            assert np.array_equal(O.top_k(pi, len(tp)).kept, tp)
+
+
+def test_decode_top_k_covering_context_equals_dense_for_retrieval_heads():
+    inp = synth.make_inputs("tiny", 0, overrides={"L": 300, "window": 16})
+    dense, _ = O.decode_inputs(inp, p=1.0)
+    out, res = O.decode_inputs(inp, k=300)
+    r = [g for g in range(inp.Hkv) if inp.head_mask[g]]
+    for g in r:
+        assert len(res[(0, g)].listed) == 300 - len(O.sink_window(300, inp.n_sink, 16))
+    np.testing.assert_allclose(out, dense, rtol=0, atol=1e-12)
+
+
 def test_sink_window_golden():
     for L, ns, w, pos in _rows("sink_window_cases.txt"):
         assert list(O.sink_window(int(L), int(ns), int(w))) == [int(x) for x in pos.split()]
