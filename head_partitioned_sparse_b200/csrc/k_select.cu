@@ -145,6 +145,12 @@ __device__ __forceinline__ void hist_desc(unsigned long long* stage, const unsig
   __syncthreads();
 }
 
+// Mass of a token in the radix select: its quantised probability for top-p, 1 for
+// top-k (the same select then counts tokens, and the target is k).
+__device__ __forceinline__ unsigned long long sel_mass(const StepParams& P, unsigned bits) {
+  return P.topk > 0 ? 1ull : mass_q(bits);
+}
+
 // ------------------------------------------------------------------ index scores
 // Scores of 16 tokens at a time on the tensor cores (mma.sync m16n8k16, bf16 in,
 // float32 accumulate): A = the 16 tokens' bf16 index rows (16 x 16 dims), B = the
@@ -727,9 +733,10 @@ __device__ void cut1_slice(const StepParams& P, SmemStage& sm, SelScalars& sc, i
   unsigned long long target = total;
   bool keep_all = P.keep_all || total == 0ull;
   if (!keep_all) {
-    target = (unsigned long long)ceil((double)P.p * (double)total);
+    // top-k: the k-th token (total = the number of tokens); top-p: the mass ceil(p total)
+    target = P.topk > 0 ? (unsigned long long)P.topk : (unsigned long long)ceil((double)P.p * (double)total);
     if (target < 1ull) target = 1ull;
-    keep_all = target > total;   // cannot happen for p < 1; keep everything if it does
+    keep_all = target >= total && P.topk > 0 ? true : target > total;   // k >= L keeps all
   }
   if (tid == 0) sc.cut_bin = -1;
   __syncthreads();
@@ -856,7 +863,8 @@ __device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
   __syncthreads();
   unsigned long long* g1 = P.ws.hist1 + (size_t)un.s * kBins1;
   for (int i = tid; i < kBins1; i += kSelThreads)
-    if (sm.cnt[i]) atomicAdd(g1 + i, bin1_mass((unsigned)i, sm.cnt[i], sm.low[i]));
+    if (sm.cnt[i])
+      atomicAdd(g1 + i, P.topk > 0 ? (unsigned long long)sm.cnt[i] : bin1_mass((unsigned)i, sm.cnt[i], sm.low[i]));
   __syncthreads();   // the histogram is reused by the next range
 }
 
@@ -947,7 +955,7 @@ __device__ void threshold_unit(const StepParams& P, SelScalars& sc, int y, int c
       for (int i = 0; i < kTokPerThread; ++i) {
         if ((cflags >> i) & 1u) {
           cand[base + __popc(masks[i] & lt)] = make_uint2(bits[i], (unsigned)(j0 + tid + kSelThreads * i));
-          atomicAdd(&h2[(bits[i] >> 6) & 0xfffu], mass_q(bits[i]));
+          atomicAdd(&h2[(bits[i] >> 6) & 0xfffu], sel_mass(P, bits[i]));
         }
         base += __popc(masks[i]);
       }
@@ -1007,7 +1015,7 @@ __device__ void refine_slice(const StepParams& P, SelSmem& smu, SelScalars& sc, 
       if (d2 > cb2) {
         if (!sw.always(pos)) atomicAdd(&chunk_sel[pos / kChunk], 1);
       } else if (d2 == cb2) {
-        atomicAdd(&sm.m3[bits & 63u], mass_q(bits));
+        atomicAdd(&sm.m3[bits & 63u], sel_mass(P, bits));
         atomicAdd(&sm.c3[bits & 63u], 1u);
         const unsigned slot = atomicAdd(&sc.small_n, 1u);
         if (slot < kSmallCap) small[slot] = make_uint2(bits, (unsigned)pos);
@@ -1044,7 +1052,7 @@ __device__ void refine_slice(const StepParams& P, SelSmem& smu, SelScalars& sc, 
       tau = ((unsigned)b1 << 18) | ((unsigned)cb2 << 6) | (unsigned)sc.b3;
       const unsigned long long m_gt = sc.above2;
       const unsigned n_eq = sm.c3[sc.b3];
-      const unsigned long long q_tau = mass_q(tau);
+      const unsigned long long q_tau = sel_mass(P, tau);
       const unsigned long long need =
           (q_tau > 0ull && target > m_gt) ? (target - m_gt + q_tau - 1ull) / q_tau : ~0ull;
       if (need < (unsigned long long)n_eq) {

@@ -166,6 +166,7 @@ struct StepArgs {
   int64_t max_seq_len;
   float p;
   int n_sink, window;
+  int64_t k;   // > 0: top-k selection with budget k (p unused)
 };
 
 spa_status check_step(spa_ctx* h, const StepArgs& a, spa::StepParams* P) {
@@ -176,7 +177,9 @@ spa_status check_step(spa_ctx* h, const StepArgs& a, spa::StepParams* P) {
     return fail(SPA_ERR_INVALID_ARG, "q_pre/idx_cache must be 16-byte aligned, seq_lens 8-byte aligned");
   if (a.B < 1 || a.B > h->cfg.max_batch)
     return fail(SPA_ERR_INVALID_ARG, "B must be in [1, max_batch=%d] (got %d)", h->cfg.max_batch, a.B);
-  if (!(a.p > 0.f) || !(a.p <= 1.f)) return fail(SPA_ERR_INVALID_ARG, "p must be in (0, 1] (got %g)", (double)a.p);
+  if (a.k < 0) return fail(SPA_ERR_INVALID_ARG, "k must be >= 1 (got %lld)", (long long)a.k);
+  if (a.k == 0 && (!(a.p > 0.f) || !(a.p <= 1.f)))
+    return fail(SPA_ERR_INVALID_ARG, "p must be in (0, 1] (got %g)", (double)a.p);
   if (a.n_sink < 0 || a.window < 0) return fail(SPA_ERR_INVALID_ARG, "n_sink and window must be >= 0");
   if ((int64_t)a.n_sink + a.window < 1)
     return fail(SPA_ERR_INVALID_ARG, "n_sink + window must be >= 1 (a streaming head needs a token)");
@@ -200,8 +203,9 @@ spa_status check_step(spa_ctx* h, const StepArgs& a, spa::StepParams* P) {
   P->Lcap = (int)(a.max_seq_len ? a.max_seq_len : h->cfg.max_ctx);
   P->n_chunks = (P->Lcap + spa::kChunk - 1) / spa::kChunk;
   P->n_slices = a.B * Hkv;
-  P->p = a.p;
-  P->keep_all = a.p >= 1.f ? 1 : 0;
+  P->p = a.k > 0 ? 1.f : a.p;
+  P->keep_all = a.k == 0 && a.p >= 1.f ? 1 : 0;
+  P->topk = a.k;
   P->n_sink = a.n_sink;
   P->window = a.window;
   P->idx_scale_log2 = h->idx_scale * 1.4426950408889634f;
@@ -215,6 +219,46 @@ spa_status run_selection(spa_ctx* h, spa::StepParams& P, cudaStream_t st) {
   const int grid = spa::select_grid(P, h->select_max_grid);
   return run(h, SPA_K_SELECT, st, "select", [&] { return spa::launch_select(P, h->cfg.kv_dtype, grid, st); });
 }
+
+spa_status select_with(spa_ctx* h, spa::StepParams& P, int32_t* sel_idx, int32_t* sel_count, spa_stream stream) {
+  if (!sel_idx || !sel_count) return fail(SPA_ERR_INVALID_ARG, "sel_idx and sel_count must be non-NULL");
+  if (!aligned16(sel_idx) || ((uintptr_t)sel_count & 3u))
+    return fail(SPA_ERR_INVALID_ARG, "sel_idx must be 16-byte aligned, sel_count 4-byte aligned");
+  P.sel_list = sel_idx;
+  P.sel_count = sel_count;
+  return run_selection(h, P, reinterpret_cast<cudaStream_t>(stream));
+}
+
+
+spa_status decode_with(spa_ctx* h, spa::StepParams& P, const void* k_cache, const void* v_cache, float* out,
+                       int32_t* sel_count_opt, spa_stream stream) {
+  spa_status r = SPA_OK;
+  if (!k_cache || !v_cache || !out) return fail(SPA_ERR_INVALID_ARG, "k_cache, v_cache and out must be non-NULL");
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return fail(SPA_ERR_INVALID_ARG, "k_cache, v_cache and out must be 16-byte aligned");
+  if (sel_count_opt && ((uintptr_t)sel_count_opt & 3u)) return fail(SPA_ERR_INVALID_ARG, "sel_count_opt misaligned");
+  P.k_cache = k_cache;
+  P.v_cache = v_cache;
+  P.out = out;
+  P.sel_list = h->ws.list;
+  P.sel_count = nullptr;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if ((r = run_selection(h, P, st))) return r;
+  // upper bound on splits: every slice has at most Lcap rows
+  const int64_t per_slice = (P.Lcap + P.split_rows - 1) / P.split_rows;
+  const int64_t max_items = per_slice * P.n_slices;
+  int64_t cap = (int64_t)h->num_sms * h->attend_occ;
+  if (cap > spa::kMaxAttendCtas) cap = spa::kMaxAttendCtas;
+  const int grid = (int)(max_items < cap ? max_items : cap);
+  // bf16 caches: the attention kernel combines the splits and reports the counts itself
+  if (h->cfg.kv_dtype == 0) P.sel_count = sel_count_opt;
+  if ((r = run(h, SPA_K_ATTEND, st, "attend", [&] { return spa::launch_attend(P, h->cfg.kv_dtype, grid, st); })))
+    return r;
+  if (h->cfg.kv_dtype == 0) return SPA_OK;
+  P.sel_count = sel_count_opt;
+  return run(h, SPA_K_COMBINE, st, "combine", [&] { return spa::launch_combine(P, st); });
+}
+
 
 }  // namespace
 
@@ -350,14 +394,19 @@ spa_status spa_select(spa_handle h, const void* q_pre, const void* idx_cache, co
                       const int64_t* seq_lens, int B, int64_t max_seq_len, float p, int n_sink, int window,
                       int32_t* sel_idx, int32_t* sel_count, spa_stream stream) {
   spa::StepParams P;
-  spa_status r = check_step(h, StepArgs{q_pre, idx_cache, head_mask, seq_lens, B, max_seq_len, p, n_sink, window}, &P);
+  spa_status r = check_step(h, StepArgs{q_pre, idx_cache, head_mask, seq_lens, B, max_seq_len, p, n_sink, window, 0}, &P);
   if (r) return r;
-  if (!sel_idx || !sel_count) return fail(SPA_ERR_INVALID_ARG, "sel_idx and sel_count must be non-NULL");
-  if (!aligned16(sel_idx) || ((uintptr_t)sel_count & 3u))
-    return fail(SPA_ERR_INVALID_ARG, "sel_idx must be 16-byte aligned, sel_count 4-byte aligned");
-  P.sel_list = sel_idx;
-  P.sel_count = sel_count;
-  return run_selection(h, P, reinterpret_cast<cudaStream_t>(stream));
+  return select_with(h, P, sel_idx, sel_count, stream);
+}
+
+spa_status spa_select_topk(spa_handle h, const void* q_pre, const void* idx_cache, const uint8_t* head_mask,
+                           const int64_t* seq_lens, int B, int64_t max_seq_len, int64_t k, int n_sink, int window,
+                           int32_t* sel_idx, int32_t* sel_count, spa_stream stream) {
+  spa::StepParams P;
+  if (k < 1) return fail(SPA_ERR_INVALID_ARG, "k must be >= 1 (got %lld)", (long long)k);
+  spa_status r = check_step(h, StepArgs{q_pre, idx_cache, head_mask, seq_lens, B, max_seq_len, 1.f, n_sink, window, k}, &P);
+  if (r) return r;
+  return select_with(h, P, sel_idx, sel_count, stream);
 }
 
 spa_status spa_decode(spa_handle h, const void* q_pre, const void* k_cache, const void* v_cache,
@@ -365,32 +414,20 @@ spa_status spa_decode(spa_handle h, const void* q_pre, const void* k_cache, cons
                       int64_t max_seq_len, float p, int n_sink, int window, float* out, int32_t* sel_count_opt,
                       spa_stream stream) {
   spa::StepParams P;
-  spa_status r = check_step(h, StepArgs{q_pre, idx_cache, head_mask, seq_lens, B, max_seq_len, p, n_sink, window}, &P);
+  spa_status r = check_step(h, StepArgs{q_pre, idx_cache, head_mask, seq_lens, B, max_seq_len, p, n_sink, window, 0}, &P);
   if (r) return r;
-  if (!k_cache || !v_cache || !out) return fail(SPA_ERR_INVALID_ARG, "k_cache, v_cache and out must be non-NULL");
-  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
-    return fail(SPA_ERR_INVALID_ARG, "k_cache, v_cache and out must be 16-byte aligned");
-  if (sel_count_opt && ((uintptr_t)sel_count_opt & 3u)) return fail(SPA_ERR_INVALID_ARG, "sel_count_opt misaligned");
-  P.k_cache = k_cache;
-  P.v_cache = v_cache;
-  P.out = out;
-  P.sel_list = h->ws.list;
-  P.sel_count = nullptr;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if ((r = run_selection(h, P, st))) return r;
-  // upper bound on splits: every slice has at most Lcap rows
-  const int64_t per_slice = (P.Lcap + P.split_rows - 1) / P.split_rows;
-  const int64_t max_items = per_slice * P.n_slices;
-  int64_t cap = (int64_t)h->num_sms * h->attend_occ;
-  if (cap > spa::kMaxAttendCtas) cap = spa::kMaxAttendCtas;
-  const int grid = (int)(max_items < cap ? max_items : cap);
-  // bf16 caches: the attention kernel combines the splits and reports the counts itself
-  if (h->cfg.kv_dtype == 0) P.sel_count = sel_count_opt;
-  if ((r = run(h, SPA_K_ATTEND, st, "attend", [&] { return spa::launch_attend(P, h->cfg.kv_dtype, grid, st); })))
-    return r;
-  if (h->cfg.kv_dtype == 0) return SPA_OK;
-  P.sel_count = sel_count_opt;
-  return run(h, SPA_K_COMBINE, st, "combine", [&] { return spa::launch_combine(P, st); });
+  return decode_with(h, P, k_cache, v_cache, out, sel_count_opt, stream);
+}
+
+spa_status spa_decode_topk(spa_handle h, const void* q_pre, const void* k_cache, const void* v_cache,
+                           const void* idx_cache, const uint8_t* head_mask, const int64_t* seq_lens, int B,
+                           int64_t max_seq_len, int64_t k, int n_sink, int window, float* out, int32_t* sel_count_opt,
+                           spa_stream stream) {
+  spa::StepParams P;
+  if (k < 1) return fail(SPA_ERR_INVALID_ARG, "k must be >= 1 (got %lld)", (long long)k);
+  spa_status r = check_step(h, StepArgs{q_pre, idx_cache, head_mask, seq_lens, B, max_seq_len, 1.f, n_sink, window, k}, &P);
+  if (r) return r;
+  return decode_with(h, P, k_cache, v_cache, out, sel_count_opt, stream);
 }
 
 spa_status spa_device_status(spa_handle h, spa_stream stream) {

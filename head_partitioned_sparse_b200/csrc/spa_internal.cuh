@@ -115,6 +115,7 @@ struct StepParams {
   int n_slices;          // B * Hkv
   float p;
   int keep_all;          // p >= 1
+  int64_t topk;          // > 0: keep the topk highest-probability tokens instead of top-p
   int n_sink, window;
   float idx_scale_log2;  // idx_scale * log2(e)
   float attn_scale_log2; // log2(e) / sqrt(128)

@@ -161,11 +161,30 @@ SPA_API spa_status spa_select(spa_handle h, const void* q_pre, const void* idx_c
  *   out             device float32 [B][Hq][128], written
  *   sel_count_opt   NULL, or device int32 [B * Hkv] receiving the selected counts
  * Attention is split over rows (split-K), each split keeping an online-softmax
- * state (m, l, acc) that a combine kernel merges with log-sum-exp weights.
+ * state (m, l, acc) merged with log-sum-exp weights (inside the attention kernel
+ * for bf16 caches, by a combine kernel for float32 caches).
  */
 SPA_API spa_status spa_decode(spa_handle h, const void* q_pre, const void* k_cache, const void* v_cache,
                       const void* idx_cache, const uint8_t* head_mask, const int64_t* seq_lens,
                       int B, int64_t max_seq_len, float p, int n_sink, int window,
+                      float* out, int32_t* sel_count_opt, spa_stream stream);
+
+/*
+ * Top-k selector variant: the fixed budget that "Full Attention Strikes Back"
+ * (RTPurbo summary), Methodology §3, contrasts with dynamic top-p.  T keeps the
+ * first k tokens of the (pi desc, position asc) order over all L tokens (every
+ * token when k >= L); sinks and window are attended anyway and the lists exclude
+ * them, as for top-p.  Every other argument, output and error is that of
+ * spa_select / spa_decode; k must be >= 1 (else SPA_ERR_INVALID_ARG).  The same
+ * exact radix select runs with every token's mass set to 1 and the target k.
+ */
+SPA_API spa_status spa_select_topk(spa_handle h, const void* q_pre, const void* idx_cache,
+                      const uint8_t* head_mask, const int64_t* seq_lens, int B, int64_t max_seq_len,
+                      int64_t k, int n_sink, int window, int32_t* sel_idx, int32_t* sel_count,
+                      spa_stream stream);
+SPA_API spa_status spa_decode_topk(spa_handle h, const void* q_pre, const void* k_cache, const void* v_cache,
+                      const void* idx_cache, const uint8_t* head_mask, const int64_t* seq_lens,
+                      int B, int64_t max_seq_len, int64_t k, int n_sink, int window,
                       float* out, int32_t* sel_count_opt, spa_stream stream);
 
 /*
