@@ -56,6 +56,7 @@ def parse_args():
     ap.add_argument("--no-sweep", action="store_true", help="skip the per-p sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-topk-sweep", action="store_true", help="skip the top-k selector measurements")
     ap.add_argument("--override", action="append", default=[], metavar="KEY=VALUE",
                     help="replace a workload field (e.g. B=1 for a small profiling case)")
     return ap.parse_args()
@@ -338,6 +339,27 @@ def main_native(args):
                                 "achieved_gbs": abw["total"] / (msw * 1e-3) / 1e9,
                                 "selected_rows": abw["selected_rows"]}
 
+    # top-k selector variant (same measurement, smaller step count)
+    topk_sweep = {}
+    if not args.no_topk_sweep:
+        for kk in (2048, 16384, 65536):
+            def step_k(i, kk=kk):
+                kc, vc, ixc = layers[i % len(layers)]
+                B.spa_decode_topk(h, q, kc, vc, ixc, head_mask, lens, inp.B, Lcap, kk, inp.n_sink, inp.window,
+                                  out, None, stream)
+            for i in range(3):
+                step_k(i)
+            n = max(10, args.steps // 4)
+            msk, _ = timed(n, step_k)
+            msk = shard.reduce_max(msk, dev) / n
+            B.spa_decode_topk(h, q, layers[0][0], layers[0][1], layers[0][2], head_mask, lens, inp.B, Lcap, kk,
+                              inp.n_sink, inp.window, out, cnt, stream)
+            torch.cuda.synchronize(dev)
+            abk = algorithmic_bytes(inp, cnt.cpu().numpy(), s_kv)
+            topk_sweep[str(kk)] = {"ms_per_step": msk, "layer_steps_per_s": world * 1e3 / msk,
+                                   "achieved_gbs": abk["total"] / (msk * 1e-3) / 1e9,
+                                   "selected_rows": abk["selected_rows"]}
+
     # end to end through the public API: pinned host inputs in, result out, every step
     e2e = None
     if not args.no_e2e:
@@ -417,6 +439,7 @@ def main_native(args):
             "gpu_launches": int(launches),
             "clocks": clk,
             "p_sweep": sweep or None,
+            "topk_sweep": topk_sweep or None,
         }
         print(json.dumps(line), flush=True)
     B.spa_destroy(h)
