@@ -8,30 +8,35 @@
 // Group mean of per-head probabilities: "Autonomy of Heads" summary, Deployment
 // strategy (GQA scores aggregated to the group by their mean).
 //
-// Phases, separated by grid-wide barriers (units: retrieval slices s = (b, g) and
-// their chunks of kChunk tokens; CTAs take units in grid-stride order):
-//   prologue  q_rot = RoPE(q_pre, L-1) for every head (angles in float64, reduced
-//             exactly in units of pi), q_idx = P_q q_pre (float64 dot products),
-//             reset of each retrieval slice's selection state;
-//   score     per chunk and head h: m = max_j l_hj, z = sum_j 2^(l_hj - m),
+// Phases (units: retrieval slices s = (b, g); the score and mass phases split the
+// slices' 16-token groups into equal ranges per CTA, the later phases work on chunks of
+// kChunk tokens):
+//   score     the leader CTA of each slice computes q_idx = P_q q_pre (float64 dot
+//             products) and publishes it (flag); every range then forms, per head h,
+//             m = max_j l_hj, z = sum_j 2^(l_hj - m),
 //             l_hj = log2(e) * idx_scale * <q_idx[h], idx_j>   (index read #1);
-//   mass      merge (m, z) over chunks -> M_h, Z_h; recompute l_hj (index read #2),
+//   -- grid barrier --
+//   mass      merge (m, z) over ranges -> M_h, Z_h; recompute l_hj (index read #2),
 //             pi_j = sum_h 2^(l_hj - M_h) / (G Z_h), stored as fp32; a mass histogram
 //             over the top 12 bits of pi_j's bit pattern, masses quantised to integer
-//             multiples of 2^-63 so every sum is exact and order independent (per chunk
+//             multiples of 2^-63 so every sum is exact and order independent (per range
 //             as a count and a sum of low significand bits per bin, 32-bit atomics);
-//   cut 1     per slice: total mass, target ceil(p * total) and the bin b1 where the
-//             descending cumulative mass reaches it;
+//   cut 1     per slice (last range, ticket): total mass, target ceil(p * total) (or k
+//             for top-k) and the bin b1 where the descending cumulative mass reaches it;
+//   -- grid barrier --
 //   threshold per chunk: tokens above b1 counted, tokens of bin b1 appended as
 //             candidates with their round-2 masses added to the slice histogram;
-//   refine    per slice: round-2 bin b2 from the histogram, one pass over the
-//             candidates for round 3 (exact cut value tau), the tie quota at tau
-//             (lowest positions first) and per-chunk output offsets;
+//   refine    per slice (last chunk, ticket): round-2 bin b2 from the histogram, one
+//             pass over the candidates for round 3 (exact cut value tau), the tie quota
+//             at tau (lowest positions first) and per-chunk output offsets; idle CTAs
+//             compute q_rot = RoPE(q_pre, L-1) for every head as duties (angles in
+//             float64, reduced exactly in units of pi);
+//   -- grid barrier --
 //   compact   per chunk: kept positions outside sinks/window, ascending.
 // One launch replaces a chain of small kernels whose fixed launch cost dominated.
-// Grid barriers spin on a generation word with a clock budget; on timeout they set a
-// device status bit and every CTA leaves the kernel.  The launch is cooperative, so
-// all CTAs are resident together.
+// Grid barriers and the q_idx flags are polled with a clock budget; on timeout they set
+// a device status bit and the kernel leaves or carries on without hanging.  The launch
+// is cooperative, so all CTAs are resident together.
 #include <climits>
 
 #include "spa_internal.cuh"
