@@ -35,6 +35,10 @@ Readings where the pages are silent (each is listed in the design notes):
     kept set is the shortest prefix whose mass is >= p; p >= 1 keeps all;
   * the top-k variant keeps the first k tokens of that same order (all L when
     k >= L), over all L tokens like top-p, sinks and window attended anyway;
+  * the block-granular variant scores blocks of 64 consecutive positions by
+    their mass (the sum of their tokens' probabilities), orders blocks by (mass
+    desc, block index asc), keeps a block iff the running mass before it is < p,
+    and keeps every token of a kept block ([HGA] routes chunks, not tokens);
   * sinks = positions [0, n_sink), window = the last ``window`` positions
     (the current token included); both are always attended, the union
     de-duplicated;
@@ -213,6 +217,35 @@ def top_k(pi: np.ndarray, k: int) -> TopP:
     return TopP(kept=kept, order=order, c_before=c_before)
 
 
+BLOCK = 64
+
+
+def block_top_p(pi: np.ndarray, p: float, block: int = BLOCK) -> TopP:
+    """Top-p over blocks of ``block`` consecutive positions, whole blocks kept.
+
+    Block b covers positions [b block, min((b + 1) block, L)); its mass is the sum
+    of its tokens' probabilities.  Blocks are ordered by (mass desc, block index
+    asc) and a block is kept iff the running mass before it is < p (p >= 1 keeps
+    all).  ``c_before`` gives, for every position, the running mass before its
+    block; ``order`` lists the blocks in that order.
+    """
+    pi = np.asarray(pi, np.float64)
+    L = pi.shape[0]
+    nb = (L + block - 1) // block
+    bmass = np.array([pi[b * block:(b + 1) * block].sum() for b in range(nb)])
+    bidx = np.arange(nb)
+    order = np.lexsort((bidx, -bmass))
+    run = np.cumsum(bmass[order])
+    before_sorted = np.concatenate([[0.0], run[:-1]])
+    b_before = np.empty(nb, np.float64)
+    b_before[order] = before_sorted
+    kept_blocks = bidx if p >= 1.0 else np.sort(order[before_sorted < p])
+    kept = np.concatenate([np.arange(b * block, min((b + 1) * block, L)) for b in kept_blocks]) \
+        if len(kept_blocks) else np.zeros(0, np.int64)
+    c_before = np.repeat(b_before, block)[:L]
+    return TopP(kept=kept.astype(np.int64), order=order, c_before=c_before)
+
+
 def sink_window(L: int, n_sink: int, window: int) -> np.ndarray:
     """Positions always attended: [0, n_sink) union [L - window, L), clipped to [0, L)."""
     s = set(range(min(max(n_sink, 0), L)))
@@ -248,10 +281,12 @@ class SliceResult:
 
 def decode(q_pre, k_cache, v_cache, idx_cache, head_mask, seq_lens, p, n_sink, window,
            P_q, rope_theta, idx_scale, *, to_f64=None, slices=None,
-           attend_sets: Optional[Dict[Tuple[int, int], np.ndarray]] = None, k: Optional[int] = None):
+           attend_sets: Optional[Dict[Tuple[int, int], np.ndarray]] = None, k: Optional[int] = None,
+           blocks: bool = False):
     """One decode step for every (b, kv head) in ``slices`` (default: all).
 
-    Retrieval heads select by top-p (``p``), or by top-k when ``k`` is given.
+    Retrieval heads select by top-p (``p``), by top-k when ``k`` is given, or by
+    block-granular top-p when ``blocks`` is set.
 
     Array arguments hold storage values; ``to_f64`` maps a storage array to its
     exact float64 values (bf16 bits -> values, or identity for float32).
@@ -280,7 +315,7 @@ def decode(q_pre, k_cache, v_cache, idx_cache, head_mask, seq_lens, p, n_sink, w
         if retrieval:
             idx = bf16_bits_to_f64(idx_cache[b, g, :L])
             pi, _ = index_probs(qp, np.asarray(P_q, np.float64)[heads], idx, idx_scale)
-            tp = top_p(pi, p) if k is None else top_k(pi, k)
+            tp = block_top_p(pi, p) if blocks else (top_p(pi, p) if k is None else top_k(pi, k))
             sr.topp, sr.pi = tp, pi
             listed = np.setdiff1d(tp.kept, base)
             if attend_sets is not None and (b, g) in attend_sets:
@@ -296,7 +331,7 @@ def decode(q_pre, k_cache, v_cache, idx_cache, head_mask, seq_lens, p, n_sink, w
 
 
 def decode_inputs(inp, *, slices=None, attend_sets=None, p=None, n_sink=None, window=None,
-                  idx_cache=None, k=None):
+                  idx_cache=None, k=None, blocks=False):
     """``decode`` on a ``synth.Inputs`` bundle (index cache built by ``index_append``)."""
     to_f64 = (lambda a: bf16_bits_to_f64(a)) if inp.dtype == "bf16" else (lambda a: np.asarray(a, np.float64))
     if idx_cache is None:
@@ -306,7 +341,7 @@ def decode_inputs(inp, *, slices=None, attend_sets=None, p=None, n_sink=None, wi
                   inp.n_sink if n_sink is None else n_sink,
                   inp.window if window is None else window,
                   inp.P_q, inp.rope_theta, inp.idx_scale, to_f64=to_f64, slices=slices,
-                  attend_sets=attend_sets, k=k)
+                  attend_sets=attend_sets, k=k, blocks=blocks)
 
 
 def index_cache_for(inp, heads: Optional[List[int]] = None, precision: str = "f32") -> np.ndarray:

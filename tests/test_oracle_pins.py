@@ -267,6 +267,62 @@ def test_decode_top_k_covering_context_equals_dense_for_retrieval_heads():
     np.testing.assert_allclose(out, dense, rtol=0, atol=1e-12)
 
 
+# ---------------------------------------------------------------- block-granular top-p
+def test_block_top_p_golden_cases():
+    n = 0
+    for p, blk, masses, kept in _rows("block_top_p_cases.txt"):
+        pi = np.array([float(m) for m in masses.split()])
+        want = [int(x) for x in kept.split()]
+        assert list(O.block_top_p(pi, float(p), int(blk)).kept) == want, (p, blk, masses)
+        n += 1
+    assert n >= 12
+
+
+def test_block_top_p_with_unit_blocks_is_top_p():
+    rng = np.random.default_rng(18)
+    for _ in range(100):
+        L = int(rng.integers(1, 200))
+        pi = rng.lognormal(0, 2, L)
+        pi /= pi.sum()
+        for p in (0.3, 0.9, 0.99, 1.0):
+            assert np.array_equal(O.block_top_p(pi, p, 1).kept, O.top_p(pi, p).kept)
+
+
+def test_block_top_p_matches_brute_force_over_blocks():
+    rng = np.random.default_rng(19)
+    for trial in range(200):
+        blk = int(rng.integers(2, 6))
+        L = int(rng.integers(1, 8 * blk))
+        pi = rng.random(L) ** 3
+        pi /= pi.sum()
+        p = float(rng.choice([0.3, 0.6, 0.9, 0.99]))
+        got = O.block_top_p(pi, p, blk).kept
+        nb = (L + blk - 1) // blk
+        mass = [pi[b * blk:(b + 1) * blk].sum() for b in range(nb)]
+        best = None   # fewest blocks reaching p, then the largest mass
+        for r in range(1, nb + 1):
+            ok = [c for c in itertools.combinations(range(nb), r) if sum(mass[b] for b in c) >= p]
+            if ok:
+                best = (r, max(sum(mass[b] for b in c) for c in ok))
+                break
+        if best is None:          # rounding left the total below p: everything is kept
+            assert len(got) == L
+            continue
+        kept_blocks = sorted({int(j) // blk for j in got})
+        assert len(kept_blocks) == best[0]
+        assert sum(mass[b] for b in kept_blocks) == pytest.approx(best[1], abs=1e-12)
+        # whole blocks only
+        for b in kept_blocks:
+            assert all(j in set(got.tolist()) for j in range(b * blk, min((b + 1) * blk, L)))
+
+
+def test_decode_blocks_p1_equals_dense_for_retrieval_heads():
+    inp = synth.make_inputs("tiny", 0, overrides={"L": 300, "window": 16})
+    dense, _ = O.decode_inputs(inp, p=1.0)
+    out, _ = O.decode_inputs(inp, p=1.0, blocks=True)
+    np.testing.assert_allclose(out, dense, rtol=0, atol=1e-12)
+
+
 def test_sink_window_golden():
     for L, ns, w, pos in _rows("sink_window_cases.txt"):
         assert list(O.sink_window(int(L), int(ns), int(w))) == [int(x) for x in pos.split()]
