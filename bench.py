@@ -57,6 +57,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-topk-sweep", action="store_true", help="skip the top-k selector measurements")
+    ap.add_argument("--no-block-sweep", action="store_true", help="skip the block-granular selector measurements")
     ap.add_argument("--override", action="append", default=[], metavar="KEY=VALUE",
                     help="replace a workload field (e.g. B=1 for a small profiling case)")
     return ap.parse_args()
@@ -360,6 +361,28 @@ def main_native(args):
                                    "achieved_gbs": abk["total"] / (msk * 1e-3) / 1e9,
                                    "selected_rows": abk["selected_rows"]}
 
+    # block-granular top-p variant (64-token blocks; same measurement, smaller step count)
+    block_sweep = {}
+    if not args.no_block_sweep:
+        for pp in (0.9, 0.99):
+            pq = float(np.float32(pp))
+            def step_b(i, pq=pq):
+                kc, vc, ixc = layers[i % len(layers)]
+                B.spa_decode_blocks(h, q, kc, vc, ixc, head_mask, lens, inp.B, Lcap, pq, inp.n_sink, inp.window,
+                                    out, None, stream)
+            for i in range(3):
+                step_b(i)
+            n = max(10, args.steps // 4)
+            msb, _ = timed(n, step_b)
+            msb = shard.reduce_max(msb, dev) / n
+            B.spa_decode_blocks(h, q, layers[0][0], layers[0][1], layers[0][2], head_mask, lens, inp.B, Lcap, pq,
+                                inp.n_sink, inp.window, out, cnt, stream)
+            torch.cuda.synchronize(dev)
+            abb = algorithmic_bytes(inp, cnt.cpu().numpy(), s_kv)
+            block_sweep[f"{pp:g}"] = {"ms_per_step": msb, "layer_steps_per_s": world * 1e3 / msb,
+                                      "achieved_gbs": abb["total"] / (msb * 1e-3) / 1e9,
+                                      "selected_rows": abb["selected_rows"]}
+
     # end to end through the public API: pinned host inputs in, result out, every step
     e2e = None
     if not args.no_e2e:
@@ -440,6 +463,7 @@ def main_native(args):
             "clocks": clk,
             "p_sweep": sweep or None,
             "topk_sweep": topk_sweep or None,
+            "block_sweep": block_sweep or None,
         }
         print(json.dumps(line), flush=True)
     B.spa_destroy(h)

@@ -67,6 +67,8 @@ _SIGS = {
     "spa_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i64, _f, _i, _i, _vp, _vp, _vp]),
     "spa_select_topk": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i64, _i64, _i, _i, _vp, _vp, _vp]),
     "spa_decode_topk": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i64, _i64, _i, _i, _vp, _vp, _vp]),
+    "spa_select_blocks": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i64, _f, _i, _i, _vp, _vp, _vp]),
+    "spa_decode_blocks": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i64, _f, _i, _i, _vp, _vp, _vp]),
     "spa_device_status": (_i, [_vp, _vp]),
     "spa_set_profiling": (_i, [_vp, ctypes.c_uint]),
     "spa_profile_read": (_i, [_vp, _i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
@@ -173,6 +175,20 @@ def spa_decode_topk(h, q_pre, k_cache, v_cache, idx_cache, head_mask, seq_lens, 
     _check(load().spa_decode_topk(h, _ptr(q_pre), _ptr(k_cache), _ptr(v_cache), _ptr(idx_cache),
                                   _host_u8(head_mask), _ptr(seq_lens), B, max_seq_len, int(k), n_sink, window,
                                   _ptr(out), _ptr(sel_count_opt), _stream(stream)))
+
+
+def spa_select_blocks(h, q_pre, idx_cache, head_mask, seq_lens, B: int, max_seq_len: int, p: float, n_sink: int,
+                      window: int, sel_idx, sel_count, stream=None) -> None:
+    _check(load().spa_select_blocks(h, _ptr(q_pre), _ptr(idx_cache), _host_u8(head_mask), _ptr(seq_lens), B,
+                                    max_seq_len, p, n_sink, window, _ptr(sel_idx), _ptr(sel_count),
+                                    _stream(stream)))
+
+
+def spa_decode_blocks(h, q_pre, k_cache, v_cache, idx_cache, head_mask, seq_lens, B: int, max_seq_len: int,
+                      p: float, n_sink: int, window: int, out, sel_count_opt=None, stream=None) -> None:
+    _check(load().spa_decode_blocks(h, _ptr(q_pre), _ptr(k_cache), _ptr(v_cache), _ptr(idx_cache),
+                                    _host_u8(head_mask), _ptr(seq_lens), B, max_seq_len, p, n_sink, window,
+                                    _ptr(out), _ptr(sel_count_opt), _stream(stream)))
 
 
 def spa_device_status(h, stream=None) -> None:

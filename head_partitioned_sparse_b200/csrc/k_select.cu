@@ -33,6 +33,12 @@
 //             float64, reduced exactly in units of pi);
 //   -- grid barrier --
 //   compact   per chunk: kept positions outside sinks/window, ascending.
+// Block mode (the block-granular variant, a second instantiation): the ranges are cut at
+// kBlock-token block boundaries, the mass phase stores and histograms each block's mass
+// (the float32 sum of its tokens' pi) instead of the tokens', the threshold, refine and
+// compact steps rank blocks and count their listed tokens, and compact lists every
+// token of a kept block.  The blocks follow the chunk routing of the "Hierarchical
+// Global Attention" summary, Central mechanism §4.
 // One launch replaces a chain of small kernels whose fixed launch cost dominated.
 // Grid barriers and the q_idx flags are polled with a clock budget; on timeout they set
 // a device status bit and the kernel leaves or carries on without hanging.  The launch
@@ -539,18 +545,22 @@ __device__ void compute_qidx(const StepParams& P, int b, int g, SelScalars& sc) 
 // each, as ngc 16-token groups; slice y = b * n_ret + r owns global groups
 // [y ngc, (y+1) ngc)) into equal contiguous group ranges, one per CTA, so every SM of a
 // full-occupancy grid gets the same share.  A range may span slices; groups past a
-// sequence's length are empty.  CTA c covers [c T / nb, (c+1) T / nb), T = n_rs ngc.
+// sequence's length are empty.  Ranges are cut at multiples of q groups (q = 1, or
+// kBlock / 16 in block mode so that no block is split; ngc is then a multiple of q):
+// CTA c covers groups [q floor(c Q / nb), q floor((c+1) Q / nb)), Q = n_rs ngc / q.
+template <bool BLK>
 struct Ranges {
-  long long ngc, total;
+  static constexpr int q = BLK ? kBlock / 16 : 1;
+  long long ngc, quanta;
   int nb;
   __device__ __forceinline__ Ranges(const StepParams& P) {
-    ngc = ((long long)P.Lcap + 15) / 16;
-    total = (long long)P.B * P.n_ret * ngc;
+    ngc = ((long long)P.Lcap + 16 * q - 1) / (16 * q) * q;
+    quanta = (long long)P.B * P.n_ret * (ngc / q);
     nb = (int)gridDim.x;
   }
-  __device__ __forceinline__ long long begin(int c) const { return (long long)c * total / nb; }
+  __device__ __forceinline__ long long begin(int c) const { return (long long)c * quanta / nb * q; }
   // CTA whose range holds global group g
-  __device__ __forceinline__ int owner(long long g) const { return (int)(((g + 1) * nb - 1) / total); }
+  __device__ __forceinline__ int owner(long long g) const { return (int)(((g / q + 1) * nb - 1) / quanta); }
   __device__ __forceinline__ int first_cta(int y) const { return owner((long long)y * ngc); }
   __device__ __forceinline__ int last_cta(int y) const { return owner((long long)(y + 1) * ngc - 1); }
 };
@@ -560,8 +570,8 @@ struct Ranges {
 __device__ __forceinline__ size_t stats_slot(int cta, int y) { return (size_t)cta + (size_t)y; }
 
 // Visits the CTA's range as segments f(y, l0, l1) of local groups [l0, l1) of slice y.
-template <class F>
-__device__ __forceinline__ void for_each_segment(const Ranges& R, F&& f) {
+template <class RT, class F>
+__device__ __forceinline__ void for_each_segment(const RT& R, F&& f) {
   const long long ge = R.begin(blockIdx.x + 1);
   for (long long g = R.begin(blockIdx.x); g < ge;) {
     const int y = (int)(g / R.ngc);
@@ -625,7 +635,8 @@ __device__ __forceinline__ void wait_qidx(const StepParams& P, int s) {
 }
 
 // Clears the CTA's share of slice y's round-1 / round-2 histograms (read after a barrier).
-__device__ __forceinline__ void clear_hist_share(const StepParams& P, const Ranges& R, int y, int s) {
+template <class RT>
+__device__ __forceinline__ void clear_hist_share(const StepParams& P, const RT& R, int y, int s) {
   static_assert(kBins1 == kBins2, "histogram reset assumes equal round-1 / round-2 bin counts");
   const int first = R.first_cta(y), n = R.last_cta(y) - first + 1, k = (int)blockIdx.x - first;
   unsigned long long* h1 = P.ws.hist1 + (size_t)s * kBins1;
@@ -641,8 +652,8 @@ __device__ __forceinline__ void clear_hist_share(const StepParams& P, const Rang
 // groups l0 + w, l0 + w + 8, ..., kGroupBatch at a time; the first batch is requested
 // before the query vectors arrive (bounded by the call's max length; rows past the
 // sequence are masked).
-template <int G>
-__device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc, const Ranges& R, int y,
+template <int G, class RT>
+__device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc, const RT& R, int y,
                               int l0, int l1) {
   constexpr int NH = IdxTiles<G>::NH, U = kGroupBatch;
   const Unit un = unit_of(P, y);
@@ -715,9 +726,9 @@ __device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc
   __syncthreads();   // sm.red reused by the next range
 }
 
-template <typename T, int G>
+template <typename T, int G, bool BLK>
 __device__ void score_phase(const StepParams& P, SmemScore& sm, SelScalars& sc) {
-  const Ranges R(P);
+  const Ranges<BLK> R(P);
   const long long ga = R.begin(blockIdx.x), ge = R.begin(blockIdx.x + 1);
   for (long long y = (ga + R.ngc - 1) / R.ngc; y * R.ngc < ge; ++y) lead_slice<T, G>(P, sc, (int)y);
   for_each_segment(R, [&](int y, int l0, int l1) { score_segment<G>(P, sm, sc, R, y, l0, l1); });
@@ -762,20 +773,26 @@ __device__ void cut1_slice(const StepParams& P, SmemStage& sm, SelScalars& sc, i
 // round-1 histogram via a per-range shared histogram of counts and low significand
 // bits (32-bit atomics; a range holds at most kMaxRangeGroups groups, so a bin's
 // low-bit sum stays below 2^32).
+// Block mode (BLK): warp w's batch is the four consecutive groups of one kBlock-token
+// block; the block's mass (the float32 sum of its tokens' pi, in a fixed order) is
+// stored at pi[block] and histogrammed instead of the tokens'.
 constexpr int kMaxRangeGroups = 1024;   // 16384 tokens: 16384 * 2^18 = 2^32
-template <int G>
-__device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, const Ranges& R, int y, int l0,
+static_assert(kGroupBatch * 16 == kBlock, "block mode: one warp batch is one block");
+template <int G, bool BLK>
+__device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, const Ranges<BLK>& R, int y, int l0,
                              int l1) {
   constexpr int NH = IdxTiles<G>::NH, U = kGroupBatch;
   const Unit un = unit_of(P, y);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, gid = lane >> 2, t4 = lane & 3;
   const uint2* rows = reinterpret_cast<const uint2*>(P.idx_cache + (size_t)un.s * P.Lmax * kIdxDim);
   const uint64_t pol = l2_policy_drop();
+  // local group of batch slot u at batch base gb
+  auto grp = [&](int gb, int u) { return BLK ? gb + U * warp + u : gb + warp + kWarps * u; };
   uint2 ra[U], rb[U];
   {
     const int jpf = min(P.Lcap, 16 * l1);
 #pragma unroll
-    for (int u = 0; u < U; ++u) load_group(rows, 16 * (l0 + warp + kWarps * u), jpf, pol, ra[u], rb[u]);
+    for (int u = 0; u < U; ++u) load_group(rows, 16 * grp(l0, u), jpf, pol, ra[u], rb[u]);
   }
   // the sequence length, the query index vectors and the slice statistics are
   // requested together; one CTA barrier publishes them
@@ -830,11 +847,12 @@ __device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
   for (int gb = l0; 16 * gb < jend; gb += kWarps * U) {
     if (gb > l0) {
 #pragma unroll
-      for (int u = 0; u < U; ++u) load_group(rows, 16 * (gb + warp + kWarps * u), jend, pol, ra[u], rb[u]);
+      for (int u = 0; u < U; ++u) load_group(rows, 16 * grp(gb, u), jend, pol, ra[u], rb[u]);
     }
+    float bsum = 0.f;
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int j = 16 * (gb + warp + kWarps * u);
+      const int j = 16 * grp(gb, u);
       float lg[NH][2];
       group_logits<G>(ra[u], rb[u], qb, scale, lg);
       // pi = sum over the group's heads of 2^(l - M_h) / (G Z_h): lane-local heads first,
@@ -852,7 +870,9 @@ __device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
         acc += __shfl_xor_sync(kFull, acc, 2);
         pr[cc] = acc;
       }
-      if (t4 < 2) {   // lane t4 = 0 stores token gid, t4 = 1 token gid + 8
+      if (BLK) {
+        bsum += (j + gid < jend ? pr[0] : 0.f) + (j + gid + 8 < jend ? pr[1] : 0.f);
+      } else if (t4 < 2) {   // lane t4 = 0 stores token gid, t4 = 1 token gid + 8
         const int jt = j + gid + 8 * t4;
         const float v = t4 == 0 ? pr[0] : pr[1];
         if (jt < jend) {
@@ -864,6 +884,19 @@ __device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
         }
       }
     }
+    if (BLK) {
+      // every lane of a token quad holds the same sums: add over the 8 token rows
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) bsum += __shfl_xor_sync(kFull, bsum, o);
+      const int jb = 16 * grp(gb, 0);
+      if (lane == 0 && jb < jend) {
+        pi[jb / kBlock] = bsum;
+        const unsigned bits = __float_as_uint(bsum);
+        const unsigned d = min(bits >> 18, (unsigned)(kBins1 - 1));
+        atomicAdd(&sm.cnt[d], 1u);
+        atomicAdd(&sm.low[d], bits & 0x3ffffu);
+      }
+    }
   }
   __syncthreads();
   unsigned long long* g1 = P.ws.hist1 + (size_t)un.s * kBins1;
@@ -873,12 +906,12 @@ __device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
   __syncthreads();   // the histogram is reused by the next range
 }
 
-template <int G>
+template <int G, bool BLK>
 __device__ void mass_phase(const StepParams& P, SelSmem& sm_all, SelScalars& sc) {
   SmemMass& sm = sm_all.mass;
-  const Ranges R(P);
+  const Ranges<BLK> R(P);
   for_each_segment(R, [&](int y, int l0, int l1) {
-    for (int a = l0; a < l1; a += kMaxRangeGroups) mass_segment<G>(P, sm, sc, R, y, a, min(l1, a + kMaxRangeGroups));
+    for (int a = l0; a < l1; a += kMaxRangeGroups) mass_segment<G, BLK>(P, sm, sc, R, y, a, min(l1, a + kMaxRangeGroups));
     const int n = R.last_cta(y) - R.first_cta(y) + 1;
     if (last_of_slice(&P.ws.st[unit_of(P, y).s].ticket_mass, (unsigned)n, &sc.ok)) cut1_slice(P, sm_all.stage, sc, y);
   });
@@ -909,8 +942,25 @@ __device__ __forceinline__ int listed_in(const SinkWindow& sw, int lo, int hi) {
   return b > a ? b - a : 0;
 }
 
+// Chunk of element e (a token, or a block in block mode).
+template <bool BLK>
+__device__ __forceinline__ int chunk_of(int e) {
+  return BLK ? e / (kChunk / kBlock) : e / kChunk;
+}
+
+// Listed positions (outside sinks and window) of element e: token e, or block e in
+// block mode.
+template <bool BLK>
+__device__ __forceinline__ int listed_of(const SinkWindow& sw, int L, int e) {
+  if (!BLK) return sw.always(e) ? 0 : 1;
+  return listed_in(sw, e * kBlock, min(L, (e + 1) * kBlock));
+}
+
 // Unit: one chunk.  Tokens above bin b1 counted (listed ones), tokens of bin b1
 // appended as candidates with their round-2 masses added to the slice histogram.
+// Block mode: the chunk's kChunk / kBlock blocks, one per thread of the first warps;
+// a block above b1 counts its listed tokens, a block of bin b1 is a candidate.
+template <bool BLK>
 __device__ void threshold_unit(const StepParams& P, SelScalars& sc, int y, int c) {
   const Unit un = unit_of(P, y);
   const int L = cta_len(P, un.b, sc);
@@ -925,7 +975,31 @@ __device__ void threshold_unit(const StepParams& P, SelScalars& sc, int y, int c
   uint2* cand = P.ws.cand + (size_t)un.s * P.Lmax;
   unsigned long long* h2 = P.ws.hist2 + (size_t)un.s * kBins2;
   int cnt = 0;
-  if (j0 < L) {
+  if (BLK && j0 < L) {
+    constexpr int kPer = kChunk / kBlock;
+    static_assert(kPer % 32 == 0 && kPer <= kSelThreads, "block mode: whole warps of blocks per chunk");
+    const int e = c * kPer + tid;
+    bool is_cand = false;
+    unsigned bits = 0u;
+    if (tid < kPer && e * kBlock < L) {
+      bits = __ldcg(pib + e);
+      const int d1 = (int)min(bits >> 18, (unsigned)(kBins1 - 1));
+      if (d1 > b1) cnt = listed_of<BLK>(sw, L, e);
+      else is_cand = d1 == b1;
+    }
+    if (tid < kPer) {   // whole warps
+      const unsigned mask = __ballot_sync(kFull, is_cand);
+      if (mask) {
+        unsigned base = 0u;
+        if (lane == 0) base = atomicAdd(&st->cand_count, (unsigned)__popc(mask));
+        base = __shfl_sync(kFull, base, 0);
+        if (is_cand) {
+          cand[base + __popc(mask & ((1u << lane) - 1u))] = make_uint2(bits, (unsigned)e);
+          atomicAdd(&h2[(bits >> 6) & 0xfffu], sel_mass(P, bits));
+        }
+      }
+    }
+  } else if (j0 < L) {
     const int jend = min(L, j0 + kChunk);
     unsigned bits[kTokPerThread];
 #pragma unroll
@@ -971,6 +1045,7 @@ __device__ void threshold_unit(const StepParams& P, SelScalars& sc, int y, int c
 }
 
 // ------------------------------------------------------------------ refine (per slice)
+template <bool BLK>
 __device__ void refine_slice(const StepParams& P, SelSmem& smu, SelScalars& sc, int y) {
   SmemRefine& sm = smu.ref;
   const Unit un = unit_of(P, y);
@@ -1018,7 +1093,8 @@ __device__ void refine_slice(const StepParams& P, SelSmem& smu, SelScalars& sc, 
     for_each_candidate(cand, n, [&](unsigned bits, int pos) {
       const int d2 = (int)((bits >> 6) & 0xfffu);
       if (d2 > cb2) {
-        if (!sw.always(pos)) atomicAdd(&chunk_sel[pos / kChunk], 1);
+        const int nl = listed_of<BLK>(sw, L, pos);
+        if (nl) atomicAdd(&chunk_sel[chunk_of<BLK>(pos)], nl);
       } else if (d2 == cb2) {
         atomicAdd(&sm.m3[bits & 63u], sel_mass(P, bits));
         atomicAdd(&sm.c3[bits & 63u], 1u);
@@ -1098,7 +1174,10 @@ __device__ void refine_slice(const StepParams& P, SelSmem& smu, SelScalars& sc, 
       const int pc = pos_cut;
       auto keep_bin = [&](unsigned bits, int pos) {
         if ((int)((bits >> 6) & 0xfffu) != cb2) return;
-        if ((bits > tau || (bits == tau && pos <= pc)) && !sw.always(pos)) atomicAdd(&chunk_sel[pos / kChunk], 1);
+        if (bits > tau || (bits == tau && pos <= pc)) {
+          const int nl = listed_of<BLK>(sw, L, pos);
+          if (nl) atomicAdd(&chunk_sel[chunk_of<BLK>(pos)], nl);
+        }
       };
       if (small_ok) {
         for (unsigned i = tid; i < sn; i += kSelThreads) keep_bin(small[i].x, (int)small[i].y);
@@ -1144,6 +1223,7 @@ __device__ void refine_slice(const StepParams& P, SelSmem& smu, SelScalars& sc, 
 }
 
 // ------------------------------------------------------------------ compact phase
+template <bool BLK>
 __device__ void compact_unit(const StepParams& P, SelScalars& sc, int y, int c) {
   const Unit un = unit_of(P, y);
   const int L = cta_len(P, un.b, sc);
@@ -1162,7 +1242,19 @@ __device__ void compact_unit(const StepParams& P, SelScalars& sc, int y, int c) 
   const unsigned* pib = reinterpret_cast<const unsigned*>(P.ws.pi + (size_t)un.s * P.ws.pi_stride);
   const int jb = j0 + threadIdx.x * kTokPerThread;  // this thread's 16 consecutive tokens
   unsigned keep = 0u;
-  if (jb < L) {
+  if (BLK && jb < L) {
+    // the 16 tokens lie in one block: kept with it
+    static_assert(kBlock % kTokPerThread == 0, "a thread's tokens must lie in one block");
+    const int e = jb / kBlock;
+    const unsigned bits = __ldcg(pib + e);
+    if (bits > tau || (bits == tau && e <= pos_cut)) {
+#pragma unroll
+      for (int i = 0; i < kTokPerThread; ++i) {
+        const int j = jb + i;
+        keep |= (j < L && !sw.always(j) ? 1u : 0u) << i;
+      }
+    }
+  } else if (jb < L) {
     // rows of the probability buffer are padded to 64 floats: four 16-byte loads stay in the row
     const uint4* v4 = reinterpret_cast<const uint4*>(pib + jb);
     unsigned bits[kTokPerThread];
@@ -1196,7 +1288,7 @@ __device__ void compact_unit(const StepParams& P, SelScalars& sc, int y, int c) 
 }
 
 // ------------------------------------------------------------------ the kernel
-template <typename T, int G>
+template <typename T, int G, bool BLK>
 __global__ void __launch_bounds__(kSelThreads, 4) k_select(StepParams P) {
   __shared__ SelSmem sm;
   __shared__ SelScalars sc;
@@ -1208,42 +1300,49 @@ __global__ void __launch_bounds__(kSelThreads, 4) k_select(StepParams P) {
   const int n_rs = P.B * P.n_ret;
   const int n_units = n_rs * P.n_chunks;
   if (blockIdx.x == 0 && threadIdx.x == 0) P.ws.bar[kBarDuty] = 0u;   // taken after two barriers
-  score_phase<T, G>(P, sm.score, sc);
+  score_phase<T, G, BLK>(P, sm.score, sc);
   if (!grid_barrier(P.ws.bar, P.ws.dev_err, &sc.ok)) return;
-  mass_phase<G>(P, sm, sc);
+  mass_phase<G, BLK>(P, sm, sc);
   if (!grid_barrier(P.ws.bar, P.ws.dev_err, &sc.ok)) return;
   for (int u = blockIdx.x; u < n_units; u += nb) {
     const int y = u / P.n_chunks;
-    threshold_unit(P, sc, y, u % P.n_chunks);
-    if (last_of_slice(&P.ws.st[unit_of(P, y).s].ticket_thr, P.n_chunks, &sc.ok)) refine_slice(P, sm, sc, y);
+    threshold_unit<BLK>(P, sc, y, u % P.n_chunks);
+    if (last_of_slice(&P.ws.st[unit_of(P, y).s].ticket_thr, P.n_chunks, &sc.ok)) refine_slice<BLK>(P, sm, sc, y);
   }
   qrot_duties<T>(P, sm.pro, sc);   // off the critical path: refine steps run meanwhile
   if (!grid_barrier(P.ws.bar, P.ws.dev_err, &sc.ok)) return;
-  for (int u = blockIdx.x; u < n_units; u += nb) compact_unit(P, sc, u / P.n_chunks, u % P.n_chunks);
+  for (int u = blockIdx.x; u < n_units; u += nb) compact_unit<BLK>(P, sc, u / P.n_chunks, u % P.n_chunks);
 }
 
 template <typename T, int G>
 cudaError_t launch_tg(const StepParams& P, int grid, cudaStream_t st) {
   StepParams local = P;
   void* args[] = {&local};
-  return cudaLaunchCooperativeKernel((const void*)k_select<T, G>, dim3(grid), dim3(kSelThreads), args, 0, st);
+  const void* fn = P.blocks ? (const void*)k_select<T, G, true> : (const void*)k_select<T, G, false>;
+  return cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(kSelThreads), args, 0, st);
 }
 
+// Co-resident CTAs per SM, the smaller of the token and block variants (one grid size
+// serves both).
 template <typename T, int G>
 int resident_tg() {
-  int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_select<T, G>, kSelThreads, 0) != cudaSuccess) return -1;
-  return n;
+  int n = 0, m = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_select<T, G, false>, kSelThreads, 0) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, k_select<T, G, true>, kSelThreads, 0) != cudaSuccess)
+    return -1;
+  return n < m ? n : m;
 }
 
 }  // namespace
 
 // Grid of the selection launch: every resident CTA (the same count on every SM, so the
 // range-partitioned score and mass phases are balanced per SM), but never more CTAs than
-// 16-token groups, so no CTA has an empty range.
+// range quanta (16-token groups, or kBlock-token blocks in block mode), so no CTA has an
+// empty range.
 int select_grid(const StepParams& P, int max_resident) {
   if (P.n_ret <= 0) return P.n_slices < max_resident ? P.n_slices : max_resident;
-  const long long groups = (long long)P.B * P.n_ret * (((long long)P.Lcap + 15) / 16);
+  const long long qt = P.blocks ? kBlock : 16;
+  const long long groups = (long long)P.B * P.n_ret * (((long long)P.Lcap + qt - 1) / qt);
   long long want = max_resident;
   if (want > groups) want = groups;
   if (want < 1) want = 1;

@@ -167,6 +167,7 @@ struct StepArgs {
   float p;
   int n_sink, window;
   int64_t k;   // > 0: top-k selection with budget k (p unused)
+  int blocks;  // 1: block-granular top-p
 };
 
 spa_status check_step(spa_ctx* h, const StepArgs& a, spa::StepParams* P) {
@@ -206,6 +207,7 @@ spa_status check_step(spa_ctx* h, const StepArgs& a, spa::StepParams* P) {
   P->p = a.k > 0 ? 1.f : a.p;
   P->keep_all = a.k == 0 && a.p >= 1.f ? 1 : 0;
   P->topk = a.k;
+  P->blocks = a.blocks;
   P->n_sink = a.n_sink;
   P->window = a.window;
   P->idx_scale_log2 = h->idx_scale * 1.4426950408889634f;
@@ -394,7 +396,7 @@ spa_status spa_select(spa_handle h, const void* q_pre, const void* idx_cache, co
                       const int64_t* seq_lens, int B, int64_t max_seq_len, float p, int n_sink, int window,
                       int32_t* sel_idx, int32_t* sel_count, spa_stream stream) {
   spa::StepParams P;
-  spa_status r = check_step(h, StepArgs{q_pre, idx_cache, head_mask, seq_lens, B, max_seq_len, p, n_sink, window, 0}, &P);
+  spa_status r = check_step(h, StepArgs{q_pre, idx_cache, head_mask, seq_lens, B, max_seq_len, p, n_sink, window, 0, 0}, &P);
   if (r) return r;
   return select_with(h, P, sel_idx, sel_count, stream);
 }
@@ -404,7 +406,7 @@ spa_status spa_select_topk(spa_handle h, const void* q_pre, const void* idx_cach
                            int32_t* sel_idx, int32_t* sel_count, spa_stream stream) {
   spa::StepParams P;
   if (k < 1) return fail(SPA_ERR_INVALID_ARG, "k must be >= 1 (got %lld)", (long long)k);
-  spa_status r = check_step(h, StepArgs{q_pre, idx_cache, head_mask, seq_lens, B, max_seq_len, 1.f, n_sink, window, k}, &P);
+  spa_status r = check_step(h, StepArgs{q_pre, idx_cache, head_mask, seq_lens, B, max_seq_len, 1.f, n_sink, window, k, 0}, &P);
   if (r) return r;
   return select_with(h, P, sel_idx, sel_count, stream);
 }
@@ -414,7 +416,7 @@ spa_status spa_decode(spa_handle h, const void* q_pre, const void* k_cache, cons
                       int64_t max_seq_len, float p, int n_sink, int window, float* out, int32_t* sel_count_opt,
                       spa_stream stream) {
   spa::StepParams P;
-  spa_status r = check_step(h, StepArgs{q_pre, idx_cache, head_mask, seq_lens, B, max_seq_len, p, n_sink, window, 0}, &P);
+  spa_status r = check_step(h, StepArgs{q_pre, idx_cache, head_mask, seq_lens, B, max_seq_len, p, n_sink, window, 0, 0}, &P);
   if (r) return r;
   return decode_with(h, P, k_cache, v_cache, out, sel_count_opt, stream);
 }
@@ -425,7 +427,26 @@ spa_status spa_decode_topk(spa_handle h, const void* q_pre, const void* k_cache,
                            spa_stream stream) {
   spa::StepParams P;
   if (k < 1) return fail(SPA_ERR_INVALID_ARG, "k must be >= 1 (got %lld)", (long long)k);
-  spa_status r = check_step(h, StepArgs{q_pre, idx_cache, head_mask, seq_lens, B, max_seq_len, 1.f, n_sink, window, k}, &P);
+  spa_status r = check_step(h, StepArgs{q_pre, idx_cache, head_mask, seq_lens, B, max_seq_len, 1.f, n_sink, window, k, 0}, &P);
+  if (r) return r;
+  return decode_with(h, P, k_cache, v_cache, out, sel_count_opt, stream);
+}
+
+spa_status spa_select_blocks(spa_handle h, const void* q_pre, const void* idx_cache, const uint8_t* head_mask,
+                             const int64_t* seq_lens, int B, int64_t max_seq_len, float p, int n_sink, int window,
+                             int32_t* sel_idx, int32_t* sel_count, spa_stream stream) {
+  spa::StepParams P;
+  spa_status r = check_step(h, StepArgs{q_pre, idx_cache, head_mask, seq_lens, B, max_seq_len, p, n_sink, window, 0, 1}, &P);
+  if (r) return r;
+  return select_with(h, P, sel_idx, sel_count, stream);
+}
+
+spa_status spa_decode_blocks(spa_handle h, const void* q_pre, const void* k_cache, const void* v_cache,
+                             const void* idx_cache, const uint8_t* head_mask, const int64_t* seq_lens, int B,
+                             int64_t max_seq_len, float p, int n_sink, int window, float* out, int32_t* sel_count_opt,
+                             spa_stream stream) {
+  spa::StepParams P;
+  spa_status r = check_step(h, StepArgs{q_pre, idx_cache, head_mask, seq_lens, B, max_seq_len, p, n_sink, window, 0, 1}, &P);
   if (r) return r;
   return decode_with(h, P, k_cache, v_cache, out, sel_count_opt, stream);
 }

@@ -19,6 +19,8 @@ constexpr int kChunk = 4096;
 constexpr int kSelThreads = 256;
 constexpr int kTokPerThread = kChunk / kSelThreads;  // 16
 constexpr int kMaxChunks = int(kMaxCtx / kChunk);    // 4096
+// Block-granular selection ranks blocks of kBlock consecutive positions of a slice.
+constexpr int kBlock = 64;
 
 // Radix digits of the fp32 bit pattern u of a probability in [0, 1]:
 // bits 31..30 are zero, digit1 = u >> 18 (12 bits), digit2 = (u >> 6) & 0xfff
@@ -116,6 +118,7 @@ struct StepParams {
   float p;
   int keep_all;          // p >= 1
   int64_t topk;          // > 0: keep the topk highest-probability tokens instead of top-p
+  int blocks;            // 1: top-p over kBlock-token blocks, whole blocks kept
   int n_sink, window;
   float idx_scale_log2;  // idx_scale * log2(e)
   float attn_scale_log2; // log2(e) / sqrt(128)

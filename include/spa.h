@@ -188,6 +188,28 @@ SPA_API spa_status spa_decode_topk(spa_handle h, const void* q_pre, const void* 
                       float* out, int32_t* sel_count_opt, spa_stream stream);
 
 /*
+ * Block-granular top-p variant.  The "Hierarchical Global Attention" summary
+ * (Central mechanism §4) routes each query to whole chunks of the context rather
+ * than to single tokens; here the chunks are blocks of 64 consecutive positions,
+ * [64 c, min(64 c + 64, L)), and the mass threshold is that of "Full Attention
+ * Strikes Back" (RTPurbo summary), Methodology §3:
+ *   pi_c = sum of pi_j over block c's tokens (pi_j as in spa_select);
+ *   blocks in (pi_c desc, c asc) order; block c is kept iff the mass of the blocks
+ *   before it is < p (every block when p >= 1);
+ *   T = every position of a kept block, minus sinks and window, ascending.
+ * The mass test runs on pi_c quantised as in spa_select (exact integer sums).
+ * Every other argument, output and error is that of spa_select / spa_decode.
+ */
+SPA_API spa_status spa_select_blocks(spa_handle h, const void* q_pre, const void* idx_cache,
+                      const uint8_t* head_mask, const int64_t* seq_lens, int B, int64_t max_seq_len,
+                      float p, int n_sink, int window, int32_t* sel_idx, int32_t* sel_count,
+                      spa_stream stream);
+SPA_API spa_status spa_decode_blocks(spa_handle h, const void* q_pre, const void* k_cache, const void* v_cache,
+                      const void* idx_cache, const uint8_t* head_mask, const int64_t* seq_lens,
+                      int B, int64_t max_seq_len, float p, int n_sink, int window,
+                      float* out, int32_t* sel_count_opt, spa_stream stream);
+
+/*
  * Synchronise `stream`, then read and clear the handle's device status word.
  * Returns SPA_ERR_DEVICE_RANGE (with the offending field named in
  * spa_last_error) if a kernel clamped an out-of-range seq_lens/start_pos value
