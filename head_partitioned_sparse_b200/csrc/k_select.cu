@@ -322,26 +322,27 @@ __device__ __forceinline__ void online_add(float& m, float& z, float l) {
 // ------------------------------------------------------------------ grid barrier
 constexpr long long kBarrierCycles = 4000000000LL;   // ~2 s bound per barrier
 
-// Sense-reversing barrier over all CTAs of a cooperative launch: bar[0] counts
-// arrivals (reset by the last arriver), bar[32] is the generation (a separate
-// 128-byte line, so polling does not delay the arrivals).  Returns false (on every
-// thread of the CTA) if the wait gave up.
+// Barrier over all CTAs of a cooperative launch on one arrival word bar[0]: CTA 0
+// adds 2^31 - (nb - 1), every other CTA adds 1, so the word's top bit flips exactly
+// when the last CTA arrives and its low 31 bits return to their value (no reset, and
+// the release is the last arrival itself).  Every CTA polls until the top bit differs
+// from the one it saw on arrival.  The CTA whose arrival flips the bit also advances
+// the generation word bar[32] (its own 128-byte line), which tags the q_idx flags of
+// a call.  Returns false (on every thread of the CTA) if the wait gave up.
 __device__ bool grid_barrier(unsigned* bar, unsigned* err, int* s_ok) {
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
-    volatile unsigned* gen = bar + 32;
-    const unsigned g = *gen;
+    const unsigned add = blockIdx.x == 0 ? 0x80000000u - (gridDim.x - 1u) : 1u;
     __threadfence();
-    const unsigned arrived = atomicAdd(bar, 1u);
-    if (arrived == gridDim.x - 1) {
-      atomicExch(bar, 0u);
-      __threadfence();
+    const unsigned old = atomicAdd(bar, add);
+    if (((old + add) ^ old) & 0x80000000u) {
       atomicAdd(bar + 32, 1u);
     } else {
+      volatile unsigned* word = bar;
       const long long t0 = clock64();
       unsigned ns = 32;
-      while (*gen == g) {
+      while (((*word ^ old) & 0x80000000u) == 0u) {
         if (clock64() - t0 > kBarrierCycles) {
           atomicOr(err, kErrTimeout);
           ok = 0;
@@ -963,27 +964,42 @@ __device__ __forceinline__ int listed_of(const SinkWindow& sw, int L, int e) {
 template <bool BLK>
 __device__ void threshold_unit(const StepParams& P, SelScalars& sc, int y, int c) {
   const Unit un = unit_of(P, y);
-  const int L = cta_len(P, un.b, sc);
   const int tid = threadIdx.x, lane = tid & 31;
   const int j0 = c * kChunk;
   SliceState* st = P.ws.st + un.s;
-  if (tid == 0) sc.b1 = __ldcg(&st->b1);
-  __syncthreads();
-  const int b1 = sc.b1;
-  const SinkWindow sw(L, P.n_sink, P.window);
   const unsigned* pib = reinterpret_cast<const unsigned*>(P.ws.pi + (size_t)un.s * P.ws.pi_stride);
+  // the chunk's probabilities are requested with L and b1 (one round trip); rows hold
+  // the call's capacity, and entries past L are masked below
+  constexpr int kPer = kChunk / kBlock;
+  static_assert(kPer % 32 == 0 && kPer <= kSelThreads, "block mode: whole warps of blocks per chunk");
+  unsigned bits[kTokPerThread];
+  if (BLK) {
+    const int e = c * kPer + tid;
+    bits[0] = tid < kPer && e * kBlock < P.Lcap ? __ldcg(pib + e) : 0u;
+  } else {
+#pragma unroll
+    for (int i = 0; i < kTokPerThread; ++i) {
+      const int j = j0 + tid + kSelThreads * i;
+      bits[i] = j < P.Lcap ? __ldcg(pib + j) : 0u;
+    }
+  }
+  __syncthreads();   // earlier readers of sc.L / sc.b1 are done
+  if (tid == 0) {
+    sc.L = load_len(P.seq_lens, un.b, P.Lcap, P.ws.dev_err);
+    sc.b1 = __ldcg(&st->b1);
+  }
+  __syncthreads();
+  const int L = sc.L, b1 = sc.b1;
+  const SinkWindow sw(L, P.n_sink, P.window);
   uint2* cand = P.ws.cand + (size_t)un.s * P.Lmax;
   unsigned long long* h2 = P.ws.hist2 + (size_t)un.s * kBins2;
   int cnt = 0;
   if (BLK && j0 < L) {
-    constexpr int kPer = kChunk / kBlock;
-    static_assert(kPer % 32 == 0 && kPer <= kSelThreads, "block mode: whole warps of blocks per chunk");
     const int e = c * kPer + tid;
     bool is_cand = false;
-    unsigned bits = 0u;
     if (tid < kPer && e * kBlock < L) {
-      bits = __ldcg(pib + e);
-      const int d1 = (int)min(bits >> 18, (unsigned)(kBins1 - 1));
+      const unsigned b = bits[0];
+      const int d1 = (int)min(b >> 18, (unsigned)(kBins1 - 1));
       if (d1 > b1) cnt = listed_of<BLK>(sw, L, e);
       else is_cand = d1 == b1;
     }
@@ -994,19 +1010,13 @@ __device__ void threshold_unit(const StepParams& P, SelScalars& sc, int y, int c
         if (lane == 0) base = atomicAdd(&st->cand_count, (unsigned)__popc(mask));
         base = __shfl_sync(kFull, base, 0);
         if (is_cand) {
-          cand[base + __popc(mask & ((1u << lane) - 1u))] = make_uint2(bits, (unsigned)e);
-          atomicAdd(&h2[(bits >> 6) & 0xfffu], sel_mass(P, bits));
+          cand[base + __popc(mask & ((1u << lane) - 1u))] = make_uint2(bits[0], (unsigned)e);
+          atomicAdd(&h2[(bits[0] >> 6) & 0xfffu], sel_mass(P, bits[0]));
         }
       }
     }
   } else if (j0 < L) {
     const int jend = min(L, j0 + kChunk);
-    unsigned bits[kTokPerThread];
-#pragma unroll
-    for (int i = 0; i < kTokPerThread; ++i) {
-      const int j = j0 + tid + kSelThreads * i;
-      bits[i] = j < jend ? __ldcg(pib + j) : 0u;
-    }
     unsigned cflags = 0u;
 #pragma unroll
     for (int i = 0; i < kTokPerThread; ++i) {
@@ -1058,17 +1068,18 @@ __device__ void refine_slice(const StepParams& P, SelSmem& smu, SelScalars& sc, 
   const unsigned n = __ldcg(&st->cand_count);
   const unsigned long long target = __ldcg(&st->target);
   const unsigned long long mab = __ldcg(&st->m_above);
+  const int b1 = __ldcg(&st->b1);
+  int64_t len = P.seq_lens[un.b];
   __syncthreads();   // earlier readers of the scalars are done
-  if (tid == 32) sc.b1 = __ldcg(&st->b1);
   if (tid == 0) {
-    sc.L = load_len(P.seq_lens, un.b, P.Lcap, P.ws.dev_err);
+    if (len < 1 || len > P.Lcap) atomicOr(P.ws.dev_err, kErrSeqLen);
     sc.b2 = -1;
     sc.b3 = -1;
     sc.small_n = 0u;
     sc.kbin = -1;
   }
   __syncthreads();
-  const int L = sc.L, b1 = sc.b1;
+  const int L = len < 1 ? 1 : (len > P.Lcap ? P.Lcap : (int)len);
   const SinkWindow sw(L, P.n_sink, P.window);
   const uint2* cand = P.ws.cand + (size_t)un.s * P.Lmax;
   if (b1 >= 0) {   // round 2 cut (the staging buffer aliases chunk_sel / cnt4k)
@@ -1196,21 +1207,27 @@ __device__ void refine_slice(const StepParams& P, SelSmem& smu, SelScalars& sc, 
                      __ldcg(&P.ws.chunk_gt[(size_t)un.s * P.n_chunks + c]);
     __syncthreads();
   }
-  // offsets: exclusive scan over chunks of (above-b1 count + kept candidates)
+  // offsets: exclusive scan over chunks of (above-b1 count + kept candidates); with one
+  // chunk per thread (up to kSelThreads chunks) the count is loaded once
   const int per = (P.n_chunks + kSelThreads - 1) / kSelThreads;
   const int c0 = tid * per;
+  const int* gt_row = P.ws.chunk_gt + (size_t)un.s * P.n_chunks;
   int loc = 0;
   for (int k = 0; k < per; ++k) {
     const int c = c0 + k;
-    if (c < P.n_chunks) loc += __ldcg(&P.ws.chunk_gt[(size_t)un.s * P.n_chunks + c]) + chunk_sel[c];
+    if (c < P.n_chunks) loc += __ldcg(gt_row + c) + chunk_sel[c];
   }
   int total = 0;
   int run = block_excl_scan(loc, sc.shi, &total);
-  for (int k = 0; k < per; ++k) {
-    const int c = c0 + k;
-    if (c < P.n_chunks) {
-      P.ws.chunk_off[(size_t)un.s * P.n_chunks + c] = run;
-      run += __ldcg(&P.ws.chunk_gt[(size_t)un.s * P.n_chunks + c]) + chunk_sel[c];
+  if (per == 1) {
+    if (c0 < P.n_chunks) P.ws.chunk_off[(size_t)un.s * P.n_chunks + c0] = run;
+  } else {
+    for (int k = 0; k < per; ++k) {
+      const int c = c0 + k;
+      if (c < P.n_chunks) {
+        P.ws.chunk_off[(size_t)un.s * P.n_chunks + c] = run;
+        run += __ldcg(gt_row + c) + chunk_sel[c];
+      }
     }
   }
   if (tid == 0) {
@@ -1225,39 +1242,18 @@ __device__ void refine_slice(const StepParams& P, SelSmem& smu, SelScalars& sc, 
 // ------------------------------------------------------------------ compact phase
 template <bool BLK>
 __device__ void compact_unit(const StepParams& P, SelScalars& sc, int y, int c) {
+  static_assert(kBlock % kTokPerThread == 0, "a thread's tokens must lie in one block");
   const Unit un = unit_of(P, y);
-  const int L = cta_len(P, un.b, sc);
   const int j0 = c * kChunk;
-  if (j0 >= L) return;
-  if (threadIdx.x == 0) {
-    const SliceState* st = P.ws.st + un.s;
-    sc.tau = __ldcg(&st->tau_bits);
-    sc.pos_cut = __ldcg(&st->pos_cut);
-    sc.off = __ldcg(&P.ws.chunk_off[(size_t)un.s * P.n_chunks + c]);
-  }
-  __syncthreads();
-  const unsigned tau = sc.tau;
-  const int pos_cut = sc.pos_cut;
-  const SinkWindow sw(L, P.n_sink, P.window);
   const unsigned* pib = reinterpret_cast<const unsigned*>(P.ws.pi + (size_t)un.s * P.ws.pi_stride);
   const int jb = j0 + threadIdx.x * kTokPerThread;  // this thread's 16 consecutive tokens
-  unsigned keep = 0u;
-  if (BLK && jb < L) {
-    // the 16 tokens lie in one block: kept with it
-    static_assert(kBlock % kTokPerThread == 0, "a thread's tokens must lie in one block");
-    const int e = jb / kBlock;
-    const unsigned bits = __ldcg(pib + e);
-    if (bits > tau || (bits == tau && e <= pos_cut)) {
-#pragma unroll
-      for (int i = 0; i < kTokPerThread; ++i) {
-        const int j = jb + i;
-        keep |= (j < L && !sw.always(j) ? 1u : 0u) << i;
-      }
-    }
-  } else if (jb < L) {
-    // rows of the probability buffer are padded to 64 floats: four 16-byte loads stay in the row
+  // the probabilities are requested with L and the slice's cut (one round trip); rows
+  // hold the call's capacity padded to 64 floats, so four 16-byte loads stay in the row
+  unsigned bits[kTokPerThread] = {};
+  if (BLK) {
+    bits[0] = jb < P.Lcap ? __ldcg(pib + jb / kBlock) : 0u;   // the 16 tokens lie in one block
+  } else if (jb < P.Lcap) {
     const uint4* v4 = reinterpret_cast<const uint4*>(pib + jb);
-    unsigned bits[kTokPerThread];
 #pragma unroll
     for (int q = 0; q < kTokPerThread / 4; ++q) {
       const uint4 v = __ldcg(v4 + q);
@@ -1266,6 +1262,32 @@ __device__ void compact_unit(const StepParams& P, SelScalars& sc, int y, int c) 
       bits[4 * q + 2] = v.z;
       bits[4 * q + 3] = v.w;
     }
+  }
+  __syncthreads();   // earlier readers of the scalars are done
+  if (threadIdx.x == 0) {
+    const SliceState* st = P.ws.st + un.s;
+    sc.L = load_len(P.seq_lens, un.b, P.Lcap, P.ws.dev_err);
+    sc.tau = __ldcg(&st->tau_bits);
+    sc.pos_cut = __ldcg(&st->pos_cut);
+    sc.off = __ldcg(&P.ws.chunk_off[(size_t)un.s * P.n_chunks + c]);
+  }
+  __syncthreads();
+  const int L = sc.L;
+  if (j0 >= L) return;
+  const unsigned tau = sc.tau;
+  const int pos_cut = sc.pos_cut;
+  const SinkWindow sw(L, P.n_sink, P.window);
+  unsigned keep = 0u;
+  if (BLK && jb < L) {
+    const int e = jb / kBlock;
+    if (bits[0] > tau || (bits[0] == tau && e <= pos_cut)) {
+#pragma unroll
+      for (int i = 0; i < kTokPerThread; ++i) {
+        const int j = jb + i;
+        keep |= (j < L && !sw.always(j) ? 1u : 0u) << i;
+      }
+    }
+  } else if (jb < L) {
 #pragma unroll
     for (int i = 0; i < kTokPerThread; ++i) {
       const int j = jb + i;
