@@ -29,8 +29,8 @@ SPA_ERR_DEVICE_RANGE = -6
 SPA_BF16 = 0
 SPA_F32 = 1
 
-SPA_K_INDEX_APPEND, SPA_K_SELECT, SPA_K_ATTEND, SPA_K_COMBINE = range(4)
-SPA_K_COUNT = 4
+SPA_K_INDEX_APPEND, SPA_K_SELECT, SPA_K_ATTEND, SPA_K_COMBINE, SPA_K_KV_APPEND = range(5)
+SPA_K_COUNT = 5
 
 
 class SpaError(RuntimeError):
@@ -69,6 +69,10 @@ _SIGS = {
     "spa_decode_topk": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i64, _i64, _i, _i, _vp, _vp, _vp]),
     "spa_select_blocks": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i64, _f, _i, _i, _vp, _vp, _vp]),
     "spa_decode_blocks": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i64, _f, _i, _i, _vp, _vp, _vp]),
+    "spa_kv_append_compact": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp]),
+    "spa_index_append_compact": (_i, [_vp, _vp, _vp, _i, _i, _vp, _vp, _vp]),
+    "spa_select_compact": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i64, _f, _i, _i, _vp, _vp, _vp]),
+    "spa_decode_compact": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i64, _f, _i, _i, _vp, _vp, _vp]),
     "spa_device_status": (_i, [_vp, _vp]),
     "spa_set_profiling": (_i, [_vp, ctypes.c_uint]),
     "spa_profile_read": (_i, [_vp, _i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
@@ -189,6 +193,33 @@ def spa_decode_blocks(h, q_pre, k_cache, v_cache, idx_cache, head_mask, seq_lens
     _check(load().spa_decode_blocks(h, _ptr(q_pre), _ptr(k_cache), _ptr(v_cache), _ptr(idx_cache),
                                     _host_u8(head_mask), _ptr(seq_lens), B, max_seq_len, p, n_sink, window,
                                     _ptr(out), _ptr(sel_count_opt), _stream(stream)))
+
+
+def spa_kv_append_compact(h, k_new, v_new, start_pos, B: int, T: int, head_mask, n_sink: int, window: int,
+                          k_ret, v_ret, k_ring, v_ring, stream=None) -> None:
+    _check(load().spa_kv_append_compact(h, _ptr(k_new), _ptr(v_new), _ptr(start_pos), B, T, _host_u8(head_mask),
+                                        n_sink, window, _ptr(k_ret), _ptr(v_ret), _ptr(k_ring), _ptr(v_ring),
+                                        _stream(stream)))
+
+
+def spa_index_append_compact(h, k_pre, start_pos, B: int, T: int, head_mask, idx_ret, stream=None) -> None:
+    _check(load().spa_index_append_compact(h, _ptr(k_pre), _ptr(start_pos), B, T, _host_u8(head_mask),
+                                           _ptr(idx_ret), _stream(stream)))
+
+
+def spa_select_compact(h, q_pre, idx_ret, head_mask, seq_lens, B: int, max_seq_len: int, p: float, n_sink: int,
+                       window: int, sel_idx, sel_count, stream=None) -> None:
+    _check(load().spa_select_compact(h, _ptr(q_pre), _ptr(idx_ret), _host_u8(head_mask), _ptr(seq_lens), B,
+                                     max_seq_len, p, n_sink, window, _ptr(sel_idx), _ptr(sel_count),
+                                     _stream(stream)))
+
+
+def spa_decode_compact(h, q_pre, k_ret, v_ret, k_ring, v_ring, idx_ret, head_mask, seq_lens, B: int,
+                       max_seq_len: int, p: float, n_sink: int, window: int, out, sel_count_opt=None,
+                       stream=None) -> None:
+    _check(load().spa_decode_compact(h, _ptr(q_pre), _ptr(k_ret), _ptr(v_ret), _ptr(k_ring), _ptr(v_ring),
+                                     _ptr(idx_ret), _host_u8(head_mask), _ptr(seq_lens), B, max_seq_len, p, n_sink,
+                                     window, _ptr(out), _ptr(sel_count_opt), _stream(stream)))
 
 
 def spa_device_status(h, stream=None) -> None:

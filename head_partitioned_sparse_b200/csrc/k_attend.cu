@@ -119,8 +119,10 @@ __global__ void __launch_bounds__(kAttnThreads) k_attend(StepParams P) {
     const int nc = sw.n_contig();
     const int v0 = (item - pref[s]) * P.split_rows;
     const int v1 = min(v0 + P.split_rows, n_rows);
-    const T* kbase = (const T*)P.k_cache + (size_t)s * P.Lmax * kHeadDim;
-    const T* vbase = (const T*)P.v_cache + (size_t)s * P.Lmax * kHeadDim;
+    const KvSlice<T> kvs = kv_slice<T>(P, s);
+    const T* kbase = kvs.k;
+    const T* vbase = kvs.v;
+    const bool ring = kvs.ring;
     const int* list = P.sel_list + (size_t)s * P.Lmax;
 
     __syncthreads();  // previous item done with qs / buffers
@@ -139,7 +141,8 @@ __global__ void __launch_bounds__(kAttnThreads) k_attend(StepParams P) {
       for (int i = tid; i < nr * kCpr; i += kAttnThreads) {
         const int r = i / kCpr, c = i % kCpr;
         const int v = r0 + r;
-        const int pos = v < nc ? sw.contig_pos(v) : list[v - nc];
+        int pos = v < nc ? sw.contig_pos(v) : list[v - nc];
+        if (ring) pos = ring_row(pos, P.n_sink, P.window);   // streaming head, compact layout
         cp_async16(kd + r * kHeadDim + c * (16 / sizeof(T)), kbase + (size_t)pos * kHeadDim + c * (16 / sizeof(T)));
         cp_async16(vd + r * kHeadDim + c * (16 / sizeof(T)), vbase + (size_t)pos * kHeadDim + c * (16 / sizeof(T)));
       }

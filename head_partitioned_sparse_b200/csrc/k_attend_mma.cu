@@ -297,8 +297,13 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
       const int r0 = pf.v0 + pf_ch * kChunkRows;
       int v = r0 + lane;
       if (v >= pf.v1) v = r0;   // rows past the item repeat row 0 (finite, masked later)
-      pos = v < pf.nc ? (v < pf.n_s ? v : pf.w_lo + (v - pf.n_s))
-                      : P.sel_list[(size_t)pf.s * P.Lmax + (v - pf.nc)];
+      if (v < pf.nc) {
+        pos = v < pf.n_s ? v : pf.w_lo + (v - pf.n_s);
+        // compact layout: a streaming head's rows sit in its ring
+        if (P.compact && !P.is_ret[pf.s % P.Hkv]) pos = ring_row(pos, P.n_sink, P.window);
+      } else {
+        pos = P.sel_list[(size_t)pf.s * P.Lmax + (v - pf.nc)];
+      }
     }
     return pos;
   };
@@ -309,8 +314,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
   auto issue_next = [&]() {
     __nv_bfloat16* dst = myring + (size_t)(issued % kStages) * kStageElems;
     if (pf_item <= s_last) {
-      const __nv_bfloat16* kb = (const __nv_bfloat16*)P.k_cache + (size_t)pf.s * P.Lmax * kHeadDim;
-      const __nv_bfloat16* vb = (const __nv_bfloat16*)P.v_cache + (size_t)pf.s * P.Lmax * kHeadDim;
+      const KvSlice<__nv_bfloat16> kv = kv_slice<__nv_bfloat16>(P, pf.s);
+      const __nv_bfloat16* kb = kv.k;
+      const __nv_bfloat16* vb = kv.v;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int idx = i * 32 + lane;   // 512 pieces of 16 bytes: [K|V][row][piece]

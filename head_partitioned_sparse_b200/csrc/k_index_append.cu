@@ -7,7 +7,9 @@
 // with each product rounded to float32 and added to a float32 running sum in
 // ascending d.
 //
-// Layout: a CTA takes 64 consecutive tokens of one (b, kv head); the key tile
+// Layout: a CTA takes 64 consecutive tokens of one (b, kv head) of the head map (all
+// heads in place, or the retrieval heads only at their rank for the compact layout);
+// the key tile
 // (as float32, rows padded to 129 floats so a warp's 8 rows hit 8 banks) and the
 // head's projector sit in shared memory; each thread produces 4 of a row's 16
 // outputs and writes them as one 8-byte store (a row is 32 contiguous bytes).
@@ -23,12 +25,13 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 k_index_append(const T* __restrict__ k_pre, const int64_t* __restrict__ start_pos, int T_, int Hkv,
                int64_t Lmax, const float* __restrict__ P_k, uint16_t* __restrict__ idx,
-               unsigned* __restrict__ err) {
+               unsigned* __restrict__ err, const HeadMap map) {
   __shared__ float ks[kRowsPerCta][kPad];
   __shared__ float ps[kIdxDim][kPad];
-  const int s = blockIdx.y;              // b * Hkv + g
-  const int g = s % Hkv;
-  const int b = s / Hkv;
+  const int b = blockIdx.y / map.n, m = blockIdx.y % map.n;
+  const int g = map.g[m];
+  const int s = b * Hkv + g;                      // source (b, head)
+  const int sd = b * map.n_slots + map.slot[m];   // destination (b, slot)
   const int t0 = blockIdx.x * kRowsPerCta;
   const int nrows = min(kRowsPerCta, T_ - t0);
   const int tid = threadIdx.x;
@@ -62,21 +65,29 @@ k_index_append(const T* __restrict__ k_pre, const int64_t* __restrict__ start_po
              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(acc[1])) << 16);
   packed.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(acc[2])) |
              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(acc[3])) << 16);
-  *reinterpret_cast<uint2*>(idx + ((size_t)s * Lmax + pos) * kIdxDim + r0) = packed;
+  *reinterpret_cast<uint2*>(idx + ((size_t)sd * Lmax + pos) * kIdxDim + r0) = packed;
 }
 
 }  // namespace
 
 cudaError_t launch_index_append(const void* k_pre, const int64_t* start_pos, int B, int T, int Hkv,
                                 int64_t Lmax, int kv_dtype, const float* P_k, uint16_t* idx_cache,
-                                unsigned* dev_err, cudaStream_t st) {
-  dim3 grid((T + kRowsPerCta - 1) / kRowsPerCta, B * Hkv);
+                                unsigned* dev_err, cudaStream_t st, const HeadMap* map) {
+  HeadMap m;
+  if (map) {
+    m = *map;
+  } else {
+    m.n = m.n_slots = Hkv;
+    for (int g = 0; g < Hkv; ++g) m.g[g] = m.slot[g] = g;
+  }
+  if (m.n == 0) return cudaSuccess;
+  dim3 grid((T + kRowsPerCta - 1) / kRowsPerCta, B * m.n);
   if (kv_dtype == 0)
     k_index_append<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)k_pre, start_pos, T, Hkv, Lmax,
-                                                          P_k, idx_cache, dev_err);
+                                                          P_k, idx_cache, dev_err, m);
   else
     k_index_append<float><<<grid, 256, 0, st>>>((const float*)k_pre, start_pos, T, Hkv, Lmax, P_k,
-                                                 idx_cache, dev_err);
+                                                 idx_cache, dev_err, m);
   return cudaGetLastError();
 }
 

@@ -660,7 +660,7 @@ __device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc
   const Unit un = unit_of(P, y);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, t4 = lane & 3, gid = lane >> 2;
   clear_hist_share(P, R, y, un.s);
-  const uint2* rows = reinterpret_cast<const uint2*>(P.idx_cache + (size_t)un.s * P.Lmax * kIdxDim);
+  const uint2* rows = reinterpret_cast<const uint2*>(idx_rows(P, y, un.s));
   const uint64_t pol = l2_policy_keep();
   uint2 ra[U], rb[U];
   {
@@ -785,7 +785,7 @@ __device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
   constexpr int NH = IdxTiles<G>::NH, U = kGroupBatch;
   const Unit un = unit_of(P, y);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, gid = lane >> 2, t4 = lane & 3;
-  const uint2* rows = reinterpret_cast<const uint2*>(P.idx_cache + (size_t)un.s * P.Lmax * kIdxDim);
+  const uint2* rows = reinterpret_cast<const uint2*>(idx_rows(P, y, un.s));
   const uint64_t pol = l2_policy_drop();
   // local group of batch slot u at batch base gb
   auto grp = [&](int gb, int u) { return BLK ? gb + U * warp + u : gb + warp + kWarps * u; };

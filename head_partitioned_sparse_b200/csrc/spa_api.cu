@@ -217,6 +217,22 @@ spa_status check_step(spa_ctx* h, const StepArgs& a, spa::StepParams* P) {
   return SPA_OK;
 }
 
+// Compact layout: ring size and each head's rank among the heads of its kind.
+spa_status setup_compact(spa::StepParams* P, const void* k_ring, const void* v_ring, bool need_ring) {
+  P->compact = 1;
+  P->n_str = P->Hkv - P->n_ret;
+  P->ring = P->n_sink + P->window;
+  int nr = 0, ns = 0;
+  for (int g = 0; g < P->Hkv; ++g) P->head_rank[g] = P->is_ret[g] ? nr++ : ns++;
+  if (need_ring && P->n_str > 0) {
+    if (!k_ring || !v_ring) return fail(SPA_ERR_INVALID_ARG, "k_ring and v_ring must be non-NULL");
+    if (!aligned16(k_ring) || !aligned16(v_ring)) return fail(SPA_ERR_INVALID_ARG, "k_ring/v_ring must be 16-byte aligned");
+  }
+  P->k_ring = k_ring;
+  P->v_ring = v_ring;
+  return SPA_OK;
+}
+
 spa_status run_selection(spa_ctx* h, spa::StepParams& P, cudaStream_t st) {
   const int grid = spa::select_grid(P, h->select_max_grid);
   return run(h, SPA_K_SELECT, st, "select", [&] { return spa::launch_select(P, h->cfg.kv_dtype, grid, st); });
@@ -451,6 +467,93 @@ spa_status spa_decode_blocks(spa_handle h, const void* q_pre, const void* k_cach
   return decode_with(h, P, k_cache, v_cache, out, sel_count_opt, stream);
 }
 
+spa_status spa_kv_append_compact(spa_handle h, const void* k_new, const void* v_new, const int64_t* start_pos,
+                                 int B, int T, const uint8_t* head_mask, int n_sink, int window, void* k_ret,
+                                 void* v_ret, void* k_ring, void* v_ring, spa_stream stream) {
+  if (!h) return fail(SPA_ERR_INVALID_ARG, "handle is NULL");
+  if (!k_new || !v_new || !start_pos || !head_mask)
+    return fail(SPA_ERR_INVALID_ARG, "k_new, v_new, start_pos and head_mask must be non-NULL");
+  if (!aligned16(k_new) || !aligned16(v_new) || ((uintptr_t)start_pos & 7u))
+    return fail(SPA_ERR_INVALID_ARG, "k_new/v_new must be 16-byte aligned, start_pos 8-byte aligned");
+  if (B < 1 || B > h->cfg.max_batch)
+    return fail(SPA_ERR_INVALID_ARG, "B must be in [1, max_batch=%d] (got %d)", h->cfg.max_batch, B);
+  if (T < 1 || (int64_t)T > h->cfg.max_ctx)
+    return fail(SPA_ERR_INVALID_ARG, "T must be in [1, max_ctx] (got %d)", T);
+  if (n_sink < 0 || window < 0 || (int64_t)n_sink + window < 1)
+    return fail(SPA_ERR_INVALID_ARG, "n_sink, window must be >= 0 with n_sink + window >= 1");
+  const int Hkv = h->cfg.n_kv_heads;
+  unsigned char is_ret[spa::kMaxKvHeads];
+  int rank[spa::kMaxKvHeads];
+  int n_ret = 0, n_str = 0;
+  for (int g = 0; g < Hkv; ++g) {
+    is_ret[g] = head_mask[g] ? 1 : 0;
+    rank[g] = is_ret[g] ? n_ret++ : n_str++;
+  }
+  if (n_ret > 0 && (!k_ret || !v_ret || !aligned16(k_ret) || !aligned16(v_ret)))
+    return fail(SPA_ERR_INVALID_ARG, "k_ret/v_ret must be non-NULL and 16-byte aligned");
+  if (n_str > 0 && (!k_ring || !v_ring || !aligned16(k_ring) || !aligned16(v_ring)))
+    return fail(SPA_ERR_INVALID_ARG, "k_ring/v_ring must be non-NULL and 16-byte aligned");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return run(h, SPA_K_KV_APPEND, st, "kv append", [&] {
+    return spa::launch_kv_append_compact(k_new, v_new, start_pos, B, T, Hkv, h->cfg.max_ctx, h->cfg.kv_dtype, is_ret,
+                                         rank, n_ret, n_str, n_sink, window, k_ret, v_ret, k_ring, v_ring,
+                                         h->ws.dev_err, st);
+  });
+}
+
+spa_status spa_index_append_compact(spa_handle h, const void* k_pre, const int64_t* start_pos, int B, int T,
+                                    const uint8_t* head_mask, void* idx_ret, spa_stream stream) {
+  if (!h) return fail(SPA_ERR_INVALID_ARG, "handle is NULL");
+  if (!k_pre || !start_pos || !idx_ret || !head_mask)
+    return fail(SPA_ERR_INVALID_ARG, "k_pre, start_pos, head_mask, idx_ret must be non-NULL");
+  if (!aligned16(k_pre) || !aligned16(idx_ret) || ((uintptr_t)start_pos & 7u))
+    return fail(SPA_ERR_INVALID_ARG, "k_pre/idx_ret must be 16-byte aligned, start_pos 8-byte aligned");
+  if (B < 1 || B > h->cfg.max_batch)
+    return fail(SPA_ERR_INVALID_ARG, "B must be in [1, max_batch=%d] (got %d)", h->cfg.max_batch, B);
+  if (T < 1 || (int64_t)T > h->cfg.max_ctx)
+    return fail(SPA_ERR_INVALID_ARG, "T must be in [1, max_ctx] (got %d)", T);
+  spa::HeadMap m;
+  m.n = 0;
+  for (int g = 0; g < h->cfg.n_kv_heads; ++g)
+    if (head_mask[g]) {
+      m.g[m.n] = g;
+      m.slot[m.n] = m.n;
+      ++m.n;
+    }
+  m.n_slots = m.n;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return run(h, SPA_K_INDEX_APPEND, st, "index append", [&] {
+    return spa::launch_index_append(k_pre, start_pos, B, T, h->cfg.n_kv_heads, h->cfg.max_ctx, h->cfg.kv_dtype,
+                                    h->ws.P_k, static_cast<uint16_t*>(idx_ret), h->ws.dev_err, st, &m);
+  });
+}
+
+spa_status spa_select_compact(spa_handle h, const void* q_pre, const void* idx_ret, const uint8_t* head_mask,
+                              const int64_t* seq_lens, int B, int64_t max_seq_len, float p, int n_sink, int window,
+                              int32_t* sel_idx, int32_t* sel_count, spa_stream stream) {
+  spa::StepParams P;
+  spa_status r = check_step(h, StepArgs{q_pre, idx_ret, head_mask, seq_lens, B, max_seq_len, p, n_sink, window, 0, 0}, &P);
+  if (r) return r;
+  if ((r = setup_compact(&P, nullptr, nullptr, false))) return r;
+  return select_with(h, P, sel_idx, sel_count, stream);
+}
+
+spa_status spa_decode_compact(spa_handle h, const void* q_pre, const void* k_ret, const void* v_ret,
+                              const void* k_ring, const void* v_ring, const void* idx_ret, const uint8_t* head_mask,
+                              const int64_t* seq_lens, int B, int64_t max_seq_len, float p, int n_sink, int window,
+                              float* out, int32_t* sel_count_opt, spa_stream stream) {
+  spa::StepParams P;
+  spa_status r = check_step(h, StepArgs{q_pre, idx_ret, head_mask, seq_lens, B, max_seq_len, p, n_sink, window, 0, 0}, &P);
+  if (r) return r;
+  if ((r = setup_compact(&P, k_ring, v_ring, true))) return r;
+  if (P.n_ret == 0) {   // no retrieval head: the retrieval caches are never read
+    static const uint4 dummy[1] = {};
+    if (!k_ret) k_ret = dummy;
+    if (!v_ret) v_ret = dummy;
+  }
+  return decode_with(h, P, k_ret, v_ret, out, sel_count_opt, stream);
+}
+
 spa_status spa_device_status(spa_handle h, spa_stream stream) {
   if (!h) return fail(SPA_ERR_INVALID_ARG, "handle is NULL");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -513,7 +616,7 @@ spa_status spa_profile_read(spa_handle h, int kernel_id, double* total_ms, int64
 }
 
 const char* spa_kernel_name(int kernel_id) {
-  static const char* names[SPA_K_COUNT] = {"index_append", "select", "attend", "combine"};
+  static const char* names[SPA_K_COUNT] = {"index_append", "select", "attend", "combine", "kv_append"};
   return (kernel_id >= 0 && kernel_id < SPA_K_COUNT) ? names[kernel_id] : "";
 }
 

@@ -126,6 +126,13 @@ struct StepParams {
   int n_ret;
   int ret_heads[kMaxKvHeads];
   unsigned char is_ret[kMaxKvHeads];
+  // compact KV layout (0: every head keeps [Bm][Hkv][Lmax] rows, index rows likewise)
+  int compact;
+  int n_str;             // streaming heads (Hkv - n_ret)
+  int ring;              // ring rows per streaming head: n_sink + window
+  int head_rank[kMaxKvHeads];   // rank of head g among the retrieval or the streaming heads
+  const void* k_ring;    // [Bm][n_str][ring][128] streaming-head keys (compact layout)
+  const void* v_ring;
   Workspace ws;
 };
 
@@ -151,6 +158,50 @@ struct SinkWindow {
   __device__ __forceinline__ bool always(int j) const { return j < n_s || j >= w_lo; }
   __device__ __forceinline__ int contig_pos(int v) const { return v < n_s ? v : w_lo + (v - n_s); }
 };
+
+// Compact KV layout.  Retrieval heads keep every position in [Bm][n_ret][Lmax][128]
+// (rank r of the head among the retrieval heads, ascending head index); streaming heads
+// keep only what they attend, in a ring [Bm][n_str][n_sink + window][128]: position t
+// at row t for t < n_sink, else at row n_sink + (t - n_sink) mod window.  Index rows of
+// the retrieval heads live in [Bm][n_ret][Lmax][16].
+__device__ __forceinline__ int ring_row(int pos, int n_sink, int window) {
+  return pos < n_sink || window <= 0 ? pos : n_sink + (pos - n_sink) % window;
+}
+// K and V rows of slice s = b * Hkv + g, and whether its positions go through the ring.
+template <typename T>
+struct KvSlice {
+  const T* k;
+  const T* v;
+  bool ring;
+};
+template <typename T>
+__device__ __forceinline__ KvSlice<T> kv_slice(const StepParams& P, int s) {
+  KvSlice<T> r;
+  if (!P.compact) {
+    const size_t off = (size_t)s * P.Lmax * kHeadDim;
+    r.k = (const T*)P.k_cache + off;
+    r.v = (const T*)P.v_cache + off;
+    r.ring = false;
+    return r;
+  }
+  const int b = s / P.Hkv, g = s % P.Hkv, rk = P.head_rank[g];
+  if (P.is_ret[g]) {
+    const size_t off = ((size_t)b * P.n_ret + rk) * P.Lmax * kHeadDim;
+    r.k = (const T*)P.k_cache + off;
+    r.v = (const T*)P.v_cache + off;
+    r.ring = false;
+  } else {
+    const size_t off = ((size_t)b * P.n_str + rk) * P.ring * kHeadDim;
+    r.k = (const T*)P.k_ring + off;
+    r.v = (const T*)P.v_ring + off;
+    r.ring = true;
+  }
+  return r;
+}
+// Index rows of retrieval slice y = b * n_ret + r (slice s = b * Hkv + g).
+__device__ __forceinline__ const uint16_t* idx_rows(const StepParams& P, int y, int s) {
+  return P.idx_cache + (size_t)(P.compact ? y : s) * P.Lmax * kIdxDim;
+}
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -198,9 +249,20 @@ __device__ __forceinline__ void merge_mz(float& m, float& z, float m2, float z2)
 
 // Launchers (defined in the kernel translation units).
 namespace spa {
+// Heads an append writes, with their destination slot (compact layout: rank).
+struct HeadMap {
+  int n;                    // heads written
+  int g[kMaxKvHeads];       // source head
+  int slot[kMaxKvHeads];    // destination head slot
+  int n_slots;              // head slots per sequence in the destination
+};
 cudaError_t launch_index_append(const void* k_pre, const int64_t* start_pos, int B, int T, int Hkv,
                                 int64_t Lmax, int kv_dtype, const float* P_k, uint16_t* idx_cache,
-                                unsigned* dev_err, cudaStream_t st);
+                                unsigned* dev_err, cudaStream_t st, const HeadMap* map = nullptr);
+cudaError_t launch_kv_append_compact(const void* k_new, const void* v_new, const int64_t* start_pos, int B, int T,
+                                     int Hkv, int64_t Lmax, int kv_dtype, const unsigned char* is_ret,
+                                     const int* head_rank, int n_ret, int n_str, int n_sink, int window, void* k_ret,
+                                     void* v_ret, void* k_ring, void* v_ring, unsigned* dev_err, cudaStream_t st);
 cudaError_t launch_select(const StepParams& P, int kv_dtype, int grid, cudaStream_t st);
 int select_grid(const StepParams& P, int max_resident);
 int select_resident_per_sm(int kv_dtype, int G);

@@ -209,6 +209,48 @@ SPA_API spa_status spa_decode_blocks(spa_handle h, const void* q_pre, const void
                       int B, int64_t max_seq_len, float p, int n_sink, int window,
                       float* out, int32_t* sel_count_opt, spa_stream stream);
 
+/* ---- compact KV layout (streaming heads keep only sinks and window) ----
+ *
+ * "Autonomy of Heads" summary, Deployment strategy: retrieval heads keep their global
+ * KV state, streaming heads keep only a fixed sink cache and a recent window.  The
+ * head partition (head_mask) fixes the layout, so every call on the same caches must
+ * pass the same head_mask, n_sink and window.  With n_ret retrieval and
+ * n_str = Hkv - n_ret streaming heads, the rank of a head is its index among the heads
+ * of its kind (ascending head index):
+ *   k_ret, v_ret   device [max_batch][n_ret][Lmax][128], kv_dtype: every position
+ *   k_ring, v_ring device [max_batch][n_str][n_sink + window][128], kv_dtype: position t
+ *                  at row t for t < n_sink, else at row n_sink + (t - n_sink) mod window
+ *   idx_ret        device bf16 [max_batch][n_ret][Lmax][16]: retrieval heads only
+ * Streaming heads then use (n_sink + window) / Lmax of their full-layout memory.
+ * Pointers are 16-byte aligned; errors as for the full-layout calls.
+ */
+
+/* Append T new positions start_pos[b] .. start_pos[b] + T - 1 of every (b, KV head):
+ *   k_new, v_new  device [B][Hkv][T][128], kv_dtype (k post-RoPE)
+ * Retrieval heads store every position; a streaming head stores position t iff
+ * t < n_sink or t >= max(n_sink, start_pos[b] + T - window) (what it still attends
+ * after the call; these never share a ring row).  Positions outside [0, Lmax) are
+ * skipped and reported by spa_device_status. */
+SPA_API spa_status spa_kv_append_compact(spa_handle h, const void* k_new, const void* v_new,
+                      const int64_t* start_pos, int B, int T, const uint8_t* head_mask, int n_sink,
+                      int window, void* k_ret, void* v_ret, void* k_ring, void* v_ring, spa_stream stream);
+
+/* spa_index_append for the retrieval heads only, into idx_ret at their rank. */
+SPA_API spa_status spa_index_append_compact(spa_handle h, const void* k_pre, const int64_t* start_pos,
+                      int B, int T, const uint8_t* head_mask, void* idx_ret, spa_stream stream);
+
+/* spa_select / spa_decode on the compact layout: the same selection and outputs
+ * (bit for bit: the same rows in the same order) as on full-layout caches holding the
+ * same values. */
+SPA_API spa_status spa_select_compact(spa_handle h, const void* q_pre, const void* idx_ret,
+                      const uint8_t* head_mask, const int64_t* seq_lens, int B, int64_t max_seq_len,
+                      float p, int n_sink, int window, int32_t* sel_idx, int32_t* sel_count,
+                      spa_stream stream);
+SPA_API spa_status spa_decode_compact(spa_handle h, const void* q_pre, const void* k_ret, const void* v_ret,
+                      const void* k_ring, const void* v_ring, const void* idx_ret, const uint8_t* head_mask,
+                      const int64_t* seq_lens, int B, int64_t max_seq_len, float p, int n_sink, int window,
+                      float* out, int32_t* sel_count_opt, spa_stream stream);
+
 /*
  * Synchronise `stream`, then read and clear the handle's device status word.
  * Returns SPA_ERR_DEVICE_RANGE (with the offending field named in
@@ -225,7 +267,8 @@ SPA_API spa_status spa_device_status(spa_handle h, spa_stream stream);
 #define SPA_K_SELECT 1
 #define SPA_K_ATTEND 2
 #define SPA_K_COMBINE 3
-#define SPA_K_COUNT 4
+#define SPA_K_KV_APPEND 4
+#define SPA_K_COUNT 5
 
 /* kernel_mask = 0 disables timing.  Otherwise every launch of a kernel whose bit
  * (1 << SPA_K_...) is set is bracketed by two CUDA events recorded on the launch
