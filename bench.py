@@ -58,6 +58,7 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-topk-sweep", action="store_true", help="skip the top-k selector measurements")
     ap.add_argument("--no-block-sweep", action="store_true", help="skip the block-granular selector measurements")
+    ap.add_argument("--no-compact", action="store_true", help="skip the compact KV layout measurement")
     ap.add_argument("--override", action="append", default=[], metavar="KEY=VALUE",
                     help="replace a workload field (e.g. B=1 for a small profiling case)")
     return ap.parse_args()
@@ -383,6 +384,43 @@ def main_native(args):
                                       "achieved_gbs": abb["total"] / (msb * 1e-3) / 1e9,
                                       "selected_rows": abb["selected_rows"]}
 
+    # compact KV layout: streaming heads keep only sinks + a ring-buffered window
+    compact = None
+    if not args.no_compact:
+        ret = [g for g in range(inp.Hkv) if head_mask[g]]
+        n_ret, n_str, ring = len(ret), inp.Hkv - len(ret), inp.n_sink + inp.window
+        c_layers = []
+        for (k, v, ix) in layers:
+            kr = torch.empty((inp.B, max(n_ret, 1), inp.Lmax, 128), dtype=k.dtype, device=dev)
+            vr = torch.empty_like(kr)
+            ks = torch.empty((inp.B, max(n_str, 1), max(ring, 1), 128), dtype=k.dtype, device=dev)
+            vs = torch.empty_like(ks)
+            for b in range(inp.B):   # prefill each sequence into its slot through the library
+                L_b = int(inp.seq_lens[b])
+                B.spa_kv_append_compact(h, k[b:b + 1, :, :L_b].contiguous(), v[b:b + 1, :, :L_b].contiguous(),
+                                        torch.zeros(1, dtype=torch.int64, device=dev), 1, L_b, head_mask,
+                                        inp.n_sink, inp.window, kr[b], vr[b], ks[b], vs[b], stream)
+            c_layers.append((kr, vr, ks, vs, ix[:, ret].contiguous()))
+        B.spa_device_status(h, stream)
+
+        def step_c(i):
+            kr, vr, ks, vs, ixr = c_layers[i % len(c_layers)]
+            B.spa_decode_compact(h, q, kr, vr, ks, vs, ixr, head_mask, lens, inp.B, Lcap, p, inp.n_sink,
+                                 inp.window, out, None, stream)
+        for i in range(3):
+            step_c(i)
+        n = max(10, args.steps // 4)
+        msc, _ = timed(n, step_c)
+        msc = shard.reduce_max(msc, dev) / n
+        row = 128 * s_kv * 2   # K + V bytes per position and head
+        full_b = inp.B * inp.Hkv * inp.Lmax * row
+        comp_b = inp.B * (n_ret * inp.Lmax + n_str * ring) * row
+        compact = {"ms_per_step": msc, "layer_steps_per_s": world * 1e3 / msc,
+                   "achieved_gbs": ab["total"] / (msc * 1e-3) / 1e9,
+                   "kv_bytes_full_layout": full_b, "kv_bytes_compact": comp_b,
+                   "kv_memory_ratio": full_b / comp_b}
+        del c_layers
+
     # end to end through the public API: pinned host inputs in, result out, every step
     e2e = None
     if not args.no_e2e:
@@ -464,6 +502,7 @@ def main_native(args):
             "p_sweep": sweep or None,
             "topk_sweep": topk_sweep or None,
             "block_sweep": block_sweep or None,
+            "compact": compact,
         }
         print(json.dumps(line), flush=True)
     B.spa_destroy(h)

@@ -246,5 +246,42 @@ def make_inputs(name: str = "tiny", seed: int = 0, *,
                   p=float(np.float32(cfg["p"])), n_sink=n_sink, window=window)
 
 
+_T_WQ, _T_WK, _T_WBASIS = 100, 101, 102
+
+
+def make_head_weights(seed: int = 0, Hq: int = 32, Hkv: int = 8, d_model: int = 4096,
+                      retrieval=(0, 4), rank: int = 8, noise: float = 0.05):
+    """Seeded synthetic query/key projections for head labelling by effective rank.
+
+    Returns (W_Q [Hq][128][d_model], W_K [Hkv][128][d_model]) as float32.  Streaming-like
+    KV heads (and their query heads) get i.i.d. N(0, 1/d_model) entries: a diffuse
+    query-key spectrum.  For a retrieval-like KV head g listed in ``retrieval``, the key
+    head and its G query heads share one rank-``rank`` row space drawn for the group:
+    W = sqrt(d_model / 128) C_W B_g + noise * N(0, 1/d_model), with B_g [rank][d_model]
+    of N(0, 1/d_model) entries and a per-matrix C_W [128][rank] of N(0, 1/rank)
+    entries, so a few query-key directions dominate (a concentrated spectrum).
+    """
+    G = Hq // Hkv
+    WQ = np.empty((Hq, HEAD_DIM, d_model), np.float32)
+    WK = np.empty((Hkv, HEAD_DIM, d_model), np.float32)
+    sd = np.float32(1.0 / np.sqrt(d_model))
+    for g in range(Hkv):
+        concentrated = g in retrieval
+        if concentrated:
+            basis = _rng(seed, _T_WBASIS, 0, g).standard_normal((rank, d_model), dtype=np.float32) * sd
+        for m in range(G + 1):   # m < G: query head g G + m; m = G: the key head
+            tid = _T_WQ if m < G else _T_WK
+            r = _rng(seed, tid, m, g)
+            w = r.standard_normal((HEAD_DIM, d_model), dtype=np.float32) * sd
+            if concentrated:
+                coef = r.standard_normal((HEAD_DIM, rank), dtype=np.float32) / np.float32(np.sqrt(rank))
+                w = coef @ basis * np.float32(np.sqrt(d_model / HEAD_DIM)) + np.float32(noise) * w
+            if m < G:
+                WQ[g * G + m] = w
+            else:
+                WK[g] = w
+    return WQ, WK
+
+
 def list_configs() -> List[str]:
     return list(CONFIGS)
