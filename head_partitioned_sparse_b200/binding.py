@@ -73,6 +73,8 @@ _SIGS = {
     "spa_index_append_compact": (_i, [_vp, _vp, _vp, _i, _i, _vp, _vp, _vp]),
     "spa_select_compact": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i64, _f, _i, _i, _vp, _vp, _vp]),
     "spa_decode_compact": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i64, _f, _i, _i, _vp, _vp, _vp]),
+    "spa_head_ranks_workspace_size": (_i, [_i, _i, ctypes.POINTER(ctypes.c_size_t)]),
+    "spa_head_effective_ranks": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp]),
     "spa_device_status": (_i, [_vp, _vp]),
     "spa_set_profiling": (_i, [_vp, ctypes.c_uint]),
     "spa_profile_read": (_i, [_vp, _i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
@@ -220,6 +222,20 @@ def spa_decode_compact(h, q_pre, k_ret, v_ret, k_ring, v_ring, idx_ret, head_mas
     _check(load().spa_decode_compact(h, _ptr(q_pre), _ptr(k_ret), _ptr(v_ret), _ptr(k_ring), _ptr(v_ring),
                                      _ptr(idx_ret), _host_u8(head_mask), _ptr(seq_lens), B, max_seq_len, p, n_sink,
                                      window, _ptr(out), _ptr(sel_count_opt), _stream(stream)))
+
+
+def spa_head_ranks_workspace_size(n_q_heads: int, n_kv_heads: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load().spa_head_ranks_workspace_size(n_q_heads, n_kv_heads, ctypes.byref(n)))
+    return n.value
+
+
+def spa_head_effective_ranks(W_Q, W_K, n_q_heads: int, n_kv_heads: int, d_model: int, n_retrieval: int,
+                             workspace, workspace_bytes: int, er_q, er_kv, head_mask, sigma_opt=None,
+                             stream=None) -> None:
+    _check(load().spa_head_effective_ranks(_ptr(W_Q), _ptr(W_K), n_q_heads, n_kv_heads, d_model, n_retrieval,
+                                           _ptr(workspace), workspace_bytes, _ptr(er_q), _ptr(er_kv),
+                                           _ptr(head_mask), _ptr(sigma_opt), _stream(stream)))
 
 
 def spa_device_status(h, stream=None) -> None:

@@ -554,6 +554,37 @@ spa_status spa_decode_compact(spa_handle h, const void* q_pre, const void* k_ret
   return decode_with(h, P, k_ret, v_ret, out, sel_count_opt, stream);
 }
 
+spa_status spa_head_ranks_workspace_size(int n_q_heads, int n_kv_heads, size_t* bytes) {
+  if (!bytes) return fail(SPA_ERR_INVALID_ARG, "bytes is NULL");
+  if (n_kv_heads < 1 || n_kv_heads > spa::kMaxKvHeads || n_q_heads < n_kv_heads || n_q_heads % n_kv_heads)
+    return fail(SPA_ERR_INVALID_ARG, "n_q_heads must be a positive multiple of n_kv_heads in [1, %d]",
+                spa::kMaxKvHeads);
+  *bytes = spa::head_rank_workspace_bytes(n_q_heads, n_kv_heads);
+  return SPA_OK;
+}
+
+spa_status spa_head_effective_ranks(const float* W_Q, const float* W_K, int n_q_heads, int n_kv_heads, int d_model,
+                                    int n_retrieval, void* workspace, size_t workspace_bytes, double* er_q,
+                                    double* er_kv, uint8_t* head_mask, double* sigma_opt, spa_stream stream) {
+  size_t need = 0;
+  spa_status r = spa_head_ranks_workspace_size(n_q_heads, n_kv_heads, &need);
+  if (r) return r;
+  if (!W_Q || !W_K || !workspace || !er_q || !er_kv || !head_mask)
+    return fail(SPA_ERR_INVALID_ARG, "W_Q, W_K, workspace, er_q, er_kv and head_mask must be non-NULL");
+  if (!aligned16(W_Q) || !aligned16(W_K) || !aligned16(workspace) || ((uintptr_t)er_q & 7u) ||
+      ((uintptr_t)er_kv & 7u) || ((uintptr_t)sigma_opt & 7u))
+    return fail(SPA_ERR_INVALID_ARG, "W_Q/W_K/workspace must be 16-byte aligned, outputs 8-byte aligned");
+  if (d_model < 1) return fail(SPA_ERR_INVALID_ARG, "d_model must be >= 1 (got %d)", d_model);
+  if (n_retrieval < 0 || n_retrieval > n_kv_heads)
+    return fail(SPA_ERR_INVALID_ARG, "n_retrieval must be in [0, n_kv_heads] (got %d)", n_retrieval);
+  if (workspace_bytes < need)
+    return fail(SPA_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
+  cudaError_t e = spa::launch_head_ranks(W_Q, W_K, n_q_heads, n_kv_heads, d_model, n_retrieval, workspace, er_q,
+                                         er_kv, head_mask, sigma_opt, nullptr, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "head ranks");
+  return SPA_OK;
+}
+
 spa_status spa_device_status(spa_handle h, spa_stream stream) {
   if (!h) return fail(SPA_ERR_INVALID_ARG, "handle is NULL");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

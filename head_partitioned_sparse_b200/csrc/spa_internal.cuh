@@ -272,4 +272,8 @@ int attend_setup(int kv_dtype, int G, int max_slices);
 cudaError_t launch_attend_bf16(const StepParams& P, int grid, cudaStream_t st);
 int attend_bf16_setup(int G, int max_slices);
 int set_last_error(int code, const char* msg);
+size_t head_rank_workspace_bytes(int Hq, int Hkv);
+cudaError_t launch_head_ranks(const float* W_Q, const float* W_K, int Hq, int Hkv, int d_model, int n_ret,
+                              void* ws, double* er_q, double* er_kv, unsigned char* mask, double* sigma,
+                              int* sweeps, cudaStream_t st);
 }  // namespace spa

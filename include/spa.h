@@ -251,6 +251,33 @@ SPA_API spa_status spa_decode_compact(spa_handle h, const void* q_pre, const voi
                       const int64_t* seq_lens, int B, int64_t max_seq_len, float p, int n_sink, int window,
                       float* out, int32_t* sel_count_opt, spa_stream stream);
 
+/* ---- head labels from frozen weights ----
+ *
+ * "Autonomy of Heads" summary, Methodology §1-§4: the effective rank of each query
+ * head's kernel operator M_h = W_K^{g T} W_Q^h (g = h / G, its key head),
+ *   ER(h) = exp(-sum_k s_k ln s_k),  s_k = sigma_k / sum_j sigma_j,
+ * sigma_k the singular values of M_h, taken as the square roots of the eigenvalues of
+ * the d_head x d_head proxy (W_Q W_Q^T)(W_K W_K^T).  Per KV head the mean ER of its G
+ * query heads; the n_retrieval KV heads of lowest mean ER (ties: lower index) get
+ * head_mask = 1 (retrieval), the others 0 (streaming).  Everything runs in float64 on
+ * the device; squaring the operator returns a zero singular value as about
+ * sqrt(eps) sigma_max, so rank-deficient heads carry an ER error of up to ~5e-4
+ * relative, full-rank heads about 1e-9.  Run once per model, off the decode path.
+ *   W_Q          device float32 [n_q_heads][128][d_model] (q = W_Q^h x)
+ *   W_K          device float32 [n_kv_heads][128][d_model]
+ *   workspace    device scratch of spa_head_ranks_workspace_size bytes, 16-byte aligned
+ *   er_q         device float64 [n_q_heads], written
+ *   er_kv        device float64 [n_kv_heads], written
+ *   head_mask    device uint8 [n_kv_heads], written
+ *   sigma_opt    NULL, or device float64 [n_q_heads][128]: singular values, descending
+ * Errors: SPA_ERR_INVALID_ARG for NULL or misaligned pointers, n_q_heads not a multiple
+ * of n_kv_heads, n_kv_heads outside [1, 64], d_model < 1, n_retrieval outside
+ * [0, n_kv_heads], or a workspace smaller than required.  The call only enqueues work. */
+SPA_API spa_status spa_head_ranks_workspace_size(int n_q_heads, int n_kv_heads, size_t* bytes);
+SPA_API spa_status spa_head_effective_ranks(const float* W_Q, const float* W_K, int n_q_heads, int n_kv_heads,
+                      int d_model, int n_retrieval, void* workspace, size_t workspace_bytes, double* er_q,
+                      double* er_kv, uint8_t* head_mask, double* sigma_opt, spa_stream stream);
+
 /*
  * Synchronise `stream`, then read and clear the handle's device status word.
  * Returns SPA_ERR_DEVICE_RANGE (with the offending field named in
