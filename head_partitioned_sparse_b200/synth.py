@@ -247,6 +247,17 @@ def make_inputs(name: str = "tiny", seed: int = 0, *,
 
 
 _T_WQ, _T_WK, _T_WBASIS = 100, 101, 102
+_T_QCHUNK = 103
+
+
+def prefill_queries(inp: "Inputs", seed: int, T: int) -> np.ndarray:
+    """Seeded pre-RoPE queries of a prefill chunk: [B][Hq][T][128] N(0, 1) entries, in the
+    bundle's storage dtype (bf16 bits or float32), one stream per (sequence, head)."""
+    q = np.empty((inp.B, inp.Hq, T, HEAD_DIM), np.float32)
+    for b in range(inp.B):
+        for h in range(inp.Hq):
+            q[b, h] = _rng(seed, _T_QCHUNK, b, h).standard_normal((T, HEAD_DIM), dtype=np.float32)
+    return _store(q, inp.dtype)
 
 
 def make_head_weights(seed: int = 0, Hq: int = 32, Hkv: int = 8, d_model: int = 4096,
