@@ -29,8 +29,8 @@ SPA_ERR_DEVICE_RANGE = -6
 SPA_BF16 = 0
 SPA_F32 = 1
 
-SPA_K_INDEX_APPEND, SPA_K_SELECT, SPA_K_ATTEND, SPA_K_COMBINE, SPA_K_KV_APPEND = range(5)
-SPA_K_COUNT = 5
+SPA_K_INDEX_APPEND, SPA_K_SELECT, SPA_K_ATTEND, SPA_K_COMBINE, SPA_K_KV_APPEND, SPA_K_PREFILL = range(6)
+SPA_K_COUNT = 6
 
 
 class SpaError(RuntimeError):
@@ -75,6 +75,7 @@ _SIGS = {
     "spa_decode_compact": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i64, _f, _i, _i, _vp, _vp, _vp]),
     "spa_head_ranks_workspace_size": (_i, [_i, _i, ctypes.POINTER(ctypes.c_size_t)]),
     "spa_head_effective_ranks": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp]),
+    "spa_prefill": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp]),
     "spa_device_status": (_i, [_vp, _vp]),
     "spa_set_profiling": (_i, [_vp, ctypes.c_uint]),
     "spa_profile_read": (_i, [_vp, _i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
@@ -236,6 +237,12 @@ def spa_head_effective_ranks(W_Q, W_K, n_q_heads: int, n_kv_heads: int, d_model:
     _check(load().spa_head_effective_ranks(_ptr(W_Q), _ptr(W_K), n_q_heads, n_kv_heads, d_model, n_retrieval,
                                            _ptr(workspace), workspace_bytes, _ptr(er_q), _ptr(er_kv),
                                            _ptr(head_mask), _ptr(sigma_opt), _stream(stream)))
+
+
+def spa_prefill(h, q_chunk, k_cache, v_cache, head_mask, start_pos, B: int, T: int, n_sink: int, window: int, out,
+                stream=None) -> None:
+    _check(load().spa_prefill(h, _ptr(q_chunk), _ptr(k_cache), _ptr(v_cache), _host_u8(head_mask), _ptr(start_pos),
+                              B, T, n_sink, window, _ptr(out), _stream(stream)))
 
 
 def spa_device_status(h, stream=None) -> None:

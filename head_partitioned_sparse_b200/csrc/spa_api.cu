@@ -585,6 +585,32 @@ spa_status spa_head_effective_ranks(const float* W_Q, const float* W_K, int n_q_
   return SPA_OK;
 }
 
+spa_status spa_prefill(spa_handle h, const void* q_chunk, const void* k_cache, const void* v_cache,
+                       const uint8_t* head_mask, const int64_t* start_pos, int B, int T, int n_sink, int window,
+                       float* out, spa_stream stream) {
+  if (!h) return fail(SPA_ERR_INVALID_ARG, "handle is NULL");
+  if (h->cfg.kv_dtype != 0) return fail(SPA_ERR_INVALID_ARG, "spa_prefill needs bf16 caches (kv_dtype = SPA_BF16)");
+  if (!q_chunk || !k_cache || !v_cache || !head_mask || !start_pos || !out)
+    return fail(SPA_ERR_INVALID_ARG, "q_chunk, k_cache, v_cache, head_mask, start_pos and out must be non-NULL");
+  if (!aligned16(q_chunk) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      ((uintptr_t)start_pos & 7u))
+    return fail(SPA_ERR_INVALID_ARG, "q_chunk/k_cache/v_cache/out must be 16-byte aligned, start_pos 8-byte aligned");
+  if (B < 1 || B > h->cfg.max_batch)
+    return fail(SPA_ERR_INVALID_ARG, "B must be in [1, max_batch=%d] (got %d)", h->cfg.max_batch, B);
+  if (T < 1 || (int64_t)T > h->cfg.max_ctx)
+    return fail(SPA_ERR_INVALID_ARG, "T must be in [1, max_ctx] (got %d)", T);
+  if (n_sink < 0 || window < 0 || (int64_t)n_sink + window < 1)
+    return fail(SPA_ERR_INVALID_ARG, "n_sink, window must be >= 0 with n_sink + window >= 1");
+  unsigned char is_ret[spa::kMaxKvHeads];
+  for (int g = 0; g < h->cfg.n_kv_heads; ++g) is_ret[g] = head_mask[g] ? 1 : 0;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return run(h, SPA_K_PREFILL, st, "prefill", [&] {
+    return spa::launch_prefill(q_chunk, k_cache, v_cache, out, start_pos, B, T, h->cfg.n_q_heads,
+                               h->cfg.n_kv_heads, h->cfg.max_ctx, n_sink, window, is_ret, h->ws.inv_freq,
+                               h->ws.dev_err, st);
+  });
+}
+
 spa_status spa_device_status(spa_handle h, spa_stream stream) {
   if (!h) return fail(SPA_ERR_INVALID_ARG, "handle is NULL");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -647,7 +673,7 @@ spa_status spa_profile_read(spa_handle h, int kernel_id, double* total_ms, int64
 }
 
 const char* spa_kernel_name(int kernel_id) {
-  static const char* names[SPA_K_COUNT] = {"index_append", "select", "attend", "combine", "kv_append"};
+  static const char* names[SPA_K_COUNT] = {"index_append", "select", "attend", "combine", "kv_append", "prefill"};
   return (kernel_id >= 0 && kernel_id < SPA_K_COUNT) ? names[kernel_id] : "";
 }
 

@@ -251,6 +251,30 @@ SPA_API spa_status spa_decode_compact(spa_handle h, const void* q_pre, const voi
                       const int64_t* seq_lens, int B, int64_t max_seq_len, float p, int n_sink, int window,
                       float* out, int32_t* sel_count_opt, spa_stream stream);
 
+/* ---- prefill ----
+ *
+ * Attention of a prefill chunk ("Full Attention Strikes Back" (RTPurbo summary),
+ * Methodology §1: retrieval heads attend the full context, local heads a sliding
+ * window with sinks; "Autonomy of Heads" summary, Deployment strategy).  Chunk row i
+ * of sequence b is the query at absolute position t = start_pos[b] + i; it attends
+ *   retrieval head (head_mask[g] = 1): keys j in [0, t]
+ *   streaming head:                    keys j <= t with j < n_sink or j > t - window
+ *   out[b][h][i] = sum_j softmax_j(<RoPE(q_chunk[b][h][i], t), k_cache[b][g][j]> / sqrt(128)) v_cache[b][g][j]
+ * The caches must already hold every position < start_pos[b] + T (append the chunk's
+ * rows first).  The rotated query and the probabilities are rounded to bf16 for the
+ * tensor cores (float32 scores and accumulation).  Requires kv_dtype = SPA_BF16.
+ *   q_chunk    device bf16 [B][Hq][T][128] pre-RoPE queries
+ *   k_cache, v_cache device bf16 [max_batch][Hkv][Lmax][128] (full layout)
+ *   head_mask  host uint8 [Hkv]
+ *   start_pos  device int64 [B]; start_pos[b] + T must not exceed Lmax (a CTA that
+ *              finds otherwise writes nothing and spa_device_status reports it)
+ *   out        device float32 [B][Hq][T][128], written
+ * Errors: SPA_ERR_INVALID_ARG for NULL or misaligned pointers, B or T out of range,
+ * n_sink < 0, window < 0, n_sink + window < 1, or float32 caches. */
+SPA_API spa_status spa_prefill(spa_handle h, const void* q_chunk, const void* k_cache, const void* v_cache,
+                      const uint8_t* head_mask, const int64_t* start_pos, int B, int T, int n_sink,
+                      int window, float* out, spa_stream stream);
+
 /* ---- head labels from frozen weights ----
  *
  * "Autonomy of Heads" summary, Methodology §1-§4: the effective rank of each query
@@ -295,7 +319,8 @@ SPA_API spa_status spa_device_status(spa_handle h, spa_stream stream);
 #define SPA_K_ATTEND 2
 #define SPA_K_COMBINE 3
 #define SPA_K_KV_APPEND 4
-#define SPA_K_COUNT 5
+#define SPA_K_PREFILL 5
+#define SPA_K_COUNT 6
 
 /* kernel_mask = 0 disables timing.  Otherwise every launch of a kernel whose bit
  * (1 << SPA_K_...) is set is bracketed by two CUDA events recorded on the launch
