@@ -59,6 +59,8 @@ def parse_args():
     ap.add_argument("--no-topk-sweep", action="store_true", help="skip the top-k selector measurements")
     ap.add_argument("--no-block-sweep", action="store_true", help="skip the block-granular selector measurements")
     ap.add_argument("--no-compact", action="store_true", help="skip the compact KV layout measurement")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill measurement")
+    ap.add_argument("--prefill-len", type=int, default=32768, help="prefill chunk length (from position 0)")
     ap.add_argument("--override", action="append", default=[], metavar="KEY=VALUE",
                     help="replace a workload field (e.g. B=1 for a small profiling case)")
     return ap.parse_args()
@@ -139,6 +141,26 @@ def measured_peaks():
         d = json.load(open(path))
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def measured_bf16_tflops():
+    """Dense bf16 tensor peak: the burst figure (a kernel timed alone), else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        return float(json.load(open(path))["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
+def prefill_flops(T: int, start: int, head_mask, G: int, n_sink: int, window: int) -> float:
+    """Algorithmic flops of a prefill chunk: 4 * 128 per attended (query, key) pair
+    (2 * 128 for q.k, 2 * 128 for p v), over every query head."""
+    t = np.arange(start, start + T, dtype=np.float64)
+    dense = (t + 1).sum()
+    ns = np.minimum(n_sink, t + 1)
+    w_lo = np.maximum(ns, t - window + 1)
+    banded = (ns + (t + 1 - w_lo)).sum()
+    n_ret = int(np.sum(np.asarray(head_mask) != 0))
+    return 4.0 * 128 * G * (n_ret * dense + (len(head_mask) - n_ret) * banded)
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -421,6 +443,34 @@ def main_native(args):
                    "kv_memory_ratio": full_b / comp_b}
         del c_layers
 
+    # prefill of one sequence's first prefill_len positions (tensor cores; reported beside)
+    prefill = None
+    if not args.no_prefill and inp.dtype == "bf16":
+        Tp = min(args.prefill_len, inp.Lmax)
+        gq = torch.Generator(device=dev)
+        gq.manual_seed(1234 + rank)
+        q_chunk = torch.randn((1, inp.Hq, Tp, 128), generator=gq, device=dev).to(torch.bfloat16)
+        out_p = torch.empty((1, inp.Hq, Tp, 128), dtype=torch.float32, device=dev)
+        kc, vc = layers[0][0][0:1].contiguous(), layers[0][1][0:1].contiguous()
+        zero1 = torch.zeros(1, dtype=torch.int64, device=dev)
+
+        def step_p(i):
+            B.spa_prefill(h, q_chunk, kc, vc, head_mask, zero1, 1, Tp, inp.n_sink, inp.window, out_p, stream)
+        for i in range(3):
+            step_p(i)
+        B.spa_device_status(h, stream)
+        n = 5
+        msp, _ = timed(n, step_p)
+        msp = shard.reduce_max(msp, dev) / n
+        fl = prefill_flops(Tp, 0, head_mask, inp.G, inp.n_sink, inp.window)
+        tpk, tpk_kind = measured_bf16_tflops()
+        prefill = {"tokens": Tp, "ms": msp, "tokens_per_s": world * Tp / (msp * 1e-3),
+                   "tflops": fl / (msp * 1e-3) / 1e12, "flops": fl, "peak_tflops": tpk, "peak_kind": tpk_kind,
+                   "frac": fl / (msp * 1e-3) / 1e12 / tpk, "bound": "tensor",
+                   "note": "one sequence from position 0: causal dense for retrieval heads, sinks + window "
+                           "for streaming heads; bf16 inputs, float32 accumulation (tcgen05 MMA, TMEM accumulators)"}
+        del q_chunk, out_p, kc, vc
+
     # end to end through the public API: pinned host inputs in, result out, every step
     e2e = None
     if not args.no_e2e:
@@ -503,6 +553,7 @@ def main_native(args):
             "topk_sweep": topk_sweep or None,
             "block_sweep": block_sweep or None,
             "compact": compact,
+            "prefill": prefill,
         }
         print(json.dumps(line), flush=True)
     B.spa_destroy(h)

@@ -1,0 +1,459 @@
+// Prefill chunk attention on the 5th-generation tensor cores (tcgen05, TMEM).
+//
+// Semantics are those of the prefill oracle ("Full Attention Strikes Back" (RTPurbo
+// summary), Methodology §1; "Autonomy of Heads" summary, Deployment strategy): a query
+// at absolute position t attends keys j <= t, every one on a retrieval head and the
+// sinks (j < n_sink) plus the window (j > t - window) on a streaming head.  The query
+// is rotated to its position (float64 angles in units of pi) and rounded to bf16; the
+// probabilities are rounded to bf16 for P V; scores and accumulators are float32.
+//
+// One CTA: one (b, KV head) and 128 query rows (the group's G heads x 128/G positions,
+// so the G heads share every K/V tile).  256 threads: row r (TMEM lane r) belongs to
+// lane r % 32 of warps r / 32 and r / 32 + 4, which take its column halves [0, 64) and
+// [64, 128) (a warp may only touch the TMEM lanes of its own quarter).  Per 128-key tile:
+//   1. thread 0 issues S = Q K^T as 8 tcgen05.mma (M = N = 128, K = 16 each) into TMEM
+//      columns [0, 128) and commits to an mbarrier;
+//   2. every thread loads its half row of S from TMEM, masks it (tiles that every row
+//      attends whole skip the mask), the two halves agree on the row maximum through
+//      shared memory, the running maximum is kept unless a score exceeds it by more than
+//      2^8 (then the O row in TMEM is rescaled), and P = 2^(s - m) is written as bf16
+//      into shared memory while each half keeps its partial row sum;
+//   3. thread 0 issues O += P V as 8 tcgen05.mma into TMEM columns [128, 256).
+// K and V tiles stream through a two-stage cp.async ring (the next tile loads during
+// the softmax).  Q, K, V and P all sit in shared memory as 128 x 128 bf16 tiles in the
+// 128-byte swizzled layout (two 64-column halves; row r of a half at (r/8)*1024 +
+// (r%8)*128, 16-byte chunk c at (c ^ r%8)*16): K-major operands for Q, K and P, and an
+// MN-major operand (N = head dim) for V.  Every mbarrier wait is bounded; a wait that
+// gives up sets the device status and the CTA frees its tensor memory and leaves.
+#include "spa_internal.cuh"
+
+namespace spa {
+namespace {
+
+constexpr int kT = 128;                       // rows per CTA = keys per tile = head dim
+constexpr int kTileBytes = kT * kT * 2;       // one bf16 128 x 128 tile (32 KB)
+constexpr int kHalf = kTileBytes / 2;         // one 64-column half
+constexpr int kThreads = 256;                  // 8 warps: two per TMEM lane group
+constexpr long long kWaitCycles = 2000000000LL;   // ~1 s at 2 GHz
+constexpr uint32_t kTmemCols = 256;           // S [0, 128), O [128, 256)
+
+struct TcParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  float* out;
+  const int64_t* start;
+  const double* inv_freq_pi;
+  unsigned* err;
+  int T, Hq, Hkv, G, n_sink, window, n_qblocks;
+  int64_t Lmax;
+  float scale_log2;
+  unsigned char is_ret[kMaxKvHeads];
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// Byte offset of (row r, 16-byte chunk c16 in [0, 16)) in a swizzled 128 x 128 bf16 tile.
+__device__ __forceinline__ uint32_t sw_off(int r, int c16) {
+  const int half = c16 >> 3, c = c16 & 7;
+  return (uint32_t)(half * kHalf + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+}
+
+// Shared-memory matrix descriptor (sm_100): start, LBO, SBO in 16-byte units, version 1,
+// 128-byte swizzle.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// Instruction descriptor, kind::f16: bf16 A and B, float32 D, M = N = 128.
+__host__ __device__ constexpr uint32_t idesc_bf16(bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(kT >> 3) << 17) |
+         ((uint32_t)(kT >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_tc(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
+      :: "r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n"
+               :: "r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" :: "r"(smem_u32(bar)), "r"(count) : "memory");
+}
+// Bounded wait for the mbarrier phase with the given parity; false if it gave up.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  const long long t0 = clock64();
+  for (;;) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred P1;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, P1;\n\t}\n"
+        : "=r"(done) : "r"(a), "r"(parity) : "memory");
+    if (done) return true;
+    if (clock64() - t0 > kWaitCycles) return false;
+  }
+}
+
+// 32 consecutive float32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n"
+      :: "r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+         "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+         "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+         "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+         "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+         "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+         "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+         "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+         "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+         "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+         "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void cp16z(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" :: "r"(dst), "l"(src), "r"(src_bytes));
+}
+__device__ __forceinline__ float ex2a(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t pk2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const TcParams P) {
+  extern __shared__ unsigned char smem_raw[];
+  // 1024-byte aligned tiles: Q | P | K0 | V0 | K1 | V1
+  unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* qs = base;
+  unsigned char* ps = base + kTileBytes;
+  unsigned char* kv0 = base + 2 * kTileBytes;
+  __shared__ uint64_t bar_s, bar_o;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+  __shared__ float xch[2][kT];   // per-row values exchanged between the two column halves
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int lg = warp & 3, ch = warp >> 2;   // TMEM lane group (rows 32 lg ..), column half
+  const int r = 32 * lg + lane;              // this thread's row (= TMEM lane)
+  const int QB = kT / P.G;
+  const int qblk = P.n_qblocks - 1 - (int)blockIdx.x;   // heaviest first
+  const int bg = blockIdx.y, b = bg / P.Hkv, g = bg % P.Hkv;
+  const bool ret = P.is_ret[g] != 0;
+  const int64_t start = P.start[b];
+  if (start < 0 || start + P.T > P.Lmax) {
+    if (tid == 0) atomicOr(P.err, kErrStartPos);
+    return;
+  }
+  const int i0 = qblk * QB;
+  const int t_first = (int)start + i0;
+  const int t_end = (int)start + min(i0 + QB, P.T);
+  const int hl = r / QB, t = t_first + r % QB, h = g * P.G + hl;
+  const bool row_ok = t < t_end;
+
+  if (tid == 0) {
+    mbar_init(&bar_s, 1);
+    mbar_init(&bar_o, 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n"
+                 :: "r"(smem_u32(&tmem_base)), "r"(kTmemCols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+  }
+
+  // ---- Q row r, dims [32 ch, 32 ch + 32) and their rotation partners: rotate to t, bf16
+  {
+    const __nv_bfloat16* src = P.q + (((size_t)b * P.Hq + h) * P.T + (t - (int)start)) * kHeadDim;
+#pragma unroll 1
+    for (int cc = 0; cc < 4; ++cc) {
+      const int c16 = 4 * ch + cc;   // dims 8 c16 .. 8 c16 + 7 and 64 + 8 c16 ..
+      uint32_t lo[4], hi[4];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        float r1[2], r2[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int i = 8 * c16 + e + u;
+          float x1 = 0.f, x2 = 0.f;
+          if (row_ok) {
+            x1 = __bfloat162float(src[i]);
+            x2 = __bfloat162float(src[i + kHeadDim / 2]);
+          }
+          const double a = (double)t * P.inv_freq_pi[i];
+          double sn, cs;
+          sincospi(a - 2.0 * rint(0.5 * a), &sn, &cs);
+          r1[u] = (float)((double)x1 * cs - (double)x2 * sn);
+          r2[u] = (float)((double)x2 * cs + (double)x1 * sn);
+        }
+        lo[e / 2] = pk2(r1[0], r1[1]);
+        hi[e / 2] = pk2(r2[0], r2[1]);
+      }
+      *reinterpret_cast<uint4*>(qs + sw_off(r, c16)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(qs + sw_off(r, c16 + 8)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    }
+  }
+
+  // ---- key tiles (CTA-uniform)
+  int sink_tiles, w_first, w_last;
+  if (ret) {
+    sink_tiles = 0;
+    w_first = 0;
+    w_last = (t_end - 1) / kT;
+  } else {
+    const int ns = min(P.n_sink, t_end);
+    sink_tiles = (ns + kT - 1) / kT;
+    const int wlo = max(ns, t_first - P.window + 1);
+    w_first = max(wlo / kT, sink_tiles);
+    w_last = wlo >= t_end ? w_first - 1 : (t_end - 1) / kT;
+  }
+  const int n_tiles = sink_tiles + (w_last >= w_first ? w_last - w_first + 1 : 0);
+  auto tile_of = [&](int it) { return it < sink_tiles ? it : w_first + (it - sink_tiles); };
+  const __nv_bfloat16* kg = P.k + ((size_t)b * P.Hkv + g) * (size_t)P.Lmax * kHeadDim;
+  const __nv_bfloat16* vg = P.v + ((size_t)b * P.Hkv + g) * (size_t)P.Lmax * kHeadDim;
+  auto issue = [&](int it) {
+    if (it < n_tiles) {
+      const int j0 = tile_of(it) * kT;
+      unsigned char* ks = kv0 + (size_t)(it & 1) * 2 * kTileBytes;
+      unsigned char* vs = ks + kTileBytes;
+#pragma unroll 4
+      for (int e = tid; e < kT * 16; e += kThreads) {   // 16-byte chunks of one tile
+        const int rr = e >> 4, c16 = e & 15, j = j0 + rr;
+        const bool ok = j < t_end;
+        const size_t off = (size_t)(ok ? j : 0) * kHeadDim + c16 * 8;
+        const uint32_t so = sw_off(rr, c16);
+        cp16z(smem_u32(ks + so), kg + off, ok ? 16 : 0);
+        cp16z(smem_u32(vs + so), vg + off, ok ? 16 : 0);
+      }
+    }
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+  };
+  issue(0);
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = tmem_base;
+  const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
+  const uint32_t t_s = tmem + lane_off + 64 * ch;          // this thread's 64 S columns
+  const uint32_t t_o = tmem + lane_off + kT + 64 * ch;     // and 64 O columns
+  constexpr uint32_t kIdK = idesc_bf16(false), kIdV = idesc_bf16(true);
+
+  float m_run = -INFINITY, l_half = 0.f;   // running maximum (log2 units), this half's sum
+  const float sl2 = P.scale_log2;
+  const int t_last = t_end - 1;
+
+  // Every tcgen05.ld / tcgen05.st below is warp-aligned: all 32 lanes execute it, so the
+  // loop trip count, the rescale decision and the epilogue are uniform per warp (abort
+  // decisions are taken from shared memory after a CTA barrier).
+  for (int it = 0; it < n_tiles; ++it) {
+    const int j0 = tile_of(it) * kT;
+    const uint32_t ks = smem_u32(kv0 + (size_t)(it & 1) * 2 * kTileBytes);
+    const uint32_t vs = ks + kTileBytes;
+    // K/V of this tile (and Q / P writes) visible to the tensor cores
+    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+    fence_proxy_async();
+    __syncthreads();
+    if (tid == 0) {
+      fence_after();
+#pragma unroll
+      for (int kk = 0; kk < kT / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+        mma_tc(tmem, sdesc(smem_u32(qs) + off, 16, 1024), sdesc(ks + off, 16, 1024), kIdK, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(&bar_s);
+    }
+    // the previous P V has finished with P and with the other K/V stage: prefetch
+    bool ok = it == 0 || mbar_wait(&bar_o, (uint32_t)((it - 1) & 1));
+    issue(it + 1);
+    ok = mbar_wait(&bar_s, (uint32_t)(it & 1)) && ok;
+    if (!ok) {   // noted here, acted on after the next CTA barrier
+      atomicOr(&abort_flag, 1);
+      atomicOr(P.err, kErrTimeout);
+    }
+    __syncwarp();   // the lanes left their waits at different times
+    fence_after();
+    // ---- this thread's half row of S
+    float s[64];
+    {
+      float v32[32];
+      tmem_ld32(t_s, v32);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) s[i] = v32[i];
+      tmem_ld32(t_s + 32, v32);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) s[32 + i] = v32[i];
+    }
+    // a tile whose every key is attended by every row needs no mask
+    const bool full = j0 + kT - 1 <= t_first && (ret || j0 + kT - 1 < P.n_sink || j0 > t_last - P.window);
+    float mx = -INFINITY;
+    if (full) {
+#pragma unroll
+      for (int i = 0; i < 64; ++i) mx = fmaxf(mx, s[i]);
+    } else {
+      const int jb = j0 + 64 * ch;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const int j = jb + i;
+        const bool okj = row_ok && j <= t && (ret || j < P.n_sink || j > t - P.window);
+        s[i] = okj ? s[i] : -INFINITY;
+        mx = fmaxf(mx, s[i]);
+      }
+    }
+    xch[ch][r] = mx;
+    __syncthreads();
+    mx = fmaxf(xch[0][r], xch[1][r]) * sl2;   // row maximum, log2 units
+    // keep the running maximum unless a score exceeds it by more than 2^8; the O rows of
+    // the lanes that move it are rescaled in TMEM by the whole warp (factor 1 elsewhere)
+    const bool raise = mx > m_run + 8.f;
+    const float corr = raise ? (m_run == -INFINITY ? 0.f : ex2a(m_run - mx)) : 1.f;
+    const bool rescale = raise && m_run != -INFINITY;
+    if (__any_sync(0xffffffffu, rescale)) {
+      const float f = rescale ? corr : 1.f;
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        float v32[32];
+        tmem_ld32(t_o + 32 * c, v32);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v32[i] *= f;
+        tmem_st32(t_o + 32 * c, v32);
+      }
+    }
+    if (raise) {
+      l_half *= corr;
+      m_run = mx;
+    }
+    // P = 2^(s sl2 - m) as bf16 into the swizzled tile, 8 chunks of 8 keys
+    const float nm = m_run == -INFINITY ? 0.f : -m_run;
+    const bool live = m_run != -INFINITY;
+    float ls = 0.f;
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float p0 = live ? ex2a(fmaf(s[8 * cc + 2 * e], sl2, nm)) : 0.f;
+        const float p1 = live ? ex2a(fmaf(s[8 * cc + 2 * e + 1], sl2, nm)) : 0.f;
+        ls += p0 + p1;
+        w[e] = pk2(p0, p1);
+      }
+      *reinterpret_cast<uint4*>(ps + sw_off(r, 8 * ch + cc)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    l_half += ls;
+    fence_before();
+    fence_proxy_async();
+    __syncthreads();
+    if (abort_flag) break;
+    if (tid == 0) {
+      fence_after();
+#pragma unroll
+      for (int kk = 0; kk < kT / 16; ++kk) {
+        // A = P (K-major, keys 16 kk ..), B = V (MN-major: 16 keys = two 8-key groups)
+        const uint32_t aoff = (kk >> 2) * kHalf + (kk & 3) * 32;
+        mma_tc(tmem + kT, sdesc(smem_u32(ps) + aoff, 16, 1024), sdesc(vs + kk * 2048, kHalf, 1024), kIdV,
+               (it > 0 || kk > 0) ? 1u : 0u);
+      }
+      mma_commit(&bar_o);
+    }
+  }
+
+  // ---- epilogue: wait for the last P V, O / l
+  if (!abort_flag && !mbar_wait(&bar_o, (uint32_t)((n_tiles - 1) & 1))) {
+    atomicOr(&abort_flag, 1);
+    atomicOr(P.err, kErrTimeout);
+  }
+  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+  xch[ch][r] = l_half;
+  __syncthreads();
+  __syncwarp();
+  fence_after();
+  if (!abort_flag) {
+    const float l = xch[0][r] + xch[1][r];
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    float* dst = P.out + (((size_t)b * P.Hq + h) * P.T + (t - (int)start)) * kHeadDim + 64 * ch;
+#pragma unroll 1
+    for (int c = 0; c < 2; ++c) {
+      float v32[32];
+      tmem_ld32(t_o + 32 * c, v32);
+      if (row_ok) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(dst + 32 * c + i) =
+              make_float4(v32[i] * inv, v32[i + 1] * inv, v32[i + 2] * inv, v32[i + 3] * inv);
+      }
+    }
+  }
+  fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" :: "r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+}  // namespace
+
+int prefill_tc_smem_bytes() { return 6 * kTileBytes + 1024; }
+
+cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, float* out, const int64_t* start, int B,
+                              int T, int Hq, int Hkv, int64_t Lmax, int n_sink, int window,
+                              const unsigned char* is_ret, const double* inv_freq_pi, unsigned* err, cudaStream_t st) {
+  TcParams P;
+  P.q = (const __nv_bfloat16*)q;
+  P.k = (const __nv_bfloat16*)k;
+  P.v = (const __nv_bfloat16*)v;
+  P.out = out;
+  P.start = start;
+  P.inv_freq_pi = inv_freq_pi;
+  P.err = err;
+  P.T = T;
+  P.Hq = Hq;
+  P.Hkv = Hkv;
+  P.G = Hq / Hkv;
+  P.n_sink = n_sink;
+  P.window = window;
+  P.Lmax = Lmax;
+  P.scale_log2 = (float)(1.4426950408889634 / 11.313708498984761);   // log2(e) / sqrt(128)
+  for (int g = 0; g < kMaxKvHeads; ++g) P.is_ret[g] = g < Hkv ? is_ret[g] : 0;
+  const int QB = kT / P.G;
+  P.n_qblocks = (T + QB - 1) / QB;
+  const int smem = prefill_tc_smem_bytes();
+  cudaError_t e = cudaFuncSetAttribute(k_prefill_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  k_prefill_tc<<<dim3(P.n_qblocks, B * Hkv), kThreads, smem, st>>>(P);
+  return cudaGetLastError();
+}
+
+}  // namespace spa

@@ -605,7 +605,7 @@ spa_status spa_prefill(spa_handle h, const void* q_chunk, const void* k_cache, c
   for (int g = 0; g < h->cfg.n_kv_heads; ++g) is_ret[g] = head_mask[g] ? 1 : 0;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   return run(h, SPA_K_PREFILL, st, "prefill", [&] {
-    return spa::launch_prefill(q_chunk, k_cache, v_cache, out, start_pos, B, T, h->cfg.n_q_heads,
+    return spa::launch_prefill_tc(q_chunk, k_cache, v_cache, out, start_pos, B, T, h->cfg.n_q_heads,
                                h->cfg.n_kv_heads, h->cfg.max_ctx, n_sink, window, is_ret, h->ws.inv_freq,
                                h->ws.dev_err, st);
   });

@@ -273,9 +273,9 @@ cudaError_t launch_attend_bf16(const StepParams& P, int grid, cudaStream_t st);
 int attend_bf16_setup(int G, int max_slices);
 int set_last_error(int code, const char* msg);
 size_t head_rank_workspace_bytes(int Hq, int Hkv);
-cudaError_t launch_prefill(const void* q, const void* k, const void* v, float* out, const int64_t* start, int B,
-                           int T, int Hq, int Hkv, int64_t Lmax, int n_sink, int window, const unsigned char* is_ret,
-                           const double* inv_freq_pi, unsigned* err, cudaStream_t st);
+cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, float* out, const int64_t* start, int B,
+                              int T, int Hq, int Hkv, int64_t Lmax, int n_sink, int window,
+                              const unsigned char* is_ret, const double* inv_freq_pi, unsigned* err, cudaStream_t st);
 cudaError_t launch_head_ranks(const float* W_Q, const float* W_K, int Hq, int Hkv, int d_model, int n_ret,
                               void* ws, double* er_q, double* er_kv, unsigned char* mask, double* sigma,
                               int* sweeps, cudaStream_t st);

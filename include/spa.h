@@ -262,7 +262,8 @@ SPA_API spa_status spa_decode_compact(spa_handle h, const void* q_pre, const voi
  *   out[b][h][i] = sum_j softmax_j(<RoPE(q_chunk[b][h][i], t), k_cache[b][g][j]> / sqrt(128)) v_cache[b][g][j]
  * The caches must already hold every position < start_pos[b] + T (append the chunk's
  * rows first).  The rotated query and the probabilities are rounded to bf16 for the
- * tensor cores (float32 scores and accumulation).  Requires kv_dtype = SPA_BF16.
+ * tensor cores (tcgen05 MMA with float32 accumulators in tensor memory; float32
+ * scores).  Requires kv_dtype = SPA_BF16.
  *   q_chunk    device bf16 [B][Hq][T][128] pre-RoPE queries
  *   k_cache, v_cache device bf16 [max_batch][Hkv][Lmax][128] (full layout)
  *   head_mask  host uint8 [Hkv]
