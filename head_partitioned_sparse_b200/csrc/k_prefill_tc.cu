@@ -35,7 +35,8 @@ constexpr int kTileBytes = kT * kT * 2;       // one bf16 128 x 128 tile (32 KB)
 constexpr int kHalf = kTileBytes / 2;         // one 64-column half
 constexpr int kThreads = 256;                  // 8 warps: two per TMEM lane group
 constexpr long long kWaitCycles = 2000000000LL;   // ~1 s at 2 GHz
-constexpr uint32_t kTmemCols = 256;           // S [0, 128), O [128, 256)
+constexpr uint32_t kTmemCols = 512;           // S0 [0, 128), S1 [128, 256), O [256, 384)
+constexpr int kKStages = 3, kVStages = 2;
 
 struct TcParams {
   const __nv_bfloat16* q;
@@ -154,11 +155,12 @@ __device__ __forceinline__ uint32_t pk2(float lo, float hi) {
 
 __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const TcParams P) {
   extern __shared__ unsigned char smem_raw[];
-  // 1024-byte aligned tiles: Q | P | K0 | V0 | K1 | V1
+  // 1024-byte aligned tiles: Q | P | K0 K1 K2 | V0 V1
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* qs = base;
   unsigned char* ps = base + kTileBytes;
-  unsigned char* kv0 = base + 2 * kTileBytes;
+  unsigned char* kst = base + 2 * kTileBytes;
+  unsigned char* vst = kst + kKStages * kTileBytes;
   __shared__ uint64_t bar_s, bar_o;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
@@ -243,33 +245,46 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const TcParams P) {
   auto tile_of = [&](int it) { return it < sink_tiles ? it : w_first + (it - sink_tiles); };
   const __nv_bfloat16* kg = P.k + ((size_t)b * P.Hkv + g) * (size_t)P.Lmax * kHeadDim;
   const __nv_bfloat16* vg = P.v + ((size_t)b * P.Hkv + g) * (size_t)P.Lmax * kHeadDim;
-  auto issue = [&](int it) {
-    if (it < n_tiles) {
-      const int j0 = tile_of(it) * kT;
-      unsigned char* ks = kv0 + (size_t)(it & 1) * 2 * kTileBytes;
-      unsigned char* vs = ks + kTileBytes;
+  // one 128-key tile of K or V (rows past t_end are zero-filled)
+  auto load_tile = [&](const __nv_bfloat16* src, unsigned char* dst, int it) {
+    if (it >= n_tiles) return;
+    const int j0 = tile_of(it) * kT;
 #pragma unroll 4
-      for (int e = tid; e < kT * 16; e += kThreads) {   // 16-byte chunks of one tile
-        const int rr = e >> 4, c16 = e & 15, j = j0 + rr;
-        const bool ok = j < t_end;
-        const size_t off = (size_t)(ok ? j : 0) * kHeadDim + c16 * 8;
-        const uint32_t so = sw_off(rr, c16);
-        cp16z(smem_u32(ks + so), kg + off, ok ? 16 : 0);
-        cp16z(smem_u32(vs + so), vg + off, ok ? 16 : 0);
-      }
+    for (int e = tid; e < kT * 16; e += kThreads) {   // 16-byte chunks of one tile
+      const int rr = e >> 4, c16 = e & 15, j = j0 + rr;
+      const bool ok = j < t_end;
+      cp16z(smem_u32(dst + sw_off(rr, c16)), src + (size_t)(ok ? j : 0) * kHeadDim + c16 * 8, ok ? 16 : 0);
     }
-    asm volatile("cp.async.commit_group;\n" ::: "memory");
   };
-  issue(0);
+  auto k_stage = [&](int it) { return kst + (size_t)(it % kKStages) * kTileBytes; };
+  auto v_stage = [&](int it) { return vst + (size_t)(it % kVStages) * kTileBytes; };
+  load_tile(kg, k_stage(0), 0);
+  load_tile(vg, v_stage(0), 0);
+  load_tile(kg, k_stage(1), 1);
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
 
+  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+  fence_proxy_async();
   fence_before();
   __syncthreads();
   fence_after();
   const uint32_t tmem = tmem_base;
   const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
-  const uint32_t t_s = tmem + lane_off + 64 * ch;          // this thread's 64 S columns
-  const uint32_t t_o = tmem + lane_off + kT + 64 * ch;     // and 64 O columns
+  const uint32_t t_o = tmem + lane_off + 2 * kT + 64 * ch;   // this thread's 64 O columns
   constexpr uint32_t kIdK = idesc_bf16(false), kIdV = idesc_bf16(true);
+  // S_it = Q K_it^T into TMEM columns [128 (it & 1), +128)
+  auto issue_qk = [&](int it) {
+    fence_after();
+    const uint32_t ks = smem_u32(k_stage(it));
+#pragma unroll
+    for (int kk = 0; kk < kT / 16; ++kk) {
+      const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+      mma_tc(tmem + kT * (it & 1), sdesc(smem_u32(qs) + off, 16, 1024), sdesc(ks + off, 16, 1024), kIdK,
+             kk > 0 ? 1u : 0u);
+    }
+    mma_commit(&bar_s);
+  };
+  if (tid == 0) issue_qk(0);
 
   float m_run = -INFINITY, l_half = 0.f;   // running maximum (log2 units), this half's sum
   const float sl2 = P.scale_log2;
@@ -278,27 +293,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const TcParams P) {
   // Every tcgen05.ld / tcgen05.st below is warp-aligned: all 32 lanes execute it, so the
   // loop trip count, the rescale decision and the epilogue are uniform per warp (abort
   // decisions are taken from shared memory after a CTA barrier).
+  // Order per tile it: S_it ready -> row maxima -> (one thread) S_{it+1} = Q K_{it+1}^T
+  // overlaps the rest of this softmax -> P V_{it-1} done -> K_{it+2}, V_{it+1} requested
+  // -> O rescale, P -> (one thread) O += P V_it.
   for (int it = 0; it < n_tiles; ++it) {
     const int j0 = tile_of(it) * kT;
-    const uint32_t ks = smem_u32(kv0 + (size_t)(it & 1) * 2 * kTileBytes);
-    const uint32_t vs = ks + kTileBytes;
-    // K/V of this tile (and Q / P writes) visible to the tensor cores
-    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
-    fence_proxy_async();
-    __syncthreads();
-    if (tid == 0) {
-      fence_after();
-#pragma unroll
-      for (int kk = 0; kk < kT / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-        mma_tc(tmem, sdesc(smem_u32(qs) + off, 16, 1024), sdesc(ks + off, 16, 1024), kIdK, kk > 0 ? 1u : 0u);
-      }
-      mma_commit(&bar_s);
-    }
-    // the previous P V has finished with P and with the other K/V stage: prefetch
-    bool ok = it == 0 || mbar_wait(&bar_o, (uint32_t)((it - 1) & 1));
-    issue(it + 1);
-    ok = mbar_wait(&bar_s, (uint32_t)(it & 1)) && ok;
+    bool ok = mbar_wait(&bar_s, (uint32_t)(it & 1));
     if (!ok) {   // noted here, acted on after the next CTA barrier
       atomicOr(&abort_flag, 1);
       atomicOr(P.err, kErrTimeout);
@@ -308,6 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const TcParams P) {
     // ---- this thread's half row of S
     float s[64];
     {
+      const uint32_t t_s = tmem + lane_off + kT * (it & 1) + 64 * ch;
       float v32[32];
       tmem_ld32(t_s, v32);
 #pragma unroll
@@ -333,8 +334,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const TcParams P) {
       }
     }
     xch[ch][r] = mx;
+    // K_{it+1} (requested one tile earlier) has landed; S_it is read by every warp
+    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+    fence_proxy_async();
+    fence_before();
     __syncthreads();
+    if (abort_flag) break;
+    if (tid == 0 && it + 1 < n_tiles) issue_qk(it + 1);
     mx = fmaxf(xch[0][r], xch[1][r]) * sl2;   // row maximum, log2 units
+    // the previous P V has finished with P, O and V_{it-1}: request the next tiles
+    ok = it == 0 || mbar_wait(&bar_o, (uint32_t)((it - 1) & 1));
+    if (!ok) {
+      atomicOr(&abort_flag, 1);
+      atomicOr(P.err, kErrTimeout);
+    }
+    load_tile(kg, k_stage(it + 2), it + 2);
+    load_tile(vg, v_stage(it + 1), it + 1);
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+    __syncwarp();
+    fence_after();
     // keep the running maximum unless a score exceeds it by more than 2^8; the O rows of
     // the lanes that move it are rescaled in TMEM by the whole warp (factor 1 elsewhere)
     const bool raise = mx > m_run + 8.f;
@@ -378,11 +396,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const TcParams P) {
     if (abort_flag) break;
     if (tid == 0) {
       fence_after();
+      const uint32_t vs = smem_u32(v_stage(it));
 #pragma unroll
       for (int kk = 0; kk < kT / 16; ++kk) {
         // A = P (K-major, keys 16 kk ..), B = V (MN-major: 16 keys = two 8-key groups)
         const uint32_t aoff = (kk >> 2) * kHalf + (kk & 3) * 32;
-        mma_tc(tmem + kT, sdesc(smem_u32(ps) + aoff, 16, 1024), sdesc(vs + kk * 2048, kHalf, 1024), kIdV,
+        mma_tc(tmem + 2 * kT, sdesc(smem_u32(ps) + aoff, 16, 1024), sdesc(vs + kk * 2048, kHalf, 1024), kIdV,
                (it > 0 || kk > 0) ? 1u : 0u);
       }
       mma_commit(&bar_o);
@@ -425,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const TcParams P) {
 
 }  // namespace
 
-int prefill_tc_smem_bytes() { return 6 * kTileBytes + 1024; }
+int prefill_tc_smem_bytes() { return (2 + kKStages + kVStages) * kTileBytes + 1024; }
 
 cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, float* out, const int64_t* start, int B,
                               int T, int Hq, int Hkv, int64_t Lmax, int n_sink, int window,
