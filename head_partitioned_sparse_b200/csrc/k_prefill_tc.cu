@@ -148,6 +148,26 @@ __device__ __forceinline__ float ex2a(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// Packed float32 pairs (one instruction for two lanes of arithmetic).
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pk2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
@@ -246,14 +266,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const TcParams P) {
   const __nv_bfloat16* kg = P.k + ((size_t)b * P.Hkv + g) * (size_t)P.Lmax * kHeadDim;
   const __nv_bfloat16* vg = P.v + ((size_t)b * P.Hkv + g) * (size_t)P.Lmax * kHeadDim;
   // one 128-key tile of K or V (rows past t_end are zero-filled)
+  // Thread tid copies 16-byte chunk tid % 16 of rows tid / 16 + 16 u, u < 8: its swizzled
+  // offset is the same in every tile (row % 8 does not change with u), plus 2048 u.
+  const uint32_t my_so = sw_off(tid >> 4, tid & 15);
+  const int my_row = tid >> 4, my_col = (tid & 15) * 8;
   auto load_tile = [&](const __nv_bfloat16* src, unsigned char* dst, int it) {
     if (it >= n_tiles) return;
-    const int j0 = tile_of(it) * kT;
-#pragma unroll 4
-    for (int e = tid; e < kT * 16; e += kThreads) {   // 16-byte chunks of one tile
-      const int rr = e >> 4, c16 = e & 15, j = j0 + rr;
-      const bool ok = j < t_end;
-      cp16z(smem_u32(dst + sw_off(rr, c16)), src + (size_t)(ok ? j : 0) * kHeadDim + c16 * 8, ok ? 16 : 0);
+    const int j = tile_of(it) * kT + my_row;
+    const uint32_t d = smem_u32(dst) + my_so;
+    const __nv_bfloat16* sp = src + my_col;
+#pragma unroll
+    for (int u = 0; u < kT / 16; ++u) {
+      const bool ok = j + 16 * u < t_end;
+      cp16z(d + 2048u * u, sp + (size_t)(ok ? j + 16 * u : 0) * kHeadDim, ok ? 16 : 0);
     }
   };
   auto k_stage = [&](int it) { return kst + (size_t)(it % kKStages) * kTileBytes; };
@@ -376,20 +401,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const TcParams P) {
     // P = 2^(s sl2 - m) as bf16 into the swizzled tile, 8 chunks of 8 keys
     const float nm = m_run == -INFINITY ? 0.f : -m_run;
     const bool live = m_run != -INFINITY;
-    float ls = 0.f;
+    const uint64_t sl2x2 = f2pack(sl2, sl2), nmx2 = f2pack(nm, nm);
+    uint64_t acc2 = f2pack(0.f, 0.f);
 #pragma unroll
     for (int cc = 0; cc < 8; ++cc) {
       uint32_t w[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float p0 = live ? ex2a(fmaf(s[8 * cc + 2 * e], sl2, nm)) : 0.f;
-        const float p1 = live ? ex2a(fmaf(s[8 * cc + 2 * e + 1], sl2, nm)) : 0.f;
-        ls += p0 + p1;
+        float z0, z1;
+        f2unpack(f2fma(f2pack(s[8 * cc + 2 * e], s[8 * cc + 2 * e + 1]), sl2x2, nmx2), z0, z1);
+        const float p0 = live ? ex2a(z0) : 0.f;
+        const float p1 = live ? ex2a(z1) : 0.f;
+        acc2 = f2add(acc2, f2pack(p0, p1));
         w[e] = pk2(p0, p1);
       }
       *reinterpret_cast<uint4*>(ps + sw_off(r, 8 * ch + cc)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
-    l_half += ls;
+    {
+      float a0, a1;
+      f2unpack(acc2, a0, a1);
+      l_half += a0 + a1;
+    }
     fence_before();
     fence_proxy_async();
     __syncthreads();
