@@ -168,6 +168,12 @@ __device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
   return r;
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pk2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
@@ -344,20 +350,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const TcParams P) {
     }
     // a tile whose every key is attended by every row needs no mask
     const bool full = j0 + kT - 1 <= t_first && (ret || j0 + kT - 1 < P.n_sink || j0 > t_last - P.window);
-    float mx = -INFINITY;
-    if (full) {
-#pragma unroll
-      for (int i = 0; i < 64; ++i) mx = fmaxf(mx, s[i]);
-    } else {
+    if (!full) {
       const int jb = j0 + 64 * ch;
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
         const int j = jb + i;
         const bool okj = row_ok && j <= t && (ret || j < P.n_sink || j > t - P.window);
         s[i] = okj ? s[i] : -INFINITY;
-        mx = fmaxf(mx, s[i]);
       }
     }
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 64; i += 2) mx = max3(mx, s[i], s[i + 1]);
     xch[ch][r] = mx;
     // K_{it+1} (requested one tile earlier) has landed; S_it is read by every warp
     asm volatile("cp.async.wait_group 0;\n" ::: "memory");
