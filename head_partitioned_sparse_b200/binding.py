@@ -77,6 +77,7 @@ _SIGS = {
     "spa_head_effective_ranks": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp]),
     "spa_prefill": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp]),
     "spa_device_status": (_i, [_vp, _vp]),
+    "spa_debug_drop_publish": (_i, [_vp, _i]),
     "spa_set_profiling": (_i, [_vp, ctypes.c_uint]),
     "spa_profile_read": (_i, [_vp, _i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
     "spa_kernel_name": (ctypes.c_char_p, [_i]),
@@ -243,6 +244,10 @@ def spa_prefill(h, q_chunk, k_cache, v_cache, head_mask, start_pos, B: int, T: i
                 stream=None) -> None:
     _check(load().spa_prefill(h, _ptr(q_chunk), _ptr(k_cache), _ptr(v_cache), _host_u8(head_mask), _ptr(start_pos),
                               B, T, n_sink, window, _ptr(out), _stream(stream)))
+
+
+def spa_debug_drop_publish(h, enable: bool) -> None:
+    _check(load().spa_debug_drop_publish(h, 1 if enable else 0))
 
 
 def spa_device_status(h, stream=None) -> None:

@@ -613,7 +613,9 @@ __device__ void lead_slice(const StepParams& P, SelScalars& sc, int y) {
     __threadfence();
   }
   __syncthreads();
-  if (threadIdx.x == 0) atomicExch(&st->qidx_ready, gen + 1u);
+  // (the failure-detection test hook leaves the flag unset: the other CTAs' bounded
+  // waits then run out and report a timeout)
+  if (threadIdx.x == 0 && !P.drop_publish) atomicExch(&st->qidx_ready, gen + 1u);
 }
 
 // Waits (thread 0, bounded) for slice s's q_idx flag of this call; the caller

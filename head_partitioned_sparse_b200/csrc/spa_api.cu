@@ -107,6 +107,7 @@ struct spa_ctx {
   std::vector<int> ev_kid;
   size_t ev_next = 0;
   int64_t launches = 0;
+  int drop_publish = 0;   // failure-detection test hook (spa_debug_drop_publish)
 };
 
 namespace {
@@ -213,6 +214,7 @@ spa_status check_step(spa_ctx* h, const StepArgs& a, spa::StepParams* P) {
   P->idx_scale_log2 = h->idx_scale * 1.4426950408889634f;
   P->attn_scale_log2 = (float)(1.4426950408889634 / std::sqrt(128.0));
   P->split_rows = h->split_rows;
+  P->drop_publish = h->drop_publish;
   P->ws = h->ws;
   return SPA_OK;
 }
@@ -609,6 +611,12 @@ spa_status spa_prefill(spa_handle h, const void* q_chunk, const void* k_cache, c
                                h->cfg.n_kv_heads, h->cfg.max_ctx, n_sink, window, is_ret, h->ws.inv_freq,
                                h->ws.dev_err, st);
   });
+}
+
+spa_status spa_debug_drop_publish(spa_handle h, int enable) {
+  if (!h) return fail(SPA_ERR_INVALID_ARG, "handle is NULL");
+  h->drop_publish = enable ? 1 : 0;
+  return SPA_OK;
 }
 
 spa_status spa_device_status(spa_handle h, spa_stream stream) {

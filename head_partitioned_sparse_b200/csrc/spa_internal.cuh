@@ -131,6 +131,7 @@ struct StepParams {
   int n_str;             // streaming heads (Hkv - n_ret)
   int ring;              // ring rows per streaming head: n_sink + window
   int head_rank[kMaxKvHeads];   // rank of head g among the retrieval or the streaming heads
+  int drop_publish;      // failure-detection test hook: leaders do not publish q_idx
   const void* k_ring;    // [Bm][n_str][ring][128] streaming-head keys (compact layout)
   const void* v_ring;
   Workspace ws;
