@@ -76,6 +76,9 @@ _SIGS = {
     "spa_head_ranks_workspace_size": (_i, [_i, _i, ctypes.POINTER(ctypes.c_size_t)]),
     "spa_head_effective_ranks": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp]),
     "spa_prefill": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp]),
+    "spa_select_compact_sel": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i64, _i, _f, _i64, _i, _i, _vp, _vp, _vp]),
+    "spa_decode_compact_sel": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i64, _i, _f, _i64, _i, _i,
+                                    _vp, _vp, _vp]),
     "spa_device_status": (_i, [_vp, _vp]),
     "spa_debug_drop_publish": (_i, [_vp, _i]),
     "spa_set_profiling": (_i, [_vp, ctypes.c_uint]),
@@ -248,6 +251,24 @@ def spa_prefill(h, q_chunk, k_cache, v_cache, head_mask, start_pos, B: int, T: i
 
 def spa_debug_drop_publish(h, enable: bool) -> None:
     _check(load().spa_debug_drop_publish(h, 1 if enable else 0))
+
+
+SPA_SELECT_TOP_P, SPA_SELECT_TOP_K, SPA_SELECT_BLOCKS = 0, 1, 2
+
+
+def spa_select_compact_sel(h, q_pre, idx_ret, head_mask, seq_lens, B: int, max_seq_len: int, selector: int,
+                           p: float, k: int, n_sink: int, window: int, sel_idx, sel_count, stream=None) -> None:
+    _check(load().spa_select_compact_sel(h, _ptr(q_pre), _ptr(idx_ret), _host_u8(head_mask), _ptr(seq_lens), B,
+                                         max_seq_len, selector, p, int(k), n_sink, window, _ptr(sel_idx),
+                                         _ptr(sel_count), _stream(stream)))
+
+
+def spa_decode_compact_sel(h, q_pre, k_ret, v_ret, k_ring, v_ring, idx_ret, head_mask, seq_lens, B: int,
+                           max_seq_len: int, selector: int, p: float, k: int, n_sink: int, window: int, out,
+                           sel_count_opt=None, stream=None) -> None:
+    _check(load().spa_decode_compact_sel(h, _ptr(q_pre), _ptr(k_ret), _ptr(v_ret), _ptr(k_ring), _ptr(v_ring),
+                                         _ptr(idx_ret), _host_u8(head_mask), _ptr(seq_lens), B, max_seq_len, selector,
+                                         p, int(k), n_sink, window, _ptr(out), _ptr(sel_count_opt), _stream(stream)))
 
 
 def spa_device_status(h, stream=None) -> None:

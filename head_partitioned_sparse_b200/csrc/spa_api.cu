@@ -280,6 +280,54 @@ spa_status decode_with(spa_ctx* h, spa::StepParams& P, const void* k_cache, cons
 }
 
 
+// Selector arguments of the compact entry points: top-p (p), top-k (k), block top-p (p).
+spa_status selector_args(int selector, float p, int64_t k, float* p_out, int64_t* k_out, int* blocks_out) {
+  switch (selector) {
+    case SPA_SELECT_TOP_P: *p_out = p; *k_out = 0; *blocks_out = 0; return SPA_OK;
+    case SPA_SELECT_TOP_K:
+      if (k < 1) return fail(SPA_ERR_INVALID_ARG, "k must be >= 1 (got %lld)", (long long)k);
+      *p_out = 1.f; *k_out = k; *blocks_out = 0; return SPA_OK;
+    case SPA_SELECT_BLOCKS: *p_out = p; *k_out = 0; *blocks_out = 1; return SPA_OK;
+  }
+  return fail(SPA_ERR_INVALID_ARG, "selector must be SPA_SELECT_TOP_P, _TOP_K or _BLOCKS (got %d)", selector);
+}
+
+spa_status select_compact_with(spa_ctx* h, const void* q_pre, const void* idx_ret, const uint8_t* head_mask,
+                               const int64_t* seq_lens, int B, int64_t max_seq_len, int selector, float p, int64_t k,
+                               int n_sink, int window, int32_t* sel_idx, int32_t* sel_count, spa_stream stream) {
+  float pp;
+  int64_t kk;
+  int blocks;
+  spa_status r = selector_args(selector, p, k, &pp, &kk, &blocks);
+  if (r) return r;
+  spa::StepParams P;
+  r = check_step(h, StepArgs{q_pre, idx_ret, head_mask, seq_lens, B, max_seq_len, pp, n_sink, window, kk, blocks}, &P);
+  if (r) return r;
+  if ((r = setup_compact(&P, nullptr, nullptr, false))) return r;
+  return select_with(h, P, sel_idx, sel_count, stream);
+}
+
+spa_status decode_compact_with(spa_ctx* h, const void* q_pre, const void* k_ret, const void* v_ret,
+                               const void* k_ring, const void* v_ring, const void* idx_ret, const uint8_t* head_mask,
+                               const int64_t* seq_lens, int B, int64_t max_seq_len, int selector, float p, int64_t k,
+                               int n_sink, int window, float* out, int32_t* sel_count_opt, spa_stream stream) {
+  float pp;
+  int64_t kk;
+  int blocks;
+  spa_status r = selector_args(selector, p, k, &pp, &kk, &blocks);
+  if (r) return r;
+  spa::StepParams P;
+  r = check_step(h, StepArgs{q_pre, idx_ret, head_mask, seq_lens, B, max_seq_len, pp, n_sink, window, kk, blocks}, &P);
+  if (r) return r;
+  if ((r = setup_compact(&P, k_ring, v_ring, true))) return r;
+  if (P.n_ret == 0) {   // no retrieval head: the retrieval caches are never read
+    static const uint4 dummy[1] = {};
+    if (!k_ret) k_ret = dummy;
+    if (!v_ret) v_ret = dummy;
+  }
+  return decode_with(h, P, k_ret, v_ret, out, sel_count_opt, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -533,27 +581,33 @@ spa_status spa_index_append_compact(spa_handle h, const void* k_pre, const int64
 spa_status spa_select_compact(spa_handle h, const void* q_pre, const void* idx_ret, const uint8_t* head_mask,
                               const int64_t* seq_lens, int B, int64_t max_seq_len, float p, int n_sink, int window,
                               int32_t* sel_idx, int32_t* sel_count, spa_stream stream) {
-  spa::StepParams P;
-  spa_status r = check_step(h, StepArgs{q_pre, idx_ret, head_mask, seq_lens, B, max_seq_len, p, n_sink, window, 0, 0}, &P);
-  if (r) return r;
-  if ((r = setup_compact(&P, nullptr, nullptr, false))) return r;
-  return select_with(h, P, sel_idx, sel_count, stream);
+  return select_compact_with(h, q_pre, idx_ret, head_mask, seq_lens, B, max_seq_len, SPA_SELECT_TOP_P, p, 0, n_sink,
+                             window, sel_idx, sel_count, stream);
 }
 
 spa_status spa_decode_compact(spa_handle h, const void* q_pre, const void* k_ret, const void* v_ret,
                               const void* k_ring, const void* v_ring, const void* idx_ret, const uint8_t* head_mask,
                               const int64_t* seq_lens, int B, int64_t max_seq_len, float p, int n_sink, int window,
                               float* out, int32_t* sel_count_opt, spa_stream stream) {
-  spa::StepParams P;
-  spa_status r = check_step(h, StepArgs{q_pre, idx_ret, head_mask, seq_lens, B, max_seq_len, p, n_sink, window, 0, 0}, &P);
-  if (r) return r;
-  if ((r = setup_compact(&P, k_ring, v_ring, true))) return r;
-  if (P.n_ret == 0) {   // no retrieval head: the retrieval caches are never read
-    static const uint4 dummy[1] = {};
-    if (!k_ret) k_ret = dummy;
-    if (!v_ret) v_ret = dummy;
-  }
-  return decode_with(h, P, k_ret, v_ret, out, sel_count_opt, stream);
+  return decode_compact_with(h, q_pre, k_ret, v_ret, k_ring, v_ring, idx_ret, head_mask, seq_lens, B, max_seq_len,
+                             SPA_SELECT_TOP_P, p, 0, n_sink, window, out, sel_count_opt, stream);
+}
+
+spa_status spa_select_compact_sel(spa_handle h, const void* q_pre, const void* idx_ret, const uint8_t* head_mask,
+                                  const int64_t* seq_lens, int B, int64_t max_seq_len, int selector, float p,
+                                  int64_t k, int n_sink, int window, int32_t* sel_idx, int32_t* sel_count,
+                                  spa_stream stream) {
+  return select_compact_with(h, q_pre, idx_ret, head_mask, seq_lens, B, max_seq_len, selector, p, k, n_sink, window,
+                             sel_idx, sel_count, stream);
+}
+
+spa_status spa_decode_compact_sel(spa_handle h, const void* q_pre, const void* k_ret, const void* v_ret,
+                                  const void* k_ring, const void* v_ring, const void* idx_ret,
+                                  const uint8_t* head_mask, const int64_t* seq_lens, int B, int64_t max_seq_len,
+                                  int selector, float p, int64_t k, int n_sink, int window, float* out,
+                                  int32_t* sel_count_opt, spa_stream stream) {
+  return decode_compact_with(h, q_pre, k_ret, v_ret, k_ring, v_ring, idx_ret, head_mask, seq_lens, B, max_seq_len,
+                             selector, p, k, n_sink, window, out, sel_count_opt, stream);
 }
 
 spa_status spa_head_ranks_workspace_size(int n_q_heads, int n_kv_heads, size_t* bytes) {

@@ -251,6 +251,23 @@ SPA_API spa_status spa_decode_compact(spa_handle h, const void* q_pre, const voi
                       const int64_t* seq_lens, int B, int64_t max_seq_len, float p, int n_sink, int window,
                       float* out, int32_t* sel_count_opt, spa_stream stream);
 
+/* The compact-layout calls with any selector of the full layout:
+ *   SPA_SELECT_TOP_P   p as in spa_select (k unused)
+ *   SPA_SELECT_TOP_K   k as in spa_select_topk (p unused; k >= 1)
+ *   SPA_SELECT_BLOCKS  p as in spa_select_blocks (k unused)
+ * Results equal the full-layout call with the same selector on the same values. */
+#define SPA_SELECT_TOP_P 0
+#define SPA_SELECT_TOP_K 1
+#define SPA_SELECT_BLOCKS 2
+SPA_API spa_status spa_select_compact_sel(spa_handle h, const void* q_pre, const void* idx_ret,
+                      const uint8_t* head_mask, const int64_t* seq_lens, int B, int64_t max_seq_len,
+                      int selector, float p, int64_t k, int n_sink, int window, int32_t* sel_idx,
+                      int32_t* sel_count, spa_stream stream);
+SPA_API spa_status spa_decode_compact_sel(spa_handle h, const void* q_pre, const void* k_ret, const void* v_ret,
+                      const void* k_ring, const void* v_ring, const void* idx_ret, const uint8_t* head_mask,
+                      const int64_t* seq_lens, int B, int64_t max_seq_len, int selector, float p, int64_t k,
+                      int n_sink, int window, float* out, int32_t* sel_count_opt, spa_stream stream);
+
 /* ---- prefill ----
  *
  * Attention of a prefill chunk ("Full Attention Strikes Back" (RTPurbo summary),

@@ -207,3 +207,44 @@ def test_compact_append_rejects_out_of_range_positions():
             B.spa_kv_append_compact(h.h, k, k, start, 1, 8, inp.head_mask, -1, inp.window,
                                     cp.k_ret, cp.v_ret, cp.k_ring, cp.v_ring)
         assert e.value.status == B.SPA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("selector", ["top_k", "blocks"])
+def test_compact_layout_with_other_selectors_matches_full(selector):
+    inp = synth.make_inputs("tiny", 9, overrides={"dtype": "bf16", "B": 2, "L": 6000, "window": 200},
+                            seq_lens=[6000, 4321])
+    ret = [g for g in range(inp.Hkv) if inp.head_mask[g]]
+    idx = oracle_idx(inp, heads=ret)
+    k_budget = 700
+    sel_code = B.SPA_SELECT_TOP_K if selector == "top_k" else B.SPA_SELECT_BLOCKS
+    with Handle(inp) as h:
+        dev = DevInputs(inp, idx)
+        cp = Compact(inp, inp.n_sink, inp.window, fill=float("nan"))
+        for b in range(inp.B):
+            append_sequence(h, inp, dev, cp, b, 0, int(inp.seq_lens[b]), inp.n_sink, inp.window)
+        idx_c = ret_idx(idx, ret, cp)
+        out_full = torch.full((inp.B, inp.Hq, 128), float("nan"), dtype=torch.float32, device="cuda")
+        cnt_full = torch.full((inp.B * inp.Hkv,), -1, dtype=torch.int32, device="cuda")
+        if selector == "top_k":
+            B.spa_decode_topk(h.h, dev.q_pre, dev.k_cache, dev.v_cache, dev.idx, inp.head_mask, dev.seq_lens, inp.B,
+                              0, k_budget, inp.n_sink, inp.window, out_full, cnt_full)
+        else:
+            B.spa_decode_blocks(h.h, dev.q_pre, dev.k_cache, dev.v_cache, dev.idx, inp.head_mask, dev.seq_lens,
+                                inp.B, 0, inp.p, inp.n_sink, inp.window, out_full, cnt_full)
+        out = torch.full_like(out_full, float("nan"))
+        cnt = torch.full_like(cnt_full, -1)
+        B.spa_decode_compact_sel(h.h, dev.q_pre, cp.k_ret, cp.v_ret, cp.k_ring, cp.v_ring, idx_c, inp.head_mask,
+                                 dev.seq_lens, inp.B, 0, sel_code, inp.p, k_budget, inp.n_sink, inp.window, out, cnt)
+        sel = torch.full((inp.B, inp.Hkv, inp.Lmax), -1, dtype=torch.int32, device="cuda")
+        cnt_s = torch.full_like(cnt_full, -1)
+        B.spa_select_compact_sel(h.h, dev.q_pre, idx_c, inp.head_mask, dev.seq_lens, inp.B, 0, sel_code, inp.p,
+                                 k_budget, inp.n_sink, inp.window, sel, cnt_s)
+        torch.cuda.synchronize()
+        B.spa_device_status(h.h)
+        with pytest.raises(B.SpaError) as e:   # a bad selector is refused before any launch
+            B.spa_select_compact_sel(h.h, dev.q_pre, idx_c, inp.head_mask, dev.seq_lens, inp.B, 0, 7, inp.p,
+                                     k_budget, inp.n_sink, inp.window, sel, cnt_s)
+        assert e.value.status == B.SPA_ERR_INVALID_ARG
+    assert np.array_equal(cnt.cpu().numpy(), cnt_full.cpu().numpy())
+    assert np.array_equal(cnt_s.cpu().numpy(), cnt_full.cpu().numpy())
+    assert np.array_equal(out.cpu().numpy(), out_full.cpu().numpy()), "compact must equal full bit for bit"
