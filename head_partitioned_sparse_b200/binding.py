@@ -29,8 +29,10 @@ SPA_ERR_DEVICE_RANGE = -6
 SPA_BF16 = 0
 SPA_F32 = 1
 
-SPA_K_INDEX_APPEND, SPA_K_SELECT, SPA_K_ATTEND, SPA_K_COMBINE, SPA_K_KV_APPEND, SPA_K_PREFILL = range(6)
-SPA_K_COUNT = 6
+SPA_K_INDEX_APPEND, SPA_K_SELECT, SPA_K_ATTEND, SPA_K_COMBINE, SPA_K_KV_APPEND, SPA_K_PREFILL, SPA_K_CP_SELECT = range(7)
+SPA_K_COUNT = 7
+SPA_CP_STATS, SPA_CP_MASS, SPA_CP_ROUND2, SPA_CP_ROUND3, SPA_CP_ATTEND = range(5)
+SPA_CP_NBUF = 6
 
 
 class SpaError(RuntimeError):
@@ -53,6 +55,33 @@ class spa_config(ctypes.Structure):
         ("split_rows", ctypes.c_int),
         ("P_q", ctypes.c_void_p),
         ("P_k", ctypes.c_void_p),
+    ]
+
+
+class spa_cp_args(ctypes.Structure):
+    _fields_ = [
+        ("q_pre", ctypes.c_void_p),
+        ("k_cache", ctypes.c_void_p),
+        ("v_cache", ctypes.c_void_p),
+        ("idx_cache", ctypes.c_void_p),
+        ("head_mask", ctypes.POINTER(ctypes.c_uint8)),
+        ("seq_lens", ctypes.c_void_p),
+        ("B", ctypes.c_int),
+        ("p", ctypes.c_float),
+        ("n_sink", ctypes.c_int),
+        ("window", ctypes.c_int),
+        ("n_ranks", ctypes.c_int),
+        ("rank", ctypes.c_int),
+        ("pos0", ctypes.c_int64),
+        ("max_seq_len", ctypes.c_int64),
+        ("stats", ctypes.c_void_p),
+        ("hist1", ctypes.c_void_p),
+        ("hist2", ctypes.c_void_p),
+        ("hist3", ctypes.c_void_p),
+        ("out_all", ctypes.c_void_p),
+        ("lse_all", ctypes.c_void_p),
+        ("sel_count_opt", ctypes.c_void_p),
+        ("list_opt", ctypes.c_void_p),
     ]
 
 
@@ -79,6 +108,9 @@ _SIGS = {
     "spa_select_compact_sel": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i64, _i, _f, _i64, _i, _i, _vp, _vp, _vp]),
     "spa_decode_compact_sel": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i64, _i, _f, _i64, _i, _i,
                                     _vp, _vp, _vp]),
+    "spa_cp_exchange_sizes": (_i, [_vp, _i, _i, ctypes.POINTER(ctypes.c_size_t)]),
+    "spa_cp_phase": (_i, [_vp, _i, ctypes.POINTER(spa_cp_args), _vp]),
+    "spa_cp_combine": (_i, [_vp, _vp, _vp, _i, _i, _vp, _vp]),
     "spa_device_status": (_i, [_vp, _vp]),
     "spa_debug_drop_publish": (_i, [_vp, _i]),
     "spa_set_profiling": (_i, [_vp, ctypes.c_uint]),
@@ -269,6 +301,34 @@ def spa_decode_compact_sel(h, q_pre, k_ret, v_ret, k_ring, v_ring, idx_ret, head
     _check(load().spa_decode_compact_sel(h, _ptr(q_pre), _ptr(k_ret), _ptr(v_ret), _ptr(k_ring), _ptr(v_ring),
                                          _ptr(idx_ret), _host_u8(head_mask), _ptr(seq_lens), B, max_seq_len, selector,
                                          p, int(k), n_sink, window, _ptr(out), _ptr(sel_count_opt), _stream(stream)))
+
+
+def spa_cp_exchange_sizes(h, B: int, n_ranks: int) -> Tuple[int, ...]:
+    """Byte sizes of the exchange buffers (stats, hist1, hist2, hist3, out_all, lse_all)."""
+    arr = (ctypes.c_size_t * SPA_CP_NBUF)()
+    _check(load().spa_cp_exchange_sizes(h, B, n_ranks, arr))
+    return tuple(int(v) for v in arr)
+
+
+def make_cp_args(*, q_pre, k_cache, v_cache, idx_cache, head_mask, seq_lens, B: int, p: float, n_sink: int,
+                 window: int, n_ranks: int, rank: int, pos0: int, max_seq_len: int, stats, hist1, hist2, hist3,
+                 out_all, lse_all, sel_count_opt=None, list_opt=None) -> spa_cp_args:
+    """The argument block of spa_cp_phase (it keeps the host head mask alive)."""
+    mask = _host_u8(head_mask)
+    a = spa_cp_args(_ptr(q_pre), _ptr(k_cache), _ptr(v_cache), _ptr(idx_cache),
+                    ctypes.cast(mask, ctypes.POINTER(ctypes.c_uint8)), _ptr(seq_lens), B, p, n_sink, window, n_ranks,
+                    rank, int(pos0), int(max_seq_len), _ptr(stats), _ptr(hist1), _ptr(hist2), _ptr(hist3),
+                    _ptr(out_all), _ptr(lse_all), _ptr(sel_count_opt), _ptr(list_opt))
+    a._mask = mask
+    return a
+
+
+def spa_cp_phase(h, phase: int, args: spa_cp_args, stream=None) -> None:
+    _check(load().spa_cp_phase(h, phase, ctypes.byref(args), _stream(stream)))
+
+
+def spa_cp_combine(h, out_all, lse_all, n_ranks: int, B: int, out, stream=None) -> None:
+    _check(load().spa_cp_combine(h, _ptr(out_all), _ptr(lse_all), n_ranks, B, _ptr(out), _stream(stream)))
 
 
 def spa_device_status(h, stream=None) -> None:

@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libspa.so")
 SOURCES = ["spa_api.cu", "k_index_append.cu", "k_kv_append.cu", "k_select.cu", "k_attend.cu", "k_attend_mma.cu",
-           "spa_noalloc.cu", "k_aoh.cu", "k_prefill_tc.cu"]
+           "spa_noalloc.cu", "k_aoh.cu", "k_prefill_tc.cu", "k_cp.cu"]
 HEADERS = ["spa_internal.cuh", os.path.join("..", "..", "include", "spa.h")]
 
 

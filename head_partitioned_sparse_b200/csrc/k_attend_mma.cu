@@ -200,6 +200,7 @@ __device__ void combine_slice(const StepParams& P, int s, int c0, int c1, float*
     const int b = s / P.Hkv, g = s % P.Hkv;
     *reinterpret_cast<float4*>(P.out + ((size_t)b * P.Hq + (size_t)g * G + h) * kHeadDim + 4 * lane) =
         make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
+    if (P.lse && lane == 0) P.lse[(size_t)b * P.Hq + (size_t)g * G + h] = M + log2f(Ls);
   }
   if (threadIdx.x == 0 && P.sel_count) {
     const int g = s % P.Hkv;
@@ -270,6 +271,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
   // CTA whose range starts exactly at a slice boundary writes an empty state into the one
   // slot (its index + s - 1) that the previous slice's range would otherwise skip.
   const long long T = rpre[NS];
+  if (T == 0) return;   // nothing to attend (a context-parallel rank past every sequence)
   const int nb = (long long)gridDim.x < T ? (int)gridDim.x : (int)T;   // active CTAs: >= 1 row each
   const long long r_lo = (long long)blockIdx.x * T / nb, r_hi = blockIdx.x < nb ? (long long)(blockIdx.x + 1) * T / nb : r_lo;
   auto owner = [&](long long r) { return (int)(((r + 1) * nb - 1) / T); };
@@ -342,6 +344,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_attend_bf16(StepParams P) {
 
   for (int ps = s_first; ps <= s_last; ++ps) {
     const ItemInfo it = piece_info(P, rpre, sinfo, r_lo, r_hi, ps);
+    // a slice with no rows (only in context-parallel steps) has no split state, no
+    // ticket and no output here: the list kernel wrote its empty result
+    if (it.v1 <= it.v0) continue;
     if (it.s != cur_slice) {
       cur_slice = it.s;
       const int b = it.s / P.Hkv, g = it.s % P.Hkv;

@@ -328,6 +328,124 @@ spa_status decode_compact_with(spa_ctx* h, const void* q_pre, const void* k_ret,
   return decode_with(h, P, k_ret, v_ret, out, sel_count_opt, stream);
 }
 
+// ---------------------------------------------------------------- context-parallel
+constexpr int kMaxRanks = 1024;
+
+size_t cp_stats_bytes(const spa_ctx* h, int B, int R, int n_chunks) {
+  return (size_t)R * B * h->cfg.n_kv_heads * n_chunks * h->G * sizeof(float2);
+}
+
+spa_status cp_check(spa_ctx* h, const spa_cp_args* a, spa::CpParams* C) {
+  if (!h) return fail(SPA_ERR_INVALID_ARG, "handle is NULL");
+  if (!a) return fail(SPA_ERR_INVALID_ARG, "args is NULL");
+  if (h->cfg.kv_dtype != SPA_BF16) return fail(SPA_ERR_UNSUPPORTED, "context-parallel decode needs bf16 caches");
+  if (h->cfg.max_ctx < 64) return fail(SPA_ERR_INVALID_ARG, "context-parallel decode needs max_ctx >= 64");
+  if (!a->q_pre || !a->k_cache || !a->v_cache || !a->idx_cache || !a->head_mask || !a->seq_lens || !a->stats ||
+      !a->hist1 || !a->hist2 || !a->hist3 || !a->out_all || !a->lse_all)
+    return fail(SPA_ERR_INVALID_ARG, "every pointer of spa_cp_args except sel_count_opt must be non-NULL");
+  if (!aligned16(a->q_pre) || !aligned16(a->k_cache) || !aligned16(a->v_cache) || !aligned16(a->idx_cache) ||
+      !aligned16(a->stats) || !aligned16(a->hist1) || !aligned16(a->hist2) || !aligned16(a->hist3) ||
+      !aligned16(a->out_all) || !aligned16(a->lse_all) || ((uintptr_t)a->seq_lens & 7u) ||
+      ((uintptr_t)a->sel_count_opt & 3u) || !aligned16(a->list_opt))
+    return fail(SPA_ERR_INVALID_ARG, "spa_cp_args pointers must be 16-byte aligned (seq_lens 8, sel_count_opt 4)");
+  if (a->B < 1 || a->B > h->cfg.max_batch)
+    return fail(SPA_ERR_INVALID_ARG, "B must be in [1, max_batch=%d] (got %d)", h->cfg.max_batch, a->B);
+  if (!(a->p > 0.f) || !(a->p <= 1.f)) return fail(SPA_ERR_INVALID_ARG, "p must be in (0, 1] (got %g)", (double)a->p);
+  if (a->n_sink < 0 || a->window < 0 || (int64_t)a->n_sink + a->window < 1)
+    return fail(SPA_ERR_INVALID_ARG, "n_sink, window must be >= 0 with n_sink + window >= 1");
+  if (a->n_ranks < 1 || a->n_ranks > kMaxRanks || a->rank < 0 || a->rank >= a->n_ranks)
+    return fail(SPA_ERR_INVALID_ARG, "need 1 <= n_ranks <= %d and 0 <= rank < n_ranks (got %d, %d)", kMaxRanks,
+                a->n_ranks, a->rank);
+  const int64_t cap = a->max_seq_len ? a->max_seq_len : a->pos0 + h->cfg.max_ctx;
+  if (a->pos0 < 0 || a->pos0 + h->cfg.max_ctx > INT32_MAX || cap < 1 || cap > INT32_MAX)
+    return fail(SPA_ERR_INVALID_ARG, "need pos0 >= 0, pos0 + max_ctx < 2^31 and max_seq_len in [1, 2^31) (got %lld, %lld)",
+                (long long)a->pos0, (long long)cap);
+  std::memset(C, 0, sizeof *C);
+  const int Hkv = h->cfg.n_kv_heads;
+  for (int g = 0; g < Hkv; ++g) C->is_ret[g] = a->head_mask[g] ? 1 : 0;
+  C->q_pre = a->q_pre;
+  C->idx = static_cast<const uint16_t*>(a->idx_cache);
+  C->seq_lens = a->seq_lens;
+  C->B = a->B;
+  C->Hq = h->cfg.n_q_heads;
+  C->Hkv = Hkv;
+  C->G = h->G;
+  C->n_slices = a->B * Hkv;
+  C->C = h->cfg.max_ctx;
+  C->n_chunks = h->n_chunks_max;
+  C->pos0 = a->pos0;
+  C->rank = a->rank;
+  C->n_ranks = a->n_ranks;
+  C->Lcap = (int)cap;
+  C->p = a->p;
+  C->keep_all = a->p >= 1.f ? 1 : 0;
+  C->n_sink = a->n_sink;
+  C->window = a->window;
+  C->idx_scale_log2 = h->idx_scale * 1.4426950408889634f;
+  const spa::Workspace& w = h->ws;
+  C->P_q = w.P_q;
+  C->inv_freq_pi = w.inv_freq;
+  C->q_rot = w.q_rot;
+  C->q_idx = w.q_idx;
+  C->pi = w.pi;
+  C->pi_stride = w.pi_stride;
+  C->stats = static_cast<float2*>(a->stats);
+  C->hist1 = static_cast<unsigned long long*>(a->hist1);
+  C->hist2 = static_cast<unsigned long long*>(a->hist2);
+  C->hist3 = static_cast<unsigned long long*>(a->hist3);
+  // the one-GPU selection's candidate buffer and round-2 histogram are free during a
+  // context-parallel step: they hold the per-chunk round-3 counts and the cut states
+  // (max_ctx >= 64 makes [slices][n_chunks][64] counts fit in [slices][max_ctx] uint2)
+  C->tab3 = reinterpret_cast<unsigned*>(w.cand);
+  C->cs = reinterpret_cast<spa::CpSlice*>(w.hist2);
+  C->chunk_cnt = w.chunk_gt;
+  C->list = a->list_opt ? a->list_opt : w.list;
+  C->st = w.st;
+  C->sel_count = a->sel_count_opt;
+  C->out_rank = a->out_all + (size_t)a->rank * a->B * C->Hq * spa::kHeadDim;
+  C->lse_rank = a->lse_all + (size_t)a->rank * a->B * C->Hq;
+  C->err = w.dev_err;
+  return SPA_OK;
+}
+
+// Attention over the rank's listed rows: every slice gathers (no contiguous rows).
+spa_status cp_attend(spa_ctx* h, const spa_cp_args* a, const spa::CpParams& C, cudaStream_t st) {
+  spa::StepParams P;
+  std::memset(&P, 0, sizeof P);
+  P.q_pre = a->q_pre;
+  P.k_cache = a->k_cache;
+  P.v_cache = a->v_cache;
+  P.idx_cache = C.idx;
+  P.seq_lens = a->seq_lens;
+  P.out = C.out_rank;
+  P.lse = C.lse_rank;
+  P.sel_list = C.list;
+  P.sel_count = nullptr;
+  P.B = C.B;
+  P.Hq = C.Hq;
+  P.Hkv = C.Hkv;
+  P.G = C.G;
+  P.Lmax = h->cfg.max_ctx;
+  P.Lcap = C.Lcap;
+  P.n_slices = C.n_slices;
+  P.p = 1.f;
+  P.n_sink = 0;    // sinks and window are in the lists
+  P.window = 0;
+  P.attn_scale_log2 = (float)(1.4426950408889634 / std::sqrt(128.0));
+  P.split_rows = h->split_rows;
+  for (int g = 0; g < C.Hkv; ++g) {
+    P.is_ret[g] = 1;
+    P.ret_heads[P.n_ret++] = g;
+  }
+  P.ws = h->ws;
+  const int64_t per_slice = (h->cfg.max_ctx + P.split_rows - 1) / P.split_rows;
+  const int64_t max_items = per_slice * P.n_slices;
+  int64_t cap = (int64_t)h->num_sms * h->attend_occ;
+  if (cap > spa::kMaxAttendCtas) cap = spa::kMaxAttendCtas;
+  const int grid = (int)(max_items < cap ? max_items : cap);
+  return run(h, SPA_K_ATTEND, st, "cp attend", [&] { return spa::launch_attend_bf16(P, grid, st); });
+}
+
 }  // namespace
 
 extern "C" {
@@ -667,6 +785,69 @@ spa_status spa_prefill(spa_handle h, const void* q_chunk, const void* k_cache, c
   });
 }
 
+spa_status spa_cp_exchange_sizes(spa_handle h, int B, int n_ranks, size_t* bytes) {
+  if (!h || !bytes) return fail(SPA_ERR_INVALID_ARG, "NULL argument");
+  if (B < 1 || B > h->cfg.max_batch)
+    return fail(SPA_ERR_INVALID_ARG, "B must be in [1, max_batch=%d] (got %d)", h->cfg.max_batch, B);
+  if (n_ranks < 1 || n_ranks > kMaxRanks) return fail(SPA_ERR_INVALID_ARG, "n_ranks must be in [1, %d]", kMaxRanks);
+  const size_t slices = (size_t)B * h->cfg.n_kv_heads, rows = (size_t)B * h->cfg.n_q_heads;
+  bytes[0] = cp_stats_bytes(h, B, n_ranks, h->n_chunks_max);
+  bytes[1] = (size_t)n_ranks * slices * spa::kBins1 * 8;
+  bytes[2] = (size_t)n_ranks * slices * spa::kBins2 * 8;
+  bytes[3] = (size_t)n_ranks * slices * spa::kBins3 * 16;
+  bytes[4] = (size_t)n_ranks * rows * spa::kHeadDim * 4;
+  bytes[5] = (size_t)n_ranks * rows * 4;
+  return SPA_OK;
+}
+
+spa_status spa_cp_phase(spa_handle h, int phase, const spa_cp_args* a, spa_stream stream) {
+  spa::CpParams C;
+  spa_status r = cp_check(h, a, &C);
+  if (r) return r;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t slices = (size_t)C.n_slices;
+  cudaError_t e;
+  switch (phase) {
+    case SPA_CP_STATS:
+      return run(h, SPA_K_CP_SELECT, st, "cp stats", [&] { return spa::launch_cp_stats(C, st); });
+    case SPA_CP_MASS:
+      if ((e = cudaMemsetAsync(C.hist1 + (size_t)C.rank * slices * spa::kBins1, 0, slices * spa::kBins1 * 8, st)))
+        return cuda_fail(e, "cp clear hist1");
+      return run(h, SPA_K_CP_SELECT, st, "cp mass", [&] { return spa::launch_cp_mass(C, st); });
+    case SPA_CP_ROUND2:
+      if ((r = run(h, SPA_K_CP_SELECT, st, "cp cut 1", [&] { return spa::launch_cp_cut(C, 1, st); }))) return r;
+      if ((e = cudaMemsetAsync(C.hist2 + (size_t)C.rank * slices * spa::kBins2, 0, slices * spa::kBins2 * 8, st)))
+        return cuda_fail(e, "cp clear hist2");
+      return run(h, SPA_K_CP_SELECT, st, "cp round 2", [&] { return spa::launch_cp_hist(C, 2, st); });
+    case SPA_CP_ROUND3:
+      if ((r = run(h, SPA_K_CP_SELECT, st, "cp cut 2", [&] { return spa::launch_cp_cut(C, 2, st); }))) return r;
+      if ((e = cudaMemsetAsync(C.hist3 + (size_t)C.rank * slices * spa::kBins3 * 2, 0, slices * spa::kBins3 * 16, st)))
+        return cuda_fail(e, "cp clear hist3");
+      return run(h, SPA_K_CP_SELECT, st, "cp round 3", [&] { return spa::launch_cp_hist(C, 3, st); });
+    case SPA_CP_ATTEND:
+      if ((r = run(h, SPA_K_CP_SELECT, st, "cp cut 3", [&] { return spa::launch_cp_cut(C, 3, st); }))) return r;
+      if ((r = run(h, SPA_K_CP_SELECT, st, "cp list count", [&] { return spa::launch_cp_list(C, 0, st); }))) return r;
+      if ((r = run(h, SPA_K_CP_SELECT, st, "cp list", [&] { return spa::launch_cp_list(C, 1, st); }))) return r;
+      return cp_attend(h, a, C, st);
+  }
+  return fail(SPA_ERR_INVALID_ARG, "phase must be SPA_CP_STATS .. SPA_CP_ATTEND (got %d)", phase);
+}
+
+spa_status spa_cp_combine(spa_handle h, const float* out_all, const float* lse_all, int n_ranks, int B, float* out,
+                          spa_stream stream) {
+  if (!h) return fail(SPA_ERR_INVALID_ARG, "handle is NULL");
+  if (!out_all || !lse_all || !out) return fail(SPA_ERR_INVALID_ARG, "out_all, lse_all and out must be non-NULL");
+  if (!aligned16(out_all) || !aligned16(lse_all) || !aligned16(out))
+    return fail(SPA_ERR_INVALID_ARG, "out_all, lse_all and out must be 16-byte aligned");
+  if (B < 1 || B > h->cfg.max_batch)
+    return fail(SPA_ERR_INVALID_ARG, "B must be in [1, max_batch=%d] (got %d)", h->cfg.max_batch, B);
+  if (n_ranks < 1 || n_ranks > kMaxRanks) return fail(SPA_ERR_INVALID_ARG, "n_ranks must be in [1, %d]", kMaxRanks);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int rows = B * h->cfg.n_q_heads;
+  return run(h, SPA_K_COMBINE, st, "cp combine",
+             [&] { return spa::launch_cp_combine(out_all, lse_all, n_ranks, rows, out, st); });
+}
+
 spa_status spa_debug_drop_publish(spa_handle h, int enable) {
   if (!h) return fail(SPA_ERR_INVALID_ARG, "handle is NULL");
   h->drop_publish = enable ? 1 : 0;
@@ -735,7 +916,8 @@ spa_status spa_profile_read(spa_handle h, int kernel_id, double* total_ms, int64
 }
 
 const char* spa_kernel_name(int kernel_id) {
-  static const char* names[SPA_K_COUNT] = {"index_append", "select", "attend", "combine", "kv_append", "prefill"};
+  static const char* names[SPA_K_COUNT] = {"index_append", "select", "attend", "combine", "kv_append", "prefill",
+                                            "cp_select"};
   return (kernel_id >= 0 && kernel_id < SPA_K_COUNT) ? names[kernel_id] : "";
 }
 

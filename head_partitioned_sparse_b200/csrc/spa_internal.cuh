@@ -73,6 +73,54 @@ struct __align__(16) SliceState {
   unsigned qidx_ready;          // barrier generation + 1 once this call's q_idx is stored
 };
 
+// Cut state of one (b, kv head) slice in a context-parallel step (each rank holds a
+// contiguous run of the slice's positions).  Written by the cut kernels, read by the
+// histogram and list kernels of the following phases.
+struct __align__(16) CpSlice {
+  unsigned long long target;   // ceil(p * total mass), total over every rank
+  unsigned long long above;    // mass of all tokens strictly above the current digit prefix
+  int b1, b2;                  // round-1 / round-2 bins; b1 = -1 keeps every token
+  unsigned tau;                // fp32 bits of the cut probability (after round 3)
+  int quota;                   // tokens at tau this rank keeps (its lowest positions first)
+};
+
+// Arguments of the context-parallel kernels of one phase on one rank.
+struct CpParams {
+  const void* q_pre;              // [B][Hq][128] bf16, identical on every rank
+  const uint16_t* idx;            // local index rows [Bm][Hkv][C][16]
+  const int64_t* seq_lens;        // [B] global sequence lengths
+  int B, Hq, Hkv, G, n_slices;
+  int64_t C;                      // local row capacity (row stride of the local caches)
+  int n_chunks;                   // ceil(C / kChunk): chunks of a slice's local rows
+  int64_t pos0;                   // global position of local row 0
+  int rank, n_ranks;
+  int Lcap;                       // largest global sequence length accepted
+  float p;
+  int keep_all;                   // p >= 1
+  int n_sink, window;
+  float idx_scale_log2;
+  unsigned char is_ret[kMaxKvHeads];
+  const float* P_q;               // [Hq][16][128]
+  const double* inv_freq_pi;      // [64] RoPE inverse frequencies / pi
+  float* q_rot;                   // [Bm][Hq][128]
+  float* q_idx;                   // [Bm][Hq][16]
+  float* pi;                      // [Bm*Hkv][pi_stride] local probabilities
+  int64_t pi_stride;
+  float2* stats;                  // exchange: [R][n_slices][n_chunks][G] (m in log2 units, z)
+  unsigned long long* hist1;      // exchange: [R][n_slices][kBins1] masses
+  unsigned long long* hist2;      // exchange: [R][n_slices][kBins2] masses
+  unsigned long long* hist3;      // exchange: [R][n_slices][kBins3][2] (mass, count)
+  unsigned* tab3;                 // [n_slices][n_chunks][kBins3] local round-3 counts per chunk
+  int* chunk_cnt;                 // [n_slices][n_chunks] listed rows per chunk
+  CpSlice* cs;                    // [n_slices]
+  int* list;                      // [n_slices][C] listed local rows, ascending
+  SliceState* st;                 // .count: listed rows of the slice (read by attention)
+  int* sel_count;                 // optional [n_slices]
+  float* out_rank;                // this rank's attention output slot [B][Hq][128]
+  float* lse_rank;                // [B][Hq] log2-sum-exp of the rank's scores
+  unsigned* err;
+};
+
 __host__ __device__ inline int64_t pi_row_stride(int64_t Lmax) { return (Lmax + 63) / 64 * 64; }
 
 // Device workspace carved out of one allocation.
@@ -134,6 +182,7 @@ struct StepParams {
   int drop_publish;      // failure-detection test hook: leaders do not publish q_idx
   const void* k_ring;    // [Bm][n_str][ring][128] streaming-head keys (compact layout)
   const void* v_ring;
+  float* lse;            // optional [B][Hq]: log2-sum-exp of each head's attended scores
   Workspace ws;
 };
 
@@ -277,6 +326,14 @@ size_t head_rank_workspace_bytes(int Hq, int Hkv);
 cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, float* out, const int64_t* start, int B,
                               int T, int Hq, int Hkv, int64_t Lmax, int n_sink, int window,
                               const unsigned char* is_ret, const double* inv_freq_pi, unsigned* err, cudaStream_t st);
+// Context-parallel phases (k_cp.cu).
+cudaError_t launch_cp_stats(const CpParams& P, cudaStream_t st);
+cudaError_t launch_cp_mass(const CpParams& P, cudaStream_t st);
+cudaError_t launch_cp_cut(const CpParams& P, int round, cudaStream_t st);
+cudaError_t launch_cp_hist(const CpParams& P, int round, cudaStream_t st);
+cudaError_t launch_cp_list(const CpParams& P, int pass, cudaStream_t st);
+cudaError_t launch_cp_combine(const float* out_all, const float* lse_all, int n_ranks, int rows, float* out,
+                              cudaStream_t st);
 cudaError_t launch_head_ranks(const float* W_Q, const float* W_K, int Hq, int Hkv, int d_model, int n_ret,
                               void* ws, double* er_q, double* er_kv, unsigned char* mask, double* sigma,
                               int* sweeps, cudaStream_t st);

@@ -293,6 +293,77 @@ SPA_API spa_status spa_prefill(spa_handle h, const void* q_chunk, const void* k_
                       const uint8_t* head_mask, const int64_t* start_pos, int B, int T, int n_sink,
                       int window, float* out, spa_stream stream);
 
+/* ---- context-parallel decode ----
+ *
+ * One decode step of long sequences whose positions are split over n_ranks ranks
+ * (one process per GPU, or several handles on one GPU): rank r holds the contiguous run
+ * of global positions [pos0, pos0 + max_ctx) of every sequence in its own caches, local
+ * row i = global position pos0 + i (the usual split is pos0 = r * max_ctx, every rank's
+ * handle created with the same configuration).  The result is the step spa_decode
+ * computes over the whole context ("Full Attention Strikes Back" (RTPurbo summary),
+ * Methodology §2, §3, §5; split over the context as in the context-parallel scaling of
+ * the "Lighthouse Attention" summary, Experimental results): the top-p set of each
+ * retrieval group is taken over all ranks' tokens, ties at the cut go to the lowest
+ * positions, sinks and window are global positions.  Top-p with bf16 caches only.
+ *
+ * The step is five phases, SPA_CP_STATS .. SPA_CP_ATTEND, run in order on every rank,
+ * each followed by an all-gather (NCCL or any other transport; on one GPU, emulated
+ * ranks share the buffers and need none) of the rank's slot of the buffer it wrote:
+ *   SPA_CP_STATS   per-head (max, sum of exp) of the local index scores -> stats
+ *   SPA_CP_MASS    local probabilities; round-1 mass histogram           -> hist1
+ *   SPA_CP_ROUND2  cut of round 1 (all ranks' hist1); round-2 histogram  -> hist2
+ *   SPA_CP_ROUND3  cut of round 2; round-3 histogram with counts         -> hist3
+ *   SPA_CP_ATTEND  final cut and this rank's share of the ties; attention over the
+ *                  local kept rows                                        -> out_all, lse_all
+ * then spa_cp_combine merges the ranks' outputs.  Histogram masses are integers, so
+ * every rank reaches the same cut.  Each exchange buffer is [n_ranks][...] with the
+ * rank's slot at index rank; a phase writes only its own slot (clearing it first) and
+ * reads the other slots, which must hold the gathered data of the previous phase.
+ * spa_cp_exchange_sizes gives the byte size of each buffer (all slots).  Every pointer
+ * is a device pointer, 16-byte aligned.  Phases and combine only enqueue work on
+ * `stream`; a phase called out of order computes garbage but stays in bounds. */
+#define SPA_CP_STATS 0
+#define SPA_CP_MASS 1
+#define SPA_CP_ROUND2 2
+#define SPA_CP_ROUND3 3
+#define SPA_CP_ATTEND 4
+#define SPA_CP_NBUF 6     /* stats, hist1, hist2, hist3, out_all, lse_all */
+typedef struct {
+  const void* q_pre;        /* bf16 [B][Hq][128] pre-RoPE queries, the same on every rank */
+  const void* k_cache;      /* bf16 [max_batch][Hkv][max_ctx][128] local post-RoPE keys */
+  const void* v_cache;      /* bf16 [max_batch][Hkv][max_ctx][128] local values */
+  const void* idx_cache;    /* bf16 [max_batch][Hkv][max_ctx][16] local index rows */
+  const uint8_t* head_mask; /* host [Hkv], 1 = retrieval head */
+  const int64_t* seq_lens;  /* device [B] GLOBAL lengths (the current token at L - 1) */
+  int B;
+  float p;                  /* in (0, 1] */
+  int n_sink, window;       /* >= 0, n_sink + window >= 1 */
+  int n_ranks, rank;        /* 1 <= n_ranks <= 1024, 0 <= rank < n_ranks */
+  int64_t pos0;             /* global position of local row 0, >= 0 */
+  int64_t max_seq_len;      /* bound on the global lengths (0: pos0 + max_ctx) */
+  void* stats;              /* [n_ranks][B][Hkv][ceil(max_ctx / 4096)][G] float2 */
+  void* hist1;              /* [n_ranks][B][Hkv][4096] uint64 */
+  void* hist2;              /* [n_ranks][B][Hkv][4096] uint64 */
+  void* hist3;              /* [n_ranks][B][Hkv][64][2] uint64 */
+  float* out_all;           /* [n_ranks][B][Hq][128] float32 */
+  float* lse_all;           /* [n_ranks][B][Hq] float32, log2 of the softmax denominator */
+  int32_t* sel_count_opt;   /* NULL or device [B][Hkv]: local rows attended (SPA_CP_ATTEND) */
+  int32_t* list_opt;        /* NULL or device [B][Hkv][max_ctx]: the local rows attended, ascending
+                               (sinks and window included; global position = pos0 + row) */
+} spa_cp_args;
+/* bytes[i] for the SPA_CP_NBUF buffers in spa_cp_args order.  Errors: NULL handle or
+ * bytes, B outside [1, max_batch], n_ranks outside [1, 1024]. */
+SPA_API spa_status spa_cp_exchange_sizes(spa_handle h, int B, int n_ranks, size_t* bytes);
+/* Runs one phase on this rank.  Errors: SPA_ERR_INVALID_ARG for a NULL or misaligned
+ * pointer, an unknown phase, B / p / n_sink / window / rank / pos0 out of range, or
+ * max_ctx < 64; SPA_ERR_UNSUPPORTED for float32 caches. */
+SPA_API spa_status spa_cp_phase(spa_handle h, int phase, const spa_cp_args* a, spa_stream stream);
+/* out[b][h] = sum_r 2^(lse_r - M) out_r / sum_r 2^(lse_r - M), M = max_r lse_r, over
+ * the gathered out_all / lse_all (ranks in order; a rank with lse = -inf attended
+ * nothing for that head).  out: device float32 [B][Hq][128]. */
+SPA_API spa_status spa_cp_combine(spa_handle h, const float* out_all, const float* lse_all, int n_ranks, int B,
+                      float* out, spa_stream stream);
+
 /* ---- head labels from frozen weights ----
  *
  * "Autonomy of Heads" summary, Methodology §1-§4: the effective rank of each query
@@ -346,7 +417,8 @@ SPA_API spa_status spa_debug_drop_publish(spa_handle h, int enable);
 #define SPA_K_COMBINE 3
 #define SPA_K_KV_APPEND 4
 #define SPA_K_PREFILL 5
-#define SPA_K_COUNT 6
+#define SPA_K_CP_SELECT 6   /* context-parallel selection phases (every kernel of them) */
+#define SPA_K_COUNT 7
 
 /* kernel_mask = 0 disables timing.  Otherwise every launch of a kernel whose bit
  * (1 << SPA_K_...) is set is bracketed by two CUDA events recorded on the launch

@@ -78,3 +78,144 @@ def test_two_rank_decode_gathers_to_the_single_process_result():
     assert err == 0.0
     assert t == 2.0
     assert all(p.exitcode == 0 for p in procs)
+
+
+# ------------------------------------------------------------------ context-parallel exchange
+# The phases of a context-parallel step run in a host model (cp_host_model) that reads
+# and writes the exchange buffers in libspa's layout; the orchestration and the
+# all-gathers are the package's own.  Rank r holds positions [r C, (r + 1) C).
+CP_CASE = dict(name="tiny", seed=5, overrides={"B": 3, "L": 9000, "window": 64, "p": 0.9}, seq_lens=[9000, 4700, 90])
+CP_C = 4500
+
+
+def _cp_inputs():
+    import oracle as O
+    from head_partitioned_sparse_b200 import synth
+    inp = synth.make_inputs(CP_CASE["name"], CP_CASE["seed"], overrides=CP_CASE["overrides"],
+                            seq_lens=CP_CASE["seq_lens"])
+    idx = O.index_cache_for(inp, heads=[g for g in range(inp.Hkv) if inp.head_mask[g]])
+    return inp, idx
+
+
+def _cp_check(inp, idx, out, rows):
+    """Union of the ranks' rows = the oracle's sets (band 1e-5 around p); output = the
+    oracle on those rows."""
+    import oracle as O
+    _, res = O.decode_inputs(inp, idx_cache=idx)
+    listed = {}
+    for b in range(inp.B):
+        sw = O.sink_window(int(inp.seq_lens[b]), inp.n_sink, inp.window)
+        for g in range(inp.Hkv):
+            got = rows[(b, g)]
+            assert np.all(np.diff(got) > 0)
+            if not inp.head_mask[g]:
+                assert np.array_equal(got, sw)
+                continue
+            assert np.isin(sw, got).all()
+            listed[(b, g)] = np.setdiff1d(got, sw)
+            diff = np.setxor1d(listed[(b, g)], res[(b, g)].listed)
+            assert np.all(np.abs(res[(b, g)].topp.c_before[diff] - inp.p) <= 1e-5)
+    ref, _ = O.decode_inputs(inp, idx_cache=idx, attend_sets=listed)
+    return float(np.abs(out - ref).max())
+
+
+def test_cp_phases_emulated_in_one_process_match_the_oracle():
+    import torch
+    import cp_host_model as M
+    from head_partitioned_sparse_b200 import context_parallel as cp
+    inp, idx = _cp_inputs()
+    R = 3
+    C = -(-int(inp.seq_lens.max()) // R)
+    bufs = {n: torch.zeros(sz, dtype=torch.uint8) for n, sz in
+            zip(cp.BUFFERS, M.exchange_sizes(inp.B, inp.Hq, inp.Hkv, C, R))}
+    ranks = [M.HostRank(inp, idx, r, R, C, bufs, p=inp.p, n_sink=inp.n_sink, window=inp.window) for r in range(R)]
+    cp.run_step(range(R), lambda ph, r: ranks[r].phase(ph), lambda name: None)
+    out = M.combine(ranks[0].out_all, ranks[0].lse_all)
+    rows = {k: np.concatenate([rk.rows[k] for rk in ranks]) for k in ranks[0].rows}
+    assert _cp_check(inp, idx, out, rows) <= 1e-5
+
+
+def _cp_worker(rank, world, port, q):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import cp_host_model as M
+    from head_partitioned_sparse_b200 import context_parallel as cp
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    try:
+        dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+        inp, idx = _cp_inputs()
+        bufs = {n: torch.zeros(sz, dtype=torch.uint8) for n, sz in
+                zip(cp.BUFFERS, M.exchange_sizes(inp.B, inp.Hq, inp.Hkv, CP_C, world))}
+        me = M.HostRank(inp, idx, rank, world, CP_C, bufs, p=inp.p, n_sink=inp.n_sink, window=inp.window)
+        cp.run_step([rank], lambda ph, r: me.phase(ph), lambda name: cp.allgather_slot(bufs[name], world, rank))
+        out = M.combine(me.out_all, me.lse_all)
+        # every rank holds the same combined output; rows are gathered to rank 0
+        gathered = [None] * world
+        dist.all_gather_object(gathered, {k: v.tolist() for k, v in me.rows.items()})
+        outs = [None] * world
+        dist.all_gather_object(outs, out.tolist())
+        if rank == 0:
+            rows = {k: np.concatenate([np.asarray(gathered[r][k], np.int64) for r in range(world)])
+                    for k in gathered[0]}
+            err = _cp_check(inp, idx, out, rows)
+            same = all(np.array_equal(np.asarray(o), out) for o in outs)
+            # the same phases emulated in one process give the same bits
+            ebufs = {n: torch.zeros(sz, dtype=torch.uint8) for n, sz in
+                     zip(cp.BUFFERS, M.exchange_sizes(inp.B, inp.Hq, inp.Hkv, CP_C, world))}
+            er = [M.HostRank(inp, idx, r, world, CP_C, ebufs, p=inp.p, n_sink=inp.n_sink, window=inp.window)
+                  for r in range(world)]
+            cp.run_step(range(world), lambda ph, r: er[r].phase(ph), lambda name: None)
+            emu = M.combine(er[0].out_all, er[0].lse_all)
+            hist_same = all(torch.equal(bufs[n], ebufs[n]) for n in cp.BUFFERS)
+            q.put(("ok", err, same and np.array_equal(emu, out) and hist_same))
+        dist.barrier()
+        dist.destroy_process_group()
+    except Exception as e:  # report to the parent instead of hanging it
+        q.put(("err", repr(e), None))
+        raise
+
+
+def test_cp_two_rank_gloo_exchange_matches_oracle_and_emulation():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_cp_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=300)
+    alive = [p for p in procs if p.is_alive()]
+    for p in alive:
+        p.kill()
+    assert not alive, "a rank did not finish"
+    status, err, same = q.get(timeout=5)
+    assert status == "ok", err
+    assert err <= 1e-5
+    assert same, "the gloo run and the one-process emulation differ"
+    assert all(p.exitcode == 0 for p in procs)
+
+
+def test_cp_phases_ties_across_ranks_go_to_the_lowest_positions():
+    """Identical index rows (pi = 1/L everywhere): the kept ties are the lowest positions
+    of the whole context, so rank 0 keeps all of its rows, rank 1 a prefix, rank 2 none."""
+    import torch
+    import cp_host_model as M
+    import oracle as O
+    from head_partitioned_sparse_b200 import context_parallel as cp
+    from head_partitioned_sparse_b200 import synth
+    inp = synth.make_inputs("tiny", 8, overrides={"L": 1000, "window": 8, "p": float(np.float32(0.7005))})
+    idx = O.index_cache_for(inp, heads=[0])
+    idx[0, 0, :1000] = idx[0, 0, 500]
+    R, C = 3, 400
+    bufs = {n: torch.zeros(sz, dtype=torch.uint8) for n, sz in
+            zip(cp.BUFFERS, M.exchange_sizes(inp.B, inp.Hq, inp.Hkv, C, R))}
+    ranks = [M.HostRank(inp, idx, r, R, C, bufs, p=inp.p, n_sink=inp.n_sink, window=8) for r in range(R)]
+    cp.run_step(range(R), lambda ph, r: ranks[r].phase(ph), lambda name: None)
+    sw = O.sink_window(1000, inp.n_sink, 8)
+    kept = np.setdiff1d(np.concatenate([rk.rows[(0, 0)] for rk in ranks]), sw)
+    assert np.array_equal(kept, np.setdiff1d(np.arange(701), sw))
+    assert len(ranks[2].rows[(0, 0)]) == len(np.intersect1d(sw, np.arange(800, 1000)))
