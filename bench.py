@@ -61,6 +61,8 @@ def parse_args():
     ap.add_argument("--no-compact", action="store_true", help="skip the compact KV layout measurement")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill measurement")
     ap.add_argument("--prefill-len", type=int, default=32768, help="prefill chunk length (from position 0)")
+    ap.add_argument("--no-cp", action="store_true", help="skip the context-parallel measurement")
+    ap.add_argument("--cp-ranks", type=int, default=4, help="ranks of the context-parallel measurement")
     ap.add_argument("--override", action="append", default=[], metavar="KEY=VALUE",
                     help="replace a workload field (e.g. B=1 for a small profiling case)")
     return ap.parse_args()
@@ -471,6 +473,76 @@ def main_native(args):
                            "for streaming heads; bf16 inputs, float32 accumulation (tcgen05 MMA, TMEM accumulators)"}
         del q_chunk, out_p, kc, vc
 
+    # context-parallel decode of the same step: the positions split over cp_ranks ranks,
+    # emulated on this GPU (one handle and one cache shard per rank, the phases run rank
+    # after rank, exchange buffers shared: no transfer is timed).  Reported: each rank's
+    # kernel time per step (CUDA events around each of its launches), the whole emulated
+    # step, the bytes each rank would all-gather, and agreement with the one-GPU step.
+    cpar = None
+    if not args.no_cp and inp.dtype == "bf16" and args.cp_ranks >= 1:
+        from head_partitioned_sparse_b200 import context_parallel as cpm
+        R = args.cp_ranks
+        C = -(-inp.Lmax // R)          # rows per rank, rounded up to 64
+        C = -(-C // 64) * 64
+        k0_, v0_, ix0_ = layers[0]
+        cp_handles, shards = [], []
+        for r in range(R):
+            cp_handles.append(B.spa_create(B.make_config(
+                max_batch=inp.B, n_q_heads=inp.Hq, n_kv_heads=inp.Hkv, max_ctx=C, kv_dtype=B.SPA_BF16, P_q=P_q,
+                P_k=P_k, rope_theta=inp.rope_theta, idx_scale=inp.idx_scale, split_rows=args.split_rows)))
+            lo, hi = r * C, min((r + 1) * C, inp.Lmax)
+
+            def sl(t):
+                z = torch.zeros((inp.B, inp.Hkv, C) + tuple(t.shape[3:]), dtype=t.dtype, device=dev)
+                if hi > lo:
+                    z[:, :, :hi - lo] = t[:, :, lo:hi]
+                return z
+            shards.append({"k": sl(k0_), "v": sl(v0_), "idx": sl(ix0_)})
+        out_cp = torch.empty_like(out)
+        cp_bufs = cpm.alloc_exchange(B.spa_cp_exchange_sizes(cp_handles[0], inp.B, R), dev)
+
+        def step_cp(i):
+            cpm.emulated_step(cp_handles, shards, q_pre=q, head_mask=head_mask, seq_lens=lens, Bsz=inp.B, p=p,
+                              n_sink=inp.n_sink, window=inp.window, capacity=C, out=out_cp, bufs=cp_bufs,
+                              max_seq_len=Lcap, stream=stream)
+        for i in range(3):
+            step_cp(i)
+        for hh in cp_handles:
+            B.spa_device_status(hh, stream)
+        n = max(10, args.steps // 10)
+        ms_cp, _ = timed(n, step_cp)
+        ms_cp = shard.reduce_max(ms_cp, dev) / n
+        mask_cp = (1 << B.SPA_K_CP_SELECT) | (1 << B.SPA_K_ATTEND) | (1 << B.SPA_K_COMBINE)
+        for hh in cp_handles:
+            B.spa_set_profiling(hh, mask_cp)
+        timed(n, step_cp)
+        rank_us, sel_us, att_us = [], [], []
+        for hh in cp_handles:
+            ts, _ = B.spa_profile_read(hh, B.SPA_K_CP_SELECT)
+            ta, _ = B.spa_profile_read(hh, B.SPA_K_ATTEND)
+            sel_us.append(1e3 * ts / n)
+            att_us.append(1e3 * ta / n)
+            rank_us.append(1e3 * (ts + ta) / n)
+        tc, _ = B.spa_profile_read(cp_handles[0], B.SPA_K_COMBINE)
+        for hh in cp_handles:
+            B.spa_set_profiling(hh, 0)
+        B.spa_decode(h, q, k0_, v0_, ix0_, head_mask, lens, inp.B, Lcap, p, inp.n_sink, inp.window, out, None,
+                     stream)
+        step_cp(0)
+        torch.cuda.synchronize(dev)
+        sizes = B.spa_cp_exchange_sizes(cp_handles[0], inp.B, R)
+        cpar = {"ranks": R, "rows_per_rank": C, "emulated_step_ms": ms_cp,
+                "rank_kernel_us": rank_us, "rank_select_us": sel_us, "rank_attend_us": att_us,
+                "max_rank_kernel_us": max(rank_us), "combine_us": 1e3 * tc / n,
+                "exchange_bytes_per_rank": int(sum(sizes) // R),
+                "one_gpu_step_ms": ms_per_step,
+                "max_abs_vs_one_gpu": float((out_cp - out).abs().max().item()),
+                "note": "ranks emulated on one GPU one after another; a rank's kernel time is what it "
+                        "spends on its own GPU per step, without the four all-gathers"}
+        for hh in cp_handles:
+            B.spa_destroy(hh)
+        del shards, cp_bufs, out_cp
+
     # end to end through the public API: pinned host inputs in, result out, every step.
     # Every step copies its own inputs (query, new pre-RoPE key, positions, new K/V rows)
     # from pinned host memory and reads its output back.  The copies run on a copy
@@ -589,6 +661,7 @@ def main_native(args):
             "block_sweep": block_sweep or None,
             "compact": compact,
             "prefill": prefill,
+            "context_parallel": cpar,
         }
         print(json.dumps(line), flush=True)
     B.spa_destroy(h)
