@@ -501,10 +501,10 @@ def main_native(args):
         out_cp = torch.empty_like(out)
         cp_bufs = cpm.alloc_exchange(B.spa_cp_exchange_sizes(cp_handles[0], inp.B, R), dev)
 
-        def step_cp(i):
+        def step_cp(i, st=stream, ranks=None, combine=True):
             cpm.emulated_step(cp_handles, shards, q_pre=q, head_mask=head_mask, seq_lens=lens, Bsz=inp.B, p=p,
                               n_sink=inp.n_sink, window=inp.window, capacity=C, out=out_cp, bufs=cp_bufs,
-                              max_seq_len=Lcap, stream=stream)
+                              max_seq_len=Lcap, stream=st, ranks=ranks, combine=combine)
         for i in range(3):
             step_cp(i)
         for hh in cp_handles:
@@ -530,15 +530,52 @@ def main_native(args):
                      stream)
         step_cp(0)
         torch.cuda.synchronize(dev)
+        # device time alone: each rank's launches (and the whole emulated step) captured
+        # in a CUDA graph and replayed, so no host launch gap is timed
+        def graph_of(fn):
+            g = torch.cuda.CUDAGraph()
+            cap = torch.cuda.Stream(device=dev)
+            cap.wait_stream(stream)
+            with torch.cuda.graph(g, stream=cap):
+                fn()
+            torch.cuda.synchronize(dev)
+            return g
+
+        def replay_us(g, reps):
+            torch.cuda.synchronize(dev)
+            a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                g.replay()
+            z.record(stream)
+            torch.cuda.synchronize(dev)
+            return 1e3 * a.elapsed_time(z) / reps
+
+        graph_step_us, graph_rank_us, graph_err = None, [], None
+        try:
+            g_all = graph_of(lambda: step_cp(0, st=None))
+            graph_step_us = replay_us(g_all, n)
+            del g_all
+            for r in range(R):
+                g_r = graph_of(lambda: step_cp(0, st=None, ranks=[r], combine=False))
+                graph_rank_us.append(replay_us(g_r, n))
+                del g_r
+        except Exception as e:   # reported, not fatal: the step itself was timed above
+            graph_err = repr(e)[:200]
+        step_cp(0)
+        torch.cuda.synchronize(dev)
         sizes = B.spa_cp_exchange_sizes(cp_handles[0], inp.B, R)
         cpar = {"ranks": R, "rows_per_rank": C, "emulated_step_ms": ms_cp,
+                "graph_step_us": graph_step_us, "graph_rank_us": graph_rank_us,
+                "max_graph_rank_us": max(graph_rank_us) if graph_rank_us else None, "graph_error": graph_err,
                 "rank_kernel_us": rank_us, "rank_select_us": sel_us, "rank_attend_us": att_us,
                 "max_rank_kernel_us": max(rank_us), "combine_us": 1e3 * tc / n,
                 "exchange_bytes_per_rank": int(sum(sizes) // R),
                 "one_gpu_step_ms": ms_per_step,
                 "max_abs_vs_one_gpu": float((out_cp - out).abs().max().item()),
-                "note": "ranks emulated on one GPU one after another; a rank's kernel time is what it "
-                        "spends on its own GPU per step, without the four all-gathers"}
+                "note": "ranks emulated on one GPU one after another, exchanges not timed (buffers shared); "
+                        "rank_*_us: CUDA events around each launch of a Python-driven step (host gaps "
+                        "included); graph_*_us: the same launches replayed from a CUDA graph (device time)"}
         for hh in cp_handles:
             B.spa_destroy(hh)
         del shards, cp_bufs, out_cp

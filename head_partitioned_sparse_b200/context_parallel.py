@@ -115,10 +115,13 @@ class ContextParallelDecoder:
 
 def emulated_step(handles: Sequence, shards: Sequence[dict], *, q_pre, head_mask, seq_lens, Bsz: int, p: float,
                   n_sink: int, window: int, capacity: int, out, bufs=None, max_seq_len: int = 0,
-                  sel_counts: Sequence = None, lists: Sequence = None, stream=None) -> dict:
+                  sel_counts: Sequence = None, lists: Sequence = None, stream=None, ranks: Sequence[int] = None,
+                  combine: bool = True) -> dict:
     """All ranks of a context-parallel step on one GPU: handles[r] and shards[r] (dict of
     ``k``, ``v``, ``idx`` device tensors) are rank r's.  Returns the exchange buffers
-    (reusable for the next call through ``bufs``)."""
+    (reusable for the next call through ``bufs``).  ``ranks`` restricts the phases to
+    some ranks (to time one rank's share: the other slots of ``bufs`` must then hold an
+    earlier step's exchanged data); ``combine=False`` skips the final merge."""
     R = len(handles)
     if bufs is None:
         bufs = alloc_exchange(spa.spa_cp_exchange_sizes(handles[0], Bsz, R), q_pre.device)
@@ -133,6 +136,8 @@ def emulated_step(handles: Sequence, shards: Sequence[dict], *, q_pre, head_mask
             hist2=bufs["hist2"], hist3=bufs["hist3"], out_all=out_all, lse_all=lse_all,
             sel_count_opt=None if sel_counts is None else sel_counts[r],
             list_opt=None if lists is None else lists[r]))
-    run_step(range(R), lambda phase, r: spa.spa_cp_phase(handles[r], phase, args[r], stream), lambda name: None)
-    spa.spa_cp_combine(handles[0], out_all, lse_all, R, Bsz, out, stream)
+    run_step(range(R) if ranks is None else ranks, lambda phase, r: spa.spa_cp_phase(handles[r], phase, args[r], stream),
+             lambda name: None)
+    if combine:
+        spa.spa_cp_combine(handles[0], out_all, lse_all, R, Bsz, out, stream)
     return bufs

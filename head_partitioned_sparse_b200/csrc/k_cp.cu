@@ -37,6 +37,11 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr int kThreads = 256;
 constexpr int kWarpsPerCta = kThreads / 32;
 constexpr int kRun = kChunk / kThreads;   // 16 consecutive rows per thread in the list passes
+// The two passes over the index rows run 512 threads per chunk, each with all of its
+// 8 rows in flight at once (the passes are bound by memory latency, not bandwidth).
+constexpr int kRowThreads = 512;
+constexpr int kRowWarps = kRowThreads / 32;
+constexpr int kRowsPer = kChunk / kRowThreads;   // 8
 
 // 2^x with the hardware approximation (relative error about 2^-22; 2^-inf = 0), used by
 // both passes over the index rows so that the sums and the probabilities agree.
@@ -110,7 +115,7 @@ __device__ void rope_heads(const CpParams& P, const __nv_bfloat16* q, int b, int
     sincospi(r, &sn[tid], &cs[tid]);
   }
   __syncthreads();
-  for (int t = tid; t < G * (kHeadDim / 2); t += kThreads) {
+  for (int t = tid; t < G * (kHeadDim / 2); t += blockDim.x) {
     const int h = t / (kHeadDim / 2), i = t % (kHeadDim / 2);
     const double x1 = __bfloat162float(q[h * kHeadDim + i]);
     const double x2 = __bfloat162float(q[h * kHeadDim + i + kHeadDim / 2]);
@@ -127,7 +132,7 @@ __device__ void rope_heads(const CpParams& P, const __nv_bfloat16* q, int b, int
 template <int G>
 __device__ void qidx_heads(const CpParams& P, const __nv_bfloat16* q, int g, float* qsm) {
   const int tid = threadIdx.x;
-  for (int w = tid; w < G * kIdxDim * 4; w += kThreads) {   // whole warps (G * 64 = 64k)
+  for (int w = tid; w < G * kIdxDim * 4; w += blockDim.x) {   // whole warps (G * 64 = 64k)
     const int o = w >> 2, qd = w & 3, h = o / kIdxDim;
     const float4* prow = reinterpret_cast<const float4*>(P.P_q + ((size_t)g * G * kIdxDim + o) * kHeadDim + 32 * qd);
     const uint4* qrow = reinterpret_cast<const uint4*>(q + h * kHeadDim + 32 * qd);
@@ -174,51 +179,63 @@ __device__ __forceinline__ void row_logits(const uint4& a, const uint4& c, const
 }
 
 // ------------------------------------------------------------------ phase: stats
-// grid (n_chunks, n_slices).  Chunk 0 of every slice (streaming ones included) writes
-// q_rot; the chunks of retrieval slices write their (m, z) to stats[rank].
+// Loads a thread's kRowsPer index rows of chunk c (row j0 + u * kRowThreads + tid).
+__device__ __forceinline__ void load_rows(const uint16_t* rows, long long j0, long long n, uint4 (&ra)[kRowsPer],
+                                          uint4 (&rc)[kRowsPer], bool last_use) {
+  const int tid = threadIdx.x;
+#pragma unroll
+  for (int u = 0; u < kRowsPer; ++u) {
+    const long long j = j0 + (long long)u * kRowThreads + tid;
+    if (j < n) {
+      const uint4* r = reinterpret_cast<const uint4*>(rows + (size_t)j * kIdxDim);
+      if (last_use) {
+        ra[u] = __ldcs(r);
+        rc[u] = __ldcs(r + 1);
+      } else {
+        ra[u] = __ldg(r);
+        rc[u] = __ldg(r + 1);
+      }
+    }
+  }
+}
+
+// grid (n_chunks, n_slices), kRowThreads threads.  Chunk 0 of every slice (streaming
+// ones included) writes q_rot; the chunks of retrieval slices write their (m, z) to
+// stats[rank].  The rows are requested before the query prologue so that the two
+// overlap; this pass keeps their lines in L2 for the mass pass.
 template <int G>
-__global__ void __launch_bounds__(kThreads) k_cp_stats(CpParams P) {
+__global__ void __launch_bounds__(kRowThreads) k_cp_stats(CpParams P) {
   __shared__ float qsm[G * kIdxDim];
   __shared__ double cs[kHeadDim / 2], sn[kHeadDim / 2];
-  __shared__ float2 wred[kWarpsPerCta][G];
+  __shared__ float2 wred[kRowWarps][G];
   __shared__ int sh_len;
   const int c = blockIdx.x, s = blockIdx.y, b = s / P.Hkv, g = s % P.Hkv, tid = threadIdx.x;
+  const long long j0 = (long long)c * kChunk;
+  uint4 ra[kRowsPer], rc[kRowsPer];
+  // rows are requested before the sequence length is known: every row below C lies in
+  // the shard; rows at or past the local length are ignored below
+  if (P.is_ret[g]) load_rows(P.idx + (size_t)s * P.C * kIdxDim, j0, P.C, ra, rc, false);
   const int L = cta_len(P, b, &sh_len);
   const __nv_bfloat16* q = (const __nv_bfloat16*)P.q_pre + ((size_t)b * P.Hq + (size_t)g * G) * kHeadDim;
+  const long long n = P.is_ret[g] ? local_rows(P, L) : 0;
   if (c == 0) rope_heads<G>(P, q, b, g, L, cs, sn);
   if (!P.is_ret[g]) return;
   qidx_heads<G>(P, q, g, qsm);
   if (c == 0 && tid < G * kIdxDim) P.q_idx[((size_t)b * P.Hq + (size_t)g * G) * kIdxDim + tid] = qsm[tid];
 
-  const long long n = local_rows(P, L);
-  const long long j0 = (long long)c * kChunk;
-  const uint16_t* rows = P.idx + (size_t)s * P.C * kIdxDim;
   float m[G], z[G];
 #pragma unroll
   for (int h = 0; h < G; ++h) { m[h] = -INFINITY; z[h] = 0.f; }
-  constexpr int kBatch = 4;
-  for (int k0 = 0; k0 < kChunk / kThreads; k0 += kBatch) {
-    uint4 ra[kBatch], rc[kBatch];
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const long long j = j0 + (long long)(k0 + u) * kThreads + tid;
-      if (j < n) {
-        const uint4* r = reinterpret_cast<const uint4*>(rows + (size_t)j * kIdxDim);
-        ra[u] = __ldg(r);
-        rc[u] = __ldg(r + 1);
-      }
-    }
+  for (int u = 0; u < kRowsPer; ++u) {
+    const long long j = j0 + (long long)u * kRowThreads + tid;
+    if (j < n) {
+      float l[G];
+      row_logits<G>(ra[u], rc[u], qsm, P.idx_scale_log2, l);
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const long long j = j0 + (long long)(k0 + u) * kThreads + tid;
-      if (j < n) {
-        float l[G];
-        row_logits<G>(ra[u], rc[u], qsm, P.idx_scale_log2, l);
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          if (l[h] > m[h]) { z[h] = z[h] * ex2(m[h] - l[h]) + 1.f; m[h] = l[h]; }
-          else z[h] += ex2(l[h] - m[h]);
-        }
+      for (int h = 0; h < G; ++h) {
+        if (l[h] > m[h]) { z[h] = z[h] * ex2(m[h] - l[h]) + 1.f; m[h] = l[h]; }
+        else z[h] += ex2(l[h] - m[h]);
       }
     }
   }
@@ -238,31 +255,36 @@ __global__ void __launch_bounds__(kThreads) k_cp_stats(CpParams P) {
   __syncthreads();
   if (tid < G) {
     float M = -INFINITY, Z = 0.f;
-    for (int w = 0; w < kWarpsPerCta; ++w) merge_mz(M, Z, wred[w][tid].x, wred[w][tid].y);
+    for (int w = 0; w < kRowWarps; ++w) merge_mz(M, Z, wred[w][tid].x, wred[w][tid].y);
     P.stats[(((size_t)P.rank * P.n_slices + s) * P.n_chunks + c) * G + tid] = make_float2(M, Z);
   }
 }
 
 // ------------------------------------------------------------------ phase: mass
-// grid (n_chunks, n_slices), retrieval slices only.  Shared histogram of the round-1
-// digit as a count and a sum of the low 18 significand bits per bin (32-bit atomics);
-// bin1_mass turns them into the exact mass.
+// grid (n_chunks, n_slices), kRowThreads threads, retrieval slices only.  Shared
+// histogram of the round-1 digit as a count and a sum of the low 18 significand bits
+// per bin (32-bit atomics); bin1_mass turns them into the exact mass.
 template <int G>
-__global__ void __launch_bounds__(kThreads) k_cp_mass(CpParams P) {
+__global__ void __launch_bounds__(kRowThreads) k_cp_mass(CpParams P) {
   __shared__ unsigned hc[kBins1], hl[kBins1];
   __shared__ float qsm[G * kIdxDim];
-  __shared__ float2 wred[kWarpsPerCta];
+  __shared__ float2 wred[kRowWarps];
   __shared__ float Msm[G], Wsm[G];
   __shared__ int sh_len;
   const int c = blockIdx.x, s = blockIdx.y, b = s / P.Hkv, g = s % P.Hkv, tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   if (!P.is_ret[g]) return;
+  const long long j0 = (long long)c * kChunk;
+  uint4 ra[kRowsPer], rc[kRowsPer];
+  // second and last read of the rows (requested before the length is known, as above)
+  load_rows(P.idx + (size_t)s * P.C * kIdxDim, j0, P.C, ra, rc, true);
   const int L = cta_len(P, b, &sh_len);
-  for (int i = tid; i < kBins1; i += kThreads) { hc[i] = 0u; hl[i] = 0u; }
+  const long long n = local_rows(P, L);
+  for (int i = tid; i < kBins1; i += kRowThreads) { hc[i] = 0u; hl[i] = 0u; }
   if (tid < G * kIdxDim) qsm[tid] = P.q_idx[((size_t)b * P.Hq + (size_t)g * G) * kIdxDim + tid];
-  // (M_h, Z_h): warp w merges head w % G over entries w / G, w / G + 8 / G, ... (all
+  // (M_h, Z_h): warp w merges head w % G over entries w / G, w / G + kWph, ... (all
   // ranks' chunks in rank-major order), then the warps of a head are merged in order.
-  constexpr int kWph = kWarpsPerCta / G;   // warps per head
+  constexpr int kWph = kRowWarps / G;   // warps per head
   const int E = P.n_ranks * P.n_chunks;
   {
     const int h = warp % G, sub = warp / G;
@@ -288,45 +310,29 @@ __global__ void __launch_bounds__(kThreads) k_cp_mass(CpParams P) {
   }
   __syncthreads();
 
-  const long long n = local_rows(P, L);
-  const long long j0 = (long long)c * kChunk;
-  const uint16_t* rows = P.idx + (size_t)s * P.C * kIdxDim;
   float* pi = P.pi + (size_t)s * P.pi_stride;
   float Mh[G], Wh[G];
 #pragma unroll
   for (int h = 0; h < G; ++h) { Mh[h] = Msm[h]; Wh[h] = Wsm[h]; }
-  constexpr int kBatch = 4;
-  for (int k0 = 0; k0 < kChunk / kThreads; k0 += kBatch) {
-    uint4 ra[kBatch], rc[kBatch];
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const long long j = j0 + (long long)(k0 + u) * kThreads + tid;
-      if (j < n) {
-        const uint4* r = reinterpret_cast<const uint4*>(rows + (size_t)j * kIdxDim);
-        ra[u] = __ldcs(r);
-        rc[u] = __ldcs(r + 1);
-      }
-    }
+  for (int u = 0; u < kRowsPer; ++u) {
+    const long long j = j0 + (long long)u * kRowThreads + tid;
+    if (j < n) {
+      float l[G];
+      row_logits<G>(ra[u], rc[u], qsm, P.idx_scale_log2, l);
+      float v = 0.f;
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const long long j = j0 + (long long)(k0 + u) * kThreads + tid;
-      if (j < n) {
-        float l[G];
-        row_logits<G>(ra[u], rc[u], qsm, P.idx_scale_log2, l);
-        float v = 0.f;
-#pragma unroll
-        for (int h = 0; h < G; ++h) v = fmaf(ex2(l[h] - Mh[h]), Wh[h], v);
-        pi[j] = v;
-        const unsigned bits = __float_as_uint(v);
-        const unsigned d = min(bits >> 18, (unsigned)kBins1 - 1u);   // probabilities are <= 1: clamp is inert
-        atomicAdd(&hc[d], 1u);
-        atomicAdd(&hl[d], bits & 0x3ffffu);
-      }
+      for (int h = 0; h < G; ++h) v = fmaf(ex2(l[h] - Mh[h]), Wh[h], v);
+      pi[j] = v;
+      const unsigned bits = __float_as_uint(v);
+      const unsigned d = min(bits >> 18, (unsigned)kBins1 - 1u);   // probabilities are <= 1: clamp is inert
+      atomicAdd(&hc[d], 1u);
+      atomicAdd(&hl[d], bits & 0x3ffffu);
     }
   }
   __syncthreads();
   unsigned long long* dst = P.hist1 + ((size_t)P.rank * P.n_slices + s) * kBins1;
-  for (int d = tid; d < kBins1; d += kThreads) {
+  for (int d = tid; d < kBins1; d += kRowThreads) {
     const unsigned cnt = hc[d];
     if (cnt) {
       const unsigned long long ms = bin1_mass((unsigned)d, cnt, hl[d]);
@@ -336,20 +342,28 @@ __global__ void __launch_bounds__(kThreads) k_cp_mass(CpParams P) {
 }
 
 // ------------------------------------------------------------------ cuts
-// Descending scan of NB bins h (shared memory): the bin d with
+// Shared-memory slot of bin d of a 4096-bin histogram: one pad word per 16 bins, so the
+// 16 consecutive bins a thread scans in cut_desc do not share a bank with its neighbours'.
+__device__ __forceinline__ int hslot(int d) { return d + (d >> 4); }
+constexpr int kHistSlots = kBins1 + kBins1 / 16;
+
+// Descending scan of NB bins h (shared memory, slot PAD ? hslot(d) : d): the bin d with
 // above + mass(bins > d) < target <= above + mass(bins >= d).  Thread t owns bins
 // NB-1-t*PER .. NB-PER-t*PER.  Result in *out_b / *out_above (untouched if target is
 // never reached).  Ends with a CTA barrier.
-template <int NB>
+template <int NB, bool PAD>
 __device__ void cut_desc(const unsigned long long* h, unsigned long long above, unsigned long long target, int* out_b,
                          unsigned long long* out_above, unsigned long long* scratch) {
   constexpr int PER = NB >= kThreads ? NB / kThreads : 1;
   const int tid = threadIdx.x;
   const bool owns = tid * PER < NB;
+  unsigned long long v[PER];
   unsigned long long mine = 0ull;
-  if (owns) {
 #pragma unroll
-    for (int k = 0; k < PER; ++k) mine += h[NB - 1 - tid * PER - k];
+  for (int k = 0; k < PER; ++k) {
+    const int d = NB - 1 - tid * PER - k;
+    v[k] = owns ? h[PAD ? hslot(d) : d] : 0ull;
+    mine += v[k];
   }
   unsigned long long total;
   const unsigned long long before = block_excl_scan<unsigned long long>(mine, scratch, &total);
@@ -357,20 +371,52 @@ __device__ void cut_desc(const unsigned long long* h, unsigned long long above, 
     unsigned long long cum = above + before;
 #pragma unroll
     for (int k = 0; k < PER; ++k) {
-      const int d = NB - 1 - tid * PER - k;
-      const unsigned long long nx = cum + h[d];
-      if (cum < target && nx >= target) { *out_b = d; *out_above = cum; }
+      const unsigned long long nx = cum + v[k];
+      if (cum < target && nx >= target) { *out_b = NB - 1 - tid * PER - k; *out_above = cum; }
       cum = nx;
     }
   }
   __syncthreads();
 }
 
+// Sum over the ranks of a [R][n_slices][4096] histogram, slice s, into shared memory
+// (padded slots); returns this thread's part of the total.  Each thread keeps its 16
+// bins' loads of one rank in flight together.
+__device__ unsigned long long gather_hist4096(const unsigned long long* hist, int R, int n_slices, int s,
+                                              unsigned long long* h) {
+  constexpr int PER = kBins1 / kThreads;
+  const int tid = threadIdx.x;
+  unsigned long long v[PER];
+#pragma unroll
+  for (int k = 0; k < PER; ++k) v[k] = 0ull;
+  constexpr int kRanksAtOnce = 4;   // 64 loads per thread in flight
+  for (int r0 = 0; r0 < R; r0 += kRanksAtOnce) {
+    unsigned long long w[kRanksAtOnce][PER];
+#pragma unroll
+    for (int i = 0; i < kRanksAtOnce; ++i) {
+      const unsigned long long* src = hist + ((size_t)(r0 + i) * n_slices + s) * kBins1 + tid;
+#pragma unroll
+      for (int k = 0; k < PER; ++k) w[i][k] = r0 + i < R ? __ldcg(src + k * kThreads) : 0ull;
+    }
+#pragma unroll
+    for (int i = 0; i < kRanksAtOnce; ++i)
+#pragma unroll
+      for (int k = 0; k < PER; ++k) v[k] += w[i][k];
+  }
+  unsigned long long mine = 0ull;
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    h[hslot(tid + k * kThreads)] = v[k];
+    mine += v[k];
+  }
+  return mine;
+}
+
 // grid (n_slices).  round 1: total mass and target from the summed round-1 histograms,
 // then bin b1; round 2: bin b2 inside b1; round 3: bin b3, tau and this rank's quota of
 // the tokens at tau.
 __global__ void __launch_bounds__(kThreads) k_cp_cut(CpParams P, int round) {
-  __shared__ unsigned long long h[kBins1];
+  __shared__ unsigned long long h[kHistSlots];
   __shared__ unsigned long long cnt3[kBins3];
   __shared__ unsigned long long scratch[kWarpsPerCta];
   __shared__ int sb;
@@ -380,21 +426,14 @@ __global__ void __launch_bounds__(kThreads) k_cp_cut(CpParams P, int round) {
   CpSlice* cs = P.cs + s;
   const int R = P.n_ranks;
   if (round == 1) {
-    for (int d = tid; d < kBins1; d += kThreads) {
-      unsigned long long v = 0ull;
-      for (int r = 0; r < R; ++r) v += __ldcg(P.hist1 + ((size_t)r * P.n_slices + s) * kBins1 + d);
-      h[d] = v;
-    }
-    __syncthreads();
-    unsigned long long mine = 0ull;
-    for (int d = tid; d < kBins1; d += kThreads) mine += h[d];
-    const unsigned long long total = block_sum<unsigned long long>(mine, scratch);
+    const unsigned long long mine = gather_hist4096(P.hist1, R, P.n_slices, s, h);
+    const unsigned long long total = block_sum<unsigned long long>(mine, scratch);   // (barrier: h complete)
     unsigned long long target = (unsigned long long)ceil((double)P.p * (double)total);
     if (target < 1ull) target = 1ull;
     const bool keep = P.keep_all || target > total;
     if (tid == 0) { sb = -1; sabove = 0ull; }
     __syncthreads();
-    if (!keep) cut_desc<kBins1>(h, 0ull, target, &sb, &sabove, scratch);
+    if (!keep) cut_desc<kBins1, true>(h, 0ull, target, &sb, &sabove, scratch);
     if (tid == 0) {
       cs->target = target;
       cs->above = sabove;
@@ -409,14 +448,10 @@ __global__ void __launch_bounds__(kThreads) k_cp_cut(CpParams P, int round) {
   if (b1 < 0) return;
   const unsigned long long target = __ldcg(&cs->target), above = __ldcg(&cs->above);
   if (round == 2) {
-    for (int d = tid; d < kBins2; d += kThreads) {
-      unsigned long long v = 0ull;
-      for (int r = 0; r < R; ++r) v += __ldcg(P.hist2 + ((size_t)r * P.n_slices + s) * kBins2 + d);
-      h[d] = v;
-    }
+    gather_hist4096(P.hist2, R, P.n_slices, s, h);
     if (tid == 0) { sb = -1; sabove = above; }
     __syncthreads();
-    cut_desc<kBins2>(h, above, target, &sb, &sabove, scratch);
+    cut_desc<kBins2, true>(h, above, target, &sb, &sabove, scratch);
     if (tid == 0) {
       if (sb < 0) atomicOr(P.err, kErrInternal);
       cs->b2 = sb < 0 ? 0 : sb;
@@ -438,7 +473,7 @@ __global__ void __launch_bounds__(kThreads) k_cp_cut(CpParams P, int round) {
   }
   if (tid == 0) { sb = -1; sabove = above; }
   __syncthreads();
-  cut_desc<kBins3>(h, above, target, &sb, &sabove, scratch);
+  cut_desc<kBins3, false>(h, above, target, &sb, &sabove, scratch);
   if (tid == 0) {
     int b3 = sb;
     if (b3 < 0) { atomicOr(P.err, kErrInternal); b3 = 0; }
@@ -469,22 +504,28 @@ __global__ void __launch_bounds__(kThreads) k_cp_hist(CpParams P, int round) {
   if (!P.is_ret[g]) return;
   const CpSlice* cs = P.cs + s;
   const int b1 = __ldcg(&cs->b1);
-  if (b1 < 0) return;
   const int b2 = __ldcg(&cs->b2);
   const int L = cta_len(P, b, &sh_len);
-  const int nb = round == 2 ? kBins2 : kBins3;
-  for (int i = tid; i < nb; i += kThreads) hm[i] = 0ull;
-  if (round == 3 && tid < kBins3) hn[tid] = 0u;
-  __syncthreads();
+  if (b1 < 0) return;
   const long long n = local_rows(P, L);
   const long long j0 = (long long)c * kChunk;
   const unsigned* pb = reinterpret_cast<const unsigned*>(P.pi + (size_t)s * P.pi_stride);
   const unsigned pre2 = (unsigned)b1, pre3 = ((unsigned)b1 << 12) | (unsigned)b2;
   bool any = false;
-  for (int k = 0; k < kChunk / kThreads; ++k) {
+  constexpr int PER = kChunk / kThreads;
+  unsigned uv[PER];   // all of the thread's probabilities in flight at once; ~0u never matches a prefix
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
     const long long j = j0 + (long long)k * kThreads + tid;
-    if (j >= n) break;
-    const unsigned u = __ldcg(pb + j);
+    uv[k] = j < n ? __ldcg(pb + j) : ~0u;
+  }
+  const int nb = round == 2 ? kBins2 : kBins3;
+  for (int i = tid; i < nb; i += kThreads) hm[i] = 0ull;
+  if (round == 3 && tid < kBins3) hn[tid] = 0u;
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const unsigned u = uv[k];
     if (round == 2) {
       if ((u >> 18) == pre2) {
         atomicAdd(&hm[(u >> 6) & 0xfffu], mass_q(u));
@@ -517,50 +558,54 @@ __global__ void __launch_bounds__(kThreads) k_cp_hist(CpParams P, int round) {
 // Returns the 16-bit mask; needs the CTA (block scans of the tied rows).
 __device__ unsigned list_mask(const CpParams& P, int s, int c, int L, unsigned* uscratch) {
   const int g = s % P.Hkv, tid = threadIdx.x;
+  const bool ret = P.is_ret[g] != 0;
   const long long n = local_rows(P, L);
   const long long r0 = (long long)c * kChunk + (long long)tid * kRun;
+  // issue every load first: the cut state, the thread's 16 probabilities (r0 is a
+  // multiple of 16 rows: four aligned 16-byte words), the earlier chunks' tie counts
+  int b1 = -1, quota = 0;
+  unsigned tau = 0u;
+  uint4 pw[kRun / 4];
+  if (ret) {
+    b1 = __ldcg(&P.cs[s].b1);
+    tau = __ldcg(&P.cs[s].tau);
+    quota = __ldcg(&P.cs[s].quota);
+    const uint4* pv = reinterpret_cast<const uint4*>(P.pi + (size_t)s * P.pi_stride + r0);
+#pragma unroll
+    for (int q4 = 0; q4 < kRun / 4; ++q4) pw[q4] = r0 < n ? __ldcg(pv + q4) : make_uint4(0u, 0u, 0u, 0u);
+  }
   const SinkWindow sw(L, P.n_sink, P.window);
   unsigned mask = 0u;
-  int b1 = -1;
-  if (P.is_ret[g]) b1 = __ldcg(&P.cs[s].b1);
-  const bool ret = P.is_ret[g] != 0;
-  if (ret && b1 < 0) {   // keep everything local
-#pragma unroll
-    for (int k = 0; k < kRun; ++k)
-      if (r0 + k < n) mask |= 1u << k;
-    return mask;
-  }
 #pragma unroll
   for (int k = 0; k < kRun; ++k) {
     const long long r = r0 + k;
     if (r < n && sw.always((int)(P.pos0 + r))) mask |= 1u << k;
   }
   if (!ret) return mask;
-  const unsigned tau = __ldcg(&P.cs[s].tau);
-  const int quota = __ldcg(&P.cs[s].quota);
+  if (b1 < 0) {   // keep everything local
+#pragma unroll
+    for (int k = 0; k < kRun; ++k)
+      if (r0 + k < n) mask |= 1u << k;
+    return mask;
+  }
   const unsigned b3 = tau & 0x3fu;
   // tied rows of the earlier chunks of this slice (local to the rank)
   unsigned earlier = 0u;
   for (int cc = tid; cc < c; cc += kThreads) earlier += __ldcg(P.tab3 + ((size_t)s * P.n_chunks + cc) * kBins3 + b3);
-  earlier = block_sum<unsigned>(earlier, uscratch);
-  const unsigned* pb = reinterpret_cast<const unsigned*>(P.pi + (size_t)s * P.pi_stride);
   unsigned gt = 0u, eq = 0u;
-  if (r0 < n) {
-    const uint4* pv = reinterpret_cast<const uint4*>(pb + r0);   // r0 is a multiple of 16 rows
 #pragma unroll
-    for (int q4 = 0; q4 < kRun / 4; ++q4) {
-      const uint4 w = __ldcg(pv + q4);
-      const unsigned v[4] = {w.x, w.y, w.z, w.w};
+  for (int q4 = 0; q4 < kRun / 4; ++q4) {
+    const unsigned v[4] = {pw[q4].x, pw[q4].y, pw[q4].z, pw[q4].w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int k = 4 * q4 + i;
-        if (r0 + k < n) {
-          if (v[i] > tau) gt |= 1u << k;
-          else if (v[i] == tau) eq |= 1u << k;
-        }
+    for (int i = 0; i < 4; ++i) {
+      const int k = 4 * q4 + i;
+      if (r0 + k < n) {
+        if (v[i] > tau) gt |= 1u << k;
+        else if (v[i] == tau) eq |= 1u << k;
       }
     }
   }
+  earlier = block_sum<unsigned>(earlier, uscratch);
   unsigned n_eq_total;
   const unsigned before = earlier + block_excl_scan<unsigned>((unsigned)__popc(eq), uscratch, &n_eq_total);
   unsigned kept_eq = 0u, seen = before;
@@ -642,10 +687,10 @@ __global__ void __launch_bounds__(32) k_cp_combine(const float* out_all, const f
 cudaError_t launch_cp_stats(const CpParams& P, cudaStream_t st) {
   const dim3 grid(P.n_chunks, P.n_slices);
   switch (P.G) {
-    case 1: k_cp_stats<1><<<grid, kThreads, 0, st>>>(P); break;
-    case 2: k_cp_stats<2><<<grid, kThreads, 0, st>>>(P); break;
-    case 4: k_cp_stats<4><<<grid, kThreads, 0, st>>>(P); break;
-    case 8: k_cp_stats<8><<<grid, kThreads, 0, st>>>(P); break;
+    case 1: k_cp_stats<1><<<grid, kRowThreads, 0, st>>>(P); break;
+    case 2: k_cp_stats<2><<<grid, kRowThreads, 0, st>>>(P); break;
+    case 4: k_cp_stats<4><<<grid, kRowThreads, 0, st>>>(P); break;
+    case 8: k_cp_stats<8><<<grid, kRowThreads, 0, st>>>(P); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -654,10 +699,10 @@ cudaError_t launch_cp_stats(const CpParams& P, cudaStream_t st) {
 cudaError_t launch_cp_mass(const CpParams& P, cudaStream_t st) {
   const dim3 grid(P.n_chunks, P.n_slices);
   switch (P.G) {
-    case 1: k_cp_mass<1><<<grid, kThreads, 0, st>>>(P); break;
-    case 2: k_cp_mass<2><<<grid, kThreads, 0, st>>>(P); break;
-    case 4: k_cp_mass<4><<<grid, kThreads, 0, st>>>(P); break;
-    case 8: k_cp_mass<8><<<grid, kThreads, 0, st>>>(P); break;
+    case 1: k_cp_mass<1><<<grid, kRowThreads, 0, st>>>(P); break;
+    case 2: k_cp_mass<2><<<grid, kRowThreads, 0, st>>>(P); break;
+    case 4: k_cp_mass<4><<<grid, kRowThreads, 0, st>>>(P); break;
+    case 8: k_cp_mass<8><<<grid, kRowThreads, 0, st>>>(P); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
