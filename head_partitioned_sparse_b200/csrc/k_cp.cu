@@ -10,7 +10,8 @@
 //   the context-parallel scaling of the "Lighthouse Attention" summary, Experimental
 //   results (1M tokens on 32 GPUs).
 //
-// Phases (per rank; the exchange after each one is an all-gather of the rank's slot):
+// Phases (per rank; the exchange after each one is an all-gather of the rank's slot; the
+// histogram rows a phase adds into were cleared by an earlier phase of the same rank):
 //   stats   q_rot = RoPE(q_pre, L-1); q_idx = P_q q_pre (float64 dots); per chunk of
 //           local rows and head h: m = max_j l_hj, z = sum_j 2^(l_hj - m),
 //           l_hj = log2(e) idx_scale <q_idx[h], idx_j>                    -> stats[rank]
@@ -220,6 +221,10 @@ __global__ void __launch_bounds__(kRowThreads) k_cp_stats(CpParams P) {
   const long long n = P.is_ret[g] ? local_rows(P, L) : 0;
   if (c == 0) rope_heads<G>(P, q, b, g, L, cs, sn);
   if (!P.is_ret[g]) return;
+  if (c == 0) {   // the rank's round-1 histogram row of this slice, filled by the next phase
+    unsigned long long* h1 = P.hist1 + ((size_t)P.rank * P.n_slices + s) * kBins1;
+    for (int i = tid; i < kBins1; i += kRowThreads) h1[i] = 0ull;
+  }
   qidx_heads<G>(P, q, g, qsm);
   if (c == 0 && tid < G * kIdxDim) P.q_idx[((size_t)b * P.Hq + (size_t)g * G) * kIdxDim + tid] = qsm[tid];
 
@@ -281,6 +286,12 @@ __global__ void __launch_bounds__(kRowThreads) k_cp_mass(CpParams P) {
   const int L = cta_len(P, b, &sh_len);
   const long long n = local_rows(P, L);
   for (int i = tid; i < kBins1; i += kRowThreads) { hc[i] = 0u; hl[i] = 0u; }
+  if (c == 0) {   // the rank's round-2 and round-3 rows of this slice, filled by later phases
+    unsigned long long* h2 = P.hist2 + ((size_t)P.rank * P.n_slices + s) * kBins2;
+    unsigned long long* h3 = P.hist3 + ((size_t)P.rank * P.n_slices + s) * kBins3 * 2;
+    for (int i = tid; i < kBins2; i += kRowThreads) h2[i] = 0ull;
+    if (tid < kBins3 * 2) h3[tid] = 0ull;
+  }
   if (tid < G * kIdxDim) qsm[tid] = P.q_idx[((size_t)b * P.Hq + (size_t)g * G) * kIdxDim + tid];
   // (M_h, Z_h): warp w merges head w % G over entries w / G, w / G + kWph, ... (all
   // ranks' chunks in rank-major order), then the warps of a head are merged in order.

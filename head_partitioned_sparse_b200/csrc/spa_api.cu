@@ -805,24 +805,16 @@ spa_status spa_cp_phase(spa_handle h, int phase, const spa_cp_args* a, spa_strea
   spa_status r = cp_check(h, a, &C);
   if (r) return r;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const size_t slices = (size_t)C.n_slices;
-  cudaError_t e;
   switch (phase) {
     case SPA_CP_STATS:
       return run(h, SPA_K_CP_SELECT, st, "cp stats", [&] { return spa::launch_cp_stats(C, st); });
-    case SPA_CP_MASS:
-      if ((e = cudaMemsetAsync(C.hist1 + (size_t)C.rank * slices * spa::kBins1, 0, slices * spa::kBins1 * 8, st)))
-        return cuda_fail(e, "cp clear hist1");
+    case SPA_CP_MASS:   // (the stats phase cleared this rank's hist1 rows)
       return run(h, SPA_K_CP_SELECT, st, "cp mass", [&] { return spa::launch_cp_mass(C, st); });
-    case SPA_CP_ROUND2:
+    case SPA_CP_ROUND2:   // (the mass phase cleared this rank's hist2 and hist3 rows)
       if ((r = run(h, SPA_K_CP_SELECT, st, "cp cut 1", [&] { return spa::launch_cp_cut(C, 1, st); }))) return r;
-      if ((e = cudaMemsetAsync(C.hist2 + (size_t)C.rank * slices * spa::kBins2, 0, slices * spa::kBins2 * 8, st)))
-        return cuda_fail(e, "cp clear hist2");
       return run(h, SPA_K_CP_SELECT, st, "cp round 2", [&] { return spa::launch_cp_hist(C, 2, st); });
     case SPA_CP_ROUND3:
       if ((r = run(h, SPA_K_CP_SELECT, st, "cp cut 2", [&] { return spa::launch_cp_cut(C, 2, st); }))) return r;
-      if ((e = cudaMemsetAsync(C.hist3 + (size_t)C.rank * slices * spa::kBins3 * 2, 0, slices * spa::kBins3 * 16, st)))
-        return cuda_fail(e, "cp clear hist3");
       return run(h, SPA_K_CP_SELECT, st, "cp round 3", [&] { return spa::launch_cp_hist(C, 3, st); });
     case SPA_CP_ATTEND:
       if ((r = run(h, SPA_K_CP_SELECT, st, "cp cut 3", [&] { return spa::launch_cp_cut(C, 3, st); }))) return r;

@@ -317,8 +317,10 @@ SPA_API spa_status spa_prefill(spa_handle h, const void* q_chunk, const void* k_
  *                  local kept rows                                        -> out_all, lse_all
  * then spa_cp_combine merges the ranks' outputs.  Histogram masses are integers, so
  * every rank reaches the same cut.  Each exchange buffer is [n_ranks][...] with the
- * rank's slot at index rank; a phase writes only its own slot (clearing it first) and
- * reads the other slots, which must hold the gathered data of the previous phase.
+ * rank's slot at index rank; a phase writes only its own slots (the histogram slots it
+ * adds into are cleared by an earlier phase of the same rank: stats clears hist1, mass
+ * clears hist2 and hist3) and reads the other slots, which must hold the gathered data
+ * of the previous phase.
  * spa_cp_exchange_sizes gives the byte size of each buffer (all slots).  Every pointer
  * is a device pointer, 16-byte aligned.  Phases and combine only enqueue work on
  * `stream`; a phase called out of order computes garbage but stays in bounds. */
