@@ -536,7 +536,9 @@ def main_native(args):
             g = torch.cuda.CUDAGraph()
             cap = torch.cuda.Stream(device=dev)
             cap.wait_stream(stream)
-            with torch.cuda.graph(g, stream=cap):
+            # thread-local capture: other threads' CUDA calls (a process group's watchdog
+            # under torchrun) stay legal while this thread captures
+            with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
                 fn()
             torch.cuda.synchronize(dev)
             return g

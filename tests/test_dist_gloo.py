@@ -219,3 +219,67 @@ def test_cp_phases_ties_across_ranks_go_to_the_lowest_positions():
     kept = np.setdiff1d(np.concatenate([rk.rows[(0, 0)] for rk in ranks]), sw)
     assert np.array_equal(kept, np.setdiff1d(np.arange(701), sw))
     assert len(ranks[2].rows[(0, 0)]) == len(np.intersect1d(sw, np.arange(800, 1000)))
+
+
+def _decoder_worker(rank, world, port, q):
+    """ContextParallelDecoder.step itself over gloo, with the library calls routed to the
+    host model of the phases (the buffers, the phase order and the all-gathers are the
+    decoder's own)."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import cp_host_model as M
+    from head_partitioned_sparse_b200 import binding as spa
+    from head_partitioned_sparse_b200 import context_parallel as cp
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    try:
+        dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+        inp, idx = _cp_inputs()
+        model = {}
+        calls = []
+        spa.spa_cp_exchange_sizes = lambda h, B, R: M.exchange_sizes(B, inp.Hq, inp.Hkv, CP_C, R)
+        spa.spa_cp_phase = lambda h, phase, args, stream=None: (calls.append(phase), model["m"].phase(phase))
+        spa.spa_cp_combine = lambda h, out_all, lse_all, R, B, out, stream=None: out.copy_(
+            torch.from_numpy(M.combine(model["m"].out_all, model["m"].lse_all)))
+        dec = cp.ContextParallelDecoder(0, B=inp.B, capacity=CP_C, device="cpu")
+        model["m"] = M.HostRank(inp, idx, rank, world, CP_C, dec.bufs, p=inp.p, n_sink=inp.n_sink,
+                                window=inp.window)
+        z = torch.zeros(16, dtype=torch.uint8)
+        out = torch.full((inp.B, inp.Hq, 128), float("nan"), dtype=torch.float32)
+        dec.step(q_pre=z, k_cache=z, v_cache=z, idx_cache=z, head_mask=inp.head_mask,
+                 seq_lens=torch.from_numpy(inp.seq_lens.astype(np.int64)), p=inp.p, n_sink=inp.n_sink,
+                 window=inp.window, out=out)
+        rows = [None] * world
+        dist.all_gather_object(rows, {k: v.tolist() for k, v in model["m"].rows.items()})
+        if rank == 0:
+            got = {k: np.concatenate([np.asarray(rows[r][k], np.int64) for r in range(world)]) for k in rows[0]}
+            err = _cp_check(inp, idx, out.numpy().astype(np.float64), got)
+            q.put(("ok", err, calls == [0, 1, 2, 3, 4]))
+        dist.barrier()
+        dist.destroy_process_group()
+    except Exception as e:  # report to the parent instead of hanging it
+        q.put(("err", repr(e), None))
+        raise
+
+
+def test_context_parallel_decoder_step_over_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_decoder_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=300)
+    alive = [p for p in procs if p.is_alive()]
+    for p in alive:
+        p.kill()
+    assert not alive, "a rank did not finish"
+    status, err, order_ok = q.get(timeout=5)
+    assert status == "ok", err
+    assert err <= 1e-5
+    assert order_ok, "the phases must run once each, in order"
+    assert all(p.exitcode == 0 for p in procs)
