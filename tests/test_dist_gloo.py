@@ -119,12 +119,12 @@ def _cp_check(inp, idx, out, rows):
     return float(np.abs(out - ref).max())
 
 
-def test_cp_phases_emulated_in_one_process_match_the_oracle():
+@pytest.mark.parametrize("R", [1, 2, 3, 5])
+def test_cp_phases_emulated_in_one_process_match_the_oracle(R):
     import torch
     import cp_host_model as M
     from head_partitioned_sparse_b200 import context_parallel as cp
     inp, idx = _cp_inputs()
-    R = 3
     C = -(-int(inp.seq_lens.max()) // R)
     bufs = {n: torch.zeros(sz, dtype=torch.uint8) for n, sz in
             zip(cp.BUFFERS, M.exchange_sizes(inp.B, inp.Hq, inp.Hkv, C, R))}
