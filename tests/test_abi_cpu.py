@@ -3,6 +3,7 @@ bad arguments on the host before touching a GPU.  No compute calls here."""
 import ctypes
 import os
 import re
+import shutil
 import subprocess
 
 import pytest
@@ -103,3 +104,31 @@ def test_create_without_device_fails_loudly(lib):
     with pytest.raises(B.SpaError) as e:
         B.spa_create(_cfg())
     assert e.value.status in (B.SPA_ERR_CUDA, B.SPA_ERR_UNSUPPORTED)
+
+
+def test_context_parallel_calls_reject_a_null_handle(lib):
+    for call in (lambda: B.spa_cp_exchange_sizes(None, 1, 2),
+                 lambda: B.spa_cp_combine(None, 16, 16, 2, 1, 16, stream=0),
+                 lambda: B.spa_cp_phase(None, B.SPA_CP_STATS, B.make_cp_args(
+                     q_pre=16, k_cache=16, v_cache=16, idx_cache=16, head_mask=[1, 0], seq_lens=16, B=1, p=0.9,
+                     n_sink=4, window=16, n_ranks=2, rank=0, pos0=0, max_seq_len=0, stats=16, hist1=16, hist2=16,
+                     hist3=16, out_all=16, lse_all=16), stream=0)):
+        with pytest.raises(B.SpaError) as e:
+            call()
+        assert e.value.status == B.SPA_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs a C compiler")
+def test_cp_args_layout_matches_the_header(tmp_path):
+    """The ctypes mirror of spa_cp_args has the C layout (size and every field offset)."""
+    fields = [f for f, _ in B.spa_cp_args._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "spa.h"\nint main(void) {\n'
+                   '  printf("%zu", sizeof(spa_cp_args));\n'
+                   + "".join(f'  printf(" %zu", offsetof(spa_cp_args, {f}));\n' for f in fields)
+                   + "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()]
+    want = [ctypes.sizeof(B.spa_cp_args)] + [getattr(B.spa_cp_args, f).offset for f in fields]
+    assert got == want
