@@ -97,11 +97,12 @@ def _cp_inputs():
     return inp, idx
 
 
-def _cp_check(inp, idx, out, rows):
+def _cp_check(inp, idx, out, rows, p=None):
     """Union of the ranks' rows = the oracle's sets (band 1e-5 around p); output = the
     oracle on those rows."""
     import oracle as O
-    _, res = O.decode_inputs(inp, idx_cache=idx)
+    p = inp.p if p is None else p
+    _, res = O.decode_inputs(inp, idx_cache=idx, p=p)
     listed = {}
     for b in range(inp.B):
         sw = O.sink_window(int(inp.seq_lens[b]), inp.n_sink, inp.window)
@@ -114,25 +115,26 @@ def _cp_check(inp, idx, out, rows):
             assert np.isin(sw, got).all()
             listed[(b, g)] = np.setdiff1d(got, sw)
             diff = np.setxor1d(listed[(b, g)], res[(b, g)].listed)
-            assert np.all(np.abs(res[(b, g)].topp.c_before[diff] - inp.p) <= 1e-5)
-    ref, _ = O.decode_inputs(inp, idx_cache=idx, attend_sets=listed)
+            assert np.all(np.abs(res[(b, g)].topp.c_before[diff] - p) <= 1e-5)
+    ref, _ = O.decode_inputs(inp, idx_cache=idx, p=p, attend_sets=listed)
     return float(np.abs(out - ref).max())
 
 
-@pytest.mark.parametrize("R", [1, 2, 3, 5])
-def test_cp_phases_emulated_in_one_process_match_the_oracle(R):
+@pytest.mark.parametrize("R,p", [(1, None), (2, None), (3, None), (5, None), (3, 0.5), (4, 0.99), (2, 1.0)])
+def test_cp_phases_emulated_in_one_process_match_the_oracle(R, p):
     import torch
     import cp_host_model as M
     from head_partitioned_sparse_b200 import context_parallel as cp
     inp, idx = _cp_inputs()
+    pp = inp.p if p is None else float(np.float32(p))
     C = -(-int(inp.seq_lens.max()) // R)
     bufs = {n: torch.zeros(sz, dtype=torch.uint8) for n, sz in
             zip(cp.BUFFERS, M.exchange_sizes(inp.B, inp.Hq, inp.Hkv, C, R))}
-    ranks = [M.HostRank(inp, idx, r, R, C, bufs, p=inp.p, n_sink=inp.n_sink, window=inp.window) for r in range(R)]
+    ranks = [M.HostRank(inp, idx, r, R, C, bufs, p=pp, n_sink=inp.n_sink, window=inp.window) for r in range(R)]
     cp.run_step(range(R), lambda ph, r: ranks[r].phase(ph), lambda name: None)
     out = M.combine(ranks[0].out_all, ranks[0].lse_all)
     rows = {k: np.concatenate([rk.rows[k] for rk in ranks]) for k in ranks[0].rows}
-    assert _cp_check(inp, idx, out, rows) <= 1e-5
+    assert _cp_check(inp, idx, out, rows, p=pp) <= 1e-5
 
 
 def _cp_worker(rank, world, port, q):
