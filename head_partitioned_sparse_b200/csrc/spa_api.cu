@@ -356,7 +356,9 @@ spa_status cp_check(spa_ctx* h, const spa_cp_args* a, spa::CpParams* C) {
   if (a->n_ranks < 1 || a->n_ranks > kMaxRanks || a->rank < 0 || a->rank >= a->n_ranks)
     return fail(SPA_ERR_INVALID_ARG, "need 1 <= n_ranks <= %d and 0 <= rank < n_ranks (got %d, %d)", kMaxRanks,
                 a->n_ranks, a->rank);
-  const int64_t cap = a->max_seq_len ? a->max_seq_len : a->pos0 + h->cfg.max_ctx;
+  // default bound: the whole contiguous split (n_ranks * max_ctx), or this rank's end
+  const int64_t split_end = (int64_t)a->n_ranks * h->cfg.max_ctx, rank_end = a->pos0 + h->cfg.max_ctx;
+  const int64_t cap = a->max_seq_len ? a->max_seq_len : (split_end > rank_end ? split_end : rank_end);
   if (a->pos0 < 0 || a->pos0 + h->cfg.max_ctx > INT32_MAX || cap < 1 || cap > INT32_MAX)
     return fail(SPA_ERR_INVALID_ARG, "need pos0 >= 0, pos0 + max_ctx < 2^31 and max_seq_len in [1, 2^31) (got %lld, %lld)",
                 (long long)a->pos0, (long long)cap);
