@@ -341,7 +341,8 @@ typedef struct {
   float p;                  /* in (0, 1] */
   int n_sink, window;       /* >= 0, n_sink + window >= 1 */
   int n_ranks, rank;        /* 1 <= n_ranks <= 1024, 0 <= rank < n_ranks */
-  int64_t pos0;             /* global position of local row 0, >= 0 */
+  int64_t pos0;             /* global position of local row 0, >= 0; must grow with rank (ties at
+                               the cut are handed out rank by rank, lowest positions first) */
   int64_t max_seq_len;      /* bound on the global lengths (0: the larger of n_ranks * max_ctx
                                and pos0 + max_ctx) */
   void* stats;              /* [n_ranks][B][Hkv][ceil(max_ctx / 4096)][G] float2 */
