@@ -285,3 +285,25 @@ def test_context_parallel_decoder_step_over_gloo():
     assert err <= 1e-5
     assert order_ok, "the phases must run once each, in order"
     assert all(p.exitcode == 0 for p in procs)
+
+
+def test_cp_host_model_masses_are_exact_fixed_point():
+    """mass_q(bits(x)) = x * 2^63 exactly for float32 x >= 2^-40, else 0 (the quantised
+    mass the histograms sum); cut_desc finds the first bin, from the top, where the
+    running mass reaches the target."""
+    from fractions import Fraction
+
+    import cp_host_model as M
+    rng = np.random.default_rng(3)
+    xs = np.concatenate([rng.random(2000, dtype=np.float32) ** 8, np.float32([1.0, 2.0 ** -40, 2.0 ** -41, 0.0])])
+    got = M.mass_q(xs.view(np.uint32))
+    for x, q in zip(xs.tolist(), got.tolist()):
+        want = int(Fraction(x) * 2 ** 63) if x >= 2.0 ** -40 else 0
+        assert q == want
+    h = np.array([5, 0, 3, 2], np.uint64)          # bins 0..3; from the top: 2, 3, 0, 5
+    assert M.cut_desc(h, 0, 1) == (3, 0)
+    assert M.cut_desc(h, 0, 3) == (2, 2)
+    assert M.cut_desc(h, 0, 5) == (2, 2)
+    assert M.cut_desc(h, 0, 6) == (0, 5)
+    assert M.cut_desc(h, 4, 10) == (0, 9)
+    assert M.cut_desc(h, 0, 11)[0] == -1
