@@ -42,6 +42,10 @@ MUTATIONS = [
      "kept_blocks = bidx if p >= 1.0 else np.sort(order[before_sorted <= p])", "block top-p keeps one block too many"),
     ("spa_oracle.py", "bmass = np.array([pi[b * block:(b + 1) * block].sum()",
      "bmass = np.array([pi[b * block:(b + 1) * block].max()", "block scored by its maximum"),
+    ("spa_oracle.py", "s.update(range(max(0, L - max(window, 0)), L))",
+     "s.update(range(max(0, L - max(window, 0) + 1), L))", "window one position short"),
+    ("spa_oracle.py", "return softmax(s, axis=-1) @ np.asarray(V, np.float64)",
+     "return softmax(s, axis=0) @ np.asarray(V, np.float64)", "attention softmax over the wrong axis"),
     ("aoh_oracle.py", "np.exp(-np.sum(p * np.log(p)))", "np.exp(-np.sum(p * np.log2(p)))", "entropy in bits"),
     ("aoh_oracle.py", "return (Wq @ Wq.T) @ (Wk @ Wk.T)", "return (Wq @ Wk.T) @ (Wk @ Wq.T)", "proxy matrix operands"),
     ("aoh_oracle.py", "_, R = np.linalg.qr(Wk.T)", "_, R = np.linalg.qr(Wq.T)", "kernel operator operands"),
