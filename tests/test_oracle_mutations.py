@@ -59,6 +59,9 @@ MUTATIONS = [
     ("prefill_oracle.py", "q = rope(to_f64(q_chunk[b, h, i]), t, rope_theta)",
      "q = rope(to_f64(q_chunk[b, h, i]), i, rope_theta)", "query rotated to its chunk row"),
     ("prefill_oracle.py", "g = h // G", "g = h % Hkv", "GQA head mapping"),
+    ("prefill_oracle.py", "keys = prefill_keys(t, bool(head_mask[g]), n_sink, window)",
+     "keys = prefill_keys(t, not head_mask[g], n_sink, window)", "retrieval and streaming heads swapped"),
+    ("aoh_oracle.py", "p = s / s.sum()", "p = s / s.max()", "singular values normalised by the largest"),
 ]
 
 
