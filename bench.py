@@ -217,7 +217,7 @@ def main_reference(args):
     inp = synth.make_inputs(args.config, shard.rank_seed(args.seed, 0), overrides=overrides(args),
                             draw_streaming_kpre=False)
     ret = [g for g in range(inp.Hkv) if inp.head_mask[g]]
-    idx = O.index_cache_for(inp, heads=ret, precision="f64")   # BLAS: fast setup, untimed
+    idx = O.index_cache_for(inp, heads=ret)   # BLAS: fast setup, untimed
     # each step: the oracle's decode of one sequence of the batch (all its KV heads);
     # a layer-step is B such samples.
     for i in range(args.warmup):
@@ -665,7 +665,7 @@ def main_native(args):
         if world == 1 and not args.no_cpu_baseline:
             import oracle as O
             ret = [g for g in range(inp.Hkv) if inp.head_mask[g]]
-            idx_o = O.index_cache_for(inp, heads=ret, precision="f64")   # untimed setup
+            idx_o = O.index_cache_for(inp, heads=ret)   # untimed setup
             t_first = run_oracle_sample(inp, idx_o, p, list(range(inp.B)))
             reps = max(1, min(8, math.ceil(10.0 / max(t_first, 1e-3)))) - 1
             tot = t_first + sum(run_oracle_sample(inp, idx_o, p, list(range(inp.B))) for _ in range(reps))

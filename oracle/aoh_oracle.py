@@ -18,7 +18,7 @@ Source: "Autonomy of Heads" (AoH) summary, Methodology:
      rest streaming; under GQA head scores are aggregated to the group by their
      mean.
 
-Readings where the summary is silent (listed in the design notes):
+Readings taken where the summary is silent:
   * W_Q^h and W_K^g are the d_head x d_model row blocks of the query and key
     projections (q = W_Q^h x); a query head uses the key head of its GQA group;
   * log is the natural logarithm (exp and log of the same base: the effective

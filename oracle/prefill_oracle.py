@@ -10,7 +10,7 @@ Sources (page title, section):
   "Autonomy of Heads" summary, Deployment strategy: streaming heads keep a sink
   cache and a recent window from the first token on, prefill included.
 
-Readings (listed in the design notes):
+Readings taken where the pages are silent:
   * a chunk holds the T queries at absolute positions start[b] .. start[b] + T - 1;
     the caches already hold every position up to the chunk's last (keys post-RoPE);
   * a query at position t attends causally: a retrieval head keys [0, t]; a

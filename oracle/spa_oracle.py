@@ -26,7 +26,7 @@ Sources (page title, section):
          aggregated to the group by their mean; streaming heads keep a sink cache
          and a recent window.
 
-Readings where the pages are silent (each is listed in the design notes):
+Readings taken where the pages are silent:
   * index softmax temperature = idx_scale (1/sqrt(16) by default);
   * per query head probabilities, averaged over the GQA group (the group mean
     of [AoH]); one selected set per (sequence, KV head);
@@ -44,9 +44,7 @@ Readings where the pages are silent (each is listed in the design notes):
     de-duplicated;
   * RoPE: rotate-half pairing (i, i + d/2), inv_freq_i = theta^(-2i/d), angle
     = position * inv_freq_i, query at position L-1, no frequency rescaling;
-  * index cache rows are bf16, rounded to nearest-even; the code is decided
-    in float32 (products and a running sum in ascending d), the precision the
-    CUDA path decides it in; the float64 definition is kept beside it.
+  * index cache rows are bf16: the exact product rounded once to nearest-even.
 """
 from __future__ import annotations
 
@@ -113,35 +111,22 @@ def rope(x: np.ndarray, pos, theta: float) -> np.ndarray:
 # --------------------------------------------------------------------------
 # Index cache  ([FASB] §2)
 # --------------------------------------------------------------------------
-def index_rows(k_pre_rows: np.ndarray, P_k_g: np.ndarray, precision: str = "f32") -> np.ndarray:
+def index_rows(k_pre_rows: np.ndarray, P_k_g: np.ndarray) -> np.ndarray:
     """bf16 bits of P_k[g] . k for each pre-RoPE key row; [n, 128] -> [n, 16].
 
-    precision="f64": the mathematical definition, bf16_rne of the exact product.
-    precision="f32": the bf16 code decided in float32, the precision the CUDA
-    path decides it in: each product P[r][d] * k[d] rounded to float32 and added
-    to a float32 running sum in ascending d (starting from 0), then bf16_rne.
-    The two agree except where the float32 sum and the exact value straddle a
-    bf16 rounding midpoint.
+    The definition: the exact (float64) product of the projector and the key,
+    rounded once to the nearest bf16, ties to even.
     """
-    if precision == "f64":
-        return f64_to_bf16_bits(np.asarray(k_pre_rows, np.float64) @ np.asarray(P_k_g, np.float64).T)
-    if precision != "f32":
-        raise ValueError(precision)
-    k = np.asarray(k_pre_rows, np.float32)          # storage values are exact in float32
-    P = np.asarray(P_k_g, np.float32)
-    acc = np.zeros((k.shape[0], P.shape[0]), np.float32)
-    for d in range(k.shape[1]):
-        acc = acc + k[:, d:d + 1] * P[None, :, d]    # float32 multiply, then float32 add
-    return f64_to_bf16_bits(acc.astype(np.float64))
+    return f64_to_bf16_bits(np.asarray(k_pre_rows, np.float64) @ np.asarray(P_k_g, np.float64).T)
 
 
-def index_append(k_pre: np.ndarray, P_k: np.ndarray, precision: str = "f32") -> np.ndarray:
+def index_append(k_pre: np.ndarray, P_k: np.ndarray) -> np.ndarray:
     """[B][Hkv][T][128] pre-RoPE keys (float64 values) -> [B][Hkv][T][16] bf16 bits."""
     B, Hkv = k_pre.shape[:2]
     out = np.empty(k_pre.shape[:3] + (IDX_DIM,), np.uint16)
     for b in range(B):
         for g in range(Hkv):
-            out[b, g] = index_rows(k_pre[b, g], P_k[g], precision)
+            out[b, g] = index_rows(k_pre[b, g], P_k[g])
     return out
 
 
@@ -344,12 +329,12 @@ def decode_inputs(inp, *, slices=None, attend_sets=None, p=None, n_sink=None, wi
                   attend_sets=attend_sets, k=k, blocks=blocks)
 
 
-def index_cache_for(inp, heads: Optional[List[int]] = None, precision: str = "f32") -> np.ndarray:
+def index_cache_for(inp, heads: Optional[List[int]] = None) -> np.ndarray:
     """bf16 index cache of a ``synth.Inputs`` bundle; rows of other heads stay 0."""
     to_f64 = (lambda a: bf16_bits_to_f64(a)) if inp.dtype == "bf16" else (lambda a: np.asarray(a, np.float64))
     out = np.zeros(inp.k_pre.shape[:3] + (IDX_DIM,), np.uint16)
     hs = range(inp.Hkv) if heads is None else heads
     for b in range(inp.B):
         for g in hs:
-            out[b, g] = index_rows(to_f64(inp.k_pre[b, g]), inp.P_k[g], precision)
+            out[b, g] = index_rows(to_f64(inp.k_pre[b, g]), inp.P_k[g])
     return out

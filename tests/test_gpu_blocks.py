@@ -112,7 +112,7 @@ def test_blocks_full_size_ctx128k():
     sample = [(0, 0), (3, 2)]
     idx = np.zeros(inp.k_pre.shape[:3] + (16,), np.uint16)
     for (b, g) in sample:
-        idx[b, g] = O.index_rows(to64(inp.k_pre[b, g]), inp.P_k[g], "f32")
+        idx[b, g] = O.index_rows(to64(inp.k_pre[b, g]), inp.P_k[g])
     with Handle(inp) as h:
         dev = DevInputs(inp, idx)
         lists, cnt = gpu_select_blocks(h, inp, dev, inp.p)

@@ -37,7 +37,7 @@ def _check(name, seed, sample, ps):
     idx = np.zeros(inp.k_pre.shape[:3] + (16,), np.uint16)
     for (b, g) in sample:
         if inp.head_mask[g]:
-            idx[b, g] = O.index_rows(to64(inp.k_pre[b, g]), inp.P_k[g], "f32")
+            idx[b, g] = O.index_rows(to64(inp.k_pre[b, g]), inp.P_k[g])
     with Handle(inp) as h:
         dev = DevInputs(inp, idx)
         for p in ps:

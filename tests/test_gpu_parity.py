@@ -11,6 +11,7 @@ import torch
 import oracle as O
 from head_partitioned_sparse_b200 import binding as B
 from head_partitioned_sparse_b200 import synth
+from index_band import check_index_codes
 from spa_testutil import (OUT_ATOL, DevInputs, Handle, check_selection, dev_storage, gpu_decode, gpu_select,
                           oracle_idx)
 
@@ -22,17 +23,6 @@ def _ret(inp):
 
 
 # ------------------------------------------------------------------ index append
-def _within_f64_bound(gpu_bits, k_f64, P_k):
-    """Every code lies between the bf16 roundings of exact -/+ the float32 accumulation
-    bound of a 128-term sum (the float64 definition, up to float32 rounding)."""
-    exact = np.einsum("bgtd,grd->bgtr", k_f64, P_k.astype(np.float64))
-    bound = 128 * 2.0 ** -24 * np.einsum("bgtd,grd->bgtr", np.abs(k_f64), np.abs(P_k.astype(np.float64))) * 1.01
-    lo = O.bf16_bits_to_f64(O.f64_to_bf16_bits(exact - bound))
-    hi = O.bf16_bits_to_f64(O.f64_to_bf16_bits(exact + bound))
-    v = O.bf16_bits_to_f64(gpu_bits)
-    assert np.all((v >= lo) & (v <= hi))
-
-
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_index_append_prefill_parity(dtype):
     inp = synth.make_inputs("tiny", 5, overrides={"L": 3000, "dtype": dtype, "B": 2})
@@ -44,9 +34,10 @@ def test_index_append_prefill_parity(dtype):
         B.spa_index_append(h.h, k, start, inp.B, inp.Lmax, idx)
         B.spa_device_status(h.h)
     got = idx.cpu().numpy().view(np.uint16)
-    want = O.index_cache_for(inp)                 # code decided in float32, as the kernel does
-    assert np.array_equal(got, want)
-    _within_f64_bound(got, to64(inp.k_pre), inp.P_k)
+    # the float64 definition, bit-exact except next to a bf16 rounding midpoint
+    n_off = sum(check_index_codes(got[:, g], to64(inp.k_pre[:, g]), inp.P_k[g]) for g in range(inp.Hkv))
+    print(f"index codes one step from the definition (next to a midpoint): {n_off} of {got.size}")
+    assert n_off <= 1e-3 * got.size
 
 
 def test_index_append_decode_rows_at_offsets():
@@ -59,9 +50,10 @@ def test_index_append_decode_rows_at_offsets():
         B.spa_index_append(h.h, dev_storage(k_new, "bf16"), torch.tensor(starts, device="cuda"), 3, T, idx)
         B.spa_device_status(h.h)
         got = idx.cpu().numpy().view(np.uint16)
-        want = O.index_cache_for(inp)
+        k64 = O.bf16_bits_to_f64(inp.k_pre)
         for b in range(3):
-            assert np.array_equal(got[b, :, starts[b]], want[b, :, starts[b]])
+            for g in range(inp.Hkv):
+                check_index_codes(got[b, g, starts[b]], k64[b, g, starts[b]], inp.P_k[g])
             mask = np.ones(512, bool)
             mask[starts[b]] = False
             assert not got[b][:, mask].any()       # nothing else written

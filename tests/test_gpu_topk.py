@@ -114,7 +114,7 @@ def test_topk_full_size_ctx128k():
     sample = [(0, 0), (3, 2)]
     idx = np.zeros(inp.k_pre.shape[:3] + (16,), np.uint16)
     for (b, g) in sample:
-        idx[b, g] = O.index_rows(to64(inp.k_pre[b, g]), inp.P_k[g], "f32")
+        idx[b, g] = O.index_rows(to64(inp.k_pre[b, g]), inp.P_k[g])
     k = 4096
     with Handle(inp) as h:
         dev = DevInputs(inp, idx)

@@ -75,7 +75,7 @@ def _scratch(tmp, oracle_file=None, old=None, new=None):
         shutil.copy(os.path.join(ROOT, "head_partitioned_sparse_b200", f), pkg)
     tests = os.path.join(tmp, "tests")
     os.makedirs(tests)
-    for f in ["conftest.py"] + sorted(set(PINS.values())):
+    for f in ["conftest.py", "index_band.py"] + sorted(set(PINS.values())):
         shutil.copy(os.path.join(ROOT, "tests", f), tests)
     shutil.copytree(os.path.join(ROOT, "tests", "golden"), os.path.join(tests, "golden"))
     if oracle_file:

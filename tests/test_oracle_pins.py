@@ -13,6 +13,7 @@ import pytest
 import torch
 
 import oracle as O
+from index_band import check_index_codes, f32_accumulation_bound, f32_sequential_codes
 from head_partitioned_sparse_b200 import synth
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -421,8 +422,8 @@ def test_planted_keys_are_recalled_in_tiny_workload():
     assert len(sr.topp.kept) < 0.05 * inp.seq_lens[0]   # concentrated: a small selected set
 
 
-# ---------------------------------------------------------------- float32-decided index code
-def test_index_rows_f32_follows_float32_sequential_rounding():
+# ---------------------------------------------------------------- float32 accumulation band
+def test_band_admits_float32_sum_that_straddles_a_midpoint():
     # fp32 inputs: 1 + 2^-8 then four 2^-30 terms.  In float32 each 2^-30 is lost
     # (spacing at 1 is 2^-23), the sum stays on the bf16 midpoint and rounds to even
     # (1.0); the exact value lies above the midpoint and rounds up to 1 + 2^-7.
@@ -430,25 +431,39 @@ def test_index_rows_f32_follows_float32_sequential_rounding():
     P[0, :5] = 1.0
     k = np.zeros((1, 128), np.float64)
     k[0, :5] = [1.0 + 2.0 ** -8] + [2.0 ** -30] * 4
-    f32 = O.bf16_bits_to_f64(O.index_rows(k, P, "f32"))[0, 0]
-    f64 = O.bf16_bits_to_f64(O.index_rows(k, P, "f64"))[0, 0]
-    assert f32 == 1.0 and f64 == 1.0 + 2.0 ** -7
+    f32 = f32_sequential_codes(k, P)
+    assert O.bf16_bits_to_f64(f32)[0, 0] == 1.0
+    assert O.bf16_bits_to_f64(O.index_rows(k, P))[0, 0] == 1.0 + 2.0 ** -7
+    assert check_index_codes(f32, k, P) == 1          # admitted, and counted as differing
 
 
-def test_index_rows_f32_matches_torch_float32_loop_and_f64_bound():
+def test_band_float32_model_matches_torch_float32_loop_and_is_admitted():
     rng = np.random.default_rng(12)
-    k = synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(rng.standard_normal((200, 128)).astype(np.float32)))
+    k = synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(rng.standard_normal((2000, 128)).astype(np.float32)))
     P = (rng.standard_normal((16, 128)) / math.sqrt(128)).astype(np.float32)
-    got = O.index_rows(k.astype(np.float64), P, "f32")
+    got = f32_sequential_codes(k.astype(np.float64), P)
     # independent float32 sequential sum with torch (no fused multiply-add on CPU tensors)
     tk, tP = torch.from_numpy(k), torch.from_numpy(P)
-    acc = torch.zeros((200, 16), dtype=torch.float32)
+    acc = torch.zeros((2000, 16), dtype=torch.float32)
     for d in range(128):
         acc = acc + tk[:, d:d + 1] * tP[None, :, d]
     ref = acc.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     assert np.array_equal(got, ref)
-    exact = k.astype(np.float64) @ P.astype(np.float64).T
-    bound = 128 * 2.0 ** -24 * (np.abs(k).astype(np.float64) @ np.abs(P).astype(np.float64).T) * 1.01
-    v = O.bf16_bits_to_f64(got)
-    assert np.all(v >= O.bf16_bits_to_f64(O.f64_to_bf16_bits(exact - bound)))
-    assert np.all(v <= O.bf16_bits_to_f64(O.f64_to_bf16_bits(exact + bound)))
+    n_off = check_index_codes(got, k.astype(np.float64), P)
+    assert n_off < 0.01 * got.size                    # rare: only next to a midpoint
+    assert check_index_codes(O.index_rows(k.astype(np.float64), P), k.astype(np.float64), P) == 0
+
+
+def test_band_rejects_a_code_one_step_off_away_from_a_midpoint():
+    rng = np.random.default_rng(13)
+    k = synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(rng.standard_normal((64, 128)).astype(np.float32)))
+    P = (rng.standard_normal((16, 128)) / math.sqrt(128)).astype(np.float32)
+    k64 = k.astype(np.float64)
+    bits = O.index_rows(k64, P).copy()
+    exact = k64 @ P.astype(np.float64).T
+    beta = f32_accumulation_bound(k64, P)
+    far = O.f64_to_bf16_bits(exact - beta) == O.f64_to_bf16_bits(exact + beta)
+    i, r = np.argwhere(far)[0]
+    bits[i, r] = bits[i, r] + 1                       # next bf16 magnitude
+    with pytest.raises(AssertionError):
+        check_index_codes(bits, k64, P)
