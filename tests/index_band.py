@@ -6,8 +6,10 @@ pre-RoPE keys; the cache is bf16).  A device that accumulates the 128 products
 in float32, in any order, with or without fused multiply-add, reaches a sum
 within gamma_128 * sum |P k| of the exact value (u = 2^-24; Higham, Accuracy
 and Stability of Numerical Algorithms, eq. 3.5).  Its code equals the defined
-code unless that interval holds a bf16 rounding midpoint; there it may be the
-neighbour on the other side of the midpoint.
+code unless that interval holds a bf16 rounding midpoint; there it may be any
+code the interval rounds to: the neighbour across the midpoint when the bound is
+below one bf16 step, several steps when the products cancel and the exact value
+is small next to the bound.
 
 Test infrastructure: numpy only, no GPU.
 """
@@ -36,8 +38,8 @@ def f32_accumulation_bound(k_f64: np.ndarray, P: np.ndarray) -> np.ndarray:
 
 def check_index_codes(got_bits: np.ndarray, k_f64: np.ndarray, P: np.ndarray) -> int:
     """Every code is the defined one, or - only where the exact value lies within the
-    float32 accumulation bound of a bf16 midpoint - one step from it inside that
-    interval.  Returns the number of codes that differ from the definition.
+    float32 accumulation bound of a bf16 midpoint - another code that interval rounds
+    to.  Returns the number of codes that differ from the definition.
 
     got_bits [..., 16] bf16 bits; k_f64 [..., 128] exact key values; P [16, 128]."""
     exact = np.einsum("...d,rd->...r", np.asarray(k_f64, np.float64), np.asarray(P, np.float64))
@@ -47,7 +49,7 @@ def check_index_codes(got_bits: np.ndarray, k_f64: np.ndarray, P: np.ndarray) ->
     hi = _ordinal(O.f64_to_bf16_bits(exact + beta))
     g, w = _ordinal(got_bits), _ordinal(want)
     near_midpoint = lo != hi
-    ok = (g == w) | (near_midpoint & (g >= lo) & (g <= hi) & (np.abs(g - w) <= 1))
+    ok = (g == w) | (near_midpoint & (g >= lo) & (g <= hi))
     assert np.all(ok), (f"{int((~ok).sum())} index codes outside the band; first at "
                         f"{np.argwhere(~ok)[:4].tolist()}")
     return int((g != w).sum())
