@@ -13,9 +13,14 @@
 // The array's name is only a host-side stand-in in host code, so its device address
 // is looked up once per device with cudaGetSymbolAddress, with that device current,
 // on the first call made on that device (do that first call before any stream
-// capture).  Every call shares the array and it keeps the last call's contents; the
-// selection kernels clear what must start at zero (histograms, counters, state) at
-// the start of each call.  Calls that overlap on the GPU (other streams, other host
+// capture).  Every call shares the array and it keeps the last call's contents.  The
+// words that must start at zero on every call (the selection kernel's grid-barrier
+// arrival and generation words, the device status word and the per-slice state with
+// its tickets and query-vector flags) sit at fixed offsets at the head of the array and
+// are cleared with one cudaMemsetAsync on the call's stream before the launch, so a
+// call never inherits a half-counted barrier, whatever the shapes of earlier calls or
+// whether one of their bounded waits gave up; the kernels clear the rest (histograms,
+// counters) themselves.  Calls that overlap on the GPU (other streams, other host
 // threads) race on the array: serialise them.
 #include <cmath>
 #include <cstring>
@@ -117,8 +122,10 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
   P.split_rows = spa::kDefaultSplitRows;
 
   int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaError_t ce = cudaGetDevice(&dev);
+  if (ce != cudaSuccess) return err(SPA_ERR_CUDA, cudaGetErrorString(ce));
+  ce = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (ce != cudaSuccess) return err(SPA_ERR_CUDA, cudaGetErrorString(ce));
   const int per_sm = spa::select_resident_per_sm(kv_dtype, G);
   if (per_sm < 1 || sms < 1) return err(SPA_ERR_UNSUPPORTED, "spa_select_noalloc: selection kernel cannot be resident");
   const int grid = spa::select_grid(P, per_sm * sms < spa::kMaxSelectGrid ? per_sm * sms : spa::kMaxSelectGrid);
@@ -127,6 +134,10 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
   spa_status r = scratch_on_current_device(&base_v);
   if (r) return r;
   char* base = static_cast<char*>(base_v);
+  // Fixed head block, cleared before every launch: barrier words, status word, the
+  // per-slice state of up to kMaxSlices slices.
+  const size_t off_bar = 0, off_err = up256(spa::kBarWords * 4), off_st = off_err + 256;
+  const size_t head_bytes = up256(off_st + (size_t)kMaxSlices * sizeof(spa::SliceState));
   const size_t sz[] = {
       64 * 8,                                                  // inv_freq (unused by selection; zero)
       (size_t)B * n_q_heads * spa::kHeadDim * 4,               // q_rot
@@ -137,13 +148,10 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
       (size_t)slices * max_ctx * 8,                            // candidates
       (size_t)slices * P.n_chunks * 4,                         // chunk_gt
       (size_t)slices * P.n_chunks * 4,                         // chunk_off
-      (size_t)slices * sizeof(spa::SliceState),                // state
-      256,                                                     // device status word
       (size_t)slices * spa::kBins2 * 8,                        // hist2
-      spa::kBarWords * 4,                                      // selection grid barrier
   };
   size_t off[sizeof sz / sizeof sz[0]];
-  size_t o = 0;
+  size_t o = head_bytes;
   for (size_t i = 0; i < sizeof sz / sizeof sz[0]; ++i) {
     off[i] = o;
     o += up256(sz[i]);
@@ -161,13 +169,15 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
   w.cand = (uint2*)(base + off[6]);
   w.chunk_gt = (int*)(base + off[7]);
   w.chunk_off = (int*)(base + off[8]);
-  w.st = (spa::SliceState*)(base + off[9]);
-  w.dev_err = (unsigned*)(base + off[10]);
-  w.hist2 = (unsigned long long*)(base + off[11]);
-  w.bar = (unsigned*)(base + off[12]);
+  w.hist2 = (unsigned long long*)(base + off[9]);
+  w.bar = (unsigned*)(base + off_bar);
+  w.dev_err = (unsigned*)(base + off_err);
+  w.st = (spa::SliceState*)(base + off_st);
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = spa::launch_select(P, kv_dtype, grid, st);
+  cudaError_t e = cudaMemsetAsync(base, 0, head_bytes, st);   // stream-ordered; allocates nothing
+  if (e != cudaSuccess) return err(SPA_ERR_CUDA, cudaGetErrorString(e));
+  e = spa::launch_select(P, kv_dtype, grid, st);
   if (e != cudaSuccess) return err(SPA_ERR_CUDA, cudaGetErrorString(e));
   return SPA_OK;
 }

@@ -457,8 +457,17 @@ SPA_API spa_status spa_launch_count(spa_handle h, int64_t* launches);
  * device address there (cudaGetSymbolAddress, with that device current): make that
  * first call before any stream capture.  Every call shares the array and the next
  * call overwrites it, so calls that overlap on the GPU race: serialise them.
- * Out-of-range seq_lens values are clamped but not reported (no handle to hold the
- * status word).
+ * Before each launch the call clears, with one cudaMemsetAsync on `stream` (which
+ * allocates nothing), the fixed block at the head of the array that holds the
+ * selection kernel's grid-barrier words, its status word and the per-slice state,
+ * so no call inherits synchronisation state from an earlier one of another shape.
+ * Device-side conditions are not reported by this entry point (there is no handle
+ * to hold a status word): out-of-range seq_lens values are clamped, and a bounded
+ * device wait that gives up (about 2 s; the kernel then leaves early and its lists
+ * and counts are not valid) or an internal consistency check that fails is dropped.
+ * In every such case the call has already returned SPA_OK; the next call starts
+ * from cleared state.  Callers that need these conditions reported use
+ * spa_create + spa_select + spa_device_status.
  */
 SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads, int n_kv_heads, int kv_dtype,
                                       float idx_scale, int64_t max_ctx, const void* q_pre,

@@ -4,7 +4,12 @@ Such callers (a host framework that has reserved the GPU's memory for its own
 pool, or a decode loop that cannot afford an allocation's implicit device
 synchronisation) get an entry point with no handle whose scratch is a static
 device array.  Its result must equal spa_select's, exactly (selection is
-integer work), on consecutive calls that reuse the same static scratch.
+integer work), on consecutive calls that reuse the same static scratch, and
+must agree with the float64 oracle under the selection band.
+
+The calls go from the largest footprint to smaller ones, so a later call lays
+its buffers over bytes an earlier call left non-zero: the synchronisation and
+per-slice state sit at fixed offsets and are cleared before every launch.
 
 This file is collected last so that, if it fails, a run that stops at the first
 failure has already run every other test.
@@ -16,7 +21,7 @@ import torch
 import oracle as O
 from head_partitioned_sparse_b200 import binding as B
 from head_partitioned_sparse_b200 import synth
-from spa_testutil import DevInputs, Handle, gpu_select, kv_dtype_code
+from spa_testutil import DevInputs, Handle, check_selection, gpu_select, kv_dtype_code
 
 pytestmark = pytest.mark.gpu
 
@@ -32,24 +37,36 @@ def _noalloc_select(inp, dev, P_q, p):
             for b in range(inp.B) for g in range(inp.Hkv)}, cnt.reshape(inp.B, inp.Hkv)
 
 
-def test_noalloc_select_matches_spa_select_on_two_calls_in_a_row():
-    cases = [
+def _cases():
+    return [
+        # largest footprint first: 2 heads x 2^18 tokens = the 2^19-token limit
+        (synth.make_inputs("tiny", 23, overrides={"dtype": "bf16", "L": 1 << 18}), 0.9),
         (synth.make_inputs("tiny", 21, overrides={"dtype": "bf16", "B": 3, "L": 2 * 4096 + 99, "window": 200},
                            seq_lens=[2 * 4096 + 99, 5000, 700]), 0.9),
         (synth.make_inputs("tiny", 22, overrides={"dtype": "bf16", "Hq": 16, "Hkv": 2, "L": 20000,
                                                   "retrieval": [0, 1], "n_planted": 16}), 0.5),
     ]
-    for inp, p in cases:                       # two calls in a row on the same static scratch
-        pp = float(np.float32(p))
-        idx = O.index_cache_for(inp, heads=[g for g in range(inp.Hkv) if inp.head_mask[g]])
-        with Handle(inp) as h:
-            dev = DevInputs(inp, idx)
-            want, want_cnt = gpu_select(h, inp, dev, p=pp)
-            got, got_cnt = _noalloc_select(inp, dev, h.P_q, pp)
-        assert np.array_equal(got_cnt, want_cnt)
-        for k in want:
-            assert np.array_equal(got[k], want[k]), k
-        assert got_cnt[:, np.asarray(inp.head_mask) == 1].min() > 0
+
+
+def test_noalloc_select_matches_spa_select_and_the_oracle_on_calls_in_a_row():
+    for rep in range(2):                       # every case twice, on the same static scratch
+        for inp, p in _cases():
+            pp = float(np.float32(p))
+            ret = [g for g in range(inp.Hkv) if inp.head_mask[g]]
+            idx = O.index_cache_for(inp, heads=ret)
+            with Handle(inp) as h:
+                dev = DevInputs(inp, idx)
+                want, want_cnt = gpu_select(h, inp, dev, p=pp)
+                got, got_cnt = _noalloc_select(inp, dev, h.P_q, pp)
+            assert np.array_equal(got_cnt, want_cnt), (rep, inp.L)
+            for k in want:
+                assert np.array_equal(got[k], want[k]), (rep, k)
+            assert got_cnt[:, np.asarray(inp.head_mask) == 1].min() > 0
+            if rep == 0:                       # against the float64 oracle, once per case
+                _, res = O.decode_inputs(inp, idx_cache=idx, p=pp,
+                                         slices=[(b, g) for b in range(inp.B) for g in ret])
+                for (b, g), sr in res.items():
+                    check_selection(got[(b, g)], sr, pp, inp.n_sink, inp.window)
 
 
 def test_noalloc_select_rejects_requests_beyond_its_static_scratch():
