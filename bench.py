@@ -63,6 +63,8 @@ def parse_args():
     ap.add_argument("--prefill-len", type=int, default=32768, help="prefill chunk length (from position 0)")
     ap.add_argument("--no-cp", action="store_true", help="skip the context-parallel measurement")
     ap.add_argument("--cp-ranks", type=int, default=4, help="ranks of the context-parallel measurement")
+    ap.add_argument("--no-index-append", action="store_true", help="skip the index-append throughput leg")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' sub-records")
     ap.add_argument("--override", action="append", default=[], metavar="KEY=VALUE",
                     help="replace a workload field (e.g. B=1 for a small profiling case)")
     return ap.parse_args()
@@ -80,6 +82,16 @@ def workload_desc(cfg: dict, name: str, p: float) -> str:
     return (f"{name}: batch {cfg['B']}, {cfg['Hq']}/{cfg['Hkv']} heads, head dim 128, context {cfg['L']}, "
             f"{cfg['dtype']}, {len(cfg['retrieval'])} retrieval KV heads, r=16 index, p={p:g}, "
             f"sinks {cfg['n_sink']}, window {cfg['window']}")
+
+
+def config_dict(cfg: dict, name: str, p: float, world: int, n_layers: int) -> dict:
+    """The ``config`` object of the JSON line, identical on both arms."""
+    s_kv = 2 if cfg["dtype"] == "bf16" else 4
+    layer_bytes = cfg["B"] * cfg["Hkv"] * cfg["L"] * (2 * 128 * s_kv + 32)
+    return {"workload": workload_desc(cfg, name, p), "batch": cfg["B"], "seq_len": cfg["L"], "p": p,
+            "storage": cfg["dtype"], "parallelism": f"dp{world}",
+            "l2": f"inputs larger than L2: {n_layers} layer copies of {layer_bytes / 1e9:.2f} GB "
+                  f"(K, V, index rows) cycled, one per step"}
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -205,6 +217,123 @@ def run_oracle_sample(inp, idx_bits, p, seqs):
     return time.perf_counter() - t0
 
 
+def selection_metrics(B, torch, h, q, idx, lens, inp, p, Lcap, dev, stream):
+    """Realised sparsity, index mass captured and planted-key recall of one step's
+    selection (the kept lists from spa_select).  Reported only: computed after timing,
+    in float32 with torch (the index distribution restated for the report)."""
+    sel = torch.full((inp.B, inp.Hkv, inp.Lmax), -1, dtype=torch.int32, device=dev)
+    cnt = torch.zeros(inp.B * inp.Hkv, dtype=torch.int32, device=dev)
+    B.spa_select(h, q, idx, inp.head_mask, lens, inp.B, Lcap, p, inp.n_sink, inp.window, sel, cnt, stream)
+    B.spa_device_status(h, stream)
+    cnt = cnt.cpu().numpy().reshape(inp.B, inp.Hkv)
+    G = inp.G
+    P_q = torch.from_numpy(inp.P_q).to(dev)
+    qf = q.float()
+    ret_tokens = ret_attended = all_attended = 0
+    mass, recall_hit, recall_n = [], 0, 0
+    for b in range(inp.B):
+        L = int(inp.seq_lens[b])
+        n_s = min(inp.n_sink, L)
+        w_lo = max(n_s, L - inp.window)
+        always = torch.zeros(L, dtype=torch.bool, device=dev)
+        always[:n_s] = True
+        always[w_lo:] = True
+        for g in range(inp.Hkv):
+            if not inp.head_mask[g]:
+                all_attended += int(always.sum())
+                continue
+            keep = always.clone()
+            lst = sel[b, g, :int(cnt[b, g])].long()
+            keep[lst] = True
+            heads = slice(g * G, (g + 1) * G)
+            q_idx = torch.einsum("hrd,hd->hr", P_q[heads], qf[b, heads])              # [G][16]
+            rows = idx[b, g, :L].view(torch.bfloat16).float()                     # bf16 bits -> values
+            s = (rows @ q_idx.T) * inp.idx_scale                                   # [L][G]
+            pi = torch.softmax(s, dim=0).mean(dim=1)
+            mass.append(float(pi[keep].sum()))
+            n_keep = int(keep.sum())
+            ret_tokens += L
+            ret_attended += n_keep
+            all_attended += n_keep
+            planted = inp.planted.get((b, g))
+            if planted is not None and len(planted):
+                pl = torch.from_numpy(np.asarray(planted)).to(dev)
+                recall_hit += int(keep[pl].sum())
+                recall_n += len(planted)
+    total = int(sum(int(inp.seq_lens[b]) for b in range(inp.B))) * inp.Hkv
+    return {"retrieval_sparsity": 1.0 - ret_attended / max(ret_tokens, 1),
+            "overall_sparsity": 1.0 - all_attended / max(total, 1),
+            "index_mass_captured": {"min": min(mass) if mass else None, "mean": float(np.mean(mass)) if mass else None},
+            "planted_recall": recall_hit / recall_n if recall_n else None, "planted_keys": recall_n,
+            "note": "sparsity: share of cached tokens not attended (retrieval heads; all heads); mass: the index "
+                    "distribution's mass on each retrieval slice's attended set (sinks, window, kept); recall: "
+                    "planted keys attended"}
+
+
+def run_config(name, args, B, torch, dev, stream, rank, world, peak, timed, capture):
+    """Headline-style measurement of another workload: graph-replayed steps over two layer
+    copies, algorithmic bytes, achieved GB/s, and the selection metrics."""
+    cfg = dict(synth.CONFIGS[name])
+    p = float(np.float32(cfg["p"]))
+    inp = synth.make_inputs(name, shard.rank_seed(args.seed, rank), draw_streaming_kpre=False)
+    s_kv = 2 if inp.dtype == "bf16" else 4
+
+    def up(a):
+        if inp.dtype == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    P_q, P_k = torch.from_numpy(inp.P_q).to(dev), torch.from_numpy(inp.P_k).to(dev)
+    h = B.spa_create(B.make_config(max_batch=inp.B, n_q_heads=inp.Hq, n_kv_heads=inp.Hkv, max_ctx=inp.Lmax,
+                                   kv_dtype=B.SPA_BF16 if inp.dtype == "bf16" else B.SPA_F32, P_q=P_q, P_k=P_k,
+                                   rope_theta=inp.rope_theta, idx_scale=inp.idx_scale))
+    try:
+        q = up(inp.q_pre)
+        lens = torch.from_numpy(inp.seq_lens).to(dev)
+        k0, v0 = up(inp.k_cache), up(inp.v_cache)
+        kp = up(inp.k_pre)
+        idx0 = torch.zeros((inp.B, inp.Hkv, inp.Lmax, 16), dtype=torch.int16, device=dev)
+        B.spa_index_append(h, kp, torch.zeros(inp.B, dtype=torch.int64, device=dev), inp.B, inp.Lmax, idx0, stream)
+        B.spa_device_status(h, stream)
+        del kp
+        layers = [(k0, v0, idx0), (k0.clone(), v0.clone(), idx0.clone())]
+        out = torch.empty((inp.B, inp.Hq, 128), dtype=torch.float32, device=dev)
+        cnt = torch.zeros(inp.B * inp.Hkv, dtype=torch.int32, device=dev)
+        Lcap = int(inp.seq_lens.max())
+
+        def step(i, st):
+            k, v, ix = layers[i % 2]
+            B.spa_decode(h, q, k, v, ix, inp.head_mask, lens, inp.B, Lcap, p, inp.n_sink, inp.window, out, None, st)
+        step(0, stream)
+        torch.cuda.synchronize(dev)
+        graphs, err = [], None
+        try:
+            graphs = [capture(lambda st, j=j: step(j, st)) for j in range(2)]
+        except Exception as e:
+            err = repr(e)[:200]
+        run = (lambda i: graphs[i % 2].replay()) if graphs else (lambda i: step(i, stream))
+        for i in range(3):
+            run(i)
+        n = max(20, args.steps)
+        ms, _ = timed(n, run)
+        ms = shard.reduce_max(ms, dev) / n
+        del graphs
+        B.spa_decode(h, q, k0, v0, idx0, inp.head_mask, lens, inp.B, Lcap, p, inp.n_sink, inp.window, out, cnt,
+                     stream)
+        B.spa_device_status(h, stream)
+        ab = algorithmic_bytes(inp, cnt.cpu().numpy(), s_kv)
+        gbs = ab["total"] / (ms * 1e-3) / 1e9
+        rec = {"workload": workload_desc(cfg, name, p), "ms_per_step": ms, "layer_steps_per_s": world * 1e3 / ms,
+               "bytes_per_step": ab, "achieved_gbs": gbs, "frac_of_peak": gbs / peak, "steps": n,
+               "timing": "CUDA graph replay, two layer copies cycled" if not err else f"eager ({err})"}
+        rec.update(selection_metrics(B, torch, h, q, idx0, lens, inp, p, Lcap, dev, stream))
+        return rec
+    finally:
+        B.spa_destroy(h)
+        torch.cuda.synchronize(dev)
+        torch.cuda.empty_cache()
+
+
 # ----------------------------------------------------------------------------- reference arm
 def main_reference(args):
     rank, _, world = shard.dist_env()
@@ -218,22 +347,28 @@ def main_reference(args):
                             draw_streaming_kpre=False)
     ret = [g for g in range(inp.Hkv) if inp.head_mask[g]]
     idx = O.index_cache_for(inp, heads=ret)   # BLAS: fast setup, untimed
-    # each step: the oracle's decode of one sequence of the batch (all its KV heads);
-    # a layer-step is B such samples.
-    for i in range(args.warmup):
-        run_oracle_sample(inp, idx, p, [i % inp.B])
-    times = [run_oracle_sample(inp, idx, p, [i % inp.B]) for i in range(args.steps)]
-    sec_per_layer_step = float(np.mean(times)) * inp.B
-    value = 1.0 / sec_per_layer_step
+    # each step: the oracle's decode of a whole layer-step (every slice of the batch), or,
+    # when K + W such steps would take more than about three minutes, of the first
+    # n_seq sequences (the value is then scaled by B / n_seq; ms_per_step is measured)
+    t_one = run_oracle_sample(inp, idx, p, list(range(inp.B)))
+    n_seq = inp.B
+    while n_seq > 1 and (args.steps + args.warmup) * t_one * n_seq / inp.B > 180.0:
+        n_seq -= 1
+    seqs = list(range(n_seq))
+    for _ in range(max(0, args.warmup - 1)):
+        run_oracle_sample(inp, idx, p, seqs)
+    times = [run_oracle_sample(inp, idx, p, seqs) for _ in range(args.steps)]
+    sec_per_step = float(np.mean(times))
+    value = (n_seq / inp.B) / sec_per_step
     cores = cpu_threads()
+    sample = (f"float64 NumPy oracle, a whole layer-step per step (all {inp.B}x{inp.Hkv} slices)" if n_seq == inp.B
+              else f"float64 NumPy oracle, {n_seq} of {inp.B} sequences (all {inp.Hkv} KV heads) per step")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec_per_layer_step * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec_per_step * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_desc(cfg, args.config, p), "batch": inp.B, "seq_len": inp.Lmax, "p": p},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"float64 NumPy oracle, one sequence (all {inp.Hkv} KV heads) per step, "
-                                   f"x{inp.B} per layer-step"},
+        "config": config_dict(cfg, args.config, p, world, args.layers),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -296,9 +431,9 @@ def main_native(args):
     cnt = torch.zeros(inp.B * inp.Hkv, dtype=torch.int32, device=dev)
     Lcap = int(inp.seq_lens.max())
 
-    def step(i, pp=p):
+    def step(i, pp=p, st=stream):
         k, v, ix = layers[i % len(layers)]
-        B.spa_decode(h, q, k, v, ix, head_mask, lens, inp.B, Lcap, pp, inp.n_sink, inp.window, out, None, stream)
+        B.spa_decode(h, q, k, v, ix, head_mask, lens, inp.B, Lcap, pp, inp.n_sink, inp.window, out, None, st)
 
     def barrier():
         if world > 1:
@@ -320,18 +455,78 @@ def main_native(args):
         launches = B.spa_launch_count(h) - n0
         return e0.elapsed_time(e1), launches
 
+    def capture(fn):
+        """fn(st) captured in a CUDA graph on a side stream (thread-local capture mode, so
+        other threads' CUDA calls, e.g. a process group's watchdog, stay legal)."""
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(device=dev)
+        cap.wait_stream(stream)
+        with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
+            fn(None)
+        torch.cuda.synchronize(dev)
+        return g
+
+    class Stepper:
+        """One step per call on layer copy i % layers, replayed from a CUDA graph per copy
+        (eager launches if capture fails; the reason is reported)."""
+
+        def __init__(self, fn):
+            self.fn, self.graphs, self.error = fn, [], None
+            n0 = B.spa_launch_count(h)
+            fn(0, stream)                       # eager warm-up step, counts the launches
+            torch.cuda.synchronize(dev)
+            self.launches = B.spa_launch_count(h) - n0
+            try:
+                self.graphs = [capture(lambda st, j=j: fn(j, st)) for j in range(len(layers))]
+            except Exception as e:
+                self.graphs, self.error = [], repr(e)[:200]
+
+        def __call__(self, i):
+            if self.graphs:
+                self.graphs[i % len(self.graphs)].replay()
+            else:
+                self.fn(i, stream)
+
+        def time(self, n, warm=3):
+            for i in range(warm):
+                self(i)
+            ms, _ = timed(n, self)
+            return shard.reduce_max(ms, dev) / n
+
+        def distribution(self, n):
+            """Per-step device times (us) from events between consecutive steps."""
+            torch.cuda.synchronize(dev)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+            ev[0].record(stream)
+            for i in range(n):
+                self(i)
+                ev[i + 1].record(stream)
+            torch.cuda.synchronize(dev)
+            return [1e3 * ev[i].elapsed_time(ev[i + 1]) for i in range(n)]
+
+        def release(self):
+            self.graphs = []
+
     clocks = ClockSampler(local) if rank == 0 else None
+    main = Stepper(lambda i, st: step(i, st=st))
     for i in range(args.warmup):
-        step(i)
-    # headline: events only around the dominant kernel (attend), on the launch stream
-    ms, launches = timed(args.steps, step, profile_mask=1 << B.SPA_K_ATTEND)
-    tot, n = B.spa_profile_read(h, B.SPA_K_ATTEND)
-    attend_us = 1e3 * tot / max(n, 1)
-    B.spa_set_profiling(h, 0)
+        main(i)
+    # headline: K steps replayed from the graphs, events only at both ends
+    ms, _ = timed(args.steps, main)
     ms_max = shard.reduce_max(ms, dev)
     ms_per_step = ms_max / args.steps
-    # per-kernel breakdown: a separate pass with events around every launch (adds stream gaps)
-    n_brk = max(10, args.steps // 4)
+    launches = main.launches * args.steps
+    # per-step distribution (events between consecutive steps), at least 200 steps
+    n_dist = max(200, args.steps)
+    per_step = np.array(main.distribution(n_dist))
+    dist_us = {"steps": n_dist, "median": float(np.median(per_step)), "p10": float(np.percentile(per_step, 10)),
+               "p90": float(np.percentile(per_step, 90)), "min": float(per_step.min()),
+               "max": float(per_step.max())}
+    # per-kernel breakdown: a separate eager pass with events around every launch
+    # (each event pair adds stream time; the attention kernel's roofline uses it)
+    n_brk = max(20, args.steps)
+    for i in range(3):
+        step(i)
     timed(n_brk, step, profile_mask=(1 << B.SPA_K_COUNT) - 1)
     kern = {}
     for kid in range(B.SPA_K_COUNT):
@@ -339,6 +534,7 @@ def main_native(args):
         if n_k:
             kern[B.spa_kernel_name(kid)] = {"launches": n_k, "avg_us": 1e3 * tot_k / n_k}
     B.spa_set_profiling(h, 0)
+    attend_us = kern.get("attend", {}).get("avg_us", float("nan"))
 
     # selected counts of this workload (identical every step)
     B.spa_decode(h, q, layers[0][0], layers[0][1], layers[0][2], head_mask, lens, inp.B, Lcap, p, inp.n_sink,
@@ -346,67 +542,61 @@ def main_native(args):
     B.spa_device_status(h, stream)
     counts = cnt.cpu().numpy().reshape(inp.B, inp.Hkv)
     ab = algorithmic_bytes(inp, counts, s_kv)
+    peak, peak_kind = measured_peaks()
+
+    def record(ms_step, abx, stepper=None):
+        gbs = abx["total"] / (ms_step * 1e-3) / 1e9
+        r = {"ms_per_step": ms_step, "layer_steps_per_s": world * 1e3 / ms_step, "achieved_gbs": gbs,
+             "frac_of_peak": gbs / peak, "selected_rows": abx["selected_rows"], "bytes_per_step": abx["total"]}
+        if stepper is not None and stepper.error:
+            r["graph_error"] = stepper.error
+        return r
 
     # p sweep (same measurement, smaller step count)
     sweep = {}
     if not args.no_sweep and "p_sweep" in cfg:
         for pp in cfg["p_sweep"]:
             pq = float(np.float32(pp))
-            for i in range(3):
-                step(i, pq)
-            n = max(10, args.steps // 4)
-            msw, _ = timed(n, lambda i: step(i, pq))
-            msw = shard.reduce_max(msw, dev) / n
+            sw = Stepper(lambda i, st, pq=pq: step(i, pq, st))
+            msw = sw.time(max(20, args.steps))
+            sw.release()
             B.spa_decode(h, q, layers[0][0], layers[0][1], layers[0][2], head_mask, lens, inp.B, Lcap, pq,
                          inp.n_sink, inp.window, out, cnt, stream)
             torch.cuda.synchronize(dev)
-            abw = algorithmic_bytes(inp, cnt.cpu().numpy(), s_kv)
-            sweep[f"{pp:g}"] = {"ms_per_step": msw, "layer_steps_per_s": world * 1e3 / msw,
-                                "achieved_gbs": abw["total"] / (msw * 1e-3) / 1e9,
-                                "selected_rows": abw["selected_rows"]}
+            sweep[f"{pp:g}"] = record(msw, algorithmic_bytes(inp, cnt.cpu().numpy(), s_kv), sw)
 
     # top-k selector variant (same measurement, smaller step count)
     topk_sweep = {}
     if not args.no_topk_sweep:
         for kk in (2048, 16384, 65536):
-            def step_k(i, kk=kk):
+            def step_k(i, st, kk=kk):
                 kc, vc, ixc = layers[i % len(layers)]
                 B.spa_decode_topk(h, q, kc, vc, ixc, head_mask, lens, inp.B, Lcap, kk, inp.n_sink, inp.window,
-                                  out, None, stream)
-            for i in range(3):
-                step_k(i)
-            n = max(10, args.steps // 4)
-            msk, _ = timed(n, step_k)
-            msk = shard.reduce_max(msk, dev) / n
+                                  out, None, st)
+            sk = Stepper(step_k)
+            msk = sk.time(max(20, args.steps))
+            sk.release()
             B.spa_decode_topk(h, q, layers[0][0], layers[0][1], layers[0][2], head_mask, lens, inp.B, Lcap, kk,
                               inp.n_sink, inp.window, out, cnt, stream)
             torch.cuda.synchronize(dev)
-            abk = algorithmic_bytes(inp, cnt.cpu().numpy(), s_kv)
-            topk_sweep[str(kk)] = {"ms_per_step": msk, "layer_steps_per_s": world * 1e3 / msk,
-                                   "achieved_gbs": abk["total"] / (msk * 1e-3) / 1e9,
-                                   "selected_rows": abk["selected_rows"]}
+            topk_sweep[str(kk)] = record(msk, algorithmic_bytes(inp, cnt.cpu().numpy(), s_kv), sk)
 
     # block-granular top-p variant (64-token blocks; same measurement, smaller step count)
     block_sweep = {}
     if not args.no_block_sweep:
         for pp in (0.9, 0.99):
             pq = float(np.float32(pp))
-            def step_b(i, pq=pq):
+            def step_b(i, st, pq=pq):
                 kc, vc, ixc = layers[i % len(layers)]
                 B.spa_decode_blocks(h, q, kc, vc, ixc, head_mask, lens, inp.B, Lcap, pq, inp.n_sink, inp.window,
-                                    out, None, stream)
-            for i in range(3):
-                step_b(i)
-            n = max(10, args.steps // 4)
-            msb, _ = timed(n, step_b)
-            msb = shard.reduce_max(msb, dev) / n
+                                    out, None, st)
+            sb = Stepper(step_b)
+            msb = sb.time(max(20, args.steps))
+            sb.release()
             B.spa_decode_blocks(h, q, layers[0][0], layers[0][1], layers[0][2], head_mask, lens, inp.B, Lcap, pq,
                                 inp.n_sink, inp.window, out, cnt, stream)
             torch.cuda.synchronize(dev)
-            abb = algorithmic_bytes(inp, cnt.cpu().numpy(), s_kv)
-            block_sweep[f"{pp:g}"] = {"ms_per_step": msb, "layer_steps_per_s": world * 1e3 / msb,
-                                      "achieved_gbs": abb["total"] / (msb * 1e-3) / 1e9,
-                                      "selected_rows": abb["selected_rows"]}
+            block_sweep[f"{pp:g}"] = record(msb, algorithmic_bytes(inp, cnt.cpu().numpy(), s_kv), sb)
 
     # compact KV layout: streaming heads keep only sinks + a ring-buffered window
     compact = None
@@ -427,15 +617,13 @@ def main_native(args):
             c_layers.append((kr, vr, ks, vs, ix[:, ret].contiguous()))
         B.spa_device_status(h, stream)
 
-        def step_c(i):
+        def step_c(i, st):
             kr, vr, ks, vs, ixr = c_layers[i % len(c_layers)]
             B.spa_decode_compact(h, q, kr, vr, ks, vs, ixr, head_mask, lens, inp.B, Lcap, p, inp.n_sink,
-                                 inp.window, out, None, stream)
-        for i in range(3):
-            step_c(i)
-        n = max(10, args.steps // 4)
-        msc, _ = timed(n, step_c)
-        msc = shard.reduce_max(msc, dev) / n
+                                 inp.window, out, None, st)
+        sc = Stepper(step_c)
+        msc = sc.time(max(20, args.steps))
+        sc.release()
         row = 128 * s_kv * 2   # K + V bytes per position and head
         full_b = inp.B * inp.Hkv * inp.Lmax * row
         comp_b = inp.B * (n_ret * inp.Lmax + n_str * ring) * row
@@ -654,10 +842,41 @@ def main_native(args):
                "d2h_bytes_per_step": int(d2h), "ms_per_step": mse,
                "note": "copies on a second stream, double-buffered: step i+1's inputs load and step i-1's "
                        "output drains while step i computes"}
+    # selection metrics of the headline workload (reported, outside every timed region)
+    sel_metrics = selection_metrics(B, torch, h, q, layers[0][2], lens, inp, p, Lcap, dev, stream)
+
+    # index append throughput: the whole prefill of every head's index rows
+    iapp = None
+    if not args.no_index_append:
+        kp = up(inp.k_pre)
+        zero = torch.zeros(inp.B, dtype=torch.int64, device=dev)
+        ix_t = torch.empty_like(layers[0][2])
+
+        def step_ia(i, st):
+            B.spa_index_append(h, kp, zero, inp.B, inp.Lmax, ix_t, st)
+        sia = Stepper(step_ia)
+        n = 10
+        msi = sia.time(n)
+        sia.release()
+        B.spa_device_status(h, stream)
+        rows = inp.B * inp.Hkv * inp.Lmax
+        byts = rows * (128 * s_kv + 32)
+        gbs = byts / (msi * 1e-3) / 1e9
+        iapp = {"rows": rows, "ms": msi, "bytes": byts, "achieved_gbs": gbs, "frac_of_peak": gbs / peak,
+                "peak": peak, "peak_kind": peak_kind, "bound": "hbm",
+                "note": f"{inp.B}x{inp.Hkv} (sequence, KV head) slices x {inp.Lmax} positions: "
+                        f"{128 * s_kv} B of pre-RoPE key read and 32 B of index row written per row"}
+        del kp, ix_t
+
+    # the other workloads, one sub-record each (a smaller step count)
+    per_config = {}
+    if not args.no_configs:
+        for name in [c for c in ("llama3_8b_32k", "batch16_64k", "ctx1m") if c != args.config]:
+            per_config[name] = run_config(name, args, B, torch, dev, stream, rank, world, peak, timed, capture)
+
     clk = clocks.stop() if clocks else None
 
     if rank == 0:
-        peak, peak_kind = measured_peaks()
         att_bytes = (ab["contig_rows"] + ab["selected_rows"]) * 2 * 128 * s_kv
         achieved = att_bytes / (attend_us * 1e-6) / 1e9
         traffic = recorded_traffic("k_attend_mma.cu", "attend_ctx128k.md") if args.config == "ctx128k" else None
@@ -677,20 +896,22 @@ def main_native(args):
             "metric": METRIC, "value": world * 1e3 / ms_per_step, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": workload_desc(cfg, args.config, p), "batch": inp.B, "seq_len": inp.Lmax,
-                       "p": p, "storage": inp.dtype, "parallelism": f"dp{world}" if world > 1 else "single",
-                       "l2": f"inputs larger than L2: {len(layers)} layer copies of "
-                             f"{(layers[0][0].numel() * 2 * s_kv + layers[0][2].numel() * 2) / 1e9:.2f} GB "
-                             f"cycled; {ab['total'] / 1e6:.0f} MB touched per step"},
+            "config": config_dict(cfg, args.config, p, world, len(layers)),
+            "timing": ("each step replayed from a CUDA graph (one per layer copy); CUDA events on the launch "
+                       "stream at both ends of the K timed steps" if main.graphs else
+                       f"eager launches (graph capture failed: {main.error}); CUDA events at both ends"),
+            "step_us_distribution": dist_us,
             "achieved_gbs": step_gbs,
             "frac_of_peak": step_gbs / peak,
             "bytes_per_step": ab,
             "selected_counts": counts.tolist(),
             "kernels_us": kern,
-            "kernels_us_note": "separate pass with CUDA events around every launch; each pair adds stream gaps",
+            "kernels_us_note": "separate eager pass with CUDA events around every launch; each pair adds stream time",
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "kernel": "attend",
-                         "avg_us": attend_us, "bytes_per_launch": att_bytes, "peak_kind": peak_kind},
+                         "avg_us": attend_us, "bytes_per_launch": att_bytes, "peak_kind": peak_kind,
+                         "step_achieved": step_gbs, "step_frac": step_gbs / peak,
+                         "step_bytes": ab["total"], "step_us": ms_per_step * 1e3},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": int(launches),
@@ -701,6 +922,9 @@ def main_native(args):
             "compact": compact,
             "prefill": prefill,
             "context_parallel": cpar,
+            "selection": sel_metrics,
+            "index_append": iapp,
+            "configs": per_config or None,
         }
         print(json.dumps(line), flush=True)
     B.spa_destroy(h)

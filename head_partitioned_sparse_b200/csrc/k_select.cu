@@ -8,47 +8,53 @@
 // Group mean of per-head probabilities: "Autonomy of Heads" summary, Deployment
 // strategy (GQA scores aggregated to the group by their mean).
 //
-// Phases (units: retrieval slices s = (b, g); the score and mass phases split the
-// slices' 16-token groups into equal ranges per CTA, the later phases work on chunks of
-// kChunk tokens):
-//   score     the leader CTA of each slice computes q_idx = P_q q_pre (float64 dot
-//             products) and publishes it (flag); every range then forms, per head h,
-//             m = max_j l_hj, z = sum_j 2^(l_hj - m),
+// Work partition: the retrieval slices' capacity, in 16-token groups, is split into
+// equal contiguous ranges, one per CTA; a range may span slices (one segment per slice
+// it touches).  Every phase works on the CTA's own range, and the probabilities of the
+// range stay in shared memory from the mass phase to the compaction.
+// Phases:
+//   score     each CTA forms the group's query index vectors q_idx = P_q q_pre itself
+//             (float64 dot products) while its first index rows are in flight, then per
+//             head h: m = max_j l_hj, z = sum_j 2^(l_hj - m),
 //             l_hj = log2(e) * idx_scale * <q_idx[h], idx_j>   (index read #1);
 //   -- grid barrier --
-//   mass      merge (m, z) over ranges -> M_h, Z_h; recompute l_hj (index read #2),
-//             pi_j = sum_h 2^(l_hj - M_h) / (G Z_h), stored as fp32; a mass histogram
-//             over the top 12 bits of pi_j's bit pattern, masses quantised to integer
-//             multiples of 2^-63 so every sum is exact and order independent (per range
-//             as a count and a sum of low significand bits per bin, 32-bit atomics);
+//   mass      merge (m, z) over the slice's ranges -> M_h, Z_h; recompute l_hj (index
+//             read #2, from L2), pi_j = sum_h 2^(l_hj - M_h) / (G Z_h), kept on chip; a
+//             mass histogram over the top 12 bits of pi_j's bit pattern, masses as
+//             integer multiples of 2^-63 so every sum is exact and order independent
+//             (per range as a count and a sum of low significand bits per bin);
 //   cut 1     per slice (last range, ticket): total mass, target ceil(p * total) (or k
 //             for top-k) and the bin b1 where the descending cumulative mass reaches it;
 //   -- grid barrier --
-//   threshold per chunk: tokens above b1 counted, tokens of bin b1 appended as
+//   threshold per range: tokens above b1 counted, tokens of bin b1 appended as
 //             candidates with their round-2 masses added to the slice histogram;
-//   refine    per slice (last chunk, ticket): round-2 bin b2 from the histogram, one
-//             pass over the candidates for round 3 (exact cut value tau), the tie quota
-//             at tau (lowest positions first) and per-chunk output offsets; idle CTAs
-//             compute q_rot = RoPE(q_pre, L-1) for every head as duties (angles in
-//             float64, reduced exactly in units of pi);
+//   refine    per slice (last range, ticket): the exact cut from the candidates - the
+//             value tau and the position up to which tokens equal to tau are kept
+//             (lowest positions first) - by an on-chip sort when they are few, else by
+//             two more radix rounds over the histogram; per-range output offsets.
+//             Meanwhile every CTA prefetches its share of the sink and window K/V rows
+//             into L2 for the attention kernel that follows (HBM is otherwise idle in
+//             these phases), and idle CTAs compute q_rot = RoPE(q_pre, L-1) for every
+//             head as duties (angles in float64, reduced exactly in units of pi);
 //   -- grid barrier --
-//   compact   per chunk: kept positions outside sinks/window, ascending.
+//   compact   per range: kept positions outside sinks/window, ascending.
 // Block mode (the block-granular variant, a second instantiation): the ranges are cut at
-// kBlock-token block boundaries, the mass phase stores and histograms each block's mass
-// (the float32 sum of its tokens' pi) instead of the tokens', the threshold, refine and
-// compact steps rank blocks and count their listed tokens, and compact lists every
-// token of a kept block.  The blocks follow the chunk routing of the "Hierarchical
-// Global Attention" summary, Central mechanism §4.
+// kBlock-token block boundaries, the mass phase keeps and histograms each block's mass
+// (the float32 sum of its tokens' pi) instead of the tokens', the threshold and refine
+// steps rank blocks and count their listed tokens, and compact lists every token of a
+// kept block.  The blocks follow the chunk routing of the "Hierarchical Global
+// Attention" summary, Central mechanism §4.
 // One launch replaces a chain of small kernels whose fixed launch cost dominated.
-// Grid barriers and the q_idx flags are polled with a clock budget; on timeout they set
-// a device status bit and the kernel leaves or carries on without hanging.  The launch
-// is cooperative, so all CTAs are resident together.
+// Grid barriers are polled with a clock budget; on timeout they set a device status bit
+// and the kernel leaves without hanging.  The launch is cooperative, so all CTAs are
+// resident together.
 #include <climits>
 
 #include "spa_internal.cuh"
 
 namespace spa {
 namespace {
+
 
 constexpr unsigned kFull = 0xffffffffu;
 
@@ -107,26 +113,6 @@ __device__ void find_cut_desc_4096(const unsigned long long (&m)[16], unsigned l
     if (cum < target && nxt >= target) {
       *out_bin = hi - k;
       *out_above = cum;
-    }
-    cum = nxt;
-  }
-  __syncthreads();
-}
-
-// Ascending count search: thread t owns bins [16 t, 16 t + 15].  Finds the bin where the
-// running count (starting at base) first reaches q.
-__device__ void find_kth_asc_4096(const unsigned (&c)[16], unsigned base, unsigned q, unsigned* sh,
-                                  int* out_bin, unsigned* out_before) {
-  unsigned s = 0;
-#pragma unroll
-  for (int k = 0; k < 16; ++k) s += c[k];
-  unsigned cum = base + block_excl_scan(s, sh, (unsigned*)nullptr);
-#pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const unsigned nxt = cum + c[k];
-    if (cum < q && nxt >= q) {
-      *out_bin = 16 * (int)threadIdx.x + k;
-      *out_before = cum;
     }
     cum = nxt;
   }
@@ -319,31 +305,35 @@ __device__ __forceinline__ void online_add(float& m, float& z, float l) {
 
 
 
-// ------------------------------------------------------------------ grid barrier
-constexpr long long kBarrierCycles = 4000000000LL;   // ~2 s bound per barrier
+// ------------------------------------------------------------------ per-slice synchronisation
+// The phases of a slice wait only for the CTA ranges of that slice: a range arrives at
+// the slice's counter for a phase once its output of that phase is stored (the counters
+// are reset by the prologue kernel before every launch), and a phase that needs the
+// whole slice waits until every range of the slice has arrived.  The launch is
+// cooperative, so every CTA that may be waited for is resident.
+constexpr long long kWaitCycles = 4000000000LL;   // ~2 s bound per wait
 
-// Barrier over all CTAs of a cooperative launch on one arrival word bar[0]: CTA 0
-// adds 2^31 - (nb - 1), every other CTA adds 1, so the word's top bit flips exactly
-// when the last CTA arrives and its low 31 bits return to their value (no reset, and
-// the release is the last arrival itself).  Every CTA polls until the top bit differs
-// from the one it saw on arrival.  The CTA whose arrival flips the bit also advances
-// the generation word bar[32] (its own 128-byte line), which tags the q_idx flags of
-// a call.  Returns false (on every thread of the CTA) if the wait gave up.
-__device__ bool grid_barrier(unsigned* bar, unsigned* err, int* s_ok) {
+// This CTA's range arrives at counter ctr (called by every thread of the CTA): every
+// thread fences its own writes of the phase, then one arrival for the CTA.
+__device__ __forceinline__ void slice_arrive(unsigned* ctr) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) atomicAdd(ctr, 1u);
+}
+
+// Waits (thread 0, polled with back-off, bounded) until n ranges have arrived at ctr;
+// returns false on every thread of the CTA if the wait gave up (the status word then
+// holds kErrTimeout).
+__device__ bool slice_wait(unsigned* ctr, unsigned n, unsigned* err, int* s_ok) {
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
-    const unsigned add = blockIdx.x == 0 ? 0x80000000u - (gridDim.x - 1u) : 1u;
-    __threadfence();
-    const unsigned old = atomicAdd(bar, add);
-    if (((old + add) ^ old) & 0x80000000u) {
-      atomicAdd(bar + 32, 1u);
-    } else {
-      volatile unsigned* word = bar;
+    volatile unsigned* w = ctr;
+    if (*w < n) {
       const long long t0 = clock64();
       unsigned ns = 32;
-      while (((*word ^ old) & 0x80000000u) == 0u) {
-        if (clock64() - t0 > kBarrierCycles) {
+      while (*w < n) {
+        if (clock64() - t0 > kWaitCycles) {
           atomicOr(err, kErrTimeout);
           ok = 0;
           break;
@@ -359,32 +349,24 @@ __device__ bool grid_barrier(unsigned* bar, unsigned* err, int* s_ok) {
   return *s_ok != 0;
 }
 
-// "Last CTA of the slice" ticket: every unit of the slice takes one; the CTA that
-// takes the last runs the per-slice step.  Called by every thread of the CTA.
-__device__ bool last_of_slice(unsigned* ticket, unsigned n_units, int* s_flag) {
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) *s_flag = atomicAdd(ticket, 1u) == n_units - 1;
-  __syncthreads();
-  if (*s_flag) __threadfence();
-  return *s_flag != 0;
-}
-
 // ------------------------------------------------------------------ shared memory
 constexpr int kWarps = kSelThreads / 32;
-constexpr int kGroupBatch = 4;                // groups per warp loaded together (8 spills at 64 registers)
-constexpr int kSmallCap = 1024;   // candidates of the round-2 cut bin held in shared memory
-constexpr int kCandBatch = 8;     // candidates loaded per thread before any is used
+constexpr int kGroupBatch = 4;    // groups per warp loaded together (8 spills at 64 registers)
+constexpr int kPiCap = 4096;      // probabilities of a range kept on chip (dynamic shared memory)
+constexpr int kPiBytes = kPiCap * 4;
+constexpr int kSmallList = 2048;  // candidates of the round-A cut digit kept on chip by the refine step
+constexpr int kTieCap = 256;      // candidates equal to the cut value ranked directly
+constexpr int kRefBatch = 8;      // candidate loads per thread issued together by the refine step
 
 struct SmemPro { double cs[kHeadDim / 2], sn[kHeadDim / 2]; };
 struct SmemScore { float2 red[kSelThreads / 32][kMaxGroup]; };
 struct SmemMass { unsigned cnt[kBins1], low[kBins1]; float Mh[kMaxGroup], Wh[kMaxGroup]; };
 struct SmemRefine {
-  int chunk_sel[kMaxChunks];      // kept candidates per chunk (listed ones)
-  unsigned cnt4k[4096];           // position-select histogram
-  uint2 small[kSmallCap];         // candidates of the round-2 cut bin
-  unsigned long long m3[kBins3];
-  unsigned c3[kBins3];
+  uint2 small[kSmallList];            // candidates of the round-A cut digit (bits, element)
+  unsigned hc[512];                   // radix round: count per digit
+  unsigned hl[512];                   // radix round: sum of the bits below the digit
+  int tie[kTieCap];                   // positions of the candidates equal to the cut value
+  int wcnt[kSelThreads / 32];         // per-warp counts
 };
 // Round-1 / round-2 histogram staged for the cut search: loaded coalesced, read back as
 // 16 consecutive bins per thread (index i stored at i + i / 16 against bank conflicts).
@@ -402,9 +384,9 @@ struct SelScalars {
   unsigned long long shl[32];
   unsigned shu[32];
   int shi[32];
-  int L, b1, b2, b3, kbin, fbin, cut_bin, pos_cut, off, ok, duty;
-  unsigned small_n, kbefore, fbefore, tau;
-  unsigned long long above2, cut_above;
+  int L, b1, cut_bin, pos_cut, off, ok, digit, ntie;
+  unsigned tau, ncand, nsmall, cbase;
+  unsigned long long cut_above, above, target, m_above;
 };
 
 // Unit coordinates: retrieval slice y -> (b, g, s).
@@ -428,8 +410,7 @@ __device__ __forceinline__ int cta_len(const StepParams& P, int b, SelScalars& s
 
 // ------------------------------------------------------------------ query rotation
 // RoPE of slice s's G query heads at position L-1 (streaming slices included), read by
-// the attention kernels after this launch; a streaming slice's selection count is 0.
-// Taken as a "duty" by CTAs that wait at the last barrier anyway.
+// the attention kernels after this launch.
 template <typename T>
 __device__ void qrot_slice(const StepParams& P, SmemPro& sm, SelScalars& sc, int s) {
   const int b = s / P.Hkv, g = s % P.Hkv, G = P.G;
@@ -453,24 +434,7 @@ __device__ void qrot_slice(const StepParams& P, SmemPro& sm, SelScalars& sc, int
     o[i] = (float)(x1 * sm.cs[i] - x2 * sm.sn[i]);
     o[i + kHeadDim / 2] = (float)(x2 * sm.cs[i] + x1 * sm.sn[i]);
   }
-  if (!P.is_ret[g] && tid == 0) {
-    P.ws.st[s].count = 0;
-    if (P.sel_count) P.sel_count[s] = 0;
-  }
-  __syncthreads();   // sm.cs / sm.sn reused by the next duty
-}
-
-// Takes q_rot duties (slices) from a grid-wide ticket until none is left.
-template <typename T>
-__device__ void qrot_duties(const StepParams& P, SmemPro& sm, SelScalars& sc) {
-  for (;;) {
-    __syncthreads();
-    if (threadIdx.x == 0) sc.duty = (int)atomicAdd(P.ws.bar + kBarDuty, 1u);
-    __syncthreads();
-    const int s = sc.duty;
-    if (s >= P.n_slices) return;
-    qrot_slice<T>(P, sm, sc, s);
-  }
+  __syncthreads();   // sm.cs / sm.sn and sc.L are reused
 }
 
 // ------------------------------------------------------------------ query index vectors
@@ -541,14 +505,56 @@ __device__ void compute_qidx(const StepParams& P, int b, int g, SelScalars& sc) 
   __syncthreads();
 }
 
+// Round-A histogram of slice s (candidates of its round-1 cut bin by bits 17..9): 512
+// counts, then 512 sums of bits 8..0.  It lives in the slice's round-2 histogram row,
+// which the one-GPU selection does not otherwise use.
+__device__ __forceinline__ unsigned* hist_a(const StepParams& P, int s) {
+  return reinterpret_cast<unsigned*>(P.ws.hist2 + (size_t)s * kBins2);
+}
+
+// ------------------------------------------------------------------ query prologue kernel
+// One CTA per (b, kv head) slice, launched before the selection kernel: q_rot for the
+// slice's G heads (decode calls), and for a retrieval slice q_idx = P_q q_pre (float64
+// dot products), the reset of its selection state (arrival counters included) and of its
+// round-1 histogram.  A streaming slice's selection count is 0.  Forming these once per
+// slice lets every CTA of the selection kernel start streaming index rows at once.
+template <typename T, int G>
+__global__ void __launch_bounds__(kSelThreads) k_qprep(StepParams P) {
+  __shared__ SmemPro sm;
+  __shared__ SelScalars sc;
+  const int s = blockIdx.x, b = s / P.Hkv, g = s % P.Hkv, tid = threadIdx.x;
+  if (P.is_ret[g]) {
+    if (tid == 0) {
+      SliceState z;
+      z.target = z.m_above = 0ull;
+      z.b1 = -1;
+      z.count = 0;
+      z.arr_score = z.arr_mass = z.arr_thr = z.arr_cnt = 0u;
+      z.ncand = z.tau_bits = 0u;
+      z.pos_cut = INT_MAX;
+      P.ws.st[s] = z;
+    }
+    unsigned long long* h1 = P.ws.hist1 + (size_t)s * kBins1;
+    for (int i = tid; i < kBins1; i += kSelThreads) h1[i] = 0ull;
+    unsigned* ha = hist_a(P, s);
+    for (int i = tid; i < 1024; i += kSelThreads) ha[i] = 0u;
+    compute_qidx<T, G>(P, b, g, sc);
+    if (tid < G * kIdxDim) P.ws.q_idx[((size_t)b * P.Hq + (size_t)g * G) * kIdxDim + tid] = sc.qsm[tid];
+  } else if (tid == 0) {
+    P.ws.st[s].count = 0;
+    if (P.sel_count) P.sel_count[s] = 0;
+  }
+  if (P.k_cache) qrot_slice<T>(P, sm, sc, s);
+}
+
 // ------------------------------------------------------------------ work partition
-// The score and mass phases split the retrieval slices' capacity (max_seq_len tokens
-// each, as ngc 16-token groups; slice y = b * n_ret + r owns global groups
-// [y ngc, (y+1) ngc)) into equal contiguous group ranges, one per CTA, so every SM of a
-// full-occupancy grid gets the same share.  A range may span slices; groups past a
-// sequence's length are empty.  Ranges are cut at multiples of q groups (q = 1, or
-// kBlock / 16 in block mode so that no block is split; ngc is then a multiple of q):
-// CTA c covers groups [q floor(c Q / nb), q floor((c+1) Q / nb)), Q = n_rs ngc / q.
+// The retrieval slices' capacity (max_seq_len tokens each, as ngc 16-token groups;
+// slice y = b * n_ret + r owns global groups [y ngc, (y+1) ngc)) is split into equal
+// contiguous group ranges, one per CTA, so every SM of a full-occupancy grid gets the
+// same share.  A range may span slices; groups past a sequence's length are empty.
+// Ranges are cut at multiples of q groups (q = 1, or kBlock / 16 in block mode so that
+// no block is split; ngc is then a multiple of q): CTA c covers groups
+// [q floor(c Q / nb), q floor((c+1) Q / nb)), Q = n_rs ngc / q.
 template <bool BLK>
 struct Ranges {
   static constexpr int q = BLK ? kBlock / 16 : 1;
@@ -565,9 +571,9 @@ struct Ranges {
   __device__ __forceinline__ int first_cta(int y) const { return owner((long long)y * ngc); }
   __device__ __forceinline__ int last_cta(int y) const { return owner((long long)(y + 1) * ngc - 1); }
 };
-// Per-range statistics of slice y live at stats[(cta + y) * G]: the CTAs of slice y
-// are consecutive and the last one of y may be the first one of y + 1, so the slots
-// of different slices never overlap (at most nb + n_rs of them).
+// Per-range values of slice y (statistics, counts, offsets) live at slot cta + y: the
+// CTAs of slice y are consecutive and the last one of y may be the first one of y + 1,
+// so the slots of different slices never overlap (at most nb + n_rs of them).
 __device__ __forceinline__ size_t stats_slot(int cta, int y) { return (size_t)cta + (size_t)y; }
 
 // Visits the CTA's range as segments f(y, l0, l1) of local groups [l0, l1) of slice y.
@@ -582,86 +588,51 @@ __device__ __forceinline__ void for_each_segment(const RT& R, F&& f) {
   }
 }
 
+// Probabilities of the CTA's range: element e of a segment's slice (token e, or block e
+// in block mode) lives on chip at its offset from the range's first token (or block),
+// or, past the first kPiCap elements of the range, in the global rows
+// [slices][pi_stride].  One view per segment: t0 = the range-relative offset of the
+// slice's element 0, s = the slice.
+extern __shared__ float s_pi[];   // dynamic shared memory of the selection kernel: kPiCap floats
+struct PiSeg {
+  int t0, s;
+};
+template <bool BLK>
+__device__ __forceinline__ PiSeg pi_seg(const Ranges<BLK>& R, int y, int s) {
+  const long long t0 = 16 * ((long long)y * R.ngc - R.begin(blockIdx.x));
+  PiSeg v;
+  v.t0 = (int)(BLK ? t0 / kBlock : t0);
+  v.s = s;
+  return v;
+}
+__device__ __forceinline__ void pi_store(const StepParams& P, PiSeg ps, int e, float v) {
+  const int loc = ps.t0 + e;
+  if (loc < kPiCap) s_pi[loc] = v;
+  else P.ws.pi[(size_t)ps.s * P.ws.pi_stride + e] = v;
+}
+__device__ __forceinline__ float pi_load(const StepParams& P, PiSeg ps, int e) {
+  const int loc = ps.t0 + e;
+  return loc < kPiCap ? s_pi[loc] : __ldcg(P.ws.pi + (size_t)ps.s * P.ws.pi_stride + e);
+}
+// elements e .. e + 3 (e a multiple of 4; token mode: t0 is a multiple of 16, so the
+// four sit on one side of kPiCap and are 16-byte aligned on either side)
+__device__ __forceinline__ float4 pi_load4(const StepParams& P, PiSeg ps, int e) {
+  const int loc = ps.t0 + e;
+  return loc < kPiCap ? *reinterpret_cast<const float4*>(s_pi + loc)
+                      : __ldcg(reinterpret_cast<const float4*>(P.ws.pi + (size_t)ps.s * P.ws.pi_stride + e));
+}
+
 // ------------------------------------------------------------------ score phase
-// The leader of slice y (the CTA holding its first group) resets the slice state,
-// computes the group's query index vectors, stores them and publishes them with a flag
-// tagged with this call's barrier generation; every range of the slice reads them after
-// the flag (bounded wait).  A CTA leads its slices before it scores any range, and only
-// waits for lower-numbered CTAs, so the waits always end.
-template <typename T, int G>
-__device__ void lead_slice(const StepParams& P, SelScalars& sc, int y) {
-  const Unit un = unit_of(P, y);
-  SliceState* st = P.ws.st + un.s;
-  unsigned gen = 0u;   // barrier generation (thread 0): constant while any CTA scores
-  if (threadIdx.x == 0) gen = *reinterpret_cast<volatile unsigned*>(P.ws.bar + 32);
-  __syncthreads();   // earlier readers of sc.qsm / sc.L are done
-  if (threadIdx.x == 0) {
-    SliceState z;
-    z.q_total = z.target = z.m_above = 0ull;
-    z.b1 = -1;
-    z.tau_bits = 0u;
-    z.pos_cut = INT_MAX;
-    z.count = 0;
-    z.cand_count = 0u;
-    z.ticket_mass = z.ticket_thr = 0u;
-    z.qidx_ready = 0u;
-    *st = z;
-  }
-  compute_qidx<T, G>(P, un.b, un.g, sc);
-  if (threadIdx.x < G * kIdxDim) {
-    P.ws.q_idx[((size_t)un.b * P.Hq + (size_t)un.g * G) * kIdxDim + threadIdx.x] = sc.qsm[threadIdx.x];
-    __threadfence();
-  }
-  __syncthreads();
-  // (the failure-detection test hook leaves the flag unset: the other CTAs' bounded
-  // waits then run out and report a timeout)
-  if (threadIdx.x == 0 && !P.drop_publish) atomicExch(&st->qidx_ready, gen + 1u);
-}
-
-// Waits (thread 0, bounded) for slice s's q_idx flag of this call; the caller
-// synchronises the CTA afterwards.  The barrier generation that tags the flag cannot
-// change before this CTA reaches the first grid barrier.
-__device__ __forceinline__ void wait_qidx(const StepParams& P, int s) {
-  volatile unsigned* flag = &P.ws.st[s].qidx_ready;
-  const unsigned want = *reinterpret_cast<volatile unsigned*>(P.ws.bar + 32) + 1u;
-  const long long t0 = clock64();
-  unsigned ns = 32;
-  while (*flag != want) {
-    if (clock64() - t0 > kBarrierCycles) {
-      atomicOr(P.ws.dev_err, kErrTimeout);
-      break;
-    }
-    __nanosleep(ns);
-    if (ns < 128) ns <<= 1;
-  }
-  __threadfence();
-}
-
-// Clears the CTA's share of slice y's round-1 / round-2 histograms (read after a barrier).
-template <class RT>
-__device__ __forceinline__ void clear_hist_share(const StepParams& P, const RT& R, int y, int s) {
-  static_assert(kBins1 == kBins2, "histogram reset assumes equal round-1 / round-2 bin counts");
-  const int first = R.first_cta(y), n = R.last_cta(y) - first + 1, k = (int)blockIdx.x - first;
-  unsigned long long* h1 = P.ws.hist1 + (size_t)s * kBins1;
-  unsigned long long* h2 = P.ws.hist2 + (size_t)s * kBins2;
-  for (int i = k * kSelThreads + (int)threadIdx.x; i < kBins1; i += n * kSelThreads) {
-    h1[i] = 0ull;
-    h2[i] = 0ull;
-  }
-}
-
 // One range of slice y: per head m = max_j l_hj, z = sum_j 2^(l_hj - m) over the tokens
 // of local groups [l0, l1), l_hj = log2(e) * idx_scale * <q_idx[h], idx_j>.  Warp w takes
 // groups l0 + w, l0 + w + 8, ..., kGroupBatch at a time; the first batch is requested
-// before the query vectors arrive (bounded by the call's max length; rows past the
-// sequence are masked).
-template <int G, class RT>
-__device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc, const RT& R, int y,
-                              int l0, int l1) {
+// before the query index vectors are read (bounded by the call's max length; rows past
+// the sequence are masked).
+template <int G>
+__device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc, int y, int l0, int l1) {
   constexpr int NH = IdxTiles<G>::NH, U = kGroupBatch;
   const Unit un = unit_of(P, y);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, t4 = lane & 3, gid = lane >> 2;
-  clear_hist_share(P, R, y, un.s);
   const uint2* rows = reinterpret_cast<const uint2*>(idx_rows(P, y, un.s));
   const uint64_t pol = l2_policy_keep();
   uint2 ra[U], rb[U];
@@ -670,10 +641,18 @@ __device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc
 #pragma unroll
     for (int u = 0; u < U; ++u) load_group(rows, 16 * (l0 + warp + kWarps * u), jpf, pol, ra[u], rb[u]);
   }
+  // the sequence length and the query index vectors (formed by the prologue kernel)
+  // are requested behind the first batch; one CTA barrier publishes them
   __syncthreads();   // earlier readers of sc.L and sc.qsm are done
+  int64_t len_raw = 0;
+  if (tid == 0) len_raw = P.seq_lens[un.b];
+  if (tid < G * kIdxDim) sc.qsm[tid] = __ldcg(&P.ws.q_idx[((size_t)un.b * P.Hq + (size_t)un.g * G) * kIdxDim + tid]);
   if (tid == 0) {
-    sc.L = load_len(P.seq_lens, un.b, P.Lcap, P.ws.dev_err);
-    if (16 * l0 < sc.L) wait_qidx(P, un.s);
+    if (len_raw < 1 || len_raw > P.Lcap) {
+      atomicOr(P.ws.dev_err, kErrSeqLen);
+      len_raw = len_raw < 1 ? 1 : P.Lcap;
+    }
+    sc.L = (int)len_raw;
   }
   __syncthreads();
   const int L = sc.L;
@@ -683,7 +662,7 @@ __device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc
     return;
   }
   uint32_t qb[IdxTiles<G>::NT][2];
-  load_qidx_frag<G>(P, un.b, un.g, sc.qsm, qb);
+  qidx_frag<G>(sc.qsm, qb);
   const float scale = P.idx_scale_log2;
   const int jend = min(L, 16 * l1);
   // two independent online accumulators per head (tokens gid and gid + 8)
@@ -726,19 +705,16 @@ __device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc
     for (int w = 0; w < kWarps; ++w) merge_mz(mm, zz, sm.red[w][tid].x, sm.red[w][tid].y);
     out[tid] = make_float2(mm, zz);
   }
-  __syncthreads();   // sm.red reused by the next range
+  __syncthreads();   // sm.red, sc.L and sc.qsm are reused by the next segment
 }
 
-template <typename T, int G, bool BLK>
-__device__ void score_phase(const StepParams& P, SmemScore& sm, SelScalars& sc) {
-  const Ranges<BLK> R(P);
-  const long long ga = R.begin(blockIdx.x), ge = R.begin(blockIdx.x + 1);
-  for (long long y = (ga + R.ngc - 1) / R.ngc; y * R.ngc < ge; ++y) lead_slice<T, G>(P, sc, (int)y);
-  for_each_segment(R, [&](int y, int l0, int l1) { score_segment<G>(P, sm, sc, R, y, l0, l1); });
-}
-
-// ------------------------------------------------------------------ cut 1 (per slice)
-__device__ void cut1_slice(const StepParams& P, SmemStage& sm, SelScalars& sc, int y) {
+// ------------------------------------------------------------------ cut 1 (per range)
+// Every CTA of a slice takes the slice's round-1 cut from the complete round-1 histogram
+// (32 KB, read from L2): total mass, target ceil(p * total) (or k for top-k) and the bin
+// b1 where the descending cumulative mass reaches it (-1: keep every token).  Results in
+// sc.b1, sc.target, sc.m_above; the slice's first CTA also stores them for the refine
+// step of every range.
+__device__ void cut1_range(const StepParams& P, SmemStage& sm, SelScalars& sc, int y, bool lead) {
   const Unit un = unit_of(P, y);
   const int tid = threadIdx.x;
   unsigned long long v[16], m16[16];
@@ -748,7 +724,6 @@ __device__ void cut1_slice(const StepParams& P, SmemStage& sm, SelScalars& sc, i
   for (int k = 0; k < 16; ++k) tsum += v[k];
   const unsigned long long total = block_sum(tsum, sc.shl);
   hist_desc(sm.h, v, m16);
-  SliceState* st = P.ws.st + un.s;
   unsigned long long target = total;
   bool keep_all = P.keep_all || total == 0ull;
   if (!keep_all) {
@@ -761,10 +736,15 @@ __device__ void cut1_slice(const StepParams& P, SmemStage& sm, SelScalars& sc, i
   __syncthreads();
   if (!keep_all) find_cut_desc_4096(m16, 0ull, target, sc.shl, &sc.cut_bin, &sc.cut_above);
   if (tid == 0) {
-    st->q_total = total;
-    st->target = target;
-    st->b1 = keep_all ? -1 : sc.cut_bin;
-    st->m_above = keep_all ? 0ull : sc.cut_above;
+    sc.b1 = keep_all ? -1 : sc.cut_bin;
+    sc.target = target;
+    sc.m_above = keep_all ? 0ull : sc.cut_above;
+    if (lead) {
+      SliceState* st = P.ws.st + un.s;
+      st->target = sc.target;
+      st->b1 = sc.b1;
+      st->m_above = sc.m_above;
+    }
   }
   __syncthreads();
 }
@@ -772,20 +752,21 @@ __device__ void cut1_slice(const StepParams& P, SmemStage& sm, SelScalars& sc, i
 // ------------------------------------------------------------------ mass phase
 // One range of slice y: M_h, Z_h merged from the slice's range statistics (fixed
 // order), the logits recomputed (index read #2, mostly from L2),
-// pi_j = sum_h 2^(l_hj - M_h) / (G Z_h) stored, and its mass added to the slice's
+// pi_j = sum_h 2^(l_hj - M_h) / (G Z_h) kept (PiSeg), and its mass added to the slice's
 // round-1 histogram via a per-range shared histogram of counts and low significand
 // bits (32-bit atomics; a range holds at most kMaxRangeGroups groups, so a bin's
 // low-bit sum stays below 2^32).
 // Block mode (BLK): warp w's batch is the four consecutive groups of one kBlock-token
 // block; the block's mass (the float32 sum of its tokens' pi, in a fixed order) is
-// stored at pi[block] and histogrammed instead of the tokens'.
+// kept for the block and histogrammed instead of the tokens'.
 constexpr int kMaxRangeGroups = 1024;   // 16384 tokens: 16384 * 2^18 = 2^32
 static_assert(kGroupBatch * 16 == kBlock, "block mode: one warp batch is one block");
 template <int G, bool BLK>
-__device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, const Ranges<BLK>& R, int y, int l0,
-                             int l1) {
+__device__ bool mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, const Ranges<BLK>& R,
+                             int y, int l0, int l1, bool wait_scores, unsigned n_ranges) {
   constexpr int NH = IdxTiles<G>::NH, U = kGroupBatch;
   const Unit un = unit_of(P, y);
+  const PiSeg ps = pi_seg<BLK>(R, y, un.s);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, gid = lane >> 2, t4 = lane & 3;
   const uint2* rows = reinterpret_cast<const uint2*>(idx_rows(P, y, un.s));
   const uint64_t pol = l2_policy_drop();
@@ -797,6 +778,8 @@ __device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
 #pragma unroll
     for (int u = 0; u < U; ++u) load_group(rows, 16 * grp(l0, u), jpf, pol, ra[u], rb[u]);
   }
+  // every range of the slice has stored its statistics (the first batch is in flight)
+  if (wait_scores && !slice_wait(&P.ws.st[un.s].arr_score, n_ranges, P.ws.dev_err, &sc.ok)) return false;
   // the sequence length, the query index vectors and the slice statistics are
   // requested together; one CTA barrier publishes them
   __syncthreads();   // earlier readers of sc.L, sc.qsm and the histogram are done
@@ -834,7 +817,7 @@ __device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
   }
   __syncthreads();
   const int L = sc.L;
-  if (16 * l0 >= L) return;
+  if (16 * l0 >= L) return true;
   uint32_t qb[IdxTiles<G>::NT][2];
   qidx_frag<G>(sc.qsm, qb);
   const float scale = P.idx_scale_log2;
@@ -846,7 +829,6 @@ __device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
     W[h] = head < G ? sm.Wh[head] : 0.f;   // lanes of absent heads contribute nothing
   }
   const int jend = min(L, 16 * l1);
-  float* pi = P.ws.pi + (size_t)un.s * P.ws.pi_stride;
   for (int gb = l0; 16 * gb < jend; gb += kWarps * U) {
     if (gb > l0) {
 #pragma unroll
@@ -875,11 +857,11 @@ __device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
       }
       if (BLK) {
         bsum += (j + gid < jend ? pr[0] : 0.f) + (j + gid + 8 < jend ? pr[1] : 0.f);
-      } else if (t4 < 2) {   // lane t4 = 0 stores token gid, t4 = 1 token gid + 8
+      } else if (t4 < 2) {   // lane t4 = 0 keeps token gid, t4 = 1 token gid + 8
         const int jt = j + gid + 8 * t4;
         const float v = t4 == 0 ? pr[0] : pr[1];
         if (jt < jend) {
-          pi[jt] = v;
+          pi_store(P, ps, jt, v);
           const unsigned bits = __float_as_uint(v);
           const unsigned d = min(bits >> 18, (unsigned)(kBins1 - 1));
           atomicAdd(&sm.cnt[d], 1u);
@@ -893,7 +875,7 @@ __device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
       for (int o = 4; o < 32; o <<= 1) bsum += __shfl_xor_sync(kFull, bsum, o);
       const int jb = 16 * grp(gb, 0);
       if (lane == 0 && jb < jend) {
-        pi[jb / kBlock] = bsum;
+        pi_store(P, ps, jb / kBlock, bsum);
         const unsigned bits = __float_as_uint(bsum);
         const unsigned d = min(bits >> 18, (unsigned)(kBins1 - 1));
         atomicAdd(&sm.cnt[d], 1u);
@@ -907,48 +889,60 @@ __device__ void mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
     if (sm.cnt[i])
       atomicAdd(g1 + i, P.topk > 0 ? (unsigned long long)sm.cnt[i] : bin1_mass((unsigned)i, sm.cnt[i], sm.low[i]));
   __syncthreads();   // the histogram is reused by the next range
+  return true;
 }
 
-template <int G, bool BLK>
-__device__ void mass_phase(const StepParams& P, SelSmem& sm_all, SelScalars& sc) {
-  SmemMass& sm = sm_all.mass;
-  const Ranges<BLK> R(P);
-  for_each_segment(R, [&](int y, int l0, int l1) {
-    for (int a = l0; a < l1; a += kMaxRangeGroups) mass_segment<G, BLK>(P, sm, sc, R, y, a, min(l1, a + kMaxRangeGroups));
-    const int n = R.last_cta(y) - R.first_cta(y) + 1;
-    if (last_of_slice(&P.ws.st[unit_of(P, y).s].ticket_mass, (unsigned)n, &sc.ok)) cut1_slice(P, sm_all.stage, sc, y);
-  });
+// ------------------------------------------------------------------ L2 prefetch
+// Bulk prefetch into L2 (no data returned to the SM): the rows are read again, from
+// L2, by the attention kernel that follows this one.
+__device__ __forceinline__ void prefetch_l2(const void* p, unsigned bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes) : "memory");
 }
 
-// ------------------------------------------------------------------ threshold phase
-// Calls f(bits, pos) for every candidate (in no particular order), kCandBatch
-// independent loads per thread at a time.
-template <class F>
-__device__ __forceinline__ void for_each_candidate(const uint2* cand, unsigned n, F&& f) {
-  for (unsigned i0 = 0; i0 < n; i0 += kSelThreads * kCandBatch) {
-    uint2 cv[kCandBatch];
-#pragma unroll
-    for (int u = 0; u < kCandBatch; ++u) {
-      const unsigned i = i0 + threadIdx.x + kSelThreads * u;
-      cv[u] = i < n ? __ldcg(cand + i) : make_uint2(0u, 0xffffffffu);
+// The sink and window K/V rows of every slice (streaming slices of the compact layout:
+// their ring), which the attention reads whatever the selection keeps, prefetched in
+// pieces of up to 64 KB.  Thread t of CTA c takes piece c + t nb, so the pieces spread
+// over every CTA.  Decode calls only (select-only calls pass no caches).
+template <typename T>
+__device__ void prefetch_attended_rows(const StepParams& P) {
+  if (!P.k_cache) return;
+  constexpr long long kRow = kHeadDim * sizeof(T);
+  constexpr long long kPiece = 65536;
+  const long long span = (long long)(P.compact ? max(P.window, P.ring) : P.window) * kRow;
+  const int per_slice = 2 * (1 + (int)((span + kPiece - 1) / kPiece));   // K and V: sinks + window pieces
+  const long long total = (long long)P.n_slices * per_slice;
+  for (long long p = blockIdx.x + (long long)threadIdx.x * gridDim.x; p < total;
+       p += (long long)gridDim.x * blockDim.x) {
+    const int s = (int)(p / per_slice), r = (int)(p % per_slice), piece = r >> 1;
+    int64_t L = P.seq_lens[s / P.Hkv];
+    L = L < 1 ? 1 : (L > P.Lcap ? P.Lcap : L);
+    const KvSlice<T> sl = kv_slice<T>(P, s);
+    const char* base = reinterpret_cast<const char*>((r & 1) ? sl.v : sl.k);
+    long long lo, hi;   // byte range in the slice's rows
+    if (sl.ring) {      // ring rows [0, min(L, ring))
+      if (piece == 0) continue;
+      lo = (long long)(piece - 1) * kPiece;
+      hi = min((long long)min((int64_t)P.ring, L) * kRow, lo + kPiece);
+    } else {
+      const SinkWindow sw((int)L, P.n_sink, P.window);
+      if (piece == 0) {
+        lo = 0;
+        hi = (long long)sw.n_s * kRow;
+      } else {
+        lo = (long long)sw.w_lo * kRow + (long long)(piece - 1) * kPiece;
+        hi = min(L * kRow, lo + kPiece);
+      }
     }
-#pragma unroll
-    for (int u = 0; u < kCandBatch; ++u)
-      if (cv[u].y != 0xffffffffu) f(cv[u].x, (int)cv[u].y);
+    if (hi > lo) prefetch_l2(base + lo, (unsigned)(hi - lo));
   }
 }
 
+// ------------------------------------------------------------------ threshold phase
 // Number of positions of [lo, hi) outside sinks and window.
 __device__ __forceinline__ int listed_in(const SinkWindow& sw, int lo, int hi) {
   if (hi <= lo) return 0;
   const int a = max(lo, sw.n_s), b = min(hi, sw.w_lo);
   return b > a ? b - a : 0;
-}
-
-// Chunk of element e (a token, or a block in block mode).
-template <bool BLK>
-__device__ __forceinline__ int chunk_of(int e) {
-  return BLK ? e / (kChunk / kBlock) : e / kChunk;
 }
 
 // Listed positions (outside sinks and window) of element e: token e, or block e in
@@ -959,355 +953,485 @@ __device__ __forceinline__ int listed_of(const SinkWindow& sw, int L, int e) {
   return listed_in(sw, e * kBlock, min(L, (e + 1) * kBlock));
 }
 
-// Unit: one chunk.  Tokens above bin b1 counted (listed ones), tokens of bin b1
-// appended as candidates with their round-2 masses added to the slice histogram.
-// Block mode: the chunk's kChunk / kBlock blocks, one per thread of the first warps;
-// a block above b1 counts its listed tokens, a block of bin b1 is a candidate.
+// Elements (tokens, or blocks in block mode) of the segment of local groups [l0, l1) of
+// a slice of length L: [e0, e1).
 template <bool BLK>
-__device__ void threshold_unit(const StepParams& P, SelScalars& sc, int y, int c) {
-  const Unit un = unit_of(P, y);
-  const int tid = threadIdx.x, lane = tid & 31;
-  const int j0 = c * kChunk;
-  SliceState* st = P.ws.st + un.s;
-  const unsigned* pib = reinterpret_cast<const unsigned*>(P.ws.pi + (size_t)un.s * P.ws.pi_stride);
-  // the chunk's probabilities are requested with L and b1 (one round trip); rows hold
-  // the call's capacity, and entries past L are masked below
-  constexpr int kPer = kChunk / kBlock;
-  static_assert(kPer % 32 == 0 && kPer <= kSelThreads, "block mode: whole warps of blocks per chunk");
-  unsigned bits[kTokPerThread];
-  if (BLK) {
-    const int e = c * kPer + tid;
-    bits[0] = tid < kPer && e * kBlock < P.Lcap ? __ldcg(pib + e) : 0u;
-  } else {
-#pragma unroll
-    for (int i = 0; i < kTokPerThread; ++i) {
-      const int j = j0 + tid + kSelThreads * i;
-      bits[i] = j < P.Lcap ? __ldcg(pib + j) : 0u;
-    }
-  }
-  __syncthreads();   // earlier readers of sc.L / sc.b1 are done
-  if (tid == 0) {
-    sc.L = load_len(P.seq_lens, un.b, P.Lcap, P.ws.dev_err);
-    sc.b1 = __ldcg(&st->b1);
-  }
-  __syncthreads();
-  const int L = sc.L, b1 = sc.b1;
-  const SinkWindow sw(L, P.n_sink, P.window);
-  uint2* cand = P.ws.cand + (size_t)un.s * P.Lmax;
-  unsigned long long* h2 = P.ws.hist2 + (size_t)un.s * kBins2;
-  int cnt = 0;
-  if (BLK && j0 < L) {
-    const int e = c * kPer + tid;
-    bool is_cand = false;
-    if (tid < kPer && e * kBlock < L) {
-      const unsigned b = bits[0];
-      const int d1 = (int)min(b >> 18, (unsigned)(kBins1 - 1));
-      if (d1 > b1) cnt = listed_of<BLK>(sw, L, e);
-      else is_cand = d1 == b1;
-    }
-    if (tid < kPer) {   // whole warps
-      const unsigned mask = __ballot_sync(kFull, is_cand);
-      if (mask) {
-        unsigned base = 0u;
-        if (lane == 0) base = atomicAdd(&st->cand_count, (unsigned)__popc(mask));
-        base = __shfl_sync(kFull, base, 0);
-        if (is_cand) {
-          cand[base + __popc(mask & ((1u << lane) - 1u))] = make_uint2(bits[0], (unsigned)e);
-          atomicAdd(&h2[(bits[0] >> 6) & 0xfffu], sel_mass(P, bits[0]));
-        }
-      }
-    }
-  } else if (j0 < L) {
-    const int jend = min(L, j0 + kChunk);
-    unsigned cflags = 0u;
-#pragma unroll
-    for (int i = 0; i < kTokPerThread; ++i) {
-      const int j = j0 + tid + kSelThreads * i;
-      if (j < jend) {
-        const int d1 = (int)min(bits[i] >> 18, (unsigned)(kBins1 - 1));
-        if (d1 > b1) cnt += sw.always(j) ? 0 : 1;
-        else if (d1 == b1) cflags |= 1u << i;
-      }
-    }
-    // one atomic per warp reserves the warp's candidate slots
-    unsigned masks[kTokPerThread];
-    unsigned warp_total = 0u;
-#pragma unroll
-    for (int i = 0; i < kTokPerThread; ++i) {
-      masks[i] = __ballot_sync(kFull, (cflags >> i) & 1u);
-      warp_total += __popc(masks[i]);
-    }
-    if (warp_total) {
-      unsigned base = 0u;
-      if (lane == 0) base = atomicAdd(&st->cand_count, warp_total);
-      base = __shfl_sync(kFull, base, 0);
-      const unsigned lt = (1u << lane) - 1u;
-#pragma unroll
-      for (int i = 0; i < kTokPerThread; ++i) {
-        if ((cflags >> i) & 1u) {
-          cand[base + __popc(masks[i] & lt)] = make_uint2(bits[i], (unsigned)(j0 + tid + kSelThreads * i));
-          atomicAdd(&h2[(bits[i] >> 6) & 0xfffu], sel_mass(P, bits[i]));
-        }
-        base += __popc(masks[i]);
-      }
-    }
-  }
-  const int chunk_total = block_sum(cnt, sc.shi);
-  if (tid == 0) P.ws.chunk_gt[(size_t)un.s * P.n_chunks + c] = chunk_total;
+__device__ __forceinline__ void seg_elems(int L, int l0, int l1, int& e0, int& e1) {
+  const int j0 = 16 * l0, j1 = min(L, 16 * l1);
+  e0 = BLK ? j0 / kBlock : j0;
+  e1 = j1 <= j0 ? e0 : (BLK ? (j1 + kBlock - 1) / kBlock : j1);
 }
 
-// ------------------------------------------------------------------ refine (per slice)
+// One range of slice y (after cut1_range of y): the elements of bin b1 are the slice's
+// candidates.  Two passes over the range's probabilities (on chip): the first counts
+// them per warp, one atomic per CTA reserves their slots in the slice's candidate array,
+// the second writes them (bits, element) in range order and adds them to the slice's
+// round-A histogram (bits 17..9: count and sum of bits 8..0).  Token mode: lane l of warp
+// w reads elements 4 l .. 4 l + 3 of the warp's 128 as one 16-byte load.
 template <bool BLK>
-__device__ void refine_slice(const StepParams& P, SelSmem& smu, SelScalars& sc, int y) {
-  SmemRefine& sm = smu.ref;
+__device__ void threshold_segment(const StepParams& P, SelScalars& sc, SmemRefine& sm, const Ranges<BLK>& R, int y,
+                                  int l0, int l1) {
+  const Unit un = unit_of(P, y);
+  const PiSeg ps = pi_seg<BLK>(R, y, un.s);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __syncthreads();   // earlier readers of the scalars are done
+  if (tid == 0) sc.L = load_len(P.seq_lens, un.b, P.Lcap, P.ws.dev_err);
+  __syncthreads();
+  const int L = sc.L, b1 = sc.b1;   // b1 from cut1_range
+  if (b1 < 0) return;               // keep everything: no candidates
+  int e0, e1;
+  seg_elems<BLK>(L, l0, l1, e0, e1);
+  constexpr int kPer = BLK ? 1 : 4;
+  // candidate mask of the thread's elements of round k0 (their bits in bits[])
+  auto cand_mask = [&](int k0, unsigned (&bits)[kPer]) {
+    const int eb = k0 + (BLK ? tid : 128 * warp + 4 * lane);
+    unsigned m = 0u;
+    if (BLK) {
+      bits[0] = eb < e1 ? __float_as_uint(pi_load(P, ps, eb)) : 0u;
+    } else if (eb < e1) {
+      const float4 v = pi_load4(P, ps, eb);
+      bits[0] = __float_as_uint(v.x);
+      bits[1] = __float_as_uint(v.y);
+      bits[2] = __float_as_uint(v.z);
+      bits[3] = __float_as_uint(v.w);
+    }
+#pragma unroll
+    for (int q = 0; q < kPer; ++q)
+      if (eb + q < e1 && (int)min(bits[q] >> 18, (unsigned)(kBins1 - 1)) == b1) m |= 1u << q;
+    return m;
+  };
+  int wc = 0;   // this warp's candidates (every lane holds the warp's sum)
+  for (int k0 = e0; k0 < e1; k0 += kSelThreads * kPer) {
+    unsigned bits[kPer];
+    int c = __popc(cand_mask(k0, bits));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(kFull, c, o);
+    wc += c;
+  }
+  if (lane == 0) sm.wcnt[warp] = wc;
+  __syncthreads();
+  unsigned total = 0u;
+  int wbase = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    total += (unsigned)sm.wcnt[w];
+    wbase += w < warp ? sm.wcnt[w] : 0;
+  }
+  if (total == 0u) return;
+  if (tid == 0) sc.cbase = atomicAdd(&P.ws.st[un.s].ncand, total);
+  __syncthreads();
+  uint2* cand = P.ws.cand + (size_t)un.s * P.Lmax;
+  unsigned* ha = hist_a(P, un.s);
+  unsigned slot = sc.cbase + (unsigned)wbase;
+  for (int k0 = e0; k0 < e1; k0 += kSelThreads * kPer) {
+    unsigned bits[kPer];
+    const unsigned m = cand_mask(k0, bits);
+    const int eb = k0 + (BLK ? tid : 128 * warp + 4 * lane);
+    // lanes in order, each lane's elements in order
+    const int c = __popc(m);
+    int x = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(kFull, x, o);
+      if (lane >= o) x += t;
+    }
+    unsigned k = slot + (unsigned)(x - c);
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      if (m >> q & 1u) {
+        cand[k++] = make_uint2(bits[q], (unsigned)(eb + q));
+        const unsigned d = (bits[q] >> 9) & 511u;
+        atomicAdd(ha + d, 1u);
+        atomicAdd(ha + 512 + d, bits[q] & 511u);
+      }
+    }
+    slot += (unsigned)__shfl_sync(kFull, x, 31);
+  }
+}
+
+// ------------------------------------------------------------------ refine (per range)
+// Mass of the round-A/B digit d of the cut bin b1: count c, sum l of the bits below the
+// digit, significand bits above them sig (implicit bit included).  Every candidate
+// shares b1's exponent field, so the digit's mass is the exact sum of its candidates'
+// mass_q: (sig * c + l) << (e - 87) (0 for e < 87), or c for top-k.
+__device__ __forceinline__ unsigned long long digit_mass(const StepParams& P, int b1, unsigned sig, unsigned c,
+                                                         unsigned l) {
+  if (P.topk > 0) return c;
+  int e = b1 >> 5;
+  if (e < kMassMinExp || c == 0u) return 0ull;
+  e = e > 127 ? 127 : e;
+  return ((unsigned long long)sig * c + l) << (e - kMassMinExp);
+}
+
+// Warp 0: the digit d of [0, 512) (visited from 511 down) where base plus the
+// cumulative mass of the digits above it first reaches target; sc.digit (-1 if never)
+// and sc.above (the mass ahead of d).  sig_of(d) gives the digit's significand bits.
+template <class SIG>
+__device__ void digit_cut_desc(const StepParams& P, const SmemRefine& sm, SelScalars& sc, int b1, SIG sig_of,
+                               unsigned long long base, unsigned long long target) {
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x >= 32) return;
+  unsigned long long sum = 0ull;
+  for (int k = 0; k < 16; ++k) {
+    const int d = 511 - 16 * lane - k;
+    sum += digit_mass(P, b1, sig_of(d), sm.hc[d], sm.hl[d]);
+  }
+  unsigned long long x = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long t = __shfl_up_sync(kFull, x, o);
+    if (lane >= o) x += t;
+  }
+  unsigned long long cum = base + x - sum;
+  if (cum < target && cum + sum >= target) {   // the crossing is in this lane's digits
+    for (int k = 0; k < 16; ++k) {
+      const int d = 511 - 16 * lane - k;
+      const unsigned long long m = digit_mass(P, b1, sig_of(d), sm.hc[d], sm.hl[d]);
+      if (cum < target && cum + m >= target) {
+        sc.digit = d;
+        sc.above = cum;
+      }
+      cum += m;
+    }
+  }
+}
+
+// Warp 0: the digit of [0, 256) (visited from 0 up) where base plus the count of the
+// digits below it first reaches need; sc.digit (-1 if never) and sc.above (the count
+// before it).
+__device__ void digit_kth_asc(const SmemRefine& sm, SelScalars& sc, unsigned long long base,
+                              unsigned long long need) {
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x >= 32) return;
+  unsigned sum = 0u;
+  for (int k = 0; k < 8; ++k) sum += sm.hc[8 * lane + k];
+  unsigned x = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned t = __shfl_up_sync(kFull, x, o);
+    if (lane >= o) x += t;
+  }
+  unsigned long long cum = base + x - sum;
+  if (cum < need && cum + sum >= need) {
+    for (int k = 0; k < 8; ++k) {
+      const unsigned c = sm.hc[8 * lane + k];
+      if (cum < need && cum + c >= need) {
+        sc.digit = 8 * lane + k;
+        sc.above = cum;
+      }
+      cum += c;
+    }
+  }
+}
+
+// The slice's exact cut, taken by every CTA of the slice for itself once every range has
+// stored its candidates.  All tokens above the round-1 bin b1 are kept; among the
+// candidates of b1, in (pi desc, position asc) order, a candidate is kept while the mass
+// ranked ahead of it (m_above plus the candidates before it) is below the target.
+// Round A: the round-A histogram (bits 17..9, exact masses from counts and sums of the
+// lower bits) gives the digit dA holding the cut.  One pass over the slice's candidate
+// array gathers the candidates of dA on chip; round B over those (bits 8..0) gives the
+// cut value tau and the mass above it; if only some of the candidates equal to tau are
+// needed, the lowest positions are kept: ranked directly when they are few, else by
+// three 8-bit rounds over their positions.  Results in sc.tau, sc.pos_cut and sc.L;
+// the slice's first CTA (lead) also stores tau and pos_cut.
+template <bool BLK>
+__device__ void refine_range(const StepParams& P, SmemRefine& sm, SelScalars& sc, int y, bool lead) {
   const Unit un = unit_of(P, y);
   const int tid = threadIdx.x;
-  SliceState* st = P.ws.st + un.s;
-  // every input of this step is requested at once: the round-2 histogram (bits 17..6,
-  // filled by the chunks), the slice state and the sequence length
-  unsigned long long v2[16];
-  hist_issue(P.ws.hist2 + (size_t)un.s * kBins2, v2);
-  const unsigned n = __ldcg(&st->cand_count);
+  const SliceState* st = P.ws.st + un.s;
   const unsigned long long target = __ldcg(&st->target);
   const unsigned long long mab = __ldcg(&st->m_above);
   const int b1 = __ldcg(&st->b1);
-  int64_t len = P.seq_lens[un.b];
-  __syncthreads();   // earlier readers of the scalars are done
+  const unsigned n = b1 >= 0 ? __ldcg(&st->ncand) : 0u;
+  const int L = load_len(P.seq_lens, un.b, P.Lcap, P.ws.dev_err);
+  const uint2* cand = P.ws.cand + (size_t)un.s * P.Lmax;
+  const unsigned* ha = hist_a(P, un.s);
+  unsigned hav[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) hav[k] = b1 >= 0 ? __ldcg(ha + tid + kSelThreads * k) : 0u;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {   // words 0..511 counts, 512..1023 low sums
+    const int w = tid + kSelThreads * k;
+    if (w < 512) sm.hc[w] = hav[k]; else sm.hl[w - 512] = hav[k];
+  }
   if (tid == 0) {
-    if (len < 1 || len > P.Lcap) atomicOr(P.ws.dev_err, kErrSeqLen);
-    sc.b2 = -1;
-    sc.b3 = -1;
-    sc.small_n = 0u;
-    sc.kbin = -1;
+    sc.digit = -1;
+    sc.pos_cut = INT_MAX;
+    sc.ntie = 0;
+    sc.nsmall = 0u;
   }
   __syncthreads();
-  const int L = len < 1 ? 1 : (len > P.Lcap ? P.Lcap : (int)len);
-  const SinkWindow sw(L, P.n_sink, P.window);
-  const uint2* cand = P.ws.cand + (size_t)un.s * P.Lmax;
-  if (b1 >= 0) {   // round 2 cut (the staging buffer aliases chunk_sel / cnt4k)
-    unsigned long long m16[16];
-    hist_desc(smu.stage.h, v2, m16);
-    find_cut_desc_4096(m16, mab, target, sc.shl, &sc.b2, &sc.above2);
-  }
-  int* chunk_sel = sm.chunk_sel;
-  unsigned* cnt4k = sm.cnt4k;
-  uint2* small = sm.small;
-  // exact cut value, tie quota, per-chunk output offsets
+  // f(v) for every candidate, kRefBatch coalesced loads per thread issued together
+  auto for_each_cand = [&](auto&& f) {
+    for (unsigned i0 = 0; i0 < n; i0 += kSelThreads * kRefBatch) {
+      uint2 v[kRefBatch];
+#pragma unroll
+      for (int u = 0; u < kRefBatch; ++u) {
+        const unsigned i = i0 + tid + kSelThreads * u;
+        v[u] = i < n ? __ldcg(cand + i) : make_uint2(0u, 0xffffffffu);
+      }
+#pragma unroll
+      for (int u = 0; u < kRefBatch; ++u)
+        if (v[u].y != 0xffffffffu) f(v[u]);
+    }
+  };
   unsigned tau = 0u;
   int pos_cut = INT_MAX;
-  for (int c = tid; c < P.n_chunks; c += kSelThreads) chunk_sel[c] = 0;
-  if (tid < kBins3) { sm.m3[tid] = 0ull; sm.c3[tid] = 0u; }
-  __syncthreads();
   bool found = b1 < 0;   // keep-everything mode needs no cut
   if (b1 >= 0) {
-    const int cb2 = sc.b2;
-    // one pass over the candidates: above the round-2 bin they are kept; inside it
-    // they feed round 3 (bits 5..0) and are parked in shared memory
-    for_each_candidate(cand, n, [&](unsigned bits, int pos) {
-      const int d2 = (int)((bits >> 6) & 0xfffu);
-      if (d2 > cb2) {
-        const int nl = listed_of<BLK>(sw, L, pos);
-        if (nl) atomicAdd(&chunk_sel[chunk_of<BLK>(pos)], nl);
-      } else if (d2 == cb2) {
-        atomicAdd(&sm.m3[bits & 63u], sel_mass(P, bits));
-        atomicAdd(&sm.c3[bits & 63u], 1u);
-        const unsigned slot = atomicAdd(&sc.small_n, 1u);
-        if (slot < kSmallCap) small[slot] = make_uint2(bits, (unsigned)pos);
-      }
-    });
+    const unsigned sig1 = (((unsigned)b1 & 31u) << 18) | 0x800000u;   // significand bits above bit 18
+    digit_cut_desc(P, sm, sc, b1, [&](int d) { return sig1 | ((unsigned)d << 9); }, mab, target);
     __syncthreads();
-    if (tid < 32 && cb2 >= 0) {
-      // round 3 (bits 5..0), descending: lane i holds bins 63 - 2i and 62 - 2i
-      const unsigned long long ma = sm.m3[63 - 2 * tid], mb = sm.m3[62 - 2 * tid];
-      unsigned long long x = ma + mb;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const unsigned long long t = __shfl_up_sync(kFull, x, o);
-        if (tid >= o) x += t;
-      }
-      const unsigned long long before = sc.above2 + x - (ma + mb);   // mass above bin 63 - 2i
-      int hit = -1;
-      unsigned long long above = 0ull;
-      if (before < target && before + ma >= target) { hit = 63 - 2 * tid; above = before; }
-      else if (before + ma < target && before + ma + mb >= target) { hit = 62 - 2 * tid; above = before + ma; }
-      const unsigned who = __ballot_sync(kFull, hit >= 0);
-      if (who != 0u && tid == __ffs(who) - 1) {
-        sc.b3 = hit;
-        sc.above2 = above;   // mass strictly above tau
-      }
-    }
-    __syncthreads();
-    // b2 and b3 always exist (the candidates carry the mass of bin b1); if a search ever
-    // failed, every token is kept rather than a missing bin indexed
-    found = cb2 >= 0 && sc.b3 >= 0;
-    const bool small_ok = sc.small_n <= (unsigned)kSmallCap;
-    const unsigned sn = small_ok ? sc.small_n : 0u;
+    const int dA = sc.digit;
+    const unsigned long long aboveA = sc.above;
+    found = dA >= 0;
     if (found) {
-      tau = ((unsigned)b1 << 18) | ((unsigned)cb2 << 6) | (unsigned)sc.b3;
-      const unsigned long long m_gt = sc.above2;
-      const unsigned n_eq = sm.c3[sc.b3];
-      const unsigned long long q_tau = sel_mass(P, tau);
-      const unsigned long long need =
-          (q_tau > 0ull && target > m_gt) ? (target - m_gt + q_tau - 1ull) / q_tau : ~0ull;
-      if (need < (unsigned long long)n_eq) {
-        // pos_cut = need-th smallest position among the candidates equal to tau
-        const unsigned qk = (unsigned)need;
-        for (int pass = 0; pass < 2; ++pass) {
-          for (int i = tid; i < 4096; i += kSelThreads) cnt4k[i] = 0u;
-          __syncthreads();
-          const int kb = sc.kbin;
-          auto add = [&](unsigned bits, int pos) {
-            if (bits != tau) return;
-            if (pass == 0) atomicAdd(&cnt4k[(unsigned)pos >> 12], 1u);
-            else if ((int)((unsigned)pos >> 12) == kb) atomicAdd(&cnt4k[(unsigned)pos & 4095u], 1u);
-          };
-          if (small_ok) {
-            for (unsigned i = tid; i < sn; i += kSelThreads) add(small[i].x, (int)small[i].y);
-          } else {
-            for_each_candidate(cand, n, add);
-          }
-          __syncthreads();
-          unsigned c16[16];
-#pragma unroll
-          for (int k = 0; k < 16; ++k) c16[k] = cnt4k[16 * tid + k];
-          if (tid == 0) sc.fbin = -1;
-          __syncthreads();
-          find_kth_asc_4096(c16, pass == 0 ? 0u : sc.kbefore, qk, sc.shu, &sc.fbin, &sc.fbefore);
-          if (tid == 0) {
-            if (sc.fbin < 0) sc.kbin = -1;
-            else if (pass == 0) { sc.kbin = sc.fbin; sc.kbefore = sc.fbefore; }
-            else if (sc.kbin >= 0) sc.kbin = (sc.kbin << 12) | sc.fbin;
-          }
-          __syncthreads();
-          if (sc.kbin < 0) break;
+      const unsigned preB = ((unsigned)b1 << 9) | (unsigned)dA;
+      // the candidates of digit dA, gathered on chip
+      for_each_cand([&](uint2 v) {
+        if ((v.x >> 9) == preB) {
+          const unsigned k = atomicAdd(&sc.nsmall, 1u);
+          if (k < (unsigned)kSmallList) sm.small[k] = v;
         }
-        pos_cut = sc.kbin >= 0 ? sc.kbin : INT_MAX;
-      }
-      // kept candidates of the round-2 cut bin
-      const int pc = pos_cut;
-      auto keep_bin = [&](unsigned bits, int pos) {
-        if ((int)((bits >> 6) & 0xfffu) != cb2) return;
-        if (bits > tau || (bits == tau && pos <= pc)) {
-          const int nl = listed_of<BLK>(sw, L, pos);
-          if (nl) atomicAdd(&chunk_sel[chunk_of<BLK>(pos)], nl);
+      });
+      for (int d = tid; d < 512; d += kSelThreads) sm.hc[d] = sm.hl[d] = 0u;
+      if (tid == 0) sc.digit = -1;
+      __syncthreads();
+      const unsigned ns = sc.nsmall;
+      const bool fits = ns <= (unsigned)kSmallList;
+      // f(v) for every candidate of digit dA: from the on-chip list, or (if it overflowed)
+      // from the candidate array
+      auto for_each_small = [&](auto&& f) {
+        if (fits) {
+          for (unsigned i = tid; i < ns; i += kSelThreads) f(sm.small[i]);
+        } else {
+          for_each_cand([&](uint2 v) { if ((v.x >> 9) == preB) f(v); });
         }
       };
-      if (small_ok) {
-        for (unsigned i = tid; i < sn; i += kSelThreads) keep_bin(small[i].x, (int)small[i].y);
-      } else {
-        for_each_candidate(cand, n, keep_bin);
+      // round B: bits 8..0 of the candidates of digit dA
+      for_each_small([&](uint2 v) { atomicAdd(&sm.hc[v.x & 511u], 1u); });
+      __syncthreads();
+      const unsigned sigA = sig1 | ((unsigned)dA << 9);
+      digit_cut_desc(P, sm, sc, b1, [&](int d) { return sigA | (unsigned)d; }, aboveA, target);
+      __syncthreads();
+      found = sc.digit >= 0;
+      if (found) {
+        const int dB = sc.digit;
+        tau = preB << 9 | (unsigned)dB;                 // fp32 bits of the cut value
+        const unsigned long long m_gt = sc.above;       // mass strictly above tau
+        const unsigned n_eq = sm.hc[dB];                 // candidates equal to tau
+        const unsigned long long q_tau = sel_mass(P, tau);
+        const unsigned long long need =
+            (q_tau > 0ull && target > m_gt) ? (target - m_gt + q_tau - 1ull) / q_tau : ~0ull;
+        __syncthreads();   // every read of sm.hc is done
+        if (need < (unsigned long long)n_eq) {
+          // keep the need lowest positions among the candidates equal to tau
+          if (n_eq <= (unsigned)kTieCap) {
+            for_each_small([&](uint2 v) {
+              if (v.x == tau) sm.tie[atomicAdd(&sc.ntie, 1)] = (int)v.y;
+            });
+            __syncthreads();
+            if (tid < (int)n_eq) {
+              const int pmine = sm.tie[tid];
+              unsigned r = 0u;
+              for (unsigned k = 0; k < n_eq; ++k) r += sm.tie[k] < pmine ? 1u : 0u;
+              if (r == (unsigned)need - 1u) sc.pos_cut = pmine;
+            }
+            __syncthreads();
+          } else {
+            unsigned pp = 0u;
+            unsigned long long before = 0ull;
+            bool ok = true;
+            for (int sh = 16; sh >= 0 && ok; sh -= 8) {   // positions < 2^24
+              for (int d = tid; d < 256; d += kSelThreads) sm.hc[d] = 0u;
+              if (tid == 0) sc.digit = -1;
+              __syncthreads();
+              for_each_small([&](uint2 v) {
+                if (v.x == tau && (v.y >> (sh + 8)) == pp) atomicAdd(&sm.hc[(v.y >> sh) & 255u], 1u);
+              });
+              __syncthreads();
+              digit_kth_asc(sm, sc, before, need);
+              __syncthreads();
+              ok = sc.digit >= 0;
+              if (ok) {
+                pp = (pp << 8) | (unsigned)sc.digit;
+                before = sc.above;
+              }
+            }
+            if (tid == 0) sc.pos_cut = ok ? (int)pp : INT_MAX;
+            __syncthreads();
+          }
+          pos_cut = sc.pos_cut;
+        }
       }
     }
-    __syncthreads();
   }
-  if (!found) {
-    // keep everything: every listed token of each chunk
+  if (!found) {   // a search that fails keeps every token rather than index a missing bin
     tau = 0u;
     pos_cut = INT_MAX;
-    for (int c = tid; c < P.n_chunks; c += kSelThreads)
-      chunk_sel[c] = listed_in(sw, c * kChunk, min(L, (c + 1) * kChunk)) -
-                     __ldcg(&P.ws.chunk_gt[(size_t)un.s * P.n_chunks + c]);
-    __syncthreads();
   }
-  // offsets: exclusive scan over chunks of (above-b1 count + kept candidates); with one
-  // chunk per thread (up to kSelThreads chunks) the count is loaded once
-  const int per = (P.n_chunks + kSelThreads - 1) / kSelThreads;
-  const int c0 = tid * per;
-  const int* gt_row = P.ws.chunk_gt + (size_t)un.s * P.n_chunks;
+  __syncthreads();   // earlier readers of the scalars are done
+  if (tid == 0) {
+    sc.tau = tau;
+    sc.pos_cut = pos_cut;
+    sc.L = L;
+    if (lead) {   // for the compaction of every range of the slice
+      SliceState* stw = P.ws.st + un.s;
+      stw->tau_bits = tau;
+      stw->pos_cut = pos_cut;
+    }
+  }
+  __syncthreads();
+}
+
+// ------------------------------------------------------------------ kept count and offset
+// Whether element e (token e, or block e) is kept by the cut (tau, pos_cut).
+__device__ __forceinline__ bool kept_by_cut(unsigned bits, int e, unsigned tau, int pos_cut) {
+  return bits > tau || (bits == tau && e <= pos_cut);
+}
+
+// One range of slice y (after refine_range of y): its kept listed tokens, counted from
+// its on-chip probabilities and stored at its slot; then it arrives at the slice's count
+// counter.
+template <bool BLK>
+__device__ void count_segment(const StepParams& P, SelScalars& sc, const Ranges<BLK>& R, int y, int l0, int l1) {
+  const Unit un = unit_of(P, y);
+  const PiSeg ps = pi_seg<BLK>(R, y, un.s);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int L = sc.L;
+  const unsigned tau = sc.tau;
+  const int pos_cut = sc.pos_cut;
+  const SinkWindow sw(L, P.n_sink, P.window);
+  int e0, e1;
+  seg_elems<BLK>(L, l0, l1, e0, e1);
+  constexpr int kPer = BLK ? 1 : 4;
+  int cnt = 0;
+  for (int k0 = e0; k0 < e1; k0 += kSelThreads * kPer) {
+    const int eb = k0 + (BLK ? tid : 128 * warp + 4 * lane);
+    if (eb >= e1) continue;
+    if (BLK) {
+      if (kept_by_cut(__float_as_uint(pi_load(P, ps, eb)), eb, tau, pos_cut)) cnt += listed_of<BLK>(sw, L, eb);
+    } else {
+      const float4 v = pi_load4(P, ps, eb);
+      const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int j = eb + q;
+        if (j < e1 && !sw.always(j) && kept_by_cut(__float_as_uint(vv[q]), j, tau, pos_cut)) ++cnt;
+      }
+    }
+  }
+  const int total = block_sum(cnt, sc.shi);
+  if (tid == 0) P.ws.seg_cnt[stats_slot(blockIdx.x, y)] = total;
+}
+
+// This range's offset in slice y's list: the kept counts of the slice's ranges before it
+// (after every range has stored its count).  The slice's first CTA stores the total.
+template <bool BLK>
+__device__ void offset_segment(const StepParams& P, SelScalars& sc, const Ranges<BLK>& R, int y) {
+  const Unit un = unit_of(P, y);
+  const int tid = threadIdx.x;
+  const int first = R.first_cta(y), n_seg = R.last_cta(y) - first + 1, mine = (int)blockIdx.x - first;
+  const int* cnt_row = P.ws.seg_cnt + stats_slot(first, y);
+  constexpr int kSegPer = kMaxSelectGrid / kSelThreads;
+  int cv[kSegPer];
   int loc = 0;
-  for (int k = 0; k < per; ++k) {
-    const int c = c0 + k;
-    if (c < P.n_chunks) loc += __ldcg(gt_row + c) + chunk_sel[c];
+#pragma unroll
+  for (int k = 0; k < kSegPer; ++k) {
+    const int c = tid * kSegPer + k;
+    cv[k] = c < n_seg ? __ldcg(cnt_row + c) : 0;
+    loc += cv[k];
   }
   int total = 0;
   int run = block_excl_scan(loc, sc.shi, &total);
-  if (per == 1) {
-    if (c0 < P.n_chunks) P.ws.chunk_off[(size_t)un.s * P.n_chunks + c0] = run;
-  } else {
-    for (int k = 0; k < per; ++k) {
-      const int c = c0 + k;
-      if (c < P.n_chunks) {
-        P.ws.chunk_off[(size_t)un.s * P.n_chunks + c] = run;
-        run += __ldcg(gt_row + c) + chunk_sel[c];
-      }
-    }
+#pragma unroll
+  for (int k = 0; k < kSegPer; ++k) {
+    const int c = tid * kSegPer + k;
+    if (c == mine) sc.off = run;
+    run += cv[k];
   }
-  if (tid == 0) {
-    st->tau_bits = tau;
-    st->pos_cut = pos_cut;
-    st->count = total;
+  if (tid == 0 && mine == 0) {
+    P.ws.st[un.s].count = total;
     if (P.sel_count) P.sel_count[un.s] = total;
   }
-  __syncthreads();   // shared memory reused by the next unit
+  __syncthreads();
 }
 
 // ------------------------------------------------------------------ compact phase
+// One range of slice y (after offset_segment of y): its kept positions outside
+// sinks/window, ascending, written at the range's offset in the slice's list.  Rounds of 1024 tokens: lane l of warp w
+// takes tokens 4 l .. 4 l + 3 of the warp's 128 (one 16-byte read of their
+// probabilities in token mode), a warp scan orders the lanes and the eight warp totals
+// order the warps.
 template <bool BLK>
-__device__ void compact_unit(const StepParams& P, SelScalars& sc, int y, int c) {
-  static_assert(kBlock % kTokPerThread == 0, "a thread's tokens must lie in one block");
+__device__ void compact_segment(const StepParams& P, SelScalars& sc, const Ranges<BLK>& R, int y, int l0, int l1) {
   const Unit un = unit_of(P, y);
-  const int j0 = c * kChunk;
-  const unsigned* pib = reinterpret_cast<const unsigned*>(P.ws.pi + (size_t)un.s * P.ws.pi_stride);
-  const int jb = j0 + threadIdx.x * kTokPerThread;  // this thread's 16 consecutive tokens
-  // the probabilities are requested with L and the slice's cut (one round trip); rows
-  // hold the call's capacity padded to 64 floats, so four 16-byte loads stay in the row
-  unsigned bits[kTokPerThread] = {};
-  if (BLK) {
-    bits[0] = jb < P.Lcap ? __ldcg(pib + jb / kBlock) : 0u;   // the 16 tokens lie in one block
-  } else if (jb < P.Lcap) {
-    const uint4* v4 = reinterpret_cast<const uint4*>(pib + jb);
-#pragma unroll
-    for (int q = 0; q < kTokPerThread / 4; ++q) {
-      const uint4 v = __ldcg(v4 + q);
-      bits[4 * q] = v.x;
-      bits[4 * q + 1] = v.y;
-      bits[4 * q + 2] = v.z;
-      bits[4 * q + 3] = v.w;
-    }
-  }
+  const PiSeg ps = pi_seg<BLK>(R, y, un.s);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   __syncthreads();   // earlier readers of the scalars are done
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     const SliceState* st = P.ws.st + un.s;
     sc.L = load_len(P.seq_lens, un.b, P.Lcap, P.ws.dev_err);
     sc.tau = __ldcg(&st->tau_bits);
     sc.pos_cut = __ldcg(&st->pos_cut);
-    sc.off = __ldcg(&P.ws.chunk_off[(size_t)un.s * P.n_chunks + c]);
   }
   __syncthreads();
-  const int L = sc.L;
-  if (j0 >= L) return;
+  const int L = sc.L;   // sc.off from offset_segment of this slice
   const unsigned tau = sc.tau;
   const int pos_cut = sc.pos_cut;
   const SinkWindow sw(L, P.n_sink, P.window);
-  unsigned keep = 0u;
-  if (BLK && jb < L) {
-    const int e = jb / kBlock;
-    if (bits[0] > tau || (bits[0] == tau && e <= pos_cut)) {
+  const int j0 = 16 * l0, j1 = min(L, 16 * l1);
+  int* dst = P.sel_list + (size_t)un.s * P.Lmax;
+  int64_t run = sc.off;
+  for (int k0 = j0; k0 < j1; k0 += 4 * kSelThreads) {   // whole CTA: the barriers below
+    const int jb = k0 + 128 * warp + 4 * lane;
+    unsigned keep = 0u;
+    if (jb < j1) {
+      float v[4];
+      if (BLK) {
 #pragma unroll
-      for (int i = 0; i < kTokPerThread; ++i) {
-        const int j = jb + i;
-        keep |= (j < L && !sw.always(j) ? 1u : 0u) << i;
+        for (int q = 0; q < 4; ++q) v[q] = jb + q < j1 ? pi_load(P, ps, (jb + q) / kBlock) : 0.f;
+      } else {
+        const float4 w = pi_load4(P, ps, jb);
+        v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w;
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int j = jb + q;
+        const int e = BLK ? j / kBlock : j;
+        const bool k = j < j1 && !sw.always(j) && kept_by_cut(__float_as_uint(v[q]), e, tau, pos_cut);
+        keep |= (k ? 1u : 0u) << q;
       }
     }
-  } else if (jb < L) {
+    // warp scan of the lanes' counts, then the warps' totals
+    const int c = __popc(keep);
+    int x = c;
 #pragma unroll
-    for (int i = 0; i < kTokPerThread; ++i) {
-      const int j = jb + i;
-      const bool k = j < L && (bits[i] > tau || (bits[i] == tau && j <= pos_cut)) && !sw.always(j);
-      keep |= (k ? 1u : 0u) << i;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(kFull, x, o);
+      if (lane >= o) x += t;
     }
-  }
-  const int off = block_excl_scan(__popc(keep), sc.shi, (int*)nullptr);
-  const int64_t first = (int64_t)sc.off + off;
-  int* dst = P.sel_list + (size_t)un.s * P.Lmax;
-  int k = 0;
+    if (lane == 31) sc.shi[warp] = x;
+    __syncthreads();
+    int wbase = 0, total = 0;
 #pragma unroll
-  for (int i = 0; i < kTokPerThread; ++i) {
-    if (keep >> i & 1u) {
-      const int64_t o = first + k++;
-      if (o < P.Lmax) dst[o] = jb + i;
-      else atomicOr(P.ws.dev_err, kErrInternal);   // offsets and predicate disagree: never write past the list
+    for (int w = 0; w < kWarps; ++w) {
+      const int t = sc.shi[w];
+      wbase += w < warp ? t : 0;
+      total += t;
     }
+    __syncthreads();   // sc.shi is rewritten by the next round
+    int64_t o = run + wbase + (x - c);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (keep >> q & 1u) {
+        if (o < P.Lmax) dst[o] = jb + q;
+        else atomicOr(P.ws.dev_err, kErrInternal);   // offsets and predicate disagree: never write past the list
+        ++o;
+      }
+    }
+    run += total;
   }
 }
 
@@ -1316,43 +1440,76 @@ template <typename T, int G, bool BLK>
 __global__ void __launch_bounds__(kSelThreads, 4) k_select(StepParams P) {
   __shared__ SelSmem sm;
   __shared__ SelScalars sc;
-  const int nb = gridDim.x;
-  if (P.n_ret == 0) {   // nothing to select: only the query rotation
-    for (int s = blockIdx.x; s < P.n_slices; s += nb) qrot_slice<T>(P, sm.pro, sc, s);
-    return;
-  }
-  const int n_rs = P.B * P.n_ret;
-  const int n_units = n_rs * P.n_chunks;
-  if (blockIdx.x == 0 && threadIdx.x == 0) P.ws.bar[kBarDuty] = 0u;   // taken after two barriers
-  score_phase<T, G, BLK>(P, sm.score, sc);
-  if (!grid_barrier(P.ws.bar, P.ws.dev_err, &sc.ok)) return;
-  mass_phase<G, BLK>(P, sm, sc);
-  if (!grid_barrier(P.ws.bar, P.ws.dev_err, &sc.ok)) return;
-  for (int u = blockIdx.x; u < n_units; u += nb) {
-    const int y = u / P.n_chunks;
-    threshold_unit<BLK>(P, sc, y, u % P.n_chunks);
-    if (last_of_slice(&P.ws.st[unit_of(P, y).s].ticket_thr, P.n_chunks, &sc.ok)) refine_slice<BLK>(P, sm, sc, y);
-  }
-  qrot_duties<T>(P, sm.pro, sc);   // off the critical path: refine steps run meanwhile
-  if (!grid_barrier(P.ws.bar, P.ws.dev_err, &sc.ok)) return;
-  for (int u = blockIdx.x; u < n_units; u += nb) compact_unit<BLK>(P, sc, u / P.n_chunks, u % P.n_chunks);
+  const Ranges<BLK> R(P);
+  auto n_ranges = [&](int y) { return (unsigned)(R.last_cta(y) - R.first_cta(y) + 1); };
+  for_each_segment(R, [&](int y, int l0, int l1) {
+    score_segment<G>(P, sm.score, sc, y, l0, l1);
+    // failure-detection test hook: CTA 0 never arrives, so the other CTAs of its slice
+    // give up their bounded waits for the slice's statistics
+    if (!(P.drop_publish && blockIdx.x == 0)) slice_arrive(&P.ws.st[unit_of(P, y).s].arr_score);
+  });
+  if (P.drop_publish && blockIdx.x == 0) return;
+  bool ok = true;
+  for_each_segment(R, [&](int y, int l0, int l1) {
+    for (int a = l0; a < l1 && ok; a += kMaxRangeGroups)
+      ok = mass_segment<G, BLK>(P, sm.mass, sc, R, y, a, min(l1, a + kMaxRangeGroups), a == l0, n_ranges(y));
+    if (ok) slice_arrive(&P.ws.st[unit_of(P, y).s].arr_mass);
+  });
+  if (!ok) return;
+  prefetch_attended_rows<T>(P);
+  for_each_segment(R, [&](int y, int l0, int l1) {
+    if (!ok) return;
+    SliceState* st = P.ws.st + unit_of(P, y).s;
+    ok = slice_wait(&st->arr_mass, n_ranges(y), P.ws.dev_err, &sc.ok);
+    if (!ok) return;
+    cut1_range(P, sm.stage, sc, y, (int)blockIdx.x == R.first_cta(y));
+    threshold_segment<BLK>(P, sc, sm.ref, R, y, l0, l1);
+    slice_arrive(&st->arr_thr);
+  });
+  if (!ok) return;
+  for_each_segment(R, [&](int y, int l0, int l1) {
+    if (!ok) return;
+    SliceState* st = P.ws.st + unit_of(P, y).s;
+    ok = slice_wait(&st->arr_thr, n_ranges(y), P.ws.dev_err, &sc.ok);
+    if (!ok) return;
+    refine_range<BLK>(P, sm.ref, sc, y, (int)blockIdx.x == R.first_cta(y));
+    count_segment<BLK>(P, sc, R, y, l0, l1);
+    slice_arrive(&st->arr_cnt);
+  });
+  if (!ok) return;
+  for_each_segment(R, [&](int y, int l0, int l1) {
+    if (!ok) return;
+    ok = slice_wait(&P.ws.st[unit_of(P, y).s].arr_cnt, n_ranges(y), P.ws.dev_err, &sc.ok);
+    if (!ok) return;
+    offset_segment<BLK>(P, sc, R, y);
+    compact_segment<BLK>(P, sc, R, y, l0, l1);
+  });
 }
 
 template <typename T, int G>
 cudaError_t launch_tg(const StepParams& P, int grid, cudaStream_t st) {
+  k_qprep<T, G><<<P.n_slices, kSelThreads, 0, st>>>(P);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || P.n_ret == 0) return e;   // nothing to select
   StepParams local = P;
   void* args[] = {&local};
   const void* fn = P.blocks ? (const void*)k_select<T, G, true> : (const void*)k_select<T, G, false>;
-  return cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(kSelThreads), args, 0, st);
+  return cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(kSelThreads), args, kPiBytes, st);
 }
 
 // Co-resident CTAs per SM, the smaller of the token and block variants (one grid size
-// serves both).
+// serves both).  Also raises the variants' dynamic shared memory limit to kPiBytes.
 template <typename T, int G>
 int resident_tg() {
   int n = 0, m = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_select<T, G, false>, kSelThreads, 0) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, k_select<T, G, true>, kSelThreads, 0) != cudaSuccess)
+  if (cudaFuncSetAttribute(k_select<T, G, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPiBytes) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(k_select<T, G, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPiBytes) !=
+          cudaSuccess)
+    return -1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_select<T, G, false>, kSelThreads, kPiBytes) !=
+          cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, k_select<T, G, true>, kSelThreads, kPiBytes) != cudaSuccess)
     return -1;
   return n < m ? n : m;
 }
@@ -1360,10 +1517,10 @@ int resident_tg() {
 }  // namespace
 
 // Grid of the selection launch: every resident CTA (the same count on every SM, so the
-// range-partitioned score and mass phases are balanced per SM), but never more CTAs than
-// range quanta (16-token groups, or kBlock-token blocks in block mode), so no CTA has an
-// empty range.
+// range-partitioned phases are balanced per SM), but never more CTAs than range quanta
+// (16-token groups, or kBlock-token blocks in block mode), so no CTA has an empty range.
 int select_grid(const StepParams& P, int max_resident) {
+  if (max_resident > kMaxSelectGrid) max_resident = kMaxSelectGrid;
   if (P.n_ret <= 0) return P.n_slices < max_resident ? P.n_slices : max_resident;
   const long long qt = P.blocks ? kBlock : 16;
   const long long groups = (long long)P.B * P.n_ret * (((long long)P.Lcap + qt - 1) / qt);

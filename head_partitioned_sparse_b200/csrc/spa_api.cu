@@ -32,7 +32,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
-  size_t off[19];
+  size_t off[20];
   size_t total;
   int64_t max_items;
   int n_chunks_max;
@@ -48,7 +48,7 @@ Layout plan(const spa_config& c, int split_rows) {
   L.max_items = (int64_t)slices * ((Lmax + split_rows - 1) / split_rows);
   const int64_t part_slots = L.max_items > (int64_t)(spa::kMaxAttendCtas + slices + 1)
                                  ? L.max_items : (int64_t)(spa::kMaxAttendCtas + slices + 1);
-  size_t sz[19] = {
+  size_t sz[20] = {
       (size_t)c.n_q_heads * 16 * 128 * 4,                  // 0 P_q
       (size_t)c.n_kv_heads * 16 * 128 * 4,                 // 1 P_k
       64 * 8,                                              // 2 inv_freq
@@ -68,9 +68,10 @@ Layout plan(const spa_config& c, int split_rows) {
       slices * spa::kBins2 * 8,                            // 16 hist2
       spa::kBarWords * 4,                                  // 17 selection grid barrier
       slices * 4,                                          // 18 attention tickets
+      (spa::kMaxSelectGrid + slices) * 4,                  // 19 per-range kept counts (selection)
   };
   size_t o = 0;
-  for (int i = 0; i < 19; ++i) {
+  for (int i = 0; i < 20; ++i) {
     L.off[i] = o;
     o += round_up(sz[i], 256);
   }
@@ -513,6 +514,7 @@ spa_status spa_create(spa_handle* out, const spa_config* cfg) {
   w.hist2 = (unsigned long long*)(base + L.off[16]);
   w.bar = (unsigned*)(base + L.off[17]);
   w.attn_ticket = (unsigned*)(base + L.off[18]);
+  w.seg_cnt = (int*)(base + L.off[19]);
   w.max_items = L.max_items;
   h->n_chunks_max = L.n_chunks_max;
 

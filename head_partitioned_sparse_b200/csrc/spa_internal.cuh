@@ -32,8 +32,9 @@ constexpr int kBins3 = 64;
 // probabilities that add up to at most 1 (plus fp32 rounding).
 constexpr int kMassMinExp = 87;
 
-// Largest grid of the selection kernel (sizes the per-range statistics).
-constexpr int kMaxSelectGrid = 8192;
+// Largest grid of the selection kernel (sizes the per-range statistics, counts and
+// offsets, and the per-range table of the per-slice refine step in shared memory).
+constexpr int kMaxSelectGrid = 1024;
 // Largest grid of the attention kernels (the bf16 kernel writes one split state per
 // (CTA, slice) it touches: at most grid + slices of them).
 constexpr int kMaxAttendCtas = 1024;
@@ -57,20 +58,21 @@ constexpr unsigned kErrStartPos = 2u;
 constexpr unsigned kErrInternal = 4u;
 constexpr unsigned kErrTimeout = 8u;   // a bounded device-side wait gave up
 
-// Per (b, kv head) selection state.  Written by the selection kernel, read by its
-// later phases and by attention.
+// Per (b, kv head) selection state, reset for every call by the selection's prologue
+// kernel.  The arrival counters take one arrival per CTA range of the slice after each
+// phase of the selection kernel; count is read by attention.
 struct __align__(16) SliceState {
-  unsigned long long q_total;   // sum of quantised masses (units of 2^-63)
-  unsigned long long target;    // ceil(p * q_total)
-  unsigned long long m_above;   // mass of all tokens in digit1 bins above b1
+  unsigned long long target;    // cut target: ceil(p * total mass), or k for top-k
+  unsigned long long m_above;   // mass of all tokens in round-1 bins above b1
   int b1;                       // round-1 bin holding the cut; -1 = keep everything
-  unsigned tau_bits;            // fp32 bits of the cut probability tau
-  int pos_cut;                  // tied tokens (prob == tau) are kept iff pos <= pos_cut
   int count;                    // listed tokens (kept, outside sinks/window)
-  unsigned ticket_mass;         // last-CTA tickets of the mass and threshold phases
-  unsigned ticket_thr;
-  unsigned cand_count;          // candidates appended (tokens in bin b1)
-  unsigned qidx_ready;          // barrier generation + 1 once this call's q_idx is stored
+  unsigned arr_score;           // ranges whose score statistics are stored
+  unsigned arr_mass;            // ranges whose round-1 masses are added
+  unsigned arr_thr;             // ranges whose candidates are stored
+  unsigned arr_cnt;             // ranges whose kept counts are stored
+  unsigned ncand;               // candidates of the round-1 cut bin (slots taken)
+  unsigned tau_bits;            // fp32 bits of the cut value tau
+  int pos_cut;                  // tokens equal to tau are kept iff their position <= pos_cut
 };
 
 // Cut state of one (b, kv head) slice in a context-parallel step (each rank holds a
@@ -143,6 +145,7 @@ struct Workspace {
   int* item_base;        // [Bm*Hkv + 1]
   unsigned* attn_ticket; // [Bm*Hkv] pieces of each slice finished (bf16 attention; reset by its combiner)
   float* part;           // [max(max_items, kMaxAttendCtas + Bm*Hkv + 1)][G][kPartStride]
+  int* seg_cnt;          // [kMaxSelectGrid + Bm*Hkv] per-range kept (listed) tokens
   unsigned* dev_err;     // [1]
   unsigned* bar;         // [kBarWords] selection kernel: grid barrier and q_rot duty ticket
   int64_t max_items;
@@ -179,7 +182,7 @@ struct StepParams {
   int n_str;             // streaming heads (Hkv - n_ret)
   int ring;              // ring rows per streaming head: n_sink + window
   int head_rank[kMaxKvHeads];   // rank of head g among the retrieval or the streaming heads
-  int drop_publish;      // failure-detection test hook: leaders do not publish q_idx
+  int drop_publish;      // failure-detection test hook: selection CTA 0 skips the first grid barrier
   const void* k_ring;    // [Bm][n_str][ring][128] streaming-head keys (compact layout)
   const void* v_ring;
   float* lse;            // optional [B][Hq]: log2-sum-exp of each head's attended scores

@@ -149,6 +149,7 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
       (size_t)slices * P.n_chunks * 4,                         // chunk_gt
       (size_t)slices * P.n_chunks * 4,                         // chunk_off
       (size_t)slices * spa::kBins2 * 8,                        // hist2
+      (size_t)(spa::kMaxSelectGrid + slices) * 4,              // per-range kept counts
   };
   size_t off[sizeof sz / sizeof sz[0]];
   size_t o = head_bytes;
@@ -170,6 +171,7 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
   w.chunk_gt = (int*)(base + off[7]);
   w.chunk_off = (int*)(base + off[8]);
   w.hist2 = (unsigned long long*)(base + off[9]);
+  w.seg_cnt = (int*)(base + off[10]);
   w.bar = (unsigned*)(base + off_bar);
   w.dev_err = (unsigned*)(base + off_err);
   w.st = (spa::SliceState*)(base + off_st);

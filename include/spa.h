@@ -403,9 +403,9 @@ SPA_API spa_status spa_head_effective_ranks(const float* W_Q, const float* W_K, 
  */
 SPA_API spa_status spa_device_status(spa_handle h, spa_stream stream);
 
-/* Failure-detection test hook (no fault, no hang): while enabled, the selection's slice
- * leaders compute their query index vectors but do not publish them, so every other CTA
- * of the slice waits on a flag that nothing sets until its bounded wait (about 2 s)
+/* Failure-detection test hook (no fault, no hang): while enabled, the first CTA of the
+ * selection kernel leaves before its first grid barrier, so every other CTA waits at
+ * that barrier for an arrival that never comes until its bounded wait (about 2 s)
  * gives up; the call completes with meaningless lists and spa_device_status reports
  * SPA_ERR_DEVICE_TIMEOUT (and resets the synchronisation state, so the next call on the
  * handle is sound).  Off by default; for tests only. */

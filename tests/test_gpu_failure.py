@@ -1,7 +1,7 @@
 """Failure detection without a GPU fault: a bounded device-side wait runs out.
 
-With the test hook on, the selection's slice leaders skip publishing their query index
-vectors, so every other CTA of a slice waits on a flag that nothing sets until its
+With the test hook on, the selection kernel's first CTA leaves before the first grid
+barrier, so every other CTA waits there for an arrival that never comes until its
 bounded wait gives up.  The kernel still completes, spa_device_status reports
 SPA_ERR_DEVICE_TIMEOUT, and the next call on the same handle is correct again.
 """
@@ -18,7 +18,7 @@ from spa_testutil import DevInputs, Handle, check_selection, gpu_decode, gpu_sel
 pytestmark = pytest.mark.gpu
 
 
-def test_unpublished_query_vectors_time_out_and_the_handle_recovers():
+def test_missing_barrier_arrival_times_out_and_the_handle_recovers():
     inp = synth.make_inputs("tiny", 0, overrides={"dtype": "bf16", "L": 8192, "window": 256})
     ret = [g for g in range(inp.Hkv) if inp.head_mask[g]]
     idx = oracle_idx(inp, heads=ret)

@@ -1,11 +1,12 @@
 """Prefill chunk attention on the GPU vs the float64 oracle.
 
-Tolerance, derived per output element from the two roundings the kernel makes
-(everything else is float32): the rotated query is rounded to bf16, which moves each
-score s_j by at most e_j = 2^-9 sum_d |q_d k_jd| / sqrt(128), so each softmax weight by a
-factor within exp(+-2 E), E = max_j e_j; and each weight is rounded to bf16 (2^-9)
+Tolerance: every checked output element is within a bound derived per element from
+the two roundings the kernel makes (everything else is float32): the rotated query is
+rounded to bf16 (unit roundoff 2^-8), which moves each
+score s_j by at most e_j = 2^-8 sum_d |q_d k_jd| / sqrt(128), so each softmax weight by a
+factor within exp(+-2 E), E = max_j e_j; and each weight is rounded to bf16 (2^-8)
 before P V.  Hence
-  |out_d - oracle_d| <= (2.02 E + 2^-9 + 1e-5) * sum_j p_j |v_jd| + 1e-6,
+  |out_d - oracle_d| <= (2.02 E + 2^-8 + 1e-5) * sum_j p_j |v_jd| + 1e-6,
 with 1e-5 covering the float32 scores, exp2 and accumulation.
 """
 import numpy as np
@@ -42,8 +43,8 @@ def check_rows(inp, q, start, got, rows, n_sink, window):
         g = h // inp.G
         qr = O.rope(f(q[b, h, i]), int(start[b]) + i, inp.rope_theta)
         K, V = f(inp.k_cache[b, g, keys]), f(inp.v_cache[b, g, keys])
-        E = 2.0 ** -9 * np.max(np.abs(K) @ np.abs(qr)) / np.sqrt(128.0)
-        bound = (2.02 * E + 2.0 ** -9 + 1e-5) * (p @ np.abs(V)) + 1e-6
+        E = 2.0 ** -8 * np.max(np.abs(K) @ np.abs(qr)) / np.sqrt(128.0)
+        bound = (2.02 * E + 2.0 ** -8 + 1e-5) * (p @ np.abs(V)) + 1e-6
         err = np.abs(got[b, h, i] - want[b, h, i])
         assert np.all(err <= bound), (b, h, i, float(err.max()), float(bound[np.argmax(err - bound)]))
         worst = max(worst, float((err / bound).max()))
