@@ -12,11 +12,13 @@
 // accumulate).  The projector is split exactly into three bf16 parts (hi + mid + lo =
 // the float32 value), so every product is exact and the three parts accumulate into
 // the same float32 sums.  A warp takes 16-token tiles; each lane loads 64 contiguous
-// bytes of two key rows straight from global memory (16-byte loads), because the
+// bytes of two key rows straight from global memory (16-byte loads; the next tile's
+// rows are requested before the current tile is computed), because the
 // 128 dims are permuted consistently in A and B: k-step s, lane t4 covers physical
 // dims 32 t4 + 4 s .. + 3.  Output columns are permuted so that a lane ends with four
 // consecutive outputs of a row and writes them as one 8-byte store.  The B fragments
-// of the head's projector are built once per CTA in shared memory, in fragment order.
+// of the head's projector are built once per CTA (2048 tokens) in shared memory, in
+// fragment order.
 //
 // float32 keys (k_index_append): a CTA takes 64 consecutive tokens of one (b, kv head);
 // the key tile (rows padded to 129 floats so a warp's 8 rows hit 8 banks) and the
@@ -81,8 +83,8 @@ k_index_append(const T* __restrict__ k_pre, const int64_t* __restrict__ start_po
 
 // ---------------------------------------------------------------- tensor-core variant
 constexpr int kIaWarps = 8;
-constexpr int kIaTiles = 2;                               // 16-token tiles per warp
-constexpr int kIaTok = kIaWarps * kIaTiles * 16;          // 256 tokens per CTA
+constexpr int kIaTiles = 16;                              // 16-token tiles per warp
+constexpr int kIaTok = kIaWarps * kIaTiles * 16;          // 2048 tokens per CTA
 
 __device__ __forceinline__ void ia_mma(float (&d)[4], const uint32_t (&a)[4], uint2 b) {
   asm volatile(
@@ -119,6 +121,21 @@ k_index_append_mma(const __nv_bfloat16* __restrict__ k_pre, const int64_t* __res
   const int s_src = b * Hkv + g;
   const int sd = b * map.n_slots + map.slot[m];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, gid = lane >> 2, t4 = lane & 3;
+  const int64_t base_pos = start_pos[b];
+  const __nv_bfloat16* src = k_pre + (size_t)s_src * T_ * kHeadDim;
+  // warp w takes tiles w, w + 8, ... of the CTA's 2048 tokens; the next tile's rows are
+  // requested before the current tile is computed (two tiles in flight per warp)
+  auto load_tile = [&](int tile, uint4 (&qa)[4], uint4 (&qb)[4]) {
+    const int tok0 = blockIdx.x * kIaTok + tile * 16;
+    const int ra = tok0 + gid, rb = ra + 8;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      qa[i] = ra < T_ ? __ldg(reinterpret_cast<const uint4*>(src + (size_t)ra * kHeadDim + 32 * t4) + i)
+                      : make_uint4(0u, 0u, 0u, 0u);
+      qb[i] = rb < T_ ? __ldg(reinterpret_cast<const uint4*>(src + (size_t)rb * kHeadDim + 32 * t4) + i)
+                      : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
   const float* Pg = P_k + (size_t)g * kIdxDim * kHeadDim;
   for (int i = tid; i < 8 * 2 * 3 * 32; i += blockDim.x) {
     const int ln = i & 31, part = (i >> 5) % 3, t = (i / 96) & 1, ks = i / 192;
@@ -132,20 +149,14 @@ k_index_append_mma(const __nv_bfloat16* __restrict__ k_pre, const int64_t* __res
     bfrag[ks][t][part][ln] = v;
   }
   __syncthreads();
-  const int64_t base_pos = start_pos[b];
-  const __nv_bfloat16* src = k_pre + (size_t)s_src * T_ * kHeadDim;
-  for (int tile = 0; tile < kIaTiles; ++tile) {
-    const int tok0 = blockIdx.x * kIaTok + (warp * kIaTiles + tile) * 16;
-    if (tok0 >= T_) break;
-    const int ra = tok0 + gid, rb = ra + 8;
-    uint4 qa[4], qb[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      qa[i] = ra < T_ ? __ldg(reinterpret_cast<const uint4*>(src + (size_t)ra * kHeadDim + 32 * t4) + i)
-                      : make_uint4(0u, 0u, 0u, 0u);
-      qb[i] = rb < T_ ? __ldg(reinterpret_cast<const uint4*>(src + (size_t)rb * kHeadDim + 32 * t4) + i)
-                      : make_uint4(0u, 0u, 0u, 0u);
-    }
+  uint4 qa[4], qb[4], na[4], nb[4];
+  int tile = warp;
+  if (blockIdx.x * kIaTok + tile * 16 < T_) load_tile(tile, qa, qb);
+  for (; tile < kIaWarps * kIaTiles && blockIdx.x * kIaTok + tile * 16 < T_; tile += kIaWarps) {
+    const int next = tile + kIaWarps;
+    const bool more = next < kIaWarps * kIaTiles && blockIdx.x * kIaTok + next * 16 < T_;
+    if (more) load_tile(next, na, nb);
+    const int ra = blockIdx.x * kIaTok + tile * 16 + gid, rb = ra + 8;
     float c[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
@@ -174,6 +185,10 @@ k_index_append_mma(const __nv_bfloat16* __restrict__ k_pre, const int64_t* __res
       packed.x = ia_pack(c[0][2 * h], c[0][2 * h + 1]);
       packed.y = ia_pack(c[1][2 * h], c[1][2 * h + 1]);
       *reinterpret_cast<uint2*>(idx + ((size_t)sd * Lmax + pos) * kIdxDim + 4 * t4) = packed;
+    }
+    if (more) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { qa[i] = na[i]; qb[i] = nb[i]; }
     }
   }
 }

@@ -9,34 +9,36 @@
 // strategy (GQA scores aggregated to the group by their mean).
 //
 // Work partition: the retrieval slices' capacity, in 16-token groups, is split into
-// equal contiguous ranges, one per CTA; a range may span slices (one segment per slice
-// it touches).  Every phase works on the CTA's own range, and the probabilities of the
-// range stay in shared memory from the mass phase to the compaction.
-// Phases:
-//   score     each CTA forms the group's query index vectors q_idx = P_q q_pre itself
-//             (float64 dot products) while its first index rows are in flight, then per
-//             head h: m = max_j l_hj, z = sum_j 2^(l_hj - m),
-//             l_hj = log2(e) * idx_scale * <q_idx[h], idx_j>   (index read #1);
-//   -- grid barrier --
+// equal contiguous ranges, one per CTA (a whole number of CTAs per slice when the grid
+// holds at least one CTA per slice); a range may span slices (one segment per slice it
+// touches).  Every phase works on the CTA's own range, and the probabilities of the range
+// stay in shared memory from the mass phase to the compaction.  A prologue kernel
+// (k_qprep) forms q_idx = P_q q_pre per slice (float64 dot products) and q_rot = RoPE(q,
+// L-1) for the attention, and clears the slice's selection state and histograms.
+// Phases of k_select (the CTAs of one slice meet at three per-slice arrival counters;
+// there is no grid-wide barrier):
+//   score     per head: m = max_j l_hj, z = sum_j 2^(l_hj - m) over the range,
+//             l_hj = log2(e) * idx_scale * <q_idx[h], idx_j>   (index read #1, HBM);
+//   -- the slice's score statistics are complete --
 //   mass      merge (m, z) over the slice's ranges -> M_h, Z_h; recompute l_hj (index
 //             read #2, from L2), pi_j = sum_h 2^(l_hj - M_h) / (G Z_h), kept on chip; a
 //             mass histogram over the top 12 bits of pi_j's bit pattern, masses as
 //             integer multiples of 2^-63 so every sum is exact and order independent
-//             (per range as a count and a sum of low significand bits per bin);
-//   cut 1     per slice (last range, ticket): total mass, target ceil(p * total) (or k
-//             for top-k) and the bin b1 where the descending cumulative mass reaches it;
-//   -- grid barrier --
-//   threshold per range: tokens above b1 counted, tokens of bin b1 appended as
-//             candidates with their round-2 masses added to the slice histogram;
-//   refine    per slice (last range, ticket): the exact cut from the candidates - the
-//             value tau and the position up to which tokens equal to tau are kept
-//             (lowest positions first) - by an on-chip sort when they are few, else by
-//             two more radix rounds over the histogram; per-range output offsets.
-//             Meanwhile every CTA prefetches its share of the sink and window K/V rows
-//             into L2 for the attention kernel that follows (HBM is otherwise idle in
-//             these phases), and idle CTAs compute q_rot = RoPE(q_pre, L-1) for every
-//             head as duties (angles in float64, reduced exactly in units of pi);
-//   -- grid barrier --
+//             (per range as a count and a sum of low significand bits per bin); then an
+//             L2 prefetch of the sink and window K/V rows the attention reads next;
+//   -- the slice's histogram is complete --
+//   cut 1     every CTA reads the slice's histogram: total mass, target ceil(p * total)
+//             (or k for top-k) and the bin b1 where the descending cumulative mass
+//             reaches it;
+//   threshold per range: the listed tokens above b1 counted, the elements of bin b1
+//             appended as candidates with their round-A masses added to the slice's
+//             second histogram;
+//   -- the slice's candidates are complete --
+//   refine    every CTA takes the exact cut from the candidates - the value tau and the
+//             position up to which tokens equal to tau are kept (lowest positions first)
+//             - by an on-chip sort when they are few, else by more radix rounds, and its
+//             range's offset in the list from the counts above b1 and the kept
+//             candidates before it;
 //   compact   per range: kept positions outside sinks/window, ascending.
 // Block mode (the block-granular variant, a second instantiation): the ranges are cut at
 // kBlock-token block boundaries, the mass phase keeps and histograms each block's mass
@@ -44,8 +46,8 @@
 // steps rank blocks and count their listed tokens, and compact lists every token of a
 // kept block.  The blocks follow the chunk routing of the "Hierarchical Global
 // Attention" summary, Central mechanism §4.
-// One launch replaces a chain of small kernels whose fixed launch cost dominated.
-// Grid barriers are polled with a clock budget; on timeout they set a device status bit
+// One launch replaces a chain of small kernels whose fixed launch cost dominated.  The
+// arrival waits are polled with a clock budget; on timeout they set a device status bit
 // and the kernel leaves without hanging.  The launch is cooperative, so all CTAs are
 // resident together.
 #include <climits>
@@ -94,52 +96,6 @@ __device__ V block_sum(V x, V* sh) {
   V tot;
   block_excl_scan(x, sh, &tot);
   return tot;
-}
-
-// Bins are visited from the highest down; thread t owns bins [hi-15, hi], hi = 4095 - 16 t.
-// Finds the bin where base + cumulative mass first reaches target.  Result in *out_bin /
-// *out_above (mass strictly above that bin, base included); untouched if never reached.
-__device__ void find_cut_desc_4096(const unsigned long long (&m)[16], unsigned long long base,
-                                   unsigned long long target, unsigned long long* sh,
-                                   int* out_bin, unsigned long long* out_above) {
-  unsigned long long s = 0;
-#pragma unroll
-  for (int k = 0; k < 16; ++k) s += m[k];
-  unsigned long long cum = base + block_excl_scan(s, sh, (unsigned long long*)nullptr);
-  const int hi = 4095 - 16 * (int)threadIdx.x;
-#pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const unsigned long long nxt = cum + m[k];
-    if (cum < target && nxt >= target) {
-      *out_bin = hi - k;
-      *out_above = cum;
-    }
-    cum = nxt;
-  }
-  __syncthreads();
-}
-
-// Thread t's 16 coalesced histogram words (bins t + 256 k), issued before they are used.
-__device__ __forceinline__ void hist_issue(const unsigned long long* g, unsigned long long (&v)[16]) {
-#pragma unroll
-  for (int k = 0; k < 16; ++k) v[k] = __ldcg(g + threadIdx.x + 256 * k);
-}
-// Redistributes them through shared memory so that thread t holds bins 4095 - 16 t - k,
-// k = 0..15 (the layout of the descending cut search).  Ends with a CTA barrier.
-__device__ __forceinline__ void hist_desc(unsigned long long* stage, const unsigned long long (&v)[16],
-                                          unsigned long long (&m)[16]) {
-#pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const int i = (int)threadIdx.x + 256 * k;
-    stage[i + (i >> 4)] = v[k];
-  }
-  __syncthreads();
-#pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const int i = 4095 - 16 * (int)threadIdx.x - k;
-    m[k] = stage[i + (i >> 4)];
-  }
-  __syncthreads();
 }
 
 // Mass of a token in the radix select: its quantised probability for top-p, 1 for
@@ -367,12 +323,9 @@ struct SmemRefine {
   unsigned hl[512];                   // radix round: sum of the bits below the digit
   int tie[kTieCap];                   // positions of the candidates equal to the cut value
   int wcnt[kSelThreads / 32];         // per-warp counts
+  int wabv[kSelThreads / 32];         // per-warp counts of listed tokens above the cut bin
 };
-// Round-1 / round-2 histogram staged for the cut search: loaded coalesced, read back as
-// 16 consecutive bins per thread (index i stored at i + i / 16 against bank conflicts).
-struct SmemStage { unsigned long long h[kBins1 + kBins1 / 16]; };
 union SelSmem {
-  SmemStage stage;
   SmemPro pro;
   SmemScore score;
   SmemMass mass;
@@ -512,6 +465,7 @@ __device__ __forceinline__ unsigned* hist_a(const StepParams& P, int s) {
   return reinterpret_cast<unsigned*>(P.ws.hist2 + (size_t)s * kBins2);
 }
 
+
 // ------------------------------------------------------------------ query prologue kernel
 // One CTA per (b, kv head) slice, launched before the selection kernel: q_rot for the
 // slice's G heads (decode calls), and for a retrieval slice q_idx = P_q q_pre (float64
@@ -529,9 +483,8 @@ __global__ void __launch_bounds__(kSelThreads) k_qprep(StepParams P) {
       z.target = z.m_above = 0ull;
       z.b1 = -1;
       z.count = 0;
-      z.arr_score = z.arr_mass = z.arr_thr = z.arr_cnt = 0u;
-      z.ncand = z.tau_bits = 0u;
-      z.pos_cut = INT_MAX;
+      z.arr_score = z.arr_mass = z.arr_thr = 0u;
+      z.ncand = 0u;
       P.ws.st[s] = z;
     }
     unsigned long long* h1 = P.ws.hist1 + (size_t)s * kBins1;
@@ -555,21 +508,43 @@ __global__ void __launch_bounds__(kSelThreads) k_qprep(StepParams P) {
 // Ranges are cut at multiples of q groups (q = 1, or kBlock / 16 in block mode so that
 // no block is split; ngc is then a multiple of q): CTA c covers groups
 // [q floor(c Q / nb), q floor((c+1) Q / nb)), Q = n_rs ngc / q.
+// When the grid gives every retrieval slice the same whole number of CTAs, cps (the
+// usual case: the launch grid is chosen so), the same partition reduces to 32-bit
+// arithmetic computed once per CTA: CTA c = y cps + k covers local groups
+// [q floor(k qs / cps), q floor((k+1) qs / cps)) of slice y, qs = ngc / q.
 template <bool BLK>
 struct Ranges {
   static constexpr int q = BLK ? kBlock / 16 : 1;
   long long ngc, quanta;
   int nb;
+  int cps;                 // CTAs per slice (0: ranges may span slices)
+  int y_me, l0_me, l1_me;  // with cps: this CTA's one segment
   __device__ __forceinline__ Ranges(const StepParams& P) {
     ngc = ((long long)P.Lcap + 16 * q - 1) / (16 * q) * q;
-    quanta = (long long)P.B * P.n_ret * (ngc / q);
+    const int n_rs = P.B * P.n_ret;
+    quanta = (long long)n_rs * (ngc / q);
     nb = (int)gridDim.x;
+    cps = (n_rs > 0 && nb % n_rs == 0) ? nb / n_rs : 0;
+    y_me = l0_me = l1_me = 0;
+    if (cps) {
+      const long long qs = ngc / q;
+      y_me = (int)blockIdx.x / cps;
+      const int k = (int)blockIdx.x - y_me * cps;
+      l0_me = (int)((long long)k * qs / cps) * q;
+      l1_me = (int)((long long)(k + 1) * qs / cps) * q;
+    }
   }
   __device__ __forceinline__ long long begin(int c) const { return (long long)c * quanta / nb * q; }
   // CTA whose range holds global group g
   __device__ __forceinline__ int owner(long long g) const { return (int)(((g / q + 1) * nb - 1) / quanta); }
-  __device__ __forceinline__ int first_cta(int y) const { return owner((long long)y * ngc); }
-  __device__ __forceinline__ int last_cta(int y) const { return owner((long long)(y + 1) * ngc - 1); }
+  __device__ __forceinline__ int first_cta(int y) const { return cps ? y * cps : owner((long long)y * ngc); }
+  __device__ __forceinline__ int last_cta(int y) const {
+    return cps ? y * cps + cps - 1 : owner((long long)(y + 1) * ngc - 1);
+  }
+  // range-relative group offset of slice y's group 0
+  __device__ __forceinline__ long long seg_origin(int y) const {
+    return cps ? -(long long)l0_me : (long long)y * ngc - begin(blockIdx.x);
+  }
 };
 // Per-range values of slice y (statistics, counts, offsets) live at slot cta + y: the
 // CTAs of slice y are consecutive and the last one of y may be the first one of y + 1,
@@ -579,6 +554,10 @@ __device__ __forceinline__ size_t stats_slot(int cta, int y) { return (size_t)ct
 // Visits the CTA's range as segments f(y, l0, l1) of local groups [l0, l1) of slice y.
 template <class RT, class F>
 __device__ __forceinline__ void for_each_segment(const RT& R, F&& f) {
+  if (R.cps) {   // one segment, no 64-bit division, no loop state kept live across f
+    f(R.y_me, R.l0_me, R.l1_me);
+    return;
+  }
   const long long ge = R.begin(blockIdx.x + 1);
   for (long long g = R.begin(blockIdx.x); g < ge;) {
     const int y = (int)(g / R.ngc);
@@ -599,7 +578,7 @@ struct PiSeg {
 };
 template <bool BLK>
 __device__ __forceinline__ PiSeg pi_seg(const Ranges<BLK>& R, int y, int s) {
-  const long long t0 = 16 * ((long long)y * R.ngc - R.begin(blockIdx.x));
+  const long long t0 = 16 * R.seg_origin(y);
   PiSeg v;
   v.t0 = (int)(BLK ? t0 / kBlock : t0);
   v.s = s;
@@ -670,15 +649,14 @@ __device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc
 #pragma unroll
   for (int h = 0; h < NH; ++h) { m[h][0] = m[h][1] = -INFINITY; z[h][0] = z[h][1] = 0.f; }
   for (int gb = l0; 16 * gb < jend; gb += kWarps * U) {
-    if (gb > l0) {
-#pragma unroll
-      for (int u = 0; u < U; ++u) load_group(rows, 16 * (gb + warp + kWarps * u), jend, pol, ra[u], rb[u]);
-    }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int j = 16 * (gb + warp + kWarps * u);
       float lg[NH][2];
       group_logits<G>(ra[u], rb[u], qb, scale, lg);
+      // refill the consumed slot with the same slot of the next batch
+      load_group(rows, 16 * (gb + kWarps * U + warp + kWarps * u), jend, pol, ra[u], rb[u]);
+
 #pragma unroll
       for (int h = 0; h < NH; ++h) {
         online_add(m[h][0], z[h][0], j + gid < jend ? lg[h][0] : -INFINITY);
@@ -709,36 +687,72 @@ __device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc
 }
 
 // ------------------------------------------------------------------ cut 1 (per range)
-// Every CTA of a slice takes the slice's round-1 cut from the complete round-1 histogram
-// (32 KB, read from L2): total mass, target ceil(p * total) (or k for top-k) and the bin
-// b1 where the descending cumulative mass reaches it (-1: keep every token).  Results in
-// sc.b1, sc.target, sc.m_above; the slice's first CTA also stores them for the refine
+// Every CTA of a slice takes the slice's round-1 cut itself from the complete round-1
+// histogram (32 KB, read from L2): thread t loads the 16 consecutive bins 4095 - 16 t - k
+// (k = 0..15, descending), a warp scan and a scan of the 8 warp totals give the mass ahead
+// of each thread's bins, and the thread whose bins hold the crossing walks them: the
+// total mass, the target ceil(p * total) (or k for top-k) and the bin b1 where the
+// descending cumulative mass reaches it (-1: keep every token).  Results in sc.b1,
+// sc.target, sc.m_above (the mass of all bins above b1) and sc.L (the sequence length,
+// read in the same round trip); the slice's first CTA also stores the cut for the refine
 // step of every range.
-__device__ void cut1_range(const StepParams& P, SmemStage& sm, SelScalars& sc, int y, bool lead) {
+__device__ void cut1_range(const StepParams& P, SelScalars& sc, int y, bool lead) {
   const Unit un = unit_of(P, y);
-  const int tid = threadIdx.x;
-  unsigned long long v[16], m16[16];
-  hist_issue(P.ws.hist1 + (size_t)un.s * kBins1, v);
-  unsigned long long tsum = 0;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const ulonglong2* h = reinterpret_cast<const ulonglong2*>(P.ws.hist1 + (size_t)un.s * kBins1 + kBins1 - 16 * (tid + 1));
+  ulonglong2 hv[8];
 #pragma unroll
-  for (int k = 0; k < 16; ++k) tsum += v[k];
-  const unsigned long long total = block_sum(tsum, sc.shl);
-  hist_desc(sm.h, v, m16);
-  unsigned long long target = total;
-  bool keep_all = P.keep_all || total == 0ull;
-  if (!keep_all) {
-    // top-k: the k-th token (total = the number of tokens); top-p: the mass ceil(p total)
-    target = P.topk > 0 ? (unsigned long long)P.topk : (unsigned long long)ceil((double)P.p * (double)total);
-    if (target < 1ull) target = 1ull;
-    keep_all = target >= total && P.topk > 0 ? true : target > total;   // k >= L keeps all
+  for (int k = 0; k < 8; ++k) hv[k] = __ldcg(h + k);   // bins 4080 - 16 t .. 4095 - 16 t, ascending
+  if (tid == 0) sc.L = load_len(P.seq_lens, un.b, P.Lcap, P.ws.dev_err);
+  unsigned long long mine = 0ull;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mine += hv[k].x + hv[k].y;
+  unsigned long long x = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long t = __shfl_up_sync(kFull, x, o);
+    if (lane >= o) x += t;
   }
+  if (lane == 31) sc.shl[warp] = x;
   if (tid == 0) sc.cut_bin = -1;
   __syncthreads();
-  if (!keep_all) find_cut_desc_4096(m16, 0ull, target, sc.shl, &sc.cut_bin, &sc.cut_above);
+  unsigned long long wbase = 0ull, tot = 0ull;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const unsigned long long t = sc.shl[w];
+    wbase += w < warp ? t : 0ull;
+    tot += t;
+  }
+  unsigned long long target = tot;
+  bool keep_all = P.keep_all || tot == 0ull;
+  if (!keep_all) {
+    // top-k: the k-th token (total = the number of tokens); top-p: the mass ceil(p total)
+    target = P.topk > 0 ? (unsigned long long)P.topk : (unsigned long long)ceil((double)P.p * (double)tot);
+    if (target < 1ull) target = 1ull;
+    keep_all = target >= tot && P.topk > 0 ? true : target > tot;   // k >= L keeps all
+  }
+  if (!keep_all) {
+    unsigned long long cum = wbase + x - mine;   // mass of the bins above this thread's
+    if (cum < target && cum + mine >= target) {
+#pragma unroll
+      for (int k = 7; k >= 0; --k) {
+        const unsigned long long b[2] = {hv[k].y, hv[k].x};   // descending: bin 2k + 1, then 2k
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          if (cum < target && cum + b[e] >= target) {
+            sc.cut_bin = kBins1 - 16 * (tid + 1) + 2 * k + 1 - e;
+            sc.cut_above = cum;
+          }
+          cum += b[e];
+        }
+      }
+    }
+  }
+  __syncthreads();
   if (tid == 0) {
-    sc.b1 = keep_all ? -1 : sc.cut_bin;
+    sc.b1 = keep_all ? -1 : sc.cut_bin;   // a search that fails keeps every token
     sc.target = target;
-    sc.m_above = keep_all ? 0ull : sc.cut_above;
+    sc.m_above = sc.b1 >= 0 ? sc.cut_above : 0ull;
     if (lead) {
       SliceState* st = P.ws.st + un.s;
       st->target = sc.target;
@@ -830,16 +844,15 @@ __device__ bool mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
   }
   const int jend = min(L, 16 * l1);
   for (int gb = l0; 16 * gb < jend; gb += kWarps * U) {
-    if (gb > l0) {
-#pragma unroll
-      for (int u = 0; u < U; ++u) load_group(rows, 16 * grp(gb, u), jend, pol, ra[u], rb[u]);
-    }
     float bsum = 0.f;
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int j = 16 * grp(gb, u);
       float lg[NH][2];
       group_logits<G>(ra[u], rb[u], qb, scale, lg);
+      // refill the consumed slot with the same slot of the next batch
+      load_group(rows, 16 * grp(gb + kWarps * U, u), jend, pol, ra[u], rb[u]);
+
       // pi = sum over the group's heads of 2^(l - M_h) / (G Z_h): lane-local heads first,
       // then the 4 lanes of a token (fixed order, identical result in every lane)
       float pr[2];
@@ -851,16 +864,27 @@ __device__ bool mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
           if (G < 4 && W[h] == 0.f) continue;   // lanes of absent heads (G < 4) add nothing
           acc += ex2(lg[h][cc] - M[h]) * W[h];
         }
-        acc += __shfl_xor_sync(kFull, acc, 1);
-        acc += __shfl_xor_sync(kFull, acc, 2);
         pr[cc] = acc;
       }
       if (BLK) {
+        // every lane ends with both tokens' sums
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          pr[cc] += __shfl_xor_sync(kFull, pr[cc], 1);
+          pr[cc] += __shfl_xor_sync(kFull, pr[cc], 2);
+        }
         bsum += (j + gid < jend ? pr[0] : 0.f) + (j + gid + 8 < jend ? pr[1] : 0.f);
-      } else if (t4 < 2) {   // lane t4 = 0 keeps token gid, t4 = 1 token gid + 8
-        const int jt = j + gid + 8 * t4;
-        const float v = t4 == 0 ? pr[0] : pr[1];
-        if (jt < jend) {
+      } else {
+        // transposed reduction: after the exchange with lane t4 ^ 1, even lanes hold token
+        // gid's pair sum and odd lanes token gid + 8's; after t4 ^ 2, lanes t4 = 0 and 1
+        // hold the two tokens' sums over the 4 lanes (the same additions in the same order
+        // as reducing each token over the 4 lanes)
+        const bool odd = (t4 & 1) != 0;
+        float v = odd ? pr[1] : pr[0];
+        v += __shfl_xor_sync(kFull, odd ? pr[0] : pr[1], 1);
+        v += __shfl_xor_sync(kFull, v, 2);
+        const int jt = j + gid + 8 * t4;   // lane t4 = 0 keeps token gid, t4 = 1 token gid + 8
+        if (t4 < 2 && jt < jend) {
           pi_store(P, ps, jt, v);
           const unsigned bits = __float_as_uint(v);
           const unsigned d = min(bits >> 18, (unsigned)(kBins1 - 1));
@@ -963,27 +987,27 @@ __device__ __forceinline__ void seg_elems(int L, int l0, int l1, int& e0, int& e
 }
 
 // One range of slice y (after cut1_range of y): the elements of bin b1 are the slice's
-// candidates.  Two passes over the range's probabilities (on chip): the first counts
-// them per warp, one atomic per CTA reserves their slots in the slice's candidate array,
-// the second writes them (bits, element) in range order and adds them to the slice's
-// round-A histogram (bits 17..9: count and sum of bits 8..0).  Token mode: lane l of warp
-// w reads elements 4 l .. 4 l + 3 of the warp's 128 as one 16-byte load.
+// candidates; the listed tokens of the elements above b1 (every element when b1 < 0) are
+// kept whatever the exact cut, and their count is stored at the range's slot.  Two passes
+// over the range's probabilities (on chip): the first counts both per warp, one atomic per
+// CTA reserves the candidates' slots in the slice's candidate array, the second writes
+// them (bits, element) in range order and adds them to the slice's round-A histogram
+// (bits 17..9: count and sum of bits 8..0).  Token mode: lane l of warp w reads elements
+// 4 l .. 4 l + 3 of the warp's 128 as one 16-byte load.
 template <bool BLK>
 __device__ void threshold_segment(const StepParams& P, SelScalars& sc, SmemRefine& sm, const Ranges<BLK>& R, int y,
                                   int l0, int l1) {
   const Unit un = unit_of(P, y);
   const PiSeg ps = pi_seg<BLK>(R, y, un.s);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  __syncthreads();   // earlier readers of the scalars are done
-  if (tid == 0) sc.L = load_len(P.seq_lens, un.b, P.Lcap, P.ws.dev_err);
-  __syncthreads();
-  const int L = sc.L, b1 = sc.b1;   // b1 from cut1_range
-  if (b1 < 0) return;               // keep everything: no candidates
+  const int L = sc.L, b1 = sc.b1;   // from cut1_range (b1 < 0: keep everything)
+  const SinkWindow sw(L, P.n_sink, P.window);
   int e0, e1;
   seg_elems<BLK>(L, l0, l1, e0, e1);
   constexpr int kPer = BLK ? 1 : 4;
-  // candidate mask of the thread's elements of round k0 (their bits in bits[])
-  auto cand_mask = [&](int k0, unsigned (&bits)[kPer]) {
+  // candidate mask of the thread's elements of round k0 (their bits in bits[]); the
+  // listed tokens of its elements above b1 are added to *above
+  auto cand_mask = [&](int k0, unsigned (&bits)[kPer], int* above) {
     const int eb = k0 + (BLK ? tid : 128 * warp + 4 * lane);
     unsigned m = 0u;
     if (BLK) {
@@ -996,27 +1020,40 @@ __device__ void threshold_segment(const StepParams& P, SelScalars& sc, SmemRefin
       bits[3] = __float_as_uint(v.w);
     }
 #pragma unroll
-    for (int q = 0; q < kPer; ++q)
-      if (eb + q < e1 && (int)min(bits[q] >> 18, (unsigned)(kBins1 - 1)) == b1) m |= 1u << q;
+    for (int q = 0; q < kPer; ++q) {
+      if (eb + q < e1) {
+        const int bin = (int)min(bits[q] >> 18, (unsigned)(kBins1 - 1));
+        if (bin == b1) m |= 1u << q;
+        if (above && bin > b1) *above += listed_of<BLK>(sw, L, eb + q);
+      }
+    }
     return m;
   };
-  int wc = 0;   // this warp's candidates (every lane holds the warp's sum)
+  int wc = 0;      // this warp's candidates (every lane holds the warp's sum)
+  int above = 0;   // this thread's listed tokens above b1
   for (int k0 = e0; k0 < e1; k0 += kSelThreads * kPer) {
     unsigned bits[kPer];
-    int c = __popc(cand_mask(k0, bits));
+    int c = __popc(cand_mask(k0, bits, &above));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(kFull, c, o);
     wc += c;
   }
-  if (lane == 0) sm.wcnt[warp] = wc;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(kFull, above, o);
+  if (lane == 0) {
+    sm.wcnt[warp] = wc;
+    sm.wabv[warp] = above;
+  }
   __syncthreads();
   unsigned total = 0u;
-  int wbase = 0;
+  int wbase = 0, above_all = 0;
 #pragma unroll
   for (int w = 0; w < kWarps; ++w) {
     total += (unsigned)sm.wcnt[w];
     wbase += w < warp ? sm.wcnt[w] : 0;
+    above_all += sm.wabv[w];
   }
+  if (tid == 0) P.ws.seg_cnt[stats_slot(blockIdx.x, y)] = above_all;
   if (total == 0u) return;
   if (tid == 0) sc.cbase = atomicAdd(&P.ws.st[un.s].ncand, total);
   __syncthreads();
@@ -1025,7 +1062,7 @@ __device__ void threshold_segment(const StepParams& P, SelScalars& sc, SmemRefin
   unsigned slot = sc.cbase + (unsigned)wbase;
   for (int k0 = e0; k0 < e1; k0 += kSelThreads * kPer) {
     unsigned bits[kPer];
-    const unsigned m = cand_mask(k0, bits);
+    const unsigned m = cand_mask(k0, bits, nullptr);
     const int eb = k0 + (BLK ? tid : 128 * warp + 4 * lane);
     // lanes in order, each lane's elements in order
     const int c = __popc(m);
@@ -1124,8 +1161,14 @@ __device__ void digit_kth_asc(const SmemRefine& sm, SelScalars& sc, unsigned lon
   }
 }
 
-// The slice's exact cut, taken by every CTA of the slice for itself once every range has
-// stored its candidates.  All tokens above the round-1 bin b1 are kept; among the
+// Whether element e (token e, or block e) is kept by the cut (tau, pos_cut).
+__device__ __forceinline__ bool kept_by_cut(unsigned bits, int e, unsigned tau, int pos_cut) {
+  return bits > tau || (bits == tau && e <= pos_cut);
+}
+
+// The slice's exact cut and this range's place in the slice's list, taken by every CTA of
+// the slice for itself once every range has stored its candidates and its count of
+// listed tokens above the round-1 bin b1.  All tokens above b1 are kept; among the
 // candidates of b1, in (pi desc, position asc) order, a candidate is kept while the mass
 // ranked ahead of it (m_above plus the candidates before it) is below the target.
 // Round A: the round-A histogram (bits 17..9, exact masses from counts and sums of the
@@ -1133,23 +1176,64 @@ __device__ void digit_kth_asc(const SmemRefine& sm, SelScalars& sc, unsigned lon
 // array gathers the candidates of dA on chip; round B over those (bits 8..0) gives the
 // cut value tau and the mass above it; if only some of the candidates equal to tau are
 // needed, the lowest positions are kept: ranked directly when they are few, else by
-// three 8-bit rounds over their positions.  Results in sc.tau, sc.pos_cut and sc.L;
-// the slice's first CTA (lead) also stores tau and pos_cut.
+// three 8-bit rounds over their positions.  The kept candidates' listed tokens, those
+// before this range and all of them, added to the ranges' counts above b1, give the
+// range's offset and the slice's total.  A search that finds no cut (inconsistent
+// masses) keeps every candidate of the last digit it reached and above, so the counts
+// and the compaction's predicate still agree.  Results in sc.tau, sc.pos_cut, sc.L and
+// sc.off; the slice's first CTA (lead) stores the total.
 template <bool BLK>
-__device__ void refine_range(const StepParams& P, SmemRefine& sm, SelScalars& sc, int y, bool lead) {
+__device__ void refine_range(const StepParams& P, SmemRefine& sm, SelScalars& sc, const Ranges<BLK>& R, int y,
+                             int l0, int l1, bool lead) {
   const Unit un = unit_of(P, y);
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const SliceState* st = P.ws.st + un.s;
+  const int first = R.first_cta(y), n_seg = R.last_cta(y) - first + 1, mine = (int)blockIdx.x - first;
+  const int* abv_row = P.ws.seg_cnt + stats_slot(first, y);
+  constexpr int kSegPer = kMaxSelectGrid / kSelThreads;
+  // one round trip: the cut state, the ranges' counts above b1, the round-A histogram
+  // (4 words per thread) and the first kRefBatch candidates per thread (read up to the
+  // row's capacity, used below n)
   const unsigned long long target = __ldcg(&st->target);
   const unsigned long long mab = __ldcg(&st->m_above);
   const int b1 = __ldcg(&st->b1);
-  const unsigned n = b1 >= 0 ? __ldcg(&st->ncand) : 0u;
+  const unsigned n_raw = __ldcg(&st->ncand);
   const int L = load_len(P.seq_lens, un.b, P.Lcap, P.ws.dev_err);
   const uint2* cand = P.ws.cand + (size_t)un.s * P.Lmax;
   const unsigned* ha = hist_a(P, un.s);
+  int av[kSegPer];
+#pragma unroll
+  for (int k = 0; k < kSegPer; ++k) {
+    const int c = tid + kSelThreads * k;
+    av[k] = c < n_seg ? __ldcg(abv_row + c) : 0;
+  }
   unsigned hav[4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) hav[k] = b1 >= 0 ? __ldcg(ha + tid + kSelThreads * k) : 0u;
+  for (int k = 0; k < 4; ++k) hav[k] = __ldcg(ha + tid + kSelThreads * k);
+  uint2 c0[kRefBatch];
+#pragma unroll
+  for (int u = 0; u < kRefBatch; ++u) {
+    const unsigned i = tid + kSelThreads * u;
+    c0[u] = i < (unsigned)P.Lmax ? __ldcg(cand + i) : make_uint2(0u, 0u);
+  }
+  const unsigned n = b1 >= 0 ? n_raw : 0u;
+  {
+    int before = 0, all = 0;
+#pragma unroll
+    for (int k = 0; k < kSegPer; ++k) {
+      all += av[k];
+      before += tid + kSelThreads * k < mine ? av[k] : 0;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      before += __shfl_xor_sync(kFull, before, o);
+      all += __shfl_xor_sync(kFull, all, o);
+    }
+    if (lane == 0) {
+      sm.wcnt[warp] = before;
+      sm.wabv[warp] = all;
+    }
+  }
 #pragma unroll
   for (int k = 0; k < 4; ++k) {   // words 0..511 counts, 512..1023 low sums
     const int w = tid + kSelThreads * k;
@@ -1162,9 +1246,29 @@ __device__ void refine_range(const StepParams& P, SmemRefine& sm, SelScalars& sc
     sc.nsmall = 0u;
   }
   __syncthreads();
-  // f(v) for every candidate, kRefBatch coalesced loads per thread issued together
+  int ab_before = 0, ab_all = 0;   // listed tokens above b1: ranges before this one, all
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    ab_before += sm.wcnt[w];
+    ab_all += sm.wabv[w];
+  }
+  // listed tokens of the kept candidates: before this range's first element, all
+  int e0, e1;
+  seg_elems<BLK>(L, l0, l1, e0, e1);
+  const SinkWindow sw(L, P.n_sink, P.window);
+  int pb = 0, pt = 0;
+  auto kept_cand = [&](uint2 v) {
+    const int c = listed_of<BLK>(sw, L, (int)v.y);
+    pt += c;
+    pb += (int)v.y < e0 ? c : 0;
+  };
+  // f(v) for every candidate, kRefBatch coalesced loads per thread issued together (the
+  // first batch is the one already loaded)
   auto for_each_cand = [&](auto&& f) {
-    for (unsigned i0 = 0; i0 < n; i0 += kSelThreads * kRefBatch) {
+#pragma unroll
+    for (int u = 0; u < kRefBatch; ++u)
+      if (tid + kSelThreads * u < n) f(c0[u]);
+    for (unsigned i0 = kSelThreads * kRefBatch; i0 < n; i0 += kSelThreads * kRefBatch) {
       uint2 v[kRefBatch];
 #pragma unroll
       for (int u = 0; u < kRefBatch; ++u) {
@@ -1176,23 +1280,28 @@ __device__ void refine_range(const StepParams& P, SmemRefine& sm, SelScalars& sc
         if (v[u].y != 0xffffffffu) f(v[u]);
     }
   };
-  unsigned tau = 0u;
+  unsigned tau = 0u;     // keep everything (b1 < 0)
   int pos_cut = INT_MAX;
-  bool found = b1 < 0;   // keep-everything mode needs no cut
   if (b1 >= 0) {
     const unsigned sig1 = (((unsigned)b1 & 31u) << 18) | 0x800000u;   // significand bits above bit 18
     digit_cut_desc(P, sm, sc, b1, [&](int d) { return sig1 | ((unsigned)d << 9); }, mab, target);
     __syncthreads();
     const int dA = sc.digit;
     const unsigned long long aboveA = sc.above;
-    found = dA >= 0;
-    if (found) {
+    if (dA < 0) {
+      tau = (unsigned)b1 << 18;   // no cut found: every candidate of b1 is kept
+      for_each_cand(kept_cand);
+    } else {
       const unsigned preB = ((unsigned)b1 << 9) | (unsigned)dA;
-      // the candidates of digit dA, gathered on chip
+      tau = preB << 9;   // until the cut is found: every candidate of dA and above is kept
+      // the candidates of digit dA gathered on chip; those above it are kept
       for_each_cand([&](uint2 v) {
-        if ((v.x >> 9) == preB) {
+        const unsigned d9 = v.x >> 9;
+        if (d9 == preB) {
           const unsigned k = atomicAdd(&sc.nsmall, 1u);
           if (k < (unsigned)kSmallList) sm.small[k] = v;
+        } else if (d9 > preB) {
+          kept_cand(v);
         }
       });
       for (int d = tid; d < 512; d += kSelThreads) sm.hc[d] = sm.hl[d] = 0u;
@@ -1209,157 +1318,144 @@ __device__ void refine_range(const StepParams& P, SmemRefine& sm, SelScalars& sc
           for_each_cand([&](uint2 v) { if ((v.x >> 9) == preB) f(v); });
         }
       };
-      // round B: bits 8..0 of the candidates of digit dA
-      for_each_small([&](uint2 v) { atomicAdd(&sm.hc[v.x & 511u], 1u); });
-      __syncthreads();
-      const unsigned sigA = sig1 | ((unsigned)dA << 9);
-      digit_cut_desc(P, sm, sc, b1, [&](int d) { return sigA | (unsigned)d; }, aboveA, target);
-      __syncthreads();
-      found = sc.digit >= 0;
-      if (found) {
-        const int dB = sc.digit;
-        tau = preB << 9 | (unsigned)dB;                 // fp32 bits of the cut value
-        const unsigned long long m_gt = sc.above;       // mass strictly above tau
-        const unsigned n_eq = sm.hc[dB];                 // candidates equal to tau
-        const unsigned long long q_tau = sel_mass(P, tau);
-        const unsigned long long need =
-            (q_tau > 0ull && target > m_gt) ? (target - m_gt + q_tau - 1ull) / q_tau : ~0ull;
-        __syncthreads();   // every read of sm.hc is done
-        if (need < (unsigned long long)n_eq) {
-          // keep the need lowest positions among the candidates equal to tau
-          if (n_eq <= (unsigned)kTieCap) {
-            for_each_small([&](uint2 v) {
-              if (v.x == tau) sm.tie[atomicAdd(&sc.ntie, 1)] = (int)v.y;
-            });
-            __syncthreads();
-            if (tid < (int)n_eq) {
-              const int pmine = sm.tie[tid];
-              unsigned r = 0u;
-              for (unsigned k = 0; k < n_eq; ++k) r += sm.tie[k] < pmine ? 1u : 0u;
-              if (r == (unsigned)need - 1u) sc.pos_cut = pmine;
-            }
-            __syncthreads();
-          } else {
-            unsigned pp = 0u;
-            unsigned long long before = 0ull;
-            bool ok = true;
-            for (int sh = 16; sh >= 0 && ok; sh -= 8) {   // positions < 2^24
-              for (int d = tid; d < 256; d += kSelThreads) sm.hc[d] = 0u;
-              if (tid == 0) sc.digit = -1;
-              __syncthreads();
-              for_each_small([&](uint2 v) {
-                if (v.x == tau && (v.y >> (sh + 8)) == pp) atomicAdd(&sm.hc[(v.y >> sh) & 255u], 1u);
-              });
-              __syncthreads();
-              digit_kth_asc(sm, sc, before, need);
-              __syncthreads();
-              ok = sc.digit >= 0;
-              if (ok) {
-                pp = (pp << 8) | (unsigned)sc.digit;
-                before = sc.above;
-              }
-            }
-            if (tid == 0) sc.pos_cut = ok ? (int)pp : INT_MAX;
-            __syncthreads();
+      if (ns <= 32u) {
+        // few: warp 0 sorts them by (pi desc, position asc) and keeps the prefix whose
+        // mass ahead stays below the target; the last kept gives tau and pos_cut
+        if (tid < 32) {
+          unsigned long long key = 0ull, m = 0ull;
+          if (lane < (int)ns) {
+            const uint2 v = sm.small[lane];
+            key = ((unsigned long long)v.x << 32) | (0xffffffffu - v.y);
+            m = sel_mass(P, v.x);
           }
+#pragma unroll
+          for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+            for (int j = k >> 1; j > 0; j >>= 1) {
+              const unsigned long long ok_ = __shfl_xor_sync(kFull, key, j);
+              const unsigned long long om = __shfl_xor_sync(kFull, m, j);
+              const bool desc = (lane & k) == 0, lower = (lane & j) == 0;
+              // lower lane of the pair keeps the larger key in a descending run
+              const bool take = lower == desc ? ok_ > key : ok_ < key;
+              if (take) { key = ok_; m = om; }
+            }
+          }
+          unsigned long long x = m;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long t = __shfl_up_sync(kFull, x, o);
+            if (lane >= o) x += t;
+          }
+          const unsigned long long before = aboveA + x - m;
+          const bool kept = key != 0ull && before < target;
+          const unsigned kmask = __ballot_sync(kFull, kept);
+          if (kmask != 0u && lane == 31 - __clz(kmask)) {   // the last kept
+            sc.tau = (unsigned)(key >> 32);
+            sc.pos_cut = (int)(0xffffffffu - (unsigned)key);
+            sc.digit = 1;
+          }
+        }
+        __syncthreads();
+        if (sc.digit >= 0) {
+          tau = sc.tau;
           pos_cut = sc.pos_cut;
         }
+      } else {
+        // round B: bits 8..0 of the candidates of digit dA
+        for_each_small([&](uint2 v) { atomicAdd(&sm.hc[v.x & 511u], 1u); });
+        __syncthreads();
+        const unsigned sigA = sig1 | ((unsigned)dA << 9);
+        digit_cut_desc(P, sm, sc, b1, [&](int d) { return sigA | (unsigned)d; }, aboveA, target);
+        __syncthreads();
+        if (sc.digit >= 0) {
+          const int dB = sc.digit;
+          tau = preB << 9 | (unsigned)dB;                 // fp32 bits of the cut value
+          const unsigned long long m_gt = sc.above;       // mass strictly above tau
+          const unsigned n_eq = sm.hc[dB];                 // candidates equal to tau
+          const unsigned long long q_tau = sel_mass(P, tau);
+          const unsigned long long need =
+              (q_tau > 0ull && target > m_gt) ? (target - m_gt + q_tau - 1ull) / q_tau : ~0ull;
+          __syncthreads();   // every read of sm.hc is done
+          if (need < (unsigned long long)n_eq) {
+            // keep the need lowest positions among the candidates equal to tau
+            if (n_eq <= (unsigned)kTieCap) {
+              for_each_small([&](uint2 v) {
+                if (v.x == tau) sm.tie[atomicAdd(&sc.ntie, 1)] = (int)v.y;
+              });
+              __syncthreads();
+              if (tid < (int)n_eq) {
+                const int pmine = sm.tie[tid];
+                unsigned r = 0u;
+                for (unsigned k = 0; k < n_eq; ++k) r += sm.tie[k] < pmine ? 1u : 0u;
+                if (r == (unsigned)need - 1u) sc.pos_cut = pmine;
+              }
+              __syncthreads();
+            } else {
+              unsigned pp = 0u;
+              unsigned long long before = 0ull;
+              bool ok = true;
+              for (int sh = 16; sh >= 0 && ok; sh -= 8) {   // positions < 2^24
+                for (int d = tid; d < 256; d += kSelThreads) sm.hc[d] = 0u;
+                if (tid == 0) sc.digit = -1;
+                __syncthreads();
+                for_each_small([&](uint2 v) {
+                  if (v.x == tau && (v.y >> (sh + 8)) == pp) atomicAdd(&sm.hc[(v.y >> sh) & 255u], 1u);
+                });
+                __syncthreads();
+                digit_kth_asc(sm, sc, before, need);
+                __syncthreads();
+                ok = sc.digit >= 0;
+                if (ok) {
+                  pp = (pp << 8) | (unsigned)sc.digit;
+                  before = sc.above;
+                }
+              }
+              if (tid == 0) sc.pos_cut = ok ? (int)pp : INT_MAX;
+              __syncthreads();
+            }
+            pos_cut = sc.pos_cut;
+          }
+        }
       }
+      // the kept candidates of digit dA
+      for_each_small([&](uint2 v) {
+        if (kept_by_cut(v.x, (int)v.y, tau, pos_cut)) kept_cand(v);
+      });
     }
   }
-  if (!found) {   // a search that fails keeps every token rather than index a missing bin
-    tau = 0u;
-    pos_cut = INT_MAX;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    pb += __shfl_xor_sync(kFull, pb, o);
+    pt += __shfl_xor_sync(kFull, pt, o);
   }
-  __syncthreads();   // earlier readers of the scalars are done
+  __syncthreads();   // earlier readers of the scalars and of the per-warp counts are done
+  if (lane == 0) {
+    sm.wcnt[warp] = pb;
+    sm.wabv[warp] = pt;
+  }
+  __syncthreads();
   if (tid == 0) {
+    int kb = 0, kt = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      kb += sm.wcnt[w];
+      kt += sm.wabv[w];
+    }
     sc.tau = tau;
     sc.pos_cut = pos_cut;
     sc.L = L;
-    if (lead) {   // for the compaction of every range of the slice
-      SliceState* stw = P.ws.st + un.s;
-      stw->tau_bits = tau;
-      stw->pos_cut = pos_cut;
+    sc.off = ab_before + kb;
+    if (lead) {   // the slice's listed count, for the attention kernel
+      const int total = ab_all + kt;
+      P.ws.st[un.s].count = total;
+      if (P.sel_count) P.sel_count[un.s] = total;
     }
-  }
-  __syncthreads();
-}
-
-// ------------------------------------------------------------------ kept count and offset
-// Whether element e (token e, or block e) is kept by the cut (tau, pos_cut).
-__device__ __forceinline__ bool kept_by_cut(unsigned bits, int e, unsigned tau, int pos_cut) {
-  return bits > tau || (bits == tau && e <= pos_cut);
-}
-
-// One range of slice y (after refine_range of y): its kept listed tokens, counted from
-// its on-chip probabilities and stored at its slot; then it arrives at the slice's count
-// counter.
-template <bool BLK>
-__device__ void count_segment(const StepParams& P, SelScalars& sc, const Ranges<BLK>& R, int y, int l0, int l1) {
-  const Unit un = unit_of(P, y);
-  const PiSeg ps = pi_seg<BLK>(R, y, un.s);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int L = sc.L;
-  const unsigned tau = sc.tau;
-  const int pos_cut = sc.pos_cut;
-  const SinkWindow sw(L, P.n_sink, P.window);
-  int e0, e1;
-  seg_elems<BLK>(L, l0, l1, e0, e1);
-  constexpr int kPer = BLK ? 1 : 4;
-  int cnt = 0;
-  for (int k0 = e0; k0 < e1; k0 += kSelThreads * kPer) {
-    const int eb = k0 + (BLK ? tid : 128 * warp + 4 * lane);
-    if (eb >= e1) continue;
-    if (BLK) {
-      if (kept_by_cut(__float_as_uint(pi_load(P, ps, eb)), eb, tau, pos_cut)) cnt += listed_of<BLK>(sw, L, eb);
-    } else {
-      const float4 v = pi_load4(P, ps, eb);
-      const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int j = eb + q;
-        if (j < e1 && !sw.always(j) && kept_by_cut(__float_as_uint(vv[q]), j, tau, pos_cut)) ++cnt;
-      }
-    }
-  }
-  const int total = block_sum(cnt, sc.shi);
-  if (tid == 0) P.ws.seg_cnt[stats_slot(blockIdx.x, y)] = total;
-}
-
-// This range's offset in slice y's list: the kept counts of the slice's ranges before it
-// (after every range has stored its count).  The slice's first CTA stores the total.
-template <bool BLK>
-__device__ void offset_segment(const StepParams& P, SelScalars& sc, const Ranges<BLK>& R, int y) {
-  const Unit un = unit_of(P, y);
-  const int tid = threadIdx.x;
-  const int first = R.first_cta(y), n_seg = R.last_cta(y) - first + 1, mine = (int)blockIdx.x - first;
-  const int* cnt_row = P.ws.seg_cnt + stats_slot(first, y);
-  constexpr int kSegPer = kMaxSelectGrid / kSelThreads;
-  int cv[kSegPer];
-  int loc = 0;
-#pragma unroll
-  for (int k = 0; k < kSegPer; ++k) {
-    const int c = tid * kSegPer + k;
-    cv[k] = c < n_seg ? __ldcg(cnt_row + c) : 0;
-    loc += cv[k];
-  }
-  int total = 0;
-  int run = block_excl_scan(loc, sc.shi, &total);
-#pragma unroll
-  for (int k = 0; k < kSegPer; ++k) {
-    const int c = tid * kSegPer + k;
-    if (c == mine) sc.off = run;
-    run += cv[k];
-  }
-  if (tid == 0 && mine == 0) {
-    P.ws.st[un.s].count = total;
-    if (P.sel_count) P.sel_count[un.s] = total;
   }
   __syncthreads();
 }
 
 // ------------------------------------------------------------------ compact phase
-// One range of slice y (after offset_segment of y): its kept positions outside
+// One range of slice y (after refine_range of y): its kept positions outside
 // sinks/window, ascending, written at the range's offset in the slice's list.  Rounds of 1024 tokens: lane l of warp w
 // takes tokens 4 l .. 4 l + 3 of the warp's 128 (one 16-byte read of their
 // probabilities in token mode), a warp scan orders the lanes and the eight warp totals
@@ -1369,15 +1465,7 @@ __device__ void compact_segment(const StepParams& P, SelScalars& sc, const Range
   const Unit un = unit_of(P, y);
   const PiSeg ps = pi_seg<BLK>(R, y, un.s);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  __syncthreads();   // earlier readers of the scalars are done
-  if (tid == 0) {
-    const SliceState* st = P.ws.st + un.s;
-    sc.L = load_len(P.seq_lens, un.b, P.Lcap, P.ws.dev_err);
-    sc.tau = __ldcg(&st->tau_bits);
-    sc.pos_cut = __ldcg(&st->pos_cut);
-  }
-  __syncthreads();
-  const int L = sc.L;   // sc.off from offset_segment of this slice
+  const int L = sc.L;   // sc.L, sc.tau, sc.pos_cut and sc.off from refine_range of this slice
   const unsigned tau = sc.tau;
   const int pos_cut = sc.pos_cut;
   const SinkWindow sw(L, P.n_sink, P.window);
@@ -1462,7 +1550,7 @@ __global__ void __launch_bounds__(kSelThreads, 4) k_select(StepParams P) {
     SliceState* st = P.ws.st + unit_of(P, y).s;
     ok = slice_wait(&st->arr_mass, n_ranges(y), P.ws.dev_err, &sc.ok);
     if (!ok) return;
-    cut1_range(P, sm.stage, sc, y, (int)blockIdx.x == R.first_cta(y));
+    cut1_range(P, sc, y, (int)blockIdx.x == R.first_cta(y));
     threshold_segment<BLK>(P, sc, sm.ref, R, y, l0, l1);
     slice_arrive(&st->arr_thr);
   });
@@ -1472,16 +1560,7 @@ __global__ void __launch_bounds__(kSelThreads, 4) k_select(StepParams P) {
     SliceState* st = P.ws.st + unit_of(P, y).s;
     ok = slice_wait(&st->arr_thr, n_ranges(y), P.ws.dev_err, &sc.ok);
     if (!ok) return;
-    refine_range<BLK>(P, sm.ref, sc, y, (int)blockIdx.x == R.first_cta(y));
-    count_segment<BLK>(P, sc, R, y, l0, l1);
-    slice_arrive(&st->arr_cnt);
-  });
-  if (!ok) return;
-  for_each_segment(R, [&](int y, int l0, int l1) {
-    if (!ok) return;
-    ok = slice_wait(&P.ws.st[unit_of(P, y).s].arr_cnt, n_ranges(y), P.ws.dev_err, &sc.ok);
-    if (!ok) return;
-    offset_segment<BLK>(P, sc, R, y);
+    refine_range<BLK>(P, sm.ref, sc, R, y, l0, l1, (int)blockIdx.x == R.first_cta(y));
     compact_segment<BLK>(P, sc, R, y, l0, l1);
   });
 }
@@ -1516,16 +1595,25 @@ int resident_tg() {
 
 }  // namespace
 
-// Grid of the selection launch: every resident CTA (the same count on every SM, so the
-// range-partitioned phases are balanced per SM), but never more CTAs than range quanta
-// (16-token groups, or kBlock-token blocks in block mode), so no CTA has an empty range.
+// Grid of the selection launch: as many resident CTAs as give every retrieval slice the
+// same whole number of CTAs (all of them when the slices do not divide the resident
+// count), but never more CTAs than range quanta (16-token groups, or kBlock-token blocks
+// in block mode), so no CTA has an empty range.
 int select_grid(const StepParams& P, int max_resident) {
   if (max_resident > kMaxSelectGrid) max_resident = kMaxSelectGrid;
   if (P.n_ret <= 0) return P.n_slices < max_resident ? P.n_slices : max_resident;
   const long long qt = P.blocks ? kBlock : 16;
-  const long long groups = (long long)P.B * P.n_ret * (((long long)P.Lcap + qt - 1) / qt);
+  const long long n_rs = (long long)P.B * P.n_ret, per_slice = ((long long)P.Lcap + qt - 1) / qt;
+  // a whole number of CTAs per retrieval slice when there are at least as many CTAs as
+  // slices: every range then lies inside one slice (the range split places the
+  // boundaries of equal shares there), so no CTA serves two slices' phases
+  if (n_rs <= max_resident) {
+    long long cps = max_resident / n_rs;
+    if (cps > per_slice) cps = per_slice;
+    return (int)(n_rs * cps);
+  }
   long long want = max_resident;
-  if (want > groups) want = groups;
+  if (want > n_rs * per_slice) want = n_rs * per_slice;
   if (want < 1) want = 1;
   return (int)want;
 }

@@ -32,7 +32,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
-  size_t off[20];
+  size_t off[18];
   size_t total;
   int64_t max_items;
   int n_chunks_max;
@@ -48,7 +48,7 @@ Layout plan(const spa_config& c, int split_rows) {
   L.max_items = (int64_t)slices * ((Lmax + split_rows - 1) / split_rows);
   const int64_t part_slots = L.max_items > (int64_t)(spa::kMaxAttendCtas + slices + 1)
                                  ? L.max_items : (int64_t)(spa::kMaxAttendCtas + slices + 1);
-  size_t sz[20] = {
+  size_t sz[18] = {
       (size_t)c.n_q_heads * 16 * 128 * 4,                  // 0 P_q
       (size_t)c.n_kv_heads * 16 * 128 * 4,                 // 1 P_k
       64 * 8,                                              // 2 inv_freq
@@ -58,20 +58,18 @@ Layout plan(const spa_config& c, int split_rows) {
       slices * (size_t)spa::pi_row_stride(Lmax) * 4,       // 6 pi
       slices * spa::kBins1 * 8,                            // 7 hist1
       slices * (size_t)Lmax * 8,                           // 8 cand
-      slices * L.n_chunks_max * 4,                         // 9 chunk_gt
-      slices * L.n_chunks_max * 4,                         // 10 chunk_off
-      slices * sizeof(spa::SliceState),                    // 11 st
-      slices * (size_t)Lmax * 4,                           // 12 list
-      (slices + 1) * 4,                                    // 13 item_base
-      (size_t)part_slots * G * spa::kPartStride * 4,       // 14 split states
-      256,                                                 // 15 dev_err
-      slices * spa::kBins2 * 8,                            // 16 hist2
-      spa::kBarWords * 4,                                  // 17 selection grid barrier
-      slices * 4,                                          // 18 attention tickets
-      (spa::kMaxSelectGrid + slices) * 4,                  // 19 per-range kept counts (selection)
+      slices * L.n_chunks_max * 4,                         // 9 chunk counts (context-parallel)
+      slices * sizeof(spa::SliceState),                    // 10 st
+      slices * (size_t)Lmax * 4,                           // 11 list
+      (slices + 1) * 4,                                    // 12 item_base
+      (size_t)part_slots * G * spa::kPartStride * 4,       // 13 split states
+      256,                                                 // 14 dev_err
+      slices * spa::kBins2 * 8,                            // 15 hist2
+      slices * 4,                                          // 16 attention tickets
+      (spa::kMaxSelectGrid + slices) * 4,                  // 17 per-range counts above the cut bin (selection)
   };
   size_t o = 0;
-  for (int i = 0; i < 20; ++i) {
+  for (int i = 0; i < 18; ++i) {
     L.off[i] = o;
     o += round_up(sz[i], 256);
   }
@@ -505,16 +503,14 @@ spa_status spa_create(spa_handle* out, const spa_config* cfg) {
   w.hist1 = (unsigned long long*)(base + L.off[7]);
   w.cand = (uint2*)(base + L.off[8]);
   w.chunk_gt = (int*)(base + L.off[9]);
-  w.chunk_off = (int*)(base + L.off[10]);
-  w.st = (spa::SliceState*)(base + L.off[11]);
-  w.list = (int*)(base + L.off[12]);
-  w.item_base = (int*)(base + L.off[13]);
-  w.part = (float*)(base + L.off[14]);
-  w.dev_err = (unsigned*)(base + L.off[15]);
-  w.hist2 = (unsigned long long*)(base + L.off[16]);
-  w.bar = (unsigned*)(base + L.off[17]);
-  w.attn_ticket = (unsigned*)(base + L.off[18]);
-  w.seg_cnt = (int*)(base + L.off[19]);
+  w.st = (spa::SliceState*)(base + L.off[10]);
+  w.list = (int*)(base + L.off[11]);
+  w.item_base = (int*)(base + L.off[12]);
+  w.part = (float*)(base + L.off[13]);
+  w.dev_err = (unsigned*)(base + L.off[14]);
+  w.hist2 = (unsigned long long*)(base + L.off[15]);
+  w.attn_ticket = (unsigned*)(base + L.off[16]);
+  w.seg_cnt = (int*)(base + L.off[17]);
   w.max_items = L.max_items;
   h->n_chunks_max = L.n_chunks_max;
 
@@ -526,8 +522,8 @@ spa_status spa_create(spa_handle* out, const spa_config* cfg) {
   if ((e = cudaMemcpy(w.P_q, cfg->P_q, pq, cudaMemcpyDeviceToDevice)) != cudaSuccess ||
       (e = cudaMemcpy(w.P_k, cfg->P_k, pk, cudaMemcpyDeviceToDevice)) != cudaSuccess ||
       (e = cudaMemcpy(w.inv_freq, invf, sizeof invf, cudaMemcpyHostToDevice)) != cudaSuccess ||
-      (e = cudaMemset(w.dev_err, 0, 4)) != cudaSuccess || (e = cudaMemset(w.bar, 0, spa::kBarWords * 4)) != cudaSuccess ||
-      (e = cudaMemset(w.st, 0, L.off[12] - L.off[11])) != cudaSuccess ||
+      (e = cudaMemset(w.dev_err, 0, 4)) != cudaSuccess ||
+      (e = cudaMemset(w.st, 0, L.off[11] - L.off[10])) != cudaSuccess ||
       (e = cudaMemset(w.attn_ticket, 0, (size_t)cfg->max_batch * cfg->n_kv_heads * 4)) != cudaSuccess ||
       (e = cudaDeviceSynchronize()) != cudaSuccess) {
     cudaFree(h->mem);
@@ -860,10 +856,9 @@ spa_status spa_device_status(spa_handle h, spa_stream stream) {
   if (flags) {
     if ((e = cudaMemset(h->ws.dev_err, 0, 4)) != cudaSuccess) return cuda_fail(e, "clear status");
     if (flags & spa::kErrTimeout) {
-      // the grid barrier may have been left mid-way: start the next call from a clean barrier
-      cudaMemset(h->ws.bar, 0, spa::kBarWords * 4);
+      // a wait that gave up may have left arrival counters or attention tickets mid-way:
+      // start the next call from clean ones (the prologue kernel also clears the counters)
       cudaMemset(h->ws.attn_ticket, 0, sizeof(unsigned) * (size_t)h->cfg.max_batch * h->cfg.n_kv_heads);
-      // q_idx flags are tagged with the barrier generation, which restarts at 0
       cudaMemset(h->ws.st, 0, sizeof(spa::SliceState) * (size_t)h->cfg.max_batch * h->cfg.n_kv_heads);
       cudaDeviceSynchronize();
       return fail(SPA_ERR_DEVICE_TIMEOUT, "a bounded device-side wait gave up (flags 0x%x)", flags);

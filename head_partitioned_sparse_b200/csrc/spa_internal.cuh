@@ -47,11 +47,6 @@ constexpr int kDefaultSplitRows = 1024;
 // One split's state per head: acc[128], m, l, 2 floats of padding (16-byte rows).
 constexpr int kPartStride = kHeadDim + 4;
 
-// Words of the selection kernel's synchronisation block, one 128-byte line each:
-// [0] barrier arrivals, [32] barrier generation, [kBarDuty] q_rot duty ticket.
-constexpr int kBarWords = 96;
-constexpr int kBarDuty = 64;
-
 // Device status bits.
 constexpr unsigned kErrSeqLen = 1u;
 constexpr unsigned kErrStartPos = 2u;
@@ -68,11 +63,8 @@ struct __align__(16) SliceState {
   int count;                    // listed tokens (kept, outside sinks/window)
   unsigned arr_score;           // ranges whose score statistics are stored
   unsigned arr_mass;            // ranges whose round-1 masses are added
-  unsigned arr_thr;             // ranges whose candidates are stored
-  unsigned arr_cnt;             // ranges whose kept counts are stored
+  unsigned arr_thr;             // ranges whose candidates and counts above b1 are stored
   unsigned ncand;               // candidates of the round-1 cut bin (slots taken)
-  unsigned tau_bits;            // fp32 bits of the cut value tau
-  int pos_cut;                  // tokens equal to tau are kept iff their position <= pos_cut
 };
 
 // Cut state of one (b, kv head) slice in a context-parallel step (each rank holds a
@@ -139,15 +131,13 @@ struct Workspace {
   unsigned long long* hist2;  // [Bm*Hkv][kBins2] round-2 masses of the round-1 cut bin
   uint2* cand;           // [Bm*Hkv][Lmax]  (prob bits, position)
   int* chunk_gt;         // [Bm*Hkv][n_chunks_max]
-  int* chunk_off;        // [Bm*Hkv][n_chunks_max]
   SliceState* st;        // [Bm*Hkv]
   int* list;             // [Bm*Hkv][Lmax]  selected positions (decode)
   int* item_base;        // [Bm*Hkv + 1]
   unsigned* attn_ticket; // [Bm*Hkv] pieces of each slice finished (bf16 attention; reset by its combiner)
   float* part;           // [max(max_items, kMaxAttendCtas + Bm*Hkv + 1)][G][kPartStride]
-  int* seg_cnt;          // [kMaxSelectGrid + Bm*Hkv] per-range kept (listed) tokens
+  int* seg_cnt;          // [kMaxSelectGrid + Bm*Hkv] per-range listed tokens above the cut bin
   unsigned* dev_err;     // [1]
-  unsigned* bar;         // [kBarWords] selection kernel: grid barrier and q_rot duty ticket
   int64_t max_items;
 };
 
@@ -182,7 +172,7 @@ struct StepParams {
   int n_str;             // streaming heads (Hkv - n_ret)
   int ring;              // ring rows per streaming head: n_sink + window
   int head_rank[kMaxKvHeads];   // rank of head g among the retrieval or the streaming heads
-  int drop_publish;      // failure-detection test hook: selection CTA 0 skips the first grid barrier
+  int drop_publish;      // failure-detection test hook: selection CTA 0 never arrives at its slice's counters
   const void* k_ring;    // [Bm][n_str][ring][128] streaming-head keys (compact layout)
   const void* v_ring;
   float* lse;            // optional [B][Hq]: log2-sum-exp of each head's attended scores

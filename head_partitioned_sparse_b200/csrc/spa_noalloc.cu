@@ -14,13 +14,12 @@
 // is looked up once per device with cudaGetSymbolAddress, with that device current,
 // on the first call made on that device (do that first call before any stream
 // capture).  Every call shares the array and it keeps the last call's contents.  The
-// words that must start at zero on every call (the selection kernel's grid-barrier
-// arrival and generation words, the device status word and the per-slice state with
-// its tickets and query-vector flags) sit at fixed offsets at the head of the array and
-// are cleared with one cudaMemsetAsync on the call's stream before the launch, so a
-// call never inherits a half-counted barrier, whatever the shapes of earlier calls or
-// whether one of their bounded waits gave up; the kernels clear the rest (histograms,
-// counters) themselves.  Calls that overlap on the GPU (other streams, other host
+// words that must start at zero on every call (the device status word and the
+// per-slice state with the selection kernel's arrival counters) sit at fixed offsets
+// at the head of the array and are cleared with one cudaMemsetAsync on the call's
+// stream before the launch, so a call never inherits a half-counted arrival, whatever
+// the shapes of earlier calls or whether one of their bounded waits gave up; the
+// kernels clear the rest (histograms, counters) themselves.  Calls that overlap on the GPU (other streams, other host
 // threads) race on the array: serialise them.
 #include <cmath>
 #include <cstring>
@@ -134,9 +133,9 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
   spa_status r = scratch_on_current_device(&base_v);
   if (r) return r;
   char* base = static_cast<char*>(base_v);
-  // Fixed head block, cleared before every launch: barrier words, status word, the
-  // per-slice state of up to kMaxSlices slices.
-  const size_t off_bar = 0, off_err = up256(spa::kBarWords * 4), off_st = off_err + 256;
+  // Fixed head block, cleared before every launch: the status word and the per-slice
+  // state (arrival counters included) of up to kMaxSlices slices.
+  const size_t off_err = 0, off_st = 256;
   const size_t head_bytes = up256(off_st + (size_t)kMaxSlices * sizeof(spa::SliceState));
   const size_t sz[] = {
       64 * 8,                                                  // inv_freq (unused by selection; zero)
@@ -146,10 +145,8 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
       (size_t)slices * spa::pi_row_stride(max_ctx) * 4,        // pi
       (size_t)slices * spa::kBins1 * 8,                        // hist1
       (size_t)slices * max_ctx * 8,                            // candidates
-      (size_t)slices * P.n_chunks * 4,                         // chunk_gt
-      (size_t)slices * P.n_chunks * 4,                         // chunk_off
       (size_t)slices * spa::kBins2 * 8,                        // hist2
-      (size_t)(spa::kMaxSelectGrid + slices) * 4,              // per-range kept counts
+      (size_t)(spa::kMaxSelectGrid + slices) * 4,              // per-range counts above the cut bin
   };
   size_t off[sizeof sz / sizeof sz[0]];
   size_t o = head_bytes;
@@ -168,11 +165,8 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
   w.pi_stride = spa::pi_row_stride(max_ctx);
   w.hist1 = (unsigned long long*)(base + off[5]);
   w.cand = (uint2*)(base + off[6]);
-  w.chunk_gt = (int*)(base + off[7]);
-  w.chunk_off = (int*)(base + off[8]);
-  w.hist2 = (unsigned long long*)(base + off[9]);
-  w.seg_cnt = (int*)(base + off[10]);
-  w.bar = (unsigned*)(base + off_bar);
+  w.hist2 = (unsigned long long*)(base + off[7]);
+  w.seg_cnt = (int*)(base + off[8]);
   w.dev_err = (unsigned*)(base + off_err);
   w.st = (spa::SliceState*)(base + off_st);
 

@@ -404,9 +404,9 @@ SPA_API spa_status spa_head_effective_ranks(const float* W_Q, const float* W_K, 
 SPA_API spa_status spa_device_status(spa_handle h, spa_stream stream);
 
 /* Failure-detection test hook (no fault, no hang): while enabled, the first CTA of the
- * selection kernel leaves before its first grid barrier, so every other CTA waits at
- * that barrier for an arrival that never comes until its bounded wait (about 2 s)
- * gives up; the call completes with meaningless lists and spa_device_status reports
+ * selection kernel leaves before its first arrival at its slice's counter, so every
+ * other CTA of that slice waits for an arrival that never comes until its bounded wait
+ * (about 2 s) gives up; the call completes with meaningless lists and spa_device_status reports
  * SPA_ERR_DEVICE_TIMEOUT (and resets the synchronisation state, so the next call on the
  * handle is sound).  Off by default; for tests only. */
 SPA_API spa_status spa_debug_drop_publish(spa_handle h, int enable);
@@ -459,7 +459,7 @@ SPA_API spa_status spa_launch_count(spa_handle h, int64_t* launches);
  * call overwrites it, so calls that overlap on the GPU race: serialise them.
  * Before each launch the call clears, with one cudaMemsetAsync on `stream` (which
  * allocates nothing), the fixed block at the head of the array that holds the
- * selection kernel's grid-barrier words, its status word and the per-slice state,
+ * status word and the per-slice state (the selection kernel's arrival counters),
  * so no call inherits synchronisation state from an earlier one of another shape.
  * Device-side conditions are not reported by this entry point (there is no handle
  * to hold a status word): out-of-range seq_lens values are clamped, and a bounded
