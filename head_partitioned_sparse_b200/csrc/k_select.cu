@@ -308,7 +308,7 @@ __device__ bool slice_wait(unsigned* ctr, unsigned n, unsigned* err, int* s_ok) 
 // ------------------------------------------------------------------ shared memory
 constexpr int kWarps = kSelThreads / 32;
 constexpr int kGroupBatch = 4;    // groups per warp loaded together (8 spills at 64 registers)
-constexpr int kPiCap = 4096;      // probabilities of a range kept on chip (dynamic shared memory)
+constexpr int kPiCap = 16 * kSelThreads;   // probabilities of a range kept on chip (dynamic shared memory)
 constexpr int kPiBytes = kPiCap * 4;
 constexpr int kSmallList = 2048;  // candidates of the round-A cut digit kept on chip by the refine step
 constexpr int kTieCap = 256;      // candidates equal to the cut value ranked directly
@@ -688,9 +688,10 @@ __device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc
 
 // ------------------------------------------------------------------ cut 1 (per range)
 // Every CTA of a slice takes the slice's round-1 cut itself from the complete round-1
-// histogram (32 KB, read from L2): thread t loads the 16 consecutive bins 4095 - 16 t - k
-// (k = 0..15, descending), a warp scan and a scan of the 8 warp totals give the mass ahead
-// of each thread's bins, and the thread whose bins hold the crossing walks them: the
+// histogram (32 KB, read from L2): thread t loads the kPer = 4096 / threads consecutive
+// bins 4095 - kPer t - k (k = 0..kPer-1, descending), a warp scan and a scan of the warp
+// totals give the mass ahead of each thread's bins, and the thread whose bins hold the
+// crossing walks them: the
 // total mass, the target ceil(p * total) (or k for top-k) and the bin b1 where the
 // descending cumulative mass reaches it (-1: keep every token).  Results in sc.b1,
 // sc.target, sc.m_above (the mass of all bins above b1) and sc.L (the sequence length,
@@ -699,14 +700,15 @@ __device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc
 __device__ void cut1_range(const StepParams& P, SelScalars& sc, int y, bool lead) {
   const Unit un = unit_of(P, y);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const ulonglong2* h = reinterpret_cast<const ulonglong2*>(P.ws.hist1 + (size_t)un.s * kBins1 + kBins1 - 16 * (tid + 1));
-  ulonglong2 hv[8];
+  constexpr int kPer = kBins1 / kSelThreads, kVec = kPer / 2;   // bins per thread, 16-byte words
+  const ulonglong2* h = reinterpret_cast<const ulonglong2*>(P.ws.hist1 + (size_t)un.s * kBins1 + kBins1 - kPer * (tid + 1));
+  ulonglong2 hv[kVec];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) hv[k] = __ldcg(h + k);   // bins 4080 - 16 t .. 4095 - 16 t, ascending
+  for (int k = 0; k < kVec; ++k) hv[k] = __ldcg(h + k);   // bins 4096 - kPer (t + 1) .. 4095 - kPer t, ascending
   if (tid == 0) sc.L = load_len(P.seq_lens, un.b, P.Lcap, P.ws.dev_err);
   unsigned long long mine = 0ull;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) mine += hv[k].x + hv[k].y;
+  for (int k = 0; k < kVec; ++k) mine += hv[k].x + hv[k].y;
   unsigned long long x = mine;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -735,12 +737,12 @@ __device__ void cut1_range(const StepParams& P, SelScalars& sc, int y, bool lead
     unsigned long long cum = wbase + x - mine;   // mass of the bins above this thread's
     if (cum < target && cum + mine >= target) {
 #pragma unroll
-      for (int k = 7; k >= 0; --k) {
+      for (int k = kVec - 1; k >= 0; --k) {
         const unsigned long long b[2] = {hv[k].y, hv[k].x};   // descending: bin 2k + 1, then 2k
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           if (cum < target && cum + b[e] >= target) {
-            sc.cut_bin = kBins1 - 16 * (tid + 1) + 2 * k + 1 - e;
+            sc.cut_bin = kBins1 - kPer * (tid + 1) + 2 * k + 1 - e;
             sc.cut_above = cum;
           }
           cum += b[e];
@@ -1192,7 +1194,7 @@ __device__ void refine_range(const StepParams& P, SmemRefine& sm, SelScalars& sc
   const int* abv_row = P.ws.seg_cnt + stats_slot(first, y);
   constexpr int kSegPer = kMaxSelectGrid / kSelThreads;
   // one round trip: the cut state, the ranges' counts above b1, the round-A histogram
-  // (4 words per thread) and the first kRefBatch candidates per thread (read up to the
+  // (1024 words over the CTA) and the first kRefBatch candidates per thread (read up to the
   // row's capacity, used below n)
   const unsigned long long target = __ldcg(&st->target);
   const unsigned long long mab = __ldcg(&st->m_above);
@@ -1207,9 +1209,10 @@ __device__ void refine_range(const StepParams& P, SmemRefine& sm, SelScalars& sc
     const int c = tid + kSelThreads * k;
     av[k] = c < n_seg ? __ldcg(abv_row + c) : 0;
   }
-  unsigned hav[4];
+  constexpr int kHaPer = 1024 / kSelThreads;
+  unsigned hav[kHaPer];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) hav[k] = __ldcg(ha + tid + kSelThreads * k);
+  for (int k = 0; k < kHaPer; ++k) hav[k] = __ldcg(ha + tid + kSelThreads * k);
   uint2 c0[kRefBatch];
 #pragma unroll
   for (int u = 0; u < kRefBatch; ++u) {
@@ -1235,7 +1238,7 @@ __device__ void refine_range(const StepParams& P, SmemRefine& sm, SelScalars& sc
     }
   }
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {   // words 0..511 counts, 512..1023 low sums
+  for (int k = 0; k < kHaPer; ++k) {   // words 0..511 counts, 512..1023 low sums
     const int w = tid + kSelThreads * k;
     if (w < 512) sm.hc[w] = hav[k]; else sm.hl[w - 512] = hav[k];
   }
@@ -1458,7 +1461,7 @@ __device__ void refine_range(const StepParams& P, SmemRefine& sm, SelScalars& sc
 // One range of slice y (after refine_range of y): its kept positions outside
 // sinks/window, ascending, written at the range's offset in the slice's list.  Rounds of 1024 tokens: lane l of warp w
 // takes tokens 4 l .. 4 l + 3 of the warp's 128 (one 16-byte read of their
-// probabilities in token mode), a warp scan orders the lanes and the eight warp totals
+// probabilities in token mode), a warp scan orders the lanes and the warp totals
 // order the warps.
 template <bool BLK>
 __device__ void compact_segment(const StepParams& P, SelScalars& sc, const Ranges<BLK>& R, int y, int l0, int l1) {
@@ -1525,7 +1528,7 @@ __device__ void compact_segment(const StepParams& P, SelScalars& sc, const Range
 
 // ------------------------------------------------------------------ the kernel
 template <typename T, int G, bool BLK>
-__global__ void __launch_bounds__(kSelThreads, 4) k_select(StepParams P) {
+__global__ void __launch_bounds__(kSelThreads, 1024 / kSelThreads) k_select(StepParams P) {
   __shared__ SelSmem sm;
   __shared__ SelScalars sc;
   const Ranges<BLK> R(P);

@@ -16,8 +16,7 @@ constexpr int64_t kMaxCtx = int64_t(1) << 24;
 
 // Selection works on chunks of kChunk consecutive tokens of one (b, kv head) slice.
 constexpr int kChunk = 4096;
-constexpr int kSelThreads = 256;
-constexpr int kTokPerThread = kChunk / kSelThreads;  // 16
+constexpr int kSelThreads = 512;   // threads of a selection CTA (2 CTAs per SM)
 constexpr int kMaxChunks = int(kMaxCtx / kChunk);    // 4096
 // Block-granular selection ranks blocks of kBlock consecutive positions of a slice.
 constexpr int kBlock = 64;
