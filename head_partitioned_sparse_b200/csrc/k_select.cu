@@ -139,9 +139,10 @@ __device__ __forceinline__ int lane_head(int t4, int nh) { return G <= 4 ? t4 : 
 
 
 // The lane's B fragments of the group's query index vectors (qsm, G * 16 floats in
-// shared memory).
+// shared memory), each scaled by `scale` (log2(e) * idx_scale) in float32 before the
+// split, so the tensor cores return log2-domain logits directly.
 template <int G>
-__device__ __forceinline__ void qidx_frag(const float* qbase, uint32_t (&qb)[IdxTiles<G>::NT][2]) {
+__device__ __forceinline__ void qidx_frag(const float* qbase, float scale, uint32_t (&qb)[IdxTiles<G>::NT][2]) {
   const int lane = threadIdx.x & 31, gid = lane >> 2, t4 = lane & 3;
 #pragma unroll
   for (int t = 0; t < IdxTiles<G>::NT; ++t) {
@@ -158,7 +159,7 @@ __device__ __forceinline__ void qidx_frag(const float* qbase, uint32_t (&qb)[Idx
     if (part >= 0) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float x = qbase[head * kIdxDim + 4 * t4 + e];
+        const float x = qbase[head * kIdxDim + 4 * t4 + e] * scale;
         const float hi = __bfloat162float(__float2bfloat16_rn(x));
         const float mid = __bfloat162float(__float2bfloat16_rn(x - hi));
         const float lo = __bfloat162float(__float2bfloat16_rn((x - hi) - mid));
@@ -170,21 +171,11 @@ __device__ __forceinline__ void qidx_frag(const float* qbase, uint32_t (&qb)[Idx
   }
 }
 
-// Stages the group's query index vectors (written by an earlier phase, read through L2)
-// in shared memory and builds the fragments.  Called by every thread of the CTA.
-template <int G>
-__device__ __forceinline__ void load_qidx_frag(const StepParams& P, int b, int g, float* qsm,
-                                               uint32_t (&qb)[IdxTiles<G>::NT][2]) {
-  if (threadIdx.x < G * kIdxDim)
-    qsm[threadIdx.x] = __ldcg(&P.ws.q_idx[((size_t)b * P.Hq + (size_t)g * G) * kIdxDim + threadIdx.x]);
-  __syncthreads();
-  qidx_frag<G>(qsm, qb);
-}
-
-// Log2-domain logits of tokens gid (ra) and gid + 8 (rb) for the lane's heads.
+// Log2-domain logits of tokens gid (ra) and gid + 8 (rb) for the lane's heads (the
+// scale is in the fragments).
 template <int G>
 __device__ __forceinline__ void group_logits(const uint2& ra, const uint2& rb,
-                                             const uint32_t (&qb)[IdxTiles<G>::NT][2], float scale,
+                                             const uint32_t (&qb)[IdxTiles<G>::NT][2],
                                              float (&lg)[IdxTiles<G>::NH][2]) {
   const uint32_t a[4] = {ra.x, rb.x, ra.y, rb.y};
   float c[IdxTiles<G>::NT][4];
@@ -194,13 +185,13 @@ __device__ __forceinline__ void group_logits(const uint2& ra, const uint2& rb,
     mma16816(c[t], a, qb[t][0], qb[t][1]);
   }
   if (G <= 4) {
-    lg[0][0] = ((c[0][0] + c[0][1]) + c[1][0]) * scale;
-    lg[0][1] = ((c[0][2] + c[0][3]) + c[1][2]) * scale;
+    lg[0][0] = (c[0][0] + c[0][1]) + c[1][0];
+    lg[0][1] = (c[0][2] + c[0][3]) + c[1][2];
   } else {
-    lg[0][0] = ((c[0][0] + c[0][1]) + c[IdxTiles<G>::NT - 1][0]) * scale;
-    lg[0][1] = ((c[0][2] + c[0][3]) + c[IdxTiles<G>::NT - 1][2]) * scale;
-    lg[IdxTiles<G>::NH - 1][0] = ((c[1][0] + c[1][1]) + c[IdxTiles<G>::NT - 1][1]) * scale;
-    lg[IdxTiles<G>::NH - 1][1] = ((c[1][2] + c[1][3]) + c[IdxTiles<G>::NT - 1][3]) * scale;
+    lg[0][0] = (c[0][0] + c[0][1]) + c[IdxTiles<G>::NT - 1][0];
+    lg[0][1] = (c[0][2] + c[0][3]) + c[IdxTiles<G>::NT - 1][2];
+    lg[IdxTiles<G>::NH - 1][0] = (c[1][0] + c[1][1]) + c[IdxTiles<G>::NT - 1][1];
+    lg[IdxTiles<G>::NH - 1][1] = (c[1][2] + c[1][3]) + c[IdxTiles<G>::NT - 1][3];
   }
 }
 
@@ -316,7 +307,7 @@ constexpr int kRefBatch = 8;      // candidate loads per thread issued together 
 
 struct SmemPro { double cs[kHeadDim / 2], sn[kHeadDim / 2]; };
 struct SmemScore { float2 red[kSelThreads / 32][kMaxGroup]; };
-struct SmemMass { unsigned cnt[kBins1], low[kBins1]; float Mh[kMaxGroup], Wh[kMaxGroup]; };
+struct SmemMass { unsigned cnt[kBins1], low[kBins1]; float Mh[kMaxGroup]; };
 struct SmemRefine {
   uint2 small[kSmallList];            // candidates of the round-A cut digit (bits, element)
   unsigned hc[512];                   // radix round: count per digit
@@ -641,8 +632,7 @@ __device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc
     return;
   }
   uint32_t qb[IdxTiles<G>::NT][2];
-  qidx_frag<G>(sc.qsm, qb);
-  const float scale = P.idx_scale_log2;
+  qidx_frag<G>(sc.qsm, P.idx_scale_log2, qb);
   const int jend = min(L, 16 * l1);
   // two independent online accumulators per head (tokens gid and gid + 8)
   float m[NH][2], z[NH][2];
@@ -653,7 +643,7 @@ __device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc
     for (int u = 0; u < U; ++u) {
       const int j = 16 * (gb + warp + kWarps * u);
       float lg[NH][2];
-      group_logits<G>(ra[u], rb[u], qb, scale, lg);
+      group_logits<G>(ra[u], rb[u], qb, lg);
       // refill the consumed slot with the same slot of the next batch
       load_group(rows, 16 * (gb + kWarps * U + warp + kWarps * u), jend, pol, ra[u], rb[u]);
 
@@ -768,7 +758,8 @@ __device__ void cut1_range(const StepParams& P, SelScalars& sc, int y, bool lead
 // ------------------------------------------------------------------ mass phase
 // One range of slice y: M_h, Z_h merged from the slice's range statistics (fixed
 // order), the logits recomputed (index read #2, mostly from L2),
-// pi_j = sum_h 2^(l_hj - M_h) / (G Z_h) kept (PiSeg), and its mass added to the slice's
+// pi_j = sum_h 2^(l_hj - M_h) / (G Z_h), evaluated as sum_h 2^(l_hj - M'_h) with
+// M'_h = M_h + log2(G Z_h), kept (PiSeg), and its mass added to the slice's
 // round-1 histogram via a per-range shared histogram of counts and low significand
 // bits (32-bit atomics; a range holds at most kMaxRangeGroups groups, so a bin's
 // low-bit sum stays below 2^32).
@@ -819,8 +810,7 @@ __device__ bool mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
       merge_mz(m, z, m2, z2);
     }
     if (lane == 0) {
-      sm.Mh[warp] = m;
-      sm.Wh[warp] = 1.f / ((float)G * z);
+      sm.Mh[warp] = m + log2f((float)G * z);
     }
   }
   if (tid < G * kIdxDim) sc.qsm[tid] = qv;
@@ -835,14 +825,12 @@ __device__ bool mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
   const int L = sc.L;
   if (16 * l0 >= L) return true;
   uint32_t qb[IdxTiles<G>::NT][2];
-  qidx_frag<G>(sc.qsm, qb);
-  const float scale = P.idx_scale_log2;
-  float M[NH], W[NH];
+  qidx_frag<G>(sc.qsm, P.idx_scale_log2, qb);
+  float M[NH];
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
     const int head = lane_head<G>(t4, h);
-    M[h] = head < G ? sm.Mh[head] : 0.f;
-    W[h] = head < G ? sm.Wh[head] : 0.f;   // lanes of absent heads contribute nothing
+    M[h] = head < G ? sm.Mh[head] : INFINITY;   // lanes of absent heads contribute nothing
   }
   const int jend = min(L, 16 * l1);
   for (int gb = l0; 16 * gb < jend; gb += kWarps * U) {
@@ -851,7 +839,7 @@ __device__ bool mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
     for (int u = 0; u < U; ++u) {
       const int j = 16 * grp(gb, u);
       float lg[NH][2];
-      group_logits<G>(ra[u], rb[u], qb, scale, lg);
+      group_logits<G>(ra[u], rb[u], qb, lg);
       // refill the consumed slot with the same slot of the next batch
       load_group(rows, 16 * grp(gb + kWarps * U, u), jend, pol, ra[u], rb[u]);
 
@@ -863,8 +851,8 @@ __device__ bool mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
         float acc = 0.f;
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
-          if (G < 4 && W[h] == 0.f) continue;   // lanes of absent heads (G < 4) add nothing
-          acc += ex2(lg[h][cc] - M[h]) * W[h];
+          if (G < 4 && M[h] == INFINITY) continue;   // lanes of absent heads (G < 4) add nothing
+          acc += ex2(lg[h][cc] - M[h]);
         }
         pr[cc] = acc;
       }
