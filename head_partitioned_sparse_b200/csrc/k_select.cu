@@ -316,7 +316,7 @@ struct SmemRefine {
   int wcnt[kSelThreads / 32];         // per-warp counts
   int wabv[kSelThreads / 32];         // per-warp counts of listed tokens above the cut bin
 };
-union SelSmem {
+union SelSmem {   // (compact_segment stages kThrRun * kSelThreads ints here)
   SmemPro pro;
   SmemScore score;
   SmemMass mass;
@@ -978,102 +978,78 @@ __device__ __forceinline__ void seg_elems(int L, int l0, int l1, int& e0, int& e
 
 // One range of slice y (after cut1_range of y): the elements of bin b1 are the slice's
 // candidates; the listed tokens of the elements above b1 (every element when b1 < 0) are
-// kept whatever the exact cut, and their count is stored at the range's slot.  Two passes
-// over the range's probabilities (on chip): the first counts both per warp, one atomic per
-// CTA reserves the candidates' slots in the slice's candidate array, the second writes
-// them (bits, element) in range order and adds them to the slice's round-A histogram
-// (bits 17..9: count and sum of bits 8..0).  Token mode: lane l of warp w reads elements
-// 4 l .. 4 l + 3 of the warp's 128 as one 16-byte load.
+// kept whatever the exact cut, and their count is stored at the range's slot.  Rounds
+// of kThrRun consecutive elements per thread (token mode; one block per thread in block
+// mode), held in registers: one CTA scan gives each thread's candidate offset and the
+// round's totals, one atomic per round reserves the candidates' slots in the slice's
+// candidate array, and the candidates (bits, element) are written in range order and
+// added to the slice's round-A histogram (bits 17..9: count and sum of bits 8..0).
+constexpr int kThrRun = 16;
 template <bool BLK>
 __device__ void threshold_segment(const StepParams& P, SelScalars& sc, SmemRefine& sm, const Ranges<BLK>& R, int y,
                                   int l0, int l1) {
+  (void)sm;
   const Unit un = unit_of(P, y);
   const PiSeg ps = pi_seg<BLK>(R, y, un.s);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int L = sc.L, b1 = sc.b1;   // from cut1_range (b1 < 0: keep everything)
   const SinkWindow sw(L, P.n_sink, P.window);
   int e0, e1;
   seg_elems<BLK>(L, l0, l1, e0, e1);
-  constexpr int kPer = BLK ? 1 : 4;
-  // candidate mask of the thread's elements of round k0 (their bits in bits[]); the
-  // listed tokens of its elements above b1 are added to *above
-  auto cand_mask = [&](int k0, unsigned (&bits)[kPer], int* above) {
-    const int eb = k0 + (BLK ? tid : 128 * warp + 4 * lane);
-    unsigned m = 0u;
-    if (BLK) {
-      bits[0] = eb < e1 ? __float_as_uint(pi_load(P, ps, eb)) : 0u;
-    } else if (eb < e1) {
-      const float4 v = pi_load4(P, ps, eb);
-      bits[0] = __float_as_uint(v.x);
-      bits[1] = __float_as_uint(v.y);
-      bits[2] = __float_as_uint(v.z);
-      bits[3] = __float_as_uint(v.w);
-    }
-#pragma unroll
-    for (int q = 0; q < kPer; ++q) {
-      if (eb + q < e1) {
-        const int bin = (int)min(bits[q] >> 18, (unsigned)(kBins1 - 1));
-        if (bin == b1) m |= 1u << q;
-        if (above && bin > b1) *above += listed_of<BLK>(sw, L, eb + q);
-      }
-    }
-    return m;
-  };
-  int wc = 0;      // this warp's candidates (every lane holds the warp's sum)
-  int above = 0;   // this thread's listed tokens above b1
-  for (int k0 = e0; k0 < e1; k0 += kSelThreads * kPer) {
-    unsigned bits[kPer];
-    int c = __popc(cand_mask(k0, bits, &above));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(kFull, c, o);
-    wc += c;
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(kFull, above, o);
-  if (lane == 0) {
-    sm.wcnt[warp] = wc;
-    sm.wabv[warp] = above;
-  }
-  __syncthreads();
-  unsigned total = 0u;
-  int wbase = 0, above_all = 0;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
-    total += (unsigned)sm.wcnt[w];
-    wbase += w < warp ? sm.wcnt[w] : 0;
-    above_all += sm.wabv[w];
-  }
-  if (tid == 0) P.ws.seg_cnt[stats_slot(blockIdx.x, y)] = above_all;
-  if (total == 0u) return;
-  if (tid == 0) sc.cbase = atomicAdd(&P.ws.st[un.s].ncand, total);
-  __syncthreads();
+  constexpr int kPer = BLK ? 1 : kThrRun;
   uint2* cand = P.ws.cand + (size_t)un.s * P.Lmax;
   unsigned* ha = hist_a(P, un.s);
-  unsigned slot = sc.cbase + (unsigned)wbase;
-  for (int k0 = e0; k0 < e1; k0 += kSelThreads * kPer) {
+  int above_all = 0;
+  for (int k0 = e0; k0 < e1; k0 += kSelThreads * kPer) {   // whole CTA: the scan below
+    const int eb = k0 + kPer * tid;
     unsigned bits[kPer];
-    const unsigned m = cand_mask(k0, bits, nullptr);
-    const int eb = k0 + (BLK ? tid : 128 * warp + 4 * lane);
-    // lanes in order, each lane's elements in order
-    const int c = __popc(m);
-    int x = c;
+    unsigned cmask = 0u;
+    int above = 0;
+    if (eb < e1) {
+      if (BLK) {
+        bits[0] = __float_as_uint(pi_load(P, ps, eb));
+      } else {
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(kFull, x, o);
-      if (lane >= o) x += t;
+        for (int q4 = 0; q4 < kPer / 4; ++q4) {   // eb is a multiple of 16: aligned 16-byte words
+          const float4 v = pi_load4(P, ps, eb + 4 * q4);
+          bits[4 * q4] = __float_as_uint(v.x);
+          bits[4 * q4 + 1] = __float_as_uint(v.y);
+          bits[4 * q4 + 2] = __float_as_uint(v.z);
+          bits[4 * q4 + 3] = __float_as_uint(v.w);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < kPer; ++q) {
+        if (eb + q < e1) {
+          const int bin = (int)min(bits[q] >> 18, (unsigned)(kBins1 - 1));
+          if (bin == b1) cmask |= 1u << q;
+          if (bin > b1) above += listed_of<BLK>(sw, L, eb + q);
+        }
+      }
     }
-    unsigned k = slot + (unsigned)(x - c);
+    // candidates before this thread (low half) and the round's totals (candidates low,
+    // listed tokens above b1 high)
+    unsigned long long tot;
+    const unsigned long long pre =
+        block_excl_scan<unsigned long long>(((unsigned long long)above << 32) | (unsigned)__popc(cmask), sc.shl, &tot);
+    above_all += (int)(tot >> 32);
+    const unsigned n_round = (unsigned)tot;
+    if (n_round == 0u) continue;   // uniform: the totals are the CTA's
+    if (tid == 0) sc.cbase = atomicAdd(&P.ws.st[un.s].ncand, n_round);
+    __syncthreads();
+    unsigned slot = sc.cbase + (unsigned)pre;
 #pragma unroll
     for (int q = 0; q < kPer; ++q) {
-      if (m >> q & 1u) {
-        cand[k++] = make_uint2(bits[q], (unsigned)(eb + q));
+      if (cmask >> q & 1u) {
+        cand[slot++] = make_uint2(bits[q], (unsigned)(eb + q));
         const unsigned d = (bits[q] >> 9) & 511u;
         atomicAdd(ha + d, 1u);
         atomicAdd(ha + 512 + d, bits[q] & 511u);
       }
     }
-    slot += (unsigned)__shfl_sync(kFull, x, 31);
+    __syncthreads();   // sc.cbase is rewritten by the next round
   }
+  if (tid == 0) P.ws.seg_cnt[stats_slot(blockIdx.x, y)] = above_all;
 }
 
 // ------------------------------------------------------------------ refine (per range)
@@ -1090,35 +1066,34 @@ __device__ __forceinline__ unsigned long long digit_mass(const StepParams& P, in
   return ((unsigned long long)sig * c + l) << (e - kMassMinExp);
 }
 
-// Warp 0: the digit d of [0, 512) (visited from 511 down) where base plus the
-// cumulative mass of the digits above it first reaches target; sc.digit (-1 if never)
-// and sc.above (the mass ahead of d).  sig_of(d) gives the digit's significand bits.
+// The digit d of [0, 512) (visited from 511 down) where base plus the cumulative mass of
+// the digits above it first reaches target; sc.digit (left as it was if never; callers
+// set -1 first) and sc.above (the mass ahead of d).  sig_of(d) gives the digit's
+// significand bits.  Called by every thread of the CTA: thread t takes digits
+// 511 - kDPer t - k, one CTA scan orders them.
 template <class SIG>
 __device__ void digit_cut_desc(const StepParams& P, const SmemRefine& sm, SelScalars& sc, int b1, SIG sig_of,
                                unsigned long long base, unsigned long long target) {
-  const int lane = threadIdx.x & 31;
-  if (threadIdx.x >= 32) return;
-  unsigned long long sum = 0ull;
-  for (int k = 0; k < 16; ++k) {
-    const int d = 511 - 16 * lane - k;
-    sum += digit_mass(P, b1, sig_of(d), sm.hc[d], sm.hl[d]);
-  }
-  unsigned long long x = sum;
+  constexpr int kDPer = 512 / kSelThreads;
+  static_assert(kDPer * kSelThreads == 512, "the CTA covers the 512 digits");
+  const int tid = threadIdx.x;
+  unsigned long long m[kDPer], sum = 0ull;
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned long long t = __shfl_up_sync(kFull, x, o);
-    if (lane >= o) x += t;
+  for (int k = 0; k < kDPer; ++k) {
+    const int d = 511 - kDPer * tid - k;
+    m[k] = digit_mass(P, b1, sig_of(d), sm.hc[d], sm.hl[d]);
+    sum += m[k];
   }
-  unsigned long long cum = base + x - sum;
-  if (cum < target && cum + sum >= target) {   // the crossing is in this lane's digits
-    for (int k = 0; k < 16; ++k) {
-      const int d = 511 - 16 * lane - k;
-      const unsigned long long m = digit_mass(P, b1, sig_of(d), sm.hc[d], sm.hl[d]);
-      if (cum < target && cum + m >= target) {
-        sc.digit = d;
+  unsigned long long tot;
+  unsigned long long cum = base + block_excl_scan<unsigned long long>(sum, sc.shl, &tot);
+  if (cum < target && cum + sum >= target) {   // the crossing is in this thread's digits
+#pragma unroll
+    for (int k = 0; k < kDPer; ++k) {
+      if (cum < target && cum + m[k] >= target) {
+        sc.digit = 511 - kDPer * tid - k;
         sc.above = cum;
       }
-      cum += m;
+      cum += m[k];
     }
   }
 }
@@ -1447,69 +1422,65 @@ __device__ void refine_range(const StepParams& P, SmemRefine& sm, SelScalars& sc
 
 // ------------------------------------------------------------------ compact phase
 // One range of slice y (after refine_range of y): its kept positions outside
-// sinks/window, ascending, written at the range's offset in the slice's list.  Rounds of 1024 tokens: lane l of warp w
-// takes tokens 4 l .. 4 l + 3 of the warp's 128 (one 16-byte read of their
-// probabilities in token mode), a warp scan orders the lanes and the warp totals
-// order the warps.
+// sinks/window, ascending, written at the range's offset in the slice's list.  Rounds of
+// kThrRun consecutive tokens per thread: the thread's keep mask from its probabilities
+// (16-byte reads in token mode, its block's one in block mode), one CTA scan of the
+// counts for the thread's offset, the kept positions staged in order in shared memory
+// (`stage`, kThrRun * threads ints), then copied to the list with coalesced stores.
 template <bool BLK>
-__device__ void compact_segment(const StepParams& P, SelScalars& sc, const Ranges<BLK>& R, int y, int l0, int l1) {
+__device__ void compact_segment(const StepParams& P, SelScalars& sc, int* stage, const Ranges<BLK>& R, int y, int l0,
+                                int l1) {
   const Unit un = unit_of(P, y);
   const PiSeg ps = pi_seg<BLK>(R, y, un.s);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int L = sc.L;   // sc.L, sc.tau, sc.pos_cut and sc.off from refine_range of this slice
   const unsigned tau = sc.tau;
   const int pos_cut = sc.pos_cut;
   const SinkWindow sw(L, P.n_sink, P.window);
   const int j0 = 16 * l0, j1 = min(L, 16 * l1);
   int* dst = P.sel_list + (size_t)un.s * P.Lmax;
-  int64_t run = sc.off;
-  for (int k0 = j0; k0 < j1; k0 += 4 * kSelThreads) {   // whole CTA: the barriers below
-    const int jb = k0 + 128 * warp + 4 * lane;
+  int run = sc.off;
+  static_assert(kBlock % kThrRun == 0, "a thread's run lies in one block");
+  static_assert(sizeof(SelSmem) >= sizeof(int) * kThrRun * kSelThreads, "a round's positions fit the stage");
+  for (int k0 = j0; k0 < j1; k0 += kThrRun * kSelThreads) {   // whole CTA: the scan below
+    const int jb = k0 + kThrRun * tid;
     unsigned keep = 0u;
     if (jb < j1) {
-      float v[4];
+      unsigned bits[kThrRun];
       if (BLK) {
+        const unsigned v = __float_as_uint(pi_load(P, ps, jb / kBlock));
 #pragma unroll
-        for (int q = 0; q < 4; ++q) v[q] = jb + q < j1 ? pi_load(P, ps, (jb + q) / kBlock) : 0.f;
+        for (int q = 0; q < kThrRun; ++q) bits[q] = v;
       } else {
-        const float4 w = pi_load4(P, ps, jb);
-        v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w;
+#pragma unroll
+        for (int q4 = 0; q4 < kThrRun / 4; ++q4) {   // jb is a multiple of 16: aligned 16-byte words
+          const float4 v = pi_load4(P, ps, jb + 4 * q4);
+          bits[4 * q4] = __float_as_uint(v.x);
+          bits[4 * q4 + 1] = __float_as_uint(v.y);
+          bits[4 * q4 + 2] = __float_as_uint(v.z);
+          bits[4 * q4 + 3] = __float_as_uint(v.w);
+        }
       }
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < kThrRun; ++q) {
         const int j = jb + q;
         const int e = BLK ? j / kBlock : j;
-        const bool k = j < j1 && !sw.always(j) && kept_by_cut(__float_as_uint(v[q]), e, tau, pos_cut);
-        keep |= (k ? 1u : 0u) << q;
+        if (j < j1 && !sw.always(j) && kept_by_cut(bits[q], e, tau, pos_cut)) keep |= 1u << q;
       }
     }
-    // warp scan of the lanes' counts, then the warps' totals
-    const int c = __popc(keep);
-    int x = c;
+    int total;
+    int o = block_excl_scan<int>(__popc(keep), sc.shi, &total);   // (ends with a CTA barrier)
+    // the round's kept positions in order in shared memory, then one coalesced copy
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(kFull, x, o);
-      if (lane >= o) x += t;
-    }
-    if (lane == 31) sc.shi[warp] = x;
+    for (int q = 0; q < kThrRun; ++q)
+      if (keep >> q & 1u) stage[o++] = jb + q;
     __syncthreads();
-    int wbase = 0, total = 0;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      const int t = sc.shi[w];
-      wbase += w < warp ? t : 0;
-      total += t;
+    if (run + total > P.Lmax) {   // offsets and predicate disagree: never write past the list
+      if (tid == 0) atomicOr(P.ws.dev_err, kErrInternal);
+      total = P.Lmax - run;
     }
-    __syncthreads();   // sc.shi is rewritten by the next round
-    int64_t o = run + wbase + (x - c);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      if (keep >> q & 1u) {
-        if (o < P.Lmax) dst[o] = jb + q;
-        else atomicOr(P.ws.dev_err, kErrInternal);   // offsets and predicate disagree: never write past the list
-        ++o;
-      }
-    }
+    for (int i = tid; i < total; i += kSelThreads) dst[run + i] = stage[i];
+    __syncthreads();   // the stage is rewritten by the next round
     run += total;
   }
 }
@@ -1552,7 +1523,7 @@ __global__ void __launch_bounds__(kSelThreads, 1024 / kSelThreads) k_select(Step
     ok = slice_wait(&st->arr_thr, n_ranges(y), P.ws.dev_err, &sc.ok);
     if (!ok) return;
     refine_range<BLK>(P, sm.ref, sc, R, y, l0, l1, (int)blockIdx.x == R.first_cta(y));
-    compact_segment<BLK>(P, sc, R, y, l0, l1);
+    compact_segment<BLK>(P, sc, reinterpret_cast<int*>(&sm), R, y, l0, l1);
   });
 }
 
