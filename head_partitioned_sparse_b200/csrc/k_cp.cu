@@ -27,8 +27,11 @@
 //           them and writes (out, log2-sum-exp)                      -> out[rank], lse[rank]
 //   combine out = sum_r 2^(lse_r - M) out_r / sum_r 2^(lse_r - M).
 // Masses are integers in units of 2^-63 (mass_q), so the summed histograms are exact
-// whatever the order, and every rank takes the same cut decisions.  The kernels never
-// wait on another launch or rank: the exchanges happen between launches.
+// whatever the order, and every rank takes the same cut decisions.  Each cut is taken
+// at the start of the launch that needs it, by every CTA of the slice (the summed
+// histogram is a few KB to 32 KB per rank), so a rank's step is seven launches: stats,
+// mass, round 2, round 3, list count, list, attention.  The kernels never wait on
+// another launch or rank: the exchanges happen between launches.
 #include "spa_internal.cuh"
 
 namespace spa {
@@ -423,55 +426,68 @@ __device__ unsigned long long gather_hist4096(const unsigned long long* hist, in
   return mine;
 }
 
-// grid (n_slices).  round 1: total mass and target from the summed round-1 histograms,
-// then bin b1; round 2: bin b2 inside b1; round 3: bin b3, tau and this rank's quota of
-// the tokens at tau.
-__global__ void __launch_bounds__(kThreads) k_cp_cut(CpParams P, int round) {
-  __shared__ unsigned long long h[kHistSlots];
-  __shared__ unsigned long long cnt3[kBins3];
-  __shared__ unsigned long long scratch[kWarpsPerCta];
-  __shared__ int sb;
-  __shared__ unsigned long long sabove;
-  const int s = blockIdx.x, g = s % P.Hkv, tid = threadIdx.x;
-  if (!P.is_ret[g]) return;
-  CpSlice* cs = P.cs + s;
+// The cuts, taken at the start of the kernel that needs them by every CTA of the slice
+// (the histograms were exchanged between the launches; every CTA reaches the same
+// result from the same data).  Chunk 0 of the slice stores the cut state for the
+// following phases.
+//
+// Cut 1: total mass and target from the summed round-1 histograms, then bin b1 (-1
+// keeps every token).  h: kHistSlots words of shared memory.  Ends with a CTA barrier.
+__device__ void cp_cut1(const CpParams& P, int s, bool store, unsigned long long* h, unsigned long long* scratch,
+                        int* sb, unsigned long long* sabove, unsigned long long* starget) {
+  const int tid = threadIdx.x;
+  const unsigned long long mine = gather_hist4096(P.hist1, P.n_ranks, P.n_slices, s, h);
+  const unsigned long long total = block_sum<unsigned long long>(mine, scratch);   // (barrier: h complete)
+  unsigned long long target = (unsigned long long)ceil((double)P.p * (double)total);
+  if (target < 1ull) target = 1ull;
+  const bool keep = P.keep_all || target > total;
+  if (tid == 0) { *sb = -1; *sabove = 0ull; *starget = target; }
+  __syncthreads();
+  if (!keep) cut_desc<kBins1, true>(h, 0ull, target, sb, sabove, scratch);
+  if (store && tid == 0) {
+    CpSlice* cs = P.cs + s;
+    cs->target = target;
+    cs->above = *sabove;
+    cs->b1 = *sb;
+    cs->b2 = -1;
+    cs->tau = 0u;
+    cs->quota = 0;
+  }
+  __syncthreads();
+}
+
+// Cut 2 (b1 >= 0): bin b2 inside b1 from the summed round-2 histograms; *sabove enters
+// as the mass above b1 and leaves as the mass above (b1, b2) (stored as above2, so the
+// launch's other CTAs still read the round-1 value).  Ends with a CTA barrier.
+__device__ void cp_cut2(const CpParams& P, int s, bool store, unsigned long long target, unsigned long long* h,
+                        unsigned long long* scratch, int* sb, unsigned long long* sabove) {
+  const int tid = threadIdx.x;
+  const unsigned long long above = *sabove;
+  gather_hist4096(P.hist2, P.n_ranks, P.n_slices, s, h);
+  if (tid == 0) *sb = -1;
+  __syncthreads();
+  cut_desc<kBins2, true>(h, above, target, sb, sabove, scratch);
+  if (tid == 0) {
+    if (*sb < 0) { atomicOr(P.err, kErrInternal); *sb = 0; }
+    if (store) {
+      CpSlice* cs = P.cs + s;
+      cs->b2 = *sb;
+      cs->above2 = *sabove;
+    }
+  }
+  __syncthreads();
+}
+
+// Cut 3 (b1 >= 0): bin b3, tau and this rank's quota of the tokens at tau (lowest
+// positions first, i.e. rank by rank) from the round-3 histograms.  Ends with a CTA
+// barrier; results in *stau and *squota.
+__device__ void cp_cut3(const CpParams& P, int s, bool store, unsigned long long* h, unsigned long long* cnt3,
+                        unsigned long long* scratch, int* sb, unsigned long long* sabove, unsigned* stau, int* squota) {
+  const int tid = threadIdx.x;
+  const CpSlice* cs = P.cs + s;
+  const int b1 = __ldcg(&cs->b1), b2 = __ldcg(&cs->b2);
+  const unsigned long long target = __ldcg(&cs->target), above = __ldcg(&cs->above2);
   const int R = P.n_ranks;
-  if (round == 1) {
-    const unsigned long long mine = gather_hist4096(P.hist1, R, P.n_slices, s, h);
-    const unsigned long long total = block_sum<unsigned long long>(mine, scratch);   // (barrier: h complete)
-    unsigned long long target = (unsigned long long)ceil((double)P.p * (double)total);
-    if (target < 1ull) target = 1ull;
-    const bool keep = P.keep_all || target > total;
-    if (tid == 0) { sb = -1; sabove = 0ull; }
-    __syncthreads();
-    if (!keep) cut_desc<kBins1, true>(h, 0ull, target, &sb, &sabove, scratch);
-    if (tid == 0) {
-      cs->target = target;
-      cs->above = sabove;
-      cs->b1 = sb;   // -1: keep every token
-      cs->b2 = -1;
-      cs->tau = 0u;
-      cs->quota = 0;
-    }
-    return;
-  }
-  const int b1 = __ldcg(&cs->b1);
-  if (b1 < 0) return;
-  const unsigned long long target = __ldcg(&cs->target), above = __ldcg(&cs->above);
-  if (round == 2) {
-    gather_hist4096(P.hist2, R, P.n_slices, s, h);
-    if (tid == 0) { sb = -1; sabove = above; }
-    __syncthreads();
-    cut_desc<kBins2, true>(h, above, target, &sb, &sabove, scratch);
-    if (tid == 0) {
-      if (sb < 0) atomicOr(P.err, kErrInternal);
-      cs->b2 = sb < 0 ? 0 : sb;
-      cs->above = sabove;
-    }
-    return;
-  }
-  // round 3
-  const int b2 = __ldcg(&cs->b2);
   if (tid < kBins3) {
     unsigned long long v = 0ull, k = 0ull;
     for (int r = 0; r < R; ++r) {
@@ -482,40 +498,60 @@ __global__ void __launch_bounds__(kThreads) k_cp_cut(CpParams P, int round) {
     h[tid] = v;
     cnt3[tid] = k;
   }
-  if (tid == 0) { sb = -1; sabove = above; }
+  if (tid == 0) { *sb = -1; *sabove = above; }
   __syncthreads();
-  cut_desc<kBins3, false>(h, above, target, &sb, &sabove, scratch);
+  cut_desc<kBins3, false>(h, above, target, sb, sabove, scratch);
   if (tid == 0) {
-    int b3 = sb;
+    int b3 = *sb;
     if (b3 < 0) { atomicOr(P.err, kErrInternal); b3 = 0; }
     const unsigned tau = ((unsigned)b1 << 18) | ((unsigned)b2 << 6) | (unsigned)b3;
     // tokens at tau, lowest positions first, while the mass before them is below target
     const unsigned long long mt = mass_q(tau);
-    const unsigned long long need = target > sabove ? target - sabove : 0ull;
+    const unsigned long long need = target > *sabove ? target - *sabove : 0ull;
     const unsigned long long ties = mt ? (need + mt - 1ull) / mt : cnt3[b3];
     unsigned long long before = 0ull;
     for (int r = 0; r < P.rank; ++r) before += __ldcg(P.hist3 + (((size_t)r * P.n_slices + s) * kBins3 + b3) * 2 + 1);
     const unsigned long long mine = __ldcg(P.hist3 + (((size_t)P.rank * P.n_slices + s) * kBins3 + b3) * 2 + 1);
     unsigned long long q = ties > before ? ties - before : 0ull;
     if (q > mine) q = mine;
-    cs->tau = tau;
-    cs->quota = (int)q;
+    *stau = tau;
+    *squota = (int)q;
+    if (store) {
+      CpSlice* w = P.cs + s;
+      w->tau = tau;
+      w->quota = (int)q;
+    }
   }
+  __syncthreads();
 }
 
 // ------------------------------------------------------------------ rounds 2 and 3
-// grid (n_chunks, n_slices), retrieval slices with a cut.  Round 2: masses of the
-// round-2 digit of the tokens in bin b1.  Round 3: masses and counts of the round-3
-// digit of the tokens in (b1, b2), plus this chunk's counts per digit (tab3).
+// grid (n_chunks, n_slices), retrieval slices.  Round 2: cut 1, then the masses of the
+// round-2 digit of the tokens in bin b1.  Round 3: cut 2, then the masses and counts of
+// the round-3 digit of the tokens in (b1, b2), plus this chunk's counts per digit
+// (tab3).  Slices whose cut keeps every token stop after the cut.
 __global__ void __launch_bounds__(kThreads) k_cp_hist(CpParams P, int round) {
-  __shared__ unsigned long long hm[kBins2];
+  __shared__ unsigned long long hm[kHistSlots];   // the cut's summed histogram, then this chunk's masses
   __shared__ unsigned hn[kBins3];
-  __shared__ int sh_len;
+  __shared__ unsigned long long scratch[kWarpsPerCta];
+  __shared__ unsigned long long sabove, starget;
+  __shared__ int sb, sh_len;
   const int c = blockIdx.x, s = blockIdx.y, b = s / P.Hkv, g = s % P.Hkv, tid = threadIdx.x;
   if (!P.is_ret[g]) return;
   const CpSlice* cs = P.cs + s;
-  const int b1 = __ldcg(&cs->b1);
-  const int b2 = __ldcg(&cs->b2);
+  int b1, b2 = 0;
+  if (round == 2) {
+    cp_cut1(P, s, c == 0, hm, scratch, &sb, &sabove, &starget);
+    b1 = sb;
+  } else {
+    b1 = __ldcg(&cs->b1);
+    if (b1 >= 0) {
+      if (tid == 0) sabove = __ldcg(&cs->above);
+      __syncthreads();
+      cp_cut2(P, s, c == 0, __ldcg(&cs->target), hm, scratch, &sb, &sabove);
+      b2 = sb;
+    }
+  }
   const int L = cta_len(P, b, &sh_len);
   if (b1 < 0) return;
   const long long n = local_rows(P, L);
@@ -567,20 +603,16 @@ __global__ void __launch_bounds__(kThreads) k_cp_hist(CpParams P, int round) {
 // window of the global positions, plus (retrieval slices) the top-p set: probability
 // above tau, or at tau within the rank's quota counted from its lowest position.
 // Returns the 16-bit mask; needs the CTA (block scans of the tied rows).
-__device__ unsigned list_mask(const CpParams& P, int s, int c, int L, unsigned* uscratch) {
+__device__ unsigned list_mask(const CpParams& P, int s, int c, int L, int b1, unsigned tau, int quota,
+                              unsigned* uscratch) {
   const int g = s % P.Hkv, tid = threadIdx.x;
   const bool ret = P.is_ret[g] != 0;
   const long long n = local_rows(P, L);
   const long long r0 = (long long)c * kChunk + (long long)tid * kRun;
-  // issue every load first: the cut state, the thread's 16 probabilities (r0 is a
-  // multiple of 16 rows: four aligned 16-byte words), the earlier chunks' tie counts
-  int b1 = -1, quota = 0;
-  unsigned tau = 0u;
+  // issue the loads first: the thread's 16 probabilities (r0 is a multiple of 16 rows:
+  // four aligned 16-byte words), the earlier chunks' tie counts
   uint4 pw[kRun / 4];
   if (ret) {
-    b1 = __ldcg(&P.cs[s].b1);
-    tau = __ldcg(&P.cs[s].tau);
-    quota = __ldcg(&P.cs[s].quota);
     const uint4* pv = reinterpret_cast<const uint4*>(P.pi + (size_t)s * P.pi_stride + r0);
 #pragma unroll
     for (int q4 = 0; q4 < kRun / 4; ++q4) pw[q4] = r0 < n ? __ldcg(pv + q4) : make_uint4(0u, 0u, 0u, 0u);
@@ -630,14 +662,32 @@ __device__ unsigned list_mask(const CpParams& P, int s, int c, int L, unsigned* 
   return mask | gt | kept_eq;
 }
 
-// pass 0: listed rows per chunk.  pass 1: the rows themselves (ascending), the slice's
+// pass 0: cut 3 (retrieval slices with a cut; chunk 0 stores tau and the quota), then
+// the listed rows per chunk.  pass 1: the rows themselves (ascending), the slice's
 // count, and (empty slices) the rank's zero output with log2-sum-exp -inf.
 __global__ void __launch_bounds__(kThreads) k_cp_list(CpParams P, int pass) {
   __shared__ unsigned uscratch[kWarpsPerCta];
-  __shared__ int sh_len;
-  const int c = blockIdx.x, s = blockIdx.y, b = s / P.Hkv, tid = threadIdx.x;
+  __shared__ unsigned long long h3[kBins3], c3[kBins3], scratch[kWarpsPerCta], sabove;
+  __shared__ unsigned stau;
+  __shared__ int sb, squota, sh_len;
+  const int c = blockIdx.x, s = blockIdx.y, b = s / P.Hkv, g = s % P.Hkv, tid = threadIdx.x;
+  int b1 = -1, quota = 0;
+  unsigned tau = 0u;
+  if (P.is_ret[g]) {
+    b1 = __ldcg(&P.cs[s].b1);
+    if (b1 >= 0) {
+      if (pass == 0) {
+        cp_cut3(P, s, c == 0, h3, c3, scratch, &sb, &sabove, &stau, &squota);
+        tau = stau;
+        quota = squota;
+      } else {
+        tau = __ldcg(&P.cs[s].tau);
+        quota = __ldcg(&P.cs[s].quota);
+      }
+    }
+  }
   const int L = cta_len(P, b, &sh_len);
-  const unsigned mask = list_mask(P, s, c, L, uscratch);
+  const unsigned mask = list_mask(P, s, c, L, b1, tau, quota, uscratch);
   unsigned n_chunk;
   const unsigned off = block_excl_scan<unsigned>((unsigned)__popc(mask), uscratch, &n_chunk);
   if (pass == 0) {
@@ -716,11 +766,6 @@ cudaError_t launch_cp_mass(const CpParams& P, cudaStream_t st) {
     case 8: k_cp_mass<8><<<grid, kRowThreads, 0, st>>>(P); break;
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
-}
-
-cudaError_t launch_cp_cut(const CpParams& P, int round, cudaStream_t st) {
-  k_cp_cut<<<P.n_slices, kThreads, 0, st>>>(P, round);
   return cudaGetLastError();
 }
 

@@ -468,6 +468,10 @@ __global__ void __launch_bounds__(kSelThreads) k_qprep(StepParams P) {
   __shared__ SmemPro sm;
   __shared__ SelScalars sc;
   const int s = blockIdx.x, b = s / P.Hkv, g = s % P.Hkv, tid = threadIdx.x;
+  // the selection kernel (launched with programmatic stream serialization) may start
+  // its CTAs and their first index-row loads now; it waits for this grid's completion
+  // before it reads anything written here
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   if (P.is_ret[g]) {
     if (tid == 0) {
       SliceState z;
@@ -509,6 +513,7 @@ struct Ranges {
   long long ngc, quanta;
   int nb;
   int cps;                 // CTAs per slice (0: ranges may span slices)
+  int me;                  // this CTA's range index
   int y_me, l0_me, l1_me;  // with cps: this CTA's one segment
   __device__ __forceinline__ Ranges(const StepParams& P) {
     ngc = ((long long)P.Lcap + 16 * q - 1) / (16 * q) * q;
@@ -516,11 +521,12 @@ struct Ranges {
     quanta = (long long)n_rs * (ngc / q);
     nb = (int)gridDim.x;
     cps = (n_rs > 0 && nb % n_rs == 0) ? nb / n_rs : 0;
+    me = (int)blockIdx.x;
     y_me = l0_me = l1_me = 0;
     if (cps) {
       const long long qs = ngc / q;
-      y_me = (int)blockIdx.x / cps;
-      const int k = (int)blockIdx.x - y_me * cps;
+      y_me = me / cps;
+      const int k = me - y_me * cps;
       l0_me = (int)((long long)k * qs / cps) * q;
       l1_me = (int)((long long)(k + 1) * qs / cps) * q;
     }
@@ -534,7 +540,7 @@ struct Ranges {
   }
   // range-relative group offset of slice y's group 0
   __device__ __forceinline__ long long seg_origin(int y) const {
-    return cps ? -(long long)l0_me : (long long)y * ngc - begin(blockIdx.x);
+    return cps ? -(long long)l0_me : (long long)y * ngc - begin(me);
   }
 };
 // Per-range values of slice y (statistics, counts, offsets) live at slot cta + y: the
@@ -549,8 +555,8 @@ __device__ __forceinline__ void for_each_segment(const RT& R, F&& f) {
     f(R.y_me, R.l0_me, R.l1_me);
     return;
   }
-  const long long ge = R.begin(blockIdx.x + 1);
-  for (long long g = R.begin(blockIdx.x); g < ge;) {
+  const long long ge = R.begin(R.me + 1);
+  for (long long g = R.begin(R.me); g < ge;) {
     const int y = (int)(g / R.ngc);
     const long long gend = min(ge, (long long)(y + 1) * R.ngc);
     f(y, (int)(g - (long long)y * R.ngc), (int)(gend - (long long)y * R.ngc));
@@ -599,7 +605,7 @@ __device__ __forceinline__ float4 pi_load4(const StepParams& P, PiSeg ps, int e)
 // before the query index vectors are read (bounded by the call's max length; rows past
 // the sequence are masked).
 template <int G>
-__device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc, int y, int l0, int l1) {
+__device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc, int me, int y, int l0, int l1) {
   constexpr int NH = IdxTiles<G>::NH, U = kGroupBatch;
   const Unit un = unit_of(P, y);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, t4 = lane & 3, gid = lane >> 2;
@@ -611,6 +617,9 @@ __device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc
 #pragma unroll
     for (int u = 0; u < U; ++u) load_group(rows, 16 * (l0 + warp + kWarps * u), jpf, pol, ra[u], rb[u]);
   }
+  // from here on the prologue kernel's writes (state reset, q_idx) are read: wait for
+  // its completion (returns at once when this launch did not overlap it)
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   // the sequence length and the query index vectors (formed by the prologue kernel)
   // are requested behind the first batch; one CTA barrier publishes them
   __syncthreads();   // earlier readers of sc.L and sc.qsm are done
@@ -626,7 +635,7 @@ __device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc
   }
   __syncthreads();
   const int L = sc.L;
-  float2* out = P.ws.stats + stats_slot(blockIdx.x, y) * G;
+  float2* out = P.ws.stats + stats_slot(me, y) * G;
   if (16 * l0 >= L) {
     if (tid < G) out[tid] = make_float2(-INFINITY, 0.f);
     return;
@@ -1049,7 +1058,7 @@ __device__ void threshold_segment(const StepParams& P, SelScalars& sc, SmemRefin
     }
     __syncthreads();   // sc.cbase is rewritten by the next round
   }
-  if (tid == 0) P.ws.seg_cnt[stats_slot(blockIdx.x, y)] = above_all;
+  if (tid == 0) P.ws.seg_cnt[stats_slot(R.me, y)] = above_all;
 }
 
 // ------------------------------------------------------------------ refine (per range)
@@ -1153,7 +1162,7 @@ __device__ void refine_range(const StepParams& P, SmemRefine& sm, SelScalars& sc
   const Unit un = unit_of(P, y);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const SliceState* st = P.ws.st + un.s;
-  const int first = R.first_cta(y), n_seg = R.last_cta(y) - first + 1, mine = (int)blockIdx.x - first;
+  const int first = R.first_cta(y), n_seg = R.last_cta(y) - first + 1, mine = R.me - first;
   const int* abv_row = P.ws.seg_cnt + stats_slot(first, y);
   constexpr int kSegPer = kMaxSelectGrid / kSelThreads;
   // one round trip: the cut state, the ranges' counts above b1, the round-A histogram
@@ -1493,7 +1502,7 @@ __global__ void __launch_bounds__(kSelThreads, 1024 / kSelThreads) k_select(Step
   const Ranges<BLK> R(P);
   auto n_ranges = [&](int y) { return (unsigned)(R.last_cta(y) - R.first_cta(y) + 1); };
   for_each_segment(R, [&](int y, int l0, int l1) {
-    score_segment<G>(P, sm.score, sc, y, l0, l1);
+    score_segment<G>(P, sm.score, sc, R.me, y, l0, l1);
     // failure-detection test hook: CTA 0 never arrives, so the other CTAs of its slice
     // give up their bounded waits for the slice's statistics
     if (!(P.drop_publish && blockIdx.x == 0)) slice_arrive(&P.ws.st[unit_of(P, y).s].arr_score);
@@ -1512,7 +1521,7 @@ __global__ void __launch_bounds__(kSelThreads, 1024 / kSelThreads) k_select(Step
     SliceState* st = P.ws.st + unit_of(P, y).s;
     ok = slice_wait(&st->arr_mass, n_ranges(y), P.ws.dev_err, &sc.ok);
     if (!ok) return;
-    cut1_range(P, sc, y, (int)blockIdx.x == R.first_cta(y));
+    cut1_range(P, sc, y, R.me == R.first_cta(y));
     threshold_segment<BLK>(P, sc, sm.ref, R, y, l0, l1);
     slice_arrive(&st->arr_thr);
   });
@@ -1522,7 +1531,7 @@ __global__ void __launch_bounds__(kSelThreads, 1024 / kSelThreads) k_select(Step
     SliceState* st = P.ws.st + unit_of(P, y).s;
     ok = slice_wait(&st->arr_thr, n_ranges(y), P.ws.dev_err, &sc.ok);
     if (!ok) return;
-    refine_range<BLK>(P, sm.ref, sc, R, y, l0, l1, (int)blockIdx.x == R.first_cta(y));
+    refine_range<BLK>(P, sm.ref, sc, R, y, l0, l1, R.me == R.first_cta(y));
     compact_segment<BLK>(P, sc, reinterpret_cast<int*>(&sm), R, y, l0, l1);
   });
 }
@@ -1535,7 +1544,22 @@ cudaError_t launch_tg(const StepParams& P, int grid, cudaStream_t st) {
   StepParams local = P;
   void* args[] = {&local};
   const void* fn = P.blocks ? (const void*)k_select<T, G, true> : (const void*)k_select<T, G, false>;
-  return cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(kSelThreads), args, kPiBytes, st);
+  // cooperative (every CTA resident: the arrival waits need it) and allowed to start
+  // before the prologue kernel ends (programmatic stream serialization; the score phase
+  // waits for the prologue's completion after requesting its first index rows)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kSelThreads);
+  cfg.dynamicSmemBytes = kPiBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeCooperative;
+  at[0].val.cooperative = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
 // Co-resident CTAs per SM, the smaller of the token and block variants (one grid size

@@ -810,14 +810,11 @@ spa_status spa_cp_phase(spa_handle h, int phase, const spa_cp_args* a, spa_strea
       return run(h, SPA_K_CP_SELECT, st, "cp stats", [&] { return spa::launch_cp_stats(C, st); });
     case SPA_CP_MASS:   // (the stats phase cleared this rank's hist1 rows)
       return run(h, SPA_K_CP_SELECT, st, "cp mass", [&] { return spa::launch_cp_mass(C, st); });
-    case SPA_CP_ROUND2:   // (the mass phase cleared this rank's hist2 and hist3 rows)
-      if ((r = run(h, SPA_K_CP_SELECT, st, "cp cut 1", [&] { return spa::launch_cp_cut(C, 1, st); }))) return r;
+    case SPA_CP_ROUND2:   // cut 1 + round 2 (the mass phase cleared this rank's hist2 and hist3 rows)
       return run(h, SPA_K_CP_SELECT, st, "cp round 2", [&] { return spa::launch_cp_hist(C, 2, st); });
-    case SPA_CP_ROUND3:
-      if ((r = run(h, SPA_K_CP_SELECT, st, "cp cut 2", [&] { return spa::launch_cp_cut(C, 2, st); }))) return r;
+    case SPA_CP_ROUND3:   // cut 2 + round 3
       return run(h, SPA_K_CP_SELECT, st, "cp round 3", [&] { return spa::launch_cp_hist(C, 3, st); });
-    case SPA_CP_ATTEND:
-      if ((r = run(h, SPA_K_CP_SELECT, st, "cp cut 3", [&] { return spa::launch_cp_cut(C, 3, st); }))) return r;
+    case SPA_CP_ATTEND:   // cut 3 + list count, list, attention
       if ((r = run(h, SPA_K_CP_SELECT, st, "cp list count", [&] { return spa::launch_cp_list(C, 0, st); }))) return r;
       if ((r = run(h, SPA_K_CP_SELECT, st, "cp list", [&] { return spa::launch_cp_list(C, 1, st); }))) return r;
       return cp_attend(h, a, C, st);

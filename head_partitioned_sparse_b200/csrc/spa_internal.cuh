@@ -67,11 +67,13 @@ struct __align__(16) SliceState {
 };
 
 // Cut state of one (b, kv head) slice in a context-parallel step (each rank holds a
-// contiguous run of the slice's positions).  Written by the cut kernels, read by the
-// histogram and list kernels of the following phases.
+// contiguous run of the slice's positions).  Written by the cuts (chunk 0 of the slice
+// in the launch that takes them), read by the histogram and list kernels of the
+// following phases.
 struct __align__(16) CpSlice {
   unsigned long long target;   // ceil(p * total mass), total over every rank
-  unsigned long long above;    // mass of all tokens strictly above the current digit prefix
+  unsigned long long above;    // mass of all tokens strictly above bin b1
+  unsigned long long above2;   // mass of all tokens strictly above the prefix (b1, b2)
   int b1, b2;                  // round-1 / round-2 bins; b1 = -1 keeps every token
   unsigned tau;                // fp32 bits of the cut probability (after round 3)
   int quota;                   // tokens at tau this rank keeps (its lowest positions first)
@@ -321,7 +323,6 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, float
 // Context-parallel phases (k_cp.cu).
 cudaError_t launch_cp_stats(const CpParams& P, cudaStream_t st);
 cudaError_t launch_cp_mass(const CpParams& P, cudaStream_t st);
-cudaError_t launch_cp_cut(const CpParams& P, int round, cudaStream_t st);
 cudaError_t launch_cp_hist(const CpParams& P, int round, cudaStream_t st);
 cudaError_t launch_cp_list(const CpParams& P, int pass, cudaStream_t st);
 cudaError_t launch_cp_combine(const float* out_all, const float* lse_all, int n_ranks, int rows, float* out,
