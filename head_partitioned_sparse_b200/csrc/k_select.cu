@@ -333,15 +333,18 @@ struct SelScalars {
   unsigned long long cut_above, above, target, m_above;
 };
 
-// Unit coordinates: retrieval slice y -> (b, g, s).
+// Unit coordinates: retrieval slice y of this launch -> (b, g, s) and its retrieval
+// slice index over the whole batch, yg (launches over part of a batch start at
+// sequence P.b_base).
 struct Unit {
-  int b, g, s;
+  int b, g, s, yg;
 };
 __device__ __forceinline__ Unit unit_of(const StepParams& P, int y) {
   Unit u;
-  u.b = y / P.n_ret;
+  u.b = P.b_base + y / P.n_ret;
   u.g = P.ret_heads[y % P.n_ret];
   u.s = u.b * P.Hkv + u.g;
+  u.yg = P.b_base * P.n_ret + y;
   return u;
 }
 // Sequence length of b, loaded by one thread and shared (every CTA of a slice needs it).
@@ -467,7 +470,7 @@ template <typename T, int G>
 __global__ void __launch_bounds__(kSelThreads) k_qprep(StepParams P) {
   __shared__ SmemPro sm;
   __shared__ SelScalars sc;
-  const int s = blockIdx.x, b = s / P.Hkv, g = s % P.Hkv, tid = threadIdx.x;
+  const int s = P.b_base * P.Hkv + (int)blockIdx.x, b = s / P.Hkv, g = s % P.Hkv, tid = threadIdx.x;
   // the selection kernel (launched with programmatic stream serialization) may start
   // its CTAs and their first index-row loads now; it waits for this grid's completion
   // before it reads anything written here
@@ -609,7 +612,7 @@ __device__ void score_segment(const StepParams& P, SmemScore& sm, SelScalars& sc
   constexpr int NH = IdxTiles<G>::NH, U = kGroupBatch;
   const Unit un = unit_of(P, y);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, t4 = lane & 3, gid = lane >> 2;
-  const uint2* rows = reinterpret_cast<const uint2*>(idx_rows(P, y, un.s));
+  const uint2* rows = reinterpret_cast<const uint2*>(idx_rows(P, un.yg, un.s));
   const uint64_t pol = l2_policy_keep();
   uint2 ra[U], rb[U];
   {
@@ -784,7 +787,7 @@ __device__ bool mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
   const Unit un = unit_of(P, y);
   const PiSeg ps = pi_seg<BLK>(R, y, un.s);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, gid = lane >> 2, t4 = lane & 3;
-  const uint2* rows = reinterpret_cast<const uint2*>(idx_rows(P, y, un.s));
+  const uint2* rows = reinterpret_cast<const uint2*>(idx_rows(P, un.yg, un.s));
   const uint64_t pol = l2_policy_drop();
   // local group of batch slot u at batch base gb
   auto grp = [&](int gb, int u) { return BLK ? gb + U * warp + u : gb + warp + kWarps * u; };
@@ -842,8 +845,11 @@ __device__ bool mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
     M[h] = head < G ? sm.Mh[head] : INFINITY;   // lanes of absent heads contribute nothing
   }
   const int jend = min(L, 16 * l1);
+  static_assert(kGroupBatch % 2 == 0, "token mode reduces the batch's groups in pairs");
   for (int gb = l0; 16 * gb < jend; gb += kWarps * U) {
     float bsum = 0.f;
+    float pa[2] = {0.f, 0.f};   // token mode: the first group of the current pair
+    int ja = 0;
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int j = 16 * grp(gb, u);
@@ -874,21 +880,28 @@ __device__ bool mass_segment(const StepParams& P, SmemMass& sm, SelScalars& sc, 
         }
         bsum += (j + gid < jend ? pr[0] : 0.f) + (j + gid + 8 < jend ? pr[1] : 0.f);
       } else {
-        // transposed reduction: after the exchange with lane t4 ^ 1, even lanes hold token
-        // gid's pair sum and odd lanes token gid + 8's; after t4 ^ 2, lanes t4 = 0 and 1
-        // hold the two tokens' sums over the 4 lanes (the same additions in the same order
-        // as reducing each token over the 4 lanes)
-        const bool odd = (t4 & 1) != 0;
-        float v = odd ? pr[1] : pr[0];
-        v += __shfl_xor_sync(kFull, odd ? pr[0] : pr[1], 1);
-        v += __shfl_xor_sync(kFull, v, 2);
-        const int jt = j + gid + 8 * t4;   // lane t4 = 0 keeps token gid, t4 = 1 token gid + 8
-        if (t4 < 2 && jt < jend) {
-          pi_store(P, ps, jt, v);
-          const unsigned bits = __float_as_uint(v);
-          const unsigned d = min(bits >> 18, (unsigned)(kBins1 - 1));
-          atomicAdd(&sm.cnt[d], 1u);
-          atomicAdd(&sm.low[d], bits & 0x3ffffu);
+        // two groups (A = slot u - 1, B = slot u) reduced together over the 4 lanes of a
+        // token row, so that every lane ends with one of the pair's 32 tokens: the
+        // exchange with lane t4 ^ 2 leaves lanes t4 < 2 with group A's two partial sums
+        // and lanes t4 >= 2 with group B's, the exchange with t4 ^ 1 leaves lane t4 with
+        // token gid (t4 even) or gid + 8 (t4 odd) of its group, summed in a fixed order
+        if ((u & 1) == 0) {
+          pa[0] = pr[0];
+          pa[1] = pr[1];
+          ja = j;
+        } else {
+          const bool hi2 = (t4 & 2) != 0, odd = (t4 & 1) != 0;
+          const float v0 = (hi2 ? pr[0] : pa[0]) + __shfl_xor_sync(kFull, hi2 ? pa[0] : pr[0], 2);
+          const float v1 = (hi2 ? pr[1] : pa[1]) + __shfl_xor_sync(kFull, hi2 ? pa[1] : pr[1], 2);
+          const float v = (odd ? v1 : v0) + __shfl_xor_sync(kFull, odd ? v0 : v1, 1);
+          const int jt = (hi2 ? j : ja) + gid + 8 * (t4 & 1);
+          if (jt < jend) {
+            pi_store(P, ps, jt, v);
+            const unsigned bits = __float_as_uint(v);
+            const unsigned d = min(bits >> 18, (unsigned)(kBins1 - 1));
+            atomicAdd(&sm.cnt[d], 1u);
+            atomicAdd(&sm.low[d], bits & 0x3ffffu);
+          }
         }
       }
     }
@@ -936,7 +949,7 @@ __device__ void prefetch_attended_rows(const StepParams& P) {
   const long long total = (long long)P.n_slices * per_slice;
   for (long long p = blockIdx.x + (long long)threadIdx.x * gridDim.x; p < total;
        p += (long long)gridDim.x * blockDim.x) {
-    const int s = (int)(p / per_slice), r = (int)(p % per_slice), piece = r >> 1;
+    const int s = P.b_base * P.Hkv + (int)(p / per_slice), r = (int)(p % per_slice), piece = r >> 1;
     int64_t L = P.seq_lens[s / P.Hkv];
     L = L < 1 ? 1 : (L > P.Lcap ? P.Lcap : L);
     const KvSlice<T> sl = kv_slice<T>(P, s);
@@ -1604,7 +1617,8 @@ int select_grid(const StepParams& P, int max_resident) {
   return (int)want;
 }
 
-cudaError_t launch_select(const StepParams& P, int kv_dtype, int grid, cudaStream_t st) {
+namespace {
+cudaError_t launch_part(const StepParams& P, int kv_dtype, int grid, cudaStream_t st) {
   if (kv_dtype == 0) {
     switch (P.G) {
       case 1: return launch_tg<__nv_bfloat16, 1>(P, grid, st);
@@ -1621,6 +1635,24 @@ cudaError_t launch_select(const StepParams& P, int kv_dtype, int grid, cudaStrea
     }
   }
   return cudaErrorInvalidValue;
+}
+}  // namespace
+
+cudaError_t launch_select(const StepParams& P, int kv_dtype, int max_resident, cudaStream_t st) {
+  if (max_resident > kMaxSelectGrid) max_resident = kMaxSelectGrid;
+  if (max_resident < 1 || P.n_ret > max_resident) return cudaErrorInvalidValue;
+  // sequences per launch: all, unless their retrieval slices outnumber the co-resident
+  // CTAs (then every launch still gets a whole number of CTAs per slice)
+  const int per = P.n_ret > 0 ? (max_resident / P.n_ret > 0 ? max_resident / P.n_ret : 1) : P.B;
+  for (int b0 = 0; b0 < P.B; b0 += per) {
+    StepParams Q = P;
+    Q.b_base = P.b_base + b0;
+    Q.B = P.B - b0 < per ? P.B - b0 : per;
+    Q.n_slices = Q.B * P.Hkv;
+    const cudaError_t e = launch_part(Q, kv_dtype, select_grid(Q, max_resident), st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 // Co-resident CTAs of the selection kernel per SM for (dtype, G), or -1.

@@ -235,8 +235,8 @@ spa_status setup_compact(spa::StepParams* P, const void* k_ring, const void* v_r
 }
 
 spa_status run_selection(spa_ctx* h, spa::StepParams& P, cudaStream_t st) {
-  const int grid = spa::select_grid(P, h->select_max_grid);
-  return run(h, SPA_K_SELECT, st, "select", [&] { return spa::launch_select(P, h->cfg.kv_dtype, grid, st); });
+  return run(h, SPA_K_SELECT, st, "select",
+             [&] { return spa::launch_select(P, h->cfg.kv_dtype, h->select_max_grid, st); });
 }
 
 spa_status select_with(spa_ctx* h, spa::StepParams& P, int32_t* sel_idx, int32_t* sel_count, spa_stream stream) {

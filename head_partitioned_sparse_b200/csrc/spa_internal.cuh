@@ -174,6 +174,7 @@ struct StepParams {
   int ring;              // ring rows per streaming head: n_sink + window
   int head_rank[kMaxKvHeads];   // rank of head g among the retrieval or the streaming heads
   int drop_publish;      // failure-detection test hook: selection CTA 0 never arrives at its slice's counters
+  int b_base;            // selection launches: first sequence of this launch's part of the batch
   const void* k_ring;    // [Bm][n_str][ring][128] streaming-head keys (compact layout)
   const void* v_ring;
   float* lse;            // optional [B][Hq]: log2-sum-exp of each head's attended scores
@@ -307,7 +308,10 @@ cudaError_t launch_kv_append_compact(const void* k_new, const void* v_new, const
                                      int Hkv, int64_t Lmax, int kv_dtype, const unsigned char* is_ret,
                                      const int* head_rank, int n_ret, int n_str, int n_sink, int window, void* k_ret,
                                      void* v_ret, void* k_ring, void* v_ring, unsigned* dev_err, cudaStream_t st);
-cudaError_t launch_select(const StepParams& P, int kv_dtype, int grid, cudaStream_t st);
+// Selection of every slice of P (prologue + selection kernel).  Batches whose retrieval
+// slices outnumber max_resident co-resident CTAs run as several launch pairs, each over
+// as many whole sequences as fit.
+cudaError_t launch_select(const StepParams& P, int kv_dtype, int max_resident, cudaStream_t st);
 int select_grid(const StepParams& P, int max_resident);
 int select_resident_per_sm(int kv_dtype, int G);
 cudaError_t launch_attend(const StepParams& P, int kv_dtype, int grid, cudaStream_t st);

@@ -127,7 +127,7 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
   if (ce != cudaSuccess) return err(SPA_ERR_CUDA, cudaGetErrorString(ce));
   const int per_sm = spa::select_resident_per_sm(kv_dtype, G);
   if (per_sm < 1 || sms < 1) return err(SPA_ERR_UNSUPPORTED, "spa_select_noalloc: selection kernel cannot be resident");
-  const int grid = spa::select_grid(P, per_sm * sms < spa::kMaxSelectGrid ? per_sm * sms : spa::kMaxSelectGrid);
+  const int max_grid = per_sm * sms < spa::kMaxSelectGrid ? per_sm * sms : spa::kMaxSelectGrid;
 
   void* base_v = nullptr;
   spa_status r = scratch_on_current_device(&base_v);
@@ -141,7 +141,7 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
       64 * 8,                                                  // inv_freq (unused by selection; zero)
       (size_t)B * n_q_heads * spa::kHeadDim * 4,               // q_rot
       (size_t)B * n_q_heads * spa::kIdxDim * 4,                // q_idx
-      (size_t)(grid + slices) * G * 8,                         // per-range statistics
+      (size_t)(max_grid + slices) * G * 8,                     // per-range statistics
       (size_t)slices * spa::pi_row_stride(max_ctx) * 4,        // pi
       (size_t)slices * spa::kBins1 * 8,                        // hist1
       (size_t)slices * max_ctx * 8,                            // candidates
@@ -173,7 +173,7 @@ extern "C" SPA_API spa_status spa_select_noalloc(const float* P_q, int n_q_heads
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(base, 0, head_bytes, st);   // stream-ordered; allocates nothing
   if (e != cudaSuccess) return err(SPA_ERR_CUDA, cudaGetErrorString(e));
-  e = spa::launch_select(P, kv_dtype, grid, st);
+  e = spa::launch_select(P, kv_dtype, max_grid, st);
   if (e != cudaSuccess) return err(SPA_ERR_CUDA, cudaGetErrorString(e));
   return SPA_OK;
 }

@@ -127,6 +127,34 @@ def test_select_and_decode_parity(prepared, case, p):
         assert np.abs(out - ref).max() <= OUT_ATOL
 
 
+def test_batch_split_over_several_selection_launches():
+    # more retrieval slices (320) than co-resident selection CTAs: the batch runs as
+    # several prologue + selection launches over whole sequences; ragged lengths catch a
+    # launch reading another launch's sequences
+    n_b = 320
+    lens = [64 + (37 * b) % 449 for b in range(n_b)]
+    inp = synth.make_inputs("tiny", 11, overrides={"B": n_b, "L": 512, "dtype": "bf16", "window": 32},
+                            seq_lens=lens)
+    idx = oracle_idx(inp, heads=_ret(inp))
+    pp = float(np.float32(inp.p))
+    with Handle(inp) as h:
+        dev = DevInputs(inp, idx)
+        lists, cnt = gpu_select(h, inp, dev, p=pp)
+        out, cnt2 = gpu_decode(h, inp, dev, p=pp)
+        B.spa_device_status(h.h)
+    assert np.array_equal(cnt, cnt2)
+    ref_on_gpu_sets, res = O.decode_inputs(inp, idx_cache=idx, p=pp,
+                                           attend_sets={k: v for k, v in lists.items() if inp.head_mask[k[1]]})
+    for b in range(inp.B):
+        for g in range(inp.Hkv):
+            if inp.head_mask[g]:
+                check_selection(lists[(b, g)], res[(b, g)], pp, inp.n_sink, inp.window)
+            else:
+                assert cnt[b, g] == 0
+    assert np.isfinite(out).all()
+    assert np.abs(out - ref_on_gpu_sets).max() <= OUT_ATOL
+
+
 @pytest.mark.parametrize("L", [1, 2, 17, 4095, 4096, 4097])
 @pytest.mark.parametrize("n_sink,window", [(4, 0), (0, 1), (4, 256), (0, 10 ** 6), (4, 64)])
 def test_edge_lengths_and_windows(L, n_sink, window):
