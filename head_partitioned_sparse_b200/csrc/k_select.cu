@@ -461,20 +461,29 @@ __device__ __forceinline__ unsigned* hist_a(const StepParams& P, int s) {
 
 
 // ------------------------------------------------------------------ query prologue kernel
-// One CTA per (b, kv head) slice, launched before the selection kernel: q_rot for the
-// slice's G heads (decode calls), and for a retrieval slice q_idx = P_q q_pre (float64
-// dot products), the reset of its selection state (arrival counters included) and of its
-// round-1 histogram.  A streaming slice's selection count is 0.  Forming these once per
-// slice lets every CTA of the selection kernel start streaming index rows at once.
+// Launched before the selection kernel: one CTA per (b, kv head) slice forms, for a
+// retrieval slice, q_idx = P_q q_pre (float64 dot products) and resets its selection
+// state (arrival counters included) and histograms (a streaming slice's selection count
+// is 0); in decode calls a second CTA per slice forms q_rot for the slice's G heads at
+// the same time.  Forming these once per slice lets every CTA of the selection kernel
+// start streaming index rows at once.
 template <typename T, int G>
 __global__ void __launch_bounds__(kSelThreads) k_qprep(StepParams P) {
   __shared__ SmemPro sm;
   __shared__ SelScalars sc;
-  const int s = P.b_base * P.Hkv + (int)blockIdx.x, b = s / P.Hkv, g = s % P.Hkv, tid = threadIdx.x;
+  // CTAs [0, n_slices) form q_idx and reset the selection state; decode calls add CTAs
+  // [n_slices, 2 n_slices) for q_rot, so the two chains run side by side
+  const bool rot = (int)blockIdx.x >= P.n_slices;
+  const int s = P.b_base * P.Hkv + (int)blockIdx.x - (rot ? P.n_slices : 0), b = s / P.Hkv, g = s % P.Hkv,
+            tid = threadIdx.x;
   // the selection kernel (launched with programmatic stream serialization) may start
   // its CTAs and their first index-row loads now; it waits for this grid's completion
   // before it reads anything written here
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  if (rot) {
+    qrot_slice<T>(P, sm, sc, s);
+    return;
+  }
   if (P.is_ret[g]) {
     if (tid == 0) {
       SliceState z;
@@ -495,7 +504,6 @@ __global__ void __launch_bounds__(kSelThreads) k_qprep(StepParams P) {
     P.ws.st[s].count = 0;
     if (P.sel_count) P.sel_count[s] = 0;
   }
-  if (P.k_cache) qrot_slice<T>(P, sm, sc, s);
 }
 
 // ------------------------------------------------------------------ work partition
@@ -1551,7 +1559,7 @@ __global__ void __launch_bounds__(kSelThreads, 1024 / kSelThreads) k_select(Step
 
 template <typename T, int G>
 cudaError_t launch_tg(const StepParams& P, int grid, cudaStream_t st) {
-  k_qprep<T, G><<<P.n_slices, kSelThreads, 0, st>>>(P);
+  k_qprep<T, G><<<P.k_cache ? 2 * P.n_slices : P.n_slices, kSelThreads, 0, st>>>(P);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || P.n_ret == 0) return e;   // nothing to select
   StepParams local = P;
