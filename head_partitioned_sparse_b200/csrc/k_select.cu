@@ -91,13 +91,6 @@ __device__ V block_excl_scan(V x, V* sh, V* total) {
   return pre + v - x;
 }
 
-template <typename V>
-__device__ V block_sum(V x, V* sh) {
-  V tot;
-  block_excl_scan(x, sh, &tot);
-  return tot;
-}
-
 // Mass of a token in the radix select: its quantised probability for top-p, 1 for
 // top-k (the same select then counts tokens, and the target is k).
 __device__ __forceinline__ unsigned long long sel_mass(const StepParams& P, unsigned bits) {
@@ -514,10 +507,11 @@ __global__ void __launch_bounds__(kSelThreads) k_qprep(StepParams P) {
 // Ranges are cut at multiples of q groups (q = 1, or kBlock / 16 in block mode so that
 // no block is split; ngc is then a multiple of q): CTA c covers groups
 // [q floor(c Q / nb), q floor((c+1) Q / nb)), Q = n_rs ngc / q.
-// When the grid gives every retrieval slice the same whole number of CTAs, cps (the
-// usual case: the launch grid is chosen so), the same partition reduces to 32-bit
-// arithmetic computed once per CTA: CTA c = y cps + k covers local groups
-// [q floor(k qs / cps), q floor((k+1) qs / cps)) of slice y, qs = ngc / q.
+// When the grid gives every retrieval slice the same whole number of CTAs, cps, the
+// same partition reduces to 32-bit arithmetic computed once per CTA: CTA c = y cps + k
+// covers local groups [q floor(k qs / cps), q floor((k+1) qs / cps)) of slice y,
+// qs = ngc / q.  launch_select sizes every launch so (it splits larger batches); the
+// general split stays correct for any grid.
 template <bool BLK>
 struct Ranges {
   static constexpr int q = BLK ? kBlock / 16 : 1;
