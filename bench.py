@@ -687,7 +687,7 @@ def main_native(args):
                 return z
             shards.append({"k": sl(k0_), "v": sl(v0_), "idx": sl(ix0_)})
         out_cp = torch.empty_like(out)
-        cp_bufs = cpm.alloc_exchange(B.spa_cp_exchange_sizes(cp_handles[0], inp.B, R), dev)
+        cp_bufs = cpm.alloc_exchange(B.spa_cp_exchange_sizes(cp_handles[0], inp.B, R, head_mask), dev)
 
         def step_cp(i, st=stream, ranks=None, combine=True):
             cpm.emulated_step(cp_handles, shards, q_pre=q, head_mask=head_mask, seq_lens=lens, Bsz=inp.B, p=p,
@@ -754,7 +754,7 @@ def main_native(args):
             graph_err = repr(e)[:200]
         step_cp(0)
         torch.cuda.synchronize(dev)
-        sizes = B.spa_cp_exchange_sizes(cp_handles[0], inp.B, R)
+        sizes = B.spa_cp_exchange_sizes(cp_handles[0], inp.B, R, head_mask)
         cpar = {"ranks": R, "rows_per_rank": C, "emulated_step_ms": ms_cp,
                 "graph_step_us": graph_step_us, "graph_rank_us": graph_rank_us,
                 "max_graph_rank_us": max(graph_rank_us) if graph_rank_us else None, "graph_error": graph_err,

@@ -108,7 +108,7 @@ _SIGS = {
     "spa_select_compact_sel": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i64, _i, _f, _i64, _i, _i, _vp, _vp, _vp]),
     "spa_decode_compact_sel": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i64, _i, _f, _i64, _i, _i,
                                     _vp, _vp, _vp]),
-    "spa_cp_exchange_sizes": (_i, [_vp, _i, _i, ctypes.POINTER(ctypes.c_size_t)]),
+    "spa_cp_exchange_sizes": (_i, [_vp, _i, _i, ctypes.POINTER(ctypes.c_uint8), ctypes.POINTER(ctypes.c_size_t)]),
     "spa_cp_phase": (_i, [_vp, _i, ctypes.POINTER(spa_cp_args), _vp]),
     "spa_cp_combine": (_i, [_vp, _vp, _vp, _i, _i, _vp, _vp]),
     "spa_device_status": (_i, [_vp, _vp]),
@@ -303,10 +303,13 @@ def spa_decode_compact_sel(h, q_pre, k_ret, v_ret, k_ring, v_ring, idx_ret, head
                                          p, int(k), n_sink, window, _ptr(out), _ptr(sel_count_opt), _stream(stream)))
 
 
-def spa_cp_exchange_sizes(h, B: int, n_ranks: int) -> Tuple[int, ...]:
-    """Byte sizes of the exchange buffers (stats, hist1, hist2, hist3, out_all, lse_all)."""
+def spa_cp_exchange_sizes(h, B: int, n_ranks: int, head_mask) -> Tuple[int, ...]:
+    """Byte sizes of the exchange buffers (stats, hist1, hist2, hist3, out_all, lse_all)
+    for the host head mask ``head_mask`` [Hkv] (the statistics and histograms hold its
+    retrieval slices only)."""
     arr = (ctypes.c_size_t * SPA_CP_NBUF)()
-    _check(load().spa_cp_exchange_sizes(h, B, n_ranks, arr))
+    mask = _host_u8(head_mask)
+    _check(load().spa_cp_exchange_sizes(h, B, n_ranks, ctypes.cast(mask, ctypes.POINTER(ctypes.c_uint8)), arr))
     return tuple(int(v) for v in arr)
 
 

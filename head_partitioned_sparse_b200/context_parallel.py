@@ -13,6 +13,9 @@ wrote in one exchange buffer, then ``spa_cp_combine``:
     SPA_CP_ROUND3  hist3     round-3 histogram with counts (ties go rank by rank)
     SPA_CP_ATTEND  out_all, lse_all   the rank's attention output and log2-sum-exp
 
+The statistics and histograms have rows for the retrieval slices only (streaming heads
+never select), so the buffers are sized for one head mask.
+
 Two drivers share that sequence (``run_step``):
   * ``ContextParallelDecoder``: one process per GPU; the exchange is
     ``torch.distributed.all_gather`` (NCCL on GPUs, gloo for the CPU tests);
@@ -60,6 +63,8 @@ def rank_span(rank: int, capacity: int) -> Tuple[int, int]:
 def allgather_slot(buf, n_ranks: int, rank: int, group=None) -> None:
     """All-gather of a [n_ranks][...] buffer whose slot ``rank`` this rank wrote."""
     import torch.distributed as dist
+    if buf.numel() == 0:   # no retrieval head: nothing to exchange (the same on every rank)
+        return
     v = buf.view(n_ranks, -1)
     mine = v[rank].clone()
     dist.all_gather(list(v.unbind(0)), mine, group=group)
@@ -72,6 +77,10 @@ def alloc_exchange(sizes: Sequence[int], device):
     return {name: torch.zeros(int(n), dtype=torch.uint8, device=device) for name, n in zip(BUFFERS, sizes)}
 
 
+def _mask_list(mask):
+    return [1 if int(v) else 0 for v in (mask.tolist() if hasattr(mask, "tolist") else mask)]
+
+
 def _views(bufs):
     import torch
     return bufs["out_all"].view(torch.float32), bufs["lse_all"].view(torch.float32)
@@ -80,12 +89,14 @@ def _views(bufs):
 class ContextParallelDecoder:
     """One rank of a context-parallel decode step (one process per GPU).
 
-    handle   -- this rank's libspa handle (max_ctx = C, the rank's share of positions)
-    B        -- batch of the steps
-    group    -- torch.distributed process group (default: the world)
+    handle    -- this rank's libspa handle (max_ctx = C, the rank's share of positions)
+    B         -- batch of the steps
+    head_mask -- [Hkv] retrieval heads of every step (the exchange buffers hold their
+                 slices only)
+    group     -- torch.distributed process group (default: the world)
     """
 
-    def __init__(self, handle, *, B: int, capacity: int, device, group=None):
+    def __init__(self, handle, *, B: int, capacity: int, device, head_mask, group=None):
         import torch.distributed as dist
         self.h = handle
         self.B = B
@@ -93,12 +104,16 @@ class ContextParallelDecoder:
         self.group = group
         self.rank = dist.get_rank(group)
         self.n_ranks = dist.get_world_size(group)
-        self.bufs = alloc_exchange(spa.spa_cp_exchange_sizes(handle, B, self.n_ranks), device)
+        self.head_mask = _mask_list(head_mask)
+        self.bufs = alloc_exchange(spa.spa_cp_exchange_sizes(handle, B, self.n_ranks, self.head_mask), device)
 
     def step(self, *, q_pre, k_cache, v_cache, idx_cache, head_mask, seq_lens, p: float, n_sink: int, window: int,
              out, max_seq_len: int = 0, sel_count=None, list_out=None) -> None:
         """Writes the step's output for every query head into ``out`` [B][Hq][128] (on
-        every rank).  k/v/idx caches are this rank's shards; seq_lens are global."""
+        every rank).  k/v/idx caches are this rank's shards; seq_lens are global;
+        head_mask must be the one the decoder was built with."""
+        if _mask_list(head_mask) != self.head_mask:
+            raise ValueError("head_mask differs from the one the exchange buffers were sized for")
         out_all, lse_all = _views(self.bufs)
         pos0, _ = rank_span(self.rank, self.C)
         args = spa.make_cp_args(q_pre=q_pre, k_cache=k_cache, v_cache=v_cache, idx_cache=idx_cache,
@@ -119,12 +134,12 @@ def emulated_step(handles: Sequence, shards: Sequence[dict], *, q_pre, head_mask
                   combine: bool = True) -> dict:
     """All ranks of a context-parallel step on one GPU: handles[r] and shards[r] (dict of
     ``k``, ``v``, ``idx`` device tensors) are rank r's.  Returns the exchange buffers
-    (reusable for the next call through ``bufs``).  ``ranks`` restricts the phases to
+    (reusable for the next call through ``bufs``, with the same ``head_mask``).  ``ranks`` restricts the phases to
     some ranks (to time one rank's share: the other slots of ``bufs`` must then hold an
     earlier step's exchanged data); ``combine=False`` skips the final merge."""
     R = len(handles)
     if bufs is None:
-        bufs = alloc_exchange(spa.spa_cp_exchange_sizes(handles[0], Bsz, R), q_pre.device)
+        bufs = alloc_exchange(spa.spa_cp_exchange_sizes(handles[0], Bsz, R, head_mask), q_pre.device)
     out_all, lse_all = _views(bufs)
     args: List[spa.spa_cp_args] = []
     for r in range(R):

@@ -26,6 +26,8 @@
 //           hist3); the rank lists its kept rows (top-p set, sinks, window), attends
 //           them and writes (out, log2-sum-exp)                      -> out[rank], lse[rank]
 //   combine out = sum_r 2^(lse_r - M) out_r / sum_r 2^(lse_r - M).
+// The exchange buffers hold one row per retrieval slice (xrow below): streaming heads
+// never select, so they neither write nor read statistics or histograms.
 // Masses are integers in units of 2^-63 (mass_q), so the summed histograms are exact
 // whatever the order, and every rank takes the same cut decisions.  Each cut is taken
 // at the start of the launch that needs it, by every CTA of the slice (the summed
@@ -58,6 +60,12 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ long long local_rows(const CpParams& P, int L) {
   long long n = (long long)L - P.pos0;
   return n < 0 ? 0 : (n > P.C ? P.C : n);
+}
+
+// Exchange row of retrieval slice s = (b, g) in rank r's slot: the exchange buffers hold
+// the retrieval slices only, sequence-major.
+__device__ __forceinline__ size_t xrow(const CpParams& P, int r, int s) {
+  return (size_t)r * P.n_xrows + (size_t)(s / P.Hkv) * P.n_ret + P.ret_ord[s % P.Hkv];
 }
 
 // Length of sequence b, validated as in the one-GPU step; shared through *sh.
@@ -225,7 +233,7 @@ __global__ void __launch_bounds__(kRowThreads) k_cp_stats(CpParams P) {
   if (c == 0) rope_heads<G>(P, q, b, g, L, cs, sn);
   if (!P.is_ret[g]) return;
   if (c == 0) {   // the rank's round-1 histogram row of this slice, filled by the next phase
-    unsigned long long* h1 = P.hist1 + ((size_t)P.rank * P.n_slices + s) * kBins1;
+    unsigned long long* h1 = P.hist1 + xrow(P, P.rank, s) * kBins1;
     for (int i = tid; i < kBins1; i += kRowThreads) h1[i] = 0ull;
   }
   qidx_heads<G>(P, q, g, qsm);
@@ -264,7 +272,7 @@ __global__ void __launch_bounds__(kRowThreads) k_cp_stats(CpParams P) {
   if (tid < G) {
     float M = -INFINITY, Z = 0.f;
     for (int w = 0; w < kRowWarps; ++w) merge_mz(M, Z, wred[w][tid].x, wred[w][tid].y);
-    P.stats[(((size_t)P.rank * P.n_slices + s) * P.n_chunks + c) * G + tid] = make_float2(M, Z);
+    P.stats[(xrow(P, P.rank, s) * P.n_chunks + c) * G + tid] = make_float2(M, Z);
   }
 }
 
@@ -290,8 +298,8 @@ __global__ void __launch_bounds__(kRowThreads) k_cp_mass(CpParams P) {
   const long long n = local_rows(P, L);
   for (int i = tid; i < kBins1; i += kRowThreads) { hc[i] = 0u; hl[i] = 0u; }
   if (c == 0) {   // the rank's round-2 and round-3 rows of this slice, filled by later phases
-    unsigned long long* h2 = P.hist2 + ((size_t)P.rank * P.n_slices + s) * kBins2;
-    unsigned long long* h3 = P.hist3 + ((size_t)P.rank * P.n_slices + s) * kBins3 * 2;
+    unsigned long long* h2 = P.hist2 + xrow(P, P.rank, s) * kBins2;
+    unsigned long long* h3 = P.hist3 + xrow(P, P.rank, s) * kBins3 * 2;
     for (int i = tid; i < kBins2; i += kRowThreads) h2[i] = 0ull;
     if (tid < kBins3 * 2) h3[tid] = 0ull;
   }
@@ -305,7 +313,7 @@ __global__ void __launch_bounds__(kRowThreads) k_cp_mass(CpParams P) {
     float m = -INFINITY, z = 0.f;
     for (int e = sub * 32 + lane; e < E; e += kWph * 32) {
       const int r = e / P.n_chunks, cc = e % P.n_chunks;
-      const float2 v = P.stats[(((size_t)r * P.n_slices + s) * P.n_chunks + cc) * G + h];
+      const float2 v = P.stats[(xrow(P, r, s) * P.n_chunks + cc) * G + h];
       merge_mz(m, z, v.x, v.y);
     }
 #pragma unroll
@@ -345,7 +353,7 @@ __global__ void __launch_bounds__(kRowThreads) k_cp_mass(CpParams P) {
     }
   }
   __syncthreads();
-  unsigned long long* dst = P.hist1 + ((size_t)P.rank * P.n_slices + s) * kBins1;
+  unsigned long long* dst = P.hist1 + xrow(P, P.rank, s) * kBins1;
   for (int d = tid; d < kBins1; d += kRowThreads) {
     const unsigned cnt = hc[d];
     if (cnt) {
@@ -393,11 +401,12 @@ __device__ void cut_desc(const unsigned long long* h, unsigned long long above, 
   __syncthreads();
 }
 
-// Sum over the ranks of a [R][n_slices][4096] histogram, slice s, into shared memory
+// Sum over the ranks of a [R][n_xrows][4096] histogram, slice s, into shared memory
 // (padded slots); returns this thread's part of the total.  Each thread keeps its 16
 // bins' loads of one rank in flight together.
-__device__ unsigned long long gather_hist4096(const unsigned long long* hist, int R, int n_slices, int s,
+__device__ unsigned long long gather_hist4096(const CpParams& P, const unsigned long long* hist, int s,
                                               unsigned long long* h) {
+  const int R = P.n_ranks;
   constexpr int PER = kBins1 / kThreads;
   const int tid = threadIdx.x;
   unsigned long long v[PER];
@@ -408,7 +417,7 @@ __device__ unsigned long long gather_hist4096(const unsigned long long* hist, in
     unsigned long long w[kRanksAtOnce][PER];
 #pragma unroll
     for (int i = 0; i < kRanksAtOnce; ++i) {
-      const unsigned long long* src = hist + ((size_t)(r0 + i) * n_slices + s) * kBins1 + tid;
+      const unsigned long long* src = hist + xrow(P, r0 + i < R ? r0 + i : 0, s) * kBins1 + tid;
 #pragma unroll
       for (int k = 0; k < PER; ++k) w[i][k] = r0 + i < R ? __ldcg(src + k * kThreads) : 0ull;
     }
@@ -436,7 +445,7 @@ __device__ unsigned long long gather_hist4096(const unsigned long long* hist, in
 __device__ void cp_cut1(const CpParams& P, int s, bool store, unsigned long long* h, unsigned long long* scratch,
                         int* sb, unsigned long long* sabove, unsigned long long* starget) {
   const int tid = threadIdx.x;
-  const unsigned long long mine = gather_hist4096(P.hist1, P.n_ranks, P.n_slices, s, h);
+  const unsigned long long mine = gather_hist4096(P, P.hist1, s, h);
   const unsigned long long total = block_sum<unsigned long long>(mine, scratch);   // (barrier: h complete)
   unsigned long long target = (unsigned long long)ceil((double)P.p * (double)total);
   if (target < 1ull) target = 1ull;
@@ -463,7 +472,7 @@ __device__ void cp_cut2(const CpParams& P, int s, bool store, unsigned long long
                         unsigned long long* scratch, int* sb, unsigned long long* sabove) {
   const int tid = threadIdx.x;
   const unsigned long long above = *sabove;
-  gather_hist4096(P.hist2, P.n_ranks, P.n_slices, s, h);
+  gather_hist4096(P, P.hist2, s, h);
   if (tid == 0) *sb = -1;
   __syncthreads();
   cut_desc<kBins2, true>(h, above, target, sb, sabove, scratch);
@@ -491,7 +500,7 @@ __device__ void cp_cut3(const CpParams& P, int s, bool store, unsigned long long
   if (tid < kBins3) {
     unsigned long long v = 0ull, k = 0ull;
     for (int r = 0; r < R; ++r) {
-      const unsigned long long* e = P.hist3 + (((size_t)r * P.n_slices + s) * kBins3 + tid) * 2;
+      const unsigned long long* e = P.hist3 + (xrow(P, r, s) * kBins3 + tid) * 2;
       v += __ldcg(e);
       k += __ldcg(e + 1);
     }
@@ -510,8 +519,8 @@ __device__ void cp_cut3(const CpParams& P, int s, bool store, unsigned long long
     const unsigned long long need = target > *sabove ? target - *sabove : 0ull;
     const unsigned long long ties = mt ? (need + mt - 1ull) / mt : cnt3[b3];
     unsigned long long before = 0ull;
-    for (int r = 0; r < P.rank; ++r) before += __ldcg(P.hist3 + (((size_t)r * P.n_slices + s) * kBins3 + b3) * 2 + 1);
-    const unsigned long long mine = __ldcg(P.hist3 + (((size_t)P.rank * P.n_slices + s) * kBins3 + b3) * 2 + 1);
+    for (int r = 0; r < P.rank; ++r) before += __ldcg(P.hist3 + (xrow(P, r, s) * kBins3 + b3) * 2 + 1);
+    const unsigned long long mine = __ldcg(P.hist3 + (xrow(P, P.rank, s) * kBins3 + b3) * 2 + 1);
     unsigned long long q = ties > before ? ties - before : 0ull;
     if (q > mine) q = mine;
     *stau = tau;
@@ -588,11 +597,11 @@ __global__ void __launch_bounds__(kThreads) k_cp_hist(CpParams P, int round) {
   if (round == 3 && tid < kBins3) P.tab3[((size_t)s * P.n_chunks + c) * kBins3 + tid] = hn[tid];
   if (!cta_any) return;
   if (round == 2) {
-    unsigned long long* dst = P.hist2 + ((size_t)P.rank * P.n_slices + s) * kBins2;
+    unsigned long long* dst = P.hist2 + xrow(P, P.rank, s) * kBins2;
     for (int d = tid; d < kBins2; d += kThreads)
       if (hm[d]) atomicAdd(dst + d, hm[d]);
   } else if (tid < kBins3 && hn[tid]) {
-    unsigned long long* e = P.hist3 + (((size_t)P.rank * P.n_slices + s) * kBins3 + tid) * 2;
+    unsigned long long* e = P.hist3 + (xrow(P, P.rank, s) * kBins3 + tid) * 2;
     atomicAdd(e, hm[tid]);
     atomicAdd(e + 1, (unsigned long long)hn[tid]);
   }

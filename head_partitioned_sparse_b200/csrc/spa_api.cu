@@ -330,8 +330,10 @@ spa_status decode_compact_with(spa_ctx* h, const void* q_pre, const void* k_ret,
 // ---------------------------------------------------------------- context-parallel
 constexpr int kMaxRanks = 1024;
 
-size_t cp_stats_bytes(const spa_ctx* h, int B, int R, int n_chunks) {
-  return (size_t)R * B * h->cfg.n_kv_heads * n_chunks * h->G * sizeof(float2);
+int count_retrieval(const spa_ctx* h, const uint8_t* head_mask) {
+  int n = 0;
+  for (int g = 0; g < h->cfg.n_kv_heads; ++g) n += head_mask[g] ? 1 : 0;
+  return n;
 }
 
 spa_status cp_check(spa_ctx* h, const spa_cp_args* a, spa::CpParams* C) {
@@ -339,9 +341,12 @@ spa_status cp_check(spa_ctx* h, const spa_cp_args* a, spa::CpParams* C) {
   if (!a) return fail(SPA_ERR_INVALID_ARG, "args is NULL");
   if (h->cfg.kv_dtype != SPA_BF16) return fail(SPA_ERR_UNSUPPORTED, "context-parallel decode needs bf16 caches");
   if (h->cfg.max_ctx < 64) return fail(SPA_ERR_INVALID_ARG, "context-parallel decode needs max_ctx >= 64");
-  if (!a->q_pre || !a->k_cache || !a->v_cache || !a->idx_cache || !a->head_mask || !a->seq_lens || !a->stats ||
-      !a->hist1 || !a->hist2 || !a->hist3 || !a->out_all || !a->lse_all)
-    return fail(SPA_ERR_INVALID_ARG, "every pointer of spa_cp_args except sel_count_opt must be non-NULL");
+  if (!a->q_pre || !a->k_cache || !a->v_cache || !a->idx_cache || !a->head_mask || !a->seq_lens || !a->out_all ||
+      !a->lse_all)
+    return fail(SPA_ERR_INVALID_ARG, "q_pre, the caches, head_mask, seq_lens, out_all and lse_all must be non-NULL");
+  const int n_ret = count_retrieval(h, a->head_mask);
+  if (n_ret > 0 && (!a->stats || !a->hist1 || !a->hist2 || !a->hist3))
+    return fail(SPA_ERR_INVALID_ARG, "stats, hist1, hist2 and hist3 must be non-NULL when a head is a retrieval head");
   if (!aligned16(a->q_pre) || !aligned16(a->k_cache) || !aligned16(a->v_cache) || !aligned16(a->idx_cache) ||
       !aligned16(a->stats) || !aligned16(a->hist1) || !aligned16(a->hist2) || !aligned16(a->hist3) ||
       !aligned16(a->out_all) || !aligned16(a->lse_all) || ((uintptr_t)a->seq_lens & 7u) ||
@@ -363,7 +368,11 @@ spa_status cp_check(spa_ctx* h, const spa_cp_args* a, spa::CpParams* C) {
                 (long long)a->pos0, (long long)cap);
   std::memset(C, 0, sizeof *C);
   const int Hkv = h->cfg.n_kv_heads;
-  for (int g = 0; g < Hkv; ++g) C->is_ret[g] = a->head_mask[g] ? 1 : 0;
+  for (int g = 0; g < Hkv; ++g) {
+    C->is_ret[g] = a->head_mask[g] ? 1 : 0;
+    C->ret_ord[g] = C->is_ret[g] ? (signed char)C->n_ret++ : (signed char)-1;
+  }
+  C->n_xrows = a->B * C->n_ret;
   C->q_pre = a->q_pre;
   C->idx = static_cast<const uint16_t*>(a->idx_cache);
   C->seq_lens = a->seq_lens;
@@ -785,16 +794,17 @@ spa_status spa_prefill(spa_handle h, const void* q_chunk, const void* k_cache, c
   });
 }
 
-spa_status spa_cp_exchange_sizes(spa_handle h, int B, int n_ranks, size_t* bytes) {
-  if (!h || !bytes) return fail(SPA_ERR_INVALID_ARG, "NULL argument");
+spa_status spa_cp_exchange_sizes(spa_handle h, int B, int n_ranks, const uint8_t* head_mask, size_t* bytes) {
+  if (!h || !head_mask || !bytes) return fail(SPA_ERR_INVALID_ARG, "NULL argument");
   if (B < 1 || B > h->cfg.max_batch)
     return fail(SPA_ERR_INVALID_ARG, "B must be in [1, max_batch=%d] (got %d)", h->cfg.max_batch, B);
   if (n_ranks < 1 || n_ranks > kMaxRanks) return fail(SPA_ERR_INVALID_ARG, "n_ranks must be in [1, %d]", kMaxRanks);
-  const size_t slices = (size_t)B * h->cfg.n_kv_heads, rows = (size_t)B * h->cfg.n_q_heads;
-  bytes[0] = cp_stats_bytes(h, B, n_ranks, h->n_chunks_max);
-  bytes[1] = (size_t)n_ranks * slices * spa::kBins1 * 8;
-  bytes[2] = (size_t)n_ranks * slices * spa::kBins2 * 8;
-  bytes[3] = (size_t)n_ranks * slices * spa::kBins3 * 16;
+  // histogram and statistics rows for the retrieval slices only
+  const size_t xrows = (size_t)n_ranks * B * count_retrieval(h, head_mask), rows = (size_t)B * h->cfg.n_q_heads;
+  bytes[0] = xrows * h->n_chunks_max * h->G * sizeof(float2);
+  bytes[1] = xrows * spa::kBins1 * 8;
+  bytes[2] = xrows * spa::kBins2 * 8;
+  bytes[3] = xrows * spa::kBins3 * 16;
   bytes[4] = (size_t)n_ranks * rows * spa::kHeadDim * 4;
   bytes[5] = (size_t)n_ranks * rows * 4;
   return SPA_OK;

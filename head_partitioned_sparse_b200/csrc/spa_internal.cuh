@@ -85,6 +85,9 @@ struct CpParams {
   const uint16_t* idx;            // local index rows [Bm][Hkv][C][16]
   const int64_t* seq_lens;        // [B] global sequence lengths
   int B, Hq, Hkv, G, n_slices;
+  int n_xrows;                    // exchange rows per rank: B * (retrieval KV heads)
+  int n_ret;                      // retrieval KV heads
+  signed char ret_ord[kMaxKvHeads];   // ordinal of KV head g among the retrieval heads (-1: streaming)
   int64_t C;                      // local row capacity (row stride of the local caches)
   int n_chunks;                   // ceil(C / kChunk): chunks of a slice's local rows
   int64_t pos0;                   // global position of local row 0
@@ -101,10 +104,12 @@ struct CpParams {
   float* q_idx;                   // [Bm][Hq][16]
   float* pi;                      // [Bm*Hkv][pi_stride] local probabilities
   int64_t pi_stride;
-  float2* stats;                  // exchange: [R][n_slices][n_chunks][G] (m in log2 units, z)
-  unsigned long long* hist1;      // exchange: [R][n_slices][kBins1] masses
-  unsigned long long* hist2;      // exchange: [R][n_slices][kBins2] masses
-  unsigned long long* hist3;      // exchange: [R][n_slices][kBins3][2] (mass, count)
+  // Exchange buffers: one row per (rank, retrieval slice), row r * n_xrows + b * n_ret
+  // + ret_ord[g]; streaming slices never write or read them.
+  float2* stats;                  // exchange: [R][n_xrows][n_chunks][G] (m in log2 units, z)
+  unsigned long long* hist1;      // exchange: [R][n_xrows][kBins1] masses
+  unsigned long long* hist2;      // exchange: [R][n_xrows][kBins2] masses
+  unsigned long long* hist3;      // exchange: [R][n_xrows][kBins3][2] (mass, count)
   unsigned* tab3;                 // [n_slices][n_chunks][kBins3] local round-3 counts per chunk
   int* chunk_cnt;                 // [n_slices][n_chunks] listed rows per chunk
   CpSlice* cs;                    // [n_slices]

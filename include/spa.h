@@ -320,8 +320,11 @@ SPA_API spa_status spa_prefill(spa_handle h, const void* q_chunk, const void* k_
  * rank's slot at index rank; a phase writes only its own slots (the histogram slots it
  * adds into are cleared by an earlier phase of the same rank: stats clears hist1, mass
  * clears hist2 and hist3) and reads the other slots, which must hold the gathered data
- * of the previous phase.
- * spa_cp_exchange_sizes gives the byte size of each buffer (all slots).  Every pointer
+ * of the previous phase.  Streaming heads never select, so stats and hist1..hist3 hold
+ * one row per retrieval slice only: slot r, row b * n_ret + j for the j-th retrieval
+ * KV head (in head order) of sequence b, n_ret the number of retrieval heads.
+ * spa_cp_exchange_sizes gives the byte size of each buffer (all slots) for a head
+ * mask; the buffers must be sized with the same mask the phases get.  Every pointer
  * is a device pointer, 16-byte aligned.  Phases and combine only enqueue work on
  * `stream`; a phase called out of order computes garbage but stays in bounds. */
 #define SPA_CP_STATS 0
@@ -345,22 +348,27 @@ typedef struct {
                                the cut are handed out rank by rank, lowest positions first) */
   int64_t max_seq_len;      /* bound on the global lengths (0: the larger of n_ranks * max_ctx
                                and pos0 + max_ctx) */
-  void* stats;              /* [n_ranks][B][Hkv][ceil(max_ctx / 4096)][G] float2 */
-  void* hist1;              /* [n_ranks][B][Hkv][4096] uint64 */
-  void* hist2;              /* [n_ranks][B][Hkv][4096] uint64 */
-  void* hist3;              /* [n_ranks][B][Hkv][64][2] uint64 */
+  void* stats;              /* [n_ranks][B][n_ret][ceil(max_ctx / 4096)][G] float2 (may be NULL, as
+                               may hist1..hist3, when head_mask has no retrieval head) */
+  void* hist1;              /* [n_ranks][B][n_ret][4096] uint64 */
+  void* hist2;              /* [n_ranks][B][n_ret][4096] uint64 */
+  void* hist3;              /* [n_ranks][B][n_ret][64][2] uint64 */
   float* out_all;           /* [n_ranks][B][Hq][128] float32 */
   float* lse_all;           /* [n_ranks][B][Hq] float32, log2 of the softmax denominator */
   int32_t* sel_count_opt;   /* NULL or device [B][Hkv]: local rows attended (SPA_CP_ATTEND) */
   int32_t* list_opt;        /* NULL or device [B][Hkv][max_ctx]: the local rows attended, ascending
                                (sinks and window included; global position = pos0 + row) */
 } spa_cp_args;
-/* bytes[i] for the SPA_CP_NBUF buffers in spa_cp_args order.  Errors: NULL handle or
- * bytes, B outside [1, max_batch], n_ranks outside [1, 1024]. */
-SPA_API spa_status spa_cp_exchange_sizes(spa_handle h, int B, int n_ranks, size_t* bytes);
+/* bytes[i] for the SPA_CP_NBUF buffers in spa_cp_args order, for the host head mask
+ * head_mask [Hkv] (1 = retrieval head; the statistics and histograms are sized for its
+ * retrieval heads, 0 bytes when it has none).  Errors: NULL handle, head_mask or bytes,
+ * B outside [1, max_batch], n_ranks outside [1, 1024]. */
+SPA_API spa_status spa_cp_exchange_sizes(spa_handle h, int B, int n_ranks, const uint8_t* head_mask,
+                                         size_t* bytes);
 /* Runs one phase on this rank.  Errors: SPA_ERR_INVALID_ARG for a NULL or misaligned
- * pointer, an unknown phase, B / p / n_sink / window / rank / pos0 out of range, or
- * max_ctx < 64; SPA_ERR_UNSUPPORTED for float32 caches. */
+ * pointer (stats and hist1..hist3 may be NULL only without retrieval heads), an
+ * unknown phase, B / p / n_sink / window / rank / pos0 out of range, or max_ctx < 64;
+ * SPA_ERR_UNSUPPORTED for float32 caches. */
 SPA_API spa_status spa_cp_phase(spa_handle h, int phase, const spa_cp_args* a, spa_stream stream);
 /* out[b][h] = sum_r 2^(lse_r - M) out_r / sum_r 2^(lse_r - M), M = max_r lse_r, over
  * the gathered out_all / lse_all (ranks in order; a rank with lse = -inf attended

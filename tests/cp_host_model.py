@@ -1,9 +1,10 @@
 """A host model of the context-parallel phases, for the CPU tests of the exchange logic.
 
 It runs the same phase sequence as libspa's context-parallel kernels and reads and
-writes the same exchange-buffer layouts (byte tensors: stats [R][S][n_chunks][G] float
-pairs, hist1/hist2 [R][S][4096] uint64, hist3 [R][S][64][2] uint64, out_all
-[R][B][Hq][128] and lse_all [R][B][Hq] float32), in float64 NumPy, so that the
+writes the same exchange-buffer layouts (byte tensors: stats [R][X][n_chunks][G] float
+pairs, hist1/hist2 [R][X][4096] uint64, hist3 [R][X][64][2] uint64, with X = B * n_ret
+rows, one per retrieval slice, sequence-major; out_all [R][B][Hq][128] and lse_all
+[R][B][Hq] float32), in float64 NumPy, so that the
 orchestration in ``head_partitioned_sparse_b200.context_parallel`` and the gloo
 all-gathers can be tested without a GPU, and so that the phase decomposition itself
 (merging per-rank softmax statistics, exact integer histograms summed over ranks, the
@@ -26,10 +27,11 @@ def n_chunks(C: int) -> int:
     return -(-C // CHUNK)
 
 
-def exchange_sizes(B: int, Hq: int, Hkv: int, C: int, R: int):
-    """Byte sizes of the exchange buffers (the layout spa_cp_exchange_sizes reports)."""
-    G, S = Hq // Hkv, B * Hkv
-    return (R * S * n_chunks(C) * G * 8, R * S * BINS1 * 8, R * S * BINS2 * 8, R * S * BINS3 * 16,
+def exchange_sizes(B: int, Hq: int, Hkv: int, C: int, R: int, head_mask):
+    """Byte sizes of the exchange buffers (the layout spa_cp_exchange_sizes reports):
+    statistics and histograms for the retrieval slices only."""
+    G, X = Hq // Hkv, B * int(sum(1 for v in head_mask if v))
+    return (R * X * n_chunks(C) * G * 8, R * X * BINS1 * 8, R * X * BINS2 * 8, R * X * BINS3 * 16,
             R * B * Hq * 128 * 4, R * B * Hq * 4)
 
 
@@ -60,17 +62,20 @@ class HostRank:
         self.inp, self.rank, self.R, self.C = inp, rank, R, C
         self.p, self.n_sink, self.window = p, n_sink, window
         self.G = inp.Hq // inp.Hkv
-        self.S = inp.B * inp.Hkv
+        # exchange row of slice (b, g): b * n_ret + (ordinal of g among the retrieval heads)
+        ret = [g for g in range(inp.Hkv) if inp.head_mask[g]]
+        self.X = inp.B * len(ret)
+        self.xrow = {b * inp.Hkv + g: b * len(ret) + j for b in range(inp.B) for j, g in enumerate(ret)}
         self.nc = n_chunks(C)
         self.pos0 = rank * C
         self.idx = idx_bits
         self.to64 = (lambda a: O.bf16_bits_to_f64(a)) if inp.dtype == "bf16" else (
             lambda a: np.asarray(a, np.float64))
         nb = lambda name: bufs[name].numpy()
-        self.stats = nb("stats").view(np.float32).reshape(R, self.S, self.nc, self.G, 2)
-        self.h1 = nb("hist1").view(np.uint64).reshape(R, self.S, BINS1)
-        self.h2 = nb("hist2").view(np.uint64).reshape(R, self.S, BINS2)
-        self.h3 = nb("hist3").view(np.uint64).reshape(R, self.S, BINS3, 2)
+        self.stats = nb("stats").view(np.float32).reshape(R, self.X, self.nc, self.G, 2)
+        self.h1 = nb("hist1").view(np.uint64).reshape(R, self.X, BINS1)
+        self.h2 = nb("hist2").view(np.uint64).reshape(R, self.X, BINS2)
+        self.h3 = nb("hist3").view(np.uint64).reshape(R, self.X, BINS3, 2)
         self.out_all = nb("out_all").view(np.float32).reshape(R, inp.B, inp.Hq, 128)
         self.lse_all = nb("lse_all").view(np.float32).reshape(R, inp.B, inp.Hq)
         self.bits = {}
@@ -102,59 +107,62 @@ class HostRank:
         for b, g, s in self._slices():
             if not self.inp.head_mask[g]:
                 continue
-            lg = self._logits(b, g)
+            lg, x = self._logits(b, g), self.xrow[s]
             for c in range(self.nc):
                 part = lg[c * CHUNK:(c + 1) * CHUNK]
                 if len(part) == 0:
-                    self.stats[self.rank, s, c, :, 0] = -np.inf
-                    self.stats[self.rank, s, c, :, 1] = 0.0
+                    self.stats[self.rank, x, c, :, 0] = -np.inf
+                    self.stats[self.rank, x, c, :, 1] = 0.0
                     continue
                 m = part.max(axis=0)
-                self.stats[self.rank, s, c, :, 0] = m
-                self.stats[self.rank, s, c, :, 1] = np.exp2(part - m).sum(axis=0)
+                self.stats[self.rank, x, c, :, 0] = m
+                self.stats[self.rank, x, c, :, 1] = np.exp2(part - m).sum(axis=0)
 
     def mass_phase(self):
         self.h1[self.rank] = 0
         for b, g, s in self._slices():
             if not self.inp.head_mask[g]:
                 continue
-            st = self.stats[:, s].reshape(-1, self.G, 2).astype(np.float64)   # all ranks, all chunks
+            x = self.xrow[s]
+            st = self.stats[:, x].reshape(-1, self.G, 2).astype(np.float64)   # all ranks, all chunks
             m, z = st[..., 0], st[..., 1]
             M = m.max(axis=0)
             Z = np.where(np.isfinite(m), z * np.exp2(m - M), 0.0).sum(axis=0)
             pi = (np.exp2(self._logits(b, g) - M) / (self.G * Z)).sum(axis=1).astype(np.float32)
             u = pi.view(np.uint32)
             self.bits[s] = u
-            np.add.at(self.h1[self.rank, s], (u >> 18).astype(np.int64), mass_q(u))
+            np.add.at(self.h1[self.rank, x], (u >> 18).astype(np.int64), mass_q(u))
 
     def round2(self):
         self.h2[self.rank] = 0
         for b, g, s in self._slices():
             if not self.inp.head_mask[g]:
                 continue
-            total = sum(int(v) for v in self.h1[:, s].sum(axis=0, dtype=np.uint64))
+            x = self.xrow[s]
+            total = sum(int(v) for v in self.h1[:, x].sum(axis=0, dtype=np.uint64))
             target = max(1, math.ceil(float(np.float32(self.p)) * float(total)))
             if self.p >= 1.0 or target > total:
                 self.cut[s] = dict(b1=-1)
                 continue
-            b1, above = cut_desc(self.h1[:, s].sum(axis=0, dtype=np.uint64), 0, target)
+            b1, above = cut_desc(self.h1[:, x].sum(axis=0, dtype=np.uint64), 0, target)
             self.cut[s] = dict(b1=b1, above=above, target=target)
             u = self.bits[s]
             sel = (u >> 18) == b1
-            np.add.at(self.h2[self.rank, s], ((u[sel] >> 6) & 0xFFF).astype(np.int64), mass_q(u[sel]))
+            np.add.at(self.h2[self.rank, x], ((u[sel] >> 6) & 0xFFF).astype(np.int64), mass_q(u[sel]))
 
     def round3(self):
         self.h3[self.rank] = 0
         for s, cs in self.cut.items():
             if cs["b1"] < 0:
                 continue
-            b2, above = cut_desc(self.h2[:, s].sum(axis=0, dtype=np.uint64), cs["above"], cs["target"])
+            x = self.xrow[s]
+            b2, above = cut_desc(self.h2[:, x].sum(axis=0, dtype=np.uint64), cs["above"], cs["target"])
             cs.update(b2=b2, above=above)
             u = self.bits[s]
             sel = (u >> 6) == ((cs["b1"] << 12) | b2)
             d = (u[sel] & 0x3F).astype(np.int64)
-            np.add.at(self.h3[self.rank, s, :, 0], d, mass_q(u[sel]))
-            np.add.at(self.h3[self.rank, s, :, 1], d, np.uint64(1))
+            np.add.at(self.h3[self.rank, x, :, 0], d, mass_q(u[sel]))
+            np.add.at(self.h3[self.rank, x, :, 1], d, np.uint64(1))
 
     def attend(self):
         inp = self.inp
@@ -170,13 +178,14 @@ class HostRank:
                 if cs["b1"] < 0:
                     keep[:] = True
                 else:
-                    b3, above = cut_desc(self.h3[:, s, :, 0].sum(axis=0, dtype=np.uint64), cs["above"],
+                    x = self.xrow[s]
+                    b3, above = cut_desc(self.h3[:, x, :, 0].sum(axis=0, dtype=np.uint64), cs["above"],
                                          cs["target"])
                     tau = (cs["b1"] << 18) | (cs["b2"] << 6) | b3
                     mt = int(mass_q(np.array([tau], np.uint32))[0])
                     ties = -(-(cs["target"] - above) // mt)
-                    before = sum(int(self.h3[r, s, b3, 1]) for r in range(self.rank))
-                    quota = min(max(ties - before, 0), int(self.h3[self.rank, s, b3, 1]))
+                    before = sum(int(self.h3[r, x, b3, 1]) for r in range(self.rank))
+                    quota = min(max(ties - before, 0), int(self.h3[self.rank, x, b3, 1]))
                     u = self.bits[s].astype(np.int64)
                     eq = u == tau
                     keep |= (u > tau) | (eq & (np.cumsum(eq) - 1 < quota))

@@ -107,7 +107,7 @@ def test_create_without_device_fails_loudly(lib):
 
 
 def test_context_parallel_calls_reject_a_null_handle(lib):
-    for call in (lambda: B.spa_cp_exchange_sizes(None, 1, 2),
+    for call in (lambda: B.spa_cp_exchange_sizes(None, 1, 2, [1, 0]),
                  lambda: B.spa_cp_combine(None, 16, 16, 2, 1, 16, stream=0),
                  lambda: B.spa_cp_phase(None, B.SPA_CP_STATS, B.make_cp_args(
                      q_pre=16, k_cache=16, v_cache=16, idx_cache=16, head_mask=[1, 0], seq_lens=16, B=1, p=0.9,

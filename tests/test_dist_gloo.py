@@ -129,12 +129,39 @@ def test_cp_phases_emulated_in_one_process_match_the_oracle(R, p):
     pp = inp.p if p is None else float(np.float32(p))
     C = -(-int(inp.seq_lens.max()) // R)
     bufs = {n: torch.zeros(sz, dtype=torch.uint8) for n, sz in
-            zip(cp.BUFFERS, M.exchange_sizes(inp.B, inp.Hq, inp.Hkv, C, R))}
+            zip(cp.BUFFERS, M.exchange_sizes(inp.B, inp.Hq, inp.Hkv, C, R, inp.head_mask))}
     ranks = [M.HostRank(inp, idx, r, R, C, bufs, p=pp, n_sink=inp.n_sink, window=inp.window) for r in range(R)]
     cp.run_step(range(R), lambda ph, r: ranks[r].phase(ph), lambda name: None)
     out = M.combine(ranks[0].out_all, ranks[0].lse_all)
     rows = {k: np.concatenate([rk.rows[k] for rk in ranks]) for k in ranks[0].rows}
     assert _cp_check(inp, idx, out, rows, p=pp) <= 1e-5
+
+
+@pytest.mark.parametrize("retrieval", [[1, 3], [0, 1, 2, 3], [2], []])
+def test_cp_exchange_rows_are_the_retrieval_slices_only(retrieval):
+    """The statistics and histograms hold one row per retrieval slice (streaming heads
+    never select): sizes scale with the retrieval heads, and the phases still reach the
+    oracle's sets with retrieval heads anywhere in the head order, all of them, or none
+    (nothing exchanged but the outputs)."""
+    import torch
+    import cp_host_model as M
+    import oracle as O
+    from head_partitioned_sparse_b200 import context_parallel as cp
+    from head_partitioned_sparse_b200 import synth
+    inp = synth.make_inputs("tiny", 6, overrides={"B": 2, "Hq": 16, "Hkv": 4, "retrieval": retrieval, "L": 6000,
+                                                   "window": 64, "p": 0.9}, seq_lens=[6000, 2500])
+    idx = O.index_cache_for(inp, heads=retrieval)
+    R, C = 3, 2000
+    sizes = M.exchange_sizes(inp.B, inp.Hq, inp.Hkv, C, R, inp.head_mask)
+    every = M.exchange_sizes(inp.B, inp.Hq, inp.Hkv, C, R, [1] * inp.Hkv)
+    assert all(sizes[i] * inp.Hkv == every[i] * len(retrieval) for i in range(4))
+    assert sizes[4:] == every[4:]
+    bufs = {n: torch.zeros(sz, dtype=torch.uint8) for n, sz in zip(cp.BUFFERS, sizes)}
+    ranks = [M.HostRank(inp, idx, r, R, C, bufs, p=inp.p, n_sink=inp.n_sink, window=inp.window) for r in range(R)]
+    cp.run_step(range(R), lambda ph, r: ranks[r].phase(ph), lambda name: None)
+    out = M.combine(ranks[0].out_all, ranks[0].lse_all)
+    rows = {k: np.concatenate([rk.rows[k] for rk in ranks]) for k in ranks[0].rows}
+    assert _cp_check(inp, idx, out, rows) <= 1e-5
 
 
 def _cp_worker(rank, world, port, q):
@@ -151,7 +178,7 @@ def _cp_worker(rank, world, port, q):
         dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
         inp, idx = _cp_inputs()
         bufs = {n: torch.zeros(sz, dtype=torch.uint8) for n, sz in
-                zip(cp.BUFFERS, M.exchange_sizes(inp.B, inp.Hq, inp.Hkv, CP_C, world))}
+                zip(cp.BUFFERS, M.exchange_sizes(inp.B, inp.Hq, inp.Hkv, CP_C, world, inp.head_mask))}
         me = M.HostRank(inp, idx, rank, world, CP_C, bufs, p=inp.p, n_sink=inp.n_sink, window=inp.window)
         cp.run_step([rank], lambda ph, r: me.phase(ph), lambda name: cp.allgather_slot(bufs[name], world, rank))
         out = M.combine(me.out_all, me.lse_all)
@@ -167,7 +194,7 @@ def _cp_worker(rank, world, port, q):
             same = all(np.array_equal(np.asarray(o), out) for o in outs)
             # the same phases emulated in one process give the same bits
             ebufs = {n: torch.zeros(sz, dtype=torch.uint8) for n, sz in
-                     zip(cp.BUFFERS, M.exchange_sizes(inp.B, inp.Hq, inp.Hkv, CP_C, world))}
+                     zip(cp.BUFFERS, M.exchange_sizes(inp.B, inp.Hq, inp.Hkv, CP_C, world, inp.head_mask))}
             er = [M.HostRank(inp, idx, r, world, CP_C, ebufs, p=inp.p, n_sink=inp.n_sink, window=inp.window)
                   for r in range(world)]
             cp.run_step(range(world), lambda ph, r: er[r].phase(ph), lambda name: None)
@@ -214,7 +241,7 @@ def test_cp_phases_ties_across_ranks_go_to_the_lowest_positions():
     idx[0, 0, :1000] = idx[0, 0, 500]
     R, C = 3, 400
     bufs = {n: torch.zeros(sz, dtype=torch.uint8) for n, sz in
-            zip(cp.BUFFERS, M.exchange_sizes(inp.B, inp.Hq, inp.Hkv, C, R))}
+            zip(cp.BUFFERS, M.exchange_sizes(inp.B, inp.Hq, inp.Hkv, C, R, inp.head_mask))}
     ranks = [M.HostRank(inp, idx, r, R, C, bufs, p=inp.p, n_sink=inp.n_sink, window=8) for r in range(R)]
     cp.run_step(range(R), lambda ph, r: ranks[r].phase(ph), lambda name: None)
     sw = O.sink_window(1000, inp.n_sink, 8)
@@ -242,11 +269,11 @@ def _decoder_worker(rank, world, port, q):
         inp, idx = _cp_inputs()
         model = {}
         calls = []
-        spa.spa_cp_exchange_sizes = lambda h, B, R: M.exchange_sizes(B, inp.Hq, inp.Hkv, CP_C, R)
+        spa.spa_cp_exchange_sizes = lambda h, B, R, mask: M.exchange_sizes(B, inp.Hq, inp.Hkv, CP_C, R, mask)
         spa.spa_cp_phase = lambda h, phase, args, stream=None: (calls.append(phase), model["m"].phase(phase))
         spa.spa_cp_combine = lambda h, out_all, lse_all, R, B, out, stream=None: out.copy_(
             torch.from_numpy(M.combine(model["m"].out_all, model["m"].lse_all)))
-        dec = cp.ContextParallelDecoder(0, B=inp.B, capacity=CP_C, device="cpu")
+        dec = cp.ContextParallelDecoder(0, B=inp.B, capacity=CP_C, device="cpu", head_mask=inp.head_mask)
         model["m"] = M.HostRank(inp, idx, rank, world, CP_C, dec.bufs, p=inp.p, n_sink=inp.n_sink,
                                 window=inp.window)
         z = torch.zeros(16, dtype=torch.uint8)

@@ -183,6 +183,23 @@ def test_context_parallel_is_deterministic():
     assert all(np.array_equal(ra[k], rb[k]) for k in ra)
 
 
+def test_exchange_rows_are_the_retrieval_slices_only():
+    """The statistics and histograms are sized for the retrieval slices of the head mask
+    (the layout of the CPU host model of the phases); a mask without retrieval heads
+    exchanges none of them (NULL buffers are accepted) and still decodes."""
+    import cp_host_model as M
+    inp, _ = _prepare("g1")
+    with Handle(inp, max_ctx=2048) as h:
+        for mask in ([1, 0, 1, 0], [0, 0, 0, 1], [1, 1, 1, 1], [0, 0, 0, 0]):
+            got = B.spa_cp_exchange_sizes(h.h, inp.B, 3, mask)
+            assert got == M.exchange_sizes(inp.B, inp.Hq, inp.Hkv, 2048, 3, mask)
+    inp0 = synth.make_inputs("tiny", 3, overrides={"dtype": "bf16", "Hq": 4, "Hkv": 4, "L": 5000, "retrieval": []})
+    idx0 = oracle_idx(inp0, heads=[])
+    for R in (1, 3):
+        out, rows = run_cp(inp0, idx0, R)
+        check_cp(inp0, idx0, out, rows, inp0.p, inp0.n_sink, inp0.window)
+
+
 def test_context_parallel_argument_errors():
     inp, idx = _prepare("g1")
     with Handle(inp, max_ctx=2048) as h:
