@@ -689,10 +689,10 @@ def main_native(args):
         out_cp = torch.empty_like(out)
         cp_bufs = cpm.alloc_exchange(B.spa_cp_exchange_sizes(cp_handles[0], inp.B, R, head_mask), dev)
 
-        def step_cp(i, st=stream, ranks=None, combine=True):
+        def step_cp(i, st=stream, ranks=None, combine=True, exchange=None):
             cpm.emulated_step(cp_handles, shards, q_pre=q, head_mask=head_mask, seq_lens=lens, Bsz=inp.B, p=p,
                               n_sink=inp.n_sink, window=inp.window, capacity=C, out=out_cp, bufs=cp_bufs,
-                              max_seq_len=Lcap, stream=st, ranks=ranks, combine=combine)
+                              max_seq_len=Lcap, stream=st, ranks=ranks, combine=combine, exchange=exchange)
         for i in range(3):
             step_cp(i)
         for hh in cp_handles:
@@ -741,15 +741,28 @@ def main_native(args):
             torch.cuda.synchronize(dev)
             return 1e3 * a.elapsed_time(z) / reps
 
-        graph_step_us, graph_rank_us, graph_err = None, [], None
+        graph_step_us, graph_rank_us, graph_err, copy_us = None, [], None, None
         try:
             g_all = graph_of(lambda: step_cp(0, st=None))
             graph_step_us = replay_us(g_all, n)
             del g_all
+            # one rank alone: the gathered buffers' other slots hold the full step's data;
+            # the summed histograms get the full step's sums back after the phase that
+            # adds into them (the all-reduce of a real step), and that copy's own time,
+            # from a graph of the copies alone, is taken off the rank's time
+            totals = {nm: cp_bufs[nm].clone() for nm in cpm.SUMMED}
+
+            def restore(name):
+                if name in totals:
+                    cp_bufs[name].copy_(totals[name])
+            g_c = graph_of(lambda: [restore(nm) for nm in cpm.SUMMED])
+            copy_us = replay_us(g_c, n)
+            del g_c
             for r in range(R):
-                g_r = graph_of(lambda: step_cp(0, st=None, ranks=[r], combine=False))
-                graph_rank_us.append(replay_us(g_r, n))
+                g_r = graph_of(lambda: step_cp(0, st=None, ranks=[r], combine=False, exchange=restore))
+                graph_rank_us.append(replay_us(g_r, n) - copy_us)
                 del g_r
+            del totals
         except Exception as e:   # reported, not fatal: the step itself was timed above
             graph_err = repr(e)[:200]
         step_cp(0)
@@ -758,14 +771,20 @@ def main_native(args):
         cpar = {"ranks": R, "rows_per_rank": C, "emulated_step_ms": ms_cp,
                 "graph_step_us": graph_step_us, "graph_rank_us": graph_rank_us,
                 "max_graph_rank_us": max(graph_rank_us) if graph_rank_us else None, "graph_error": graph_err,
+                "rank_graph_sum_copy_us": copy_us,
                 "rank_kernel_us": rank_us, "rank_select_us": sel_us, "rank_attend_us": att_us,
                 "max_rank_kernel_us": max(rank_us), "combine_us": 1e3 * tc / n,
-                "exchange_bytes_per_rank": int(sum(sizes) // R),
+                "exchange_bytes_per_rank": int(sum(sz // (1 if nm in cpm.SUMMED else R)
+                                                   for nm, sz in zip(cpm.BUFFERS, sizes))),
                 "one_gpu_step_ms": ms_per_step,
                 "max_abs_vs_one_gpu": float((out_cp - out).abs().max().item()),
                 "note": "ranks emulated on one GPU one after another, exchanges not timed (buffers shared); "
                         "rank_*_us: CUDA events around each launch of a Python-driven step (host gaps "
-                        "included); graph_*_us: the same launches replayed from a CUDA graph (device time)"}
+                        "included); graph_*_us: the same launches replayed from a CUDA graph (device time; "
+                        "graph_rank_us: one rank's launches alone, the summed histograms set to the full "
+                        "step's sums after the phase that adds into them and that copy's time taken off); "
+                        "exchange_bytes_per_rank: the rank's slot of each gathered buffer plus the whole of "
+                        "each all-reduced one"}
         for hh in cp_handles:
             B.spa_destroy(hh)
         del shards, cp_bufs, out_cp

@@ -3,18 +3,19 @@ across ranks (host orchestration of the ``spa_cp_*`` phases of libspa).
 
 Rank r holds positions [r C, (r + 1) C) of every sequence in its own caches (C = its
 handle's ``max_ctx``; every rank's handle has the same configuration).  A step is the
-five phases of ``spa_cp_phase``, each followed by an all-gather of the slot the rank
-wrote in one exchange buffer, then ``spa_cp_combine``:
+five phases of ``spa_cp_phase``, each followed by the exchange of the buffer it wrote,
+then ``spa_cp_combine``:
 
     phase          exchanged after it
-    SPA_CP_STATS   stats     per-head (max, sum of exp) of the local index scores
-    SPA_CP_MASS    hist1     round-1 mass histogram of the local probabilities
-    SPA_CP_ROUND2  hist2     round-2 histogram inside the round-1 cut bin
-    SPA_CP_ROUND3  hist3     round-3 histogram with counts (ties go rank by rank)
-    SPA_CP_ATTEND  out_all, lse_all   the rank's attention output and log2-sum-exp
+    SPA_CP_STATS   stats     all-gather: per-head (max, sum of exp) of the local scores
+    SPA_CP_MASS    hist1     all-reduce: round-1 mass histogram of the probabilities
+    SPA_CP_ROUND2  hist2     all-reduce: round-2 histogram inside the round-1 cut bin
+    SPA_CP_ROUND3  hist3     all-gather: round-3 histogram with counts (ties go rank by rank)
+    SPA_CP_ATTEND  out_all, lse_all   all-gather: the rank's output and log2-sum-exp
 
-The statistics and histograms have rows for the retrieval slices only (streaming heads
-never select), so the buffers are sized for one head mask.
+The histograms hold integer masses, so the all-reduced sums are exact.  The statistics
+and histograms have rows for the retrieval slices only (streaming heads never select),
+so the buffers are sized for one head mask.
 
 Two drivers share that sequence (``run_step``):
   * ``ContextParallelDecoder``: one process per GPU; the exchange is
@@ -58,6 +59,28 @@ def run_step(ranks: Iterable[int], run_phase: Callable[[int, int], None], exchan
 def rank_span(rank: int, capacity: int) -> Tuple[int, int]:
     """Global positions [pos0, pos0 + capacity) held by ``rank`` in the contiguous split."""
     return rank * capacity, (rank + 1) * capacity
+
+
+# buffers summed over the ranks (all-reduce); the others have a slot per rank (all-gather)
+SUMMED = ("hist1", "hist2")
+
+
+def allreduce_sum(buf, group=None) -> None:
+    """All-reduce (sum) of a buffer of uint64 words, done as int64: two's complement
+    addition is unsigned addition modulo 2^64, so the bits are the unsigned sum."""
+    import torch
+    import torch.distributed as dist
+    if buf.numel() == 0:   # no retrieval head: nothing to exchange (the same on every rank)
+        return
+    dist.all_reduce(buf.view(torch.int64), op=dist.ReduceOp.SUM, group=group)
+
+
+def exchange_buffer(bufs, name: str, n_ranks: int, rank: int, group=None) -> None:
+    """The exchange of buffer ``name`` after the phase that wrote it."""
+    if name in SUMMED:
+        allreduce_sum(bufs[name], group)
+    else:
+        allgather_slot(bufs[name], n_ranks, rank, group)
 
 
 def allgather_slot(buf, n_ranks: int, rank: int, group=None) -> None:
@@ -124,19 +147,21 @@ class ContextParallelDecoder:
                               hist3=self.bufs["hist3"], out_all=out_all, lse_all=lse_all,
                               sel_count_opt=sel_count, list_opt=list_out)
         run_step([self.rank], lambda phase, r: spa.spa_cp_phase(self.h, phase, args),
-                 lambda name: allgather_slot(self.bufs[name], self.n_ranks, self.rank, self.group))
+                 lambda name: exchange_buffer(self.bufs, name, self.n_ranks, self.rank, self.group))
         spa.spa_cp_combine(self.h, out_all, lse_all, self.n_ranks, self.B, out)
 
 
 def emulated_step(handles: Sequence, shards: Sequence[dict], *, q_pre, head_mask, seq_lens, Bsz: int, p: float,
                   n_sink: int, window: int, capacity: int, out, bufs=None, max_seq_len: int = 0,
                   sel_counts: Sequence = None, lists: Sequence = None, stream=None, ranks: Sequence[int] = None,
-                  combine: bool = True) -> dict:
+                  combine: bool = True, exchange: Callable[[str], None] = None) -> dict:
     """All ranks of a context-parallel step on one GPU: handles[r] and shards[r] (dict of
     ``k``, ``v``, ``idx`` device tensors) are rank r's.  Returns the exchange buffers
-    (reusable for the next call through ``bufs``, with the same ``head_mask``).  ``ranks`` restricts the phases to
-    some ranks (to time one rank's share: the other slots of ``bufs`` must then hold an
-    earlier step's exchanged data); ``combine=False`` skips the final merge."""
+    (reusable for the next call through ``bufs``, with the same ``head_mask``).
+    ``ranks`` restricts the phases to some ranks (to time one rank's share: the other
+    slots of ``bufs`` must then hold an earlier step's exchanged data, and ``exchange``,
+    called with each buffer's name after the phase that wrote it, must put the sums
+    over all ranks into the summed buffers); ``combine=False`` skips the final merge."""
     R = len(handles)
     if bufs is None:
         bufs = alloc_exchange(spa.spa_cp_exchange_sizes(handles[0], Bsz, R, head_mask), q_pre.device)
@@ -152,7 +177,7 @@ def emulated_step(handles: Sequence, shards: Sequence[dict], *, q_pre, head_mask
             sel_count_opt=None if sel_counts is None else sel_counts[r],
             list_opt=None if lists is None else lists[r]))
     run_step(range(R) if ranks is None else ranks, lambda phase, r: spa.spa_cp_phase(handles[r], phase, args[r], stream),
-             lambda name: None)
+             exchange or (lambda name: None))
     if combine:
         spa.spa_cp_combine(handles[0], out_all, lse_all, R, Bsz, out, stream)
     return bufs

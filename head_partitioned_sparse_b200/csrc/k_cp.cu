@@ -1,6 +1,6 @@
 // Context-parallel decode: the positions of every sequence are split over ranks (rank r
 // holds the contiguous run [pos0, pos0 + C) in its own caches), and one decode step runs
-// as phases of local launches with a small all-gather between them.
+// as phases of local launches with a small exchange between them.
 //
 // What is computed is the selection and attention of the one-GPU step:
 //   "Full Attention Strikes Back" (RTPurbo summary), Methodology §2 (index scores in a
@@ -10,16 +10,17 @@
 //   the context-parallel scaling of the "Lighthouse Attention" summary, Experimental
 //   results (1M tokens on 32 GPUs).
 //
-// Phases (per rank; the exchange after each one is an all-gather of the rank's slot; the
-// histogram rows a phase adds into were cleared by an earlier phase of the same rank):
+// Phases (per rank; after each one an exchange: an all-gather of the rank's slot of
+// stats, hist3 and the outputs, an all-reduce (sum) of hist1 and hist2; the histogram
+// rows a phase adds into were cleared by an earlier phase of the same rank):
 //   stats   q_rot = RoPE(q_pre, L-1); q_idx = P_q q_pre (float64 dots); per chunk of
 //           local rows and head h: m = max_j l_hj, z = sum_j 2^(l_hj - m),
 //           l_hj = log2(e) idx_scale <q_idx[h], idx_j>                    -> stats[rank]
 //   mass    every rank merges all ranks' (m, z) in the same order -> (M_h, Z_h);
 //           pi_j = sum_h 2^(l_hj - M_h) / (G Z_h) (fp32, kept locally); masses of the
-//           round-1 digit (bits 31..18 of pi's pattern)                  -> hist1[rank]
+//           round-1 digit (bits 31..18 of pi's pattern)                  -> hist1 (summed)
 //   round 2 cut 1 over the summed round-1 histogram (target ceil(p * total)); masses
-//           of the round-2 digit (bits 17..6) of the tokens in the cut bin -> hist2[rank]
+//           of the round-2 digit (bits 17..6) of the tokens in the cut bin -> hist2 (summed)
 //   round 3 cut 2; masses and counts of the round-3 digit (bits 5..0)   -> hist3[rank]
 //   attend  cut 3 -> tau; the tokens at tau that the selection still needs are taken
 //           from the lowest positions first, i.e. rank by rank (their counts are in
@@ -29,7 +30,8 @@
 // The exchange buffers hold one row per retrieval slice (xrow below): streaming heads
 // never select, so they neither write nor read statistics or histograms.
 // Masses are integers in units of 2^-63 (mass_q), so the summed histograms are exact
-// whatever the order, and every rank takes the same cut decisions.  Each cut is taken
+// whatever the order of the additions, and every rank takes the same cut decisions.
+// The round-3 counts stay per rank: the tie quota hands ties out rank by rank.  Each cut is taken
 // at the start of the launch that needs it, by every CTA of the slice (the summed
 // histogram is a few KB to 32 KB per rank), so a rank's step is seven launches: stats,
 // mass, round 2, round 3, list count, list, attention.  The kernels never wait on
@@ -62,11 +64,13 @@ __device__ __forceinline__ long long local_rows(const CpParams& P, int L) {
   return n < 0 ? 0 : (n > P.C ? P.C : n);
 }
 
-// Exchange row of retrieval slice s = (b, g) in rank r's slot: the exchange buffers hold
-// the retrieval slices only, sequence-major.
-__device__ __forceinline__ size_t xrow(const CpParams& P, int r, int s) {
-  return (size_t)r * P.n_xrows + (size_t)(s / P.Hkv) * P.n_ret + P.ret_ord[s % P.Hkv];
+// Exchange row of retrieval slice s = (b, g): the exchange buffers hold the retrieval
+// slices only, sequence-major.  xslot is the row of a summed buffer (hist1, hist2),
+// xrow the row in rank r's slot of a gathered one (stats, hist3).
+__device__ __forceinline__ size_t xslot(const CpParams& P, int s) {
+  return (size_t)(s / P.Hkv) * P.n_ret + P.ret_ord[s % P.Hkv];
 }
+__device__ __forceinline__ size_t xrow(const CpParams& P, int r, int s) { return (size_t)r * P.n_xrows + xslot(P, s); }
 
 // Length of sequence b, validated as in the one-GPU step; shared through *sh.
 __device__ __forceinline__ int cta_len(const CpParams& P, int b, int* sh) {
@@ -232,8 +236,8 @@ __global__ void __launch_bounds__(kRowThreads) k_cp_stats(CpParams P) {
   const long long n = P.is_ret[g] ? local_rows(P, L) : 0;
   if (c == 0) rope_heads<G>(P, q, b, g, L, cs, sn);
   if (!P.is_ret[g]) return;
-  if (c == 0) {   // the rank's round-1 histogram row of this slice, filled by the next phase
-    unsigned long long* h1 = P.hist1 + xrow(P, P.rank, s) * kBins1;
+  if (c == 0) {   // the slice's round-1 histogram row in this rank's buffer, filled by the next phase
+    unsigned long long* h1 = P.hist1 + xslot(P, s) * kBins1;
     for (int i = tid; i < kBins1; i += kRowThreads) h1[i] = 0ull;
   }
   qidx_heads<G>(P, q, g, qsm);
@@ -297,8 +301,8 @@ __global__ void __launch_bounds__(kRowThreads) k_cp_mass(CpParams P) {
   const int L = cta_len(P, b, &sh_len);
   const long long n = local_rows(P, L);
   for (int i = tid; i < kBins1; i += kRowThreads) { hc[i] = 0u; hl[i] = 0u; }
-  if (c == 0) {   // the rank's round-2 and round-3 rows of this slice, filled by later phases
-    unsigned long long* h2 = P.hist2 + xrow(P, P.rank, s) * kBins2;
+  if (c == 0) {   // the slice's round-2 row and the rank's round-3 row, filled by later phases
+    unsigned long long* h2 = P.hist2 + xslot(P, s) * kBins2;
     unsigned long long* h3 = P.hist3 + xrow(P, P.rank, s) * kBins3 * 2;
     for (int i = tid; i < kBins2; i += kRowThreads) h2[i] = 0ull;
     if (tid < kBins3 * 2) h3[tid] = 0ull;
@@ -353,7 +357,7 @@ __global__ void __launch_bounds__(kRowThreads) k_cp_mass(CpParams P) {
     }
   }
   __syncthreads();
-  unsigned long long* dst = P.hist1 + xrow(P, P.rank, s) * kBins1;
+  unsigned long long* dst = P.hist1 + xslot(P, s) * kBins1;
   for (int d = tid; d < kBins1; d += kRowThreads) {
     const unsigned cnt = hc[d];
     if (cnt) {
@@ -401,31 +405,17 @@ __device__ void cut_desc(const unsigned long long* h, unsigned long long above, 
   __syncthreads();
 }
 
-// Sum over the ranks of a [R][n_xrows][4096] histogram, slice s, into shared memory
-// (padded slots); returns this thread's part of the total.  Each thread keeps its 16
-// bins' loads of one rank in flight together.
-__device__ unsigned long long gather_hist4096(const CpParams& P, const unsigned long long* hist, int s,
-                                              unsigned long long* h) {
-  const int R = P.n_ranks;
+// Slice s's row of a summed [n_xrows][4096] histogram (every rank's masses added, by
+// the all-reduce between the launches, or directly when emulated ranks share the
+// buffer) into shared memory (padded slots); returns this thread's part of the total.
+__device__ unsigned long long load_hist4096(const CpParams& P, const unsigned long long* hist, int s,
+                                            unsigned long long* h) {
   constexpr int PER = kBins1 / kThreads;
   const int tid = threadIdx.x;
+  const unsigned long long* src = hist + xslot(P, s) * kBins1 + tid;
   unsigned long long v[PER];
 #pragma unroll
-  for (int k = 0; k < PER; ++k) v[k] = 0ull;
-  constexpr int kRanksAtOnce = 4;   // 64 loads per thread in flight
-  for (int r0 = 0; r0 < R; r0 += kRanksAtOnce) {
-    unsigned long long w[kRanksAtOnce][PER];
-#pragma unroll
-    for (int i = 0; i < kRanksAtOnce; ++i) {
-      const unsigned long long* src = hist + xrow(P, r0 + i < R ? r0 + i : 0, s) * kBins1 + tid;
-#pragma unroll
-      for (int k = 0; k < PER; ++k) w[i][k] = r0 + i < R ? __ldcg(src + k * kThreads) : 0ull;
-    }
-#pragma unroll
-    for (int i = 0; i < kRanksAtOnce; ++i)
-#pragma unroll
-      for (int k = 0; k < PER; ++k) v[k] += w[i][k];
-  }
+  for (int k = 0; k < PER; ++k) v[k] = __ldcg(src + k * kThreads);
   unsigned long long mine = 0ull;
 #pragma unroll
   for (int k = 0; k < PER; ++k) {
@@ -445,7 +435,7 @@ __device__ unsigned long long gather_hist4096(const CpParams& P, const unsigned 
 __device__ void cp_cut1(const CpParams& P, int s, bool store, unsigned long long* h, unsigned long long* scratch,
                         int* sb, unsigned long long* sabove, unsigned long long* starget) {
   const int tid = threadIdx.x;
-  const unsigned long long mine = gather_hist4096(P, P.hist1, s, h);
+  const unsigned long long mine = load_hist4096(P, P.hist1, s, h);
   const unsigned long long total = block_sum<unsigned long long>(mine, scratch);   // (barrier: h complete)
   unsigned long long target = (unsigned long long)ceil((double)P.p * (double)total);
   if (target < 1ull) target = 1ull;
@@ -472,7 +462,7 @@ __device__ void cp_cut2(const CpParams& P, int s, bool store, unsigned long long
                         unsigned long long* scratch, int* sb, unsigned long long* sabove) {
   const int tid = threadIdx.x;
   const unsigned long long above = *sabove;
-  gather_hist4096(P, P.hist2, s, h);
+  load_hist4096(P, P.hist2, s, h);
   if (tid == 0) *sb = -1;
   __syncthreads();
   cut_desc<kBins2, true>(h, above, target, sb, sabove, scratch);
@@ -597,7 +587,7 @@ __global__ void __launch_bounds__(kThreads) k_cp_hist(CpParams P, int round) {
   if (round == 3 && tid < kBins3) P.tab3[((size_t)s * P.n_chunks + c) * kBins3 + tid] = hn[tid];
   if (!cta_any) return;
   if (round == 2) {
-    unsigned long long* dst = P.hist2 + xrow(P, P.rank, s) * kBins2;
+    unsigned long long* dst = P.hist2 + xslot(P, s) * kBins2;
     for (int d = tid; d < kBins2; d += kThreads)
       if (hm[d]) atomicAdd(dst + d, hm[d]);
   } else if (tid < kBins3 && hn[tid]) {

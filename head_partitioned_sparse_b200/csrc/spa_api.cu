@@ -799,12 +799,13 @@ spa_status spa_cp_exchange_sizes(spa_handle h, int B, int n_ranks, const uint8_t
   if (B < 1 || B > h->cfg.max_batch)
     return fail(SPA_ERR_INVALID_ARG, "B must be in [1, max_batch=%d] (got %d)", h->cfg.max_batch, B);
   if (n_ranks < 1 || n_ranks > kMaxRanks) return fail(SPA_ERR_INVALID_ARG, "n_ranks must be in [1, %d]", kMaxRanks);
-  // histogram and statistics rows for the retrieval slices only
-  const size_t xrows = (size_t)n_ranks * B * count_retrieval(h, head_mask), rows = (size_t)B * h->cfg.n_q_heads;
-  bytes[0] = xrows * h->n_chunks_max * h->G * sizeof(float2);
+  // histogram and statistics rows for the retrieval slices only; hist1 and hist2 are
+  // summed over the ranks (no slot per rank)
+  const size_t xrows = (size_t)B * count_retrieval(h, head_mask), rows = (size_t)B * h->cfg.n_q_heads;
+  bytes[0] = (size_t)n_ranks * xrows * h->n_chunks_max * h->G * sizeof(float2);
   bytes[1] = xrows * spa::kBins1 * 8;
   bytes[2] = xrows * spa::kBins2 * 8;
-  bytes[3] = xrows * spa::kBins3 * 16;
+  bytes[3] = (size_t)n_ranks * xrows * spa::kBins3 * 16;
   bytes[4] = (size_t)n_ranks * rows * spa::kHeadDim * 4;
   bytes[5] = (size_t)n_ranks * rows * 4;
   return SPA_OK;

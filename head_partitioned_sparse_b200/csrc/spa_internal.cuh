@@ -104,12 +104,13 @@ struct CpParams {
   float* q_idx;                   // [Bm][Hq][16]
   float* pi;                      // [Bm*Hkv][pi_stride] local probabilities
   int64_t pi_stride;
-  // Exchange buffers: one row per (rank, retrieval slice), row r * n_xrows + b * n_ret
-  // + ret_ord[g]; streaming slices never write or read them.
-  float2* stats;                  // exchange: [R][n_xrows][n_chunks][G] (m in log2 units, z)
-  unsigned long long* hist1;      // exchange: [R][n_xrows][kBins1] masses
-  unsigned long long* hist2;      // exchange: [R][n_xrows][kBins2] masses
-  unsigned long long* hist3;      // exchange: [R][n_xrows][kBins3][2] (mass, count)
+  // Exchange buffers: rows for the retrieval slices only (row b * n_ret + ret_ord[g]);
+  // streaming slices never write or read them.  Gathered buffers have a slot per rank
+  // (row r * n_xrows + ...); summed ones (all-reduced between the launches) do not.
+  float2* stats;                  // gathered: [R][n_xrows][n_chunks][G] (m in log2 units, z)
+  unsigned long long* hist1;      // summed: [n_xrows][kBins1] masses
+  unsigned long long* hist2;      // summed: [n_xrows][kBins2] masses
+  unsigned long long* hist3;      // gathered: [R][n_xrows][kBins3][2] (mass, count)
   unsigned* tab3;                 // [n_slices][n_chunks][kBins3] local round-3 counts per chunk
   int* chunk_cnt;                 // [n_slices][n_chunks] listed rows per chunk
   CpSlice* cs;                    // [n_slices]

@@ -307,24 +307,29 @@ SPA_API spa_status spa_prefill(spa_handle h, const void* q_chunk, const void* k_
  * positions, sinks and window are global positions.  Top-p with bf16 caches only.
  *
  * The step is five phases, SPA_CP_STATS .. SPA_CP_ATTEND, run in order on every rank,
- * each followed by an all-gather (NCCL or any other transport; on one GPU, emulated
- * ranks share the buffers and need none) of the rank's slot of the buffer it wrote:
- *   SPA_CP_STATS   per-head (max, sum of exp) of the local index scores -> stats
- *   SPA_CP_MASS    local probabilities; round-1 mass histogram           -> hist1
- *   SPA_CP_ROUND2  cut of round 1 (all ranks' hist1); round-2 histogram  -> hist2
- *   SPA_CP_ROUND3  cut of round 2; round-3 histogram with counts         -> hist3
+ * each followed by an exchange of the buffer it wrote (NCCL or any other transport; on
+ * one GPU, emulated ranks share the buffers and need none):
+ *   SPA_CP_STATS   per-head (max, sum of exp) of the local index scores -> stats   (gather)
+ *   SPA_CP_MASS    local probabilities; round-1 mass histogram           -> hist1   (sum)
+ *   SPA_CP_ROUND2  cut of round 1 (summed hist1); round-2 histogram      -> hist2   (sum)
+ *   SPA_CP_ROUND3  cut of round 2; round-3 histogram with counts         -> hist3   (gather)
  *   SPA_CP_ATTEND  final cut and this rank's share of the ties; attention over the
- *                  local kept rows                                        -> out_all, lse_all
- * then spa_cp_combine merges the ranks' outputs.  Histogram masses are integers, so
- * every rank reaches the same cut.  Each exchange buffer is [n_ranks][...] with the
- * rank's slot at index rank; a phase writes only its own slots (the histogram slots it
- * adds into are cleared by an earlier phase of the same rank: stats clears hist1, mass
- * clears hist2 and hist3) and reads the other slots, which must hold the gathered data
- * of the previous phase.  Streaming heads never select, so stats and hist1..hist3 hold
- * one row per retrieval slice only: slot r, row b * n_ret + j for the j-th retrieval
- * KV head (in head order) of sequence b, n_ret the number of retrieval heads.
- * spa_cp_exchange_sizes gives the byte size of each buffer (all slots) for a head
- * mask; the buffers must be sized with the same mask the phases get.  Every pointer
+ *                  local kept rows                                -> out_all, lse_all (gather)
+ * then spa_cp_combine merges the ranks' outputs.  A gathered buffer is [n_ranks][...]
+ * with the rank's slot at index rank: the phase writes its own slot and reads the
+ * others, which must hold the other ranks' data of the previous phase (an all-gather).
+ * A summed buffer (hist1, hist2) has no slots: the phase adds this rank's masses into
+ * it and the exchange must leave every rank's copy holding the sum over the ranks (an
+ * all-reduce; the words are uint64 and an int64 sum gives the same bits, as two's
+ * complement addition is unsigned addition modulo 2^64).  Histogram masses are
+ * integers, so the sums are exact and every rank reaches the same cut.  The rows a
+ * phase adds into are cleared by an earlier phase of the same rank (stats clears
+ * hist1, mass clears hist2 and its hist3 slot), so emulated ranks that share the
+ * buffers add into one sum.  Streaming heads never select, so stats and hist1..hist3
+ * hold one row per retrieval slice only: row b * n_ret + j (in slot r for the gathered
+ * ones) for the j-th retrieval KV head (in head order) of sequence b, n_ret the number
+ * of retrieval heads.  spa_cp_exchange_sizes gives the byte size of each buffer (all
+ * slots) for a head mask; the buffers must be sized with the same mask the phases get.  Every pointer
  * is a device pointer, 16-byte aligned.  Phases and combine only enqueue work on
  * `stream`; a phase called out of order computes garbage but stays in bounds. */
 #define SPA_CP_STATS 0
@@ -350,8 +355,8 @@ typedef struct {
                                and pos0 + max_ctx) */
   void* stats;              /* [n_ranks][B][n_ret][ceil(max_ctx / 4096)][G] float2 (may be NULL, as
                                may hist1..hist3, when head_mask has no retrieval head) */
-  void* hist1;              /* [n_ranks][B][n_ret][4096] uint64 */
-  void* hist2;              /* [n_ranks][B][n_ret][4096] uint64 */
+  void* hist1;              /* [B][n_ret][4096] uint64, summed over the ranks */
+  void* hist2;              /* [B][n_ret][4096] uint64, summed over the ranks */
   void* hist3;              /* [n_ranks][B][n_ret][64][2] uint64 */
   float* out_all;           /* [n_ranks][B][Hq][128] float32 */
   float* lse_all;           /* [n_ranks][B][Hq] float32, log2 of the softmax denominator */

@@ -2,9 +2,9 @@
 
 It runs the same phase sequence as libspa's context-parallel kernels and reads and
 writes the same exchange-buffer layouts (byte tensors: stats [R][X][n_chunks][G] float
-pairs, hist1/hist2 [R][X][4096] uint64, hist3 [R][X][64][2] uint64, with X = B * n_ret
-rows, one per retrieval slice, sequence-major; out_all [R][B][Hq][128] and lse_all
-[R][B][Hq] float32), in float64 NumPy, so that the
+pairs, hist1/hist2 [X][4096] uint64 summed over the ranks, hist3 [R][X][64][2] uint64,
+with X = B * n_ret rows, one per retrieval slice, sequence-major; out_all
+[R][B][Hq][128] and lse_all [R][B][Hq] float32), in float64 NumPy, so that the
 orchestration in ``head_partitioned_sparse_b200.context_parallel`` and the gloo
 all-gathers can be tested without a GPU, and so that the phase decomposition itself
 (merging per-rank softmax statistics, exact integer histograms summed over ranks, the
@@ -29,9 +29,10 @@ def n_chunks(C: int) -> int:
 
 def exchange_sizes(B: int, Hq: int, Hkv: int, C: int, R: int, head_mask):
     """Byte sizes of the exchange buffers (the layout spa_cp_exchange_sizes reports):
-    statistics and histograms for the retrieval slices only."""
+    statistics and histograms for the retrieval slices only, hist1 and hist2 without a
+    slot per rank (summed)."""
     G, X = Hq // Hkv, B * int(sum(1 for v in head_mask if v))
-    return (R * X * n_chunks(C) * G * 8, R * X * BINS1 * 8, R * X * BINS2 * 8, R * X * BINS3 * 16,
+    return (R * X * n_chunks(C) * G * 8, X * BINS1 * 8, X * BINS2 * 8, R * X * BINS3 * 16,
             R * B * Hq * 128 * 4, R * B * Hq * 4)
 
 
@@ -73,8 +74,8 @@ class HostRank:
             lambda a: np.asarray(a, np.float64))
         nb = lambda name: bufs[name].numpy()
         self.stats = nb("stats").view(np.float32).reshape(R, self.X, self.nc, self.G, 2)
-        self.h1 = nb("hist1").view(np.uint64).reshape(R, self.X, BINS1)
-        self.h2 = nb("hist2").view(np.uint64).reshape(R, self.X, BINS2)
+        self.h1 = nb("hist1").view(np.uint64).reshape(self.X, BINS1)   # summed over the ranks
+        self.h2 = nb("hist2").view(np.uint64).reshape(self.X, BINS2)
         self.h3 = nb("hist3").view(np.uint64).reshape(R, self.X, BINS3, 2)
         self.out_all = nb("out_all").view(np.float32).reshape(R, inp.B, inp.Hq, 128)
         self.lse_all = nb("lse_all").view(np.float32).reshape(R, inp.B, inp.Hq)
@@ -102,8 +103,11 @@ class HostRank:
     def phase(self, ph: int) -> None:
         getattr(self, ("stats_phase", "mass_phase", "round2", "round3", "attend")[ph])()
 
+    # Each phase clears the summed rows the next phase adds into (as the kernels do), so
+    # ranks that share the buffers add into one sum.
     def stats_phase(self):
         self.stats[self.rank] = 0
+        self.h1[:] = 0
         for b, g, s in self._slices():
             if not self.inp.head_mask[g]:
                 continue
@@ -119,7 +123,8 @@ class HostRank:
                 self.stats[self.rank, x, c, :, 1] = np.exp2(part - m).sum(axis=0)
 
     def mass_phase(self):
-        self.h1[self.rank] = 0
+        self.h2[:] = 0
+        self.h3[self.rank] = 0
         for b, g, s in self._slices():
             if not self.inp.head_mask[g]:
                 continue
@@ -131,32 +136,30 @@ class HostRank:
             pi = (np.exp2(self._logits(b, g) - M) / (self.G * Z)).sum(axis=1).astype(np.float32)
             u = pi.view(np.uint32)
             self.bits[s] = u
-            np.add.at(self.h1[self.rank, x], (u >> 18).astype(np.int64), mass_q(u))
+            np.add.at(self.h1[x], (u >> 18).astype(np.int64), mass_q(u))
 
     def round2(self):
-        self.h2[self.rank] = 0
         for b, g, s in self._slices():
             if not self.inp.head_mask[g]:
                 continue
             x = self.xrow[s]
-            total = sum(int(v) for v in self.h1[:, x].sum(axis=0, dtype=np.uint64))
+            total = sum(int(v) for v in self.h1[x])
             target = max(1, math.ceil(float(np.float32(self.p)) * float(total)))
             if self.p >= 1.0 or target > total:
                 self.cut[s] = dict(b1=-1)
                 continue
-            b1, above = cut_desc(self.h1[:, x].sum(axis=0, dtype=np.uint64), 0, target)
+            b1, above = cut_desc(self.h1[x], 0, target)
             self.cut[s] = dict(b1=b1, above=above, target=target)
             u = self.bits[s]
             sel = (u >> 18) == b1
-            np.add.at(self.h2[self.rank, x], ((u[sel] >> 6) & 0xFFF).astype(np.int64), mass_q(u[sel]))
+            np.add.at(self.h2[x], ((u[sel] >> 6) & 0xFFF).astype(np.int64), mass_q(u[sel]))
 
     def round3(self):
-        self.h3[self.rank] = 0
         for s, cs in self.cut.items():
             if cs["b1"] < 0:
                 continue
             x = self.xrow[s]
-            b2, above = cut_desc(self.h2[:, x].sum(axis=0, dtype=np.uint64), cs["above"], cs["target"])
+            b2, above = cut_desc(self.h2[x], cs["above"], cs["target"])
             cs.update(b2=b2, above=above)
             u = self.bits[s]
             sel = (u >> 6) == ((cs["b1"] << 12) | b2)

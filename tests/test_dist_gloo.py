@@ -180,7 +180,7 @@ def _cp_worker(rank, world, port, q):
         bufs = {n: torch.zeros(sz, dtype=torch.uint8) for n, sz in
                 zip(cp.BUFFERS, M.exchange_sizes(inp.B, inp.Hq, inp.Hkv, CP_C, world, inp.head_mask))}
         me = M.HostRank(inp, idx, rank, world, CP_C, bufs, p=inp.p, n_sink=inp.n_sink, window=inp.window)
-        cp.run_step([rank], lambda ph, r: me.phase(ph), lambda name: cp.allgather_slot(bufs[name], world, rank))
+        cp.run_step([rank], lambda ph, r: me.phase(ph), lambda name: cp.exchange_buffer(bufs, name, world, rank))
         out = M.combine(me.out_all, me.lse_all)
         # every rank holds the same combined output; rows are gathered to rank 0
         gathered = [None] * world
@@ -225,6 +225,60 @@ def test_cp_two_rank_gloo_exchange_matches_oracle_and_emulation():
     assert status == "ok", err
     assert err <= 1e-5
     assert same, "the gloo run and the one-process emulation differ"
+    assert all(p.exitcode == 0 for p in procs)
+
+
+def _sum_worker(rank, world, port, q):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from head_partitioned_sparse_b200 import context_parallel as cp
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    try:
+        dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+        words = np.array(_SUM_WORDS[rank], np.uint64)
+        bufs = {"hist1": torch.from_numpy(words.view(np.uint8).copy()),
+                "hist3": torch.zeros(world * 16, dtype=torch.uint8)}
+        bufs["hist3"][rank * 16:(rank + 1) * 16] = rank + 1
+        cp.exchange_buffer(bufs, "hist1", world, rank)
+        cp.exchange_buffer(bufs, "hist3", world, rank)
+        q.put((rank, bufs["hist1"].numpy().view(np.uint64).tolist(), bufs["hist3"].tolist()))
+        dist.barrier()
+        dist.destroy_process_group()
+    except Exception as e:  # report to the parent instead of hanging it
+        q.put((rank, "err", repr(e)))
+        raise
+
+
+# uint64 words at and above 2^63, whose sums wrap modulo 2^64
+_SUM_WORDS = [[2 ** 63, 2 ** 64 - 1, 5, 2 ** 62], [2 ** 63 + 3, 2, 2 ** 64 - 5, 2 ** 62 + 2 ** 61]]
+
+
+def test_cp_summed_buffers_all_reduce_as_unsigned_64_bit_words():
+    """The summed histograms go through an int64 all-reduce: every rank must end with the
+    unsigned sum modulo 2^64 of every rank's words (two's complement addition), and a
+    gathered buffer with every rank's slot."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_sum_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    alive = [p for p in procs if p.is_alive()]
+    for p in alive:
+        p.kill()
+    assert not alive, "a rank did not finish"
+    want = [(a + b) % 2 ** 64 for a, b in zip(*_SUM_WORDS)]
+    got = sorted(q.get(timeout=5) for _ in range(2))
+    for rank, words, gathered in got:
+        assert words != "err", gathered
+        assert words == want
+        assert gathered == [1] * 16 + [2] * 16
     assert all(p.exitcode == 0 for p in procs)
 
 
