@@ -163,8 +163,13 @@ def emulated_step(handles: Sequence, shards: Sequence[dict], *, q_pre, head_mask
     called with each buffer's name after the phase that wrote it, must put the sums
     over all ranks into the summed buffers); ``combine=False`` skips the final merge."""
     R = len(handles)
+    need = spa.spa_cp_exchange_sizes(handles[0], Bsz, R, head_mask)
     if bufs is None:
-        bufs = alloc_exchange(spa.spa_cp_exchange_sizes(handles[0], Bsz, R, head_mask), q_pre.device)
+        bufs = alloc_exchange(need, q_pre.device)
+    else:   # reused buffers: the kernels index them by this step's batch and head mask
+        short = [name for name, n in zip(BUFFERS, need) if bufs[name].numel() < int(n)]
+        if short:
+            raise ValueError(f"exchange buffers {short} are smaller than this step's batch and head mask need")
     out_all, lse_all = _views(bufs)
     args: List[spa.spa_cp_args] = []
     for r in range(R):

@@ -368,6 +368,30 @@ def test_context_parallel_decoder_step_over_gloo():
     assert all(p.exitcode == 0 for p in procs)
 
 
+def test_emulated_step_rejects_exchange_buffers_sized_for_another_mask(monkeypatch):
+    """Buffers reused from a step with fewer retrieval heads are too small for this one:
+    the driver refuses before any phase is launched."""
+    import torch
+    import cp_host_model as M
+    from head_partitioned_sparse_b200 import binding as spa
+    from head_partitioned_sparse_b200 import context_parallel as cp
+    B, Hq, Hkv, C, R = 2, 16, 4, 2000, 3
+    calls = []
+    monkeypatch.setattr(spa, "spa_cp_exchange_sizes", lambda h, b, r, mask: M.exchange_sizes(b, Hq, Hkv, C, r, mask))
+    monkeypatch.setattr(spa, "spa_cp_phase", lambda *a, **k: calls.append(a))
+    monkeypatch.setattr(spa, "make_cp_args", lambda **k: None)
+    small = {n: torch.zeros(sz, dtype=torch.uint8) for n, sz in
+             zip(cp.BUFFERS, M.exchange_sizes(B, Hq, Hkv, C, R, [1, 0, 0, 0]))}
+    z = torch.zeros(16, dtype=torch.uint8)
+    shards = [{"k": z, "v": z, "idx": z}] * R
+    kw = dict(q_pre=z, seq_lens=z, Bsz=B, p=0.9, n_sink=4, window=64, capacity=C, out=z, combine=False)
+    with pytest.raises(ValueError, match="hist1"):
+        cp.emulated_step([0] * R, shards, head_mask=[1, 0, 1, 0], bufs=small, **kw)
+    assert calls == []
+    cp.emulated_step([0] * R, shards, head_mask=[0, 0, 1, 0], bufs=small, **kw)   # same size: accepted
+    assert len(calls) == 5 * R
+
+
 def test_cp_host_model_masses_are_exact_fixed_point():
     """mass_q(bits(x)) = x * 2^63 exactly for float32 x >= 2^-40, else 0 (the quantised
     mass the histograms sum); cut_desc finds the first bin, from the top, where the
