@@ -19,7 +19,8 @@ so the buffers are sized for one head mask.
 
 Two drivers share that sequence (``run_step``):
   * ``ContextParallelDecoder``: one process per GPU; the exchange is
-    ``torch.distributed.all_gather`` (NCCL on GPUs, gloo for the CPU tests);
+    ``torch.distributed.all_gather`` or ``all_reduce`` (NCCL on GPUs, gloo for the
+    CPU tests);
   * ``emulated_step``: several handles on one GPU, run phase by phase, every rank in
     turn; the ranks share the exchange buffers, so nothing has to move.  No kernel
     waits on another, so this is a plain sequence of launches.
