@@ -43,6 +43,47 @@ def test_library_exports_every_declared_symbol(lib):
     assert exported == set(declared_functions())
 
 
+def declared_prototypes():
+    """name -> (return type, [parameter types]) of every SPA_API function in the header."""
+    text = re.sub(r"/\*.*?\*/", " ", open(HEADER).read(), flags=re.S)
+    protos = {}
+    for ret, name, params in re.findall(r"^SPA_API\s+([\w\s\*]+?)\b(spa_\w+)\s*\(([^;{]*?)\)\s*;", text, flags=re.M):
+        params = " ".join(params.split())
+        types = [] if params in ("", "void") else [p.strip().rsplit(" ", 1)[0] if not p.strip().endswith("*")
+                                                  else p.strip() for p in params.split(",")]
+        # a parameter "const float* x" keeps its type part: drop the name after the last '*'
+        types = [re.sub(r"\s*\b\w+$", "", t) if "*" in t and not t.endswith("*") else t for t in types]
+        protos[name] = (" ".join(ret.split()), types)
+    return protos
+
+
+def _ctype_kind(c_type: str) -> str:
+    t = c_type.replace("const ", "").strip()
+    if "*" in t or t in ("spa_handle", "spa_stream"):
+        return "ptr"
+    return {"int": "i32", "int64_t": "i64", "float": "f32", "double": "f64", "unsigned": "u32",
+            "size_t": "size"}[t]
+
+
+def _py_kind(ct) -> str:
+    if ct in (ctypes.c_void_p, ctypes.c_char_p) or isinstance(ct, type) and issubclass(ct, ctypes._Pointer):
+        return "ptr"
+    return {ctypes.c_int: "i32", ctypes.c_int64: "i64", ctypes.c_float: "f32", ctypes.c_double: "f64",
+            ctypes.c_uint: "u32", ctypes.c_size_t: "size"}[ct]
+
+
+def test_binding_signatures_match_the_header_prototypes():
+    """Every ctypes signature has the header's parameter count and, position by position,
+    the same kind of argument (pointer, 32/64-bit integer, float, double, size)."""
+    protos = declared_prototypes()
+    assert sorted(protos) == sorted(B._SIGS)
+    for name, (ret, params) in protos.items():
+        py_ret, py_args = B._SIGS[name]
+        assert len(py_args) == len(params), (name, params)
+        assert [_py_kind(a) for a in py_args] == [_ctype_kind(t) for t in params], name
+        assert _py_kind(py_ret) == ("i32" if ret == "spa_status" else _ctype_kind(ret)), name
+
+
 def _cfg(**kw):
     base = dict(max_batch=2, n_q_heads=8, n_kv_heads=2, max_ctx=4096, kv_dtype=B.SPA_BF16,
                 P_q=0x10000, P_k=0x20000)   # never dereferenced by the host checks
